@@ -1,0 +1,457 @@
+"""Pins of the CPU oracle against definitions other than itself (no GPU).
+
+Each test ties one oracle function to an independent statement of what it
+must compute: brute force on small inputs, a library routine for a special
+case (torch bfloat16 casts, torch scaled-dot-product attention, complex
+rotation), closed-form invariants, or the dense looped forward that the lazy
+method must reduce to when nothing is skipped.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from cross_loop_sparsity_b200 import synth
+from oracle import flashloop_oracle as orc
+
+F32 = np.float32
+
+
+# ----------------------------------------------------------------------------
+# selection: top-k by (fp32 bit pattern desc, index asc)
+# ----------------------------------------------------------------------------
+
+def _select_by_counting(keys, k):
+    """Element i is selected iff fewer than k elements beat it (brute force)."""
+    bits = keys.astype(F32).view(np.uint32).astype(np.int64)
+    n = len(keys)
+    out = []
+    for i in range(n):
+        beats = sum(1 for j in range(n) if bits[j] > bits[i] or (bits[j] == bits[i] and j < i))
+        if beats < k:
+            out.append(i)
+    return np.array(out, dtype=np.int32)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_select_matches_counting_every_k(seed):
+    for n in (1, 2, 7, 33, 64):
+        keys = synth.make_keys(seed * 100 + n, n, "ties")
+        for k in range(0, n + 1):
+            assert np.array_equal(orc.select_top(keys, k), _select_by_counting(keys, k))
+
+
+def test_select_large_ties_matches_python_sort():
+    keys = synth.make_keys(7, 70000, "ties")
+    bits = keys.view(np.uint32)
+    order = sorted(range(len(keys)), key=lambda i: (-int(bits[i]), i))
+    for k in (1, 10, 4097, 35000, 70000):
+        assert np.array_equal(orc.select_top(keys, k), np.sort(np.array(order[:k], dtype=np.int32)))
+
+
+def test_select_nan_inf_zero_order():
+    keys = np.array([0.0, np.inf, np.nan, 1.0, 0.0, np.inf], dtype=F32)
+    assert list(orc.select_top(keys, 1)) == [2]          # NaN bit pattern above +inf
+    assert list(orc.select_top(keys, 3)) == [1, 2, 5]
+    assert list(orc.select_top(keys, 5)) == [0, 1, 2, 3, 5]   # zero tie -> lower index
+
+
+def test_n_select_rule():
+    assert orc.n_select(0.25, 128) == 32
+    assert orc.n_select(0.10, 8) == 1
+    assert orc.n_select(0.15, 16384) == 2458
+    assert orc.n_select(0.05, 4) == 1
+    assert orc.n_select(0.05, 1) == 1
+    assert orc.n_select(1.0, 5) == 5
+    assert orc.n_select(1e-9, 5) == 1
+    assert orc.n_select(0.5, 0) == 0
+
+
+# ----------------------------------------------------------------------------
+# number formats
+# ----------------------------------------------------------------------------
+
+def test_bf16_round_matches_torch():
+    rng = np.random.default_rng(3)
+    x = np.concatenate([rng.standard_normal(100000).astype(F32) * F32(10.0) ** rng.integers(-30, 30, 100000),
+                        np.array([0.0, -0.0, 1.0, 3.0e38, 1e-40, -2.5], F32)])
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = orc.bf16_round(x)
+    assert np.array_equal(got, ref)
+
+
+def _fp16_table():
+    allv = np.arange(0, 0x7C01, dtype=np.uint16).view(np.float16).astype(np.float64)  # +0 .. +inf
+    return np.sort(allv)
+
+
+def test_fp16_round_up_brute_force():
+    table = _fp16_table()
+    rng = np.random.default_rng(4)
+    xs = [rng.uniform(0, 1, 20000), 10.0 ** rng.uniform(-9, 4.8, 20000),
+          table[1:-1][rng.integers(0, len(table) - 2, 5000)],                   # exact fp16 values
+          (table[1:-2] + table[2:-1])[rng.integers(0, len(table) - 3, 5000)] / 2.0]  # midpoints
+    x = np.concatenate(xs).astype(F32)
+    x = np.concatenate([x, np.array([0.0, 65504.0, 65504.5, 70000.0, 5.9604645e-08, 1e-12], F32)])
+    got = orc.fp16_round_up(x).astype(np.float64)
+    want = table[np.searchsorted(table, x.astype(np.float64), side="left")]
+    assert np.array_equal(got, want)
+
+
+def test_fp16_round_up_overflow_is_inf():
+    assert np.isinf(orc.fp16_round_up(np.array([65520.0], F32))[0])
+
+
+# ----------------------------------------------------------------------------
+# quantiser
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("bits,g", [(4, 32), (4, 64), (4, 128), (2, 64)])
+def test_quantizer_brute_force_and_bounds(bits, g):
+    qm = (1 << (bits - 1)) - 1
+    r = synth.make_residuals(11 + bits + g, 300, 128)
+    codes, s16 = orc.quantize_groups(r, bits, g)
+    table = _fp16_table()
+    rg = r.reshape(300, 128 // g, g)
+    amax = np.abs(rg).max(axis=-1)
+    q32 = (amax / F32(qm)).astype(F32)
+    # scale: the smallest fp16 value >= fp32(absmax/qmax), by table search
+    want_s = table[np.searchsorted(table, q32.astype(np.float64), side="left")]
+    assert np.array_equal(s16.astype(np.float64), want_s)
+    s = s16.astype(F32)
+    cg = codes.reshape(300, 128 // g, g).astype(np.int64)
+    assert np.all(np.abs(cg) <= qm)
+    # code: the integer in [-qmax, qmax] nearest the fp32 quotient, ties to even (brute force)
+    for row in range(0, 300, 7):
+        for gi in range(128 // g):
+            if s[row, gi] == 0:
+                assert np.all(cg[row, gi] == 0)
+                continue
+            quot = (rg[row, gi] / s[row, gi]).astype(F32).astype(np.float64)
+            for e in range(g):
+                best = min(range(-qm, qm + 1), key=lambda c: (abs(quot[e] - c), c % 2, c))
+                assert cg[row, gi, e] == best
+    # error bound |r - code*s| <= s/2 * (1 + 2^-20), in exact (fp64) arithmetic
+    err = np.abs(rg.astype(np.float64) - cg * s[..., None].astype(np.float64))
+    assert np.all(err <= s[..., None].astype(np.float64) / 2 * (1 + 2.0 ** -20))
+
+
+def test_quantizer_zero_group_and_exact_grid():
+    r = np.zeros((2, 64), F32)
+    r[1, :32] = np.arange(-7, 9, dtype=F32).repeat(2)[:32] * F32(0.5)   # multiples of 0.5 up to 4
+    codes, s = orc.quantize_groups(r, 4, 32)
+    assert np.all(codes[0] == 0) and np.all(s[0] == 0)
+    assert s[1, 0] == np.float16(4.0 / 7.0) or s[1, 0] >= np.float32(4.0 / 7.0)
+    deq = orc.dequant_groups(codes, s, 32)
+    assert np.all(np.abs(deq - r) <= s.astype(F32).repeat(32, axis=-1) / 2 * (1 + 2 ** -20))
+
+
+def test_pack_layout_and_roundtrip():
+    assert orc.pack_codes(np.array([1, -1, 7, -7], np.int8), 4).tolist() == [0xF1, 0x97]
+    assert orc.pack_codes(np.array([1, -1, 0, 1], np.int8), 2).tolist() == [0x4D]
+    rng = np.random.default_rng(5)
+    for bits in (4, 2):
+        qm = (1 << (bits - 1)) - 1
+        c = rng.integers(-qm, qm + 1, size=(17, 128)).astype(np.int8)
+        p = orc.pack_codes(c, bits)
+        assert p.shape == (17, 128 * bits // 8)
+        assert np.array_equal(orc.unpack_codes(p, bits), c)
+
+
+# ----------------------------------------------------------------------------
+# layer pieces
+# ----------------------------------------------------------------------------
+
+def test_rope_matches_complex_rotation_and_relative_position():
+    rng = np.random.default_rng(6)
+    hd, theta = 64, 10000.0
+    x = rng.standard_normal((5, 3, hd))
+    pos = np.array([0, 1, 17, 4095, 65536])
+    got = orc.apply_rope(x, pos, theta)
+    z = x[..., :hd // 2] + 1j * x[..., hd // 2:]
+    freqs = theta ** (-np.arange(0, hd, 2) / hd)
+    z = z * np.exp(1j * pos[:, None, None] * freqs[None, None, :])
+    want = np.concatenate([z.real, z.imag], axis=-1)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-12)
+    # <rope(q, p1), rope(k, p2)> depends on p1 - p2 only
+    q, k = rng.standard_normal((1, 1, hd)), rng.standard_normal((1, 1, hd))
+    a = np.sum(orc.apply_rope(q, np.array([10]), theta) * orc.apply_rope(k, np.array([3]), theta))
+    b = np.sum(orc.apply_rope(q, np.array([107]), theta) * orc.apply_rope(k, np.array([100]), theta))
+    assert abs(a - b) < 1e-10
+
+
+def _torch_block_forward(cfg, W, h):
+    """A plain pre-norm Llama-style layer stack written with torch library ops (fp64)."""
+    H, Hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    T = h.shape[0]
+    x = torch.from_numpy(np.asarray(h, np.float64))
+    freqs = cfg.rope_theta ** (-torch.arange(0, hd, 2, dtype=torch.float64) / hd)
+    rot = torch.polar(torch.ones(T, hd // 2, dtype=torch.float64),
+                      torch.arange(T, dtype=torch.float64)[:, None] * freqs[None, :])
+
+    def rope(t):   # t [T, heads, hd] in rotate-half pairing
+        z = torch.complex(t[..., :hd // 2], t[..., hd // 2:]) * rot[:, None, :]
+        return torch.cat([z.real, z.imag], dim=-1)
+
+    for lw in W["layers"]:
+        a = torch.nn.functional.rms_norm(x, (cfg.d_model,), torch.from_numpy(lw["attn_norm"]), cfg.rms_eps)
+        y = a @ torch.from_numpy(lw["w_qkv"]).T
+        q = rope(y[:, :H * hd].reshape(T, H, hd))
+        k = rope(y[:, H * hd:(H + Hkv) * hd].reshape(T, Hkv, hd))
+        v = y[:, (H + Hkv) * hd:].reshape(T, Hkv, hd)
+        o = torch.nn.functional.scaled_dot_product_attention(
+            q.transpose(0, 1)[None], k.transpose(0, 1)[None], v.transpose(0, 1)[None],
+            is_causal=True, enable_gqa=True)[0].transpose(0, 1).reshape(T, H * hd)
+        x = x + cfg.resid_scale * (o @ torch.from_numpy(lw["w_o"]).T)
+        m = torch.nn.functional.rms_norm(x, (cfg.d_model,), torch.from_numpy(lw["mlp_norm"]), cfg.rms_eps)
+        act = torch.nn.functional.silu(m @ torch.from_numpy(lw["w_gate"]).T) * (m @ torch.from_numpy(lw["w_up"]).T)
+        x = x + cfg.resid_scale * (act @ torch.from_numpy(lw["w_down"]).T)
+    return x.numpy()
+
+
+def _tiny_cfg(**kw):
+    base = dict(d_model=32, n_heads=4, n_kv_heads=2, head_dim=8, ffn_dim=48, n_layers=2, n_loops=3,
+                rho=0.25, c_cols=4, resid_bits=4, group_size=8, q_tile=8, vocab=40, sigma=0.2,
+                seed=9, mode="prefill", batch=1, seq_len=16)
+    base.update(kw)
+    return synth.LoopConfig("tiny", **base)
+
+
+def _weights(cfg):
+    w = synth.make_weights(cfg)
+    return orc.prepare_weights(w), w["rng"]
+
+
+@pytest.mark.parametrize("K", [1, 3])
+def test_dense_looped_forward_is_k_plain_blocks(K):
+    cfg = _tiny_cfg(n_loops=K, resid_bits=16)
+    W, rng = _weights(cfg)
+    h0 = synth.make_h0(cfg, rng, cfg.seq_len)
+    cache = orc.KVCache(cfg, 1, cfg.seq_len, kv_exact=True)
+    res = orc.prefill(cfg, W, cache, h0, 1, cfg.seq_len)
+    want = np.asarray(h0, np.float64)
+    for _ in range(K):
+        want = _torch_block_forward(cfg, W, want)
+    np.testing.assert_allclose(res.h, want, rtol=0, atol=1e-11 * np.abs(want).max())
+    assert res.trace["applications"] == cfg.n_layers * K
+    x = want[-1] / np.sqrt(np.mean(want[-1] ** 2) + cfg.rms_eps)
+    np.testing.assert_allclose(res.logits[0], W["w_out"] @ x, atol=1e-11)
+
+
+def test_block_applications_golden():
+    rows = [tuple(int(v) for v in ln.split()) for ln in open(
+        __file__.replace("test_oracle_pins.py", "golden/block_applications.txt"))
+        if ln.strip() and not ln.startswith("#")]
+    for M, K, apps in rows:
+        cfg = _tiny_cfg(d_model=16, n_heads=2, n_kv_heads=1, head_dim=8, ffn_dim=16, n_layers=M,
+                        n_loops=K, seq_len=4, q_tile=4, rho=0.5, c_cols=2, group_size=8)
+        W, rng = _weights(cfg)
+        h0 = synth.make_h0(cfg, rng, 4)
+        res = orc.prefill(cfg, W, orc.KVCache(cfg, 1, 4), h0, 1, 4)
+        assert res.trace["applications"] == apps
+
+
+# ----------------------------------------------------------------------------
+# dense limit: rho = 1, every column, exact residual  ==  dense looped forward
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("B,T,qt", [(1, 16, 8), (2, 12, 16)])
+def test_lazy_prefill_dense_limit(B, T, qt):
+    cfg = _tiny_cfg(rho=1.0, c_cols=10 ** 6, resid_bits=32, q_tile=qt, seq_len=T, batch=B, n_loops=4)
+    W, rng = _weights(cfg)
+    h0 = synth.make_h0(cfg, rng, B * T)
+    lazy = orc.prefill(cfg, W, orc.KVCache(cfg, B, T, kv_exact=True), h0, B, T)
+    dcfg = cfg.with_(resid_bits=16)
+    dense = orc.prefill(dcfg, W, orc.KVCache(dcfg, B, T, kv_exact=True), h0, B, T)
+    scale = np.sqrt(np.mean(dense.h ** 2))
+    assert np.max(np.abs(lazy.h - dense.h)) <= 1e-9 * scale
+    np.testing.assert_allclose(lazy.logits, dense.logits, atol=1e-9 * np.abs(dense.logits).max())
+
+
+def test_lazy_decode_dense_limit():
+    cfg = _tiny_cfg(rho=1.0, c_cols=10 ** 6, resid_bits=32, mode="decode", batch=3, ctx_len=9, seq_len=0,
+                    n_loops=4)
+    W, rng = _weights(cfg)
+    lens = np.array([9, 5, 1])
+    tmax = 10
+    M, K, Hkv, hd = cfg.n_layers, cfg.n_loops, cfg.n_kv_heads, cfg.head_dim
+    lazy_c = orc.KVCache(cfg, 3, tmax, kv_exact=True)
+    dcfg = cfg.with_(resid_bits=16)
+    dense_c = orc.KVCache(dcfg, 3, tmax, kv_exact=True)
+    base_k = rng.standard_normal((M, 3, Hkv, tmax, hd))
+    base_v = rng.standard_normal((M, 3, Hkv, tmax, hd))
+    res_k = rng.standard_normal((M, K - 1, 3, Hkv, tmax, hd)) * 0.1
+    res_v = rng.standard_normal((M, K - 1, 3, Hkv, tmax, hd)) * 0.1
+    for b in range(3):
+        base_k[:, b, :, lens[b]:] = base_v[:, b, :, lens[b]:] = 0
+        res_k[:, :, b, :, lens[b]:] = res_v[:, :, b, :, lens[b]:] = 0
+    lazy_c.base_k[:], lazy_c.base_v[:], lazy_c.res_k[:], lazy_c.res_v[:] = base_k, base_v, res_k, res_v
+    # dense per-loop context KV = base + sum of residuals up to that loop (independent cumulative sum)
+    dense_c.kv_k[:, 0], dense_c.kv_v[:, 0] = base_k, base_v
+    dense_c.kv_k[:, 1:] = base_k[:, None] + np.cumsum(res_k, axis=1)
+    dense_c.kv_v[:, 1:] = base_v[:, None] + np.cumsum(res_v, axis=1)
+    lazy_c.lens[:] = lens
+    dense_c.lens[:] = lens
+    h0 = synth.make_h0(cfg, rng, 3)
+    a = orc.decode_step(cfg, W, lazy_c, h0)
+    b = orc.decode_step(dcfg, W, dense_c, h0)
+    assert np.max(np.abs(a.h - b.h)) <= 1e-9 * np.sqrt(np.mean(b.h ** 2))
+    np.testing.assert_allclose(a.logits, b.logits, atol=1e-9 * np.abs(b.logits).max())
+
+
+# ----------------------------------------------------------------------------
+# materialised brute force of the lazy path (independent restatement)
+# ----------------------------------------------------------------------------
+
+def _brute_lazy_prefill(cfg, W, h0, T, quant):
+    """Tiny lazy prefill (B = 1) holding each query's score vector and value rows explicitly.
+
+    Every query keeps, per layer and head, the score and the value row of every
+    causal column as last written; its attention output is the softmax of that
+    vector.  Recomputing a query overwrites the entries of its tile's column set
+    with the new loop's scores and values.  The column set is the top-c columns
+    by max |new score - stored score|, chosen once per tile.  Written without
+    the running (O, lse) form that the oracle uses.
+    """
+    H, Hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    grp, tau, M = H // Hkv, 1 / math.sqrt(hd), cfg.n_layers
+    pos = np.arange(T)
+    tiles = pos // cfg.q_tile
+    h = np.asarray(h0, np.float64).copy()
+    # chain[j] = list over loops of (K, V) [Hkv, T, hd] reconstructed values
+    chain = [[] for _ in range(M)]
+    scores = np.zeros((M, T, H, T))
+    values = np.zeros((M, T, H, T, hd))
+    colset = {}
+
+    def out_of(j, i):
+        s = scores[j, i][:, :i + 1]
+        w = np.exp(s - s.max(axis=1, keepdims=True))
+        w /= w.sum(axis=1, keepdims=True)
+        return np.einsum("ht,htd->hd", w, values[j, i][:, :i + 1])
+
+    def layer_tail(lw, hs, o):
+        hs = hs + cfg.resid_scale * (o.reshape(len(hs), H * hd) @ lw["w_o"].T)
+        return orc._mlp_update(cfg, lw, hs)
+
+    for j, lw in enumerate(W["layers"]):
+        q, k, v = orc._qkv(cfg, lw, h, pos)
+        kb, vb = orc.bf16_round(k).transpose(1, 0, 2), orc.bf16_round(v).transpose(1, 0, 2)
+        chain[j].append((kb, vb))
+        for i in range(T):
+            for hh in range(H):
+                scores[j, i, hh, :i + 1] = tau * (kb[hh // grp, :i + 1] @ q[i, hh])
+                values[j, i, hh, :i + 1] = vb[hh // grp, :i + 1]
+        o = np.stack([out_of(j, i) for i in range(T)])
+        h = layer_tail(lw, h, o)
+    key = np.sum((h - h0) ** 2, axis=1).astype(F32)
+    n_sel = max(1, min(T, math.ceil(cfg.rho * T - 1e-9)))
+    sels = {}
+    for l in range(2, cfg.n_loops + 1):
+        bits = key.view(np.uint32)
+        S = np.array(sorted(sorted(range(T), key=lambda t: (-int(bits[t]), t))[:n_sel]))
+        sels[l] = S
+        hprev = h[S].copy()
+        for j, lw in enumerate(W["layers"]):
+            q, k, v = orc._qkv(cfg, lw, h[S], pos[S])
+            kp, vp = chain[j][-1]
+            kn, vn = kp.copy(), vp.copy()
+            for a, t in enumerate(S):
+                for arr, new, prev in ((kn, k[a], kp), (vn, v[a], vp)):
+                    r = (new.astype(F32) - prev[:, t].astype(F32)).astype(F32)
+                    c, s = quant(r)
+                    arr[:, t] = (prev[:, t].astype(F32) + orc.dequant_groups(c, s, cfg.group_size)).astype(F32)
+            chain[j].append((kn, vn))
+            for tl in sorted(set(tiles[S])):
+                if (j, tl) in colset:
+                    continue
+                mem = [a for a, t in enumerate(S) if tiles[t] == tl]
+                mp = max(S[a] for a in mem)
+                for gk in range(Hkv):
+                    ck = np.full(mp + 1, -np.inf)
+                    for a in mem:
+                        t = S[a]
+                        for hh in range(gk * grp, (gk + 1) * grp):
+                            d = np.abs(tau * (kn[gk, :t + 1] @ q[a, hh]) - scores[j, t, hh, :t + 1])
+                            ck[:t + 1] = np.maximum(ck[:t + 1], d)
+                    ck = ck.astype(F32)
+                    if mp + 1 <= cfg.c_cols:
+                        colset[(j, tl, gk)] = np.arange(mp + 1)
+                    else:
+                        b2 = ck.view(np.uint32)
+                        colset[(j, tl, gk)] = np.array(sorted(sorted(range(mp + 1),
+                                                                     key=lambda c: (-int(b2[c]), c))[:cfg.c_cols]))
+                colset[(j, tl)] = True
+            for a, t in enumerate(S):
+                for hh in range(H):
+                    C = colset[(j, tiles[t], hh // grp)]
+                    C = C[C <= t]
+                    scores[j, t, hh, C] = tau * (kn[hh // grp, C] @ q[a, hh])
+                    values[j, t, hh, C] = vn[hh // grp, C]
+            o = np.stack([out_of(j, t) for t in S])
+            h[S] = layer_tail(lw, h[S], o)
+        key = np.zeros(T, F32)
+        key[S] = np.sum((h[S] - hprev) ** 2, axis=1).astype(F32)
+    return h, sels, colset
+
+
+@pytest.mark.parametrize("seed,T,qt,c", [(21, 16, 8, 3), (22, 20, 16, 5), (23, 12, 4, 2)])
+def test_lazy_prefill_matches_materialised_brute_force(seed, T, qt, c):
+    cfg = _tiny_cfg(seed=seed, seq_len=T, q_tile=qt, c_cols=c, rho=0.3, n_loops=4)
+    W, rng = _weights(cfg)
+    h0 = synth.make_h0(cfg, rng, T)
+    res = orc.prefill(cfg, W, orc.KVCache(cfg, 1, T), h0, 1, T)
+    quant = lambda r: orc.quantize_groups(r, cfg.resid_bits, cfg.group_size)
+    bh, bsel, bcols = _brute_lazy_prefill(cfg, W, h0, T, quant)
+    for l, S in bsel.items():
+        assert np.array_equal(res.trace["sel"][l], S)
+    for key_, C in res.trace["cols"].items():
+        assert np.array_equal(C, bcols[key_])
+    assert np.max(np.abs(res.h - bh)) <= 1e-9 * np.sqrt(np.mean(bh ** 2))
+
+
+# ----------------------------------------------------------------------------
+# invariants of the lazy path
+# ----------------------------------------------------------------------------
+
+def test_lazy_invariants_carry_and_keys():
+    cfg = _tiny_cfg(seed=31, seq_len=24, q_tile=8, c_cols=6, rho=0.25, n_loops=4)
+    W, rng = _weights(cfg)
+    h0 = synth.make_h0(cfg, rng, 24)
+    cache = orc.KVCache(cfg, 1, 24)
+    res = orc.prefill(cfg, W, cache, h0, 1, 24)
+    n_sel = orc.n_select(cfg.rho, 24)
+    hs = res.trace["h"]
+    for l in range(2, cfg.n_loops + 1):
+        S = res.trace["sel"][l]
+        assert len(S) == n_sel
+        carried = np.setdiff1d(np.arange(24), S)
+        assert np.array_equal(hs[l][carried], hs[l - 1][carried])        # bit-identical carry
+        if l + 1 in res.trace["keys"]:
+            assert np.all(res.trace["keys"][l + 1][carried] == 0)
+        for j in range(cfg.n_layers):
+            nz = np.any(cache.codes_k[j, l - 2, 0] != 0, axis=(0, 2)) | np.any(
+                cache.scales_k[j, l - 2, 0] != 0, axis=(0, 2))
+            assert np.all(np.isin(np.nonzero(nz)[0], S))
+            assert nz.sum() <= n_sel
+    np.testing.assert_array_equal(res.h, hs[cfg.n_loops])
+
+
+def test_correction_identity_full_columns_equals_softmax():
+    """With C = every column, the corrected output equals softmax attention on the new scores."""
+    cfg = _tiny_cfg(seed=41, seq_len=10, q_tile=16, c_cols=10 ** 6, rho=1.0, n_loops=2)
+    W, rng = _weights(cfg)
+    h0 = synth.make_h0(cfg, rng, 10)
+    cache = orc.KVCache(cfg, 1, 10)
+    res = orc.prefill(cfg, W, cache, h0, 1, 10)
+    # recompute loop 2's attention of layer 0 directly from the cache and loop-1 state
+    lw = W["layers"][0]
+    q, _, _ = orc._qkv(cfg, lw, res.trace["h"][1], np.arange(10))
+    tau = 1 / math.sqrt(cfg.head_dim)
+    for i in range(10):
+        kk = cache.chain("k", 0, 2, 0, np.arange(i + 1))
+        vv = cache.chain("v", 0, 2, 0, np.arange(i + 1))
+        o, lse = orc._attn_full(q[i], kk, vv, tau)
+        np.testing.assert_allclose(res.trace["O"][0, i], o, atol=1e-12)
+        np.testing.assert_allclose(res.trace["lse"][0, i], lse, atol=1e-12)
