@@ -1,0 +1,115 @@
+// fl_cache.cuh -- layout of the KV cache in HBM and the per-lane chain
+// reconstruction shared by the attention-side kernels.
+//
+// Lazy layout (resid_bits 4 or 2):
+//   base   bf16  [M][2][B][Hkv][T][hd]            loop-1 K (0) and V (1)
+//   codes  u8    [M][K-1][2][B][Hkv][T][hd*b/8]   residual codes of loops 2..K
+//   scales fp16  [M][K-1][2][B][Hkv][T][hd/g]     per-group scales of loops 2..K
+// Dense per-loop layout (resid_bits 16):
+//   base   bf16  [M][K][2][B][Hkv][T][hd]
+// Tokens of one (sequence, KV head) are contiguous so a decode step streams them.
+// The reconstructed KV of loop m is base + code*scale of loops 2..m, added in
+// loop order in fp32 ("FlashLoop ...", abstract: KV residuals between
+// adjacent loops).  code*scale is exact in fp32 (|code| <= 7, 11-bit scale).
+#pragma once
+#include "fl_device.cuh"
+
+namespace fl {
+
+struct CacheView {
+  int M, K, B, Hkv, T, hd, g, bits, dense;
+  uint16_t* base;
+  uint8_t* codes;
+  uint16_t* scales;
+
+  __host__ __device__ size_t row_bytes_codes() const { return static_cast<size_t>(hd) * bits / 8; }
+  __host__ __device__ uint16_t* base_row(int j, int kv, int b, int h, int t) const {
+    return base + ((((static_cast<size_t>(j) * 2 + kv) * B + b) * Hkv + h) * T + t) * hd;
+  }
+  // dense per-loop KV, loop l in 1..K
+  __host__ __device__ uint16_t* dense_row(int j, int l, int kv, int b, int h, int t) const {
+    return base + (((((static_cast<size_t>(j) * K + (l - 1)) * 2 + kv) * B + b) * Hkv + h) * T + t) * hd;
+  }
+  __host__ __device__ size_t res_index(int j, int l, int kv, int b, int h, int t) const {
+    return ((((static_cast<size_t>(j) * (K - 1) + (l - 2)) * 2 + kv) * B + b) * Hkv + h) * T + t;
+  }
+  __host__ __device__ uint8_t* code_row(int j, int l, int kv, int b, int h, int t) const {
+    return codes + res_index(j, l, kv, b, h, t) * row_bytes_codes();
+  }
+  __host__ __device__ uint16_t* scale_row(int j, int l, int kv, int b, int h, int t) const {
+    return scales + res_index(j, l, kv, b, h, t) * (hd / g);
+  }
+};
+
+__device__ __forceinline__ int sext(int v, int bits) { return (v << (32 - bits)) >> (32 - bits); }
+
+// The EPL codes of one lane (elements lane*EPL .. +EPL-1) of a packed row.
+template <int EPL>
+__device__ __forceinline__ void lane_codes(const uint8_t* row, int bits, int lane, int* c) {
+  if (EPL == 4) {
+    if (bits == 4) {
+      const uint32_t u = *reinterpret_cast<const uint16_t*>(row + lane * 2);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) c[e] = sext((u >> (4 * e)) & 0xF, 4);
+    } else {
+      const uint32_t u = row[lane];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) c[e] = sext((u >> (2 * e)) & 0x3, 2);
+    }
+  } else {  // EPL == 2
+    if (bits == 4) {
+      const uint32_t u = row[lane];
+      c[0] = sext(u & 0xF, 4);
+      c[1] = sext((u >> 4) & 0xF, 4);
+    } else {
+      const uint32_t u = (row[lane >> 1] >> ((lane & 1) * 4)) & 0xF;
+      c[0] = sext(u & 0x3, 2);
+      c[1] = sext((u >> 2) & 0x3, 2);
+    }
+  }
+}
+
+// Reconstructed lazy KV of loop m (1 = base) for one row; lane holds EPL values.
+template <int EPL>
+__device__ __forceinline__ void chain_lane(const CacheView& cv, int j, int kv, int b, int h, int t, int m, int lane,
+                                           float* out) {
+  const uint16_t* br = cv.base_row(j, kv, b, h, t) + lane * EPL;
+  if (EPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(br);
+    out[0] = bf16_to_f(u.x & 0xFFFF);
+    out[1] = bf16_to_f(u.x >> 16);
+    out[2] = bf16_to_f(u.y & 0xFFFF);
+    out[3] = bf16_to_f(u.y >> 16);
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(br);
+    out[0] = bf16_to_f(u & 0xFFFF);
+    out[1] = bf16_to_f(u >> 16);
+  }
+  const int gi = (lane * EPL) / cv.g;
+  for (int l = 2; l <= m; ++l) {
+    int c[EPL];
+    lane_codes<EPL>(cv.code_row(j, l, kv, b, h, t), cv.bits, lane, c);
+    const float s = half_bits_to_f(cv.scale_row(j, l, kv, b, h, t)[gi]);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) out[e] = __fadd_rn(out[e], __fmul_rn(static_cast<float>(c[e]), s));
+  }
+}
+
+// Base and loop-m reconstruction of one row in one pass (lane holds EPL values each).
+template <int EPL>
+__device__ __forceinline__ void chain_lane2(const CacheView& cv, int j, int kv, int b, int h, int t, int m_lo,
+                                            int m_hi, int lane, float* lo, float* hi) {
+  chain_lane<EPL>(cv, j, kv, b, h, t, m_lo, lane, lo);
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) hi[e] = lo[e];
+  const int gi = (lane * EPL) / cv.g;
+  for (int l = m_lo + 1; l <= m_hi; ++l) {
+    int c[EPL];
+    lane_codes<EPL>(cv.code_row(j, l, kv, b, h, t), cv.bits, lane, c);
+    const float s = half_bits_to_f(cv.scale_row(j, l, kv, b, h, t)[gi]);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) hi[e] = __fadd_rn(hi[e], __fmul_rn(static_cast<float>(c[e]), s));
+  }
+}
+
+}  // namespace fl

@@ -1,0 +1,339 @@
+// fl_gemm.cu -- the shared-block GEMMs on 5th-generation tensor cores.
+//
+// One CTA computes one 128 x BN output tile (or one K-split of it):
+//   warp 0      : TMA producer (one thread) filling a STAGES-deep shared-memory ring
+//   warp 1      : TMEM owner and MMA issuer (one thread issues tcgen05.mma)
+//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4) .. +31 with tcgen05.ld
+// Operands are bf16, K-major, 128-byte swizzled (64 elements per row of a box),
+// accumulation is fp32 in TMEM.  The epilogue is fused: plain fp32 store (QKV,
+// logits), scaled residual scatter-add into the fp32 hidden state (O-proj,
+// down-proj), or SiLU(gate) * up into the bf16 MLP activation (gate/up, which
+// keeps two accumulators).  Split-K partials go to a scratch buffer and the
+// last CTA of a tile (an atomic ticket, no waiting) reduces them in split
+// order, so results do not depend on CTA timing.
+#include "fl_device.cuh"
+#include "fl_internal.h"
+
+namespace fl {
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kBoxK = 64;             // bf16 elements per 128-byte swizzled row
+constexpr int kABytes = 128 * kBoxK * 2;
+constexpr int kSmemBudget = 200 * 1024;
+
+template <int BN, bool DA, bool DB>
+struct Cfg {
+  static constexpr int kNA = DA ? 2 : 1;
+  static constexpr int kNB = DB ? 2 : 1;
+  static constexpr int kBBytes = BN * kBoxK * 2;
+  static constexpr int kStageBytes = kNA * kABytes + kNB * kBBytes;
+  static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
+  static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
+  static constexpr int kNAcc = (DA || DB) ? 2 : 1;
+  static constexpr int kColsNeeded = kNAcc * BN;
+  static constexpr uint32_t kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
+                                        : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
+  static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + 256;
+  static_assert(kBBytes % 1024 == 0, "B box must keep 1024-byte alignment of the swizzle atoms");
+  static_assert(kStages >= 2, "pipeline needs two stages");
+};
+
+__device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
+
+template <bool SWAP>
+__device__ __forceinline__ void epi_apply(const GemmArgs& p, int row, int col0, int tile_m, int tile_n, int BN,
+                                          const float* v0, const float* v1) {
+  // row: accumulator row within the 128-row tile; columns col0 .. col0+15
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    int tok, feat;
+    if (SWAP) {
+      feat = tile_m * 128 + row;
+      tok = col0 + c;
+    } else {
+      tok = tile_m * 128 + row;
+      feat = tile_n * BN + col0 + c;
+    }
+    if (tok >= p.n_tok || feat >= p.n_feat) continue;
+    if (p.epi == kEpiStore) {
+      p.out[static_cast<size_t>(tok) * p.ldo + feat] = v0[c];
+    } else if (p.epi == kEpiResid) {
+      const int r = p.idx ? p.idx[tok] : tok;
+      float* dst = p.h + static_cast<size_t>(r) * p.ldh + feat;
+      *dst = *dst + p.scale * v0[c];
+    } else {
+      p.act[static_cast<size_t>(tok) * p.ld_act + feat] = f_to_bf16(silu_f(v0[c]) * v1[c]);
+    }
+  }
+}
+
+template <int BN, bool DA, bool DB, bool SWAP>
+__global__ void __launch_bounds__(kThreads, 1)
+k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+          const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
+          const GemmArgs p, const int a_3d, const int b_3d) {
+  using C = Cfg<BN, DA, DB>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* done = empty + C::kStages;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(done + 1);
+  volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort, [1] last-split
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile_m = blockIdx.x, tile_n = blockIdx.y, split = blockIdx.z;
+  const int c0 = (split * p.k_chunks) / p.splits;
+  const int c1 = ((split + 1) * p.k_chunks) / p.splits;
+  const int nch = c1 - c0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    mbar_init(smem_u32(done), 1);
+    flags[0] = 0;
+    flags[1] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmB0);
+    int issued = 0;
+    for (int i = 0; i < nch; ++i) {
+      const int s = i % C::kStages;
+      const uint32_t ph = (i / C::kStages) & 1;
+      if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.status)) {
+        flags[0] = 1;
+        break;
+      }
+      uint8_t* st = smem + s * C::kStageBytes;
+      const uint32_t fb = smem_u32(&full[s]);
+      mbar_arrive_expect_tx(fb, C::kStageBytes);
+      const int kx = (c0 + i) * kBoxK;
+      const int ya = tile_m * 128;
+      const int yb = tile_n * BN;
+      if (a_3d) {
+        tma_load_3d(smem_u32(st), &tmA0, fb, kx, ya, p.a_z);
+        if (DA) tma_load_3d(smem_u32(st + kABytes), &tmA1, fb, kx, ya, p.a_z);
+      } else {
+        tma_load_2d(smem_u32(st), &tmA0, fb, kx, ya);
+        if (DA) tma_load_2d(smem_u32(st + kABytes), &tmA1, fb, kx, ya);
+      }
+      uint8_t* sb = st + C::kNA * kABytes;
+      if (b_3d) {
+        tma_load_3d(smem_u32(sb), &tmB0, fb, kx, yb, p.b_z);
+        if (DB) tma_load_3d(smem_u32(sb + C::kBBytes), &tmB1, fb, kx, yb, p.b_z);
+      } else {
+        tma_load_2d(smem_u32(sb), &tmB0, fb, kx, yb);
+        if (DB) tma_load_2d(smem_u32(sb + C::kBBytes), &tmB1, fb, kx, yb);
+      }
+      ++issued;
+    }
+    if (flags[0]) {
+      // Give the copies still in flight a bounded chance to land before exit.
+      for (int i = (issued > C::kStages ? issued - C::kStages : 0); i < issued; ++i)
+        mbar_wait(smem_u32(&full[i % C::kStages]), (i / C::kStages) & 1, nullptr);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc = umma_idesc_bf16(128, BN);
+    for (int i = 0; i < nch; ++i) {
+      const int s = i % C::kStages;
+      const uint32_t ph = (i / C::kStages) & 1;
+      if (!mbar_wait(smem_u32(&full[s]), ph, p.status)) {
+        flags[0] = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(smem + s * C::kStageBytes);
+      const uint32_t a1 = a0 + kABytes;
+      const uint32_t b0 = a0 + C::kNA * kABytes;
+      const uint32_t b1 = b0 + C::kBBytes;
+#pragma unroll
+      for (int kk = 0; kk < kBoxK / 16; ++kk) {
+        const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+        const uint64_t da = umma_desc_sw128(a0 + kk * 32);
+        const uint64_t db = umma_desc_sw128(b0 + kk * 32);
+        tc_mma_bf16(tmem, da, db, idesc, acc);
+        if (C::kNAcc == 2) {
+          const uint64_t da1 = DA ? umma_desc_sw128(a1 + kk * 32) : da;
+          const uint64_t db1 = DB ? umma_desc_sw128(b1 + kk * 32) : db;
+          tc_mma_bf16(tmem + BN, da1, db1, idesc, acc);
+        }
+      }
+      tc_commit(smem_u32(&empty[s]));
+    }
+    tc_commit(smem_u32(done));
+  } else if (warp >= 2) {
+    // ---------------- epilogue
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const bool ok = mbar_wait(smem_u32(done), 0, p.status);
+    __syncwarp();   // tcgen05.ld below is warp-collective (.sync.aligned)
+    tc_fence_after();
+    const bool valid = ok && !flags[0] && nch > 0;
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    float v0[16], v1[16];
+    if (p.splits == 1) {
+      for (int c = 0; c < BN; c += 16) {
+        tmem_ld16(tbase + c, v0);
+        if (C::kNAcc == 2) tmem_ld16(tbase + BN + c, v1);
+        tc_wait_ld();
+        if (valid) epi_apply<SWAP>(p, row, c, tile_m, tile_n, BN, v0, v1);
+      }
+    } else {
+      // split-K: write this split's partial tile, take a ticket, the last CTA reduces.
+      const size_t tile_floats = static_cast<size_t>(C::kNAcc) * BN * 128;
+      float* mine = p.partial + (static_cast<size_t>(split) * gridDim.x + tile_m) * tile_floats;
+      for (int c = 0; c < BN; c += 16) {
+        tmem_ld16(tbase + c, v0);
+        if (C::kNAcc == 2) tmem_ld16(tbase + BN + c, v1);
+        tc_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          mine[static_cast<size_t>(c + j) * 128 + row] = valid ? v0[j] : 0.f;
+          if (C::kNAcc == 2) mine[static_cast<size_t>(BN + c + j) * 128 + row] = valid ? v1[j] : 0.f;
+        }
+      }
+      __threadfence();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (warp == 2 && lane == 0) {
+        const int old = atomicAdd(&p.counters[tile_m], 1);
+        flags[1] = (old == p.splits - 1) ? 1 : 0;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (flags[1]) {
+        __threadfence();
+        for (int c = 0; c < BN; c += 16) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            v0[j] = 0.f;
+            v1[j] = 0.f;
+          }
+          for (int s = 0; s < p.splits; ++s) {
+            const float* src = p.partial + (static_cast<size_t>(s) * gridDim.x + tile_m) * tile_floats;
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              v0[j] += __ldcg(src + static_cast<size_t>(c + j) * 128 + row);
+              if (C::kNAcc == 2) v1[j] += __ldcg(src + static_cast<size_t>(BN + c + j) * 128 + row);
+            }
+          }
+          epi_apply<SWAP>(p, row, c, tile_m, tile_n, BN, v0, v1);
+        }
+        if (warp == 2 && lane == 0) p.counters[tile_m] = 0;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int BN, bool DA, bool DB, bool SWAP>
+cudaError_t launch_one(const GemmLaunch& g, cudaStream_t stream) {
+  using C = Cfg<BN, DA, DB>;
+  auto kern = k_gemm_tc<BN, DA, DB, SWAP>;
+  const CUtensorMap& a1 = g.a1 ? *g.a1 : *g.a0;
+  const CUtensorMap& b1 = g.b1 ? *g.b1 : *g.b0;
+  kern<<<g.grid, kThreads, C::kSmemBytes, stream>>>(*g.a0, a1, *g.b0, b1, g.args, g.a_3d, g.b_3d);
+  return cudaGetLastError();
+}
+
+template <int BN, bool DA, bool DB, bool SWAP>
+void set_attr() {
+  cudaFuncSetAttribute(k_gemm_tc<BN, DA, DB, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       Cfg<BN, DA, DB>::kSmemBytes);
+}
+
+}  // namespace
+
+// Opt every GEMM instantiation in to its dynamic shared memory once, outside any capture.
+void gemm_init_attrs() {
+  static bool done = false;
+  if (done) return;
+  set_attr<16, true, false, true>();
+  set_attr<16, false, false, true>();
+  set_attr<32, true, false, true>();
+  set_attr<32, false, false, true>();
+  set_attr<64, true, false, true>();
+  set_attr<64, false, false, true>();
+  set_attr<128, false, true, false>();
+  set_attr<128, false, false, false>();
+  done = true;
+}
+
+size_t gemm_partial_floats(int bn, int dual, int tiles, int splits) {
+  if (splits <= 1) return 0;
+  return static_cast<size_t>(splits) * tiles * (dual ? 2 : 1) * bn * 128;
+}
+
+cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
+  const bool da = g.a1 != nullptr, db = g.b1 != nullptr;
+  if (da && db) return cudaErrorInvalidValue;
+  if (g.args.swap) {
+    if (db) return cudaErrorInvalidValue;
+    switch (g.bn) {
+      case 16: return da ? launch_one<16, true, false, true>(g, stream) : launch_one<16, false, false, true>(g, stream);
+      case 32: return da ? launch_one<32, true, false, true>(g, stream) : launch_one<32, false, false, true>(g, stream);
+      case 64: return da ? launch_one<64, true, false, true>(g, stream) : launch_one<64, false, false, true>(g, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  if (da || g.bn != 128 || g.args.splits != 1) return cudaErrorInvalidValue;
+  return db ? launch_one<128, false, true, false>(g, stream) : launch_one<128, false, false, false>(g, stream);
+}
+
+// ---------------------------------------------------------------- tensor maps
+namespace {
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeFn get_encode() {
+  static EncodeFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeFn>(ptr);
+  }
+  return fn;
+}
+}  // namespace
+
+bool encode_tmap_bf16(CUtensorMap* map, const void* base, uint64_t k, uint64_t rows, uint64_t layers,
+                      uint32_t box_rows) {
+  EncodeFn fn = get_encode();
+  if (!fn || !base || (reinterpret_cast<uintptr_t>(base) & 15) || (k * 2) % 16 != 0 || box_rows == 0 ||
+      box_rows > 256)
+    return false;
+  const cuuint32_t rank = layers > 0 ? 3 : 2;
+  cuuint64_t dims[3] = {k, rows, layers > 0 ? layers : 1};
+  cuuint64_t strides[2] = {k * 2, k * 2 * rows};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(kBoxK), box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace fl

@@ -1,0 +1,70 @@
+// fl_internal.h -- declarations shared by the library's translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+namespace fl {
+
+// ------------------------------------------------------------------ GEMM
+// D = A * B^T on tcgen05 (bf16 operands, fp32 accumulate in TMEM).  A and B
+// are K-major bf16 tiles streamed by TMA: A boxes are 128 rows x 64, B boxes
+// BN rows x 64.  The accumulator row is an A row and its column a B row.
+//   swap = 1: A = weights (row = output feature), B = tokens (<= BN of them).
+//   swap = 0: A = tokens, B = weights (BN = 128 features per tile).
+enum Epi : int {
+  kEpiStore = 0,   // out[tok * ldo + feat] = acc
+  kEpiResid = 1,   // h[row(tok) * ldh + feat] += scale * acc, row(tok) = idx ? idx[tok] : tok
+  kEpiSwiglu = 2,  // act[tok * ld_act + feat] = bf16(silu(acc0) * acc1)
+};
+
+struct GemmArgs {
+  int k_chunks;   // ceil(K / 64)
+  int splits;     // split-K factor (grid.z); > 1 only with swap = 1
+  int a_z, b_z;   // layer coordinate for 3-D (layer-stacked) tensor maps
+  int swap;
+  int epi;
+  int n_feat;     // valid output features
+  int n_tok;      // valid tokens
+  float* out;
+  int ldo;
+  float* h;
+  const int* idx;
+  float scale;
+  int ldh;
+  uint16_t* act;
+  int ld_act;
+  float* partial;   // split-K scratch: splits * grid.x * NACC * BN * 128 fp32
+  int* counters;    // one per grid.x tile; zero between launches
+  int* status;
+};
+
+struct GemmLaunch {
+  const CUtensorMap* a0;
+  const CUtensorMap* a1;   // second A operand (dual, swap: gate / up weights) or nullptr
+  const CUtensorMap* b0;
+  const CUtensorMap* b1;   // second B operand (dual, normal: gate / up weights) or nullptr
+  int bn;                  // 16, 32, 64 (swap) or 128 (normal)
+  int a_3d, b_3d;          // operand maps are layer-stacked (rank 3)
+  dim3 grid;
+  GemmArgs args;
+};
+
+cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream);
+// Largest split-K scratch (floats) one launch with these sizes may use.
+size_t gemm_partial_floats(int bn, int dual, int tiles, int splits);
+
+// Tensor map over a bf16 matrix [layers][rows][k] (rank 3 when layers > 0,
+// else [rows][k] rank 2), 128-byte swizzle, box 64 x box_rows (x 1).
+bool encode_tmap_bf16(CUtensorMap* map, const void* base, uint64_t k, uint64_t rows, uint64_t layers,
+                      uint32_t box_rows);
+
+// ------------------------------------------------------------------ other kernels
+struct SelectSeg;  // fwd
+
+cudaError_t launch_topk(const float* keys, int n_seg, int n, int k, int32_t* idx, cudaStream_t s);
+cudaError_t launch_quantize_rows(const float* r, int rows, int width, int g, int bits, uint8_t* codes,
+                                 uint16_t* scales, cudaStream_t s);
+
+}  // namespace fl

@@ -1,0 +1,1090 @@
+// fl_kernels.cu -- every step of the lazy-update looped step except the GEMMs:
+// pre-norm gather, RoPE + KV store / residual quantise, top-k selection,
+// decode and prefill attention, delta-score column keys, sparse-column
+// correction, and the per-token change keys.  Method: "FlashLoop: Fast and
+// Memory-Efficient Looped Transformers via Lazy Updates" (abstract).
+#include "fl_cache.cuh"
+#include "fl_kernels.h"
+
+namespace fl {
+
+// ============================================================================
+// block helpers
+// ============================================================================
+
+// Exclusive prefix sum over the block (blockDim.x multiple of 32, <= 1024).
+// Returns the exclusive prefix of v; *total receives the block total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* total, int* warp_buf /*[33]*/) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_buf[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    int t = lane < nw ? warp_buf[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    if (lane < nw) warp_buf[lane] = t;  // inclusive warp totals
+    if (lane == 31) warp_buf[32] = t;
+  }
+  __syncthreads();
+  const int base = w > 0 ? warp_buf[w - 1] : 0;
+  *total = warp_buf[32];
+  const int r = base + x - v;
+  __syncthreads();  // warp_buf reusable after return
+  return r;
+}
+
+__device__ __forceinline__ float block_sum(float v, float* buf /*[32]*/) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum(v);
+  if (lane == 0) buf[w] = v;
+  __syncthreads();
+  float t = lane < nw ? buf[lane] : 0.f;
+  t = warp_sum(t);
+  __syncthreads();
+  return t;
+}
+
+// ============================================================================
+// top-k selection: the k largest fp32 keys by (bit pattern desc, index asc),
+// written in ascending index order.  Radix select on 8-bit digits finds the
+// k-th key's bit pattern T; then one ordered pass takes every key above T and
+// the lowest-index keys equal to T.  Deterministic; no atomics in the output.
+// ============================================================================
+
+__device__ int block_topk(const float* __restrict__ keys, int n, int k, int32_t* __restrict__ out) {
+  __shared__ int hist[256];
+  __shared__ int sh_sel, sh_cum;
+  __shared__ int scan_buf[33];
+  if (k >= n) {
+    for (int i = threadIdx.x; i < n; i += blockDim.x) out[i] = i;
+    __syncthreads();
+    return n;
+  }
+  if (k <= 0) return 0;
+  const uint32_t* kb = reinterpret_cast<const uint32_t*>(keys);
+  uint32_t prefix = 0, mask = 0;
+  int k_rem = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint32_t u = kb[i];
+      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 0xFF], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int cum = 0, sel = 0;
+      for (int d = 255; d >= 0; --d) {
+        if (cum + hist[d] >= k_rem) {
+          sel = d;
+          break;
+        }
+        cum += hist[d];
+      }
+      sh_sel = sel;
+      sh_cum = cum;
+    }
+    __syncthreads();
+    k_rem -= sh_cum;
+    prefix |= static_cast<uint32_t>(sh_sel) << shift;
+    mask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  // prefix = bit pattern of the k-th largest key; take k_rem of the keys equal to it.
+  int eq_off = 0, out_off = 0;
+  for (int base = 0; base < n; base += blockDim.x) {
+    const int i = base + threadIdx.x;
+    const uint32_t u = i < n ? kb[i] : 0u;
+    const int gt = (i < n && u > prefix) ? 1 : 0;
+    const int eq = (i < n && u == prefix) ? 1 : 0;
+    int eq_total;
+    const int eq_rank = eq_off + block_exclusive_scan(eq, &eq_total, scan_buf);
+    const int take = gt | (eq & (eq_rank < k_rem ? 1 : 0));
+    int take_total;
+    const int pos = out_off + block_exclusive_scan(take, &take_total, scan_buf);
+    if (take) out[pos] = i;
+    eq_off += eq_total;
+    out_off += take_total;
+  }
+  __syncthreads();
+  return k;
+}
+
+__global__ void __launch_bounds__(1024) k_topk_segments(const float* __restrict__ keys, int n, int k,
+                                                        int32_t* __restrict__ idx) {
+  const int s = blockIdx.x;
+  block_topk(keys + static_cast<size_t>(s) * n, n, k, idx + static_cast<size_t>(s) * (k < n ? k : n));
+}
+
+// Token selection of a lazy loop: top-n_sel over the N keys, or the forced
+// indices when forced_on[0] is set.
+__global__ void __launch_bounds__(1024) k_select_tokens(const float* __restrict__ keys, int N, int n_sel,
+                                                        int32_t* __restrict__ idx, const int* forced_on,
+                                                        const int32_t* __restrict__ forced) {
+  if (forced_on && forced_on[0]) {
+    for (int i = threadIdx.x; i < n_sel; i += blockDim.x) idx[i] = forced[i];
+    return;
+  }
+  block_topk(keys, N, n_sel, idx);
+}
+
+// ============================================================================
+// pre-norm gather: x[i] = bf16(gain * h[idx[i]] / sqrt(mean(h^2) + eps)); rows
+// n..gridDim.x-1 are zero padding for the MMA tile.
+// ============================================================================
+__global__ void __launch_bounds__(256) k_rmsnorm_rows(const float* __restrict__ h, const int* __restrict__ idx,
+                                                      int n, int d, const float* __restrict__ gain, float eps,
+                                                      uint16_t* __restrict__ x) {
+  __shared__ float buf[32];
+  const int i = blockIdx.x;
+  uint16_t* xr = x + static_cast<size_t>(i) * d;
+  if (i >= n) {
+    for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4)
+      *reinterpret_cast<uint2*>(xr + c) = make_uint2(0u, 0u);
+    return;
+  }
+  const int r = idx ? idx[i] : i;
+  const float* hr = h + static_cast<size_t>(r) * d;
+  float ss = 0.f;
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(hr + c);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  const float tot = block_sum(ss, buf);
+  const float inv = rsqrtf(tot / static_cast<float>(d) + eps);
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(hr + c);
+    const float4 gv = *reinterpret_cast<const float4*>(gain + c);
+    const uint32_t lo = f_to_bf16(v.x * inv * gv.x) | (static_cast<uint32_t>(f_to_bf16(v.y * inv * gv.y)) << 16);
+    const uint32_t hi = f_to_bf16(v.z * inv * gv.z) | (static_cast<uint32_t>(f_to_bf16(v.w * inv * gv.w)) << 16);
+    *reinterpret_cast<uint2*>(xr + c) = make_uint2(lo, hi);
+  }
+}
+
+// ============================================================================
+// residual quantiser of one group, lane-distributed: the group is GL = g/EPL
+// consecutive lanes.  s = fp16_RU(fp32(absmax / qmax)) (0 if absmax is 0),
+// code = clamp(rint(fp32(r / s)), -qmax, qmax), ties to even.
+// Returns the lane's codes and the group's fp16 scale bits.
+// ============================================================================
+template <int EPL>
+__device__ __forceinline__ uint16_t quantize_lane(const float* r, int g, int bits, int* code) {
+  const int GL = g / EPL;
+  float am = 0.f;
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) am = fmaxf(am, fabsf(r[e]));
+  for (int o = GL >> 1; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const int qm = (1 << (bits - 1)) - 1;
+  const __half sh = __float2half_ru(__fdiv_rn(am, static_cast<float>(qm)));
+  const float s = __half2float(sh);
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) {
+    int c = 0;
+    if (s > 0.f) {
+      c = __float2int_rn(__fdiv_rn(r[e], s));
+      c = c > qm ? qm : (c < -qm ? -qm : c);
+    }
+    code[e] = c;
+  }
+  return __half_as_ushort(sh);
+}
+
+// Pack the lane's codes (two's complement, element order low bits first) and
+// store them into a packed row; for EPL=2 with 2-bit codes two lanes share a byte.
+template <int EPL>
+__device__ __forceinline__ void store_lane_codes(uint8_t* row, int bits, int lane, const int* c) {
+  if (EPL == 4) {
+    if (bits == 4) {
+      const uint32_t u = (c[0] & 0xF) | ((c[1] & 0xF) << 4) | ((c[2] & 0xF) << 8) | ((c[3] & 0xF) << 12);
+      *reinterpret_cast<uint16_t*>(row + lane * 2) = static_cast<uint16_t>(u);
+    } else {
+      row[lane] = static_cast<uint8_t>((c[0] & 3) | ((c[1] & 3) << 2) | ((c[2] & 3) << 4) | ((c[3] & 3) << 6));
+    }
+  } else {
+    if (bits == 4) {
+      row[lane] = static_cast<uint8_t>((c[0] & 0xF) | ((c[1] & 0xF) << 4));
+    } else {
+      const uint32_t nib = (c[0] & 3) | ((c[1] & 3) << 2);
+      const uint32_t other = __shfl_down_sync(0xffffffffu, nib, 1);
+      if ((lane & 1) == 0) row[lane >> 1] = static_cast<uint8_t>(nib | (other << 4));
+    }
+  }
+}
+
+template <int EPL>
+__global__ void __launch_bounds__(128) k_quantize_rows(const float* __restrict__ r, int rows, int width, int g,
+                                                       int bits, uint8_t* __restrict__ codes,
+                                                       uint16_t* __restrict__ scales) {
+  const int warp_global = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  const int chunks = width / (32 * EPL);
+  if (warp_global >= rows * chunks) return;
+  const int row = warp_global / chunks, ch = warp_global % chunks;
+  const float* src = r + static_cast<size_t>(row) * width + ch * 32 * EPL + lane * EPL;
+  float v[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) v[e] = src[e];
+  int c[EPL];
+  const uint16_t s = quantize_lane<EPL>(v, g, bits, c);
+  uint8_t* crow = codes + (static_cast<size_t>(row) * width + ch * 32 * EPL) * bits / 8;
+  store_lane_codes<EPL>(crow, bits, lane, c);
+  const int GL = g / EPL;
+  if ((lane % GL) == 0) scales[static_cast<size_t>(row) * (width / g) + (ch * 32 * EPL) / g + lane / GL] = s;
+}
+
+// ============================================================================
+// RoPE + KV store / residual quantise (one warp per (GEMM row, head)).
+//   q heads : rotate, write q_cur (and q_last at loop 1 of the lazy path)
+//   k heads : rotate; v heads: as is.  Then
+//     dense   : store bf16 into this loop's own KV
+//     lazy l=1: store bf16 base; zero the residual rows of loops 2..K
+//     lazy l>1: r = kv - reconstructed(loop l-1); quantise; store codes+scale
+// ============================================================================
+template <int EPL>
+__global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
+  const int lane = threadIdx.x & 31;
+  const int item = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int heads = a.H + 2 * a.Hkv;
+  if (item >= a.n * heads) return;
+  const int i = item / heads, hh = item % heads;
+  const int tok = a.idx ? a.idx[i] : i;
+  const int b = a.seq[tok], t = a.pos[tok];
+  const int hd = a.hd, half = hd / 2;
+  const float* src = a.qkv + static_cast<size_t>(i) * a.ldq + static_cast<size_t>(hh) * hd + lane * EPL;
+  float x[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) x[e] = src[e];
+  const bool is_v = hh >= a.H + a.Hkv;
+  if (!is_v) {
+    float y[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) y[e] = __shfl_xor_sync(0xffffffffu, x[e], 16);
+    const int ai = (lane & 15) * EPL;
+    const float* cs = a.rope_cos + static_cast<size_t>(t) * half + ai;
+    const float* sn = a.rope_sin + static_cast<size_t>(t) * half + ai;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) x[e] = lane < 16 ? x[e] * cs[e] - y[e] * sn[e] : x[e] * cs[e] + y[e] * sn[e];
+  }
+  if (hh < a.H) {
+    float* dq = a.q_cur + (static_cast<size_t>(i) * a.H + hh) * hd + lane * EPL;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) dq[e] = x[e];
+    if (a.lazy && a.loop == 1 && a.q_last) {
+      float* ql = a.q_last + (static_cast<size_t>(tok) * a.H + hh) * hd + lane * EPL;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) ql[e] = x[e];
+    }
+    return;
+  }
+  const int kv = is_v ? 1 : 0;
+  const int gk = is_v ? hh - a.H - a.Hkv : hh - a.H;
+  const CacheView& cv = a.cv;
+  if (!a.lazy || a.loop == 1) {
+    uint16_t* dst = (a.lazy ? cv.base_row(a.j, kv, b, gk, t) : cv.dense_row(a.j, a.loop, kv, b, gk, t)) + lane * EPL;
+    if (EPL == 4) {
+      const uint32_t lo = f_to_bf16(x[0]) | (static_cast<uint32_t>(f_to_bf16(x[1])) << 16);
+      const uint32_t hi = f_to_bf16(x[2]) | (static_cast<uint32_t>(f_to_bf16(x[3])) << 16);
+      *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
+    } else {
+      *reinterpret_cast<uint32_t*>(dst) = f_to_bf16(x[0]) | (static_cast<uint32_t>(f_to_bf16(x[1])) << 16);
+    }
+    if (a.lazy) {
+      const int rb = static_cast<int>(cv.row_bytes_codes());
+      const int ns = hd / cv.g;
+      for (int l = 2; l <= cv.K; ++l) {
+        uint8_t* cr = cv.code_row(a.j, l, kv, b, gk, t);
+        for (int o = lane; o < rb; o += 32) cr[o] = 0;
+        uint16_t* sr = cv.scale_row(a.j, l, kv, b, gk, t);
+        if (lane < ns) sr[lane] = 0;
+      }
+    }
+    return;
+  }
+  float prev[EPL];
+  chain_lane<EPL>(cv, a.j, kv, b, gk, t, a.loop - 1, lane, prev);
+  float r[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) r[e] = __fsub_rn(x[e], prev[e]);
+  int c[EPL];
+  const uint16_t s = quantize_lane<EPL>(r, cv.g, cv.bits, c);
+  store_lane_codes<EPL>(cv.code_row(a.j, a.loop, kv, b, gk, t), cv.bits, lane, c);
+  const int GL = cv.g / EPL;
+  if ((lane % GL) == 0) cv.scale_row(a.j, a.loop, kv, b, gk, t)[lane / GL] = s;
+}
+
+// ============================================================================
+// decode attention over one cache (lazy base at loop 1, or the dense
+// baseline's own per-loop KV): grid (n*Hkv, splits); each CTA handles the
+// group's query heads over one column range, 64-column tiles staged in
+// shared memory; the last CTA of a (token, KV head) merges the splits.
+// ============================================================================
+constexpr int kDecTile = 64;
+constexpr int kDecPad = 8;  // bf16 elements of padding per staged row
+
+template <int HD>
+__global__ void __launch_bounds__(128) k_attn_decode(const AttnDecArgs a) {
+  constexpr int RS = HD + kDecPad;                 // staged row stride (bf16)
+  constexpr int GMAX = 8;
+  __shared__ __align__(16) uint16_t Ks[kDecTile * RS];
+  __shared__ __align__(16) uint16_t Vs[kDecTile * RS];
+  __shared__ float Qs[GMAX * HD];
+  __shared__ float S[GMAX][kDecTile];
+  __shared__ float m_run[GMAX], l_run[GMAX], alpha[GMAX];
+  __shared__ int is_last;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv, sp = blockIdx.y;
+  const int grp = a.H / a.Hkv;
+  const int tok = a.idx ? a.idx[i] : i;
+  const int b = a.seq[tok], P = a.pos[tok];
+  const int c_begin = sp * a.split_len;
+  const int c_end = min(c_begin + a.split_len, P + 1);
+  const CacheView& cv = a.cv;
+
+  for (int e = tid; e < grp * HD; e += 128)
+    Qs[e] = a.q_cur[(static_cast<size_t>(i) * a.H + g * grp) * HD + e];
+  if (tid < GMAX) {
+    m_run[tid] = -INFINITY;
+    l_run[tid] = 0.f;
+  }
+  // thread -> (output dim d, head slot) for the PV accumulation
+  constexpr int HS = 128 / HD;                  // head slots: 1 (hd 128) or 2 (hd 64)
+  const int d = tid % HD, hslot = tid / HD;
+  float acc[GMAX];
+#pragma unroll
+  for (int h = 0; h < GMAX; ++h) acc[h] = 0.f;
+  __syncthreads();
+
+  for (int c0 = c_begin; c0 < c_end; c0 += kDecTile) {
+    const int nc = min(kDecTile, c_end - c0);
+    // stage K and V rows (16-byte chunks)
+    constexpr int CH = HD / 8;  // 16-byte chunks per row
+    for (int e = tid; e < nc * CH; e += 128) {
+      const int r = e / CH, cc = e % CH;
+      const uint16_t* kr = a.dense ? cv.dense_row(a.j, a.loop, 0, b, g, c0 + r) : cv.base_row(a.j, 0, b, g, c0 + r);
+      const uint16_t* vr = a.dense ? cv.dense_row(a.j, a.loop, 1, b, g, c0 + r) : cv.base_row(a.j, 1, b, g, c0 + r);
+      *reinterpret_cast<uint4*>(&Ks[r * RS + cc * 8]) = *reinterpret_cast<const uint4*>(kr + cc * 8);
+      *reinterpret_cast<uint4*>(&Vs[r * RS + cc * 8]) = *reinterpret_cast<const uint4*>(vr + cc * 8);
+    }
+    __syncthreads();
+    // scores: thread -> column tid % 64, heads tid/64, tid/64 + 2, ...
+    {
+      const int c = tid % kDecTile, h0 = tid / kDecTile;
+      for (int h = h0; h < grp; h += 2) {
+        float s = -INFINITY;
+        if (c < nc) {
+          float dot = 0.f;
+          const uint16_t* kr = &Ks[c * RS];
+          const float* q = &Qs[h * HD];
+#pragma unroll 8
+          for (int e = 0; e < HD; e += 8) {
+            const uint4 u = *reinterpret_cast<const uint4*>(kr + e);
+            dot += q[e + 0] * bf16_to_f(u.x & 0xFFFF) + q[e + 1] * bf16_to_f(u.x >> 16);
+            dot += q[e + 2] * bf16_to_f(u.y & 0xFFFF) + q[e + 3] * bf16_to_f(u.y >> 16);
+            dot += q[e + 4] * bf16_to_f(u.z & 0xFFFF) + q[e + 5] * bf16_to_f(u.z >> 16);
+            dot += q[e + 6] * bf16_to_f(u.w & 0xFFFF) + q[e + 7] * bf16_to_f(u.w >> 16);
+          }
+          s = dot * a.tau;
+        }
+        S[h][c] = s;
+      }
+    }
+    __syncthreads();
+    // online softmax per head: warp w handles heads w, w+4
+    for (int h = warp; h < grp; h += 4) {
+      const float s0 = S[h][lane], s1 = S[h][lane + 32];
+      const float tmax = warp_max(fmaxf(s0, s1));
+      const float mnew = fmaxf(m_run[h], tmax);
+      const float p0 = s0 == -INFINITY ? 0.f : expf(s0 - mnew);
+      const float p1 = s1 == -INFINITY ? 0.f : expf(s1 - mnew);
+      const float psum = warp_sum(p0 + p1);
+      S[h][lane] = p0;
+      S[h][lane + 32] = p1;
+      __syncwarp();
+      if (lane == 0) {
+        const float al = m_run[h] == -INFINITY ? 0.f : expf(m_run[h] - mnew);
+        alpha[h] = al;
+        l_run[h] = l_run[h] * al + psum;
+        m_run[h] = mnew;
+      }
+    }
+    __syncthreads();
+    for (int h = hslot; h < grp; h += HS) {
+      float sacc = acc[h] * alpha[h];
+      for (int c = 0; c < nc; ++c) sacc += S[h][c] * bf16_to_f(Vs[c * RS + d]);
+      acc[h] = sacc;
+    }
+    __syncthreads();
+  }
+  // write this split's partial (m, l, unnormalised o)
+  const size_t pbase = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits + sp;
+  for (int h = hslot; h < grp; h += HS) a.part_o[(pbase * GMAX + h) * HD + d] = acc[h];
+  if (tid < grp) {
+    a.part_ml[(pbase * GMAX + tid) * 2 + 0] = m_run[tid];
+    a.part_ml[(pbase * GMAX + tid) * 2 + 1] = l_run[tid];
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int old = atomicAdd(&a.counters[i * a.Hkv + g], 1);
+    is_last = (old == a.n_splits - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const size_t q0 = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits;
+  for (int h = hslot; h < grp; h += HS) {
+    float M = -INFINITY;
+    for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, __ldcg(&a.part_ml[((q0 + s) * GMAX + h) * 2]));
+    float L = 0.f, o = 0.f;
+    for (int s = 0; s < a.n_splits; ++s) {
+      const float ms = __ldcg(&a.part_ml[((q0 + s) * GMAX + h) * 2]);
+      if (ms == -INFINITY) continue;
+      const float w = expf(ms - M);
+      L += w * __ldcg(&a.part_ml[((q0 + s) * GMAX + h) * 2 + 1]);
+      o += w * __ldcg(&a.part_o[((q0 + s) * GMAX + h) * HD + d]);
+    }
+    const int hq = g * grp + h;
+    const float ov = o / L;
+    if (a.o_state) a.o_state[(static_cast<size_t>(tok) * a.H + hq) * HD + d] = ov;
+    a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + d] = f_to_bf16(ov);
+    if (d == 0 && a.lse_state) a.lse_state[static_cast<size_t>(tok) * a.H + hq] = M + logf(L);
+  }
+  if (tid == 0) a.counters[i * a.Hkv + g] = 0;
+}
+
+// ============================================================================
+// prefill causal attention (loop 1 of the lazy path; every loop of the dense
+// baseline).  grid (ceil(T/64), H, B); 256 threads: thread (r = tid/4, c4 =
+// tid%4) owns query row r, 16 score columns and HD/4 output dims.
+// ============================================================================
+template <int HD>
+__global__ void __launch_bounds__(256) k_attn_prefill(const AttnPreArgs a) {
+  constexpr int BQ = 64, BK = 64;
+  constexpr int RS = HD + kDecPad;
+  constexpr int DV = HD / 4;
+  extern __shared__ __align__(16) uint8_t sm[];
+  float* Qs = reinterpret_cast<float*>(sm);                         // [BQ][HD+1]
+  float* Ps = Qs + BQ * (HD + 1);                                   // [BQ][BK+1]
+  uint16_t* Ks = reinterpret_cast<uint16_t*>(Ps + BQ * (BK + 1));   // [BK][RS]
+  uint16_t* Vs = Ks + BK * RS;                                      // [BK][RS]
+
+  const int tid = threadIdx.x;
+  const int qb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int grp = a.H / a.Hkv, g = h / grp;
+  const int T = a.T;
+  const int r = tid >> 2, c4 = tid & 3;
+  const int q0 = qb * BQ;
+  const int qpos = q0 + r;
+  const CacheView& cv = a.cv;
+
+  for (int e = tid; e < BQ * HD; e += 256) {
+    const int rr = e / HD, dd = e % HD;
+    const int qp = q0 + rr;
+    Qs[rr * (HD + 1) + dd] = qp < T ? a.q_cur[((static_cast<size_t>(b) * T + qp) * a.H + h) * HD + dd] : 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  float acc[DV];
+#pragma unroll
+  for (int e = 0; e < DV; ++e) acc[e] = 0.f;
+  const int kt_end = min(T, q0 + BQ);
+  for (int k0 = 0; k0 < kt_end; k0 += BK) {
+    __syncthreads();
+    constexpr int CH = HD / 8;
+    for (int e = tid; e < BK * CH; e += 256) {
+      const int rr = e / CH, cc = e % CH;
+      const int kp = k0 + rr;
+      uint4 ku = make_uint4(0, 0, 0, 0), vu = make_uint4(0, 0, 0, 0);
+      if (kp < T) {
+        const uint16_t* kr = a.dense ? cv.dense_row(a.j, a.loop, 0, b, g, kp) : cv.base_row(a.j, 0, b, g, kp);
+        const uint16_t* vr = a.dense ? cv.dense_row(a.j, a.loop, 1, b, g, kp) : cv.base_row(a.j, 1, b, g, kp);
+        ku = *reinterpret_cast<const uint4*>(kr + cc * 8);
+        vu = *reinterpret_cast<const uint4*>(vr + cc * 8);
+      }
+      *reinterpret_cast<uint4*>(&Ks[rr * RS + cc * 8]) = ku;
+      *reinterpret_cast<uint4*>(&Vs[rr * RS + cc * 8]) = vu;
+    }
+    __syncthreads();
+    float s[16];
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int c = c4 * 16 + j;
+      const int kp = k0 + c;
+      float dot = 0.f;
+      const uint16_t* kr = &Ks[c * RS];
+      const float* q = &Qs[r * (HD + 1)];
+#pragma unroll 8
+      for (int e = 0; e < HD; e += 2) {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(kr + e);
+        dot += q[e] * bf16_to_f(u & 0xFFFF) + q[e + 1] * bf16_to_f(u >> 16);
+      }
+      s[j] = (kp <= qpos && kp < T && qpos < T) ? dot * a.tau : -INFINITY;
+      tmax = fmaxf(tmax, s[j]);
+    }
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
+    tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
+    const float mnew = fmaxf(m, tmax);
+    float psum = 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float p = s[j] == -INFINITY ? 0.f : expf(s[j] - mnew);
+      Ps[r * (BK + 1) + c4 * 16 + j] = p;
+      psum += p;
+    }
+    psum += __shfl_xor_sync(0xffffffffu, psum, 1);
+    psum += __shfl_xor_sync(0xffffffffu, psum, 2);
+    const float al = m == -INFINITY ? 0.f : expf(m - mnew);
+    l = l * al + psum;
+    m = mnew;
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < DV; ++e) acc[e] *= al;
+    for (int c = 0; c < BK; ++c) {
+      const float p = Ps[r * (BK + 1) + c];
+      const uint16_t* vr = &Vs[c * RS + c4 * DV];
+#pragma unroll
+      for (int e = 0; e < DV; e += 2) {
+        const uint32_t u = *reinterpret_cast<const uint32_t*>(vr + e);
+        acc[e] += p * bf16_to_f(u & 0xFFFF);
+        acc[e + 1] += p * bf16_to_f(u >> 16);
+      }
+    }
+  }
+  if (qpos >= T) return;
+  const size_t tok = static_cast<size_t>(b) * T + qpos;
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int e = 0; e < DV; ++e) {
+    const int dd = c4 * DV + e;
+    const float ov = acc[e] * inv;
+    if (a.o_state) a.o_state[(tok * a.H + h) * HD + dd] = ov;
+    a.o_bf16[tok * a.H * HD + static_cast<size_t>(h) * HD + dd] = f_to_bf16(ov);
+  }
+  if (c4 == 0 && a.lse_state) a.lse_state[tok * a.H + h] = m + logf(l);
+}
+
+// ============================================================================
+// per-call token bookkeeping
+// ============================================================================
+__global__ void k_setup_call(int N, int mode_decode, int T, int tiles_per_seq, int q_tile,
+                             const int* __restrict__ seq_len, int* seq, int* pos, int* tile, int* last,
+                             int n_tiles, int* has_c) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < N) {
+    if (mode_decode) {
+      seq[t] = t;
+      pos[t] = seq_len[t];
+      tile[t] = t;
+    } else {
+      const int b = t / T, p = t % T;
+      seq[t] = b;
+      pos[t] = p;
+      tile[t] = b * tiles_per_seq + p / q_tile;
+    }
+    last[t] = 1;
+  }
+  if (t < n_tiles) has_c[t] = 0;
+}
+
+__global__ void k_set_lens(int B, int* seq_len, int add, int value) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) seq_len[b] = add ? seq_len[b] + 1 : value;
+}
+
+// slot of each token in the selection (or -1), and the snapshot of selected rows
+__global__ void k_after_select(const int32_t* __restrict__ idx, int n_sel, int N, int d, int* sel_slot,
+                               const float* __restrict__ h, float* __restrict__ h_snap, int slot_blocks) {
+  if (static_cast<int>(blockIdx.x) < slot_blocks) {
+    const int t = blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= N) return;
+    int lo = 0, hi = n_sel;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (idx[mid] < t) lo = mid + 1; else hi = mid;
+    }
+    sel_slot[t] = (lo < n_sel && idx[lo] == t) ? lo : -1;
+    return;
+  }
+  const int row = blockIdx.x - slot_blocks;
+  if (row >= n_sel) return;
+  const float* src = h + static_cast<size_t>(idx[row]) * d;
+  float* dst = h_snap + static_cast<size_t>(row) * d;
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4)
+    *reinterpret_cast<float4*>(dst + c) = *reinterpret_cast<const float4*>(src + c);
+}
+
+// Change keys: loop 1 -> ||h - h_in||^2 for every token; loop l -> ||h - h_snap||^2
+// for selected tokens and 0 for carried ones; selected tokens record last = l and
+// mark their query tile as having a column set.
+__global__ void __launch_bounds__(128) k_change_keys(const float* __restrict__ h, const float* __restrict__ ref,
+                                                     const int* __restrict__ sel_slot, int N, int d, int loop,
+                                                     float* __restrict__ key, int* last, const int* tile,
+                                                     int* has_c) {
+  const int t = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (t >= N) return;
+  const float* other;
+  if (loop == 1) {
+    other = ref + static_cast<size_t>(t) * d;
+  } else {
+    const int s = sel_slot[t];
+    if (s < 0) {
+      if (lane == 0) key[t] = 0.f;
+      return;
+    }
+    other = ref + static_cast<size_t>(s) * d;
+  }
+  const float* hr = h + static_cast<size_t>(t) * d;
+  float acc = 0.f;
+  for (int c = lane * 4; c < d; c += 128) {
+    const float4 x = *reinterpret_cast<const float4*>(hr + c);
+    const float4 y = *reinterpret_cast<const float4*>(other + c);
+    const float a0 = x.x - y.x, a1 = x.y - y.y, a2 = x.z - y.z, a3 = x.w - y.w;
+    acc += a0 * a0 + a1 * a1 + a2 * a2 + a3 * a3;
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) {
+    key[t] = acc;
+    if (loop > 1) {
+      last[t] = loop;
+      has_c[tile[t]] = 1;
+    }
+  }
+}
+
+// ============================================================================
+// query-tile plan of a lazy loop: the selected tokens (ascending) grouped by
+// query tile; tiles recomputed for the first time need a column set.
+// ============================================================================
+__global__ void __launch_bounds__(1024) k_plan_tiles(const int32_t* __restrict__ idx, int n_sel,
+                                                     const int* __restrict__ tile, const int* __restrict__ has_c,
+                                                     TilePlan plan) {
+  __shared__ int scan_buf[33];
+  __shared__ int base_p, base_need;
+  if (threadIdx.x == 0) {
+    base_p = 0;
+    base_need = 0;
+  }
+  __syncthreads();
+  for (int c0 = 0; c0 < n_sel; c0 += blockDim.x) {
+    const int i = c0 + threadIdx.x;
+    int tl = -1, start = 0, need = 0;
+    if (i < n_sel) {
+      tl = tile[idx[i]];
+      start = (i == 0 || tile[idx[i - 1]] != tl) ? 1 : 0;
+      need = start && !has_c[tl];
+    }
+    int tot_p, tot_n;
+    const int p = base_p + block_exclusive_scan(start, &tot_p, scan_buf);
+    const int q = base_need + block_exclusive_scan(need, &tot_n, scan_buf);
+    if (start) {
+      plan.tile[p] = tl;
+      plan.qb[p] = i;
+      if (p > 0) plan.qe[p - 1] = i;
+    }
+    if (need) plan.need[q] = p;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      base_p += tot_p;
+      base_need += tot_n;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    if (base_p > 0) plan.qe[base_p - 1] = n_sel;
+    plan.counts[0] = base_p;
+    plan.counts[1] = base_need;
+  }
+}
+
+// ============================================================================
+// delta-score column keys of tiles recomputed for the first time:
+//   key[k] = max over the tile's selected queries i (with k <= pos(i)) and the
+//   group's heads h of | tau*(q_l[i,h] . K_l[k] - q_last[i,h] . K_base[k]) |
+// ("attention-output differences are dominated by a sparse and stable subset
+// of key columns", "FlashLoop ...", abstract).  grid (max_need*Hkv, chunks).
+// ============================================================================
+template <int HD, int EPL>
+__global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
+  constexpr int CC = 64;      // columns per CTA
+  constexpr int QP = 16;      // (query, head) pairs staged per batch
+  extern __shared__ __align__(16) uint8_t sm[];
+  float* Kn = reinterpret_cast<float*>(sm);      // [CC][HD+1]
+  float* Kb = Kn + CC * (HD + 1);                // [CC][HD+1]
+  float* Qn = Kb + CC * (HD + 1);                // [QP][HD]
+  float* Qo = Qn + QP * HD;                      // [QP][HD]
+  float* Mx = Qo + QP * HD;                      // [4][CC]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int seg = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
+  if (seg >= a.plan.counts[1]) return;
+  const int p = a.plan.need[seg];
+  const int qb = a.plan.qb[p], qe = a.plan.qe[p];
+  const int tok_last = a.idx[qe - 1];
+  const int b = a.seq[tok_last], maxpos = a.pos[tok_last];
+  const int c0 = blockIdx.y * CC;
+  if (c0 > maxpos) return;
+  const int nc = min(CC, maxpos + 1 - c0);
+  const int grp = a.H / a.Hkv;
+  const CacheView& cv = a.cv;
+  // reconstruct K of loop l and the base for this column chunk
+  for (int rr = warp; rr < nc; rr += 8) {
+    float lo[EPL], hi[EPL];
+    chain_lane2<EPL>(cv, a.j, 0, b, g, c0 + rr, 1, a.loop, lane, lo, hi);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      Kb[rr * (HD + 1) + lane * EPL + e] = lo[e];
+      Kn[rr * (HD + 1) + lane * EPL + e] = hi[e];
+    }
+  }
+  const int c = tid % CC, slot = tid / CC;
+  float best = 0.f;
+  const int npairs = (qe - qb) * grp;
+  for (int pb = 0; pb < npairs; pb += QP) {
+    __syncthreads();
+    const int np = min(QP, npairs - pb);
+    for (int e = tid; e < np * HD; e += 256) {
+      const int pr = e / HD, dd = e % HD;
+      const int qi = qb + (pb + pr) / grp, hh = g * grp + (pb + pr) % grp;
+      const int tk = a.idx[qi];
+      Qn[pr * HD + dd] = a.q_cur[(static_cast<size_t>(qi) * a.H + hh) * HD + dd];
+      Qo[pr * HD + dd] = a.q_last[(static_cast<size_t>(tk) * a.H + hh) * HD + dd];
+    }
+    __syncthreads();
+    if (c < nc) {
+      for (int pr = slot; pr < np; pr += 4) {
+        const int qi = qb + (pb + pr) / grp;
+        if (a.pos[a.idx[qi]] < c0 + c) continue;
+        float dn = 0.f, db = 0.f;
+        const float* kn = &Kn[c * (HD + 1)];
+        const float* kb = &Kb[c * (HD + 1)];
+        const float* qn = &Qn[pr * HD];
+        const float* qo = &Qo[pr * HD];
+#pragma unroll 8
+        for (int e = 0; e < HD; ++e) {
+          dn += kn[e] * qn[e];
+          db += kb[e] * qo[e];
+        }
+        best = fmaxf(best, fabsf(a.tau * (dn - db)));
+      }
+    }
+  }
+  Mx[slot * CC + c] = best;
+  __syncthreads();
+  if (tid < nc) {
+    const float v = fmaxf(fmaxf(Mx[tid], Mx[CC + tid]), fmaxf(Mx[2 * CC + tid], Mx[3 * CC + tid]));
+    a.col_keys[(static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols + c0 + tid] = v;
+  }
+}
+
+// top-c columns of each (tile, KV head) that needs a column set
+__global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
+  const int seg = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
+  if (seg >= a.plan.counts[1]) return;
+  const int p = a.plan.need[seg];
+  const int tl = a.plan.tile[p];
+  const int tok_last = a.idx[a.plan.qe[p] - 1];
+  const int n = a.pos[tok_last] + 1;
+  int32_t* out = a.cols + ((static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g) * a.c;
+  int* nout = a.ncols + (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
+  if (a.forced_on && a.forced_on[0]) {
+    const size_t off = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
+    const int fn = a.forced_ncols[off];
+    for (int e = threadIdx.x; e < fn; e += blockDim.x) out[e] = a.forced_cols[off * a.c + e];
+    if (threadIdx.x == 0) *nout = fn;
+    return;
+  }
+  const int got = block_topk(a.col_keys + (static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols, n, a.c, out);
+  if (threadIdx.x == 0) *nout = got;
+}
+
+// ============================================================================
+// sparse-column correction of (O, lse) for one selected query and KV group:
+//   Mx = max(lse, s_new, s_old) over the query's columns C (k <= pos)
+//   Z' = e^(lse-Mx) - sum_C e^(s_old-Mx) + sum_C e^(s_new-Mx)
+//   N' = e^(lse-Mx) O - sum_C e^(s_old-Mx) V_last + sum_C e^(s_new-Mx) V_l
+//   O = N'/Z', lse = Mx + ln Z', q_last = q_l
+// with s_new = tau q_l.K_l, s_old = tau q_last.K_last.  grid (n_sel*Hkv), 128 threads.
+// ============================================================================
+template <int HD, int EPL>
+__global__ void __launch_bounds__(128) k_correct(const CorrectArgs a) {
+  constexpr int CC = 32;
+  constexpr int GMAX = 8;
+  extern __shared__ __align__(16) uint8_t sm[];
+  float* An = reinterpret_cast<float*>(sm);       // [CC][HD+1] new rows (K then V)
+  float* Ao = An + CC * (HD + 1);                 // [CC][HD+1] old rows
+  float* Qn = Ao + CC * (HD + 1);                 // [GMAX][HD]
+  float* Qo = Qn + GMAX * HD;                     // [GMAX][HD]
+  const int grp = a.H / a.Hkv;
+  float* Sn = Qo + GMAX * HD;                     // [grp][c]
+  float* So = Sn + grp * a.c;                     // [grp][c]
+  __shared__ float mx[GMAX], zz[GMAX], el[GMAX];
+  __shared__ int ncs;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
+  const int tok = a.idx[i];
+  const int b = a.seq[tok], P = a.pos[tok], tl = a.tile[tok];
+  const int m_old = a.last[tok];
+  const CacheView& cv = a.cv;
+  const int32_t* C = a.cols + ((static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g) * a.c;
+  const int ncol = a.ncols[(static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g];
+  if (tid == 0) {
+    int n = 0;
+    while (n < ncol && C[n] <= P) ++n;   // C is ascending
+    ncs = n;
+  }
+  for (int e = tid; e < grp * HD; e += 128) {
+    const int hh = g * grp + e / HD, dd = e % HD;
+    Qn[e] = a.q_cur[(static_cast<size_t>(i) * a.H + hh) * HD + dd];
+    Qo[e] = a.q_last[(static_cast<size_t>(tok) * a.H + hh) * HD + dd];
+  }
+  __syncthreads();
+  const int nc = ncs;
+  // pass 1: scores over C
+  for (int c0 = 0; c0 < nc; c0 += CC) {
+    const int cn = min(CC, nc - c0);
+    for (int rr = warp; rr < cn; rr += 4) {
+      float lo[EPL], hi[EPL];
+      chain_lane2<EPL>(cv, a.j, 0, b, g, C[c0 + rr], m_old, a.loop, lane, lo, hi);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        Ao[rr * (HD + 1) + lane * EPL + e] = lo[e];
+        An[rr * (HD + 1) + lane * EPL + e] = hi[e];
+      }
+    }
+    __syncthreads();
+    {
+      const int cc = tid % CC, hs = tid / CC;
+      if (cc < cn) {
+        for (int h = hs; h < grp; h += 4) {
+          float dn = 0.f, dl = 0.f;
+#pragma unroll 8
+          for (int e = 0; e < HD; ++e) {
+            dn += An[cc * (HD + 1) + e] * Qn[h * HD + e];
+            dl += Ao[cc * (HD + 1) + e] * Qo[h * HD + e];
+          }
+          Sn[h * a.c + c0 + cc] = dn * a.tau;
+          So[h * a.c + c0 + cc] = dl * a.tau;
+        }
+      }
+    }
+    __syncthreads();
+  }
+  // Mx, Z' per head (warp per head)
+  for (int h = warp; h < grp; h += 4) {
+    const size_t so = (static_cast<size_t>(tok) * a.H + g * grp + h);
+    const float L = a.lse_state[so];
+    float m = L;
+    for (int e = lane; e < nc; e += 32) m = fmaxf(m, fmaxf(Sn[h * a.c + e], So[h * a.c + e]));
+    m = warp_max(m);
+    float zs = 0.f;
+    for (int e = lane; e < nc; e += 32) {
+      const float en = expf(Sn[h * a.c + e] - m), eo = expf(So[h * a.c + e] - m);
+      Sn[h * a.c + e] = en;
+      So[h * a.c + e] = eo;
+      zs += en - eo;
+    }
+    zs = warp_sum(zs);
+    if (lane == 0) {
+      const float e0 = expf(L - m);
+      mx[h] = m;
+      el[h] = e0;
+      zz[h] = e0 + zs;
+    }
+  }
+  __syncthreads();
+  // pass 2: values over C
+  constexpr int HS = 128 / HD;
+  const int d = tid % HD, hslot = tid / HD;
+  float acc[GMAX];
+#pragma unroll
+  for (int h = 0; h < GMAX; ++h) acc[h] = 0.f;
+  for (int c0 = 0; c0 < nc; c0 += CC) {
+    const int cn = min(CC, nc - c0);
+    __syncthreads();
+    for (int rr = warp; rr < cn; rr += 4) {
+      float lo[EPL], hi[EPL];
+      chain_lane2<EPL>(cv, a.j, 1, b, g, C[c0 + rr], m_old, a.loop, lane, lo, hi);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        Ao[rr * (HD + 1) + lane * EPL + e] = lo[e];
+        An[rr * (HD + 1) + lane * EPL + e] = hi[e];
+      }
+    }
+    __syncthreads();
+    for (int h = hslot; h < grp; h += HS) {
+      float s = acc[h];
+      for (int cc = 0; cc < cn; ++cc)
+        s += Sn[h * a.c + c0 + cc] * An[cc * (HD + 1) + d] - So[h * a.c + c0 + cc] * Ao[cc * (HD + 1) + d];
+      acc[h] = s;
+    }
+  }
+  __syncthreads();
+  for (int h = hslot; h < grp; h += HS) {
+    const int hq = g * grp + h;
+    const size_t so = static_cast<size_t>(tok) * a.H + hq;
+    const float z = zz[h];
+    if (!(z > 0.f) && a.status) atomicOr(a.status, kErrBadIndex);
+    const float ov = (el[h] * a.o_state[so * HD + d] + acc[h]) / z;
+    a.o_state[so * HD + d] = ov;
+    a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + d] = f_to_bf16(ov);
+    a.q_last[so * HD + d] = Qn[h * HD + d];
+    if (d == 0) a.lse_state[so] = mx[h] + logf(z);
+  }
+}
+
+// ============================================================================
+// cache import helpers
+// ============================================================================
+template <int EPL>
+__global__ void k_pack_codes(const int8_t* __restrict__ src, int rows, int hd, int bits, uint8_t* __restrict__ dst,
+                             size_t dst_row_stride) {
+  const int w = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (w >= rows) return;
+  int c[EPL];
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) c[e] = src[static_cast<size_t>(w) * hd + lane * EPL + e];
+  store_lane_codes<EPL>(dst + static_cast<size_t>(w) * dst_row_stride, bits, lane, c);
+}
+
+// ============================================================================
+// launchers
+// ============================================================================
+cudaError_t launch_topk(const float* keys, int n_seg, int n, int k, int32_t* idx, cudaStream_t s) {
+  k_topk_segments<<<n_seg, 1024, 0, s>>>(keys, n, k, idx);
+  return cudaGetLastError();
+}
+cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* idx, const int* forced_on,
+                                 const int32_t* forced, cudaStream_t s) {
+  k_select_tokens<<<1, 1024, 0, s>>>(keys, N, n_sel, idx, forced_on, forced);
+  return cudaGetLastError();
+}
+cudaError_t launch_quantize_rows(const float* r, int rows, int width, int g, int bits, uint8_t* codes,
+                                 uint16_t* scales, cudaStream_t s) {
+  if (width % 128 == 0) {
+    const int warps = rows * (width / 128);
+    k_quantize_rows<4><<<(warps + 3) / 4, 128, 0, s>>>(r, rows, width, g, bits, codes, scales);
+  } else {
+    const int warps = rows * (width / 64);
+    k_quantize_rows<2><<<(warps + 3) / 4, 128, 0, s>>>(r, rows, width, g, bits, codes, scales);
+  }
+  return cudaGetLastError();
+}
+cudaError_t launch_rmsnorm_rows(const float* h, const int* idx, int n, int n_pad, int d, const float* gain, float eps,
+                                uint16_t* x, cudaStream_t s) {
+  k_rmsnorm_rows<<<n_pad, 256, 0, s>>>(h, idx, n, d, gain, eps, x);
+  return cudaGetLastError();
+}
+cudaError_t launch_qkv_post(const QkvPostArgs& a, cudaStream_t s) {
+  const int warps = a.n * (a.H + 2 * a.Hkv);
+  if (a.hd == 128) k_qkv_post<4><<<(warps + 3) / 4, 128, 0, s>>>(a);
+  else k_qkv_post<2><<<(warps + 3) / 4, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+cudaError_t launch_attn_decode(const AttnDecArgs& a, int n, cudaStream_t s) {
+  dim3 grid(n * a.Hkv, a.n_splits);
+  if (a.hd == 128) k_attn_decode<128><<<grid, 128, 0, s>>>(a);
+  else k_attn_decode<64><<<grid, 128, 0, s>>>(a);
+  return cudaGetLastError();
+}
+size_t attn_prefill_smem(int hd) {
+  return static_cast<size_t>(64) * (hd + 1) * 4 + 64 * 65 * 4 + 2 * 64 * (hd + kDecPad) * 2;
+}
+cudaError_t launch_attn_prefill(const AttnPreArgs& a, int B, cudaStream_t s) {
+  dim3 grid((a.T + 63) / 64, a.H, B);
+  const size_t sm = attn_prefill_smem(a.hd);
+  if (a.hd == 128) {
+    k_attn_prefill<128><<<grid, 256, sm, s>>>(a);
+  } else {
+    k_attn_prefill<64><<<grid, 256, sm, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+cudaError_t launch_setup_call(int N, int decode, int T, int tiles_per_seq, int q_tile, const int* seq_len, int* seq,
+                              int* pos, int* tile, int* last, int n_tiles, int* has_c, cudaStream_t s) {
+  const int n = N > n_tiles ? N : n_tiles;
+  k_setup_call<<<(n + 255) / 256, 256, 0, s>>>(N, decode, T, tiles_per_seq, q_tile, seq_len, seq, pos, tile, last,
+                                               n_tiles, has_c);
+  return cudaGetLastError();
+}
+cudaError_t launch_set_lens(int B, int* seq_len, int add, int value, cudaStream_t s) {
+  k_set_lens<<<(B + 127) / 128, 128, 0, s>>>(B, seq_len, add, value);
+  return cudaGetLastError();
+}
+cudaError_t launch_after_select(const int32_t* idx, int n_sel, int N, int d, int* sel_slot, const float* h,
+                                float* h_snap, cudaStream_t s) {
+  const int slot_blocks = (N + 255) / 256;
+  k_after_select<<<slot_blocks + n_sel, 256, 0, s>>>(idx, n_sel, N, d, sel_slot, h, h_snap, slot_blocks);
+  return cudaGetLastError();
+}
+cudaError_t launch_change_keys(const float* h, const float* ref, const int* sel_slot, int N, int d, int loop,
+                               float* key, int* last, const int* tile, int* has_c, cudaStream_t s) {
+  k_change_keys<<<(N + 3) / 4, 128, 0, s>>>(h, ref, sel_slot, N, d, loop, key, last, tile, has_c);
+  return cudaGetLastError();
+}
+cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, const int* has_c, const TilePlan& p,
+                              cudaStream_t s) {
+  k_plan_tiles<<<1, 1024, 0, s>>>(idx, n_sel, tile, has_c, p);
+  return cudaGetLastError();
+}
+size_t dscore_smem(int hd) {
+  return (static_cast<size_t>(2) * 64 * (hd + 1) + 2 * 16 * hd + 4 * 64) * 4;
+}
+cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s) {
+  dim3 grid(max_need * a.Hkv, max_chunks);
+  const size_t sm = dscore_smem(a.hd);
+  if (a.hd == 128) {
+    k_dscore<128, 4><<<grid, 256, sm, s>>>(a);
+  } else {
+    k_dscore<64, 2><<<grid, 256, sm, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t s) {
+  k_select_cols<<<max_need * a.Hkv, 1024, 0, s>>>(a);
+  return cudaGetLastError();
+}
+size_t correct_smem(int hd, int grp, int c) {
+  return (static_cast<size_t>(2) * 32 * (hd + 1) + 2 * 8 * hd + 2 * static_cast<size_t>(grp) * c) * 4;
+}
+cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
+  const size_t sm = correct_smem(a.hd, a.H / a.Hkv, a.c);
+  if (a.hd == 128) {
+    k_correct<128, 4><<<n_sel * a.Hkv, 128, sm, s>>>(a);
+  } else {
+    k_correct<64, 2><<<n_sel * a.Hkv, 128, sm, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+// Opt every large-shared-memory kernel in to its dynamic shared memory once,
+// outside any stream capture.
+void kernels_init_attrs() {
+  static bool done = false;
+  if (done) return;
+  const int pre128 = static_cast<int>(attn_prefill_smem(128)), pre64 = static_cast<int>(attn_prefill_smem(64));
+  cudaFuncSetAttribute(k_attn_prefill<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, pre128);
+  cudaFuncSetAttribute(k_attn_prefill<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, pre64);
+  cudaFuncSetAttribute(k_dscore<128, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dscore_smem(128)));
+  cudaFuncSetAttribute(k_dscore<64, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dscore_smem(64)));
+  // the correction kernel's score buffers grow with c; allow the device maximum
+  // (configs whose need exceeds it are refused at init)
+  cudaFuncSetAttribute(k_correct<128, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+  cudaFuncSetAttribute(k_correct<64, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
+  done = true;
+}
+
+cudaError_t launch_pack_codes(const int8_t* src, int rows, int hd, int bits, uint8_t* dst, size_t dst_row_stride,
+                              cudaStream_t s) {
+  if (hd == 128) k_pack_codes<4><<<(rows + 3) / 4, 128, 0, s>>>(src, rows, hd, bits, dst, dst_row_stride);
+  else k_pack_codes<2><<<(rows + 3) / 4, 128, 0, s>>>(src, rows, hd, bits, dst, dst_row_stride);
+  return cudaGetLastError();
+}
+
+}  // namespace fl

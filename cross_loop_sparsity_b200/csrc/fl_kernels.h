@@ -1,0 +1,136 @@
+// fl_kernels.h -- argument blocks and launchers of the non-GEMM kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "fl_cache.cuh"
+#include "fl_internal.h"
+
+namespace fl {
+
+struct QkvPostArgs {
+  const float* qkv;   // [n][(H+2Hkv)*hd] fp32, GEMM row order
+  int ldq;
+  const int* idx;     // GEMM row -> call token (nullptr = identity)
+  int n;
+  const int* seq;     // call token -> sequence
+  const int* pos;     // call token -> position
+  int H, Hkv, hd;
+  const float* rope_cos;  // [max_ctx][hd/2]
+  const float* rope_sin;
+  CacheView cv;
+  int j, loop, lazy;
+  float* q_cur;       // [n][H][hd] GEMM order
+  float* q_last;      // [N][H][hd] token order (this layer), written at loop 1
+};
+
+struct AttnDecArgs {
+  const float* q_cur;
+  const int* idx;
+  const int* seq;
+  const int* pos;
+  CacheView cv;
+  int j, loop, dense;
+  int H, Hkv, hd;
+  float tau;
+  int split_len, n_splits;
+  float* part_o;      // [n][Hkv][splits][8][hd]
+  float* part_ml;     // [n][Hkv][splits][8][2]
+  int* counters;      // [n][Hkv], zero between launches
+  float* o_state;     // [N][H][hd] token order (nullptr for the dense baseline)
+  float* lse_state;   // [N][H]
+  uint16_t* o_bf16;   // [n][H*hd] GEMM order
+};
+
+struct AttnPreArgs {
+  const float* q_cur;  // [B*T][H][hd] token order
+  CacheView cv;
+  int j, loop, dense;
+  int T, H, Hkv, hd;
+  float tau;
+  float* o_state;
+  float* lse_state;
+  uint16_t* o_bf16;
+};
+
+struct TilePlan {
+  int* tile;    // [max_tiles] query tile of plan entry p
+  int* qb;      // first / one-past-last index into the selection of its queries
+  int* qe;
+  int* need;    // plan entries whose tile needs a column set
+  int* counts;  // [0] entries, [1] entries needing a column set
+};
+
+struct DScoreArgs {
+  TilePlan plan;
+  const int32_t* idx;
+  const int* seq;
+  const int* pos;
+  const float* q_cur;   // GEMM order
+  const float* q_last;  // token order (this layer)
+  CacheView cv;
+  int j, loop, H, Hkv, hd;
+  float tau;
+  float* col_keys;      // [max_need][Hkv][max_cols]
+  int max_cols;
+};
+
+struct SelColsArgs {
+  TilePlan plan;
+  const int32_t* idx;
+  const int* pos;
+  const float* col_keys;
+  int max_cols, Hkv, c, j, n_tiles;
+  int32_t* cols;        // [M][n_tiles][Hkv][c]
+  int* ncols;           // [M][n_tiles][Hkv]
+  const int* forced_on;
+  const int32_t* forced_cols;
+  const int* forced_ncols;
+};
+
+struct CorrectArgs {
+  const int32_t* idx;
+  const int* seq;
+  const int* pos;
+  const int* tile;
+  const int* last;
+  const float* q_cur;
+  float* q_last;
+  float* o_state;
+  float* lse_state;
+  uint16_t* o_bf16;
+  const int32_t* cols;
+  const int* ncols;
+  CacheView cv;
+  int j, loop, H, Hkv, hd, c, n_tiles;
+  float tau;
+  int* status;
+};
+
+constexpr int kMaxDynSmem = 232448;  // 227 KB: the per-block dynamic shared memory limit of sm_100
+size_t correct_smem(int hd, int grp, int c);
+
+cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* idx, const int* forced_on,
+                                 const int32_t* forced, cudaStream_t s);
+cudaError_t launch_rmsnorm_rows(const float* h, const int* idx, int n, int n_pad, int d, const float* gain, float eps,
+                                uint16_t* x, cudaStream_t s);
+cudaError_t launch_qkv_post(const QkvPostArgs& a, cudaStream_t s);
+cudaError_t launch_attn_decode(const AttnDecArgs& a, int n, cudaStream_t s);
+cudaError_t launch_attn_prefill(const AttnPreArgs& a, int B, cudaStream_t s);
+cudaError_t launch_setup_call(int N, int decode, int T, int tiles_per_seq, int q_tile, const int* seq_len, int* seq,
+                              int* pos, int* tile, int* last, int n_tiles, int* has_c, cudaStream_t s);
+cudaError_t launch_set_lens(int B, int* seq_len, int add, int value, cudaStream_t s);
+cudaError_t launch_after_select(const int32_t* idx, int n_sel, int N, int d, int* sel_slot, const float* h,
+                                float* h_snap, cudaStream_t s);
+cudaError_t launch_change_keys(const float* h, const float* ref, const int* sel_slot, int N, int d, int loop,
+                               float* key, int* last, const int* tile, int* has_c, cudaStream_t s);
+cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, const int* has_c, const TilePlan& p,
+                              cudaStream_t s);
+cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s);
+cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t s);
+cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s);
+cudaError_t launch_pack_codes(const int8_t* src, int rows, int hd, int bits, uint8_t* dst, size_t dst_row_stride,
+                              cudaStream_t s);
+
+}  // namespace fl

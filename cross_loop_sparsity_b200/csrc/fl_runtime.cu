@@ -1,0 +1,948 @@
+// fl_runtime.cu -- host runtime and C ABI: configuration checks, workspace
+// layout, TMA descriptors, the per-call kernel sequence (prefill and decode),
+// CUDA-graph capture of decode steps, cache import/export and test entry points.
+//
+// One call runs the looped block K times over its tokens ("FlashLoop: Fast and
+// Memory-Efficient Looped Transformers via Lazy Updates", abstract):
+//   loop 1     : every token, dense attention; writes the bf16 base KV
+//   loop l >= 2: top ceil(rho*N) tokens by ||h_{l-1} - h_{l-2}||^2 recompute;
+//                their KV is stored as a quantised residual; their attention is
+//                corrected over the fixed top-c key columns of their query tile
+// The dense baseline (resid_bits 16) recomputes every token every loop with a
+// per-loop bf16 KV ("Looped Transformer 教程", 第一步 / 第四步).
+#include <cmath>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "flashloop.h"
+#include "fl_kernels.h"
+
+using namespace fl;
+
+namespace fl {
+void gemm_init_attrs();
+void kernels_init_attrs();
+}  // namespace fl
+
+struct flashloop_ctx {
+  flashloop_config cfg;
+  flashloop_weights w;
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+  int device = 0;
+  CacheView cv{};
+  bool lazy = true;
+  int qkv_rows = 0, N_max = 0, N_pad = 0, n_tiles_max = 0, max_need = 0;
+  int dec_splits = 1, dec_split_len = 64;
+  // workspace regions
+  float *rope_cos = nullptr, *rope_sin = nullptr;
+  int *seq_len = nullptr, *status = nullptr;
+  float *h = nullptr, *h_in = nullptr, *h_snap = nullptr;
+  uint16_t *x = nullptr, *obf = nullptr, *act = nullptr;
+  float *qkv = nullptr, *q_cur = nullptr;
+  float *o_state = nullptr, *lse_state = nullptr, *q_last = nullptr;
+  int *seq = nullptr, *pos = nullptr, *tile = nullptr, *last = nullptr, *sel_slot = nullptr;
+  float *key = nullptr, *keys_trace = nullptr;
+  int32_t *idx_all = nullptr, *idx_sel = nullptr, *idx_last = nullptr;
+  int* has_c = nullptr;
+  TilePlan plan{};
+  int32_t* cols = nullptr;
+  int* ncols = nullptr;
+  float* col_keys = nullptr;
+  int* forced_on = nullptr;
+  int32_t *forced_sel = nullptr, *forced_cols = nullptr;
+  int* forced_ncols = nullptr;
+  float *part_o = nullptr, *part_ml = nullptr;
+  int* attn_counters = nullptr;
+  float* gemm_partial = nullptr;
+  size_t gemm_partial_cap = 0;
+  int* gemm_counters = nullptr;
+  float* logits_ws = nullptr;
+  // descriptors
+  CUtensorMap tm_qkv, tm_o, tm_gate, tm_up, tm_down, tm_out;
+  CUtensorMap tm_x_a, tm_obf_a, tm_act_a;
+  CUtensorMap tm_x_b[3], tm_obf_b[3], tm_act_b[3];
+  // host state
+  std::vector<int> lens;
+  std::vector<int> graph_b;
+  std::vector<cudaGraphExec_t> graph_exec;
+  std::vector<int> eager_seen;
+  int use_graph = 1;
+  std::string last_err;
+  int last_N = 0, last_nsel = 0, last_decode = 0, last_tiles = 0;
+};
+
+namespace {
+
+constexpr int kNumSM = 148;
+constexpr int kCountersGemm = 4096;
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+int n_select(double rho, int n) {
+  if (n <= 0) return 0;
+  int k = static_cast<int>(std::ceil(rho * n - 1e-9));
+  if (k < 1) k = 1;
+  if (k > n) k = n;
+  return k;
+}
+
+bool valid_config(const flashloop_config* c) {
+  if (!c) return false;
+  if (c->d_model < 64 || c->d_model % 64) return false;
+  if (c->head_dim != 64 && c->head_dim != 128) return false;
+  if (c->n_heads < 1 || c->n_kv_heads < 1 || c->n_heads % c->n_kv_heads) return false;
+  if (c->n_heads / c->n_kv_heads > 8) return false;
+  if (c->ffn_dim < 8 || c->ffn_dim % 8) return false;
+  if (c->n_layers < 1 || c->n_loops < 1 || c->n_loops > 16) return false;
+  if (c->resid_bits != 2 && c->resid_bits != 4 && c->resid_bits != 16) return false;
+  if (c->resid_bits != 16) {
+    if (!(c->rho > 0.0 && c->rho <= 1.0)) return false;
+    if (c->c_cols < 1 || c->c_cols > 4096) return false;
+    if (c->group_size != 32 && c->group_size != 64 && c->group_size != 128) return false;
+    if (c->group_size > c->head_dim || c->head_dim % c->group_size) return false;
+    if (c->q_tile < 1) return false;
+  }
+  if (c->vocab < 1 || c->max_batch < 1 || c->max_ctx < 1 || c->max_tokens < 0) return false;
+  if (!(c->rms_eps > 0.f) || !(c->rope_theta > 0.f)) return false;
+  return true;
+}
+
+int swap_bn(int n) { return n <= 16 ? 16 : n <= 32 ? 32 : 64; }
+
+// split-K factor of a skinny GEMM with `tiles` 128-row feature tiles
+int split_factor(int tiles, int k_chunks) {
+  if (tiles >= kNumSM) return 1;
+  int s = kNumSM / tiles;
+  if (s > k_chunks) s = k_chunks;
+  return s < 1 ? 1 : s;
+}
+
+// Walk the workspace regions; assign pointers when ctx is given.  Returns the byte total.
+size_t layout(const flashloop_config& c, flashloop_ctx* x) {
+  const int M = c.n_layers, K = c.n_loops, Hkv = c.n_kv_heads, H = c.n_heads, hd = c.head_dim, d = c.d_model;
+  const bool lazy = c.resid_bits != 16;
+  const size_t B = c.max_batch, T = c.max_ctx;
+  const int N = c.max_tokens > c.max_batch ? c.max_tokens : c.max_batch;
+  const int Npad = ceil_div(N > 64 ? N : 64, 128) * 128;
+  const int qkv_rows = (H + 2 * Hkv) * hd;
+  const int q_tile = lazy ? c.q_tile : 128;
+  const int n_tiles = (c.max_batch > ceil_div(c.max_tokens, q_tile) + c.max_batch)
+                          ? c.max_batch : ceil_div(c.max_tokens, q_tile) + c.max_batch;
+  const int nsel_max = lazy ? n_select(c.rho, N) : N;
+  const int max_need = nsel_max < n_tiles ? nsel_max : n_tiles;
+  const int cc = lazy ? c.c_cols : 1;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> uint8_t* {
+    uint8_t* p = x ? x->ws + off : nullptr;
+    off = align256(off + bytes);
+    return p;
+  };
+  // KV cache
+  const size_t rows = static_cast<size_t>(M) * 2 * B * Hkv * T;
+  uint8_t *base, *codes = nullptr, *scales = nullptr;
+  if (lazy) {
+    base = take(rows * hd * 2);
+    codes = take(rows * (K - 1) * (static_cast<size_t>(hd) * c.resid_bits / 8));
+    scales = take(rows * (K - 1) * (hd / c.group_size) * 2);
+  } else {
+    base = take(rows * K * hd * 2);
+  }
+  uint8_t* rc = take(T * (hd / 2) * 4);
+  uint8_t* rs = take(T * (hd / 2) * 4);
+  uint8_t* seq_len = take(B * 4);
+  uint8_t* status = take(16);
+  uint8_t* h = take(static_cast<size_t>(N) * d * 4);
+  uint8_t* h_in = take(static_cast<size_t>(N) * d * 4);
+  uint8_t* h_snap = take(static_cast<size_t>(N) * d * 4);
+  uint8_t* xb = take(static_cast<size_t>(Npad) * d * 2);
+  uint8_t* obf = take(static_cast<size_t>(Npad) * H * hd * 2);
+  uint8_t* act = take(static_cast<size_t>(Npad) * c.ffn_dim * 2);
+  uint8_t* qkv = take(static_cast<size_t>(Npad) * qkv_rows * 4);
+  uint8_t* q_cur = take(static_cast<size_t>(N) * H * hd * 4);
+  uint8_t *o_state = nullptr, *lse = nullptr, *q_last = nullptr;
+  if (lazy) {
+    o_state = take(static_cast<size_t>(M) * N * H * hd * 4);
+    lse = take(static_cast<size_t>(M) * N * H * 4);
+    q_last = take(static_cast<size_t>(M) * N * H * hd * 4);
+  }
+  uint8_t* seq = take(N * 4);
+  uint8_t* pos = take(N * 4);
+  uint8_t* tile = take(N * 4);
+  uint8_t* last = take(N * 4);
+  uint8_t* sel_slot = take(N * 4);
+  uint8_t* key = take(N * 4);
+  uint8_t* keys_trace = take(static_cast<size_t>(K) * N * 4);
+  uint8_t* idx_all = take(N * 4);
+  uint8_t* idx_sel = take(static_cast<size_t>(K) * N * 4);
+  uint8_t* idx_last = take(B * 4);
+  uint8_t* has_c = take(n_tiles * 4);
+  uint8_t* p_tile = take(n_tiles * 4);
+  uint8_t* p_qb = take(n_tiles * 4);
+  uint8_t* p_qe = take(n_tiles * 4);
+  uint8_t* p_need = take(n_tiles * 4);
+  uint8_t* p_counts = take(16);
+  uint8_t* cols = take(static_cast<size_t>(M) * n_tiles * Hkv * cc * 4);
+  uint8_t* ncols = take(static_cast<size_t>(M) * n_tiles * Hkv * 4);
+  uint8_t* col_keys = take(lazy ? static_cast<size_t>(max_need) * Hkv * T * 4 : 4);
+  uint8_t* forced_on = take(16);
+  uint8_t* forced_sel = take(static_cast<size_t>(K) * N * 4);
+  uint8_t* forced_cols = take(static_cast<size_t>(M) * n_tiles * Hkv * cc * 4);
+  uint8_t* forced_ncols = take(static_cast<size_t>(M) * n_tiles * Hkv * 4);
+  // decode attention split partials
+  int splits = ceil_div(4 * kNumSM, c.max_batch * Hkv);
+  const int max_splits = ceil_div(c.max_ctx, 64);
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  const int split_len = ceil_div(ceil_div(c.max_ctx, splits), 64) * 64;
+  splits = ceil_div(c.max_ctx, split_len);
+  uint8_t* part_o = take(B * Hkv * splits * 8 * hd * 4);
+  uint8_t* part_ml = take(B * Hkv * splits * 8 * 2 * 4);
+  uint8_t* attn_counters = take(B * Hkv * 4);
+  // GEMM split-K partials (skinny orientation only)
+  size_t gp = 0;
+  if (N <= 64 || c.max_batch <= 64) {
+    const int n_sk = c.max_batch <= 64 ? c.max_batch : 64;
+    const int bn = swap_bn(n_sk);
+    const int feats[5] = {qkv_rows, d, c.ffn_dim, d, c.vocab};
+    const int ks[5] = {d, H * hd, d, c.ffn_dim, d};
+    const int dual[5] = {0, 0, 1, 0, 0};
+    for (int o = 0; o < 5; ++o) {
+      const int tiles = ceil_div(feats[o], 128);
+      const size_t f = gemm_partial_floats(bn, dual[o], tiles, split_factor(tiles, ceil_div(ks[o], 64)));
+      if (f > gp) gp = f;
+    }
+    // prefill loops >= 2 and the last-row logits may also take the skinny path with up to 64 rows
+    const int feats2[5] = {qkv_rows, d, c.ffn_dim, d, c.vocab};
+    for (int o = 0; o < 5; ++o) {
+      const int tiles = ceil_div(feats2[o], 128);
+      const size_t f = gemm_partial_floats(64, dual[o], tiles, split_factor(tiles, ceil_div(ks[o], 64)));
+      if (f > gp) gp = f;
+    }
+  }
+  uint8_t* gpart = take((gp > 0 ? gp : 1) * 4);
+  uint8_t* gcnt = take(kCountersGemm * 4);
+  uint8_t* logits = take(B * c.vocab * 4);
+  if (x) {
+    x->lazy = lazy;
+    x->qkv_rows = qkv_rows;
+    x->N_max = N;
+    x->N_pad = Npad;
+    x->n_tiles_max = n_tiles;
+    x->max_need = max_need;
+    x->dec_splits = splits;
+    x->dec_split_len = split_len;
+    x->cv.M = M; x->cv.K = K; x->cv.B = c.max_batch; x->cv.Hkv = Hkv; x->cv.T = c.max_ctx; x->cv.hd = hd;
+    x->cv.g = lazy ? c.group_size : hd;
+    x->cv.bits = lazy ? c.resid_bits : 16;
+    x->cv.dense = lazy ? 0 : 1;
+    x->cv.base = reinterpret_cast<uint16_t*>(base);
+    x->cv.codes = codes;
+    x->cv.scales = reinterpret_cast<uint16_t*>(scales);
+    x->rope_cos = reinterpret_cast<float*>(rc);
+    x->rope_sin = reinterpret_cast<float*>(rs);
+    x->seq_len = reinterpret_cast<int*>(seq_len);
+    x->status = reinterpret_cast<int*>(status);
+    x->h = reinterpret_cast<float*>(h);
+    x->h_in = reinterpret_cast<float*>(h_in);
+    x->h_snap = reinterpret_cast<float*>(h_snap);
+    x->x = reinterpret_cast<uint16_t*>(xb);
+    x->obf = reinterpret_cast<uint16_t*>(obf);
+    x->act = reinterpret_cast<uint16_t*>(act);
+    x->qkv = reinterpret_cast<float*>(qkv);
+    x->q_cur = reinterpret_cast<float*>(q_cur);
+    x->o_state = reinterpret_cast<float*>(o_state);
+    x->lse_state = reinterpret_cast<float*>(lse);
+    x->q_last = reinterpret_cast<float*>(q_last);
+    x->seq = reinterpret_cast<int*>(seq);
+    x->pos = reinterpret_cast<int*>(pos);
+    x->tile = reinterpret_cast<int*>(tile);
+    x->last = reinterpret_cast<int*>(last);
+    x->sel_slot = reinterpret_cast<int*>(sel_slot);
+    x->key = reinterpret_cast<float*>(key);
+    x->keys_trace = reinterpret_cast<float*>(keys_trace);
+    x->idx_all = reinterpret_cast<int32_t*>(idx_all);
+    x->idx_sel = reinterpret_cast<int32_t*>(idx_sel);
+    x->idx_last = reinterpret_cast<int32_t*>(idx_last);
+    x->has_c = reinterpret_cast<int*>(has_c);
+    x->plan.tile = reinterpret_cast<int*>(p_tile);
+    x->plan.qb = reinterpret_cast<int*>(p_qb);
+    x->plan.qe = reinterpret_cast<int*>(p_qe);
+    x->plan.need = reinterpret_cast<int*>(p_need);
+    x->plan.counts = reinterpret_cast<int*>(p_counts);
+    x->cols = reinterpret_cast<int32_t*>(cols);
+    x->ncols = reinterpret_cast<int*>(ncols);
+    x->col_keys = reinterpret_cast<float*>(col_keys);
+    x->forced_on = reinterpret_cast<int*>(forced_on);
+    x->forced_sel = reinterpret_cast<int32_t*>(forced_sel);
+    x->forced_cols = reinterpret_cast<int32_t*>(forced_cols);
+    x->forced_ncols = reinterpret_cast<int*>(forced_ncols);
+    x->part_o = reinterpret_cast<float*>(part_o);
+    x->part_ml = reinterpret_cast<float*>(part_ml);
+    x->attn_counters = reinterpret_cast<int*>(attn_counters);
+    x->gemm_partial = reinterpret_cast<float*>(gpart);
+    x->gemm_partial_cap = gp;
+    x->gemm_counters = reinterpret_cast<int*>(gcnt);
+    x->logits_ws = reinterpret_cast<float*>(logits);
+  }
+  return off;
+}
+
+#define FL_TRY(expr)                                   \
+  do {                                                 \
+    cudaError_t e_ = (expr);                           \
+    if (e_ != cudaSuccess) {                           \
+      ctx->last_err = cudaGetErrorString(e_);          \
+      return FL_ERR_CUDA;                              \
+    }                                                  \
+  } while (0)
+
+enum GemmOpKind { kOpQKV, kOpO, kOpGU, kOpDown, kOpOut };
+
+fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, cudaStream_t s) {
+  const flashloop_config& c = ctx->cfg;
+  GemmLaunch g{};
+  GemmArgs& a = g.args;
+  const CUtensorMap *w0 = nullptr, *w1 = nullptr, *xa = nullptr;
+  const CUtensorMap* xb = nullptr;
+  int feat = 0, K = 0;
+  switch (op) {
+    case kOpQKV:
+      w0 = &ctx->tm_qkv; feat = ctx->qkv_rows; K = c.d_model; xa = &ctx->tm_x_a; xb = ctx->tm_x_b;
+      a.epi = kEpiStore; a.out = ctx->qkv; a.ldo = ctx->qkv_rows;
+      break;
+    case kOpO:
+      w0 = &ctx->tm_o; feat = c.d_model; K = c.n_heads * c.head_dim; xa = &ctx->tm_obf_a; xb = ctx->tm_obf_b;
+      a.epi = kEpiResid; a.h = ctx->h; a.idx = idx; a.scale = c.resid_scale; a.ldh = c.d_model;
+      break;
+    case kOpGU:
+      w0 = &ctx->tm_gate; w1 = &ctx->tm_up; feat = c.ffn_dim; K = c.d_model; xa = &ctx->tm_x_a; xb = ctx->tm_x_b;
+      a.epi = kEpiSwiglu; a.act = ctx->act; a.ld_act = c.ffn_dim;
+      break;
+    case kOpDown:
+      w0 = &ctx->tm_down; feat = c.d_model; K = c.ffn_dim; xa = &ctx->tm_act_a; xb = ctx->tm_act_b;
+      a.epi = kEpiResid; a.h = ctx->h; a.idx = idx; a.scale = c.resid_scale; a.ldh = c.d_model;
+      break;
+    case kOpOut:
+      w0 = &ctx->tm_out; feat = c.vocab; K = c.d_model; xa = &ctx->tm_x_a; xb = ctx->tm_x_b;
+      a.epi = kEpiStore; a.out = ctx->logits_ws; a.ldo = c.vocab;
+      break;
+  }
+  a.k_chunks = ceil_div(K, 64);
+  a.n_feat = feat;
+  a.n_tok = n;
+  a.status = ctx->status;
+  const int w3d = op != kOpOut;
+  if (n <= 64) {
+    const int bn = swap_bn(n);
+    const int bi = bn == 16 ? 0 : bn == 32 ? 1 : 2;
+    const int tiles = ceil_div(feat, 128);
+    const int splits = split_factor(tiles, a.k_chunks);
+    if (gemm_partial_floats(bn, w1 != nullptr, tiles, splits) > ctx->gemm_partial_cap || tiles > kCountersGemm)
+      return FL_ERR_CAPACITY;
+    g.a0 = w0; g.a1 = w1; g.b0 = &xb[bi]; g.b1 = nullptr;
+    g.a_3d = w3d; g.b_3d = 0;
+    a.a_z = j; a.b_z = 0; a.swap = 1; a.splits = splits;
+    a.partial = ctx->gemm_partial; a.counters = ctx->gemm_counters;
+    g.bn = bn;
+    g.grid = dim3(tiles, 1, splits);
+  } else {
+    g.a0 = xa; g.a1 = nullptr; g.b0 = w0; g.b1 = w1;
+    g.a_3d = 0; g.b_3d = w3d;
+    a.a_z = 0; a.b_z = j; a.swap = 0; a.splits = 1;
+    g.bn = 128;
+    g.grid = dim3(ceil_div(n, 128), ceil_div(feat, 128), 1);
+  }
+  FL_TRY(launch_gemm(g, s));
+  return FL_OK;
+}
+
+__global__ void k_fill_last_rows(int B, int T, int32_t* rows) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B) rows[b] = b * T + T - 1;
+}
+
+#define FL_STEP(expr)                 \
+  do {                                \
+    fl_status st_ = (expr);           \
+    if (st_ != FL_OK) return st_;     \
+  } while (0)
+
+// The whole looped block over one call's tokens, enqueued on s.  The input
+// hidden states are in h_in; the result is left in h and logits_ws.
+fl_status run_call(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s) {
+  const flashloop_config& c = ctx->cfg;
+  const int M = c.n_layers, K = c.n_loops, d = c.d_model, H = c.n_heads, Hkv = c.n_kv_heads, hd = c.head_dim;
+  const bool lazy = ctx->lazy;
+  const int N = decode ? B : B * T;
+  const int q_tile = lazy ? c.q_tile : 128;
+  const int tiles_per_seq = decode ? 1 : ceil_div(T, q_tile);
+  const int n_tiles = decode ? B : B * tiles_per_seq;
+  const int n_sel = lazy ? n_select(c.rho, N) : N;
+  const float tau = 1.0f / std::sqrt(static_cast<float>(hd));
+  const size_t st_o = static_cast<size_t>(ctx->N_max) * H * hd, st_l = static_cast<size_t>(ctx->N_max) * H;
+  auto pad = [&](int n) { return n <= 64 ? swap_bn(n) : ceil_div(n, 128) * 128; };
+  const int max_need = n_sel < n_tiles ? n_sel : n_tiles;
+  const int col_span = decode ? c.max_ctx : T;   // columns a query tile can see
+  const int max_chunks = ceil_div(col_span, 64);
+
+  FL_TRY(launch_setup_call(N, decode, T, tiles_per_seq, q_tile, ctx->seq_len, ctx->seq, ctx->pos, ctx->tile,
+                           ctx->last, n_tiles, ctx->has_c, s));
+  FL_TRY(cudaMemcpyAsync(ctx->h, ctx->h_in, static_cast<size_t>(N) * d * 4, cudaMemcpyDeviceToDevice, s));
+  for (int l = 1; l <= K; ++l) {
+    const bool full = !lazy || l == 1;
+    const int32_t* idx = ctx->idx_all;
+    int n = N;
+    if (!full) {
+      int32_t* sel = ctx->idx_sel + static_cast<size_t>(l - 2) * ctx->N_max;
+      FL_TRY(cudaMemcpyAsync(ctx->keys_trace + static_cast<size_t>(l - 2) * ctx->N_max, ctx->key,
+                             static_cast<size_t>(N) * 4, cudaMemcpyDeviceToDevice, s));
+      FL_TRY(launch_select_tokens(ctx->key, N, n_sel, sel, ctx->forced_on,
+                                  ctx->forced_sel + static_cast<size_t>(l - 2) * ctx->N_max, s));
+      FL_TRY(launch_after_select(sel, n_sel, N, d, ctx->sel_slot, ctx->h, ctx->h_snap, s));
+      FL_TRY(launch_plan_tiles(sel, n_sel, ctx->tile, ctx->has_c, ctx->plan, s));
+      idx = sel;
+      n = n_sel;
+    }
+    for (int j = 0; j < M; ++j) {
+      float* o_st = lazy ? ctx->o_state + j * st_o : nullptr;
+      float* l_st = lazy ? ctx->lse_state + j * st_l : nullptr;
+      float* ql = lazy ? ctx->q_last + j * st_o : nullptr;
+      // attention branch
+      FL_TRY(launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d, ctx->w.attn_norm + static_cast<size_t>(j) * d,
+                                 c.rms_eps, ctx->x, s));
+      FL_STEP(gemm(ctx, kOpQKV, j, n, idx, s));
+      QkvPostArgs qa{};
+      qa.qkv = ctx->qkv; qa.ldq = ctx->qkv_rows; qa.idx = idx; qa.n = n; qa.seq = ctx->seq; qa.pos = ctx->pos;
+      qa.H = H; qa.Hkv = Hkv; qa.hd = hd; qa.rope_cos = ctx->rope_cos; qa.rope_sin = ctx->rope_sin;
+      qa.cv = ctx->cv; qa.j = j; qa.loop = l; qa.lazy = lazy ? 1 : 0; qa.q_cur = ctx->q_cur; qa.q_last = ql;
+      FL_TRY(launch_qkv_post(qa, s));
+      if (full) {
+        if (decode) {
+          AttnDecArgs aa{};
+          aa.q_cur = ctx->q_cur; aa.idx = idx; aa.seq = ctx->seq; aa.pos = ctx->pos; aa.cv = ctx->cv;
+          aa.j = j; aa.loop = l; aa.dense = lazy ? 0 : 1; aa.H = H; aa.Hkv = Hkv; aa.hd = hd; aa.tau = tau;
+          aa.split_len = ctx->dec_split_len; aa.n_splits = ctx->dec_splits;
+          aa.part_o = ctx->part_o; aa.part_ml = ctx->part_ml; aa.counters = ctx->attn_counters;
+          aa.o_state = o_st; aa.lse_state = l_st; aa.o_bf16 = ctx->obf;
+          FL_TRY(launch_attn_decode(aa, n, s));
+        } else {
+          AttnPreArgs pa{};
+          pa.q_cur = ctx->q_cur; pa.cv = ctx->cv; pa.j = j; pa.loop = l; pa.dense = lazy ? 0 : 1;
+          pa.T = T; pa.H = H; pa.Hkv = Hkv; pa.hd = hd; pa.tau = tau;
+          pa.o_state = o_st; pa.lse_state = l_st; pa.o_bf16 = ctx->obf;
+          FL_TRY(launch_attn_prefill(pa, B, s));
+        }
+      } else {
+        DScoreArgs da{};
+        da.plan = ctx->plan; da.idx = idx; da.seq = ctx->seq; da.pos = ctx->pos; da.q_cur = ctx->q_cur;
+        da.q_last = ql; da.cv = ctx->cv; da.j = j; da.loop = l; da.H = H; da.Hkv = Hkv; da.hd = hd; da.tau = tau;
+        da.col_keys = ctx->col_keys; da.max_cols = c.max_ctx;
+        FL_TRY(launch_dscore(da, max_need, max_chunks, s));
+        SelColsArgs sa{};
+        sa.plan = ctx->plan; sa.idx = idx; sa.pos = ctx->pos; sa.col_keys = ctx->col_keys; sa.max_cols = c.max_ctx;
+        sa.Hkv = Hkv; sa.c = c.c_cols; sa.j = j; sa.n_tiles = ctx->n_tiles_max; sa.cols = ctx->cols;
+        sa.ncols = ctx->ncols; sa.forced_on = ctx->forced_on; sa.forced_cols = ctx->forced_cols;
+        sa.forced_ncols = ctx->forced_ncols;
+        FL_TRY(launch_select_cols(sa, max_need, s));
+        CorrectArgs ca{};
+        ca.idx = idx; ca.seq = ctx->seq; ca.pos = ctx->pos; ca.tile = ctx->tile; ca.last = ctx->last;
+        ca.q_cur = ctx->q_cur; ca.q_last = ql; ca.o_state = o_st; ca.lse_state = l_st; ca.o_bf16 = ctx->obf;
+        ca.cols = ctx->cols; ca.ncols = ctx->ncols; ca.cv = ctx->cv; ca.j = j; ca.loop = l; ca.H = H; ca.Hkv = Hkv;
+        ca.hd = hd; ca.c = c.c_cols; ca.n_tiles = ctx->n_tiles_max; ca.tau = tau; ca.status = ctx->status;
+        FL_TRY(launch_correct(ca, n, s));
+      }
+      FL_STEP(gemm(ctx, kOpO, j, n, idx, s));
+      // MLP branch
+      FL_TRY(launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d, ctx->w.mlp_norm + static_cast<size_t>(j) * d, c.rms_eps,
+                                 ctx->x, s));
+      FL_STEP(gemm(ctx, kOpGU, j, n, idx, s));
+      FL_STEP(gemm(ctx, kOpDown, j, n, idx, s));
+    }
+    if (lazy && l < K)
+      FL_TRY(launch_change_keys(ctx->h, l == 1 ? ctx->h_in : ctx->h_snap, ctx->sel_slot, N, d, l, ctx->key, ctx->last,
+                                ctx->tile, ctx->has_c, s));
+  }
+  // final norm + LM head on the output rows
+  const int32_t* rows = ctx->idx_all;
+  if (!decode) {
+    k_fill_last_rows<<<ceil_div(B, 128), 128, 0, s>>>(B, T, ctx->idx_last);
+    FL_TRY(cudaGetLastError());
+    rows = ctx->idx_last;
+  }
+  FL_TRY(launch_rmsnorm_rows(ctx->h, rows, B, pad(B), d, ctx->w.final_norm, c.rms_eps, ctx->x, s));
+  FL_STEP(gemm(ctx, kOpOut, 0, B, rows, s));
+  FL_TRY(launch_set_lens(B, ctx->seq_len, decode ? 1 : 0, T, s));
+  return FL_OK;
+}
+
+bool build_tmaps(flashloop_ctx* ctx) {
+  const flashloop_config& c = ctx->cfg;
+  const flashloop_weights& w = ctx->w;
+  const uint64_t M = c.n_layers, d = c.d_model, f = c.ffn_dim, hq = static_cast<uint64_t>(c.n_heads) * c.head_dim;
+  bool ok = true;
+  ok &= encode_tmap_bf16(&ctx->tm_qkv, w.w_qkv, d, ctx->qkv_rows, M, 128);
+  ok &= encode_tmap_bf16(&ctx->tm_o, w.w_o, hq, d, M, 128);
+  ok &= encode_tmap_bf16(&ctx->tm_gate, w.w_gate, d, f, M, 128);
+  ok &= encode_tmap_bf16(&ctx->tm_up, w.w_up, d, f, M, 128);
+  ok &= encode_tmap_bf16(&ctx->tm_down, w.w_down, f, d, M, 128);
+  ok &= encode_tmap_bf16(&ctx->tm_out, w.w_out, d, c.vocab, 0, 128);
+  const uint64_t R = ctx->N_pad;
+  ok &= encode_tmap_bf16(&ctx->tm_x_a, ctx->x, d, R, 0, 128);
+  ok &= encode_tmap_bf16(&ctx->tm_obf_a, ctx->obf, hq, R, 0, 128);
+  ok &= encode_tmap_bf16(&ctx->tm_act_a, ctx->act, f, R, 0, 128);
+  const uint32_t bns[3] = {16, 32, 64};
+  for (int i = 0; i < 3; ++i) {
+    ok &= encode_tmap_bf16(&ctx->tm_x_b[i], ctx->x, d, R, 0, bns[i]);
+    ok &= encode_tmap_bf16(&ctx->tm_obf_b[i], ctx->obf, hq, R, 0, bns[i]);
+    ok &= encode_tmap_bf16(&ctx->tm_act_b[i], ctx->act, f, R, 0, bns[i]);
+  }
+  return ok;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+size_t flashloop_workspace_bytes(const flashloop_config* cfg) {
+  if (!valid_config(cfg)) return 0;
+  return layout(*cfg, nullptr);
+}
+
+const char* flashloop_status_string(fl_status s) {
+  switch (s) {
+    case FL_OK: return "ok";
+    case FL_ERR_INVALID_ARG: return "invalid argument";
+    case FL_ERR_CAPACITY: return "capacity exceeded";
+    case FL_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case FL_ERR_CUDA: return "CUDA error";
+    case FL_ERR_TIMEOUT: return "a kernel wait timed out";
+    case FL_ERR_NONFINITE: return "non-finite value";
+    case FL_ERR_UNSUPPORTED: return "unsupported configuration";
+  }
+  return "unknown status";
+}
+
+const char* flashloop_last_cuda_error(const flashloop_ctx* ctx) { return ctx ? ctx->last_err.c_str() : ""; }
+
+fl_status flashloop_init(const flashloop_config* cfg, const flashloop_weights* w, void* workspace,
+                         size_t workspace_bytes, fl_stream_t stream, flashloop_ctx** out) {
+  if (!out) return FL_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!valid_config(cfg) || !w) return FL_ERR_INVALID_ARG;
+  if (cfg->resid_bits != 16 &&
+      correct_smem(cfg->head_dim, cfg->n_heads / cfg->n_kv_heads, cfg->c_cols) > static_cast<size_t>(kMaxDynSmem))
+    return FL_ERR_UNSUPPORTED;
+  const void* wp[9] = {w->attn_norm, w->w_qkv, w->w_o, w->mlp_norm, w->w_gate, w->w_up, w->w_down, w->final_norm,
+                       w->w_out};
+  for (const void* p : wp)
+    if (!p || !aligned16(p)) return FL_ERR_INVALID_ARG;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255)) return FL_ERR_WORKSPACE;
+  const size_t need = layout(*cfg, nullptr);
+  if (workspace_bytes < need) return FL_ERR_WORKSPACE;
+  flashloop_ctx* ctx = new (std::nothrow) flashloop_ctx();
+  if (!ctx) return FL_ERR_CUDA;
+  ctx->cfg = *cfg;
+  ctx->w = *w;
+  ctx->ws = static_cast<uint8_t*>(workspace);
+  ctx->ws_bytes = workspace_bytes;
+  cudaGetDevice(&ctx->device);
+  layout(*cfg, ctx);
+  ctx->lens.assign(cfg->max_batch, 0);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  auto fail = [&](fl_status st) {
+    if (st == FL_ERR_CUDA && ctx->last_err.empty()) ctx->last_err = cudaGetErrorString(cudaGetLastError());
+    delete ctx;
+    return st;
+  };
+  gemm_init_attrs();
+  kernels_init_attrs();
+  if (cudaGetLastError() != cudaSuccess) return fail(FL_ERR_CUDA);
+  if (!build_tmaps(ctx)) return fail(FL_ERR_CUDA);
+  if (cudaMemsetAsync(ctx->ws, 0, need, s) != cudaSuccess) return fail(FL_ERR_CUDA);
+  // RoPE table: angle = pos * theta^(-2i/hd), computed in double, stored fp32
+  const int half = cfg->head_dim / 2;
+  std::vector<float> rc(static_cast<size_t>(cfg->max_ctx) * half), rs(rc.size());
+  for (int t = 0; t < cfg->max_ctx; ++t)
+    for (int i = 0; i < half; ++i) {
+      const double inv = std::pow(static_cast<double>(cfg->rope_theta), -2.0 * i / cfg->head_dim);
+      const double a = static_cast<double>(t) * inv;
+      rc[static_cast<size_t>(t) * half + i] = static_cast<float>(std::cos(a));
+      rs[static_cast<size_t>(t) * half + i] = static_cast<float>(std::sin(a));
+    }
+  if (cudaMemcpyAsync(ctx->rope_cos, rc.data(), rc.size() * 4, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(ctx->rope_sin, rs.data(), rs.size() * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return fail(FL_ERR_CUDA);
+  std::vector<int32_t> ident(ctx->N_max);
+  for (int i = 0; i < ctx->N_max; ++i) ident[i] = i;
+  if (cudaMemcpyAsync(ctx->idx_all, ident.data(), ident.size() * 4, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return fail(FL_ERR_CUDA);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return fail(FL_ERR_CUDA);
+  *out = ctx;
+  return FL_OK;
+}
+
+void flashloop_destroy(flashloop_ctx* ctx) {
+  if (!ctx) return;
+  for (cudaGraphExec_t e : ctx->graph_exec)
+    if (e) cudaGraphExecDestroy(e);
+  delete ctx;
+}
+
+fl_status flashloop_set_option(flashloop_ctx* ctx, fl_option opt, int value) {
+  if (!ctx) return FL_ERR_INVALID_ARG;
+  if (opt == FL_OPT_USE_GRAPH) {
+    ctx->use_graph = value ? 1 : 0;
+    return FL_OK;
+  }
+  return FL_ERR_INVALID_ARG;
+}
+
+fl_status flashloop_prefill(flashloop_ctx* ctx, const float* h0, int B, int T, float* h_out, float* logits_last,
+                            fl_stream_t stream) {
+  if (!ctx || !h0 || B < 1 || T < 1) return FL_ERR_INVALID_ARG;
+  const flashloop_config& c = ctx->cfg;
+  if (B > c.max_batch || static_cast<long long>(B) * T > c.max_tokens || T > c.max_ctx) return FL_ERR_CAPACITY;
+  for (int b = 0; b < B; ++b)
+    if (ctx->lens[b] != 0) return FL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(B) * T * c.d_model * 4;
+  FL_TRY(cudaMemcpyAsync(ctx->h_in, h0, bytes, cudaMemcpyDefault, s));
+  FL_STEP(run_call(ctx, 0, B, T, s));
+  if (h_out) FL_TRY(cudaMemcpyAsync(h_out, ctx->h, bytes, cudaMemcpyDefault, s));
+  if (logits_last)
+    FL_TRY(cudaMemcpyAsync(logits_last, ctx->logits_ws, static_cast<size_t>(B) * c.vocab * 4, cudaMemcpyDefault, s));
+  for (int b = 0; b < B; ++b) ctx->lens[b] = T;
+  ctx->last_N = B * T;
+  ctx->last_nsel = ctx->lazy ? n_select(c.rho, B * T) : B * T;
+  ctx->last_decode = 0;
+  ctx->last_tiles = B * ceil_div(T, ctx->lazy ? c.q_tile : 128);
+  return FL_OK;
+}
+
+fl_status flashloop_decode_step(flashloop_ctx* ctx, const float* h0, int B, float* h_out, float* logits,
+                                fl_stream_t stream) {
+  if (!ctx || !h0 || B < 1) return FL_ERR_INVALID_ARG;
+  const flashloop_config& c = ctx->cfg;
+  if (B > c.max_batch) return FL_ERR_CAPACITY;
+  for (int b = 0; b < B; ++b)
+    if (ctx->lens[b] + 1 > c.max_ctx) return FL_ERR_CAPACITY;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FL_TRY(cudaMemcpyAsync(ctx->h_in, h0, static_cast<size_t>(B) * c.d_model * 4, cudaMemcpyDefault, s));
+  // A decode step's launch sequence depends on B only; after one direct run it
+  // is captured once into a CUDA graph and replayed (not on the legacy stream).
+  size_t gi = 0;
+  while (gi < ctx->graph_b.size() && ctx->graph_b[gi] != B) ++gi;
+  bool seen = false;
+  for (int v : ctx->eager_seen) seen |= (v == B);
+  if (ctx->use_graph && s != nullptr && seen) {
+    if (gi == ctx->graph_b.size()) {
+      cudaGraph_t graph = nullptr;
+      FL_TRY(cudaStreamBeginCapture(s, cudaStreamCaptureModeThreadLocal));
+      fl_status st = run_call(ctx, 1, B, 0, s);
+      cudaError_t e = cudaStreamEndCapture(s, &graph);
+      if (st != FL_OK) {
+        if (graph) cudaGraphDestroy(graph);
+        return st;
+      }
+      FL_TRY(e);
+      cudaGraphExec_t exec = nullptr;
+      e = cudaGraphInstantiate(&exec, graph, 0);
+      cudaGraphDestroy(graph);
+      FL_TRY(e);
+      ctx->graph_b.push_back(B);
+      ctx->graph_exec.push_back(exec);
+    }
+    FL_TRY(cudaGraphLaunch(ctx->graph_exec[gi], s));
+  } else {
+    FL_STEP(run_call(ctx, 1, B, 0, s));
+    if (!seen) ctx->eager_seen.push_back(B);
+  }
+  if (h_out) FL_TRY(cudaMemcpyAsync(h_out, ctx->h, static_cast<size_t>(B) * c.d_model * 4, cudaMemcpyDefault, s));
+  if (logits)
+    FL_TRY(cudaMemcpyAsync(logits, ctx->logits_ws, static_cast<size_t>(B) * c.vocab * 4, cudaMemcpyDefault, s));
+  for (int b = 0; b < B; ++b) ctx->lens[b] += 1;
+  ctx->last_N = B;
+  ctx->last_nsel = ctx->lazy ? n_select(c.rho, B) : B;
+  ctx->last_decode = 1;
+  ctx->last_tiles = B;
+  return FL_OK;
+}
+
+fl_status flashloop_kv_bytes_for(const flashloop_config* cfg, size_t* total, double* per_token_per_layer,
+                                 double* dense_per_token_per_layer) {
+  if (!valid_config(cfg)) return FL_ERR_INVALID_ARG;
+  const flashloop_config& c = *cfg;
+  const double hd = c.head_dim, kv = 2.0 * c.n_kv_heads;
+  const double dense = kv * c.n_loops * hd * 2.0;
+  double per = dense;
+  if (c.resid_bits != 16)
+    per = kv * (hd * 2.0 + (c.n_loops - 1) * (hd * c.resid_bits / 8.0 + (hd / c.group_size) * 2.0));
+  if (per_token_per_layer) *per_token_per_layer = per;
+  if (dense_per_token_per_layer) *dense_per_token_per_layer = dense;
+  if (total) *total = static_cast<size_t>(per * c.n_layers * c.max_batch * static_cast<double>(c.max_ctx));
+  return FL_OK;
+}
+
+fl_status flashloop_kv_bytes(const flashloop_ctx* ctx, size_t* total, double* per_token_per_layer,
+                             double* dense_per_token_per_layer) {
+  if (!ctx) return FL_ERR_INVALID_ARG;
+  return flashloop_kv_bytes_for(&ctx->cfg, total, per_token_per_layer, dense_per_token_per_layer);
+}
+
+fl_status flashloop_reset(flashloop_ctx* ctx, const int* seq_len, fl_stream_t stream) {
+  if (!ctx) return FL_ERR_INVALID_ARG;
+  const int B = ctx->cfg.max_batch;
+  std::vector<int> v(B, 0);
+  if (seq_len)
+    for (int b = 0; b < B; ++b) {
+      if (seq_len[b] < 0 || seq_len[b] > ctx->cfg.max_ctx) return FL_ERR_CAPACITY;
+      v[b] = seq_len[b];
+    }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FL_TRY(cudaMemcpyAsync(ctx->seq_len, v.data(), B * 4, cudaMemcpyHostToDevice, s));
+  FL_TRY(cudaStreamSynchronize(s));
+  ctx->lens = v;
+  return FL_OK;
+}
+
+fl_status flashloop_sync_status(flashloop_ctx* ctx, fl_stream_t stream) {
+  if (!ctx) return FL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FL_TRY(cudaStreamSynchronize(s));
+  int st = 0;
+  FL_TRY(cudaMemcpy(&st, ctx->status, 4, cudaMemcpyDeviceToHost));
+  if (st) {
+    const int zero = 0;
+    FL_TRY(cudaMemcpy(ctx->status, &zero, 4, cudaMemcpyHostToDevice));
+  }
+  if (st & kErrWaitTimeout) return FL_ERR_TIMEOUT;
+  if (st) return FL_ERR_NONFINITE;
+  return FL_OK;
+}
+
+fl_status flashloop_import_lazy(flashloop_ctx* ctx, int layer, int seq, int n, const uint16_t* base_k,
+                                const uint16_t* base_v, const int8_t* codes_k, const int8_t* codes_v,
+                                const uint16_t* scales_k, const uint16_t* scales_v, fl_stream_t stream) {
+  if (!ctx || !ctx->lazy) return FL_ERR_INVALID_ARG;
+  const flashloop_config& c = ctx->cfg;
+  if (layer < 0 || layer >= c.n_layers || seq < 0 || seq >= c.max_batch || n < 0 || n > c.max_ctx)
+    return FL_ERR_INVALID_ARG;
+  if (!base_k || !base_v || (c.n_loops > 1 && (!codes_k || !codes_v || !scales_k || !scales_v)))
+    return FL_ERR_INVALID_ARG;
+  if (n == 0) return FL_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int Hkv = c.n_kv_heads, hd = c.head_dim, ns = hd / c.group_size;
+  const CacheView& cv = ctx->cv;
+  for (int kv = 0; kv < 2; ++kv) {
+    const uint16_t* base = kv ? base_v : base_k;
+    for (int h = 0; h < Hkv; ++h)
+      FL_TRY(cudaMemcpyAsync(cv.base_row(layer, kv, seq, h, 0), base + static_cast<size_t>(h) * n * hd,
+                             static_cast<size_t>(n) * hd * 2, cudaMemcpyDefault, s));
+    const int8_t* codes = kv ? codes_v : codes_k;
+    const uint16_t* scales = kv ? scales_v : scales_k;
+    for (int l = 2; l <= c.n_loops; ++l)
+      for (int h = 0; h < Hkv; ++h) {
+        const size_t src = (static_cast<size_t>(l - 2) * Hkv + h) * n;
+        FL_TRY(launch_pack_codes(codes + src * hd, n, hd, c.resid_bits, cv.code_row(layer, l, kv, seq, h, 0),
+                                 cv.row_bytes_codes(), s));
+        FL_TRY(cudaMemcpyAsync(cv.scale_row(layer, l, kv, seq, h, 0), scales + src * ns,
+                               static_cast<size_t>(n) * ns * 2, cudaMemcpyDefault, s));
+      }
+  }
+  return FL_OK;
+}
+
+fl_status flashloop_import_dense(flashloop_ctx* ctx, int layer, int seq, int n, const uint16_t* kv_k,
+                                 const uint16_t* kv_v, fl_stream_t stream) {
+  if (!ctx || ctx->lazy) return FL_ERR_INVALID_ARG;
+  const flashloop_config& c = ctx->cfg;
+  if (layer < 0 || layer >= c.n_layers || seq < 0 || seq >= c.max_batch || n < 0 || n > c.max_ctx || !kv_k || !kv_v)
+    return FL_ERR_INVALID_ARG;
+  if (n == 0) return FL_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int Hkv = c.n_kv_heads, hd = c.head_dim;
+  for (int kv = 0; kv < 2; ++kv) {
+    const uint16_t* src = kv ? kv_v : kv_k;
+    for (int l = 1; l <= c.n_loops; ++l)
+      for (int h = 0; h < Hkv; ++h)
+        FL_TRY(cudaMemcpyAsync(ctx->cv.dense_row(layer, l, kv, seq, h, 0),
+                               src + (static_cast<size_t>(l - 1) * Hkv + h) * n * hd, static_cast<size_t>(n) * hd * 2,
+                               cudaMemcpyDefault, s));
+  }
+  return FL_OK;
+}
+
+fl_status flashloop_export_slice(const flashloop_ctx* ctx, int layer, int loop, int seq, int which, int n,
+                                 void* codes, void* scales, fl_stream_t stream) {
+  if (!ctx || !codes) return FL_ERR_INVALID_ARG;
+  const flashloop_config& c = ctx->cfg;
+  if (layer < 0 || layer >= c.n_layers || loop < 1 || loop > c.n_loops || seq < 0 || seq >= c.max_batch || n < 0 ||
+      n > c.max_ctx || (which != 0 && which != 1))
+    return FL_ERR_INVALID_ARG;
+  flashloop_ctx* mctx = const_cast<flashloop_ctx*>(ctx);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int Hkv = c.n_kv_heads, hd = c.head_dim;
+  const CacheView& cv = ctx->cv;
+  if (!ctx->lazy || loop == 1) {
+    for (int h = 0; h < Hkv; ++h) {
+      const uint16_t* src = ctx->lazy ? cv.base_row(layer, which, seq, h, 0) : cv.dense_row(layer, loop, which, seq, h, 0);
+      if (cudaMemcpyAsync(static_cast<uint16_t*>(codes) + static_cast<size_t>(h) * n * hd, src,
+                          static_cast<size_t>(n) * hd * 2, cudaMemcpyDefault, s) != cudaSuccess) {
+        mctx->last_err = "export copy failed";
+        return FL_ERR_CUDA;
+      }
+    }
+    return FL_OK;
+  }
+  if (!scales) return FL_ERR_INVALID_ARG;
+  const size_t rb = cv.row_bytes_codes();
+  const int ns = hd / c.group_size;
+  for (int h = 0; h < Hkv; ++h) {
+    if (cudaMemcpyAsync(static_cast<uint8_t*>(codes) + static_cast<size_t>(h) * n * rb,
+                        cv.code_row(layer, loop, which, seq, h, 0), static_cast<size_t>(n) * rb, cudaMemcpyDefault,
+                        s) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint16_t*>(scales) + static_cast<size_t>(h) * n * ns,
+                        cv.scale_row(layer, loop, which, seq, h, 0), static_cast<size_t>(n) * ns * 2,
+                        cudaMemcpyDefault, s) != cudaSuccess) {
+      mctx->last_err = "export copy failed";
+      return FL_ERR_CUDA;
+    }
+  }
+  return FL_OK;
+}
+
+fl_status flashloop_force_selection(flashloop_ctx* ctx, const int32_t* sel, int n_sel_loops, int n_sel,
+                                    const int32_t* cols, const int32_t* ncols, int n_tiles) {
+  if (!ctx || !ctx->lazy) return FL_ERR_INVALID_ARG;
+  const flashloop_config& c = ctx->cfg;
+  const int on = (sel && cols && ncols) ? 1 : 0;
+  if (on) {
+    if (n_sel_loops != c.n_loops - 1 || n_sel < 1 || n_sel > ctx->N_max || n_tiles < 1 || n_tiles > ctx->n_tiles_max)
+      return FL_ERR_INVALID_ARG;
+    for (int l = 0; l < n_sel_loops; ++l)
+      FL_TRY(cudaMemcpy(ctx->forced_sel + static_cast<size_t>(l) * ctx->N_max, sel + static_cast<size_t>(l) * n_sel,
+                        static_cast<size_t>(n_sel) * 4, cudaMemcpyHostToDevice));
+    const size_t per_tile = static_cast<size_t>(c.n_kv_heads) * c.c_cols;
+    for (int j = 0; j < c.n_layers; ++j) {
+      FL_TRY(cudaMemcpy(ctx->forced_cols + static_cast<size_t>(j) * ctx->n_tiles_max * per_tile,
+                        cols + static_cast<size_t>(j) * n_tiles * per_tile, n_tiles * per_tile * 4,
+                        cudaMemcpyHostToDevice));
+      FL_TRY(cudaMemcpy(ctx->forced_ncols + static_cast<size_t>(j) * ctx->n_tiles_max * c.n_kv_heads,
+                        ncols + static_cast<size_t>(j) * n_tiles * c.n_kv_heads,
+                        static_cast<size_t>(n_tiles) * c.n_kv_heads * 4, cudaMemcpyHostToDevice));
+    }
+  }
+  FL_TRY(cudaMemcpy(ctx->forced_on, &on, 4, cudaMemcpyHostToDevice));
+  return FL_OK;
+}
+
+fl_status flashloop_read_trace(flashloop_ctx* ctx, int32_t* sel, float* keys, int32_t* cols, int32_t* ncols,
+                               fl_stream_t stream) {
+  if (!ctx || !ctx->lazy) return FL_ERR_INVALID_ARG;
+  const flashloop_config& c = ctx->cfg;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FL_TRY(cudaStreamSynchronize(s));
+  const int L = c.n_loops - 1, n_sel = ctx->last_nsel, N = ctx->last_N, nt = ctx->last_tiles;
+  for (int l = 0; l < L; ++l) {
+    if (sel)
+      FL_TRY(cudaMemcpy(sel + static_cast<size_t>(l) * n_sel, ctx->idx_sel + static_cast<size_t>(l) * ctx->N_max,
+                        static_cast<size_t>(n_sel) * 4, cudaMemcpyDeviceToHost));
+    if (keys)
+      FL_TRY(cudaMemcpy(keys + static_cast<size_t>(l) * N, ctx->keys_trace + static_cast<size_t>(l) * ctx->N_max,
+                        static_cast<size_t>(N) * 4, cudaMemcpyDeviceToHost));
+  }
+  const size_t per_tile = static_cast<size_t>(c.n_kv_heads) * c.c_cols;
+  for (int j = 0; j < c.n_layers; ++j) {
+    if (cols)
+      FL_TRY(cudaMemcpy(cols + static_cast<size_t>(j) * nt * per_tile,
+                        ctx->cols + static_cast<size_t>(j) * ctx->n_tiles_max * per_tile, nt * per_tile * 4,
+                        cudaMemcpyDeviceToHost));
+    if (ncols)
+      FL_TRY(cudaMemcpy(ncols + static_cast<size_t>(j) * nt * c.n_kv_heads,
+                        ctx->ncols + static_cast<size_t>(j) * ctx->n_tiles_max * c.n_kv_heads,
+                        static_cast<size_t>(nt) * c.n_kv_heads * 4, cudaMemcpyDeviceToHost));
+  }
+  return FL_OK;
+}
+
+// ---------------------------------------------------------------- unit entry points
+fl_status fl_test_topk(const float* keys, int n_seg, int n, int k, int32_t* idx, fl_stream_t stream) {
+  if (!keys || !idx || n_seg < 0 || n < 0 || k < 0) return FL_ERR_INVALID_ARG;
+  if (n_seg == 0 || n == 0 || k == 0) return FL_OK;
+  fl::kernels_init_attrs();
+  return launch_topk(keys, n_seg, n, k, idx, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? FL_OK
+                                                                                                   : FL_ERR_CUDA;
+}
+
+fl_status fl_test_quantize(const float* r, int rows, int width, int g, int bits, uint8_t* codes, uint16_t* scales,
+                           fl_stream_t stream) {
+  if (!r || !codes || !scales || rows < 0 || width <= 0) return FL_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 4) return FL_ERR_INVALID_ARG;
+  if (g != 32 && g != 64 && g != 128) return FL_ERR_INVALID_ARG;
+  if (width % g) return FL_ERR_INVALID_ARG;
+  if (width % 128 != 0 && width != 64) return FL_ERR_INVALID_ARG;
+  if (width == 64 && g > 64) return FL_ERR_INVALID_ARG;
+  if (rows == 0) return FL_OK;
+  return launch_quantize_rows(r, rows, width, g, bits, codes, scales, reinterpret_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess ? FL_OK : FL_ERR_CUDA;
+}
+
+size_t fl_test_gemm_scratch_bytes(int m, int n, int k, int swap_ab) {
+  if (!swap_ab || m < 1 || m > 64 || n < 1 || k < 1) return 0;
+  const int tiles = ceil_div(n, 128);
+  const int splits = split_factor(tiles, ceil_div(k, 64));
+  return gemm_partial_floats(swap_bn(m), 0, tiles, splits) * 4 + static_cast<size_t>(tiles) * 4 + 256;
+}
+
+fl_status fl_test_gemm(const uint16_t* A, const uint16_t* B, float* D, int m, int n, int k, int swap_ab,
+                       void* scratch, size_t scratch_bytes, fl_stream_t stream) {
+  if (!A || !B || !D || m < 1 || n < 1 || k < 8 || k % 8) return FL_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return FL_ERR_INVALID_ARG;
+  if (swap_ab && m > 64) return FL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  fl::gemm_init_attrs();
+  GemmLaunch g{};
+  GemmArgs& a = g.args;
+  CUtensorMap ta, tb;
+  a.k_chunks = ceil_div(k, 64);
+  a.epi = kEpiStore;
+  a.out = D;
+  a.ldo = n;
+  a.n_feat = n;
+  a.n_tok = m;
+  if (swap_ab) {
+    const int bn = swap_bn(m);
+    const int tiles = ceil_div(n, 128);
+    const int splits = split_factor(tiles, a.k_chunks);
+    const size_t need = fl_test_gemm_scratch_bytes(m, n, k, 1);
+    if (splits > 1 && (!scratch || scratch_bytes < need || (reinterpret_cast<uintptr_t>(scratch) & 255)))
+      return FL_ERR_WORKSPACE;
+    if (!encode_tmap_bf16(&ta, B, k, n, 0, 128) || !encode_tmap_bf16(&tb, A, k, m, 0, bn)) return FL_ERR_INVALID_ARG;
+    g.a0 = &ta; g.b0 = &tb; g.bn = bn;
+    a.swap = 1; a.splits = splits;
+    if (splits > 1) {
+      a.partial = static_cast<float*>(scratch);
+      a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(scratch) +
+                                          ((gemm_partial_floats(bn, 0, tiles, splits) * 4 + 255) & ~size_t(255)));
+      if (cudaMemsetAsync(a.counters, 0, static_cast<size_t>(tiles) * 4, s) != cudaSuccess) return FL_ERR_CUDA;
+    }
+    g.grid = dim3(tiles, 1, splits);
+  } else {
+    if (!encode_tmap_bf16(&ta, A, k, m, 0, 128) || !encode_tmap_bf16(&tb, B, k, n, 0, 128)) return FL_ERR_INVALID_ARG;
+    g.a0 = &ta; g.b0 = &tb; g.bn = 128;
+    a.swap = 0; a.splits = 1;
+    g.grid = dim3(ceil_div(m, 128), ceil_div(n, 128), 1);
+  }
+  return launch_gemm(g, s) == cudaSuccess ? FL_OK : FL_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,302 @@
+"""ctypes binding of ``libflashloop.so`` (declared in ``include/flashloop.h``).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  torch provides device memory (the workspace and the weight tensors)
+and streams.  Loading fails loudly when the library is missing; there is no
+fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libflashloop.so")
+
+FL_OK = 0
+FL_OPT_USE_GRAPH = 1
+STATUS = {0: "ok", 1: "invalid argument", 2: "capacity exceeded", 3: "workspace", 4: "cuda error",
+          5: "timeout", 6: "nonfinite", 7: "unsupported"}
+
+
+class FlashLoopError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: str = ""):
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({status}) {detail}".strip())
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [("d_model", ctypes.c_int), ("n_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("ffn_dim", ctypes.c_int), ("n_layers", ctypes.c_int),
+                ("n_loops", ctypes.c_int), ("rho", ctypes.c_double), ("c_cols", ctypes.c_int),
+                ("q_tile", ctypes.c_int), ("resid_bits", ctypes.c_int), ("group_size", ctypes.c_int),
+                ("resid_scale", ctypes.c_float), ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
+                ("vocab", ctypes.c_int), ("max_batch", ctypes.c_int), ("max_ctx", ctypes.c_int),
+                ("max_tokens", ctypes.c_int)]
+
+
+class Weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("attn_norm", "w_qkv", "w_o", "mlp_norm", "w_gate", "w_up",
+                                               "w_down", "final_norm", "w_out")]
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SIG = {
+    "flashloop_workspace_bytes": (ctypes.c_size_t, [ctypes.POINTER(Config)]),
+    "flashloop_init": (_I, [ctypes.POINTER(Config), ctypes.POINTER(Weights), _P, ctypes.c_size_t, _P,
+                            ctypes.POINTER(_P)]),
+    "flashloop_prefill": (_I, [_P, _P, _I, _I, _P, _P, _P]),
+    "flashloop_decode_step": (_I, [_P, _P, _I, _P, _P, _P]),
+    "flashloop_kv_bytes": (_I, [_P, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_double),
+                                ctypes.POINTER(ctypes.c_double)]),
+    "flashloop_kv_bytes_for": (_I, [ctypes.POINTER(Config), ctypes.POINTER(ctypes.c_size_t),
+                                    ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
+    "flashloop_reset": (_I, [_P, _P, _P]),
+    "flashloop_sync_status": (_I, [_P, _P]),
+    "flashloop_destroy": (None, [_P]),
+    "flashloop_status_string": (ctypes.c_char_p, [_I]),
+    "flashloop_last_cuda_error": (ctypes.c_char_p, [_P]),
+    "flashloop_import_lazy": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
+    "flashloop_import_dense": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "flashloop_export_slice": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "flashloop_force_selection": (_I, [_P, _P, _I, _I, _P, _P, _I]),
+    "flashloop_read_trace": (_I, [_P, _P, _P, _P, _P, _P]),
+    "flashloop_set_option": (_I, [_P, _I, _I]),
+    "fl_test_topk": (_I, [_P, _I, _I, _I, _P, _P]),
+    "fl_test_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
+    "fl_test_gemm_scratch_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "fl_test_gemm": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_size_t, _P]),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise FileNotFoundError(f"{LIB_PATH} is missing: run `python -m cross_loop_sparsity_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIG.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(st: int, what: str, ctx=None):
+    if st != FL_OK:
+        detail = ""
+        if ctx:
+            e = lib().flashloop_last_cuda_error(ctx)
+            detail = e.decode() if e else ""
+        raise FlashLoopError(st, what, detail)
+
+
+def make_config(cfg, max_batch: int, max_ctx: int, max_tokens: int = 0, resid_bits: int | None = None) -> Config:
+    """Fill the C config from a ``synth.LoopConfig``-like object."""
+    return Config(cfg.d_model, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.ffn_dim, cfg.n_layers, cfg.n_loops,
+                  float(cfg.rho), cfg.c_cols, cfg.q_tile, cfg.resid_bits if resid_bits is None else resid_bits,
+                  cfg.group_size, float(cfg.resid_scale), float(cfg.rms_eps), float(cfg.rope_theta), cfg.vocab,
+                  max_batch, max_ctx, max_tokens)
+
+
+def workspace_bytes(c: Config) -> int:
+    return int(lib().flashloop_workspace_bytes(ctypes.byref(c)))
+
+
+def kv_bytes_for(c: Config):
+    tot, per, dense = ctypes.c_size_t(), ctypes.c_double(), ctypes.c_double()
+    _check(lib().flashloop_kv_bytes_for(ctypes.byref(c), ctypes.byref(tot), ctypes.byref(per), ctypes.byref(dense)),
+           "kv_bytes_for")
+    return int(tot.value), per.value, dense.value
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream):
+    return None if stream is None else ctypes.c_void_p(stream.cuda_stream)
+
+
+def upload_weights(w: dict, device="cuda"):
+    """Stack the generator's per-layer weights into device tensors (bf16 bits as int16)."""
+    import torch
+
+    def stack(name, dt=np.uint16):
+        a = np.stack([lw[name] for lw in w["layers"]]).astype(dt, copy=False)
+        if dt == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(device)
+        return torch.from_numpy(a).to(device)
+
+    return {
+        "attn_norm": stack("attn_norm", np.float32), "w_qkv": stack("w_qkv"), "w_o": stack("w_o"),
+        "mlp_norm": stack("mlp_norm", np.float32), "w_gate": stack("w_gate"), "w_up": stack("w_up"),
+        "w_down": stack("w_down"),
+        "final_norm": torch.from_numpy(np.asarray(w["final_norm"], np.float32)).to(device),
+        "w_out": torch.from_numpy(np.asarray(w["w_out"]).view(np.int16)).to(device),
+    }
+
+
+class FlashLoop:
+    """One context: a KV cache and the per-call state in a torch-owned workspace."""
+
+    def __init__(self, cfg, dev_weights: dict, max_batch: int, max_ctx: int, max_tokens: int = 0,
+                 resid_bits: int | None = None, stream=None):
+        import torch
+        self.cfg = cfg
+        self.c = make_config(cfg, max_batch, max_ctx, max_tokens, resid_bits)
+        self.weights = dev_weights  # keep alive: the library borrows these pointers
+        nbytes = workspace_bytes(self.c)
+        if nbytes == 0:
+            raise FlashLoopError(1, "workspace_bytes", "invalid config")
+        self.workspace = torch.empty(nbytes + 256, dtype=torch.uint8, device="cuda")
+        off = (-self.workspace.data_ptr()) % 256
+        self._ws_ptr = self.workspace.data_ptr() + off
+        self._ws_bytes = nbytes
+        wt = Weights(*[dev_weights[n].data_ptr() for n, _ in Weights._fields_])
+        self._wstruct = wt
+        ctx = ctypes.c_void_p()
+        st = lib().flashloop_init(ctypes.byref(self.c), ctypes.byref(wt), ctypes.c_void_p(self._ws_ptr),
+                                  ctypes.c_size_t(nbytes), _stream_ptr(stream), ctypes.byref(ctx))
+        _check(st, "flashloop_init")
+        self.ctx = ctx
+        self.lazy = self.c.resid_bits != 16
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            lib().flashloop_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- calls ---------------------------------------------------------------
+    def prefill(self, h0, B: int, T: int, h_out=None, logits=None, stream=None):
+        _check(lib().flashloop_prefill(self.ctx, _ptr(h0), B, T, _ptr(h_out), _ptr(logits), _stream_ptr(stream)),
+               "flashloop_prefill", self.ctx)
+
+    def decode_step(self, h0, B: int, h_out=None, logits=None, stream=None):
+        _check(lib().flashloop_decode_step(self.ctx, _ptr(h0), B, _ptr(h_out), _ptr(logits), _stream_ptr(stream)),
+               "flashloop_decode_step", self.ctx)
+
+    def kv_bytes(self):
+        tot, per, dense = ctypes.c_size_t(), ctypes.c_double(), ctypes.c_double()
+        _check(lib().flashloop_kv_bytes(self.ctx, ctypes.byref(tot), ctypes.byref(per), ctypes.byref(dense)),
+               "flashloop_kv_bytes")
+        return int(tot.value), per.value, dense.value
+
+    def reset(self, lens=None, stream=None):
+        arr = None
+        if lens is not None:
+            v = np.zeros(self.c.max_batch, np.int32)
+            v[:len(lens)] = np.asarray(lens, np.int32)
+            arr = v.ctypes.data_as(ctypes.c_void_p)
+            self._lens_keep = v
+        _check(lib().flashloop_reset(self.ctx, arr, _stream_ptr(stream)), "flashloop_reset", self.ctx)
+
+    def sync_status(self, stream=None) -> int:
+        return int(lib().flashloop_sync_status(self.ctx, _stream_ptr(stream)))
+
+    def set_option(self, opt: int, value: int):
+        _check(lib().flashloop_set_option(self.ctx, opt, value), "flashloop_set_option")
+
+    # -- cache import / export --------------------------------------------------
+    def import_lazy(self, layer, seq, base_k, base_v, codes_k, codes_v, scales_k, scales_v, stream=None):
+        n = base_k.shape[1]
+        _check(lib().flashloop_import_lazy(self.ctx, layer, seq, n, _ptr(base_k), _ptr(base_v), _ptr(codes_k),
+                                           _ptr(codes_v), _ptr(scales_k), _ptr(scales_v), _stream_ptr(stream)),
+               "flashloop_import_lazy", self.ctx)
+
+    def import_dense(self, layer, seq, kv_k, kv_v, stream=None):
+        n = kv_k.shape[2]
+        _check(lib().flashloop_import_dense(self.ctx, layer, seq, n, _ptr(kv_k), _ptr(kv_v), _stream_ptr(stream)),
+               "flashloop_import_dense", self.ctx)
+
+    def export_slice(self, layer, loop, seq, which, n, stream=None):
+        """Returns (codes, scales) numpy arrays; loop 1 (or dense) returns (bf16 bits [Hkv][n][hd], None)."""
+        import torch
+        c = self.c
+        if not self.lazy or loop == 1:
+            out = torch.empty((c.n_kv_heads, n, c.head_dim), dtype=torch.int16, device="cuda")
+            _check(lib().flashloop_export_slice(self.ctx, layer, loop, seq, which, n, _ptr(out), None,
+                                                _stream_ptr(stream)), "export", self.ctx)
+            torch.cuda.synchronize()
+            return out.cpu().numpy().view(np.uint16), None
+        rb = c.head_dim * c.resid_bits // 8
+        codes = torch.empty((c.n_kv_heads, n, rb), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((c.n_kv_heads, n, c.head_dim // c.group_size), dtype=torch.int16, device="cuda")
+        _check(lib().flashloop_export_slice(self.ctx, layer, loop, seq, which, n, _ptr(codes), _ptr(scales),
+                                            _stream_ptr(stream)), "export", self.ctx)
+        torch.cuda.synchronize()
+        return codes.cpu().numpy(), scales.cpu().numpy().view(np.float16)
+
+    def force_selection(self, sel=None, cols=None, ncols=None, n_tiles: int = 0):
+        if sel is None:
+            _check(lib().flashloop_force_selection(self.ctx, None, 0, 0, None, None, 0), "force_selection")
+            return
+        sel = np.ascontiguousarray(sel, np.int32)
+        cols = np.ascontiguousarray(cols, np.int32)
+        ncols = np.ascontiguousarray(ncols, np.int32)
+        self._forced_keep = (sel, cols, ncols)
+        _check(lib().flashloop_force_selection(self.ctx, sel.ctypes.data_as(ctypes.c_void_p), sel.shape[0],
+                                               sel.shape[1], cols.ctypes.data_as(ctypes.c_void_p),
+                                               ncols.ctypes.data_as(ctypes.c_void_p), n_tiles),
+               "force_selection", self.ctx)
+
+    def read_trace(self, N: int, n_sel: int, n_tiles: int, stream=None):
+        c = self.c
+        L = c.n_loops - 1
+        sel = np.zeros((L, n_sel), np.int32)
+        keys = np.zeros((L, N), np.float32)
+        cols = np.zeros((c.n_layers, n_tiles, c.n_kv_heads, c.c_cols), np.int32)
+        ncols = np.zeros((c.n_layers, n_tiles, c.n_kv_heads), np.int32)
+        _check(lib().flashloop_read_trace(self.ctx, sel.ctypes.data_as(ctypes.c_void_p),
+                                          keys.ctypes.data_as(ctypes.c_void_p), cols.ctypes.data_as(ctypes.c_void_p),
+                                          ncols.ctypes.data_as(ctypes.c_void_p), _stream_ptr(stream)),
+               "read_trace", self.ctx)
+        return sel, keys, cols, ncols
+
+
+# ---------------------------------------------------------------------------- unit entry points
+def topk(keys, k: int, stream=None):
+    """keys: cuda float32 [n_seg, n]; returns cuda int32 [n_seg, min(k, n)]."""
+    import torch
+    n_seg, n = keys.shape
+    out = torch.empty((n_seg, min(k, n)), dtype=torch.int32, device=keys.device)
+    _check(lib().fl_test_topk(_ptr(keys), n_seg, n, k, _ptr(out), _stream_ptr(stream)), "fl_test_topk")
+    return out
+
+
+def quantize(r, g: int, bits: int, stream=None):
+    """r: cuda float32 [rows, width]; returns (packed codes uint8, fp16 scale bits int16)."""
+    import torch
+    rows, width = r.shape
+    codes = torch.empty((rows, width * bits // 8), dtype=torch.uint8, device=r.device)
+    scales = torch.empty((rows, width // g), dtype=torch.int16, device=r.device)
+    _check(lib().fl_test_quantize(_ptr(r), rows, width, g, bits, _ptr(codes), _ptr(scales), _stream_ptr(stream)),
+           "fl_test_quantize")
+    return codes, scales
+
+
+def gemm(A, B, swap_ab: bool = False, stream=None):
+    """D = A @ B.T on the tcgen05 kernel; A [m,k], B [n,k] bf16 (cuda); returns fp32 [m,n]."""
+    import torch
+    m, k = A.shape
+    n = B.shape[0]
+    D = torch.empty((m, n), dtype=torch.float32, device=A.device)
+    nb = int(lib().fl_test_gemm_scratch_bytes(m, n, k, int(swap_ab)))
+    scratch = torch.empty(max(nb, 256) + 256, dtype=torch.uint8, device=A.device)
+    sp = scratch.data_ptr() + ((-scratch.data_ptr()) % 256)
+    _check(lib().fl_test_gemm(_ptr(A), _ptr(B), _ptr(D), m, n, k, int(swap_ab), ctypes.c_void_p(sp), nb,
+                              _stream_ptr(stream)), "fl_test_gemm")
+    return D

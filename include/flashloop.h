@@ -1,0 +1,226 @@
+/*
+ * flashloop.h -- C ABI of the B200 (sm_100a) lazy-update looped-Transformer
+ * inference library.
+ *
+ * The method is the one in "FlashLoop: Fast and Memory-Efficient Looped
+ * Transformers via Lazy Updates" (abstract): a shared Transformer block is
+ * applied K times; after the first loop only the tokens whose hidden state
+ * changed most are recomputed (token-sparse updates), their attention output
+ * is corrected over a sparse, stable set of key columns (sparse attention),
+ * and each loop's KV cache is the previous loop's plus a low-bit residual
+ * (KV-residual quantisation).  The dense baseline is the plain looped forward
+ * with a per-loop KV cache ("Looped Transformer 教程：权重共享、循环次数与推理
+ * 成本怎么读", 第一步 and 第四步).
+ *
+ * Conventions for every entry point:
+ *  - Device pointers are CUDA global-memory addresses on the device that was
+ *    current at flashloop_init.  Where an argument says "host or device", the
+ *    library asks CUDA which it is and stages host buffers through its
+ *    workspace (pinned host memory makes those copies asynchronous).
+ *  - bf16 tensors are passed as uint16_t bit patterns; linear weights are
+ *    row-major [out_features][in_features], stacked over layers.
+ *  - All work is enqueued on the given stream and returns without waiting,
+ *    except where stated.  One context is used from one stream at a time.
+ *  - Nothing aborts and no C++ exception crosses this boundary: every
+ *    failure is a fl_status.  The library never allocates device memory; the
+ *    caller provides one workspace buffer and owns every buffer it passes.
+ */
+#ifndef FLASHLOOP_H
+#define FLASHLOOP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* fl_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+  FL_OK = 0,
+  FL_ERR_INVALID_ARG = 1, /* a NULL/misaligned pointer, an out-of-range size or knob */
+  FL_ERR_CAPACITY = 2,    /* batch > max_batch, tokens > max_tokens, or context > max_ctx */
+  FL_ERR_WORKSPACE = 3,   /* workspace smaller than flashloop_workspace_bytes() or misaligned */
+  FL_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (see flashloop_last_cuda_error) */
+  FL_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out; the kernel returned early */
+  FL_ERR_NONFINITE = 6,   /* reserved: non-finite value detected by a checking build */
+  FL_ERR_UNSUPPORTED = 7  /* a configuration this build does not implement */
+} fl_status;
+
+/* Model and method knobs.  resid_bits: 4 or 2 = lazy path with int4/int2 KV
+ * residuals; 16 = dense looped baseline (every loop recomputes every token and
+ * keeps its own bf16 KV; rho and c_cols are ignored). */
+typedef struct {
+  int d_model;      /* d; multiple of 64 */
+  int n_heads;      /* H query heads */
+  int n_kv_heads;   /* Hkv; H % Hkv == 0 (grouped-query attention) */
+  int head_dim;     /* hd: 64 or 128 */
+  int ffn_dim;      /* SwiGLU hidden size; multiple of 8 */
+  int n_layers;     /* M: layers of the shared block */
+  int n_loops;      /* K: block applications per token, 1..16 */
+  double rho;       /* fraction of tokens recomputed at loops >= 2, in (0, 1] */
+  int c_cols;       /* key columns kept per (query tile, KV head), >= 1 */
+  int q_tile;       /* prefill query-tile length in positions (128) */
+  int resid_bits;   /* 4, 2 or 16 (see above) */
+  int group_size;   /* quantiser group along head_dim; divides hd, multiple of 32 */
+  float resid_scale;/* s: h += s * branch output (0.3) */
+  float rms_eps;    /* RMSNorm epsilon (1e-6) */
+  float rope_theta; /* RoPE base (10000) */
+  int vocab;        /* LM-head rows V */
+  int max_batch;    /* sequences held in the cache */
+  int max_ctx;      /* positions per sequence held in the cache */
+  int max_tokens;   /* largest B*T of one prefill call (decode needs max_batch) */
+} flashloop_config;
+
+/* Device pointers to the weights (borrowed for the context's lifetime). */
+typedef struct {
+  const float* attn_norm;     /* [M][d] fp32 gains */
+  const uint16_t* w_qkv;      /* [M][(H+2Hkv)*hd][d] bf16; rows: q heads, k heads, v heads */
+  const uint16_t* w_o;        /* [M][d][H*hd] bf16 */
+  const float* mlp_norm;      /* [M][d] fp32 gains */
+  const uint16_t* w_gate;     /* [M][ffn][d] bf16 */
+  const uint16_t* w_up;       /* [M][ffn][d] bf16 */
+  const uint16_t* w_down;     /* [M][d][ffn] bf16 */
+  const float* final_norm;    /* [d] fp32 gains */
+  const uint16_t* w_out;      /* [V][d] bf16 */
+} flashloop_weights;
+
+typedef struct flashloop_ctx flashloop_ctx;
+
+/* Bytes of device workspace a context with this config needs (host arithmetic
+ * only; 0 if the config is invalid).  The workspace holds the KV cache, the
+ * per-call attention state, activations, selection buffers and split-K
+ * scratch; it must be 256-byte aligned. */
+size_t flashloop_workspace_bytes(const flashloop_config* cfg);
+
+/* Validate cfg, lay out the workspace, build TMA descriptors for the weights
+ * and zero the cache.  Enqueues on `stream` (the zeroing and the RoPE table
+ * upload) and waits for it before returning.  *out receives a host-allocated
+ * context (free with flashloop_destroy). */
+fl_status flashloop_init(const flashloop_config* cfg, const flashloop_weights* w,
+                         void* workspace, size_t workspace_bytes, fl_stream_t stream,
+                         flashloop_ctx** out);
+
+/* Prefill T tokens into each of B empty sequences (lengths must be 0).
+ * h0: [B*T][d] fp32 input hidden states, sequence-major (host or device).
+ * h_out: [B*T][d] fp32 final hidden states after K loops (host or device, may be NULL).
+ * logits_last: [B][V] fp32 logits of each sequence's last position (host or device, may be NULL).
+ * Loop 1 is dense; loops 2..K recompute ceil(rho*B*T) tokens (pooled over the
+ * call, ties to the lower flat index b*T+t).  Query tiles are q_tile
+ * positions of one sequence.  On return the sequences' lengths are T. */
+fl_status flashloop_prefill(flashloop_ctx* ctx, const float* h0, int B, int T,
+                            float* h_out, float* logits_last, fl_stream_t stream);
+
+/* Append one token to each of sequences 0..B-1 at position len_b.
+ * h0: [B][d] fp32 (host or device); h_out: [B][d] fp32 or NULL; logits: [B][V]
+ * fp32 or NULL (host or device).  The ranking pools the B new tokens; each new
+ * token is its own query tile.  The step's kernels are captured once per B
+ * into a CUDA graph and replayed.  Lengths advance by one. */
+fl_status flashloop_decode_step(flashloop_ctx* ctx, const float* h0, int B,
+                                float* h_out, float* logits, fl_stream_t stream);
+
+/* KV-cache bytes: *total = bytes of the allocated cache layout; per token and
+ * layer: *per_token_per_layer for this config and *dense_per_token_per_layer
+ * for dense per-loop bf16 KV (K * 2 * Hkv * hd * 2 bytes).  Host arithmetic. */
+fl_status flashloop_kv_bytes(const flashloop_ctx* ctx, size_t* total, double* per_token_per_layer,
+                             double* dense_per_token_per_layer);
+
+/* The same figures from a config alone (host arithmetic, no context needed):
+ * total = bytes of the cache layout flashloop_init would lay out. */
+fl_status flashloop_kv_bytes_for(const flashloop_config* cfg, size_t* total, double* per_token_per_layer,
+                                 double* dense_per_token_per_layer);
+
+/* Set every sequence length (seq_len: [max_batch] host array, or NULL for all
+ * zero).  Cache contents are kept; used to replay a decode step at a fixed
+ * context.  Enqueued on `stream`. */
+fl_status flashloop_reset(flashloop_ctx* ctx, const int* seq_len, fl_stream_t stream);
+
+/* Synchronise `stream` and report the first error a kernel recorded since
+ * the last call (FL_ERR_TIMEOUT for a bounded wait that ran out), clearing it. */
+fl_status flashloop_sync_status(flashloop_ctx* ctx, fl_stream_t stream);
+
+void flashloop_destroy(flashloop_ctx* ctx);
+const char* flashloop_status_string(fl_status s);
+/* The last CUDA error string seen by this context ("" if none). */
+const char* flashloop_last_cuda_error(const flashloop_ctx* ctx);
+
+/* ------------------------------------------------------------------------ */
+/* Cache import / export (synthetic decode contexts; checks).               */
+/* ------------------------------------------------------------------------ */
+
+/* Load one (layer, sequence) slice of a lazy cache from device buffers:
+ * base_k/base_v: [Hkv][n][hd] bf16; codes_k/v: [K-1][Hkv][n][hd] int8 codes in
+ * [-qmax, qmax] (packed by the library); scales_k/v: [K-1][Hkv][n][hd/g] fp16
+ * bits.  Rows 0..n-1 of that sequence are written.  resid_bits 2/4 only. */
+fl_status flashloop_import_lazy(flashloop_ctx* ctx, int layer, int seq, int n,
+                                const uint16_t* base_k, const uint16_t* base_v,
+                                const int8_t* codes_k, const int8_t* codes_v,
+                                const uint16_t* scales_k, const uint16_t* scales_v,
+                                fl_stream_t stream);
+
+/* Load one (layer, sequence) slice of a dense per-loop cache: kv_k/kv_v
+ * [K][Hkv][n][hd] bf16.  resid_bits 16 only. */
+fl_status flashloop_import_dense(flashloop_ctx* ctx, int layer, int seq, int n,
+                                 const uint16_t* kv_k, const uint16_t* kv_v, fl_stream_t stream);
+
+/* Copy one (layer, loop, sequence) slice of the residual store to device
+ * buffers: codes [Hkv][n][hd*bits/8] packed bytes, scales [Hkv][n][hd/g] fp16
+ * bits (loop 2..K); loop 1 copies the base: base [2][Hkv][n][hd] bf16 into
+ * `codes` (K then V) and leaves `scales` untouched.  `which`: 0 = K, 1 = V. */
+fl_status flashloop_export_slice(const flashloop_ctx* ctx, int layer, int loop, int seq, int which,
+                                 int n, void* codes, void* scales, fl_stream_t stream);
+
+/* Force the selections of the next call (checks only): sel [K-1][n_sel]
+ * ascending token indices for loops 2..K; cols [M][n_tiles][Hkv][c_cols]
+ * ascending column indices with ncols [M][n_tiles][Hkv] valid entries (host
+ * arrays; NULL clears).  n_tiles is B for decode, B*ceil(T/q_tile) for
+ * prefill.  The kernels still compute every key; only the chosen indices are
+ * replaced. */
+fl_status flashloop_force_selection(flashloop_ctx* ctx, const int32_t* sel, int n_sel_loops, int n_sel,
+                                    const int32_t* cols, const int32_t* ncols, int n_tiles);
+
+/* Read back the last call's choices (host buffers): sel [K-1][n_sel]; keys
+ * [K-1][N] fp32 selection keys of loops 2..K; cols/ncols as above.  Any may be
+ * NULL.  Synchronises `stream`. */
+fl_status flashloop_read_trace(flashloop_ctx* ctx, int32_t* sel, float* keys, int32_t* cols,
+                               int32_t* ncols, fl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Unit entry points on caller buffers (device pointers).                    */
+/* ------------------------------------------------------------------------ */
+
+/* Top-k selection per segment: keys fp32 [n_seg][n]; for segment s the k
+ * largest by (IEEE bit pattern as uint32 descending, index ascending), written
+ * in ascending index order to idx [n_seg][k] (k = min(k, n)).  Token-sparse
+ * updates and the top-c key columns ("FlashLoop ...", abstract). */
+fl_status fl_test_topk(const float* keys, int n_seg, int n, int k, int32_t* idx, fl_stream_t stream);
+
+/* Per-group absmax quantiser: r fp32 [rows][width] (width % g == 0); writes
+ * packed codes [rows][width*bits/8] and fp16 scale bits [rows][width/g]:
+ * s = fp16_RU(fp32(absmax/qmax)), code = clamp(rint(fp32(r/s))) (KV-residual
+ * quantisation, "FlashLoop ...", abstract).  bits 4 or 2; g multiple of 32. */
+fl_status fl_test_quantize(const float* r, int rows, int width, int g, int bits,
+                           uint8_t* codes, uint16_t* scales, fl_stream_t stream);
+
+/* tcgen05 GEMM: D[m][n] = sum_k A[m][k] * B[n][k] (bf16 operands, fp32
+ * accumulate); A [m][k] and B [n][k] row-major bf16, D fp32 [m][n]; k % 8 == 0,
+ * all pointers 16-byte aligned.  swap_ab = 0: A's rows on the MMA M side
+ * (128-row tiles), B in 128-row tiles.  swap_ab = 1: the skinny orientation
+ * used for decode (B's rows on the MMA M side, m <= 64 rows of A as the MMA N
+ * side), with the reduction split across CTAs; `scratch` must then hold
+ * fl_test_gemm_scratch_bytes() bytes (caller-allocated device memory). */
+size_t fl_test_gemm_scratch_bytes(int m, int n, int k, int swap_ab);
+fl_status fl_test_gemm(const uint16_t* A, const uint16_t* B, float* D, int m, int n, int k, int swap_ab,
+                       void* scratch, size_t scratch_bytes, fl_stream_t stream);
+
+/* Runtime options of a context. */
+typedef enum {
+  FL_OPT_USE_GRAPH = 1 /* 1 (default): capture decode steps into CUDA graphs; 0: launch directly */
+} fl_option;
+fl_status flashloop_set_option(flashloop_ctx* ctx, fl_option opt, int value);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FLASHLOOP_H */
