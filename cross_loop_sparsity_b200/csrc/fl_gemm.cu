@@ -258,26 +258,25 @@ cudaError_t launch_one(const GemmLaunch& g, cudaStream_t stream) {
 }
 
 template <int BN, bool DA, bool DB, bool SWAP>
-void set_attr() {
-  cudaFuncSetAttribute(k_gemm_tc<BN, DA, DB, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       Cfg<BN, DA, DB>::kSmemBytes);
+cudaError_t set_attr() {
+  return cudaFuncSetAttribute(k_gemm_tc<BN, DA, DB, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Cfg<BN, DA, DB>::kSmemBytes);
 }
 
 }  // namespace
 
 // Opt every GEMM instantiation in to its dynamic shared memory once, outside any capture.
-void gemm_init_attrs() {
-  static bool done = false;
-  if (done) return;
-  set_attr<16, true, false, true>();
-  set_attr<16, false, false, true>();
-  set_attr<32, true, false, true>();
-  set_attr<32, false, false, true>();
-  set_attr<64, true, false, true>();
-  set_attr<64, false, false, true>();
-  set_attr<128, false, true, false>();
-  set_attr<128, false, false, false>();
-  done = true;
+cudaError_t gemm_init_attrs() {
+  static cudaError_t done = cudaErrorNotReady;
+  if (done == cudaSuccess) return done;
+  const cudaError_t r[8] = {set_attr<16, true, false, true>(),   set_attr<16, false, false, true>(),
+                            set_attr<32, true, false, true>(),   set_attr<32, false, false, true>(),
+                            set_attr<64, true, false, true>(),   set_attr<64, false, false, true>(),
+                            set_attr<128, false, true, false>(), set_attr<128, false, false, false>()};
+  done = cudaSuccess;
+  for (cudaError_t e : r)
+    if (e != cudaSuccess) done = e;
+  return done;
 }
 
 size_t gemm_partial_floats(int bn, int dual, int tiles, int splits) {

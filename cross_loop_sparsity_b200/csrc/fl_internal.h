@@ -52,6 +52,7 @@ struct GemmLaunch {
 };
 
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream);
+cudaError_t gemm_init_attrs();   // opt the GEMM kernels in to their shared memory (once)
 // Largest split-K scratch (floats) one launch with these sizes may use.
 size_t gemm_partial_floats(int bn, int dual, int tiles, int splits);
 

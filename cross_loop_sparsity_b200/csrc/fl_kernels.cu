@@ -1063,21 +1063,42 @@ cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
   }
   return cudaGetLastError();
 }
+// Largest dynamic shared memory a kernel may opt in to: the device's per-block
+// opt-in limit less the kernel's own static shared memory.
+template <typename F>
+int max_dyn_smem(F* kern) {
+  int dev = 0, optin = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  cudaFuncAttributes fa{};
+  cudaFuncGetAttributes(&fa, kern);
+  return optin - static_cast<int>(fa.sharedSizeBytes);
+}
+
 // Opt every large-shared-memory kernel in to its dynamic shared memory once,
-// outside any stream capture.
-void kernels_init_attrs() {
-  static bool done = false;
-  if (done) return;
-  const int pre128 = static_cast<int>(attn_prefill_smem(128)), pre64 = static_cast<int>(attn_prefill_smem(64));
-  cudaFuncSetAttribute(k_attn_prefill<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, pre128);
-  cudaFuncSetAttribute(k_attn_prefill<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, pre64);
-  cudaFuncSetAttribute(k_dscore<128, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dscore_smem(128)));
-  cudaFuncSetAttribute(k_dscore<64, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(dscore_smem(64)));
-  // the correction kernel's score buffers grow with c; allow the device maximum
-  // (configs whose need exceeds it are refused at init)
-  cudaFuncSetAttribute(k_correct<128, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-  cudaFuncSetAttribute(k_correct<64, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxDynSmem);
-  done = true;
+// outside any stream capture.  Returns the first error.
+cudaError_t kernels_init_attrs() {
+  static cudaError_t done = cudaErrorNotReady;
+  if (done == cudaSuccess) return done;
+  cudaError_t e = cudaSuccess;
+  auto set = [&](auto* kern, int bytes) {
+    const cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = r;
+  };
+  set(k_attn_prefill<128>, static_cast<int>(attn_prefill_smem(128)));
+  set(k_attn_prefill<64>, static_cast<int>(attn_prefill_smem(64)));
+  set(k_dscore<128, 4>, static_cast<int>(dscore_smem(128)));
+  set(k_dscore<64, 2>, static_cast<int>(dscore_smem(64)));
+  // the correction kernel's score buffers grow with c: allow what the device allows
+  // (configurations that need more are refused at init)
+  set(k_correct<128, 4>, max_dyn_smem(k_correct<128, 4>));
+  set(k_correct<64, 2>, max_dyn_smem(k_correct<64, 2>));
+  done = e;
+  return e;
+}
+
+size_t correct_smem_limit(int hd) {
+  return static_cast<size_t>(hd == 128 ? max_dyn_smem(k_correct<128, 4>) : max_dyn_smem(k_correct<64, 2>));
 }
 
 cudaError_t launch_pack_codes(const int8_t* src, int rows, int hd, int bits, uint8_t* dst, size_t dst_row_stride,

@@ -108,8 +108,9 @@ struct CorrectArgs {
   int* status;
 };
 
-constexpr int kMaxDynSmem = 232448;  // 227 KB: the per-block dynamic shared memory limit of sm_100
 size_t correct_smem(int hd, int grp, int c);
+size_t correct_smem_limit(int hd);   // the most the correction kernel may opt in to on this device
+cudaError_t kernels_init_attrs();
 
 cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* idx, const int* forced_on,
                                  const int32_t* forced, cudaStream_t s);

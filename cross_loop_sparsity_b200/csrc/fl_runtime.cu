@@ -21,10 +21,9 @@
 
 using namespace fl;
 
-namespace fl {
-void gemm_init_attrs();
-void kernels_init_attrs();
-}  // namespace fl
+namespace {
+std::string g_last_error;  // last CUDA error of an entry point that has no context
+}  // namespace
 
 struct flashloop_ctx {
   flashloop_config cfg;
@@ -531,16 +530,16 @@ const char* flashloop_status_string(fl_status s) {
   return "unknown status";
 }
 
-const char* flashloop_last_cuda_error(const flashloop_ctx* ctx) { return ctx ? ctx->last_err.c_str() : ""; }
+const char* flashloop_last_cuda_error(const flashloop_ctx* ctx) {
+  return ctx ? ctx->last_err.c_str() : g_last_error.c_str();
+}
 
 fl_status flashloop_init(const flashloop_config* cfg, const flashloop_weights* w, void* workspace,
                          size_t workspace_bytes, fl_stream_t stream, flashloop_ctx** out) {
   if (!out) return FL_ERR_INVALID_ARG;
   *out = nullptr;
   if (!valid_config(cfg) || !w) return FL_ERR_INVALID_ARG;
-  if (cfg->resid_bits != 16 &&
-      correct_smem(cfg->head_dim, cfg->n_heads / cfg->n_kv_heads, cfg->c_cols) > static_cast<size_t>(kMaxDynSmem))
-    return FL_ERR_UNSUPPORTED;
+
   const void* wp[9] = {w->attn_norm, w->w_qkv, w->w_o, w->mlp_norm, w->w_gate, w->w_up, w->w_down, w->final_norm,
                        w->w_out};
   for (const void* p : wp)
@@ -560,12 +559,21 @@ fl_status flashloop_init(const flashloop_config* cfg, const flashloop_weights* w
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   auto fail = [&](fl_status st) {
     if (st == FL_ERR_CUDA && ctx->last_err.empty()) ctx->last_err = cudaGetErrorString(cudaGetLastError());
+    g_last_error = ctx->last_err;
     delete ctx;
     return st;
   };
-  gemm_init_attrs();
-  kernels_init_attrs();
-  if (cudaGetLastError() != cudaSuccess) return fail(FL_ERR_CUDA);
+  {
+    cudaError_t e = gemm_init_attrs();
+    if (e == cudaSuccess) e = kernels_init_attrs();
+    if (e != cudaSuccess) {
+      ctx->last_err = cudaGetErrorString(e);
+      return fail(FL_ERR_CUDA);
+    }
+  }
+  if (ctx->lazy && correct_smem(cfg->head_dim, cfg->n_heads / cfg->n_kv_heads, cfg->c_cols) >
+                       correct_smem_limit(cfg->head_dim))
+    return fail(FL_ERR_UNSUPPORTED);
   if (!build_tmaps(ctx)) return fail(FL_ERR_CUDA);
   if (cudaMemsetAsync(ctx->ws, 0, need, s) != cudaSuccess) return fail(FL_ERR_CUDA);
   // RoPE table: angle = pos * theta^(-2i/hd), computed in double, stored fp32
@@ -875,12 +883,16 @@ fl_status flashloop_read_trace(flashloop_ctx* ctx, int32_t* sel, float* keys, in
 }
 
 // ---------------------------------------------------------------- unit entry points
+static fl_status record(cudaError_t e) {
+  if (e == cudaSuccess) return FL_OK;
+  g_last_error = cudaGetErrorString(e);
+  return FL_ERR_CUDA;
+}
+
 fl_status fl_test_topk(const float* keys, int n_seg, int n, int k, int32_t* idx, fl_stream_t stream) {
   if (!keys || !idx || n_seg < 0 || n < 0 || k < 0) return FL_ERR_INVALID_ARG;
   if (n_seg == 0 || n == 0 || k == 0) return FL_OK;
-  fl::kernels_init_attrs();
-  return launch_topk(keys, n_seg, n, k, idx, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess ? FL_OK
-                                                                                                   : FL_ERR_CUDA;
+  return record(launch_topk(keys, n_seg, n, k, idx, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 fl_status fl_test_quantize(const float* r, int rows, int width, int g, int bits, uint8_t* codes, uint16_t* scales,
@@ -892,8 +904,7 @@ fl_status fl_test_quantize(const float* r, int rows, int width, int g, int bits,
   if (width % 128 != 0 && width != 64) return FL_ERR_INVALID_ARG;
   if (width == 64 && g > 64) return FL_ERR_INVALID_ARG;
   if (rows == 0) return FL_OK;
-  return launch_quantize_rows(r, rows, width, g, bits, codes, scales, reinterpret_cast<cudaStream_t>(stream)) ==
-                 cudaSuccess ? FL_OK : FL_ERR_CUDA;
+  return record(launch_quantize_rows(r, rows, width, g, bits, codes, scales, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t fl_test_gemm_scratch_bytes(int m, int n, int k, int swap_ab) {
@@ -909,7 +920,10 @@ fl_status fl_test_gemm(const uint16_t* A, const uint16_t* B, float* D, int m, in
   if (!aligned16(A) || !aligned16(B) || !aligned16(D)) return FL_ERR_INVALID_ARG;
   if (swap_ab && m > 64) return FL_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  fl::gemm_init_attrs();
+  {
+    const cudaError_t e = gemm_init_attrs();
+    if (e != cudaSuccess) return record(e);
+  }
   GemmLaunch g{};
   GemmArgs& a = g.args;
   CUtensorMap ta, tb;
@@ -933,7 +947,8 @@ fl_status fl_test_gemm(const uint16_t* A, const uint16_t* B, float* D, int m, in
       a.partial = static_cast<float*>(scratch);
       a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(scratch) +
                                           ((gemm_partial_floats(bn, 0, tiles, splits) * 4 + 255) & ~size_t(255)));
-      if (cudaMemsetAsync(a.counters, 0, static_cast<size_t>(tiles) * 4, s) != cudaSuccess) return FL_ERR_CUDA;
+      const cudaError_t e = cudaMemsetAsync(a.counters, 0, static_cast<size_t>(tiles) * 4, s);
+      if (e != cudaSuccess) return record(e);
     }
     g.grid = dim3(tiles, 1, splits);
   } else {
@@ -942,7 +957,7 @@ fl_status fl_test_gemm(const uint16_t* A, const uint16_t* B, float* D, int m, in
     a.swap = 0; a.splits = 1;
     g.grid = dim3(ceil_div(m, 128), ceil_div(n, 128), 1);
   }
-  return launch_gemm(g, s) == cudaSuccess ? FL_OK : FL_ERR_CUDA;
+  return record(launch_gemm(g, s));
 }
 
 }  // extern "C"

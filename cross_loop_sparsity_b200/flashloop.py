@@ -91,10 +91,8 @@ def lib() -> ctypes.CDLL:
 
 def _check(st: int, what: str, ctx=None):
     if st != FL_OK:
-        detail = ""
-        if ctx:
-            e = lib().flashloop_last_cuda_error(ctx)
-            detail = e.decode() if e else ""
+        e = lib().flashloop_last_cuda_error(ctx)
+        detail = e.decode() if e else ""
         raise FlashLoopError(st, what, detail)
 
 
