@@ -1,0 +1,126 @@
+"""Shared drivers for the end-to-end GPU parity tests.
+
+Each driver draws one seeded workload from ``synth``, runs the CPU oracle on
+it, runs the CUDA library on the same arrays through the C ABI, and returns
+both.  In "forced" mode the library is handed the oracle's own token and
+column selections (the oracle's outputs become the library's inputs, never
+the reverse), so the comparison is of arithmetic rather than of near-tie
+choices; the library still computes every key itself.
+"""
+import numpy as np
+
+from cross_loop_sparsity_b200 import synth
+
+TOL = 2e-2   # max |gpu - oracle| <= TOL * RMS(oracle), for hidden states and logits
+
+
+def rel_err(got, want):
+    want = np.asarray(want, np.float64)
+    rms = float(np.sqrt(np.mean(want ** 2)))
+    return float(np.max(np.abs(np.asarray(got, np.float64) - want))) / rms
+
+
+def top_valid(keys, k, chosen):
+    """True when `chosen` (ascending) is a valid top-k of fp32 `keys` under
+    (bit pattern desc, index asc) -- checked with a plain sort, not the oracle."""
+    keys = np.ascontiguousarray(keys, np.float32)
+    bits = keys.view(np.uint32).astype(np.int64)
+    order = np.lexsort((np.arange(len(keys)), -bits))
+    return np.array_equal(np.sort(order[:k]).astype(np.int32), np.asarray(chosen, np.int32))
+
+
+def forced_arrays(cfg, trace, n_tiles):
+    sel = np.stack([trace["sel"][l] for l in range(2, cfg.n_loops + 1)])
+    cols = np.zeros((cfg.n_layers, n_tiles, cfg.n_kv_heads, cfg.c_cols), np.int32)
+    ncols = np.zeros((cfg.n_layers, n_tiles, cfg.n_kv_heads), np.int32)
+    for key, C in trace["cols"].items():
+        j, t, g = key
+        cols[j, t, g, :len(C)] = C
+        ncols[j, t, g] = len(C)
+    return sel, cols, ncols
+
+
+def run_prefill(cfg, B, T, forced=True, dense=False):
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    from oracle import flashloop_oracle as orc
+    if dense:
+        cfg = cfg.with_(resid_bits=16)
+    w = synth.make_weights(cfg)
+    h0 = synth.make_h0(cfg, w["rng"], B * T)
+    W = orc.prepare_weights(w)
+    ref = orc.prefill(cfg, W, orc.KVCache(cfg, B, T), h0, B, T)
+    eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=T, max_tokens=B * T)
+    n_tiles = B * ((T + cfg.q_tile - 1) // cfg.q_tile)
+    if forced and not dense and cfg.n_loops > 1:
+        eng.force_selection(*forced_arrays(cfg, ref.trace, n_tiles), n_tiles=n_tiles)
+    h_out = torch.empty((B * T, cfg.d_model), dtype=torch.float32, device="cuda")
+    logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    eng.prefill(torch.from_numpy(h0).cuda(), B, T, h_out, logits)
+    torch.cuda.synchronize()
+    out = {"h": h_out.cpu().numpy(), "logits": logits.cpu().numpy(), "status": eng.sync_status(),
+           "n_tiles": n_tiles}
+    if not dense:
+        n_sel = orc.n_select(cfg.rho, B * T)
+        out["sel"], out["keys"], out["cols"], out["ncols"] = eng.read_trace(B * T, n_sel, n_tiles)
+    return cfg, ref, eng, out
+
+
+def load_context(eng, cfg, ctx, dense=False):
+    """Import a synthetic context into the library's cache (device buffers)."""
+    import torch
+    lens = ctx["lens"]
+    for j in range(cfg.n_layers):
+        for b, n in enumerate(lens):
+            n = int(n)
+            if n == 0:
+                continue
+            if dense:
+                kk = torch.from_numpy(np.ascontiguousarray(ctx["kv_k"][j, :, b, :, :n]).view(np.int16)).cuda()
+                vv = torch.from_numpy(np.ascontiguousarray(ctx["kv_v"][j, :, b, :, :n]).view(np.int16)).cuda()
+                eng.import_dense(j, b, kk, vv)
+                continue
+            arr = {}
+            for nm in ("k", "v"):
+                arr["base_" + nm] = torch.from_numpy(
+                    np.ascontiguousarray(ctx["base_" + nm][j, b, :, :n]).view(np.int16)).cuda()
+                arr["codes_" + nm] = torch.from_numpy(np.ascontiguousarray(ctx["codes_" + nm][j, :, b, :, :n])).cuda()
+                arr["scales_" + nm] = torch.from_numpy(
+                    np.ascontiguousarray(ctx["scales_" + nm][j, :, b, :, :n]).view(np.int16)).cuda()
+            eng.import_lazy(j, b, arr["base_k"], arr["base_v"], arr["codes_k"], arr["codes_v"], arr["scales_k"],
+                            arr["scales_v"])
+    torch.cuda.synchronize()
+    eng.reset(list(int(x) for x in lens))
+
+
+def run_decode(cfg, lens, forced=True, dense=False, steps=1, extra_ctx=0):
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    from oracle import flashloop_oracle as orc
+    if dense:
+        cfg = cfg.with_(resid_bits=16)
+    B = len(lens)
+    w = synth.make_weights(cfg)
+    rng = w["rng"]
+    W = orc.prepare_weights(w)
+    tmax = int(max(lens)) + steps + extra_ctx
+    ctx = synth.make_dense_context(cfg, rng, lens) if dense else synth.make_context(cfg, rng, lens)
+    cache = orc.KVCache.from_dense_context(cfg, ctx, tmax) if dense else orc.KVCache.from_context(cfg, ctx, tmax)
+    eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=tmax, max_tokens=0)
+    load_context(eng, cfg, ctx, dense)
+    results = []
+    for _ in range(steps):
+        h0 = synth.make_h0(cfg, rng, B)
+        ref = orc.decode_step(cfg, W, cache, h0)
+        if forced and not dense and cfg.n_loops > 1:
+            eng.force_selection(*forced_arrays(cfg, ref.trace, B), n_tiles=B)
+        h_out = torch.empty((B, cfg.d_model), dtype=torch.float32, device="cuda")
+        logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+        eng.decode_step(torch.from_numpy(h0).cuda(), B, h_out, logits)
+        torch.cuda.synchronize()
+        out = {"h": h_out.cpu().numpy(), "logits": logits.cpu().numpy(), "status": eng.sync_status()}
+        if not dense:
+            n_sel = orc.n_select(cfg.rho, B)
+            out["sel"], out["keys"], out["cols"], out["ncols"] = eng.read_trace(B, n_sel, B)
+        results.append((ref, out))
+    return cfg, cache, eng, results

@@ -1,0 +1,142 @@
+"""End-to-end GPU parity through the C ABI against the CPU oracle.
+
+Hidden states and logits must agree within 2e-2 x RMS of the oracle's (bf16
+operands against an fp64 oracle).  Forced runs hand the library the oracle's
+selections; free runs check that the library's own selections are a valid
+top-k of the library's own keys.
+"""
+import numpy as np
+import pytest
+
+import e2e_common as E
+from cross_loop_sparsity_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from cross_loop_sparsity_b200 import build
+    build.build()
+
+
+def _check_outputs(ref, out, tol=E.TOL):
+    assert out["status"] == 0
+    eh, el = E.rel_err(out["h"], ref.h), E.rel_err(out["logits"], ref.logits)
+    assert eh <= tol, eh
+    assert el <= tol, el
+
+
+def _check_keys(cfg, ref, out, N):
+    # the library's change keys track the oracle's (they come from hidden states within tolerance)
+    for l in range(2, cfg.n_loops + 1):
+        want = ref.trace["keys"][l].astype(np.float64)
+        got = out["keys"][l - 2].astype(np.float64)
+        scale = max(float(np.max(want)), 1e-30)
+        assert np.max(np.abs(got - want)) <= 5e-2 * scale, l
+
+
+# ---------------------------------------------------------------- prefill
+def test_prefill_c1_forced():
+    cfg = synth.config("c1")
+    cfg, ref, eng, out = E.run_prefill(cfg, 1, cfg.seq_len)
+    _check_outputs(ref, out)
+    _check_keys(cfg, ref, out, cfg.seq_len)
+    for l in range(2, cfg.n_loops + 1):
+        assert np.array_equal(out["sel"][l - 2], ref.trace["sel"][l])
+
+
+def test_prefill_two_sequences_ragged_tiles_forced():
+    cfg = synth.config("c1").with_(seq_len=200, seed=5, n_loops=3)
+    cfg, ref, eng, out = E.run_prefill(cfg, 2, 200)
+    _check_outputs(ref, out)
+    assert out["n_tiles"] == 4
+    # every tile that was recomputed got a column set of min(c, eligible) columns
+    for (j, t, g), C in ref.trace["cols"].items():
+        assert out["ncols"][j, t, g] == len(C)
+        assert np.array_equal(out["cols"][j, t, g, :len(C)], C)
+
+
+def test_prefill_free_running_selection_is_valid():
+    cfg = synth.config("c1").with_(seed=11)
+    cfg, ref, eng, out = E.run_prefill(cfg, 1, cfg.seq_len, forced=False)
+    assert out["status"] == 0
+    from oracle import flashloop_oracle as orc
+    n_sel = orc.n_select(cfg.rho, cfg.seq_len)
+    agree = True
+    for l in range(2, cfg.n_loops + 1):
+        assert E.top_valid(out["keys"][l - 2], n_sel, out["sel"][l - 2]), l
+        agree &= np.array_equal(out["sel"][l - 2], ref.trace["sel"][l])
+    if agree and all(np.array_equal(out["cols"][j, t, g, :len(C)], C) for (j, t, g), C in ref.trace["cols"].items()):
+        _check_outputs(ref, out)
+
+
+def test_prefill_dense_baseline():
+    cfg = synth.config("c1").with_(seq_len=160, n_loops=3, seed=3)
+    cfg, ref, eng, out = E.run_prefill(cfg, 1, 160, dense=True)
+    _check_outputs(ref, out)
+
+
+def test_prefill_single_loop_is_a_plain_block():
+    cfg = synth.config("c1").with_(n_loops=1, seq_len=130)
+    cfg, ref, eng, out = E.run_prefill(cfg, 1, 130)
+    _check_outputs(ref, out)
+
+
+# ---------------------------------------------------------------- decode
+def test_decode_ragged_lengths_forced():
+    cfg = synth.config("c1").with_(mode="decode", batch=3, rho=0.5, c_cols=24, seed=7, seq_len=0)
+    cfg, cache, eng, results = E.run_decode(cfg, [300, 77, 1], steps=2)
+    for ref, out in results:
+        _check_outputs(ref, out)
+
+
+def test_decode_c2_full_size_forced():
+    cfg = synth.config("c2")
+    cfg, cache, eng, results = E.run_decode(cfg, [cfg.ctx_len] * cfg.batch)
+    for ref, out in results:
+        _check_outputs(ref, out)
+        _check_keys(cfg, ref, out, cfg.batch)
+
+
+def test_decode_c2_dense_baseline():
+    cfg = synth.config("c2").with_(ctx_len=1024)
+    cfg, cache, eng, results = E.run_decode(cfg, [1024] * cfg.batch, dense=True)
+    for ref, out in results:
+        _check_outputs(ref, out)
+
+
+@pytest.mark.parametrize("name", ["c5", "c5_int2"])
+def test_decode_c5_full_size_forced(name):
+    cfg = synth.config(name)
+    cfg, cache, eng, results = E.run_decode(cfg, [cfg.ctx_len])
+    for ref, out in results:
+        _check_outputs(ref, out)
+
+
+def test_decode_graph_replay_matches_direct_launches():
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    cfg = synth.config("c1").with_(mode="decode", batch=4, rho=0.25, c_cols=16, seed=13, seq_len=0)
+    lens = [64, 40, 9, 100]
+    outs = []
+    for use_graph in (1, 0):
+        w = synth.make_weights(cfg)
+        rng = w["rng"]
+        ctx = synth.make_context(cfg, rng, lens)
+        eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=4, max_ctx=128)
+        E.load_context(eng, cfg, ctx)
+        eng.set_option(fl.FL_OPT_USE_GRAPH, use_graph)
+        s = torch.cuda.Stream()
+        res = []
+        for _ in range(3):
+            h0 = torch.from_numpy(synth.make_h0(cfg, rng, 4)).cuda()
+            lg = torch.empty((4, cfg.vocab), dtype=torch.float32, device="cuda")
+            torch.cuda.synchronize()
+            eng.decode_step(h0, 4, None, lg, stream=s)
+            s.synchronize()
+            res.append(lg.cpu().numpy())
+        assert eng.sync_status(s) == 0
+        outs.append(res)
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)
