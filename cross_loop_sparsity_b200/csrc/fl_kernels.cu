@@ -600,6 +600,11 @@ __global__ void k_set_lens(int B, int* seq_len, int add, int value) {
   if (b < B) seq_len[b] = add ? seq_len[b] + 1 : value;
 }
 
+__global__ void k_reset_lens(const LensArg a, int* seq_len) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < a.n) seq_len[b] = a.v[b];
+}
+
 // slot of each token in the selection (or -1), and the snapshot of selected rows
 __global__ void k_after_select(const int32_t* __restrict__ idx, int n_sel, int N, int d, int* sel_slot,
                                const float* __restrict__ h, float* __restrict__ h_snap, int slot_blocks) {
@@ -1016,6 +1021,10 @@ cudaError_t launch_setup_call(int N, int decode, int T, int tiles_per_seq, int q
 }
 cudaError_t launch_set_lens(int B, int* seq_len, int add, int value, cudaStream_t s) {
   k_set_lens<<<(B + 127) / 128, 128, 0, s>>>(B, seq_len, add, value);
+  return cudaGetLastError();
+}
+cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s) {
+  k_reset_lens<<<1, kLensByValue, 0, s>>>(a, seq_len);
   return cudaGetLastError();
 }
 cudaError_t launch_after_select(const int32_t* idx, int n_sel, int N, int d, int* sel_slot, const float* h,

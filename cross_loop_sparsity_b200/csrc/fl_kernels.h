@@ -112,6 +112,13 @@ size_t correct_smem(int hd, int grp, int c);
 size_t correct_smem_limit(int hd);   // the most the correction kernel may opt in to on this device
 cudaError_t kernels_init_attrs();
 
+constexpr int kLensByValue = 256;
+struct LensArg {
+  int n;
+  int v[kLensByValue];
+};
+cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s);
+
 cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* idx, const int* forced_on,
                                  const int32_t* forced, cudaStream_t s);
 cudaError_t launch_rmsnorm_rows(const float* h, const int* idx, int n, int n_pad, int d, const float* gain, float eps,

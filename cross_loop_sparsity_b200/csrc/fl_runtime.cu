@@ -69,6 +69,11 @@ struct flashloop_ctx {
   std::vector<cudaGraphExec_t> graph_exec;
   std::vector<int> eager_seen;
   int use_graph = 1;
+  int prof = 0;                       // FL_OPT_PROFILE
+  std::vector<cudaEvent_t> ev;        // start/end pairs of the last profiled call
+  std::vector<int> ev_kind;
+  int ev_used = 0;
+  int launches = 0;                   // kernels enqueued by the last call
   std::string last_err;
   int last_N = 0, last_nsel = 0, last_decode = 0, last_tiles = 0;
 };
@@ -364,6 +369,54 @@ __global__ void k_fill_last_rows(int B, int T, int32_t* rows) {
   if (b < B) rows[b] = b * T + T - 1;
 }
 
+// Profiling brackets: an event pair around each kernel.  While the stream is
+// being captured the events become event-record nodes of the graph.
+cudaError_t record_event(cudaEvent_t e, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  const cudaError_t q = cudaStreamIsCapturing(s, &cs);
+  if (q != cudaSuccess) return q;
+  return cs == cudaStreamCaptureStatusActive ? cudaEventRecordWithFlags(e, s, cudaEventRecordExternal)
+                                             : cudaEventRecord(e, s);
+}
+cudaError_t prof_begin(flashloop_ctx* ctx, int kind, cudaStream_t s) {
+  if (!ctx->prof) return cudaSuccess;
+  const size_t need = static_cast<size_t>(ctx->ev_used + 1) * 2;
+  while (ctx->ev.size() < need) {
+    cudaEvent_t e = nullptr;
+    const cudaError_t r = cudaEventCreate(&e);
+    if (r != cudaSuccess) return r;
+    ctx->ev.push_back(e);
+  }
+  if (ctx->ev_kind.size() < static_cast<size_t>(ctx->ev_used + 1)) ctx->ev_kind.resize(ctx->ev_used + 1);
+  ctx->ev_kind[ctx->ev_used] = kind;
+  return record_event(ctx->ev[2 * ctx->ev_used], s);
+}
+cudaError_t prof_end(flashloop_ctx* ctx, cudaStream_t s) {
+  if (!ctx->prof) return cudaSuccess;
+  const cudaError_t r = record_event(ctx->ev[2 * ctx->ev_used + 1], s);
+  ++ctx->ev_used;
+  return r;
+}
+
+// Launch one kernel (an expression returning cudaError_t) of a given kind.
+#define FL_LAUNCH(kind, expr)                  \
+  do {                                         \
+    FL_TRY(prof_begin(ctx, (kind), s));        \
+    FL_TRY(expr);                              \
+    FL_TRY(prof_end(ctx, s));                  \
+    ++ctx->launches;                           \
+  } while (0)
+
+// Launch one GEMM (an expression returning fl_status).
+#define FL_GEMM(expr)                                  \
+  do {                                                 \
+    FL_TRY(prof_begin(ctx, FL_KIND_GEMM, s));          \
+    fl_status st_g = (expr);                           \
+    if (st_g != FL_OK) return st_g;                    \
+    FL_TRY(prof_end(ctx, s));                          \
+    ++ctx->launches;                                   \
+  } while (0)
+
 #define FL_STEP(expr)                 \
   do {                                \
     fl_status st_ = (expr);           \
@@ -388,8 +441,10 @@ fl_status run_call(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s)
   const int col_span = decode ? c.max_ctx : T;   // columns a query tile can see
   const int max_chunks = ceil_div(col_span, 64);
 
-  FL_TRY(launch_setup_call(N, decode, T, tiles_per_seq, q_tile, ctx->seq_len, ctx->seq, ctx->pos, ctx->tile,
-                           ctx->last, n_tiles, ctx->has_c, s));
+  ctx->launches = 0;
+  ctx->ev_used = 0;
+  FL_LAUNCH(FL_KIND_OTHER, launch_setup_call(N, decode, T, tiles_per_seq, q_tile, ctx->seq_len, ctx->seq, ctx->pos,
+                                             ctx->tile, ctx->last, n_tiles, ctx->has_c, s));
   FL_TRY(cudaMemcpyAsync(ctx->h, ctx->h_in, static_cast<size_t>(N) * d * 4, cudaMemcpyDeviceToDevice, s));
   for (int l = 1; l <= K; ++l) {
     const bool full = !lazy || l == 1;
@@ -399,10 +454,10 @@ fl_status run_call(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s)
       int32_t* sel = ctx->idx_sel + static_cast<size_t>(l - 2) * ctx->N_max;
       FL_TRY(cudaMemcpyAsync(ctx->keys_trace + static_cast<size_t>(l - 2) * ctx->N_max, ctx->key,
                              static_cast<size_t>(N) * 4, cudaMemcpyDeviceToDevice, s));
-      FL_TRY(launch_select_tokens(ctx->key, N, n_sel, sel, ctx->forced_on,
-                                  ctx->forced_sel + static_cast<size_t>(l - 2) * ctx->N_max, s));
-      FL_TRY(launch_after_select(sel, n_sel, N, d, ctx->sel_slot, ctx->h, ctx->h_snap, s));
-      FL_TRY(launch_plan_tiles(sel, n_sel, ctx->tile, ctx->has_c, ctx->plan, s));
+      FL_LAUNCH(FL_KIND_SELECT, launch_select_tokens(ctx->key, N, n_sel, sel, ctx->forced_on,
+                                                     ctx->forced_sel + static_cast<size_t>(l - 2) * ctx->N_max, s));
+      FL_LAUNCH(FL_KIND_SELECT, launch_after_select(sel, n_sel, N, d, ctx->sel_slot, ctx->h, ctx->h_snap, s));
+      FL_LAUNCH(FL_KIND_SELECT, launch_plan_tiles(sel, n_sel, ctx->tile, ctx->has_c, ctx->plan, s));
       idx = sel;
       n = n_sel;
     }
@@ -411,14 +466,14 @@ fl_status run_call(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s)
       float* l_st = lazy ? ctx->lse_state + j * st_l : nullptr;
       float* ql = lazy ? ctx->q_last + j * st_o : nullptr;
       // attention branch
-      FL_TRY(launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d, ctx->w.attn_norm + static_cast<size_t>(j) * d,
-                                 c.rms_eps, ctx->x, s));
-      FL_STEP(gemm(ctx, kOpQKV, j, n, idx, s));
+      FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d,
+                                                  ctx->w.attn_norm + static_cast<size_t>(j) * d, c.rms_eps, ctx->x, s));
+      FL_GEMM(gemm(ctx, kOpQKV, j, n, idx, s));
       QkvPostArgs qa{};
       qa.qkv = ctx->qkv; qa.ldq = ctx->qkv_rows; qa.idx = idx; qa.n = n; qa.seq = ctx->seq; qa.pos = ctx->pos;
       qa.H = H; qa.Hkv = Hkv; qa.hd = hd; qa.rope_cos = ctx->rope_cos; qa.rope_sin = ctx->rope_sin;
       qa.cv = ctx->cv; qa.j = j; qa.loop = l; qa.lazy = lazy ? 1 : 0; qa.q_cur = ctx->q_cur; qa.q_last = ql;
-      FL_TRY(launch_qkv_post(qa, s));
+      FL_LAUNCH(FL_KIND_KV, launch_qkv_post(qa, s));
       if (full) {
         if (decode) {
           AttnDecArgs aa{};
@@ -427,54 +482,54 @@ fl_status run_call(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s)
           aa.split_len = ctx->dec_split_len; aa.n_splits = ctx->dec_splits;
           aa.part_o = ctx->part_o; aa.part_ml = ctx->part_ml; aa.counters = ctx->attn_counters;
           aa.o_state = o_st; aa.lse_state = l_st; aa.o_bf16 = ctx->obf;
-          FL_TRY(launch_attn_decode(aa, n, s));
+          FL_LAUNCH(FL_KIND_ATTN, launch_attn_decode(aa, n, s));
         } else {
           AttnPreArgs pa{};
           pa.q_cur = ctx->q_cur; pa.cv = ctx->cv; pa.j = j; pa.loop = l; pa.dense = lazy ? 0 : 1;
           pa.T = T; pa.H = H; pa.Hkv = Hkv; pa.hd = hd; pa.tau = tau;
           pa.o_state = o_st; pa.lse_state = l_st; pa.o_bf16 = ctx->obf;
-          FL_TRY(launch_attn_prefill(pa, B, s));
+          FL_LAUNCH(FL_KIND_ATTN, launch_attn_prefill(pa, B, s));
         }
       } else {
         DScoreArgs da{};
         da.plan = ctx->plan; da.idx = idx; da.seq = ctx->seq; da.pos = ctx->pos; da.q_cur = ctx->q_cur;
         da.q_last = ql; da.cv = ctx->cv; da.j = j; da.loop = l; da.H = H; da.Hkv = Hkv; da.hd = hd; da.tau = tau;
         da.col_keys = ctx->col_keys; da.max_cols = c.max_ctx;
-        FL_TRY(launch_dscore(da, max_need, max_chunks, s));
+        FL_LAUNCH(FL_KIND_DSCORE, launch_dscore(da, max_need, max_chunks, s));
         SelColsArgs sa{};
         sa.plan = ctx->plan; sa.idx = idx; sa.pos = ctx->pos; sa.col_keys = ctx->col_keys; sa.max_cols = c.max_ctx;
         sa.Hkv = Hkv; sa.c = c.c_cols; sa.j = j; sa.n_tiles = ctx->n_tiles_max; sa.cols = ctx->cols;
         sa.ncols = ctx->ncols; sa.forced_on = ctx->forced_on; sa.forced_cols = ctx->forced_cols;
         sa.forced_ncols = ctx->forced_ncols;
-        FL_TRY(launch_select_cols(sa, max_need, s));
+        FL_LAUNCH(FL_KIND_SELECT, launch_select_cols(sa, max_need, s));
         CorrectArgs ca{};
         ca.idx = idx; ca.seq = ctx->seq; ca.pos = ctx->pos; ca.tile = ctx->tile; ca.last = ctx->last;
         ca.q_cur = ctx->q_cur; ca.q_last = ql; ca.o_state = o_st; ca.lse_state = l_st; ca.o_bf16 = ctx->obf;
         ca.cols = ctx->cols; ca.ncols = ctx->ncols; ca.cv = ctx->cv; ca.j = j; ca.loop = l; ca.H = H; ca.Hkv = Hkv;
         ca.hd = hd; ca.c = c.c_cols; ca.n_tiles = ctx->n_tiles_max; ca.tau = tau; ca.status = ctx->status;
-        FL_TRY(launch_correct(ca, n, s));
+        FL_LAUNCH(FL_KIND_CORRECT, launch_correct(ca, n, s));
       }
-      FL_STEP(gemm(ctx, kOpO, j, n, idx, s));
+      FL_GEMM(gemm(ctx, kOpO, j, n, idx, s));
       // MLP branch
-      FL_TRY(launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d, ctx->w.mlp_norm + static_cast<size_t>(j) * d, c.rms_eps,
-                                 ctx->x, s));
-      FL_STEP(gemm(ctx, kOpGU, j, n, idx, s));
-      FL_STEP(gemm(ctx, kOpDown, j, n, idx, s));
+      FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d,
+                                                  ctx->w.mlp_norm + static_cast<size_t>(j) * d, c.rms_eps, ctx->x, s));
+      FL_GEMM(gemm(ctx, kOpGU, j, n, idx, s));
+      FL_GEMM(gemm(ctx, kOpDown, j, n, idx, s));
     }
     if (lazy && l < K)
-      FL_TRY(launch_change_keys(ctx->h, l == 1 ? ctx->h_in : ctx->h_snap, ctx->sel_slot, N, d, l, ctx->key, ctx->last,
-                                ctx->tile, ctx->has_c, s));
+      FL_LAUNCH(FL_KIND_OTHER, launch_change_keys(ctx->h, l == 1 ? ctx->h_in : ctx->h_snap, ctx->sel_slot, N, d, l,
+                                                  ctx->key, ctx->last, ctx->tile, ctx->has_c, s));
   }
   // final norm + LM head on the output rows
   const int32_t* rows = ctx->idx_all;
   if (!decode) {
-    k_fill_last_rows<<<ceil_div(B, 128), 128, 0, s>>>(B, T, ctx->idx_last);
-    FL_TRY(cudaGetLastError());
+    FL_LAUNCH(FL_KIND_OTHER, (k_fill_last_rows<<<ceil_div(B, 128), 128, 0, s>>>(B, T, ctx->idx_last),
+                              cudaGetLastError()));
     rows = ctx->idx_last;
   }
-  FL_TRY(launch_rmsnorm_rows(ctx->h, rows, B, pad(B), d, ctx->w.final_norm, c.rms_eps, ctx->x, s));
-  FL_STEP(gemm(ctx, kOpOut, 0, B, rows, s));
-  FL_TRY(launch_set_lens(B, ctx->seq_len, decode ? 1 : 0, T, s));
+  FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, rows, B, pad(B), d, ctx->w.final_norm, c.rms_eps, ctx->x, s));
+  FL_GEMM(gemm(ctx, kOpOut, 0, B, rows, s));
+  FL_LAUNCH(FL_KIND_OTHER, launch_set_lens(B, ctx->seq_len, decode ? 1 : 0, T, s));
   return FL_OK;
 }
 
@@ -602,6 +657,8 @@ void flashloop_destroy(flashloop_ctx* ctx) {
   if (!ctx) return;
   for (cudaGraphExec_t e : ctx->graph_exec)
     if (e) cudaGraphExecDestroy(e);
+  for (cudaEvent_t e : ctx->ev)
+    if (e) cudaEventDestroy(e);
   delete ctx;
 }
 
@@ -609,6 +666,10 @@ fl_status flashloop_set_option(flashloop_ctx* ctx, fl_option opt, int value) {
   if (!ctx) return FL_ERR_INVALID_ARG;
   if (opt == FL_OPT_USE_GRAPH) {
     ctx->use_graph = value ? 1 : 0;
+    return FL_OK;
+  }
+  if (opt == FL_OPT_PROFILE) {
+    ctx->prof = value ? 1 : 0;
     return FL_OK;
   }
   return FL_ERR_INVALID_ARG;
@@ -647,10 +708,11 @@ fl_status flashloop_decode_step(flashloop_ctx* ctx, const float* h0, int B, floa
   FL_TRY(cudaMemcpyAsync(ctx->h_in, h0, static_cast<size_t>(B) * c.d_model * 4, cudaMemcpyDefault, s));
   // A decode step's launch sequence depends on B only; after one direct run it
   // is captured once into a CUDA graph and replayed (not on the legacy stream).
+  const int gkey = B * 2 + (ctx->prof ? 1 : 0);
   size_t gi = 0;
-  while (gi < ctx->graph_b.size() && ctx->graph_b[gi] != B) ++gi;
+  while (gi < ctx->graph_b.size() && ctx->graph_b[gi] != gkey) ++gi;
   bool seen = false;
-  for (int v : ctx->eager_seen) seen |= (v == B);
+  for (int v : ctx->eager_seen) seen |= (v == gkey);
   if (ctx->use_graph && s != nullptr && seen) {
     if (gi == ctx->graph_b.size()) {
       cudaGraph_t graph = nullptr;
@@ -666,13 +728,13 @@ fl_status flashloop_decode_step(flashloop_ctx* ctx, const float* h0, int B, floa
       e = cudaGraphInstantiate(&exec, graph, 0);
       cudaGraphDestroy(graph);
       FL_TRY(e);
-      ctx->graph_b.push_back(B);
+      ctx->graph_b.push_back(gkey);
       ctx->graph_exec.push_back(exec);
     }
     FL_TRY(cudaGraphLaunch(ctx->graph_exec[gi], s));
   } else {
     FL_STEP(run_call(ctx, 1, B, 0, s));
-    if (!seen) ctx->eager_seen.push_back(B);
+    if (!seen) ctx->eager_seen.push_back(gkey);
   }
   if (h_out) FL_TRY(cudaMemcpyAsync(h_out, ctx->h, static_cast<size_t>(B) * c.d_model * 4, cudaMemcpyDefault, s));
   if (logits)
@@ -716,11 +778,37 @@ fl_status flashloop_reset(flashloop_ctx* ctx, const int* seq_len, fl_stream_t st
       v[b] = seq_len[b];
     }
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  FL_TRY(cudaMemcpyAsync(ctx->seq_len, v.data(), B * 4, cudaMemcpyHostToDevice, s));
-  FL_TRY(cudaStreamSynchronize(s));
+  if (B <= kLensByValue) {
+    LensArg a{};
+    a.n = B;
+    for (int b = 0; b < B; ++b) a.v[b] = v[b];
+    FL_TRY(launch_reset_lens(a, ctx->seq_len, s));
+  } else {
+    FL_TRY(cudaMemcpyAsync(ctx->seq_len, v.data(), B * 4, cudaMemcpyHostToDevice, s));
+    FL_TRY(cudaStreamSynchronize(s));
+  }
   ctx->lens = v;
   return FL_OK;
 }
+
+fl_status flashloop_profile(flashloop_ctx* ctx, fl_stream_t stream, float* ms, int* launches) {
+  if (!ctx || !ms || !launches) return FL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FL_TRY(cudaStreamSynchronize(s));
+  for (int k = 0; k < FL_NUM_KINDS; ++k) {
+    ms[k] = 0.f;
+    launches[k] = 0;
+  }
+  for (int i = 0; i < ctx->ev_used; ++i) {
+    float t = 0.f;
+    FL_TRY(cudaEventElapsedTime(&t, ctx->ev[2 * i], ctx->ev[2 * i + 1]));
+    ms[ctx->ev_kind[i]] += t;
+    launches[ctx->ev_kind[i]] += 1;
+  }
+  return FL_OK;
+}
+
+int flashloop_kernels_per_call(const flashloop_ctx* ctx) { return ctx ? ctx->launches : 0; }
 
 fl_status flashloop_sync_status(flashloop_ctx* ctx, fl_stream_t stream) {
   if (!ctx) return FL_ERR_INVALID_ARG;

@@ -17,6 +17,8 @@ LIB_PATH = os.path.join(_HERE, "libflashloop.so")
 
 FL_OK = 0
 FL_OPT_USE_GRAPH = 1
+FL_OPT_PROFILE = 2
+KINDS = ["gemm", "attn", "dscore", "correct", "kv", "select", "norm", "other"]
 STATUS = {0: "ok", 1: "invalid argument", 2: "capacity exceeded", 3: "workspace", 4: "cuda error",
           5: "timeout", 6: "nonfinite", 7: "unsupported"}
 
@@ -65,6 +67,8 @@ _SIG = {
     "flashloop_force_selection": (_I, [_P, _P, _I, _I, _P, _P, _I]),
     "flashloop_read_trace": (_I, [_P, _P, _P, _P, _P, _P]),
     "flashloop_set_option": (_I, [_P, _I, _I]),
+    "flashloop_profile": (_I, [_P, _P, _P, _P]),
+    "flashloop_kernels_per_call": (_I, [_P]),
     "fl_test_topk": (_I, [_P, _I, _I, _I, _P, _P]),
     "fl_test_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "fl_test_gemm_scratch_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
@@ -205,6 +209,16 @@ class FlashLoop:
     def sync_status(self, stream=None) -> int:
         return int(lib().flashloop_sync_status(self.ctx, _stream_ptr(stream)))
 
+    def profile(self, stream=None):
+        """{kind: (ms, launches)} of the last call made with FL_OPT_PROFILE on."""
+        ms = (ctypes.c_float * len(KINDS))()
+        n = (ctypes.c_int * len(KINDS))()
+        _check(lib().flashloop_profile(self.ctx, _stream_ptr(stream), ms, n), "flashloop_profile", self.ctx)
+        return {k: (float(ms[i]), int(n[i])) for i, k in enumerate(KINDS)}
+
+    def kernels_per_call(self) -> int:
+        return int(lib().flashloop_kernels_per_call(self.ctx))
+
     def set_option(self, opt: int, value: int):
         _check(lib().flashloop_set_option(self.ctx, opt, value), "flashloop_set_option")
 
@@ -219,6 +233,36 @@ class FlashLoop:
         n = kv_k.shape[2]
         _check(lib().flashloop_import_dense(self.ctx, layer, seq, n, _ptr(kv_k), _ptr(kv_v), _stream_ptr(stream)),
                "flashloop_import_dense", self.ctx)
+
+    def load_context(self, ctx: dict, dense: bool = False):
+        """Import a cache given as host arrays (the layout ``synth.make_context`` /
+        ``make_dense_context`` returns) slice by slice, then set the lengths."""
+        import torch
+        cfg = self.cfg
+        lens = ctx["lens"]
+        for j in range(cfg.n_layers):
+            for b, n in enumerate(lens):
+                n = int(n)
+                if n == 0:
+                    continue
+                if dense:
+                    kk = torch.from_numpy(np.ascontiguousarray(ctx["kv_k"][j, :, b, :, :n]).view(np.int16)).cuda()
+                    vv = torch.from_numpy(np.ascontiguousarray(ctx["kv_v"][j, :, b, :, :n]).view(np.int16)).cuda()
+                    self.import_dense(j, b, kk, vv)
+                    continue
+                a = {}
+                for nm in ("k", "v"):
+                    a["base_" + nm] = torch.from_numpy(
+                        np.ascontiguousarray(ctx["base_" + nm][j, b, :, :n]).view(np.int16)).cuda()
+                    a["codes_" + nm] = torch.from_numpy(np.ascontiguousarray(ctx["codes_" + nm][j, :, b, :, :n])).cuda()
+                    a["scales_" + nm] = torch.from_numpy(
+                        np.ascontiguousarray(ctx["scales_" + nm][j, :, b, :, :n]).view(np.int16)).cuda()
+                self.import_lazy(j, b, a["base_k"], a["base_v"], a["codes_k"], a["codes_v"], a["scales_k"],
+                                 a["scales_v"])
+                torch.cuda.synchronize()   # the import copies read the staged tensors
+        torch.cuda.synchronize()
+        self.reset([int(x) for x in lens])
+        torch.cuda.synchronize()
 
     def export_slice(self, layer, loop, seq, which, n, stream=None):
         """Returns (codes, scales) numpy arrays; loop 1 (or dense) returns (bf16 bits [Hkv][n][hd], None)."""

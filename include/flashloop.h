@@ -133,7 +133,8 @@ fl_status flashloop_kv_bytes_for(const flashloop_config* cfg, size_t* total, dou
 
 /* Set every sequence length (seq_len: [max_batch] host array, or NULL for all
  * zero).  Cache contents are kept; used to replay a decode step at a fixed
- * context.  Enqueued on `stream`. */
+ * context.  Enqueued on `stream` as one small kernel (max_batch <= 256),
+ * without waiting. */
 fl_status flashloop_reset(flashloop_ctx* ctx, const int* seq_len, fl_stream_t stream);
 
 /* Synchronise `stream` and report the first error a kernel recorded since
@@ -216,9 +217,32 @@ fl_status fl_test_gemm(const uint16_t* A, const uint16_t* B, float* D, int m, in
 
 /* Runtime options of a context. */
 typedef enum {
-  FL_OPT_USE_GRAPH = 1 /* 1 (default): capture decode steps into CUDA graphs; 0: launch directly */
+  FL_OPT_USE_GRAPH = 1, /* 1 (default): capture decode steps into CUDA graphs; 0: launch directly */
+  FL_OPT_PROFILE = 2    /* 1: bracket every kernel of a call with CUDA events (read with flashloop_profile) */
 } fl_option;
 fl_status flashloop_set_option(flashloop_ctx* ctx, fl_option opt, int value);
+
+/* Kernel kinds reported by flashloop_profile. */
+enum {
+  FL_KIND_GEMM = 0,      /* tcgen05 GEMMs (QKV, O, gate/up, down, LM head) */
+  FL_KIND_ATTN = 1,      /* dense attention (decode splits + merge, or prefill) */
+  FL_KIND_DSCORE = 2,    /* delta-score column keys */
+  FL_KIND_CORRECT = 3,   /* sparse-column correction */
+  FL_KIND_KV = 4,        /* RoPE + KV store / residual quantise */
+  FL_KIND_SELECT = 5,    /* token / column top-k, tile plan, snapshots */
+  FL_KIND_NORM = 6,      /* RMSNorm gathers */
+  FL_KIND_OTHER = 7,     /* change keys, bookkeeping */
+  FL_NUM_KINDS = 8
+};
+
+/* Per-kind kernel time of the last prefill / decode call made with
+ * FL_OPT_PROFILE on: synchronises `stream`, then writes ms[kind] (summed
+ * device time of that kind's kernels, from CUDA events recorded around each
+ * launch) and launches[kind].  Arrays have FL_NUM_KINDS entries. */
+fl_status flashloop_profile(flashloop_ctx* ctx, fl_stream_t stream, float* ms, int* launches);
+
+/* Number of kernels the last prefill / decode call enqueued (all kinds). */
+int flashloop_kernels_per_call(const flashloop_ctx* ctx);
 
 #ifdef __cplusplus
 }

@@ -68,29 +68,7 @@ def run_prefill(cfg, B, T, forced=True, dense=False):
 
 def load_context(eng, cfg, ctx, dense=False):
     """Import a synthetic context into the library's cache (device buffers)."""
-    import torch
-    lens = ctx["lens"]
-    for j in range(cfg.n_layers):
-        for b, n in enumerate(lens):
-            n = int(n)
-            if n == 0:
-                continue
-            if dense:
-                kk = torch.from_numpy(np.ascontiguousarray(ctx["kv_k"][j, :, b, :, :n]).view(np.int16)).cuda()
-                vv = torch.from_numpy(np.ascontiguousarray(ctx["kv_v"][j, :, b, :, :n]).view(np.int16)).cuda()
-                eng.import_dense(j, b, kk, vv)
-                continue
-            arr = {}
-            for nm in ("k", "v"):
-                arr["base_" + nm] = torch.from_numpy(
-                    np.ascontiguousarray(ctx["base_" + nm][j, b, :, :n]).view(np.int16)).cuda()
-                arr["codes_" + nm] = torch.from_numpy(np.ascontiguousarray(ctx["codes_" + nm][j, :, b, :, :n])).cuda()
-                arr["scales_" + nm] = torch.from_numpy(
-                    np.ascontiguousarray(ctx["scales_" + nm][j, :, b, :, :n]).view(np.int16)).cuda()
-            eng.import_lazy(j, b, arr["base_k"], arr["base_v"], arr["codes_k"], arr["codes_v"], arr["scales_k"],
-                            arr["scales_v"])
-    torch.cuda.synchronize()
-    eng.reset(list(int(x) for x in lens))
+    eng.load_context(ctx, dense)
 
 
 def run_decode(cfg, lens, forced=True, dense=False, steps=1, extra_ctx=0):
