@@ -816,133 +816,147 @@ __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
 //   Z' = e^(lse-Mx) - sum_C e^(s_old-Mx) + sum_C e^(s_new-Mx)
 //   N' = e^(lse-Mx) O - sum_C e^(s_old-Mx) V_last + sum_C e^(s_new-Mx) V_l
 //   O = N'/Z', lse = Mx + ln Z', q_last = q_l
-// with s_new = tau q_l.K_l, s_old = tau q_last.K_last.  grid (n_sel*Hkv), 128 threads.
+// with s_new = tau q_l.K_l, s_old = tau q_last.K_last.  The column set is
+// split across CTAs (grid.y); each warp takes one column at a time and keeps a
+// running per-head maximum, so the sums above are accumulated in pieces that
+// are rescaled to the common maximum when merged.  The last CTA of a (query,
+// group) -- an atomic ticket, no waiting -- merges the pieces with the stored
+// (O, lse) term and writes the new state.
 // ============================================================================
-template <int HD, int EPL>
-__global__ void __launch_bounds__(128) k_correct(const CorrectArgs a) {
-  constexpr int CC = 32;
-  constexpr int GMAX = 8;
-  extern __shared__ __align__(16) uint8_t sm[];
-  float* An = reinterpret_cast<float*>(sm);       // [CC][HD+1] new rows (K then V)
-  float* Ao = An + CC * (HD + 1);                 // [CC][HD+1] old rows
-  float* Qn = Ao + CC * (HD + 1);                 // [GMAX][HD]
-  float* Qo = Qn + GMAX * HD;                     // [GMAX][HD]
-  const int grp = a.H / a.Hkv;
-  float* Sn = Qo + GMAX * HD;                     // [grp][c]
-  float* So = Sn + grp * a.c;                     // [grp][c]
-  __shared__ float mx[GMAX], zz[GMAX], el[GMAX];
-  __shared__ int ncs;
+template <int HD, int EPL, int GRP>
+__global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
+  constexpr int GMAX = 8, NW = 8;
+  __shared__ float sm_m[NW][GMAX], sm_z[NW][GMAX];
+  __shared__ float sm_acc[NW][GMAX][HD];
+  __shared__ int ncs, is_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int i = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
+  const int i = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv, sp = blockIdx.y;
+  constexpr int grp = GRP;
   const int tok = a.idx[i];
   const int b = a.seq[tok], P = a.pos[tok], tl = a.tile[tok];
   const int m_old = a.last[tok];
   const CacheView& cv = a.cv;
-  const int32_t* C = a.cols + ((static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g) * a.c;
-  const int ncol = a.ncols[(static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g];
+  const size_t cset = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
+  const int32_t* C = a.cols + cset * a.c;
   if (tid == 0) {
-    int n = 0;
-    while (n < ncol && C[n] <= P) ++n;   // C is ascending
-    ncs = n;
+    // C is ascending: the query's columns are its prefix with C[k] <= pos
+    int lo = 0, hi = a.ncols[cset];
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (C[mid] <= P) lo = mid + 1; else hi = mid;
+    }
+    ncs = lo;
   }
-  for (int e = tid; e < grp * HD; e += 128) {
-    const int hh = g * grp + e / HD, dd = e % HD;
-    Qn[e] = a.q_cur[(static_cast<size_t>(i) * a.H + hh) * HD + dd];
-    Qo[e] = a.q_last[(static_cast<size_t>(tok) * a.H + hh) * HD + dd];
+  // the group's query heads (new and last) in registers
+  float qn[GRP][EPL], qo[GRP][EPL];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    const size_t hq = static_cast<size_t>(g * grp + h);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      qn[h][e] = a.q_cur[(static_cast<size_t>(i) * a.H + hq) * HD + lane * EPL + e];
+      qo[h][e] = a.q_last[(static_cast<size_t>(tok) * a.H + hq) * HD + lane * EPL + e];
+    }
   }
   __syncthreads();
   const int nc = ncs;
-  // pass 1: scores over C
-  for (int c0 = 0; c0 < nc; c0 += CC) {
-    const int cn = min(CC, nc - c0);
-    for (int rr = warp; rr < cn; rr += 4) {
-      float lo[EPL], hi[EPL];
-      chain_lane2<EPL>(cv, a.j, 0, b, g, C[c0 + rr], m_old, a.loop, lane, lo, hi);
+  const int k0 = sp * a.cols_per_cta, k1 = min(nc, k0 + a.cols_per_cta);
+  float m[GRP], z[GRP], acc[GRP][EPL];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    m[h] = -INFINITY;
+    z[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
+  }
+  for (int k = k0 + warp; k < k1; k += NW) {
+    const int col = C[k];
+    float klo[EPL], khi[EPL], vlo[EPL], vhi[EPL];
+    chain_lane2<EPL>(cv, a.j, 0, b, g, col, m_old, a.loop, lane, klo, khi);
+    chain_lane2<EPL>(cv, a.j, 1, b, g, col, m_old, a.loop, lane, vlo, vhi);
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) {
+      float dn = 0.f, dl = 0.f;
 #pragma unroll
       for (int e = 0; e < EPL; ++e) {
-        Ao[rr * (HD + 1) + lane * EPL + e] = lo[e];
-        An[rr * (HD + 1) + lane * EPL + e] = hi[e];
+        dn += qn[h][e] * khi[e];
+        dl += qo[h][e] * klo[e];
       }
+      dn = warp_sum(dn) * a.tau;
+      dl = warp_sum(dl) * a.tau;
+      const float mn = fmaxf(m[h], fmaxf(dn, dl));
+      const float sc = m[h] == -INFINITY ? 0.f : expf(m[h] - mn);
+      const float en = expf(dn - mn), eo = expf(dl - mn);
+      z[h] = z[h] * sc + (en - eo);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) acc[h][e] = acc[h][e] * sc + en * vhi[e] - eo * vlo[e];
+      m[h] = mn;
     }
-    __syncthreads();
-    {
-      const int cc = tid % CC, hs = tid / CC;
-      if (cc < cn) {
-        for (int h = hs; h < grp; h += 4) {
-          float dn = 0.f, dl = 0.f;
-#pragma unroll 8
-          for (int e = 0; e < HD; ++e) {
-            dn += An[cc * (HD + 1) + e] * Qn[h * HD + e];
-            dl += Ao[cc * (HD + 1) + e] * Qo[h * HD + e];
-          }
-          Sn[h * a.c + c0 + cc] = dn * a.tau;
-          So[h * a.c + c0 + cc] = dl * a.tau;
-        }
-      }
-    }
-    __syncthreads();
   }
-  // Mx, Z' per head (warp per head)
-  for (int h = warp; h < grp; h += 4) {
-    const size_t so = (static_cast<size_t>(tok) * a.H + g * grp + h);
-    const float L = a.lse_state[so];
-    float m = L;
-    for (int e = lane; e < nc; e += 32) m = fmaxf(m, fmaxf(Sn[h * a.c + e], So[h * a.c + e]));
-    m = warp_max(m);
-    float zs = 0.f;
-    for (int e = lane; e < nc; e += 32) {
-      const float en = expf(Sn[h * a.c + e] - m), eo = expf(So[h * a.c + e] - m);
-      Sn[h * a.c + e] = en;
-      So[h * a.c + e] = eo;
-      zs += en - eo;
-    }
-    zs = warp_sum(zs);
+  // merge the warps of this CTA
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
     if (lane == 0) {
-      const float e0 = expf(L - m);
-      mx[h] = m;
-      el[h] = e0;
-      zz[h] = e0 + zs;
+      sm_m[warp][h] = m[h];
+      sm_z[warp][h] = z[h];
     }
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) sm_acc[warp][h][lane * EPL + e] = acc[h][e];
   }
   __syncthreads();
-  // pass 2: values over C
-  constexpr int HS = 128 / HD;
-  const int d = tid % HD, hslot = tid / HD;
-  float acc[GMAX];
-#pragma unroll
-  for (int h = 0; h < GMAX; ++h) acc[h] = 0.f;
-  for (int c0 = 0; c0 < nc; c0 += CC) {
-    const int cn = min(CC, nc - c0);
-    __syncthreads();
-    for (int rr = warp; rr < cn; rr += 4) {
-      float lo[EPL], hi[EPL];
-      chain_lane2<EPL>(cv, a.j, 1, b, g, C[c0 + rr], m_old, a.loop, lane, lo, hi);
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        Ao[rr * (HD + 1) + lane * EPL + e] = lo[e];
-        An[rr * (HD + 1) + lane * EPL + e] = hi[e];
+  const size_t pbase = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits + sp;
+  for (int e = tid; e < grp * HD; e += 256) {
+    const int h = e / HD, dd = e % HD;
+    float M = -INFINITY;
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][h]);
+    float A = 0.f, Z = 0.f;
+    if (M != -INFINITY)
+      for (int w = 0; w < NW; ++w) {
+        if (sm_m[w][h] == -INFINITY) continue;
+        const float f = expf(sm_m[w][h] - M);
+        A += sm_acc[w][h][dd] * f;
+        Z += sm_z[w][h] * f;
       }
-    }
-    __syncthreads();
-    for (int h = hslot; h < grp; h += HS) {
-      float s = acc[h];
-      for (int cc = 0; cc < cn; ++cc)
-        s += Sn[h * a.c + c0 + cc] * An[cc * (HD + 1) + d] - So[h * a.c + c0 + cc] * Ao[cc * (HD + 1) + d];
-      acc[h] = s;
+    a.part_acc[(pbase * GMAX + h) * HD + dd] = A;
+    if (dd == 0) {
+      a.part_mz[(pbase * GMAX + h) * 2 + 0] = M;
+      a.part_mz[(pbase * GMAX + h) * 2 + 1] = Z;
     }
   }
+  __threadfence();
   __syncthreads();
-  for (int h = hslot; h < grp; h += HS) {
+  if (tid == 0) {
+    const int old = atomicAdd(&a.counters[i * a.Hkv + g], 1);
+    is_last = (old == a.n_splits - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const size_t q0 = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits;
+  for (int e = tid; e < grp * HD; e += 256) {
+    const int h = e / HD, dd = e % HD;
     const int hq = g * grp + h;
     const size_t so = static_cast<size_t>(tok) * a.H + hq;
-    const float z = zz[h];
-    if (!(z > 0.f) && a.status) atomicOr(a.status, kErrBadIndex);
-    const float ov = (el[h] * a.o_state[so * HD + d] + acc[h]) / z;
-    a.o_state[so * HD + d] = ov;
-    a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + d] = f_to_bf16(ov);
-    a.q_last[so * HD + d] = Qn[h * HD + d];
-    if (d == 0) a.lse_state[so] = mx[h] + logf(z);
+    const float L = a.lse_state[so];
+    float M = L;
+    for (int s2 = 0; s2 < a.n_splits; ++s2) M = fmaxf(M, __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2]));
+    const float el = expf(L - M);
+    float Z = el, N = el * a.o_state[so * HD + dd];
+    for (int s2 = 0; s2 < a.n_splits; ++s2) {
+      const float ms = __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2]);
+      if (ms == -INFINITY) continue;
+      const float f = expf(ms - M);
+      Z += f * __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2 + 1]);
+      N += f * __ldcg(&a.part_acc[((q0 + s2) * GMAX + h) * HD + dd]);
+    }
+    if (!(Z > 0.f) && a.status) atomicOr(a.status, kErrBadIndex);
+    const float ov = N / Z;
+    a.o_state[so * HD + dd] = ov;
+    a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + dd] = f_to_bf16(ov);
+    a.q_last[so * HD + dd] = a.q_cur[(static_cast<size_t>(i) * a.H + hq) * HD + dd];
+    if (dd == 0) a.lse_state[so] = M + logf(Z);
   }
+  if (tid == 0) a.counters[i * a.Hkv + g] = 0;
 }
 
 // ============================================================================
@@ -1060,28 +1074,23 @@ cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t 
   k_select_cols<<<max_need * a.Hkv, 1024, 0, s>>>(a);
   return cudaGetLastError();
 }
-size_t correct_smem(int hd, int grp, int c) {
-  return (static_cast<size_t>(2) * 32 * (hd + 1) + 2 * 8 * hd + 2 * static_cast<size_t>(grp) * c) * 4;
-}
 cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
-  const size_t sm = correct_smem(a.hd, a.H / a.Hkv, a.c);
-  if (a.hd == 128) {
-    k_correct<128, 4><<<n_sel * a.Hkv, 128, sm, s>>>(a);
-  } else {
-    k_correct<64, 2><<<n_sel * a.Hkv, 128, sm, s>>>(a);
+  dim3 grid(n_sel * a.Hkv, a.n_splits);
+  const int grp = a.H / a.Hkv;
+#define FL_CORR(G)                                                   \
+  case G:                                                            \
+    if (a.hd == 128) k_correct<128, 4, G><<<grid, 256, 0, s>>>(a);   \
+    else k_correct<64, 2, G><<<grid, 256, 0, s>>>(a);                \
+    break;
+  switch (grp) {
+    FL_CORR(1)
+    FL_CORR(2)
+    FL_CORR(4)
+    FL_CORR(8)
+    default: return cudaErrorInvalidValue;
   }
+#undef FL_CORR
   return cudaGetLastError();
-}
-// Largest dynamic shared memory a kernel may opt in to: the device's per-block
-// opt-in limit less the kernel's own static shared memory.
-template <typename F>
-int max_dyn_smem(F* kern) {
-  int dev = 0, optin = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
-  cudaFuncAttributes fa{};
-  cudaFuncGetAttributes(&fa, kern);
-  return optin - static_cast<int>(fa.sharedSizeBytes);
 }
 
 // Opt every large-shared-memory kernel in to its dynamic shared memory once,
@@ -1098,16 +1107,8 @@ cudaError_t kernels_init_attrs() {
   set(k_attn_prefill<64>, static_cast<int>(attn_prefill_smem(64)));
   set(k_dscore<128, 4>, static_cast<int>(dscore_smem(128)));
   set(k_dscore<64, 2>, static_cast<int>(dscore_smem(64)));
-  // the correction kernel's score buffers grow with c: allow what the device allows
-  // (configurations that need more are refused at init)
-  set(k_correct<128, 4>, max_dyn_smem(k_correct<128, 4>));
-  set(k_correct<64, 2>, max_dyn_smem(k_correct<64, 2>));
   done = e;
   return e;
-}
-
-size_t correct_smem_limit(int hd) {
-  return static_cast<size_t>(hd == 128 ? max_dyn_smem(k_correct<128, 4>) : max_dyn_smem(k_correct<64, 2>));
 }
 
 cudaError_t launch_pack_codes(const int8_t* src, int rows, int hd, int bits, uint8_t* dst, size_t dst_row_stride,

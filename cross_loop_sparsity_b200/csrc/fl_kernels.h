@@ -105,11 +105,13 @@ struct CorrectArgs {
   CacheView cv;
   int j, loop, H, Hkv, hd, c, n_tiles;
   float tau;
+  int cols_per_cta, n_splits;   // column split: grid.y = n_splits = ceil(c / cols_per_cta)
+  float* part_acc;              // [n_sel][Hkv][n_splits][8][hd]
+  float* part_mz;               // [n_sel][Hkv][n_splits][8][2]
+  int* counters;                // [n_sel][Hkv], zero between launches
   int* status;
 };
 
-size_t correct_smem(int hd, int grp, int c);
-size_t correct_smem_limit(int hd);   // the most the correction kernel may opt in to on this device
 cudaError_t kernels_init_attrs();
 
 constexpr int kLensByValue = 256;

@@ -10,6 +10,7 @@
 //                corrected over the fixed top-c key columns of their query tile
 // The dense baseline (resid_bits 16) recomputes every token every loop with a
 // per-loop bf16 KV ("Looped Transformer 教程", 第一步 / 第四步).
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <new>
@@ -55,6 +56,8 @@ struct flashloop_ctx {
   int* forced_ncols = nullptr;
   float *part_o = nullptr, *part_ml = nullptr;
   int* attn_counters = nullptr;
+  float *corr_acc = nullptr, *corr_mz = nullptr;
+  int* corr_counters = nullptr;
   float* gemm_partial = nullptr;
   size_t gemm_partial_cap = 0;
   int* gemm_counters = nullptr;
@@ -81,6 +84,9 @@ struct flashloop_ctx {
 namespace {
 
 constexpr int kNumSM = 148;
+// Sparse-column correction: columns per CTA.  Few selected queries (decode)
+// get narrow splits for parallelism; many (prefill) get wide ones.
+constexpr int kCorrColsSmall = 16, kCorrColsBig = 128, kCorrSmallQueries = 64;
 constexpr int kCountersGemm = 4096;
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -99,7 +105,10 @@ bool valid_config(const flashloop_config* c) {
   if (c->d_model < 64 || c->d_model % 64) return false;
   if (c->head_dim != 64 && c->head_dim != 128) return false;
   if (c->n_heads < 1 || c->n_kv_heads < 1 || c->n_heads % c->n_kv_heads) return false;
-  if (c->n_heads / c->n_kv_heads > 8) return false;
+  {
+    const int grp = c->n_heads / c->n_kv_heads;   // query heads per KV head: 1, 2, 4 or 8
+    if (grp != 1 && grp != 2 && grp != 4 && grp != 8) return false;
+  }
   if (c->ffn_dim < 8 || c->ffn_dim % 8) return false;
   if (c->n_layers < 1 || c->n_loops < 1 || c->n_loops > 16) return false;
   if (c->resid_bits != 2 && c->resid_bits != 4 && c->resid_bits != 16) return false;
@@ -206,6 +215,17 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   uint8_t* part_o = take(B * Hkv * splits * 8 * hd * 4);
   uint8_t* part_ml = take(B * Hkv * splits * 8 * 2 * 4);
   uint8_t* attn_counters = take(B * Hkv * 4);
+  // correction column-split partials (the larger of the two split shapes)
+  size_t cp_rows = 0;
+  if (lazy) {
+    const int ns_small = ceil_div(cc, kCorrColsSmall), ns_big = ceil_div(cc, kCorrColsBig);
+    const size_t small_rows = static_cast<size_t>(std::min(nsel_max, kCorrSmallQueries)) * Hkv * ns_small;
+    const size_t big_rows = static_cast<size_t>(nsel_max) * Hkv * ns_big;
+    cp_rows = std::max(small_rows, big_rows);
+  }
+  uint8_t* corr_acc = take(std::max<size_t>(cp_rows, 1) * 8 * hd * 4);
+  uint8_t* corr_mz = take(std::max<size_t>(cp_rows, 1) * 8 * 2 * 4);
+  uint8_t* corr_counters = take(static_cast<size_t>(std::max(nsel_max, 1)) * Hkv * 4);
   // GEMM split-K partials (skinny orientation only)
   size_t gp = 0;
   if (N <= 64 || c.max_batch <= 64) {
@@ -287,6 +307,9 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->part_o = reinterpret_cast<float*>(part_o);
     x->part_ml = reinterpret_cast<float*>(part_ml);
     x->attn_counters = reinterpret_cast<int*>(attn_counters);
+    x->corr_acc = reinterpret_cast<float*>(corr_acc);
+    x->corr_mz = reinterpret_cast<float*>(corr_mz);
+    x->corr_counters = reinterpret_cast<int*>(corr_counters);
     x->gemm_partial = reinterpret_cast<float*>(gpart);
     x->gemm_partial_cap = gp;
     x->gemm_counters = reinterpret_cast<int*>(gcnt);
@@ -507,6 +530,9 @@ fl_status run_call(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s)
         ca.q_cur = ctx->q_cur; ca.q_last = ql; ca.o_state = o_st; ca.lse_state = l_st; ca.o_bf16 = ctx->obf;
         ca.cols = ctx->cols; ca.ncols = ctx->ncols; ca.cv = ctx->cv; ca.j = j; ca.loop = l; ca.H = H; ca.Hkv = Hkv;
         ca.hd = hd; ca.c = c.c_cols; ca.n_tiles = ctx->n_tiles_max; ca.tau = tau; ca.status = ctx->status;
+        ca.cols_per_cta = n_sel <= kCorrSmallQueries ? kCorrColsSmall : kCorrColsBig;
+        ca.n_splits = ceil_div(c.c_cols, ca.cols_per_cta);
+        ca.part_acc = ctx->corr_acc; ca.part_mz = ctx->corr_mz; ca.counters = ctx->corr_counters;
         FL_LAUNCH(FL_KIND_CORRECT, launch_correct(ca, n, s));
       }
       FL_GEMM(gemm(ctx, kOpO, j, n, idx, s));
@@ -626,9 +652,7 @@ fl_status flashloop_init(const flashloop_config* cfg, const flashloop_weights* w
       return fail(FL_ERR_CUDA);
     }
   }
-  if (ctx->lazy && correct_smem(cfg->head_dim, cfg->n_heads / cfg->n_kv_heads, cfg->c_cols) >
-                       correct_smem_limit(cfg->head_dim))
-    return fail(FL_ERR_UNSUPPORTED);
+
   if (!build_tmaps(ctx)) return fail(FL_ERR_CUDA);
   if (cudaMemsetAsync(ctx->ws, 0, need, s) != cudaSuccess) return fail(FL_ERR_CUDA);
   // RoPE table: angle = pos * theta^(-2i/hd), computed in double, stored fp32
