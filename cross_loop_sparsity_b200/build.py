@@ -17,7 +17,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libflashloop.so")
-SOURCES = ["fl_gemm.cu", "fl_kernels.cu", "fl_runtime.cu"]
+SOURCES = ["fl_gemm.cu", "fl_kernels.cu", "fl_runtime.cu", "fl_noalloc.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "-Xptxas", "-O3",

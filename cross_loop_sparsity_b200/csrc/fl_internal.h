@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
+#include <string>
 
 namespace fl {
 
@@ -60,6 +61,10 @@ size_t gemm_partial_floats(int bn, int dual, int tiles, int splits);
 // else [rows][k] rank 2), 128-byte swizzle, box 64 x box_rows (x 1).
 bool encode_tmap_bf16(CUtensorMap* map, const void* base, uint64_t k, uint64_t rows, uint64_t layers,
                       uint32_t box_rows);
+
+// Record the reason of a failure of an entry point that has no context
+// (reported by flashloop_last_cuda_error(NULL)).
+void set_last_error(const std::string& why);
 
 // ------------------------------------------------------------------ other kernels
 struct SelectSeg;  // fwd

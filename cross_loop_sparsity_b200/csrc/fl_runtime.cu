@@ -26,6 +26,8 @@ namespace {
 std::string g_last_error;  // last CUDA error of an entry point that has no context
 }  // namespace
 
+void fl::set_last_error(const std::string& why) { g_last_error = why; }
+
 struct flashloop_ctx {
   flashloop_config cfg;
   flashloop_weights w;

@@ -73,6 +73,7 @@ _SIG = {
     "fl_test_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "fl_test_gemm_scratch_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fl_test_gemm": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_size_t, _P]),
+    "fl_gemm_skinny_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _P]),
 }
 
 _lib = None
@@ -341,4 +342,17 @@ def gemm(A, B, swap_ab: bool = False, stream=None):
     sp = scratch.data_ptr() + ((-scratch.data_ptr()) % 256)
     _check(lib().fl_test_gemm(_ptr(A), _ptr(B), _ptr(D), m, n, k, int(swap_ab), ctypes.c_void_p(sp), nb,
                               _stream_ptr(stream)), "fl_test_gemm")
+    return D
+
+
+def gemm_noalloc(A, B, out=None, stream=None):
+    """D = A @ B.T (m <= 64) through the entry point that allocates nothing:
+    its split-K scratch is an array inside the library.  ``out`` (fp32 [m, n])
+    may be given so the call itself allocates nothing on the torch side either."""
+    import torch
+    m, k = A.shape
+    n = B.shape[0]
+    D = out if out is not None else torch.empty((m, n), dtype=torch.float32, device=A.device)
+    _check(lib().fl_gemm_skinny_noalloc(_ptr(A), _ptr(B), _ptr(D), m, n, k, _stream_ptr(stream)),
+           "fl_gemm_skinny_noalloc")
     return D

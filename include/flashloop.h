@@ -215,6 +215,32 @@ size_t fl_test_gemm_scratch_bytes(int m, int n, int k, int swap_ab);
 fl_status fl_test_gemm(const uint16_t* A, const uint16_t* B, float* D, int m, int n, int k, int swap_ab,
                        void* scratch, size_t scratch_bytes, fl_stream_t stream);
 
+/* Decode-shaped GEMM for callers that cannot allocate device memory.  The
+ * paper has no counterpart: this is a service of the library, not a step of
+ * the method.  Some callers may not call cudaMalloc at all -- code running in
+ * another framework's memory pool that already owns the device memory,
+ * latency-critical paths that cannot afford cudaMalloc's implicit device
+ * synchronisation, plugin hosts that forbid allocation -- yet the skinny
+ * split-K GEMM (fl_test_gemm with swap_ab = 1) needs scratch for its partial
+ * tiles and tickets.  This variant computes the same D[m][n] = sum_k A[m][k] *
+ * B[n][k] (bf16 in, fp32 out; 1 <= m <= 64, k % 8 == 0, pointers 16-byte
+ * aligned, all device memory owned by the caller) with its scratch in an
+ * array compiled into the library: FL_NOALLOC_SCRATCH_BYTES of split-K
+ * partials plus 16 KiB of tickets, held on every GPU that loads the library
+ * until the process exits.  It allocates nothing.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Shapes whose partials exceed FL_NOALLOC_SCRATCH_BYTES are refused with
+ *    FL_ERR_CAPACITY and a reason in flashloop_last_cuda_error(NULL); use
+ *    fl_test_gemm with caller scratch for those.
+ *  - Every call shares the one array and leaves its contents behind; the
+ *    tickets are cleared on the call's stream before each launch.  Calls that
+ *    overlap on the GPU (other streams, other host threads) race on it. */
+#define FL_NOALLOC_SCRATCH_BYTES (2u << 20)
+fl_status fl_gemm_skinny_noalloc(const uint16_t* A, const uint16_t* B, float* D, int m, int n, int k,
+                                 fl_stream_t stream);
+
 /* Runtime options of a context. */
 typedef enum {
   FL_OPT_USE_GRAPH = 1, /* 1 (default): capture decode steps into CUDA graphs; 0: launch directly */

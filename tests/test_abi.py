@@ -23,7 +23,7 @@ def L():
 def _declared():
     src = open(os.path.join(ROOT, "include", "flashloop.h")).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b((?:flashloop|fl_test)_[a-z_]+)\s*\(", src)))
+    return sorted(set(re.findall(r"\b((?:flashloop|fl_test|fl_gemm)_[a-z_]+)\s*\(", src)))
 
 
 def test_every_declared_symbol_is_exported(L):
