@@ -95,21 +95,79 @@ __device__ __forceinline__ void chain_lane(const CacheView& cv, int j, int kv, i
   }
 }
 
-// Base and loop-m reconstruction of one row in one pass (lane holds EPL values each).
+// Maximum loops K the reconstruction below unrolls for.
+constexpr int kMaxLoops = 16;
+
+// Reconstructions to loop m_lo and to loop m_hi (m_lo <= m_hi) of one row;
+// lane holds EPL values of each.  All loads (base row, residual codes and
+// scales of loops 2..m_hi) are issued before any arithmetic so their latencies
+// overlap; the adds then run in loop order, as the definition requires.
 template <int EPL>
 __device__ __forceinline__ void chain_lane2(const CacheView& cv, int j, int kv, int b, int h, int t, int m_lo,
                                             int m_hi, int lane, float* lo, float* hi) {
-  chain_lane<EPL>(cv, j, kv, b, h, t, m_lo, lane, lo);
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) hi[e] = lo[e];
-  const int gi = (lane * EPL) / cv.g;
-  for (int l = m_lo + 1; l <= m_hi; ++l) {
-    int c[EPL];
-    lane_codes<EPL>(cv.code_row(j, l, kv, b, h, t), cv.bits, lane, c);
-    const float s = half_bits_to_f(cv.scale_row(j, l, kv, b, h, t)[gi]);
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) hi[e] = __fadd_rn(hi[e], __fmul_rn(static_cast<float>(c[e]), s));
+  const uint16_t* br = cv.base_row(j, kv, b, h, t) + lane * EPL;
+  uint32_t braw[EPL == 4 ? 2 : 1];
+  if (EPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(br);
+    braw[0] = u.x;
+    braw[EPL == 4 ? 1 : 0] = u.y;
+  } else {
+    braw[0] = *reinterpret_cast<const uint32_t*>(br);
   }
+  const int gi = (lane * EPL) / cv.g;
+  const size_t rb = cv.row_bytes_codes(), ns = cv.hd / cv.g;
+  const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * cv.T;   // rows between consecutive loops
+  const size_t r0 = cv.res_index(j, 2, kv, b, h, t);
+  uint32_t craw[kMaxLoops - 1];
+  uint16_t sraw[kMaxLoops - 1];
+#pragma unroll
+  for (int q = 0; q < kMaxLoops - 1; ++q) {
+    craw[q] = 0u;
+    sraw[q] = 0;
+    if (q + 2 <= m_hi) {
+      const uint8_t* row = cv.codes + (r0 + q * step) * rb;
+      if (EPL == 4) {
+        craw[q] = cv.bits == 4 ? static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(row + lane * 2))
+                               : static_cast<uint32_t>(row[lane]);
+      } else {
+        craw[q] = cv.bits == 4 ? static_cast<uint32_t>(row[lane])
+                               : static_cast<uint32_t>((row[lane >> 1] >> ((lane & 1) * 4)) & 0xF);
+      }
+      sraw[q] = cv.scales[(r0 + q * step) * ns + gi];
+    }
+  }
+  float acc[EPL];
+  if (EPL == 4) {
+    acc[0] = bf16_to_f(braw[0] & 0xFFFF);
+    acc[1] = bf16_to_f(braw[0] >> 16);
+    acc[EPL == 4 ? 2 : 0] = bf16_to_f(braw[EPL == 4 ? 1 : 0] & 0xFFFF);
+    acc[EPL == 4 ? 3 : 1] = bf16_to_f(braw[EPL == 4 ? 1 : 0] >> 16);
+  } else {
+    acc[0] = bf16_to_f(braw[0] & 0xFFFF);
+    acc[1] = bf16_to_f(braw[0] >> 16);
+  }
+  if (m_lo <= 1) {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) lo[e] = acc[e];
+  }
+  const int fb = cv.bits;
+#pragma unroll
+  for (int q = 0; q < kMaxLoops - 1; ++q) {
+    if (q + 2 <= m_hi) {
+      const float sc = half_bits_to_f(sraw[q]);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        const int c = sext(static_cast<int>((craw[q] >> (fb * e)) & ((1u << fb) - 1)), fb);
+        acc[e] = __fadd_rn(acc[e], __fmul_rn(static_cast<float>(c), sc));
+      }
+      if (q + 2 == m_lo) {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) lo[e] = acc[e];
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EPL; ++e) hi[e] = acc[e];
 }
 
 }  // namespace fl

@@ -21,10 +21,16 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kBoxK = 64;             // bf16 elements per 128-byte swizzled row
 constexpr int kABytes = 128 * kBoxK * 2;
-constexpr int kSmemBudget = 200 * 1024;
+// Shared-memory ring budget: the skinny (decode) orientation keeps two CTAs per
+// SM so that a dependent GEMM can become resident and start streaming its
+// weights while the previous kernel still runs; the 128x128 orientation uses
+// one deep ring per SM.
+constexpr int kSmemBudgetSkinny = 100 * 1024;
+constexpr int kSmemBudgetWide = 200 * 1024;
 
 template <int BN, bool DA, bool DB>
 struct Cfg {
+  static constexpr int kSmemBudget = BN <= 64 ? kSmemBudgetSkinny : kSmemBudgetWide;
   static constexpr int kNA = DA ? 2 : 1;
   static constexpr int kNB = DB ? 2 : 1;
   static constexpr int kBBytes = BN * kBoxK * 2;
@@ -70,7 +76,7 @@ __device__ __forceinline__ void epi_apply(const GemmArgs& p, int row, int col0, 
 }
 
 template <int BN, bool DA, bool DB, bool SWAP>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
           const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
           const GemmArgs p, const int a_3d, const int b_3d) {
@@ -83,6 +89,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(done + 1);
   volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort, [1] last-split
 
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tile_m = blockIdx.x, tile_n = blockIdx.y, split = blockIdx.z;
   const int c0 = (split * p.k_chunks) / p.splits;
@@ -112,8 +119,52 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
     // ---------------- TMA producer
     tma_prefetch_desc(&tmA0);
     tma_prefetch_desc(&tmB0);
-    int issued = 0;
-    for (int i = 0; i < nch; ++i) {
+    // Weights never depend on an earlier kernel: the weight tiles of the first
+    // ring slots are requested before waiting on the predecessor grid; the
+    // activation tiles follow once it has completed.
+    auto load_w = [&](int i, uint8_t* st, uint32_t fb) {
+      const int kx = (c0 + i) * kBoxK;
+      if (SWAP) {
+        if (a_3d) {
+          tma_load_3d(smem_u32(st), &tmA0, fb, kx, tile_m * 128, p.a_z);
+          if (DA) tma_load_3d(smem_u32(st + kABytes), &tmA1, fb, kx, tile_m * 128, p.a_z);
+        } else {
+          tma_load_2d(smem_u32(st), &tmA0, fb, kx, tile_m * 128);
+          if (DA) tma_load_2d(smem_u32(st + kABytes), &tmA1, fb, kx, tile_m * 128);
+        }
+      } else {
+        uint8_t* sb = st + C::kNA * kABytes;
+        if (b_3d) {
+          tma_load_3d(smem_u32(sb), &tmB0, fb, kx, tile_n * BN, p.b_z);
+          if (DB) tma_load_3d(smem_u32(sb + C::kBBytes), &tmB1, fb, kx, tile_n * BN, p.b_z);
+        } else {
+          tma_load_2d(smem_u32(sb), &tmB0, fb, kx, tile_n * BN);
+          if (DB) tma_load_2d(smem_u32(sb + C::kBBytes), &tmB1, fb, kx, tile_n * BN);
+        }
+      }
+    };
+    auto load_x = [&](int i, uint8_t* st, uint32_t fb) {
+      const int kx = (c0 + i) * kBoxK;
+      if (SWAP) {
+        uint8_t* sb = st + C::kNA * kABytes;
+        if (b_3d) tma_load_3d(smem_u32(sb), &tmB0, fb, kx, tile_n * BN, p.b_z);
+        else tma_load_2d(smem_u32(sb), &tmB0, fb, kx, tile_n * BN);
+      } else {
+        if (a_3d) tma_load_3d(smem_u32(st), &tmA0, fb, kx, tile_m * 128, p.a_z);
+        else tma_load_2d(smem_u32(st), &tmA0, fb, kx, tile_m * 128);
+      }
+    };
+    const int pre = nch < C::kStages ? nch : C::kStages;
+    for (int i = 0; i < pre; ++i) {
+      uint8_t* st = smem + i * C::kStageBytes;
+      const uint32_t fb = smem_u32(&full[i]);
+      mbar_arrive_expect_tx(fb, C::kStageBytes);
+      load_w(i, st, fb);
+    }
+    pdl_wait();
+    for (int i = 0; i < pre; ++i) load_x(i, smem + i * C::kStageBytes, smem_u32(&full[i]));
+    int issued = pre;
+    for (int i = pre; i < nch; ++i) {
       const int s = i % C::kStages;
       const uint32_t ph = (i / C::kStages) & 1;
       if (!mbar_wait(smem_u32(&empty[s]), ph ^ 1u, p.status)) {
@@ -123,24 +174,8 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
       uint8_t* st = smem + s * C::kStageBytes;
       const uint32_t fb = smem_u32(&full[s]);
       mbar_arrive_expect_tx(fb, C::kStageBytes);
-      const int kx = (c0 + i) * kBoxK;
-      const int ya = tile_m * 128;
-      const int yb = tile_n * BN;
-      if (a_3d) {
-        tma_load_3d(smem_u32(st), &tmA0, fb, kx, ya, p.a_z);
-        if (DA) tma_load_3d(smem_u32(st + kABytes), &tmA1, fb, kx, ya, p.a_z);
-      } else {
-        tma_load_2d(smem_u32(st), &tmA0, fb, kx, ya);
-        if (DA) tma_load_2d(smem_u32(st + kABytes), &tmA1, fb, kx, ya);
-      }
-      uint8_t* sb = st + C::kNA * kABytes;
-      if (b_3d) {
-        tma_load_3d(smem_u32(sb), &tmB0, fb, kx, yb, p.b_z);
-        if (DB) tma_load_3d(smem_u32(sb + C::kBBytes), &tmB1, fb, kx, yb, p.b_z);
-      } else {
-        tma_load_2d(smem_u32(sb), &tmB0, fb, kx, yb);
-        if (DB) tma_load_2d(smem_u32(sb + C::kBBytes), &tmB1, fb, kx, yb);
-      }
+      load_w(i, st, fb);
+      load_x(i, st, fb);
       ++issued;
     }
     if (flags[0]) {
@@ -182,6 +217,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
     // ---------------- epilogue
     const int q = warp & 3;
     const int row = q * 32 + lane;
+    pdl_wait();
     const bool ok = mbar_wait(smem_u32(done), 0, p.status);
     __syncwarp();   // tcgen05.ld below is warp-collective (.sync.aligned)
     tc_fence_after();
@@ -224,6 +260,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
             v0[j] = 0.f;
             v1[j] = 0.f;
           }
+#pragma unroll 2
           for (int s = 0; s < p.splits; ++s) {
             const float* src = p.partial + (static_cast<size_t>(s) * gridDim.x + tile_m) * tile_floats;
 #pragma unroll
@@ -253,8 +290,8 @@ cudaError_t launch_one(const GemmLaunch& g, cudaStream_t stream) {
   auto kern = k_gemm_tc<BN, DA, DB, SWAP>;
   const CUtensorMap& a1 = g.a1 ? *g.a1 : *g.a0;
   const CUtensorMap& b1 = g.b1 ? *g.b1 : *g.b0;
-  kern<<<g.grid, kThreads, C::kSmemBytes, stream>>>(*g.a0, a1, *g.b0, b1, g.args, g.a_3d, g.b_3d);
-  return cudaGetLastError();
+  return launch_k(g.pdl, kern, g.grid, dim3(kThreads), C::kSmemBytes, stream, *g.a0, a1, *g.b0, b1, g.args,
+                  g.a_3d, g.b_3d);
 }
 
 template <int BN, bool DA, bool DB, bool SWAP>

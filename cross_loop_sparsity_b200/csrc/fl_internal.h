@@ -50,9 +50,29 @@ struct GemmLaunch {
   int a_3d, b_3d;          // operand maps are layer-stacked (rank 3)
   dim3 grid;
   GemmArgs args;
+  bool pdl = false;        // launched as a programmatic dependent of the previous kernel
 };
 
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream);
+
+// Launch a kernel, with programmatic stream serialisation when `pdl` is set
+// (only for launches whose predecessor in the stream is one of this
+// library's kernels that follows the pdl_wait discipline).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 cudaError_t gemm_init_attrs();   // opt the GEMM kernels in to their shared memory (once)
 // Largest split-K scratch (floats) one launch with these sizes may use.
 size_t gemm_partial_floats(int bn, int dual, int tiles, int splits);

@@ -64,6 +64,7 @@ __device__ int block_topk(const float* __restrict__ keys, int n, int k, int32_t*
   __shared__ int hist[256];
   __shared__ int sh_sel, sh_cum;
   __shared__ int scan_buf[33];
+  __shared__ uint32_t small_keys[1024];
   if (k >= n) {
     for (int i = threadIdx.x; i < n; i += blockDim.x) out[i] = i;
     __syncthreads();
@@ -71,6 +72,27 @@ __device__ int block_topk(const float* __restrict__ keys, int n, int k, int32_t*
   }
   if (k <= 0) return 0;
   const uint32_t* kb = reinterpret_cast<const uint32_t*>(keys);
+  if (n <= static_cast<int>(blockDim.x)) {
+    // one key per thread: its rank is the number of keys that precede it in
+    // (bit pattern desc, index asc) order; the k of rank < k are taken, in
+    // index order by a block scan
+    const int i = threadIdx.x;
+    const uint32_t u = i < n ? kb[i] : 0u;
+    if (i < n) small_keys[i] = u;
+    __syncthreads();
+    int rank = 0;
+    if (i < n)
+      for (int j = 0; j < n; ++j) {
+        const uint32_t v = small_keys[j];
+        rank += (v > u || (v == u && j < i)) ? 1 : 0;
+      }
+    const int take = (i < n && rank < k) ? 1 : 0;
+    int total;
+    const int pos = block_exclusive_scan(take, &total, scan_buf);
+    if (take) out[pos] = i;
+    __syncthreads();
+    return k;
+  }
   uint32_t prefix = 0, mask = 0;
   int k_rem = k;
   for (int shift = 24; shift >= 0; shift -= 8) {
@@ -81,17 +103,14 @@ __device__ int block_topk(const float* __restrict__ keys, int n, int k, int32_t*
       if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 0xFF], 1);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int cum = 0, sel = 0;
-      for (int d = 255; d >= 0; --d) {
-        if (cum + hist[d] >= k_rem) {
-          sel = d;
-          break;
-        }
-        cum += hist[d];
-      }
-      sh_sel = sel;
-      sh_cum = cum;
+    // the digit holding the k_rem-th largest key: a scan over the bins in
+    // descending digit order (thread t < 256 holds digit 255 - t)
+    const int cnt = threadIdx.x < 256 ? hist[255 - threadIdx.x] : 0;
+    int tot;
+    const int before = block_exclusive_scan(cnt, &tot, scan_buf);
+    if (threadIdx.x < 256 && before < k_rem && before + cnt >= k_rem) {
+      sh_sel = 255 - threadIdx.x;
+      sh_cum = before;
     }
     __syncthreads();
     k_rem -= sh_cum;
@@ -121,6 +140,8 @@ __device__ int block_topk(const float* __restrict__ keys, int n, int k, int32_t*
 
 __global__ void __launch_bounds__(1024) k_topk_segments(const float* __restrict__ keys, int n, int k,
                                                         int32_t* __restrict__ idx) {
+  pdl_trigger();
+  pdl_wait();
   const int s = blockIdx.x;
   block_topk(keys + static_cast<size_t>(s) * n, n, k, idx + static_cast<size_t>(s) * (k < n ? k : n));
 }
@@ -130,6 +151,8 @@ __global__ void __launch_bounds__(1024) k_topk_segments(const float* __restrict_
 __global__ void __launch_bounds__(1024) k_select_tokens(const float* __restrict__ keys, int N, int n_sel,
                                                         int32_t* __restrict__ idx, const int* forced_on,
                                                         const int32_t* __restrict__ forced) {
+  pdl_trigger();
+  pdl_wait();
   if (forced_on && forced_on[0]) {
     for (int i = threadIdx.x; i < n_sel; i += blockDim.x) idx[i] = forced[i];
     return;
@@ -144,6 +167,8 @@ __global__ void __launch_bounds__(1024) k_select_tokens(const float* __restrict_
 __global__ void __launch_bounds__(256) k_rmsnorm_rows(const float* __restrict__ h, const int* __restrict__ idx,
                                                       int n, int d, const float* __restrict__ gain, float eps,
                                                       uint16_t* __restrict__ x) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float buf[32];
   const int i = blockIdx.x;
   uint16_t* xr = x + static_cast<size_t>(i) * d;
@@ -224,6 +249,8 @@ template <int EPL>
 __global__ void __launch_bounds__(128) k_quantize_rows(const float* __restrict__ r, int rows, int width, int g,
                                                        int bits, uint8_t* __restrict__ codes,
                                                        uint16_t* __restrict__ scales) {
+  pdl_trigger();
+  pdl_wait();
   const int warp_global = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   const int chunks = width / (32 * EPL);
   if (warp_global >= rows * chunks) return;
@@ -250,6 +277,8 @@ __global__ void __launch_bounds__(128) k_quantize_rows(const float* __restrict__
 // ============================================================================
 template <int EPL>
 __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int heads = a.H + 2 * a.Hkv;
@@ -322,84 +351,123 @@ __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
 
 // ============================================================================
 // decode attention over one cache (lazy base at loop 1, or the dense
-// baseline's own per-loop KV): grid (n*Hkv, splits); each CTA handles the
-// group's query heads over one column range, 64-column tiles staged in
-// shared memory; the last CTA of a (token, KV head) merges the splits.
+// baseline's own per-loop KV): grid (n*Hkv, splits), 256 threads.  Each CTA
+// takes the group's query heads over one column range in 64-column tiles;
+// K/V tiles are double-buffered in shared memory with cp.async so the next
+// tile streams in while the current one is scored and accumulated.  The last
+// CTA of a (token, KV head) -- an atomic ticket, no waiting -- merges the
+// splits' (max, sum, unnormalised output) and writes O, lse.
 // ============================================================================
 constexpr int kDecTile = 64;
-constexpr int kDecPad = 8;  // bf16 elements of padding per staged row
+constexpr int kDecPad = 8;  // bf16 elements of padding per staged row (16-byte skew)
 
-template <int HD>
-__global__ void __launch_bounds__(128) k_attn_decode(const AttnDecArgs a) {
-  constexpr int RS = HD + kDecPad;                 // staged row stride (bf16)
-  constexpr int GMAX = 8;
-  __shared__ __align__(16) uint16_t Ks[kDecTile * RS];
-  __shared__ __align__(16) uint16_t Vs[kDecTile * RS];
-  __shared__ float Qs[GMAX * HD];
-  __shared__ float S[GMAX][kDecTile];
-  __shared__ float m_run[GMAX], l_run[GMAX], alpha[GMAX];
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int HD, int GRP>
+__global__ void __launch_bounds__(256) k_attn_decode(const AttnDecArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int RS = HD + kDecPad;
+  constexpr int CH = HD / 8;         // 16-byte chunks per row
+  constexpr int DQ = HD / 4;         // dims per quarter (score phase)
+  constexpr int NP = HD / 2;         // dim pairs (PV phase)
+  constexpr int CQ = 256 / NP;       // column groups of the PV phase: 4 (hd 128) or 8 (hd 64)
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint16_t* Kst = reinterpret_cast<uint16_t*>(sm);          // [2][64][RS]
+  uint16_t* Vst = Kst + 2 * kDecTile * RS;                  // [2][64][RS]
+  __shared__ float Qs[GRP * HD];
+  __shared__ float S[GRP][kDecTile];
+  __shared__ float m_run[GRP], l_run[GRP], alpha[GRP];
+  __shared__ float red[CQ][GRP][HD];
+  __shared__ float sm_m[GRP], sm_l[GRP];
   __shared__ int is_last;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int i = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv, sp = blockIdx.y;
-  const int grp = a.H / a.Hkv;
   const int tok = a.idx ? a.idx[i] : i;
   const int b = a.seq[tok], P = a.pos[tok];
   const int c_begin = sp * a.split_len;
   const int c_end = min(c_begin + a.split_len, P + 1);
   const CacheView& cv = a.cv;
+  const uint16_t* kbase = a.dense ? cv.dense_row(a.j, a.loop, 0, b, g, 0) : cv.base_row(a.j, 0, b, g, 0);
+  const uint16_t* vbase = a.dense ? cv.dense_row(a.j, a.loop, 1, b, g, 0) : cv.base_row(a.j, 1, b, g, 0);
 
-  for (int e = tid; e < grp * HD; e += 128)
-    Qs[e] = a.q_cur[(static_cast<size_t>(i) * a.H + g * grp) * HD + e];
-  if (tid < GMAX) {
+  for (int e = tid; e < GRP * HD; e += 256) Qs[e] = a.q_cur[(static_cast<size_t>(i) * a.H + g * GRP) * HD + e];
+  if (tid < GRP) {
     m_run[tid] = -INFINITY;
     l_run[tid] = 0.f;
   }
-  // thread -> (output dim d, head slot) for the PV accumulation
-  constexpr int HS = 128 / HD;                  // head slots: 1 (hd 128) or 2 (hd 64)
-  const int d = tid % HD, hslot = tid / HD;
-  float acc[GMAX];
+  // PV phase: thread -> dim pair dp, column group cq; all GRP heads
+  const int dp = tid % NP, cq = tid / NP;
+  float acc[GRP][2];
 #pragma unroll
-  for (int h = 0; h < GMAX; ++h) acc[h] = 0.f;
-  __syncthreads();
+  for (int h = 0; h < GRP; ++h) acc[h][0] = acc[h][1] = 0.f;
 
-  for (int c0 = c_begin; c0 < c_end; c0 += kDecTile) {
+  auto stage = [&](int buf, int c0) {
     const int nc = min(kDecTile, c_end - c0);
-    // stage K and V rows (16-byte chunks)
-    constexpr int CH = HD / 8;  // 16-byte chunks per row
-    for (int e = tid; e < nc * CH; e += 128) {
+    for (int e = tid; e < kDecTile * CH; e += 256) {
       const int r = e / CH, cc = e % CH;
-      const uint16_t* kr = a.dense ? cv.dense_row(a.j, a.loop, 0, b, g, c0 + r) : cv.base_row(a.j, 0, b, g, c0 + r);
-      const uint16_t* vr = a.dense ? cv.dense_row(a.j, a.loop, 1, b, g, c0 + r) : cv.base_row(a.j, 1, b, g, c0 + r);
-      *reinterpret_cast<uint4*>(&Ks[r * RS + cc * 8]) = *reinterpret_cast<const uint4*>(kr + cc * 8);
-      *reinterpret_cast<uint4*>(&Vs[r * RS + cc * 8]) = *reinterpret_cast<const uint4*>(vr + cc * 8);
+      const bool in = r < nc;
+      const size_t off = static_cast<size_t>(in ? c0 + r : c0) * HD + cc * 8;
+      cp_async16(smem_u32(Kst + (buf * kDecTile + r) * RS + cc * 8), kbase + off, in ? 16u : 0u);
+      cp_async16(smem_u32(Vst + (buf * kDecTile + r) * RS + cc * 8), vbase + off, in ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+
+  const int n_tiles = c_end > c_begin ? (c_end - c_begin + kDecTile - 1) / kDecTile : 0;
+  if (n_tiles > 0) stage(0, c_begin);
+  __syncthreads();
+  for (int t = 0; t < n_tiles; ++t) {
+    const int buf = t & 1;
+    const int c0 = c_begin + t * kDecTile;
+    const int nc = min(kDecTile, c_end - c0);
+    if (t + 1 < n_tiles) {
+      stage(buf ^ 1, c0 + kDecTile);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
-    // scores: thread -> column tid % 64, heads tid/64, tid/64 + 2, ...
+    const uint16_t* Ks = Kst + buf * kDecTile * RS;
+    const uint16_t* Vs = Vst + buf * kDecTile * RS;
+    // scores: thread -> column c = tid / 4, dim quarter tid % 4, every head; the
+    // four quarters are summed by shuffles (they are adjacent lanes)
     {
-      const int c = tid % kDecTile, h0 = tid / kDecTile;
-      for (int h = h0; h < grp; h += 2) {
-        float s = -INFINITY;
-        if (c < nc) {
-          float dot = 0.f;
-          const uint16_t* kr = &Ks[c * RS];
-          const float* q = &Qs[h * HD];
-#pragma unroll 8
-          for (int e = 0; e < HD; e += 8) {
-            const uint4 u = *reinterpret_cast<const uint4*>(kr + e);
-            dot += q[e + 0] * bf16_to_f(u.x & 0xFFFF) + q[e + 1] * bf16_to_f(u.x >> 16);
-            dot += q[e + 2] * bf16_to_f(u.y & 0xFFFF) + q[e + 3] * bf16_to_f(u.y >> 16);
-            dot += q[e + 4] * bf16_to_f(u.z & 0xFFFF) + q[e + 5] * bf16_to_f(u.z >> 16);
-            dot += q[e + 6] * bf16_to_f(u.w & 0xFFFF) + q[e + 7] * bf16_to_f(u.w >> 16);
-          }
-          s = dot * a.tau;
+      const int c = tid >> 2, qd = tid & 3;
+      float dot[GRP];
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) dot[h] = 0.f;
+      const uint16_t* kr = Ks + c * RS + qd * DQ;
+#pragma unroll
+      for (int e = 0; e < DQ; e += 8) {
+        const uint4 u = *reinterpret_cast<const uint4*>(kr + e);
+        const float k0 = __uint_as_float(u.x << 16), k1 = __uint_as_float(u.x & 0xFFFF0000u);
+        const float k2 = __uint_as_float(u.y << 16), k3 = __uint_as_float(u.y & 0xFFFF0000u);
+        const float k4 = __uint_as_float(u.z << 16), k5 = __uint_as_float(u.z & 0xFFFF0000u);
+        const float k6 = __uint_as_float(u.w << 16), k7 = __uint_as_float(u.w & 0xFFFF0000u);
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) {
+          const float* q = &Qs[h * HD + qd * DQ + e];
+          dot[h] += q[0] * k0 + q[1] * k1 + q[2] * k2 + q[3] * k3 + q[4] * k4 + q[5] * k5 + q[6] * k6 + q[7] * k7;
         }
-        S[h][c] = s;
+      }
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) {
+        float v = dot[h];
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        if (qd == 0) S[h][c] = c < nc ? v * a.tau : -INFINITY;
       }
     }
     __syncthreads();
-    // online softmax per head: warp w handles heads w, w+4
-    for (int h = warp; h < grp; h += 4) {
+    // online softmax per head: warp h handles head h
+    for (int h = warp; h < GRP; h += 8) {
       const float s0 = S[h][lane], s1 = S[h][lane + 32];
       const float tmax = warp_max(fmaxf(s0, s1));
       const float mnew = fmaxf(m_run[h], tmax);
@@ -417,19 +485,42 @@ __global__ void __launch_bounds__(128) k_attn_decode(const AttnDecArgs a) {
       }
     }
     __syncthreads();
-    for (int h = hslot; h < grp; h += HS) {
-      float sacc = acc[h] * alpha[h];
-      for (int c = 0; c < nc; ++c) sacc += S[h][c] * bf16_to_f(Vs[c * RS + d]);
-      acc[h] = sacc;
+    // PV: this thread's dim pair over its column group, every head
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) {
+      acc[h][0] *= alpha[h];
+      acc[h][1] *= alpha[h];
+    }
+    for (int c = cq; c < kDecTile; c += CQ) {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(Vs + c * RS + 2 * dp);
+      const float v0 = __uint_as_float(u << 16), v1 = __uint_as_float(u & 0xFFFF0000u);
+#pragma unroll
+      for (int h = 0; h < GRP; ++h) {
+        const float p = S[h][c];
+        acc[h][0] += p * v0;
+        acc[h][1] += p * v1;
+      }
     }
     __syncthreads();
   }
-  // write this split's partial (m, l, unnormalised o)
+  // sum the column groups, then write this split's partial (m, l, unnormalised o)
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    red[cq][h][2 * dp] = acc[h][0];
+    red[cq][h][2 * dp + 1] = acc[h][1];
+  }
+  __syncthreads();
   const size_t pbase = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits + sp;
-  for (int h = hslot; h < grp; h += HS) a.part_o[(pbase * GMAX + h) * HD + d] = acc[h];
-  if (tid < grp) {
-    a.part_ml[(pbase * GMAX + tid) * 2 + 0] = m_run[tid];
-    a.part_ml[(pbase * GMAX + tid) * 2 + 1] = l_run[tid];
+  for (int e = tid; e < GRP * HD; e += 256) {
+    const int h = e / HD, d = e % HD;
+    float o = 0.f;
+#pragma unroll
+    for (int q = 0; q < CQ; ++q) o += red[q][h][d];
+    a.part_o[(pbase * 8 + h) * HD + d] = o;
+  }
+  if (tid < GRP) {
+    a.part_ml[(pbase * 8 + tid) * 2 + 0] = m_run[tid];
+    a.part_ml[(pbase * 8 + tid) * 2 + 1] = l_run[tid];
   }
   __threadfence();
   __syncthreads();
@@ -441,22 +532,38 @@ __global__ void __launch_bounds__(128) k_attn_decode(const AttnDecArgs a) {
   if (!is_last) return;
   __threadfence();
   const size_t q0 = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits;
-  for (int h = hslot; h < grp; h += HS) {
+  // merge: warp h finds head h's maximum and total over the splits (lanes over splits)
+  for (int h = warp; h < GRP; h += 8) {
     float M = -INFINITY;
-    for (int s = 0; s < a.n_splits; ++s) M = fmaxf(M, __ldcg(&a.part_ml[((q0 + s) * GMAX + h) * 2]));
-    float L = 0.f, o = 0.f;
-    for (int s = 0; s < a.n_splits; ++s) {
-      const float ms = __ldcg(&a.part_ml[((q0 + s) * GMAX + h) * 2]);
-      if (ms == -INFINITY) continue;
-      const float w = expf(ms - M);
-      L += w * __ldcg(&a.part_ml[((q0 + s) * GMAX + h) * 2 + 1]);
-      o += w * __ldcg(&a.part_o[((q0 + s) * GMAX + h) * HD + d]);
+    for (int s2 = lane; s2 < a.n_splits; s2 += 32) M = fmaxf(M, __ldcg(&a.part_ml[((q0 + s2) * 8 + h) * 2]));
+    M = warp_max(M);
+    float L = 0.f;
+    for (int s2 = lane; s2 < a.n_splits; s2 += 32) {
+      const float ms = __ldcg(&a.part_ml[((q0 + s2) * 8 + h) * 2]);
+      if (ms != -INFINITY) L += expf(ms - M) * __ldcg(&a.part_ml[((q0 + s2) * 8 + h) * 2 + 1]);
     }
-    const int hq = g * grp + h;
-    const float ov = o / L;
+    L = warp_sum(L);
+    if (lane == 0) {
+      sm_m[h] = M;
+      sm_l[h] = L;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < GRP * HD; e += 256) {
+    const int h = e / HD, d = e % HD;
+    const float M = sm_m[h];
+    float o = 0.f;
+#pragma unroll 8
+    for (int s2 = 0; s2 < a.n_splits; ++s2) {
+      const float ms = __ldcg(&a.part_ml[((q0 + s2) * 8 + h) * 2]);
+      const float po = __ldcg(&a.part_o[((q0 + s2) * 8 + h) * HD + d]);
+      o += ms == -INFINITY ? 0.f : expf(ms - M) * po;
+    }
+    const int hq = g * GRP + h;
+    const float ov = o / sm_l[h];
     if (a.o_state) a.o_state[(static_cast<size_t>(tok) * a.H + hq) * HD + d] = ov;
     a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + d] = f_to_bf16(ov);
-    if (d == 0 && a.lse_state) a.lse_state[static_cast<size_t>(tok) * a.H + hq] = M + logf(L);
+    if (d == 0 && a.lse_state) a.lse_state[static_cast<size_t>(tok) * a.H + hq] = M + logf(sm_l[h]);
   }
   if (tid == 0) a.counters[i * a.Hkv + g] = 0;
 }
@@ -468,6 +575,8 @@ __global__ void __launch_bounds__(128) k_attn_decode(const AttnDecArgs a) {
 // ============================================================================
 template <int HD>
 __global__ void __launch_bounds__(256) k_attn_prefill(const AttnPreArgs a) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int BQ = 64, BK = 64;
   constexpr int RS = HD + kDecPad;
   constexpr int DV = HD / 4;
@@ -578,6 +687,8 @@ __global__ void __launch_bounds__(256) k_attn_prefill(const AttnPreArgs a) {
 __global__ void k_setup_call(int N, int mode_decode, int T, int tiles_per_seq, int q_tile,
                              const int* __restrict__ seq_len, int* seq, int* pos, int* tile, int* last,
                              int n_tiles, int* has_c) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t < N) {
     if (mode_decode) {
@@ -596,11 +707,15 @@ __global__ void k_setup_call(int N, int mode_decode, int T, int tiles_per_seq, i
 }
 
 __global__ void k_set_lens(int B, int* seq_len, int add, int value) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) seq_len[b] = add ? seq_len[b] + 1 : value;
 }
 
 __global__ void k_reset_lens(const LensArg a, int* seq_len) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < a.n) seq_len[b] = a.v[b];
 }
@@ -608,6 +723,8 @@ __global__ void k_reset_lens(const LensArg a, int* seq_len) {
 // slot of each token in the selection (or -1), and the snapshot of selected rows
 __global__ void k_after_select(const int32_t* __restrict__ idx, int n_sel, int N, int d, int* sel_slot,
                                const float* __restrict__ h, float* __restrict__ h_snap, int slot_blocks) {
+  pdl_trigger();
+  pdl_wait();
   if (static_cast<int>(blockIdx.x) < slot_blocks) {
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= N) return;
@@ -634,6 +751,8 @@ __global__ void __launch_bounds__(128) k_change_keys(const float* __restrict__ h
                                                      const int* __restrict__ sel_slot, int N, int d, int loop,
                                                      float* __restrict__ key, int* last, const int* tile,
                                                      int* has_c) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (t >= N) return;
   const float* other;
@@ -672,6 +791,8 @@ __global__ void __launch_bounds__(128) k_change_keys(const float* __restrict__ h
 __global__ void __launch_bounds__(1024) k_plan_tiles(const int32_t* __restrict__ idx, int n_sel,
                                                      const int* __restrict__ tile, const int* __restrict__ has_c,
                                                      TilePlan plan) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int scan_buf[33];
   __shared__ int base_p, base_need;
   if (threadIdx.x == 0) {
@@ -719,6 +840,8 @@ __global__ void __launch_bounds__(1024) k_plan_tiles(const int32_t* __restrict__
 // ============================================================================
 template <int HD, int EPL>
 __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int CC = 64;      // columns per CTA
   constexpr int QP = 16;      // (query, head) pairs staged per batch
   extern __shared__ __align__(16) uint8_t sm[];
@@ -791,6 +914,8 @@ __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
 
 // top-c columns of each (tile, KV head) that needs a column set
 __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
+  pdl_trigger();
+  pdl_wait();
   const int seg = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
   if (seg >= a.plan.counts[1]) return;
   const int p = a.plan.need[seg];
@@ -825,6 +950,8 @@ __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
 // ============================================================================
 template <int HD, int EPL, int GRP>
 __global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
+  pdl_trigger();
+  pdl_wait();
   constexpr int GMAX = 8, NW = 8;
   __shared__ float sm_m[NW][GMAX], sm_z[NW][GMAX];
   __shared__ float sm_acc[NW][GMAX][HD];
@@ -933,21 +1060,39 @@ __global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
   if (!is_last) return;
   __threadfence();
   const size_t q0 = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits;
+  // merge: warp h finds head h's common maximum and denominator (lanes over splits)
+  __shared__ float mg[GMAX], zg[GMAX], eg[GMAX];
+  for (int h = warp; h < grp; h += NW) {
+    const size_t so = static_cast<size_t>(tok) * a.H + g * grp + h;
+    const float L = a.lse_state[so];
+    float M = L;
+    for (int s2 = lane; s2 < a.n_splits; s2 += 32) M = fmaxf(M, __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2]));
+    M = warp_max(M);
+    float Z = 0.f;
+    for (int s2 = lane; s2 < a.n_splits; s2 += 32) {
+      const float ms = __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2]);
+      if (ms != -INFINITY) Z += expf(ms - M) * __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2 + 1]);
+    }
+    Z = warp_sum(Z);
+    if (lane == 0) {
+      const float el = expf(L - M);
+      mg[h] = M;
+      eg[h] = el;
+      zg[h] = el + Z;
+    }
+  }
+  __syncthreads();
   for (int e = tid; e < grp * HD; e += 256) {
     const int h = e / HD, dd = e % HD;
     const int hq = g * grp + h;
     const size_t so = static_cast<size_t>(tok) * a.H + hq;
-    const float L = a.lse_state[so];
-    float M = L;
-    for (int s2 = 0; s2 < a.n_splits; ++s2) M = fmaxf(M, __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2]));
-    const float el = expf(L - M);
-    float Z = el, N = el * a.o_state[so * HD + dd];
+    const float M = mg[h], Z = zg[h];
+    float N = eg[h] * a.o_state[so * HD + dd];
+#pragma unroll 8
     for (int s2 = 0; s2 < a.n_splits; ++s2) {
       const float ms = __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2]);
-      if (ms == -INFINITY) continue;
-      const float f = expf(ms - M);
-      Z += f * __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2 + 1]);
-      N += f * __ldcg(&a.part_acc[((q0 + s2) * GMAX + h) * HD + dd]);
+      const float pa = __ldcg(&a.part_acc[((q0 + s2) * GMAX + h) * HD + dd]);
+      N += ms == -INFINITY ? 0.f : expf(ms - M) * pa;
     }
     if (!(Z > 0.f) && a.status) atomicOr(a.status, kErrBadIndex);
     const float ov = N / Z;
@@ -965,6 +1110,8 @@ __global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
 template <int EPL>
 __global__ void k_pack_codes(const int8_t* __restrict__ src, int rows, int hd, int bits, uint8_t* __restrict__ dst,
                              size_t dst_row_stride) {
+  pdl_trigger();
+  pdl_wait();
   const int w = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (w >= rows) return;
   int c[EPL];
@@ -976,42 +1123,53 @@ __global__ void k_pack_codes(const int8_t* __restrict__ src, int rows, int hd, i
 // ============================================================================
 // launchers
 // ============================================================================
+thread_local bool g_pdl = false;
+void set_pdl(bool on) { g_pdl = on; }
+
 cudaError_t launch_topk(const float* keys, int n_seg, int n, int k, int32_t* idx, cudaStream_t s) {
-  k_topk_segments<<<n_seg, 1024, 0, s>>>(keys, n, k, idx);
-  return cudaGetLastError();
+  return launch_k(false, k_topk_segments, dim3(n_seg), dim3(1024), 0, s, keys, n, k, idx);
 }
 cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* idx, const int* forced_on,
                                  const int32_t* forced, cudaStream_t s) {
-  k_select_tokens<<<1, 1024, 0, s>>>(keys, N, n_sel, idx, forced_on, forced);
-  return cudaGetLastError();
+  return launch_k(g_pdl, k_select_tokens, dim3(1), dim3(1024), 0, s, keys, N, n_sel, idx, forced_on, forced);
 }
 cudaError_t launch_quantize_rows(const float* r, int rows, int width, int g, int bits, uint8_t* codes,
                                  uint16_t* scales, cudaStream_t s) {
   if (width % 128 == 0) {
     const int warps = rows * (width / 128);
-    k_quantize_rows<4><<<(warps + 3) / 4, 128, 0, s>>>(r, rows, width, g, bits, codes, scales);
-  } else {
-    const int warps = rows * (width / 64);
-    k_quantize_rows<2><<<(warps + 3) / 4, 128, 0, s>>>(r, rows, width, g, bits, codes, scales);
+    return launch_k(false, k_quantize_rows<4>, dim3((warps + 3) / 4), dim3(128), 0, s, r, rows, width, g, bits,
+                    codes, scales);
   }
-  return cudaGetLastError();
+  const int warps = rows * (width / 64);
+  return launch_k(false, k_quantize_rows<2>, dim3((warps + 3) / 4), dim3(128), 0, s, r, rows, width, g, bits, codes,
+                  scales);
 }
 cudaError_t launch_rmsnorm_rows(const float* h, const int* idx, int n, int n_pad, int d, const float* gain, float eps,
                                 uint16_t* x, cudaStream_t s) {
-  k_rmsnorm_rows<<<n_pad, 256, 0, s>>>(h, idx, n, d, gain, eps, x);
-  return cudaGetLastError();
+  return launch_k(g_pdl, k_rmsnorm_rows, dim3(n_pad), dim3(256), 0, s, h, idx, n, d, gain, eps, x);
 }
 cudaError_t launch_qkv_post(const QkvPostArgs& a, cudaStream_t s) {
   const int warps = a.n * (a.H + 2 * a.Hkv);
-  if (a.hd == 128) k_qkv_post<4><<<(warps + 3) / 4, 128, 0, s>>>(a);
-  else k_qkv_post<2><<<(warps + 3) / 4, 128, 0, s>>>(a);
-  return cudaGetLastError();
+  if (a.hd == 128) return launch_k(g_pdl, k_qkv_post<4>, dim3((warps + 3) / 4), dim3(128), 0, s, a);
+  return launch_k(g_pdl, k_qkv_post<2>, dim3((warps + 3) / 4), dim3(128), 0, s, a);
 }
+size_t attn_decode_smem(int hd) { return static_cast<size_t>(2) * 2 * kDecTile * (hd + kDecPad) * 2; }
 cudaError_t launch_attn_decode(const AttnDecArgs& a, int n, cudaStream_t s) {
   dim3 grid(n * a.Hkv, a.n_splits);
-  if (a.hd == 128) k_attn_decode<128><<<grid, 128, 0, s>>>(a);
-  else k_attn_decode<64><<<grid, 128, 0, s>>>(a);
-  return cudaGetLastError();
+  const size_t sm = attn_decode_smem(a.hd);
+  const int grp = a.H / a.Hkv;
+#define FL_ATT(G)                                                                           \
+  case G:                                                                                   \
+    return a.hd == 128 ? launch_k(g_pdl, k_attn_decode<128, G>, grid, dim3(256), sm, s, a)  \
+                       : launch_k(g_pdl, k_attn_decode<64, G>, grid, dim3(256), sm, s, a);
+  switch (grp) {
+    FL_ATT(1)
+    FL_ATT(2)
+    FL_ATT(4)
+    FL_ATT(8)
+    default: return cudaErrorInvalidValue;
+  }
+#undef FL_ATT
 }
 size_t attn_prefill_smem(int hd) {
   return static_cast<size_t>(64) * (hd + 1) * 4 + 64 * 65 * 4 + 2 * 64 * (hd + kDecPad) * 2;
@@ -1019,43 +1177,35 @@ size_t attn_prefill_smem(int hd) {
 cudaError_t launch_attn_prefill(const AttnPreArgs& a, int B, cudaStream_t s) {
   dim3 grid((a.T + 63) / 64, a.H, B);
   const size_t sm = attn_prefill_smem(a.hd);
-  if (a.hd == 128) {
-    k_attn_prefill<128><<<grid, 256, sm, s>>>(a);
-  } else {
-    k_attn_prefill<64><<<grid, 256, sm, s>>>(a);
-  }
-  return cudaGetLastError();
+  if (a.hd == 128) return launch_k(g_pdl, k_attn_prefill<128>, grid, dim3(256), sm, s, a);
+  return launch_k(g_pdl, k_attn_prefill<64>, grid, dim3(256), sm, s, a);
 }
 cudaError_t launch_setup_call(int N, int decode, int T, int tiles_per_seq, int q_tile, const int* seq_len, int* seq,
                               int* pos, int* tile, int* last, int n_tiles, int* has_c, cudaStream_t s) {
   const int n = N > n_tiles ? N : n_tiles;
-  k_setup_call<<<(n + 255) / 256, 256, 0, s>>>(N, decode, T, tiles_per_seq, q_tile, seq_len, seq, pos, tile, last,
-                                               n_tiles, has_c);
-  return cudaGetLastError();
+  return launch_k(g_pdl, k_setup_call, dim3((n + 255) / 256), dim3(256), 0, s, N, decode, T, tiles_per_seq, q_tile,
+                  seq_len, seq, pos, tile, last, n_tiles, has_c);
 }
 cudaError_t launch_set_lens(int B, int* seq_len, int add, int value, cudaStream_t s) {
-  k_set_lens<<<(B + 127) / 128, 128, 0, s>>>(B, seq_len, add, value);
-  return cudaGetLastError();
+  return launch_k(g_pdl, k_set_lens, dim3((B + 127) / 128), dim3(128), 0, s, B, seq_len, add, value);
 }
 cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s) {
-  k_reset_lens<<<1, kLensByValue, 0, s>>>(a, seq_len);
-  return cudaGetLastError();
+  return launch_k(false, k_reset_lens, dim3(1), dim3(kLensByValue), 0, s, a, seq_len);
 }
 cudaError_t launch_after_select(const int32_t* idx, int n_sel, int N, int d, int* sel_slot, const float* h,
                                 float* h_snap, cudaStream_t s) {
   const int slot_blocks = (N + 255) / 256;
-  k_after_select<<<slot_blocks + n_sel, 256, 0, s>>>(idx, n_sel, N, d, sel_slot, h, h_snap, slot_blocks);
-  return cudaGetLastError();
+  return launch_k(g_pdl, k_after_select, dim3(slot_blocks + n_sel), dim3(256), 0, s, idx, n_sel, N, d, sel_slot, h,
+                  h_snap, slot_blocks);
 }
 cudaError_t launch_change_keys(const float* h, const float* ref, const int* sel_slot, int N, int d, int loop,
                                float* key, int* last, const int* tile, int* has_c, cudaStream_t s) {
-  k_change_keys<<<(N + 3) / 4, 128, 0, s>>>(h, ref, sel_slot, N, d, loop, key, last, tile, has_c);
-  return cudaGetLastError();
+  return launch_k(g_pdl, k_change_keys, dim3((N + 3) / 4), dim3(128), 0, s, h, ref, sel_slot, N, d, loop, key, last,
+                  tile, has_c);
 }
 cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, const int* has_c, const TilePlan& p,
                               cudaStream_t s) {
-  k_plan_tiles<<<1, 1024, 0, s>>>(idx, n_sel, tile, has_c, p);
-  return cudaGetLastError();
+  return launch_k(g_pdl, k_plan_tiles, dim3(1), dim3(1024), 0, s, idx, n_sel, tile, has_c, p);
 }
 size_t dscore_smem(int hd) {
   return (static_cast<size_t>(2) * 64 * (hd + 1) + 2 * 16 * hd + 4 * 64) * 4;
@@ -1063,25 +1213,19 @@ size_t dscore_smem(int hd) {
 cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s) {
   dim3 grid(max_need * a.Hkv, max_chunks);
   const size_t sm = dscore_smem(a.hd);
-  if (a.hd == 128) {
-    k_dscore<128, 4><<<grid, 256, sm, s>>>(a);
-  } else {
-    k_dscore<64, 2><<<grid, 256, sm, s>>>(a);
-  }
-  return cudaGetLastError();
+  if (a.hd == 128) return launch_k(g_pdl, k_dscore<128, 4>, grid, dim3(256), sm, s, a);
+  return launch_k(g_pdl, k_dscore<64, 2>, grid, dim3(256), sm, s, a);
 }
 cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t s) {
-  k_select_cols<<<max_need * a.Hkv, 1024, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(g_pdl, k_select_cols, dim3(max_need * a.Hkv), dim3(1024), 0, s, a);
 }
 cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
   dim3 grid(n_sel * a.Hkv, a.n_splits);
   const int grp = a.H / a.Hkv;
-#define FL_CORR(G)                                                   \
-  case G:                                                            \
-    if (a.hd == 128) k_correct<128, 4, G><<<grid, 256, 0, s>>>(a);   \
-    else k_correct<64, 2, G><<<grid, 256, 0, s>>>(a);                \
-    break;
+#define FL_CORR(G)                                                                  \
+  case G:                                                                           \
+    return a.hd == 128 ? launch_k(g_pdl, k_correct<128, 4, G>, grid, dim3(256), 0, s, a) \
+                       : launch_k(g_pdl, k_correct<64, 2, G>, grid, dim3(256), 0, s, a);
   switch (grp) {
     FL_CORR(1)
     FL_CORR(2)
@@ -1090,7 +1234,6 @@ cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
     default: return cudaErrorInvalidValue;
   }
 #undef FL_CORR
-  return cudaGetLastError();
 }
 
 // Opt every large-shared-memory kernel in to its dynamic shared memory once,
@@ -1103,6 +1246,14 @@ cudaError_t kernels_init_attrs() {
     const cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess) e = r;
   };
+  set(k_attn_decode<128, 1>, static_cast<int>(attn_decode_smem(128)));
+  set(k_attn_decode<128, 2>, static_cast<int>(attn_decode_smem(128)));
+  set(k_attn_decode<128, 4>, static_cast<int>(attn_decode_smem(128)));
+  set(k_attn_decode<128, 8>, static_cast<int>(attn_decode_smem(128)));
+  set(k_attn_decode<64, 1>, static_cast<int>(attn_decode_smem(64)));
+  set(k_attn_decode<64, 2>, static_cast<int>(attn_decode_smem(64)));
+  set(k_attn_decode<64, 4>, static_cast<int>(attn_decode_smem(64)));
+  set(k_attn_decode<64, 8>, static_cast<int>(attn_decode_smem(64)));
   set(k_attn_prefill<128>, static_cast<int>(attn_prefill_smem(128)));
   set(k_attn_prefill<64>, static_cast<int>(attn_prefill_smem(64)));
   set(k_dscore<128, 4>, static_cast<int>(dscore_smem(128)));
@@ -1113,9 +1264,11 @@ cudaError_t kernels_init_attrs() {
 
 cudaError_t launch_pack_codes(const int8_t* src, int rows, int hd, int bits, uint8_t* dst, size_t dst_row_stride,
                               cudaStream_t s) {
-  if (hd == 128) k_pack_codes<4><<<(rows + 3) / 4, 128, 0, s>>>(src, rows, hd, bits, dst, dst_row_stride);
-  else k_pack_codes<2><<<(rows + 3) / 4, 128, 0, s>>>(src, rows, hd, bits, dst, dst_row_stride);
-  return cudaGetLastError();
+  if (hd == 128)
+    return launch_k(false, k_pack_codes<4>, dim3((rows + 3) / 4), dim3(128), 0, s, src, rows, hd, bits, dst,
+                    dst_row_stride);
+  return launch_k(false, k_pack_codes<2>, dim3((rows + 3) / 4), dim3(128), 0, s, src, rows, hd, bits, dst,
+                  dst_row_stride);
 }
 
 }  // namespace fl

@@ -120,6 +120,9 @@ struct LensArg {
   int v[kLensByValue];
 };
 cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s);
+// Launches made while this is on (the kernels of one call) are programmatic
+// dependents of the previous kernel; thread-local.
+void set_pdl(bool on);
 
 cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* idx, const int* forced_on,
                                  const int32_t* forced, cudaStream_t s);

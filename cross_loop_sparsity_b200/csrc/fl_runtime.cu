@@ -74,6 +74,7 @@ struct flashloop_ctx {
   std::vector<cudaGraphExec_t> graph_exec;
   std::vector<int> eager_seen;
   int use_graph = 1;
+  int pdl = 1;                        // FL_OPT_PDL
   int prof = 0;                       // FL_OPT_PROFILE
   std::vector<cudaEvent_t> ev;        // start/end pairs of the last profiled call
   std::vector<int> ev_kind;
@@ -385,11 +386,14 @@ fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, 
     g.bn = 128;
     g.grid = dim3(ceil_div(n, 128), ceil_div(feat, 128), 1);
   }
+  g.pdl = ctx->pdl;
   FL_TRY(launch_gemm(g, s));
   return FL_OK;
 }
 
 __global__ void k_fill_last_rows(int B, int T, int32_t* rows) {
+  pdl_trigger();
+  pdl_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < B) rows[b] = b * T + T - 1;
 }
@@ -448,9 +452,21 @@ cudaError_t prof_end(flashloop_ctx* ctx, cudaStream_t s) {
     if (st_ != FL_OK) return st_;     \
   } while (0)
 
+fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s);
+
 // The whole looped block over one call's tokens, enqueued on s.  The input
-// hidden states are in h_in; the result is left in h and logits_ws.
+// hidden states are in h_in; the result is left in h and logits_ws.  Kernels
+// of the call are launched as programmatic dependents of their predecessor
+// (when the option is on) so each one's launch and set-up overlap the
+// previous kernel.
 fl_status run_call(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s) {
+  set_pdl(ctx->pdl != 0);
+  const fl_status st = run_call_body(ctx, decode, B, T, s);
+  set_pdl(false);
+  return st;
+}
+
+fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s) {
   const flashloop_config& c = ctx->cfg;
   const int M = c.n_layers, K = c.n_loops, d = c.d_model, H = c.n_heads, Hkv = c.n_kv_heads, hd = c.head_dim;
   const bool lazy = ctx->lazy;
@@ -551,8 +567,8 @@ fl_status run_call(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s)
   // final norm + LM head on the output rows
   const int32_t* rows = ctx->idx_all;
   if (!decode) {
-    FL_LAUNCH(FL_KIND_OTHER, (k_fill_last_rows<<<ceil_div(B, 128), 128, 0, s>>>(B, T, ctx->idx_last),
-                              cudaGetLastError()));
+    FL_LAUNCH(FL_KIND_OTHER, launch_k(ctx->pdl, k_fill_last_rows, dim3(ceil_div(B, 128)), dim3(128), 0, s, B, T,
+                                      ctx->idx_last));
     rows = ctx->idx_last;
   }
   FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, rows, B, pad(B), d, ctx->w.final_norm, c.rms_eps, ctx->x, s));
@@ -698,6 +714,10 @@ fl_status flashloop_set_option(flashloop_ctx* ctx, fl_option opt, int value) {
     ctx->prof = value ? 1 : 0;
     return FL_OK;
   }
+  if (opt == FL_OPT_PDL) {
+    ctx->pdl = value ? 1 : 0;
+    return FL_OK;
+  }
   return FL_ERR_INVALID_ARG;
 }
 
@@ -734,7 +754,7 @@ fl_status flashloop_decode_step(flashloop_ctx* ctx, const float* h0, int B, floa
   FL_TRY(cudaMemcpyAsync(ctx->h_in, h0, static_cast<size_t>(B) * c.d_model * 4, cudaMemcpyDefault, s));
   // A decode step's launch sequence depends on B only; after one direct run it
   // is captured once into a CUDA graph and replayed (not on the legacy stream).
-  const int gkey = B * 2 + (ctx->prof ? 1 : 0);
+  const int gkey = B * 4 + (ctx->prof ? 1 : 0) + (ctx->pdl ? 2 : 0);
   size_t gi = 0;
   while (gi < ctx->graph_b.size() && ctx->graph_b[gi] != gkey) ++gi;
   bool seen = false;

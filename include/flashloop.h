@@ -244,7 +244,9 @@ fl_status fl_gemm_skinny_noalloc(const uint16_t* A, const uint16_t* B, float* D,
 /* Runtime options of a context. */
 typedef enum {
   FL_OPT_USE_GRAPH = 1, /* 1 (default): capture decode steps into CUDA graphs; 0: launch directly */
-  FL_OPT_PROFILE = 2    /* 1: bracket every kernel of a call with CUDA events (read with flashloop_profile) */
+  FL_OPT_PROFILE = 2,   /* 1: bracket every kernel of a call with CUDA events (read with flashloop_profile) */
+  FL_OPT_PDL = 3        /* 1 (default): launch each kernel of a call as a programmatic dependent of the
+                           previous one, so its launch and set-up overlap the predecessor */
 } fl_option;
 fl_status flashloop_set_option(flashloop_ctx* ctx, fl_option opt, int value);
 
