@@ -16,7 +16,6 @@ The `reference` arm times the CPU oracle on the host cores (rank 0 only).
 from __future__ import annotations
 
 import argparse
-import datetime
 import hashlib
 import json
 import math
@@ -149,34 +148,11 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-# ------------------------------------------------------------------ distributed plumbing
-def dist_setup(n_gpus):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import torch
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    return world, rank, local
+# ------------------------------------------------------------------ replicas (one per GPU)
+from cross_loop_sparsity_b200 import replicas  # noqa: E402
 
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-
-
-def max_over_ranks(world, v):
-    if world == 1:
-        return v
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+barrier = replicas.barrier
+max_over_ranks = replicas.max_over_ranks
 
 
 # ------------------------------------------------------------------ the library arm
@@ -296,7 +272,7 @@ def run_library(args, world, rank, local):
     if rank == 0 and world == 1 and not args.no_cpu:
         cpu = cpu_baseline(cfg, w, 1)
     out = {
-        "metric": METRIC, "value": world * B / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": replicas.job_throughput(world, B, ms_step), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": workload_desc(cfg), "global_batch": world * B, "ctx": cfg.ctx_len,
@@ -420,16 +396,14 @@ def run_reference(args, world, rank):
 
 def main():
     args = parse()
-    world, rank, local = dist_setup(args.gpus)
+    world, rank, local = replicas.init()
     try:
         if args.impl == "reference":
             run_reference(args, world, rank)
         else:
             run_library(args, world, rank, local)
     finally:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        replicas.finish(world)
 
 
 if __name__ == "__main__":

@@ -11,8 +11,12 @@
 // keeps two accumulators).  Split-K partials go to a scratch buffer and the
 // last CTA of a tile (an atomic ticket, no waiting) reduces them in split
 // order, so results do not depend on CTA timing.
+#include <cooperative_groups.h>
+
 #include "fl_device.cuh"
 #include "fl_internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace fl {
 
@@ -231,6 +235,21 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
         tc_wait_ld();
         if (valid) epi_apply<SWAP>(p, row, c, tile_m, tile_n, BN, v0, v1);
       }
+    } else if (p.cluster) {
+      // cluster split-K: park this split's partial tile in shared memory
+      // ([acc][col][row], the ring is free once every MMA has completed); the
+      // reduction runs after the cluster barrier below
+      float* red = reinterpret_cast<float*>(smem);
+      for (int c = 0; c < BN; c += 16) {
+        tmem_ld16(tbase + c, v0);
+        if (C::kNAcc == 2) tmem_ld16(tbase + BN + c, v1);
+        tc_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          red[(c + j) * 128 + row] = valid ? v0[j] : 0.f;
+          if (C::kNAcc == 2) red[(BN + c + j) * 128 + row] = valid ? v1[j] : 0.f;
+        }
+      }
     } else {
       // split-K: write this split's partial tile, take a ticket, the last CTA reduces.
       const size_t tile_floats = static_cast<size_t>(C::kNAcc) * BN * 128;
@@ -275,6 +294,40 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
       }
     }
   }
+  if (p.splits > 1 && p.cluster) {
+    // every split of this tile is a CTA of one cluster: rank r sums the
+    // partials of all ranks (in rank order) for its slice of token columns,
+    // reading them from the peers' shared memory, and applies the epilogue
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    if (warp >= 2) {
+      const int row = (warp & 3) * 32 + lane;
+      const int S = p.splits, r = static_cast<int>(cluster.block_rank());
+      const int per = (BN + S - 1) / S;
+      const int col0 = r * per, col1 = min(BN, col0 + per);
+      float* red = reinterpret_cast<float*>(smem);
+      for (int c = col0; c < col1; c += 16) {
+        float a0[16], a1[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) a0[j] = a1[j] = 0.f;
+        for (int q = 0; q < S; ++q) {
+          const float* peer = cluster.map_shared_rank(red, q);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (c + j < col1) {
+              a0[j] += peer[(c + j) * 128 + row];
+              if (C::kNAcc == 2) a1[j] += peer[(BN + c + j) * 128 + row];
+            }
+          }
+        }
+        // columns past col1 belong to the next rank: mark them out of range
+        GemmArgs pc = p;
+        pc.n_tok = min(p.n_tok, col1);
+        epi_apply<SWAP>(pc, row, c, tile_m, tile_n, BN, a0, a1);
+      }
+    }
+    cluster.sync();
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -290,6 +343,23 @@ cudaError_t launch_one(const GemmLaunch& g, cudaStream_t stream) {
   auto kern = k_gemm_tc<BN, DA, DB, SWAP>;
   const CUtensorMap& a1 = g.a1 ? *g.a1 : *g.a0;
   const CUtensorMap& b1 = g.b1 ? *g.b1 : *g.b0;
+  if (g.args.cluster && g.args.splits > 1) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = g.grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = g.args.splits;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = g.pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, *g.a0, a1, *g.b0, b1, g.args, g.a_3d, g.b_3d);
+  }
   return launch_k(g.pdl, kern, g.grid, dim3(kThreads), C::kSmemBytes, stream, *g.a0, a1, *g.b0, b1, g.args,
                   g.a_3d, g.b_3d);
 }

@@ -36,8 +36,10 @@ struct GemmArgs {
   int ldh;
   uint16_t* act;
   int ld_act;
-  float* partial;   // split-K scratch: splits * grid.x * NACC * BN * 128 fp32
-  int* counters;    // one per grid.x tile; zero between launches
+  float* partial;   // split-K scratch: splits * grid.x * NACC * BN * 128 fp32 (ticket path)
+  int* counters;    // one per grid.x tile; zero between launches (ticket path)
+  int cluster;      // split-K through a (1,1,splits) cluster and distributed shared memory
+                    // instead of global partials and tickets (splits <= kMaxClusterSplits)
   int* status;
 };
 
@@ -53,6 +55,7 @@ struct GemmLaunch {
   bool pdl = false;        // launched as a programmatic dependent of the previous kernel
 };
 
+constexpr int kMaxClusterSplits = 8;  // portable cluster size
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream);
 
 // Launch a kernel, with programmatic stream serialisation when `pdl` is set

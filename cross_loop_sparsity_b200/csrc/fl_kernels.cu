@@ -380,8 +380,8 @@ __global__ void __launch_bounds__(256) k_attn_decode(const AttnDecArgs a) {
   extern __shared__ __align__(16) uint8_t sm[];
   uint16_t* Kst = reinterpret_cast<uint16_t*>(sm);          // [2][64][RS]
   uint16_t* Vst = Kst + 2 * kDecTile * RS;                  // [2][64][RS]
-  __shared__ float Qs[GRP * HD];
-  __shared__ float S[GRP][kDecTile];
+  __shared__ __align__(16) float Qs[GRP * HD];
+  __shared__ __align__(16) float S[kDecTile][GRP];   // column-major: one vector load gives every head
   __shared__ float m_run[GRP], l_run[GRP], alpha[GRP];
   __shared__ float red[CQ][GRP][HD];
   __shared__ float sm_m[GRP], sm_l[GRP];
@@ -436,10 +436,11 @@ __global__ void __launch_bounds__(256) k_attn_decode(const AttnDecArgs a) {
     __syncthreads();
     const uint16_t* Ks = Kst + buf * kDecTile * RS;
     const uint16_t* Vs = Vst + buf * kDecTile * RS;
-    // scores: thread -> column c = tid / 4, dim quarter tid % 4, every head; the
-    // four quarters are summed by shuffles (they are adjacent lanes)
+    // scores: lane -> column warp*8 + lane%8, dim quarter lane/8, every head.  A
+    // quarter-warp reads eight consecutive staged rows (distinct banks) and one
+    // broadcast q chunk; the four quarters are summed by shuffles.
     {
-      const int c = tid >> 2, qd = tid & 3;
+      const int c = warp * 8 + (lane & 7), qd = lane >> 3;
       float dot[GRP];
 #pragma unroll
       for (int h = 0; h < GRP; ++h) dot[h] = 0.f;
@@ -453,29 +454,30 @@ __global__ void __launch_bounds__(256) k_attn_decode(const AttnDecArgs a) {
         const float k6 = __uint_as_float(u.w << 16), k7 = __uint_as_float(u.w & 0xFFFF0000u);
 #pragma unroll
         for (int h = 0; h < GRP; ++h) {
-          const float* q = &Qs[h * HD + qd * DQ + e];
-          dot[h] += q[0] * k0 + q[1] * k1 + q[2] * k2 + q[3] * k3 + q[4] * k4 + q[5] * k5 + q[6] * k6 + q[7] * k7;
+          const float4 qa = *reinterpret_cast<const float4*>(&Qs[h * HD + qd * DQ + e]);
+          const float4 qb = *reinterpret_cast<const float4*>(&Qs[h * HD + qd * DQ + e + 4]);
+          dot[h] += qa.x * k0 + qa.y * k1 + qa.z * k2 + qa.w * k3 + qb.x * k4 + qb.y * k5 + qb.z * k6 + qb.w * k7;
         }
       }
 #pragma unroll
       for (int h = 0; h < GRP; ++h) {
         float v = dot[h];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        if (qd == 0) S[h][c] = c < nc ? v * a.tau : -INFINITY;
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        if (qd == 0) S[c][h] = c < nc ? v * a.tau : -INFINITY;
       }
     }
     __syncthreads();
     // online softmax per head: warp h handles head h
     for (int h = warp; h < GRP; h += 8) {
-      const float s0 = S[h][lane], s1 = S[h][lane + 32];
+      const float s0 = S[lane][h], s1 = S[lane + 32][h];
       const float tmax = warp_max(fmaxf(s0, s1));
       const float mnew = fmaxf(m_run[h], tmax);
       const float p0 = s0 == -INFINITY ? 0.f : expf(s0 - mnew);
       const float p1 = s1 == -INFINITY ? 0.f : expf(s1 - mnew);
       const float psum = warp_sum(p0 + p1);
-      S[h][lane] = p0;
-      S[h][lane + 32] = p1;
+      S[lane][h] = p0;
+      S[lane + 32][h] = p1;
       __syncwarp();
       if (lane == 0) {
         const float al = m_run[h] == -INFINITY ? 0.f : expf(m_run[h] - mnew);
@@ -494,11 +496,21 @@ __global__ void __launch_bounds__(256) k_attn_decode(const AttnDecArgs a) {
     for (int c = cq; c < kDecTile; c += CQ) {
       const uint32_t u = *reinterpret_cast<const uint32_t*>(Vs + c * RS + 2 * dp);
       const float v0 = __uint_as_float(u << 16), v1 = __uint_as_float(u & 0xFFFF0000u);
+      float p[GRP];
+      if (GRP % 4 == 0) {
+#pragma unroll
+        for (int h = 0; h < GRP; h += 4) {
+          const float4 q4 = *reinterpret_cast<const float4*>(&S[c][h]);
+          p[h] = q4.x; p[(h + 1) % GRP] = q4.y; p[(h + 2) % GRP] = q4.z; p[(h + 3) % GRP] = q4.w;
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) p[h] = S[c][h];
+      }
 #pragma unroll
       for (int h = 0; h < GRP; ++h) {
-        const float p = S[h][c];
-        acc[h][0] += p * v0;
-        acc[h][1] += p * v1;
+        acc[h][0] += p[h] * v0;
+        acc[h][1] += p[h] * v1;
       }
     }
     __syncthreads();
@@ -965,15 +977,15 @@ __global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
   const CacheView& cv = a.cv;
   const size_t cset = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
   const int32_t* C = a.cols + cset * a.c;
-  if (tid == 0) {
-    // C is ascending: the query's columns are its prefix with C[k] <= pos
-    int lo = 0, hi = a.ncols[cset];
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (C[mid] <= P) lo = mid + 1; else hi = mid;
-    }
-    ncs = lo;
-  }
+  // C is ascending: the query's columns are its prefix with C[k] <= pos; only
+  // this CTA's slice of C is needed, so count within the slice in parallel
+  const int ncol_all = a.ncols[cset];
+  const int k0s = sp * a.cols_per_cta;
+  const int kend = min(ncol_all, k0s + a.cols_per_cta);
+  const int kk = k0s + tid;
+  const int in_slice = (kk < kend && C[kk] <= P) ? 1 : 0;
+  const int cnt = __syncthreads_count(in_slice);
+  if (tid == 0) ncs = k0s + cnt;
   // the group's query heads (new and last) in registers
   float qn[GRP][EPL], qo[GRP][EPL];
 #pragma unroll
@@ -986,8 +998,7 @@ __global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
     }
   }
   __syncthreads();
-  const int nc = ncs;
-  const int k0 = sp * a.cols_per_cta, k1 = min(nc, k0 + a.cols_per_cta);
+  const int k0 = k0s, k1 = ncs;
   float m[GRP], z[GRP], acc[GRP][EPL];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {

@@ -370,7 +370,9 @@ fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, 
     const int bn = swap_bn(n);
     const int bi = bn == 16 ? 0 : bn == 32 ? 1 : 2;
     const int tiles = ceil_div(feat, 128);
-    const int splits = split_factor(tiles, a.k_chunks);
+    int splits = split_factor(tiles, a.k_chunks);
+    if (splits > kMaxClusterSplits) splits = kMaxClusterSplits;   // splits of a tile form one cluster
+    a.cluster = 1;
     if (gemm_partial_floats(bn, w1 != nullptr, tiles, splits) > ctx->gemm_partial_cap || tiles > kCountersGemm)
       return FL_ERR_CAPACITY;
     g.a0 = w0; g.a1 = w1; g.b0 = &xb[bi]; g.b1 = nullptr;
