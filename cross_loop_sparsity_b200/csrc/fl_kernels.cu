@@ -3,8 +3,12 @@
 // decode and prefill attention, delta-score column keys, sparse-column
 // correction, and the per-token change keys.  Method: "FlashLoop: Fast and
 // Memory-Efficient Looped Transformers via Lazy Updates" (abstract).
+#include <cooperative_groups.h>
+
 #include "fl_cache.cuh"
 #include "fl_kernels.h"
+
+namespace cg = cooperative_groups;
 
 namespace fl {
 
@@ -800,11 +804,8 @@ __global__ void __launch_bounds__(128) k_change_keys(const float* __restrict__ h
 // query-tile plan of a lazy loop: the selected tokens (ascending) grouped by
 // query tile; tiles recomputed for the first time need a column set.
 // ============================================================================
-__global__ void __launch_bounds__(1024) k_plan_tiles(const int32_t* __restrict__ idx, int n_sel,
-                                                     const int* __restrict__ tile, const int* __restrict__ has_c,
-                                                     TilePlan plan) {
-  pdl_trigger();
-  pdl_wait();
+__device__ void block_plan(const int32_t* __restrict__ idx, int n_sel, const int* __restrict__ tile,
+                           const int* __restrict__ has_c, const TilePlan& plan) {
   __shared__ int scan_buf[33];
   __shared__ int base_p, base_need;
   if (threadIdx.x == 0) {
@@ -841,6 +842,79 @@ __global__ void __launch_bounds__(1024) k_plan_tiles(const int32_t* __restrict__
     plan.counts[0] = base_p;
     plan.counts[1] = base_need;
   }
+}
+
+__global__ void __launch_bounds__(1024) k_plan_tiles(const int32_t* __restrict__ idx, int n_sel,
+                                                     const int* __restrict__ tile, const int* __restrict__ has_c,
+                                                     TilePlan plan) {
+  pdl_trigger();
+  pdl_wait();
+  block_plan(idx, n_sel, tile, has_c, plan);
+}
+
+// One lazy loop's token bookkeeping for a call of at most blockDim.x tokens
+// (decode), in one CTA: the change keys of the previous loop (against h_in
+// after loop 1, against the selected rows' snapshot after a lazy loop, zero for
+// carried tokens), the previously selected tokens' `last` and tile flags, the
+// top-n_sel selection (or the forced one), the selection slots, the snapshot
+// of the selected rows and the query-tile plan.
+__global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int t = warp; t < a.N; t += nw) {
+    const float* other = nullptr;
+    int slot = -1;
+    if (a.loop == 2) {
+      other = a.h_in + static_cast<size_t>(t) * a.d;
+    } else {
+      slot = a.sel_slot[t];
+      if (slot >= 0) other = a.h_snap + static_cast<size_t>(slot) * a.d;
+    }
+    float acc = 0.f;
+    if (other) {
+      const float* hr = a.h + static_cast<size_t>(t) * a.d;
+      for (int c = lane * 4; c < a.d; c += 128) {
+        const float4 x = *reinterpret_cast<const float4*>(hr + c);
+        const float4 y = *reinterpret_cast<const float4*>(other + c);
+        const float a0 = x.x - y.x, a1 = x.y - y.y, a2 = x.z - y.z, a3 = x.w - y.w;
+        acc += a0 * a0 + a1 * a1 + a2 * a2 + a3 * a3;
+      }
+      acc = warp_sum(acc);
+    }
+    if (lane == 0) {
+      a.key[t] = acc;
+      a.keys_trace[t] = acc;
+      if (slot >= 0) {
+        a.last[t] = a.loop - 1;
+        a.has_c[a.tile[t]] = 1;
+      }
+    }
+  }
+  __syncthreads();
+  if (a.forced_on && a.forced_on[0]) {
+    for (int i = threadIdx.x; i < a.n_sel; i += blockDim.x) a.idx[i] = a.forced[i];
+    __syncthreads();
+  } else {
+    block_topk(a.key, a.N, a.n_sel, a.idx);
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < a.N; t += blockDim.x) {
+    int lo = 0, hi = a.n_sel;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (a.idx[mid] < t) lo = mid + 1; else hi = mid;
+    }
+    a.sel_slot[t] = (lo < a.n_sel && a.idx[lo] == t) ? lo : -1;
+  }
+  for (int r = warp; r < a.n_sel; r += nw) {
+    const float* src = a.h + static_cast<size_t>(a.idx[r]) * a.d;
+    float* dst = a.h_snap + static_cast<size_t>(r) * a.d;
+    for (int c = lane * 4; c < a.d; c += 128)
+      *reinterpret_cast<float4*>(dst + c) = *reinterpret_cast<const float4*>(src + c);
+  }
+  __syncthreads();
+  block_plan(a.idx, a.n_sel, a.tile, a.has_c, a.plan);
 }
 
 // ============================================================================
@@ -1116,6 +1190,148 @@ __global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
 }
 
 // ============================================================================
+// The same correction for few selected queries (decode): the column slices of
+// one (query, KV group) are the CTAs of one cluster.  Each CTA leaves its
+// piece (per-head max, denominator, numerator) in shared memory; after the
+// cluster barrier rank 0 merges the pieces of every rank, in rank order, over
+// distributed shared memory, together with the stored (O, lse) term.  No
+// global scratch, fence or ticket.  grid (kCorrCluster, n_sel * Hkv).
+// ============================================================================
+template <int HD, int EPL, int GRP>
+__global__ void __launch_bounds__(256) k_correct_cluster(const CorrectArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int NW = 8;
+  __shared__ float sm_m[NW][GRP], sm_z[NW][GRP];
+  __shared__ float sm_acc[NW][GRP][HD];
+  __shared__ float pm[GRP], pz[GRP];
+  __shared__ float pacc[GRP][HD];
+  __shared__ int nvalid_sh;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rank = static_cast<int>(cluster.block_rank()), CS = static_cast<int>(cluster.num_blocks());
+  const int i = blockIdx.y / a.Hkv, g = blockIdx.y % a.Hkv;
+  const int tok = a.idx[i];
+  const int b = a.seq[tok], P = a.pos[tok], tl = a.tile[tok];
+  const int m_old = a.last[tok];
+  const CacheView& cv = a.cv;
+  const size_t cset = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
+  const int32_t* C = a.cols + cset * a.c;
+  // the query's columns: the prefix of the ascending set C with C[k] <= pos
+  const int ncol_all = a.ncols[cset];
+  int nv = 0;
+  for (int base = 0; base < ncol_all; base += 256) {
+    const int k = base + tid;
+    nv += __syncthreads_count(k < ncol_all && C[k] <= P);
+  }
+  if (tid == 0) nvalid_sh = nv;
+  float qn[GRP][EPL], qo[GRP][EPL];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    const size_t hq = static_cast<size_t>(g * GRP + h);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      qn[h][e] = a.q_cur[(static_cast<size_t>(i) * a.H + hq) * HD + lane * EPL + e];
+      qo[h][e] = a.q_last[(static_cast<size_t>(tok) * a.H + hq) * HD + lane * EPL + e];
+    }
+  }
+  __syncthreads();
+  const int nvalid = nvalid_sh;
+  const int per = (nvalid + CS - 1) / CS;
+  const int k0 = rank * per, k1 = min(nvalid, k0 + per);
+  float m[GRP], z[GRP], acc[GRP][EPL];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    m[h] = -INFINITY;
+    z[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
+  }
+  for (int k = k0 + warp; k < k1; k += NW) {
+    const int col = C[k];
+    float klo[EPL], khi[EPL], vlo[EPL], vhi[EPL];
+    chain_lane2<EPL>(cv, a.j, 0, b, g, col, m_old, a.loop, lane, klo, khi);
+    chain_lane2<EPL>(cv, a.j, 1, b, g, col, m_old, a.loop, lane, vlo, vhi);
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) {
+      float dn = 0.f, dl = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        dn += qn[h][e] * khi[e];
+        dl += qo[h][e] * klo[e];
+      }
+      dn = warp_sum(dn) * a.tau;
+      dl = warp_sum(dl) * a.tau;
+      const float mn = fmaxf(m[h], fmaxf(dn, dl));
+      const float sc = m[h] == -INFINITY ? 0.f : expf(m[h] - mn);
+      const float en = expf(dn - mn), eo = expf(dl - mn);
+      z[h] = z[h] * sc + (en - eo);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) acc[h][e] = acc[h][e] * sc + en * vhi[e] - eo * vlo[e];
+      m[h] = mn;
+    }
+  }
+  // this CTA's piece: merge its warps
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    if (lane == 0) {
+      sm_m[warp][h] = m[h];
+      sm_z[warp][h] = z[h];
+    }
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) sm_acc[warp][h][lane * EPL + e] = acc[h][e];
+  }
+  __syncthreads();
+  for (int e = tid; e < GRP * HD; e += 256) {
+    const int h = e / HD, dd = e % HD;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][h]);
+    float A = 0.f, Z = 0.f;
+    if (M != -INFINITY)
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        if (sm_m[w][h] == -INFINITY) continue;
+        const float f = expf(sm_m[w][h] - M);
+        A += sm_acc[w][h][dd] * f;
+        Z += sm_z[w][h] * f;
+      }
+    pacc[h][dd] = A;
+    if (dd == 0) {
+      pm[h] = M;
+      pz[h] = Z;
+    }
+  }
+  cluster.sync();
+  if (rank == 0) {
+    for (int e = tid; e < GRP * HD; e += 256) {
+      const int h = e / HD, dd = e % HD;
+      const int hq = g * GRP + h;
+      const size_t so = static_cast<size_t>(tok) * a.H + hq;
+      const float L = a.lse_state[so];
+      float M = L;
+      for (int r = 0; r < CS; ++r) M = fmaxf(M, *cluster.map_shared_rank(&pm[h], r));
+      const float el = expf(L - M);
+      float Z = el, N = el * a.o_state[so * HD + dd];
+      for (int r = 0; r < CS; ++r) {
+        const float mr = *cluster.map_shared_rank(&pm[h], r);
+        if (mr == -INFINITY) continue;
+        const float f = expf(mr - M);
+        Z += f * *cluster.map_shared_rank(&pz[h], r);
+        N += f * *cluster.map_shared_rank(&pacc[h][dd], r);
+      }
+      if (!(Z > 0.f) && a.status) atomicOr(a.status, kErrBadIndex);
+      const float ov = N / Z;
+      a.o_state[so * HD + dd] = ov;
+      a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + dd] = f_to_bf16(ov);
+      a.q_last[so * HD + dd] = a.q_cur[(static_cast<size_t>(i) * a.H + hq) * HD + dd];
+      if (dd == 0) a.lse_state[so] = M + logf(Z);
+    }
+  }
+  cluster.sync();
+}
+
+// ============================================================================
 // cache import helpers
 // ============================================================================
 template <int EPL>
@@ -1214,6 +1430,9 @@ cudaError_t launch_change_keys(const float* h, const float* ref, const int* sel_
   return launch_k(g_pdl, k_change_keys, dim3((N + 3) / 4), dim3(128), 0, s, h, ref, sel_slot, N, d, loop, key, last,
                   tile, has_c);
 }
+cudaError_t launch_select_step(const SelectStepArgs& a, cudaStream_t s) {
+  return launch_k(g_pdl, k_select_step, dim3(1), dim3(1024), 0, s, a);
+}
 cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, const int* has_c, const TilePlan& p,
                               cudaStream_t s) {
   return launch_k(g_pdl, k_plan_tiles, dim3(1), dim3(1024), 0, s, idx, n_sel, tile, has_c, p);
@@ -1230,9 +1449,43 @@ cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cud
 cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t s) {
   return launch_k(g_pdl, k_select_cols, dim3(max_need * a.Hkv), dim3(1024), 0, s, a);
 }
+template <typename K>
+cudaError_t launch_cluster(K kern, dim3 grid, dim3 block, int cluster_x, cudaStream_t s, const CorrectArgs& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster_x;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = g_pdl ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
 cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
-  dim3 grid(n_sel * a.Hkv, a.n_splits);
   const int grp = a.H / a.Hkv;
+  if (a.cluster) {
+    dim3 grid(kCorrCluster, n_sel * a.Hkv);
+#define FL_CORRC(G)                                                                                      \
+  case G:                                                                                                \
+    return a.hd == 128 ? launch_cluster(k_correct_cluster<128, 4, G>, grid, dim3(256), kCorrCluster, s, a) \
+                       : launch_cluster(k_correct_cluster<64, 2, G>, grid, dim3(256), kCorrCluster, s, a);
+    switch (grp) {
+      FL_CORRC(1)
+      FL_CORRC(2)
+      FL_CORRC(4)
+      FL_CORRC(8)
+      default: return cudaErrorInvalidValue;
+    }
+#undef FL_CORRC
+  }
+  dim3 grid(n_sel * a.Hkv, a.n_splits);
 #define FL_CORR(G)                                                                  \
   case G:                                                                           \
     return a.hd == 128 ? launch_k(g_pdl, k_correct<128, 4, G>, grid, dim3(256), 0, s, a) \

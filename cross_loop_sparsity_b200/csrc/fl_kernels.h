@@ -62,6 +62,23 @@ struct TilePlan {
   int* counts;  // [0] entries, [1] entries needing a column set
 };
 
+struct SelectStepArgs {
+  const float* h;        // [N][d] current hidden states
+  const float* h_in;     // [N][d] call inputs (change after loop 1)
+  float* h_snap;         // [n_sel][d] loop-start rows of the selected tokens (read, then rewritten)
+  int* sel_slot;         // [N] slot of each token in the selection, or -1 (read, then rewritten)
+  int N, d, loop, n_sel;
+  float* key;            // [N]
+  float* keys_trace;     // [N] this loop's keys, kept for read-back
+  int32_t* idx;          // [n_sel] this loop's selection
+  int* last;             // [N]
+  const int* tile;       // [N]
+  int* has_c;            // [tiles]
+  const int* forced_on;
+  const int32_t* forced;
+  TilePlan plan;
+};
+
 struct DScoreArgs {
   TilePlan plan;
   const int32_t* idx;
@@ -106,6 +123,7 @@ struct CorrectArgs {
   int j, loop, H, Hkv, hd, c, n_tiles;
   float tau;
   int cols_per_cta, n_splits;   // column split: grid.y = n_splits = ceil(c / cols_per_cta)
+  int cluster;                  // few queries: one kCorrCluster-CTA cluster per (query, group)
   float* part_acc;              // [n_sel][Hkv][n_splits][8][hd]
   float* part_mz;               // [n_sel][Hkv][n_splits][8][2]
   int* counters;                // [n_sel][Hkv], zero between launches
@@ -120,6 +138,7 @@ struct LensArg {
   int v[kLensByValue];
 };
 cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s);
+constexpr int kCorrCluster = 8;   // CTAs per (query, KV group) in the clustered correction
 // Launches made while this is on (the kernels of one call) are programmatic
 // dependents of the previous kernel; thread-local.
 void set_pdl(bool on);
@@ -138,6 +157,7 @@ cudaError_t launch_after_select(const int32_t* idx, int n_sel, int N, int d, int
                                 float* h_snap, cudaStream_t s);
 cudaError_t launch_change_keys(const float* h, const float* ref, const int* sel_slot, int N, int d, int loop,
                                float* key, int* last, const int* tile, int* has_c, cudaStream_t s);
+cudaError_t launch_select_step(const SelectStepArgs& a, cudaStream_t s);
 cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, const int* has_c, const TilePlan& p,
                               cudaStream_t s);
 cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s);

@@ -90,6 +90,8 @@ constexpr int kNumSM = 148;
 // Sparse-column correction: columns per CTA.  Few selected queries (decode)
 // get narrow splits for parallelism; many (prefill) get wide ones.
 constexpr int kCorrColsSmall = 16, kCorrColsBig = 128, kCorrSmallQueries = 64;
+// Calls of at most this many tokens do a lazy loop's bookkeeping in one CTA.
+constexpr int kSelectStepMaxTokens = 1024;
 constexpr int kCountersGemm = 4096;
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -493,7 +495,19 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
     const bool full = !lazy || l == 1;
     const int32_t* idx = ctx->idx_all;
     int n = N;
-    if (!full) {
+    if (!full && N <= kSelectStepMaxTokens) {
+      // few tokens (decode): keys, selection, snapshot and tile plan in one kernel
+      int32_t* sel = ctx->idx_sel + static_cast<size_t>(l - 2) * ctx->N_max;
+      SelectStepArgs sa{};
+      sa.h = ctx->h; sa.h_in = ctx->h_in; sa.h_snap = ctx->h_snap; sa.sel_slot = ctx->sel_slot;
+      sa.N = N; sa.d = d; sa.loop = l; sa.n_sel = n_sel; sa.key = ctx->key;
+      sa.keys_trace = ctx->keys_trace + static_cast<size_t>(l - 2) * ctx->N_max; sa.idx = sel;
+      sa.last = ctx->last; sa.tile = ctx->tile; sa.has_c = ctx->has_c; sa.forced_on = ctx->forced_on;
+      sa.forced = ctx->forced_sel + static_cast<size_t>(l - 2) * ctx->N_max; sa.plan = ctx->plan;
+      FL_LAUNCH(FL_KIND_SELECT, launch_select_step(sa, s));
+      idx = sel;
+      n = n_sel;
+    } else if (!full) {
       int32_t* sel = ctx->idx_sel + static_cast<size_t>(l - 2) * ctx->N_max;
       FL_TRY(cudaMemcpyAsync(ctx->keys_trace + static_cast<size_t>(l - 2) * ctx->N_max, ctx->key,
                              static_cast<size_t>(N) * 4, cudaMemcpyDeviceToDevice, s));
@@ -553,6 +567,7 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
         ca.cols_per_cta = n_sel <= kCorrSmallQueries ? kCorrColsSmall : kCorrColsBig;
         ca.n_splits = ceil_div(c.c_cols, ca.cols_per_cta);
         ca.part_acc = ctx->corr_acc; ca.part_mz = ctx->corr_mz; ca.counters = ctx->corr_counters;
+        ca.cluster = n_sel <= kCorrSmallQueries ? 1 : 0;
         FL_LAUNCH(FL_KIND_CORRECT, launch_correct(ca, n, s));
       }
       FL_GEMM(gemm(ctx, kOpO, j, n, idx, s));
@@ -562,7 +577,7 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
       FL_GEMM(gemm(ctx, kOpGU, j, n, idx, s));
       FL_GEMM(gemm(ctx, kOpDown, j, n, idx, s));
     }
-    if (lazy && l < K)
+    if (lazy && l < K && N > kSelectStepMaxTokens)
       FL_LAUNCH(FL_KIND_OTHER, launch_change_keys(ctx->h, l == 1 ? ctx->h_in : ctx->h_snap, ctx->sel_slot, N, d, l,
                                                   ctx->key, ctx->last, ctx->tile, ctx->has_c, s));
   }

@@ -1,0 +1,145 @@
+"""Kernel-level measurements against the B200 roofline (one JSON line per kernel).
+
+  python -m cross_loop_sparsity_b200.kernel_bench [--reps N]
+
+* ``gemm_wide``: the 128x128 tcgen05 GEMM at the long-prefill shapes
+  (16384 tokens x d_model 2048: QKV 3072, O 2048, gate or up 5632, down from
+  5632), TFLOP/s against the measured dense bf16 peak.
+* ``gemm_skinny``: the split-K swap-AB GEMM at the decode shapes (8 tokens),
+  weight GB/s against the measured HBM bandwidth.
+* ``quantize``: the KV-residual quantiser over a residual shaped like the
+  65536-token context (65536 tokens x 4 layers x 2 (K, V) x 4 KV heads rows of
+  128 fp32, int4 / int2, group 64), bytes moved against HBM.
+
+Every operand set is rotated over copies whose total exceeds L2 (126 MB), so
+each timed launch reads from HBM; times are CUDA events around ``reps``
+launches after warm-up, on one stream.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def _time(fn, reps, warmup=3):
+    import torch
+    for i in range(warmup):
+        fn(i)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(reps):
+        fn(i)
+    b.record()
+    b.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def gemm_wide(reps):
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    hbm, tc, src = _peaks()
+    out = []
+    M = 16384
+    for name, n, k in (("qkv", 3072, 2048), ("o", 2048, 2048), ("gate_or_up", 5632, 2048), ("down", 2048, 5632)):
+        A = torch.randn((M, k), device="cuda").to(torch.bfloat16)
+        Bs = [torch.randn((n, k), device="cuda").mul_(0.02).to(torch.bfloat16) for _ in range(2)]
+        D = torch.empty((M, n), dtype=torch.float32, device="cuda")
+        import ctypes
+        L = fl.lib()
+
+        def run(i, B=Bs):
+            st = L.fl_test_gemm(ctypes.c_void_p(A.data_ptr()), ctypes.c_void_p(B[i % 2].data_ptr()),
+                                ctypes.c_void_p(D.data_ptr()), M, n, k, 0, None, 0, None)
+            assert st == 0
+        ms = _time(run, reps)
+        tflops = 2.0 * M * n * k / (ms * 1e-3) / 1e12
+        out.append({"kernel": "gemm_wide", "shape": f"{name}: {M}x{n}x{k}", "ms": ms, "achieved": tflops,
+                    "unit": "TFLOP/s", "peak": tc, "frac": tflops / tc, "peak_source": f"{src} bf16_tflops"})
+    return out
+
+
+def gemm_skinny(reps):
+    import ctypes
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    hbm, tc, src = _peaks()
+    L = fl.lib()
+    out = []
+    m = 8
+    for name, n, k in (("qkv", 3072, 2048), ("o", 2048, 2048), ("gate_or_up", 5632, 2048), ("down", 2048, 5632),
+                       ("lm_head", 32000, 2048)):
+        copies = max(2, int(np.ceil(300e6 / (n * k * 2))))
+        Bs = [torch.randn((n, k), device="cuda").mul_(0.02).to(torch.bfloat16) for _ in range(copies)]
+        A = torch.randn((m, k), device="cuda").to(torch.bfloat16)
+        D = torch.empty((m, n), dtype=torch.float32, device="cuda")
+        nb = int(L.fl_test_gemm_scratch_bytes(m, n, k, 1))
+        scratch = torch.empty(max(nb, 256) + 256, dtype=torch.uint8, device="cuda")
+        sp = scratch.data_ptr() + ((-scratch.data_ptr()) % 256)
+
+        def run(i):
+            st = L.fl_test_gemm(ctypes.c_void_p(A.data_ptr()), ctypes.c_void_p(Bs[i % copies].data_ptr()),
+                                ctypes.c_void_p(D.data_ptr()), m, n, k, 1, ctypes.c_void_p(sp), nb, None)
+            assert st == 0
+        ms = _time(run, reps)
+        gbs = (n * k * 2 + m * k * 2 + m * n * 4) / (ms * 1e-3) / 1e9
+        out.append({"kernel": "gemm_skinny", "shape": f"{name}: {m}x{n}x{k}", "ms": ms, "achieved": gbs,
+                    "unit": "GB/s", "peak": hbm, "frac": gbs / hbm, "peak_source": f"{src} hbm_gbs",
+                    "note": "standalone launch (ticket split-K path, no programmatic overlap)"})
+        del Bs
+        torch.cuda.empty_cache()
+    return out
+
+
+def quantize(reps):
+    import ctypes
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    hbm, tc, src = _peaks()
+    L = fl.lib()
+    out = []
+    rows, width, g = 65536 * 4 * 2 * 4, 128, 64
+    r = torch.randn((rows, width), device="cuda")
+    for bits in (4, 2):
+        codes = torch.empty((rows, width * bits // 8), dtype=torch.uint8, device="cuda")
+        scales = torch.empty((rows, width // g), dtype=torch.int16, device="cuda")
+
+        def run(i):
+            st = L.fl_test_quantize(ctypes.c_void_p(r.data_ptr()), rows, width, g, bits,
+                                    ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()), None)
+            assert st == 0
+        ms = _time(run, reps)
+        moved = rows * width * 4 + rows * width * bits // 8 + rows * (width // g) * 2
+        gbs = moved / (ms * 1e-3) / 1e9
+        out.append({"kernel": "quantize", "shape": f"int{bits}: {rows} rows x {width}, g{g}", "ms": ms,
+                    "achieved": gbs, "unit": "GB/s", "peak": hbm, "frac": gbs / hbm,
+                    "peak_source": f"{src} hbm_gbs"})
+    return out
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--reps", type=int, default=20)
+    args = ap.parse_args()
+    from cross_loop_sparsity_b200 import build
+    build.build()
+    for fn in (gemm_wide, gemm_skinny, quantize):
+        for line in fn(args.reps):
+            print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

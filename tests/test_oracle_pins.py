@@ -181,8 +181,11 @@ def test_rope_matches_complex_rotation_and_relative_position():
     assert abs(a - b) < 1e-10
 
 
-def _torch_block_forward(cfg, W, h):
-    """A plain pre-norm Llama-style layer stack written with torch library ops (fp64)."""
+def _torch_block_forward(cfg, W, h, bf16_ops=False):
+    """A plain pre-norm Llama-style layer stack written with torch library ops (fp64).
+
+    bf16_ops: the four GEMM input activations pass through torch's bf16 cast."""
+    op = (lambda t: t.to(torch.bfloat16).to(torch.float64)) if bf16_ops else (lambda t: t)
     H, Hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
     T = h.shape[0]
     x = torch.from_numpy(np.asarray(h, np.float64))
@@ -195,7 +198,7 @@ def _torch_block_forward(cfg, W, h):
         return torch.cat([z.real, z.imag], dim=-1)
 
     for lw in W["layers"]:
-        a = torch.nn.functional.rms_norm(x, (cfg.d_model,), torch.from_numpy(lw["attn_norm"]), cfg.rms_eps)
+        a = op(torch.nn.functional.rms_norm(x, (cfg.d_model,), torch.from_numpy(lw["attn_norm"]), cfg.rms_eps))
         y = a @ torch.from_numpy(lw["w_qkv"]).T
         q = rope(y[:, :H * hd].reshape(T, H, hd))
         k = rope(y[:, H * hd:(H + Hkv) * hd].reshape(T, Hkv, hd))
@@ -203,9 +206,9 @@ def _torch_block_forward(cfg, W, h):
         o = torch.nn.functional.scaled_dot_product_attention(
             q.transpose(0, 1)[None], k.transpose(0, 1)[None], v.transpose(0, 1)[None],
             is_causal=True, enable_gqa=True)[0].transpose(0, 1).reshape(T, H * hd)
-        x = x + cfg.resid_scale * (o @ torch.from_numpy(lw["w_o"]).T)
-        m = torch.nn.functional.rms_norm(x, (cfg.d_model,), torch.from_numpy(lw["mlp_norm"]), cfg.rms_eps)
-        act = torch.nn.functional.silu(m @ torch.from_numpy(lw["w_gate"]).T) * (m @ torch.from_numpy(lw["w_up"]).T)
+        x = x + cfg.resid_scale * (op(o) @ torch.from_numpy(lw["w_o"]).T)
+        m = op(torch.nn.functional.rms_norm(x, (cfg.d_model,), torch.from_numpy(lw["mlp_norm"]), cfg.rms_eps))
+        act = op(torch.nn.functional.silu(m @ torch.from_numpy(lw["w_gate"]).T) * (m @ torch.from_numpy(lw["w_up"]).T))
         x = x + cfg.resid_scale * (act @ torch.from_numpy(lw["w_down"]).T)
     return x.numpy()
 
@@ -237,6 +240,22 @@ def test_dense_looped_forward_is_k_plain_blocks(K):
     assert res.trace["applications"] == cfg.n_layers * K
     x = want[-1] / np.sqrt(np.mean(want[-1] ** 2) + cfg.rms_eps)
     np.testing.assert_allclose(res.logits[0], W["w_out"] @ x, atol=1e-11)
+
+
+@pytest.mark.parametrize("K", [1, 3])
+def test_bf16_operand_mode_matches_torch_bf16_casts(K):
+    """With bf16_ops the dense forward equals the torch restatement that rounds
+    the same four GEMM operands with torch's own bf16 cast."""
+    cfg = _tiny_cfg(n_loops=K, resid_bits=16, seed=17)
+    W, rng = _weights(cfg)
+    h0 = synth.make_h0(cfg, rng, cfg.seq_len)
+    res = orc.prefill(cfg, W, orc.KVCache(cfg, 1, cfg.seq_len, kv_exact=True), h0, 1, cfg.seq_len, bf16_ops=True)
+    want = np.asarray(h0, np.float64)
+    for _ in range(K):
+        want = _torch_block_forward(cfg, W, want, bf16_ops=True)
+    np.testing.assert_allclose(res.h, want, rtol=0, atol=1e-9 * np.abs(want).max())
+    plain = orc.prefill(cfg, W, orc.KVCache(cfg, 1, cfg.seq_len, kv_exact=True), h0, 1, cfg.seq_len)
+    assert np.max(np.abs(plain.h - res.h)) > 0      # the rounding is really applied
 
 
 def test_block_applications_golden():
