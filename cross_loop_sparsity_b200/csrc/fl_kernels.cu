@@ -341,13 +341,23 @@ __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
     }
     return;
   }
-  float prev[EPL];
-  chain_lane<EPL>(cv, a.j, kv, b, gk, t, a.loop - 1, lane, prev);
-  float r[EPL];
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) r[e] = __fsub_rn(x[e], prev[e]);
   int c[EPL];
-  const uint16_t s = quantize_lane<EPL>(r, cv.g, cv.bits, c);
+  uint16_t s;
+  if (a.forced_on && a.forced_on[0]) {
+    // checks only: the caller's codes for this selection slot
+    const size_t row = (((static_cast<size_t>(a.j) * (cv.K - 1) + (a.loop - 2)) * a.forced_ns + i) * 2 + kv) *
+                           a.Hkv + gk;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) c[e] = a.forced_codes[row * hd + lane * EPL + e];
+    s = a.forced_scales[row * (hd / cv.g) + (lane * EPL) / cv.g];
+  } else {
+    float prev[EPL];
+    chain_lane<EPL>(cv, a.j, kv, b, gk, t, a.loop - 1, lane, prev);
+    float r[EPL];
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) r[e] = __fsub_rn(x[e], prev[e]);
+    s = quantize_lane<EPL>(r, cv.g, cv.bits, c);
+  }
   store_lane_codes<EPL>(cv.code_row(a.j, a.loop, kv, b, gk, t), cv.bits, lane, c);
   const int GL = cv.g / EPL;
   if ((lane % GL) == 0) cv.scale_row(a.j, a.loop, kv, b, gk, t)[lane / GL] = s;

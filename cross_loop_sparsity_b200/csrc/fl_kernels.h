@@ -23,6 +23,10 @@ struct QkvPostArgs {
   int j, loop, lazy;
   float* q_cur;       // [n][H][hd] GEMM order
   float* q_last;      // [N][H][hd] token order (this layer), written at loop 1
+  const int* forced_on;           // forced residual codes (checks): [0] != 0 when on
+  const int8_t* forced_codes;     // [M][K-1][ns][2][Hkv][hd]
+  const uint16_t* forced_scales;  // [M][K-1][ns][2][Hkv][hd/g]
+  int forced_ns;                  // selection-slot stride ns
 };
 
 struct AttnDecArgs {

@@ -56,6 +56,10 @@ struct flashloop_ctx {
   int* forced_on = nullptr;
   int32_t *forced_sel = nullptr, *forced_cols = nullptr;
   int* forced_ncols = nullptr;
+  int8_t* forced_codes = nullptr;
+  uint16_t* forced_scales = nullptr;
+  int* forced_codes_on = nullptr;
+  int nsel_max = 0;
   float *part_o = nullptr, *part_ml = nullptr;
   int* attn_counters = nullptr;
   float *corr_acc = nullptr, *corr_mz = nullptr;
@@ -210,6 +214,10 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   uint8_t* forced_sel = take(static_cast<size_t>(K) * N * 4);
   uint8_t* forced_cols = take(static_cast<size_t>(M) * n_tiles * Hkv * cc * 4);
   uint8_t* forced_ncols = take(static_cast<size_t>(M) * n_tiles * Hkv * 4);
+  const size_t fc_rows = lazy ? static_cast<size_t>(M) * (K - 1) * nsel_max * 2 * Hkv : 0;
+  uint8_t* forced_codes = take(std::max<size_t>(fc_rows * hd, 16));
+  uint8_t* forced_scales = take(std::max<size_t>(fc_rows * (lazy ? hd / c.group_size : 1) * 2, 16));
+  uint8_t* forced_codes_on = take(16);
   // decode attention split partials
   int splits = ceil_div(4 * kNumSM, c.max_batch * Hkv);
   const int max_splits = ceil_div(c.max_ctx, 64);
@@ -309,6 +317,10 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->forced_sel = reinterpret_cast<int32_t*>(forced_sel);
     x->forced_cols = reinterpret_cast<int32_t*>(forced_cols);
     x->forced_ncols = reinterpret_cast<int*>(forced_ncols);
+    x->forced_codes = reinterpret_cast<int8_t*>(forced_codes);
+    x->forced_scales = reinterpret_cast<uint16_t*>(forced_scales);
+    x->forced_codes_on = reinterpret_cast<int*>(forced_codes_on);
+    x->nsel_max = nsel_max;
     x->part_o = reinterpret_cast<float*>(part_o);
     x->part_ml = reinterpret_cast<float*>(part_ml);
     x->attn_counters = reinterpret_cast<int*>(attn_counters);
@@ -530,6 +542,8 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
       qa.qkv = ctx->qkv; qa.ldq = ctx->qkv_rows; qa.idx = idx; qa.n = n; qa.seq = ctx->seq; qa.pos = ctx->pos;
       qa.H = H; qa.Hkv = Hkv; qa.hd = hd; qa.rope_cos = ctx->rope_cos; qa.rope_sin = ctx->rope_sin;
       qa.cv = ctx->cv; qa.j = j; qa.loop = l; qa.lazy = lazy ? 1 : 0; qa.q_cur = ctx->q_cur; qa.q_last = ql;
+      qa.forced_on = ctx->forced_codes_on; qa.forced_codes = ctx->forced_codes;
+      qa.forced_scales = ctx->forced_scales; qa.forced_ns = ctx->nsel_max;
       FL_LAUNCH(FL_KIND_KV, launch_qkv_post(qa, s));
       if (full) {
         if (decode) {
@@ -1001,6 +1015,27 @@ fl_status flashloop_force_selection(flashloop_ctx* ctx, const int32_t* sel, int 
     }
   }
   FL_TRY(cudaMemcpy(ctx->forced_on, &on, 4, cudaMemcpyHostToDevice));
+  return FL_OK;
+}
+
+fl_status flashloop_force_codes(flashloop_ctx* ctx, const int8_t* codes, const uint16_t* scales, int n_sel) {
+  if (!ctx || !ctx->lazy) return FL_ERR_INVALID_ARG;
+  const flashloop_config& c = ctx->cfg;
+  const int on = (codes && scales) ? 1 : 0;
+  if (on) {
+    if (n_sel < 1 || n_sel > ctx->nsel_max || c.n_loops < 2) return FL_ERR_INVALID_ARG;
+    const size_t per = static_cast<size_t>(2) * c.n_kv_heads;   // rows per selection slot
+    const size_t ns_code = c.head_dim, ns_scale = c.head_dim / c.group_size;
+    for (int jl = 0; jl < c.n_layers * (c.n_loops - 1); ++jl) {
+      FL_TRY(cudaMemcpy(ctx->forced_codes + static_cast<size_t>(jl) * ctx->nsel_max * per * ns_code,
+                        codes + static_cast<size_t>(jl) * n_sel * per * ns_code, n_sel * per * ns_code,
+                        cudaMemcpyHostToDevice));
+      FL_TRY(cudaMemcpy(ctx->forced_scales + static_cast<size_t>(jl) * ctx->nsel_max * per * ns_scale,
+                        scales + static_cast<size_t>(jl) * n_sel * per * ns_scale, n_sel * per * ns_scale * 2,
+                        cudaMemcpyHostToDevice));
+    }
+  }
+  FL_TRY(cudaMemcpy(ctx->forced_codes_on, &on, 4, cudaMemcpyHostToDevice));
   return FL_OK;
 }
 

@@ -66,6 +66,7 @@ _SIG = {
     "flashloop_export_slice": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "flashloop_force_selection": (_I, [_P, _P, _I, _I, _P, _P, _I]),
     "flashloop_read_trace": (_I, [_P, _P, _P, _P, _P, _P]),
+    "flashloop_force_codes": (_I, [_P, _P, _P, _I]),
     "flashloop_set_option": (_I, [_P, _I, _I]),
     "flashloop_profile": (_I, [_P, _P, _P, _P]),
     "flashloop_kernels_per_call": (_I, [_P]),
@@ -295,6 +296,18 @@ class FlashLoop:
                                                sel.shape[1], cols.ctypes.data_as(ctypes.c_void_p),
                                                ncols.ctypes.data_as(ctypes.c_void_p), n_tiles),
                "force_selection", self.ctx)
+
+    def force_codes(self, codes=None, scales=None):
+        """codes int8 [M][K-1][n_sel][2][Hkv][hd], scales float16 [M][K-1][n_sel][2][Hkv][hd/g]; None clears."""
+        if codes is None:
+            _check(lib().flashloop_force_codes(self.ctx, None, None, 0), "force_codes")
+            return
+        codes = np.ascontiguousarray(codes, np.int8)
+        scales = np.ascontiguousarray(scales, np.float16).view(np.uint16)
+        self._forced_codes_keep = (codes, scales)
+        _check(lib().flashloop_force_codes(self.ctx, codes.ctypes.data_as(ctypes.c_void_p),
+                                           scales.ctypes.data_as(ctypes.c_void_p), codes.shape[2]),
+               "force_codes", self.ctx)
 
     def read_trace(self, N: int, n_sel: int, n_tiles: int, stream=None):
         c = self.c

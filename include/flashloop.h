@@ -181,6 +181,16 @@ fl_status flashloop_export_slice(const flashloop_ctx* ctx, int layer, int loop, 
 fl_status flashloop_force_selection(flashloop_ctx* ctx, const int32_t* sel, int n_sel_loops, int n_sel,
                                     const int32_t* cols, const int32_t* ncols, int n_tiles);
 
+/* Force the residual codes of the next call's recomputed tokens (checks
+ * only): codes int8 [M][K-1][n_sel][2][Hkv][hd] in [-qmax, qmax] and fp16 scale
+ * bits [M][K-1][n_sel][2][Hkv][hd/g], for layer, loop 2..K, selection slot,
+ * K (0) / V (1), KV head (host arrays; NULL clears).  The quantiser's decisions
+ * turn small floating-point differences into whole code steps, so a check of a
+ * call's arithmetic against another implementation hands over these integer
+ * decisions along with the selections; the quantiser itself is checked
+ * bit-exactly on identical inputs (fl_test_quantize). */
+fl_status flashloop_force_codes(flashloop_ctx* ctx, const int8_t* codes, const uint16_t* scales, int n_sel);
+
 /* Read back the last call's choices (host buffers): sel [K-1][n_sel]; keys
  * [K-1][N] fp32 selection keys of loops 2..K; cols/ncols as above.  Any may be
  * NULL.  Synchronises `stream`. */

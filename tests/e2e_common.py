@@ -2,10 +2,14 @@
 
 Each driver draws one seeded workload from ``synth``, runs the CPU oracle on
 it, runs the CUDA library on the same arrays through the C ABI, and returns
-both.  In "forced" mode the library is handed the oracle's own token and
-column selections (the oracle's outputs become the library's inputs, never
-the reverse), so the comparison is of arithmetic rather than of near-tie
-choices; the library still computes every key itself.
+both.  In "forced" mode the library is handed the oracle's own integer
+decisions -- token selections, column sets and residual codes with their
+scales (the oracle's outputs become the library's inputs, never the reverse)
+-- so the comparison is of arithmetic rather than of decisions that small
+floating-point differences flip (a perturbation of 1e-6 of the inputs moves
+the oracle's own early-position states by 2% of RMS through code flips).  The
+library still computes every key and every residual itself; its selection and
+quantiser are checked bit-exactly on identical inputs elsewhere.
 """
 import numpy as np
 
@@ -50,6 +54,22 @@ def forced_arrays(cfg, trace, n_tiles):
     return sel, cols, ncols
 
 
+def forced_codes(cfg, cache, trace, seq, pos):
+    """The oracle's residual codes and scales of each loop's recomputed tokens,
+    in selection order: [M][K-1][n_sel][2][Hkv][hd] and [..][hd/g]."""
+    M, K = cfg.n_layers, cfg.n_loops
+    S2 = trace["sel"][2]
+    n_sel = len(S2)
+    codes = np.zeros((M, K - 1, n_sel, 2, cfg.n_kv_heads, cfg.head_dim), np.int8)
+    scales = np.zeros((M, K - 1, n_sel, 2, cfg.n_kv_heads, cfg.head_dim // cfg.group_size), np.float16)
+    for l in range(2, K + 1):
+        for a, t in enumerate(trace["sel"][l]):
+            for kv, nm in enumerate(("k", "v")):
+                codes[:, l - 2, a, kv] = getattr(cache, "codes_" + nm)[:, l - 2, seq[t], :, pos[t]]
+                scales[:, l - 2, a, kv] = getattr(cache, "scales_" + nm)[:, l - 2, seq[t], :, pos[t]]
+    return codes, scales
+
+
 def run_prefill(cfg, B, T, forced=True, dense=False):
     import torch
     from cross_loop_sparsity_b200 import flashloop as fl
@@ -59,11 +79,14 @@ def run_prefill(cfg, B, T, forced=True, dense=False):
     w = synth.make_weights(cfg)
     h0 = synth.make_h0(cfg, w["rng"], B * T)
     W = orc.prepare_weights(w)
-    ref = orc.prefill(cfg, W, orc.KVCache(cfg, B, T), h0, B, T, bf16_ops=bf16_ops(cfg))
+    ocache = orc.KVCache(cfg, B, T)
+    ref = orc.prefill(cfg, W, ocache, h0, B, T, bf16_ops=bf16_ops(cfg))
     eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=T, max_tokens=B * T)
     n_tiles = B * ((T + cfg.q_tile - 1) // cfg.q_tile)
     if forced and not dense and cfg.n_loops > 1:
         eng.force_selection(*forced_arrays(cfg, ref.trace, n_tiles), n_tiles=n_tiles)
+        seq, pos = np.repeat(np.arange(B), T), np.tile(np.arange(T), B)
+        eng.force_codes(*forced_codes(cfg, ocache, ref.trace, seq, pos))
     h_out = torch.empty((B * T, cfg.d_model), dtype=torch.float32, device="cuda")
     logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
     eng.prefill(torch.from_numpy(h0).cuda(), B, T, h_out, logits)
@@ -99,9 +122,11 @@ def run_decode(cfg, lens, forced=True, dense=False, steps=1, extra_ctx=0):
     results = []
     for _ in range(steps):
         h0 = synth.make_h0(cfg, rng, B)
+        pos = cache.lens[:B].copy()
         ref = orc.decode_step(cfg, W, cache, h0, bf16_ops=bf16_ops(cfg))
         if forced and not dense and cfg.n_loops > 1:
             eng.force_selection(*forced_arrays(cfg, ref.trace, B), n_tiles=B)
+            eng.force_codes(*forced_codes(cfg, cache, ref.trace, np.arange(B), pos))
         h_out = torch.empty((B, cfg.d_model), dtype=torch.float32, device="cuda")
         logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
         eng.decode_step(torch.from_numpy(h0).cuda(), B, h_out, logits)
