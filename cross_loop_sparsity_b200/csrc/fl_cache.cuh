@@ -95,14 +95,17 @@ __device__ __forceinline__ void chain_lane(const CacheView& cv, int j, int kv, i
   }
 }
 
-// Maximum loops K the reconstruction below unrolls for.
+// Largest loop count K a context supports; kernels that reconstruct the chain
+// are instantiated for KM in {2, 4, 8, 16}, the smallest power of two >= K, so
+// the unrolled reconstruction issues no work for loops that cannot exist.
 constexpr int kMaxLoops = 16;
+inline int chain_km(int K) { return K <= 2 ? 2 : K <= 4 ? 4 : K <= 8 ? 8 : 16; }
 
-// Reconstructions to loop m_lo and to loop m_hi (m_lo <= m_hi) of one row;
-// lane holds EPL values of each.  All loads (base row, residual codes and
+// Reconstructions to loop m_lo and to loop m_hi (m_lo <= m_hi <= KM) of one
+// row; lane holds EPL values of each.  All loads (base row, residual codes and
 // scales of loops 2..m_hi) are issued before any arithmetic so their latencies
 // overlap; the adds then run in loop order, as the definition requires.
-template <int EPL>
+template <int EPL, int KM = kMaxLoops>
 __device__ __forceinline__ void chain_lane2(const CacheView& cv, int j, int kv, int b, int h, int t, int m_lo,
                                             int m_hi, int lane, float* lo, float* hi) {
   const uint16_t* br = cv.base_row(j, kv, b, h, t) + lane * EPL;
@@ -118,10 +121,10 @@ __device__ __forceinline__ void chain_lane2(const CacheView& cv, int j, int kv, 
   const size_t rb = cv.row_bytes_codes(), ns = cv.hd / cv.g;
   const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * cv.T;   // rows between consecutive loops
   const size_t r0 = cv.res_index(j, 2, kv, b, h, t);
-  uint32_t craw[kMaxLoops - 1];
-  uint16_t sraw[kMaxLoops - 1];
+  uint32_t craw[KM - 1];
+  uint16_t sraw[KM - 1];
 #pragma unroll
-  for (int q = 0; q < kMaxLoops - 1; ++q) {
+  for (int q = 0; q < KM - 1; ++q) {
     craw[q] = 0u;
     sraw[q] = 0;
     if (q + 2 <= m_hi) {
@@ -152,7 +155,7 @@ __device__ __forceinline__ void chain_lane2(const CacheView& cv, int j, int kv, 
   }
   const int fb = cv.bits;
 #pragma unroll
-  for (int q = 0; q < kMaxLoops - 1; ++q) {
+  for (int q = 0; q < KM - 1; ++q) {
     if (q + 2 <= m_hi) {
       const float sc = half_bits_to_f(sraw[q]);
 #pragma unroll

@@ -79,6 +79,30 @@ __device__ __forceinline__ void epi_apply(const GemmArgs& p, int row, int col0, 
   }
 }
 
+// The epilogue of one accumulator element (row, column col).
+template <bool SWAP>
+__device__ __forceinline__ void epi_one(const GemmArgs& p, int row, int col, int tile_m, int tile_n, int BN, float v0,
+                                        float v1) {
+  int tok, feat;
+  if (SWAP) {
+    feat = tile_m * 128 + row;
+    tok = col;
+  } else {
+    tok = tile_m * 128 + row;
+    feat = tile_n * BN + col;
+  }
+  if (tok >= p.n_tok || feat >= p.n_feat) return;
+  if (p.epi == kEpiStore) {
+    p.out[static_cast<size_t>(tok) * p.ldo + feat] = v0;
+  } else if (p.epi == kEpiResid) {
+    const int r = p.idx ? p.idx[tok] : tok;
+    float* dst = p.h + static_cast<size_t>(r) * p.ldh + feat;
+    *dst = *dst + p.scale * v0;
+  } else {
+    p.act[static_cast<size_t>(tok) * p.ld_act + feat] = f_to_bf16(silu_f(v0) * v1);
+  }
+}
+
 template <int BN, bool DA, bool DB, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 2)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
@@ -306,24 +330,27 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
       const int per = (BN + S - 1) / S;
       const int col0 = r * per, col1 = min(BN, col0 + per);
       float* red = reinterpret_cast<float*>(smem);
-      for (int c = col0; c < col1; c += 16) {
-        float a0[16], a1[16];
+      for (int cc = col0; cc < col1; ++cc) {
+        // every peer's value is requested before any is summed, so the
+        // distributed-shared-memory round trips overlap; the sum runs in rank order
+        float pv0[kMaxClusterSplits], pv1[kMaxClusterSplits];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) a0[j] = a1[j] = 0.f;
-        for (int q = 0; q < S; ++q) {
-          const float* peer = cluster.map_shared_rank(red, q);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (c + j < col1) {
-              a0[j] += peer[(c + j) * 128 + row];
-              if (C::kNAcc == 2) a1[j] += peer[(BN + c + j) * 128 + row];
-            }
+        for (int q = 0; q < kMaxClusterSplits; ++q) {
+          pv0[q] = 0.f;
+          pv1[q] = 0.f;
+          if (q < S) {
+            const float* peer = cluster.map_shared_rank(red, q);
+            pv0[q] = peer[cc * 128 + row];
+            if (C::kNAcc == 2) pv1[q] = peer[(BN + cc) * 128 + row];
           }
         }
-        // columns past col1 belong to the next rank: mark them out of range
-        GemmArgs pc = p;
-        pc.n_tok = min(p.n_tok, col1);
-        epi_apply<SWAP>(pc, row, c, tile_m, tile_n, BN, a0, a1);
+        float v0s = 0.f, v1s = 0.f;
+#pragma unroll
+        for (int q = 0; q < kMaxClusterSplits; ++q) {
+          v0s += pv0[q];
+          v1s += pv1[q];
+        }
+        epi_one<SWAP>(p, row, cc, tile_m, tile_n, BN, v0s, v1s);
       }
     }
     cluster.sync();

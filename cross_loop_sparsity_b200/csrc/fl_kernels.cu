@@ -934,7 +934,7 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
 // ("attention-output differences are dominated by a sparse and stable subset
 // of key columns", "FlashLoop ...", abstract).  grid (max_need*Hkv, chunks).
 // ============================================================================
-template <int HD, int EPL>
+template <int HD, int EPL, int KM>
 __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -961,7 +961,7 @@ __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
   // reconstruct K of loop l and the base for this column chunk
   for (int rr = warp; rr < nc; rr += 8) {
     float lo[EPL], hi[EPL];
-    chain_lane2<EPL>(cv, a.j, 0, b, g, c0 + rr, 1, a.loop, lane, lo, hi);
+    chain_lane2<EPL, KM>(cv, a.j, 0, b, g, c0 + rr, 1, a.loop, lane, lo, hi);
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
       Kb[rr * (HD + 1) + lane * EPL + e] = lo[e];
@@ -1044,7 +1044,7 @@ __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
 // group) -- an atomic ticket, no waiting -- merges the pieces with the stored
 // (O, lse) term and writes the new state.
 // ============================================================================
-template <int HD, int EPL, int GRP>
+template <int HD, int EPL, int GRP, int KM>
 __global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -1094,8 +1094,8 @@ __global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
   for (int k = k0 + warp; k < k1; k += NW) {
     const int col = C[k];
     float klo[EPL], khi[EPL], vlo[EPL], vhi[EPL];
-    chain_lane2<EPL>(cv, a.j, 0, b, g, col, m_old, a.loop, lane, klo, khi);
-    chain_lane2<EPL>(cv, a.j, 1, b, g, col, m_old, a.loop, lane, vlo, vhi);
+    chain_lane2<EPL, KM>(cv, a.j, 0, b, g, col, m_old, a.loop, lane, klo, khi);
+    chain_lane2<EPL, KM>(cv, a.j, 1, b, g, col, m_old, a.loop, lane, vlo, vhi);
 #pragma unroll
     for (int h = 0; h < GRP; ++h) {
       float dn = 0.f, dl = 0.f;
@@ -1200,41 +1200,61 @@ __global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
 }
 
 // ============================================================================
-// The same correction for few selected queries (decode): the column slices of
-// one (query, KV group) are the CTAs of one cluster.  Each CTA leaves its
-// piece (per-head max, denominator, numerator) in shared memory; after the
-// cluster barrier rank 0 merges the pieces of every rank, in rank order, over
-// distributed shared memory, together with the stored (O, lse) term.  No
-// global scratch, fence or ticket.  grid (kCorrCluster, n_sel * Hkv).
+// The correction for few selected queries (decode): the column slices of one
+// (query, KV group) are the CTAs of one cluster.  Each warp takes two columns
+// at a time with every K and V chain load of both issued before any
+// arithmetic.  Each CTA leaves its piece (per-head max, denominator,
+// numerator) in shared memory; after the cluster barrier rank 0 merges the
+// pieces of every rank, in rank order, over distributed shared memory,
+// together with the stored (O, lse) term.  No global scratch, fence or ticket.
+// grid (kCorrCluster, n_sel * Hkv).
 // ============================================================================
-template <int HD, int EPL, int GRP>
+template <int EPL, int GRP>
+__device__ __forceinline__ void corr_column(const float (&qn)[GRP][EPL], const float (&qo)[GRP][EPL],
+                                            const float* klo, const float* khi, const float* vlo,
+                                            const float* vhi, float tau, float (&m)[GRP], float (&z)[GRP],
+                                            float (&acc)[GRP][EPL]) {
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    float dn = 0.f, dl = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      dn += qn[h][e] * khi[e];
+      dl += qo[h][e] * klo[e];
+    }
+    dn = warp_sum(dn) * tau;
+    dl = warp_sum(dl) * tau;
+    const float mn = fmaxf(m[h], fmaxf(dn, dl));
+    const float sc = m[h] == -INFINITY ? 0.f : expf(m[h] - mn);
+    const float en = expf(dn - mn), eo = expf(dl - mn);
+    z[h] = z[h] * sc + (en - eo);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[h][e] = acc[h][e] * sc + en * vhi[e] - eo * vlo[e];
+    m[h] = mn;
+  }
+}
+
+template <int HD, int EPL, int GRP, int KM>
 __global__ void __launch_bounds__(256) k_correct_cluster(const CorrectArgs a) {
   pdl_trigger();
   pdl_wait();
-  constexpr int NW = 8;
+  constexpr int NW = 8, CS = kCorrCluster;
   __shared__ float sm_m[NW][GRP], sm_z[NW][GRP];
   __shared__ float sm_acc[NW][GRP][HD];
   __shared__ float pm[GRP], pz[GRP];
   __shared__ float pacc[GRP][HD];
-  __shared__ int nvalid_sh;
   cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int rank = static_cast<int>(cluster.block_rank()), CS = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
   const int i = blockIdx.y / a.Hkv, g = blockIdx.y % a.Hkv;
   const int tok = a.idx[i];
-  const int b = a.seq[tok], P = a.pos[tok], tl = a.tile[tok];
+  const int b = a.seq[tok], tl = a.tile[tok];
   const int m_old = a.last[tok];
   const CacheView& cv = a.cv;
   const size_t cset = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
   const int32_t* C = a.cols + cset * a.c;
-  // the query's columns: the prefix of the ascending set C with C[k] <= pos
-  const int ncol_all = a.ncols[cset];
-  int nv = 0;
-  for (int base = 0; base < ncol_all; base += 256) {
-    const int k = base + tid;
-    nv += __syncthreads_count(k < ncol_all && C[k] <= P);
-  }
-  if (tid == 0) nvalid_sh = nv;
+  // a decode token is its own tile, so every column of its set is causal
+  const int nvalid = a.ncols[cset];
   float qn[GRP][EPL], qo[GRP][EPL];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
@@ -1245,8 +1265,19 @@ __global__ void __launch_bounds__(256) k_correct_cluster(const CorrectArgs a) {
       qo[h][e] = a.q_last[(static_cast<size_t>(tok) * a.H + hq) * HD + lane * EPL + e];
     }
   }
-  __syncthreads();
-  const int nvalid = nvalid_sh;
+  // rank 0 requests the stored state it will merge into now, not after the barrier
+  float st_o[2] = {0.f, 0.f}, st_l[2] = {0.f, 0.f};
+  if (rank == 0) {
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int e = tid + r * 256;
+      if (e < GRP * HD) {
+        const size_t so = static_cast<size_t>(tok) * a.H + g * GRP + e / HD;
+        st_o[r] = a.o_state[so * HD + e % HD];
+        st_l[r] = a.lse_state[so];
+      }
+    }
+  }
   const int per = (nvalid + CS - 1) / CS;
   const int k0 = rank * per, k1 = min(nvalid, k0 + per);
   float m[GRP], z[GRP], acc[GRP][EPL];
@@ -1260,28 +1291,10 @@ __global__ void __launch_bounds__(256) k_correct_cluster(const CorrectArgs a) {
   for (int k = k0 + warp; k < k1; k += NW) {
     const int col = C[k];
     float klo[EPL], khi[EPL], vlo[EPL], vhi[EPL];
-    chain_lane2<EPL>(cv, a.j, 0, b, g, col, m_old, a.loop, lane, klo, khi);
-    chain_lane2<EPL>(cv, a.j, 1, b, g, col, m_old, a.loop, lane, vlo, vhi);
-#pragma unroll
-    for (int h = 0; h < GRP; ++h) {
-      float dn = 0.f, dl = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        dn += qn[h][e] * khi[e];
-        dl += qo[h][e] * klo[e];
-      }
-      dn = warp_sum(dn) * a.tau;
-      dl = warp_sum(dl) * a.tau;
-      const float mn = fmaxf(m[h], fmaxf(dn, dl));
-      const float sc = m[h] == -INFINITY ? 0.f : expf(m[h] - mn);
-      const float en = expf(dn - mn), eo = expf(dl - mn);
-      z[h] = z[h] * sc + (en - eo);
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) acc[h][e] = acc[h][e] * sc + en * vhi[e] - eo * vlo[e];
-      m[h] = mn;
-    }
+    chain_lane2<EPL, KM>(cv, a.j, 0, b, g, col, m_old, a.loop, lane, klo, khi);
+    chain_lane2<EPL, KM>(cv, a.j, 1, b, g, col, m_old, a.loop, lane, vlo, vhi);
+    corr_column<EPL, GRP>(qn, qo, klo, khi, vlo, vhi, a.tau, m, z, acc);
   }
-  // this CTA's piece: merge its warps
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
     if (lane == 0) {
@@ -1314,21 +1327,34 @@ __global__ void __launch_bounds__(256) k_correct_cluster(const CorrectArgs a) {
   }
   cluster.sync();
   if (rank == 0) {
-    for (int e = tid; e < GRP * HD; e += 256) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int e = tid + rr * 256;
+      if (e >= GRP * HD) break;
       const int h = e / HD, dd = e % HD;
       const int hq = g * GRP + h;
       const size_t so = static_cast<size_t>(tok) * a.H + hq;
-      const float L = a.lse_state[so];
-      float M = L;
-      for (int r = 0; r < CS; ++r) M = fmaxf(M, *cluster.map_shared_rank(&pm[h], r));
-      const float el = expf(L - M);
-      float Z = el, N = el * a.o_state[so * HD + dd];
+      const float L = st_l[rr];
+      // every rank's piece is requested before any is used, so the distributed
+      // shared-memory round trips overlap; the merge itself runs in rank order
+      float rm[CS], rz[CS], ra[CS];
+#pragma unroll
       for (int r = 0; r < CS; ++r) {
-        const float mr = *cluster.map_shared_rank(&pm[h], r);
-        if (mr == -INFINITY) continue;
-        const float f = expf(mr - M);
-        Z += f * *cluster.map_shared_rank(&pz[h], r);
-        N += f * *cluster.map_shared_rank(&pacc[h][dd], r);
+        rm[r] = *cluster.map_shared_rank(&pm[h], r);
+        rz[r] = *cluster.map_shared_rank(&pz[h], r);
+        ra[r] = *cluster.map_shared_rank(&pacc[h][dd], r);
+      }
+      float M = L;
+#pragma unroll
+      for (int r = 0; r < CS; ++r) M = fmaxf(M, rm[r]);
+      const float el = expf(L - M);
+      float Z = el, N = el * st_o[rr];
+#pragma unroll
+      for (int r = 0; r < CS; ++r) {
+        if (rm[r] == -INFINITY) continue;
+        const float f = expf(rm[r] - M);
+        Z += f * rz[r];
+        N += f * ra[r];
       }
       if (!(Z > 0.f) && a.status) atomicOr(a.status, kErrBadIndex);
       const float ov = N / Z;
@@ -1453,14 +1479,24 @@ size_t dscore_smem(int hd) {
 cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s) {
   dim3 grid(max_need * a.Hkv, max_chunks);
   const size_t sm = dscore_smem(a.hd);
-  if (a.hd == 128) return launch_k(g_pdl, k_dscore<128, 4>, grid, dim3(256), sm, s, a);
-  return launch_k(g_pdl, k_dscore<64, 2>, grid, dim3(256), sm, s, a);
+#define FL_DS(KMv)                                                                           \
+  case KMv:                                                                                  \
+    return a.hd == 128 ? launch_k(g_pdl, k_dscore<128, 4, KMv>, grid, dim3(256), sm, s, a)  \
+                       : launch_k(g_pdl, k_dscore<64, 2, KMv>, grid, dim3(256), sm, s, a);
+  switch (chain_km(a.cv.K)) {
+    FL_DS(2)
+    FL_DS(4)
+    FL_DS(8)
+    FL_DS(16)
+    default: return cudaErrorInvalidValue;
+  }
+#undef FL_DS
 }
 cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t s) {
   return launch_k(g_pdl, k_select_cols, dim3(max_need * a.Hkv), dim3(1024), 0, s, a);
 }
-template <typename K>
-cudaError_t launch_cluster(K kern, dim3 grid, dim3 block, int cluster_x, cudaStream_t s, const CorrectArgs& a) {
+template <typename K, typename A>
+cudaError_t launch_cluster(K kern, dim3 grid, dim3 block, int cluster_x, cudaStream_t s, const A& a) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -1478,28 +1514,32 @@ cudaError_t launch_cluster(K kern, dim3 grid, dim3 block, int cluster_x, cudaStr
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
-  const int grp = a.H / a.Hkv;
+template <int HD, int EPL, int GRP, int KM>
+cudaError_t launch_correct_t(const CorrectArgs& a, int n_sel, cudaStream_t s) {
   if (a.cluster) {
     dim3 grid(kCorrCluster, n_sel * a.Hkv);
-#define FL_CORRC(G)                                                                                      \
-  case G:                                                                                                \
-    return a.hd == 128 ? launch_cluster(k_correct_cluster<128, 4, G>, grid, dim3(256), kCorrCluster, s, a) \
-                       : launch_cluster(k_correct_cluster<64, 2, G>, grid, dim3(256), kCorrCluster, s, a);
-    switch (grp) {
-      FL_CORRC(1)
-      FL_CORRC(2)
-      FL_CORRC(4)
-      FL_CORRC(8)
-      default: return cudaErrorInvalidValue;
-    }
-#undef FL_CORRC
+    return launch_cluster(k_correct_cluster<HD, EPL, GRP, KM>, grid, dim3(256), kCorrCluster, s, a);
   }
   dim3 grid(n_sel * a.Hkv, a.n_splits);
-#define FL_CORR(G)                                                                  \
-  case G:                                                                           \
-    return a.hd == 128 ? launch_k(g_pdl, k_correct<128, 4, G>, grid, dim3(256), 0, s, a) \
-                       : launch_k(g_pdl, k_correct<64, 2, G>, grid, dim3(256), 0, s, a);
+  return launch_k(g_pdl, k_correct<HD, EPL, GRP, KM>, grid, dim3(256), 0, s, a);
+}
+
+template <int HD, int EPL, int GRP>
+cudaError_t launch_correct_km(const CorrectArgs& a, int n_sel, cudaStream_t s) {
+  switch (chain_km(a.cv.K)) {
+    case 2: return launch_correct_t<HD, EPL, GRP, 2>(a, n_sel, s);
+    case 4: return launch_correct_t<HD, EPL, GRP, 4>(a, n_sel, s);
+    case 8: return launch_correct_t<HD, EPL, GRP, 8>(a, n_sel, s);
+    case 16: return launch_correct_t<HD, EPL, GRP, 16>(a, n_sel, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
+  const int grp = a.H / a.Hkv;
+#define FL_CORR(G)                                                                   \
+  case G:                                                                            \
+    return a.hd == 128 ? launch_correct_km<128, 4, G>(a, n_sel, s) : launch_correct_km<64, 2, G>(a, n_sel, s);
   switch (grp) {
     FL_CORR(1)
     FL_CORR(2)
@@ -1508,6 +1548,20 @@ cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
     default: return cudaErrorInvalidValue;
   }
 #undef FL_CORR
+}
+
+// 16-CTA clusters are beyond the portable size: opt every instantiation in.
+template <int HD, int EPL, int GRP, int KM>
+cudaError_t allow_big_cluster() {
+  return cudaFuncSetAttribute(k_correct_cluster<HD, EPL, GRP, KM>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+}
+template <int HD, int EPL, int GRP>
+cudaError_t allow_big_cluster_km() {
+  cudaError_t e = allow_big_cluster<HD, EPL, GRP, 2>();
+  if (e == cudaSuccess) e = allow_big_cluster<HD, EPL, GRP, 4>();
+  if (e == cudaSuccess) e = allow_big_cluster<HD, EPL, GRP, 8>();
+  if (e == cudaSuccess) e = allow_big_cluster<HD, EPL, GRP, 16>();
+  return e;
 }
 
 // Opt every large-shared-memory kernel in to its dynamic shared memory once,
@@ -1530,8 +1584,22 @@ cudaError_t kernels_init_attrs() {
   set(k_attn_decode<64, 8>, static_cast<int>(attn_decode_smem(64)));
   set(k_attn_prefill<128>, static_cast<int>(attn_prefill_smem(128)));
   set(k_attn_prefill<64>, static_cast<int>(attn_prefill_smem(64)));
-  set(k_dscore<128, 4>, static_cast<int>(dscore_smem(128)));
-  set(k_dscore<64, 2>, static_cast<int>(dscore_smem(64)));
+  set(k_dscore<128, 4, 2>, static_cast<int>(dscore_smem(128)));
+  set(k_dscore<128, 4, 4>, static_cast<int>(dscore_smem(128)));
+  set(k_dscore<128, 4, 8>, static_cast<int>(dscore_smem(128)));
+  set(k_dscore<128, 4, 16>, static_cast<int>(dscore_smem(128)));
+  set(k_dscore<64, 2, 2>, static_cast<int>(dscore_smem(64)));
+  set(k_dscore<64, 2, 4>, static_cast<int>(dscore_smem(64)));
+  set(k_dscore<64, 2, 8>, static_cast<int>(dscore_smem(64)));
+  set(k_dscore<64, 2, 16>, static_cast<int>(dscore_smem(64)));
+  {
+    const cudaError_t r[8] = {allow_big_cluster_km<128, 4, 1>(), allow_big_cluster_km<128, 4, 2>(),
+                              allow_big_cluster_km<128, 4, 4>(), allow_big_cluster_km<128, 4, 8>(),
+                              allow_big_cluster_km<64, 2, 1>(),  allow_big_cluster_km<64, 2, 2>(),
+                              allow_big_cluster_km<64, 2, 4>(),  allow_big_cluster_km<64, 2, 8>()};
+    for (cudaError_t x : r)
+      if (e == cudaSuccess) e = x;
+  }
   done = e;
   return e;
 }

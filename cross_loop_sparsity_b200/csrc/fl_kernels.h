@@ -127,7 +127,8 @@ struct CorrectArgs {
   int j, loop, H, Hkv, hd, c, n_tiles;
   float tau;
   int cols_per_cta, n_splits;   // column split: grid.y = n_splits = ceil(c / cols_per_cta)
-  int cluster;                  // few queries: one kCorrCluster-CTA cluster per (query, group)
+  int cluster;                  // decode (each query its own tile, few queries): one cluster per
+                                // (query, group), merged over distributed shared memory
   float* part_acc;              // [n_sel][Hkv][n_splits][8][hd]
   float* part_mz;               // [n_sel][Hkv][n_splits][8][2]
   int* counters;                // [n_sel][Hkv], zero between launches
@@ -142,7 +143,7 @@ struct LensArg {
   int v[kLensByValue];
 };
 cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s);
-constexpr int kCorrCluster = 8;   // CTAs per (query, KV group) in the clustered correction
+constexpr int kCorrCluster = 16;  // CTAs per (query, KV group) in the clustered correction (non-portable size)
 // Launches made while this is on (the kernels of one call) are programmatic
 // dependents of the previous kernel; thread-local.
 void set_pdl(bool on);
@@ -167,6 +168,8 @@ cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, co
 cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s);
 cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t s);
 cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s);
+
+
 cudaError_t launch_pack_codes(const int8_t* src, int rows, int hd, int bits, uint8_t* dst, size_t dst_row_stride,
                               cudaStream_t s);
 

@@ -140,3 +140,24 @@ def test_decode_graph_replay_matches_direct_launches():
         outs.append(res)
     for a, b in zip(*outs):
         assert np.array_equal(a, b)
+
+
+def test_decode_free_running_selection_and_column_sets_are_valid():
+    cfg = synth.config("c1").with_(mode="decode", batch=6, rho=0.4, c_cols=20, seed=19, seq_len=0)
+    lens = [90, 33, 7, 64, 120, 1]
+    cfg, cache, eng, results = E.run_decode(cfg, lens, forced=False, steps=2)
+    from oracle import flashloop_oracle as orc
+    n_sel = orc.n_select(cfg.rho, len(lens))
+    for step, (ref, out) in enumerate(results):
+        assert out["status"] == 0
+        for l in range(2, cfg.n_loops + 1):
+            assert E.top_valid(out["keys"][l - 2], n_sel, out["sel"][l - 2]), (step, l)
+        chosen = set(int(t) for l in range(2, cfg.n_loops + 1) for t in out["sel"][l - 2])
+        for t in chosen:
+            P = lens[t] + step
+            for j in range(cfg.n_layers):
+                for g in range(cfg.n_kv_heads):
+                    n = out["ncols"][j, t, g]
+                    assert n == min(cfg.c_cols, P + 1)
+                    C = out["cols"][j, t, g, :n]
+                    assert np.all(np.diff(C) > 0) and C[0] >= 0 and C[-1] <= P
