@@ -28,8 +28,10 @@ constexpr int kABytes = 128 * kBoxK * 2;
 // Shared-memory ring budget: the skinny (decode) orientation keeps two CTAs per
 // SM so that a dependent GEMM can become resident and start streaming its
 // weights while the previous kernel still runs; the 128x128 orientation uses
-// one deep ring per SM.
-constexpr int kSmemBudgetSkinny = 100 * 1024;
+// one deep ring per SM.  Two skinny CTAs fit one SM's 228 KB with the 1 KB the
+// hardware reserves per CTA and this kernel's 1.25 KB of slack and barriers:
+// 2 * (ring + 2304 + 1024) <= 233472.
+constexpr int kSmemBudgetSkinny = 113408;
 constexpr int kSmemBudgetWide = 200 * 1024;
 
 template <int BN, bool DA, bool DB>
@@ -45,7 +47,10 @@ struct Cfg {
   static constexpr int kColsNeeded = kNAcc * BN;
   static constexpr uint32_t kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
                                         : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
-  static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + 256;
+  // barriers, TMEM slot, flags [0, 256); token scales [256, 512); warp sums [512, 528);
+  // partial sums of squares [768, 1280)
+  static constexpr int kTailBytes = 1280;
+  static constexpr int kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kTailBytes;
   static_assert(kBBytes % 1024 == 0, "B box must keep 1024-byte alignment of the swizzle atoms");
   static_assert(kStages >= 2, "pipeline needs two stages");
 };
@@ -79,10 +84,12 @@ __device__ __forceinline__ void epi_apply(const GemmArgs& p, int row, int col0, 
   }
 }
 
-// The epilogue of one accumulator element (row, column col).
+// The epilogue of one accumulator element (row, column col).  Returns the
+// updated hidden-state value of a residual epilogue (0 otherwise or if the
+// element is outside the output).
 template <bool SWAP>
-__device__ __forceinline__ void epi_one(const GemmArgs& p, int row, int col, int tile_m, int tile_n, int BN, float v0,
-                                        float v1) {
+__device__ __forceinline__ float epi_one(const GemmArgs& p, int row, int col, int tile_m, int tile_n, int BN, float v0,
+                                         float v1) {
   int tok, feat;
   if (SWAP) {
     feat = tile_m * 128 + row;
@@ -91,16 +98,113 @@ __device__ __forceinline__ void epi_one(const GemmArgs& p, int row, int col, int
     tok = tile_m * 128 + row;
     feat = tile_n * BN + col;
   }
-  if (tok >= p.n_tok || feat >= p.n_feat) return;
+  if (tok >= p.n_tok || feat >= p.n_feat) return 0.f;
   if (p.epi == kEpiStore) {
     p.out[static_cast<size_t>(tok) * p.ldo + feat] = v0;
   } else if (p.epi == kEpiResid) {
     const int r = p.idx ? p.idx[tok] : tok;
     float* dst = p.h + static_cast<size_t>(r) * p.ldh + feat;
-    *dst = *dst + p.scale * v0;
+    const float hn = *dst + p.scale * v0;
+    *dst = hn;
+    return hn;
   } else {
     p.act[static_cast<size_t>(tok) * p.ld_act + feat] = f_to_bf16(silu_f(v0) * v1);
   }
+  return 0.f;
+}
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
+
+// The token operand of a swap-orientation GEMM with an input RMSNorm, built by
+// the four epilogue warps (t4 = 0..127) while the TMA producer streams only
+// weights.  For ring slot s of k-chunk i the BN x 64 bf16 tile is written in
+// the layout a 128-byte-swizzling TMA load would leave: row r at r * 128 bytes,
+// 16-byte chunk j at ((j ^ (r % 8)) * 16).  The slot's full barrier expects
+// this arrival besides the producer's.  Returns false if a wait ran out.
+template <int BN, int STAGES, int STAGE_BYTES, int B_OFF>
+__device__ __forceinline__ bool build_tokens(const GemmArgs& p, uint8_t* smem, uint64_t* full, uint64_t* empty,
+                                             float* rs, float* ss_red, volatile int* xabort, int c0, int nch,
+                                             int t4) {
+  {
+    // thread (slot, token) sums parts slot, slot + SL, ...; the SL slot sums
+    // are then added in slot order, so the total has a fixed order
+    constexpr int SL = 128 / BN;
+    const int tok = t4 % BN, slot = t4 / BN;
+    float part = 0.f;
+    if (tok < p.n_tok) {
+      for (int q0 = slot; q0 < p.ss_parts; q0 += 4 * SL) {
+        float v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int q = q0 + u * SL;
+          v[u] = q < p.ss_parts ? p.ss_in[q * p.ss_ld + tok] : 0.f;
+        }
+        part += (v[0] + v[1]) + (v[2] + v[3]);
+      }
+    }
+    ss_red[slot * BN + tok] = part;
+    epi_bar();
+    if (t4 < BN) {
+      float r = 0.f;
+      if (t4 < p.n_tok) {
+        float ss = 0.f;
+#pragma unroll
+        for (int q = 0; q < SL; ++q) ss += ss_red[q * BN + t4];
+        r = rsqrtf(ss / static_cast<float>(p.in_ld) + p.in_eps);
+      }
+      rs[t4] = r;
+    }
+    epi_bar();
+  }
+  constexpr int EP = BN / 16;    // (row, 16-byte chunk) items per thread and k-chunk
+  constexpr int CPB = 4 / EP;    // k-chunks per batch of four items
+  for (int i0 = 0; i0 < nch; i0 += CPB) {
+    float4 hv[4][2], gv[4][2];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u / EP, item = t4 + (u % EP) * 128;
+      const int r = item >> 3, j = item & 7;
+      if (i < nch && r < p.n_tok) {
+        const int k = (c0 + i) * kBoxK + j * 8;
+        const float* hr = p.in_h + static_cast<size_t>(p.in_idx ? p.in_idx[r] : r) * p.in_ld + k;
+        hv[u][0] = *reinterpret_cast<const float4*>(hr);
+        hv[u][1] = *reinterpret_cast<const float4*>(hr + 4);
+        gv[u][0] = *reinterpret_cast<const float4*>(p.in_gain + k);
+        gv[u][1] = *reinterpret_cast<const float4*>(p.in_gain + k + 4);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + u / EP, e = u % EP;
+      if (i >= nch) break;   // uniform over the 128 threads
+      const int s = i % STAGES;
+      if (e == 0 && i >= STAGES) {
+        // the slot is reused: wait until the MMAs of k-chunk i - STAGES have read it
+        if (t4 == 0) *xabort = mbar_wait(smem_u32(&empty[s]), ((i / STAGES) & 1) ^ 1u, p.status) ? 0 : 1;
+        epi_bar();
+        if (*xabort) return false;
+      }
+      const int item = t4 + e * 128;
+      const int r = item >> 3, j = item & 7;
+      uint4 w = make_uint4(0u, 0u, 0u, 0u);
+      if (r < p.n_tok) {
+        const float sc = rs[r];
+        const float4 a = hv[u][0], b = hv[u][1], ga = gv[u][0], gb = gv[u][1];
+        w.x = f_to_bf16(a.x * sc * ga.x) | (static_cast<uint32_t>(f_to_bf16(a.y * sc * ga.y)) << 16);
+        w.y = f_to_bf16(a.z * sc * ga.z) | (static_cast<uint32_t>(f_to_bf16(a.w * sc * ga.w)) << 16);
+        w.z = f_to_bf16(b.x * sc * gb.x) | (static_cast<uint32_t>(f_to_bf16(b.y * sc * gb.y)) << 16);
+        w.w = f_to_bf16(b.z * sc * gb.z) | (static_cast<uint32_t>(f_to_bf16(b.w * sc * gb.w)) << 16);
+      }
+      *reinterpret_cast<uint4*>(smem + s * STAGE_BYTES + B_OFF + r * 128 + ((j ^ (r & 7)) << 4)) = w;
+      if (e == EP - 1) {
+        // generic-proxy stores, then visible to the tensor cores' (async-proxy) reads
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        epi_bar();
+        if (t4 == 0) mbar_arrive(smem_u32(&full[s]));
+      }
+    }
+  }
+  return true;
 }
 
 template <int BN, bool DA, bool DB, bool SWAP>
@@ -115,7 +219,11 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
   uint64_t* empty = full + C::kStages;
   uint64_t* done = empty + C::kStages;
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(done + 1);
-  volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort, [1] last-split
+  volatile int* flags = reinterpret_cast<volatile int*>(tmem_slot + 1);  // [0] abort, [1] last-split, [2] x abort
+  uint8_t* tail = smem + C::kStages * C::kStageBytes;
+  float* tok_scale = reinterpret_cast<float*>(tail + 256);   // [BN] input-norm scales
+  float* ssum = reinterpret_cast<float*>(tail + 512);        // [4] per-warp sums of squares
+  const bool in_norm = SWAP && p.in_h != nullptr;
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,7 +234,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&full[s]), in_norm ? 2 : 1);   // + the token builders' arrival
       mbar_init(smem_u32(&empty[s]), 1);
     }
     mbar_init(smem_u32(done), 1);
@@ -182,15 +290,20 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
         else tma_load_2d(smem_u32(st), &tmA0, fb, kx, tile_m * 128);
       }
     };
+    // with an input norm the token operand is built in shared memory, so the
+    // producer moves weights only and never waits on the predecessor grid
+    const uint32_t tx = in_norm ? C::kNA * kABytes : C::kStageBytes;
     const int pre = nch < C::kStages ? nch : C::kStages;
     for (int i = 0; i < pre; ++i) {
       uint8_t* st = smem + i * C::kStageBytes;
       const uint32_t fb = smem_u32(&full[i]);
-      mbar_arrive_expect_tx(fb, C::kStageBytes);
+      mbar_arrive_expect_tx(fb, tx);
       load_w(i, st, fb);
     }
-    pdl_wait();
-    for (int i = 0; i < pre; ++i) load_x(i, smem + i * C::kStageBytes, smem_u32(&full[i]));
+    if (!in_norm) {
+      pdl_wait();
+      for (int i = 0; i < pre; ++i) load_x(i, smem + i * C::kStageBytes, smem_u32(&full[i]));
+    }
     int issued = pre;
     for (int i = pre; i < nch; ++i) {
       const int s = i % C::kStages;
@@ -201,9 +314,9 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
       }
       uint8_t* st = smem + s * C::kStageBytes;
       const uint32_t fb = smem_u32(&full[s]);
-      mbar_arrive_expect_tx(fb, C::kStageBytes);
+      mbar_arrive_expect_tx(fb, tx);
       load_w(i, st, fb);
-      load_x(i, st, fb);
+      if (!in_norm) load_x(i, st, fb);
       ++issued;
     }
     if (flags[0]) {
@@ -246,6 +359,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
     const int q = warp & 3;
     const int row = q * 32 + lane;
     pdl_wait();
+    if (in_norm) {
+      if (!build_tokens<BN, C::kStages, C::kStageBytes, C::kNA * kABytes>(
+              p, smem, full, empty, tok_scale, reinterpret_cast<float*>(tail + 768), flags + 2, c0, nch,
+              (warp - 2) * 32 + lane))
+        flags[0] = 1;
+    }
     const bool ok = mbar_wait(smem_u32(done), 0, p.status);
     __syncwarp();   // tcgen05.ld below is warp-collective (.sync.aligned)
     tc_fence_after();
@@ -350,7 +469,16 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
           v0s += pv0[q];
           v1s += pv1[q];
         }
-        epi_one<SWAP>(p, row, cc, tile_m, tile_n, BN, v0s, v1s);
+        const float hn = epi_one<SWAP>(p, row, cc, tile_m, tile_n, BN, v0s, v1s);
+        if (p.ss_out) {
+          // this tile's share of the token's sum of squares, in a fixed order
+          const float qs = warp_sum(hn * hn);
+          if (lane == 0) ssum[warp - 2] = qs;
+          epi_bar();
+          if (warp == 2 && lane == 0 && cc < p.n_tok)
+            p.ss_out[tile_m * p.ss_ld + cc] = (ssum[0] + ssum[1]) + (ssum[2] + ssum[3]);
+          epi_bar();
+        }
       }
     }
     cluster.sync();
@@ -393,8 +521,14 @@ cudaError_t launch_one(const GemmLaunch& g, cudaStream_t stream) {
 
 template <int BN, bool DA, bool DB, bool SWAP>
 cudaError_t set_attr() {
-  return cudaFuncSetAttribute(k_gemm_tc<BN, DA, DB, SWAP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Cfg<BN, DA, DB>::kSmemBytes);
+  auto kern = k_gemm_tc<BN, DA, DB, SWAP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN, DA, DB>::kSmemBytes);
+  // all of the SM's unified L1/shared storage as shared memory, so two skinny CTAs are resident
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+  // split-K clusters of the skinny orientation may hold up to 16 CTAs
+  if (e == cudaSuccess && SWAP) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return e;
 }
 
 }  // namespace

@@ -41,6 +41,21 @@ struct GemmArgs {
   int cluster;      // split-K through a (1,1,splits) cluster and distributed shared memory
                     // instead of global partials and tickets (splits <= kMaxClusterSplits)
   int* status;
+  // Sums of squares for the next RMSNorm, written by a residual epilogue of the
+  // cluster split-K path: ss_out[tile_m * ss_ld + tok] = sum over the tile's
+  // 128 features of the updated h[r_tok][feat]^2 (nullptr: not written).
+  float* ss_out;
+  int ss_ld;
+  // Input RMSNorm (swap orientation): the token operand is built in shared
+  // memory from fp32 hidden rows instead of loaded by TMA:
+  //   x[t][k] = bf16(h[r_t][k] * rsqrt(sum_p ss_in[p * ss_ld + t] / K + in_eps) * in_gain[k])
+  // with r_t = in_idx ? in_idx[t] : t, p < ss_parts, and zero rows t >= n_tok.
+  const float* in_h;   // nullptr: TMA operand
+  const int* in_idx;
+  const float* in_gain;
+  const float* ss_in;
+  int in_ld, ss_parts;
+  float in_eps;
 };
 
 struct GemmLaunch {
@@ -55,7 +70,7 @@ struct GemmLaunch {
   bool pdl = false;        // launched as a programmatic dependent of the previous kernel
 };
 
-constexpr int kMaxClusterSplits = 8;  // portable cluster size
+constexpr int kMaxClusterSplits = 16;  // non-portable cluster size, opted in per kernel
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream);
 
 // Launch a kernel, with programmatic stream serialisation when `pdl` is set

@@ -215,11 +215,19 @@ __device__ __forceinline__ uint16_t quantize_lane(const float* r, int g, int bit
   const int qm = (1 << (bits - 1)) - 1;
   const __half sh = __float2half_ru(__fdiv_rn(am, static_cast<float>(qm)));
   const float s = __half2float(sh);
+  // code = rint of the correctly rounded quotient r/s.  r * (1/s), with 1/s
+  // correctly rounded, is within 2 ulp of that quotient (|r/s| <= qmax + tiny,
+  // so an ulp is at most 2^-21); the nearest integers can differ only when the
+  // product lies within a few ulp of a half-integer, and only then is the
+  // quotient computed exactly.
+  const float inv = s > 0.f ? __frcp_rn(s) : 0.f;
 #pragma unroll
   for (int e = 0; e < EPL; ++e) {
     int c = 0;
     if (s > 0.f) {
-      c = __float2int_rn(__fdiv_rn(r[e], s));
+      float q = r[e] * inv;
+      if (fabsf(q - (floorf(q) + 0.5f)) <= 0x1p-18f) q = __fdiv_rn(r[e], s);
+      c = __float2int_rn(q);
       c = c > qm ? qm : (c < -qm ? -qm : c);
     }
     code[e] = c;
@@ -250,25 +258,44 @@ __device__ __forceinline__ void store_lane_codes(uint8_t* row, int bits, int lan
 }
 
 template <int EPL>
-__global__ void __launch_bounds__(128) k_quantize_rows(const float* __restrict__ r, int rows, int width, int g,
+__global__ void __launch_bounds__(256) k_quantize_rows(const float* __restrict__ r, int rows, int width, int g,
                                                        int bits, uint8_t* __restrict__ codes,
                                                        uint16_t* __restrict__ scales) {
   pdl_trigger();
   pdl_wait();
-  const int warp_global = blockIdx.x * 4 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  constexpr int PER = 4;   // row chunks per warp, loaded together
+  const int lane = threadIdx.x & 31;
   const int chunks = width / (32 * EPL);
-  if (warp_global >= rows * chunks) return;
-  const int row = warp_global / chunks, ch = warp_global % chunks;
-  const float* src = r + static_cast<size_t>(row) * width + ch * 32 * EPL + lane * EPL;
-  float v[EPL];
+  const long long total = static_cast<long long>(rows) * chunks;
+  const long long w0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * PER;
+  float v[PER][EPL];
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) v[e] = src[e];
-  int c[EPL];
-  const uint16_t s = quantize_lane<EPL>(v, g, bits, c);
-  uint8_t* crow = codes + (static_cast<size_t>(row) * width + ch * 32 * EPL) * bits / 8;
-  store_lane_codes<EPL>(crow, bits, lane, c);
+  for (int u = 0; u < PER; ++u) {
+    const long long w = w0 + u;
+    if (w < total) {
+      const int row = static_cast<int>(w / chunks), ch = static_cast<int>(w % chunks);
+      const float* src = r + static_cast<size_t>(row) * width + ch * 32 * EPL + lane * EPL;
+      if (EPL == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        v[u][0] = x.x; v[u][EPL > 1 ? 1 : 0] = x.y; v[u][EPL > 2 ? 2 : 0] = x.z; v[u][EPL > 3 ? 3 : 0] = x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(src);
+        v[u][0] = x.x; v[u][EPL > 1 ? 1 : 0] = x.y;
+      }
+    }
+  }
   const int GL = g / EPL;
-  if ((lane % GL) == 0) scales[static_cast<size_t>(row) * (width / g) + (ch * 32 * EPL) / g + lane / GL] = s;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    const long long w = w0 + u;
+    if (w >= total) break;   // warp-uniform
+    const int row = static_cast<int>(w / chunks), ch = static_cast<int>(w % chunks);
+    int c[EPL];
+    const uint16_t sc = quantize_lane<EPL>(v[u], g, bits, c);
+    uint8_t* crow = codes + (static_cast<size_t>(row) * width + ch * 32 * EPL) * bits / 8;
+    store_lane_codes<EPL>(crow, bits, lane, c);
+    if ((lane % GL) == 0) scales[static_cast<size_t>(row) * (width / g) + (ch * 32 * EPL) / g + lane / GL] = sc;
+  }
 }
 
 // ============================================================================
@@ -363,17 +390,9 @@ __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
   if ((lane % GL) == 0) cv.scale_row(a.j, a.loop, kv, b, gk, t)[lane / GL] = s;
 }
 
-// ============================================================================
-// decode attention over one cache (lazy base at loop 1, or the dense
-// baseline's own per-loop KV): grid (n*Hkv, splits), 256 threads.  Each CTA
-// takes the group's query heads over one column range in 64-column tiles;
-// K/V tiles are double-buffered in shared memory with cp.async so the next
-// tile streams in while the current one is scored and accumulated.  The last
-// CTA of a (token, KV head) -- an atomic ticket, no waiting -- merges the
-// splits' (max, sum, unnormalised output) and writes O, lse.
-// ============================================================================
 constexpr int kDecTile = 64;
-constexpr int kDecPad = 8;  // bf16 elements of padding per staged row (16-byte skew)
+constexpr int kDecPad = 8;     // bf16 elements of padding per staged row (16-byte skew)
+constexpr int kDecStages = 3;  // K/V tiles in flight per CTA (two CTAs per SM)
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -382,214 +401,344 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-template <int HD, int GRP>
-__global__ void __launch_bounds__(256) k_attn_decode(const AttnDecArgs a) {
-  pdl_trigger();
-  pdl_wait();
-  constexpr int RS = HD + kDecPad;
-  constexpr int CH = HD / 8;         // 16-byte chunks per row
-  constexpr int DQ = HD / 4;         // dims per quarter (score phase)
-  constexpr int NP = HD / 2;         // dim pairs (PV phase)
-  constexpr int CQ = 256 / NP;       // column groups of the PV phase: 4 (hd 128) or 8 (hd 64)
-  extern __shared__ __align__(16) uint8_t sm[];
-  uint16_t* Kst = reinterpret_cast<uint16_t*>(sm);          // [2][64][RS]
-  uint16_t* Vst = Kst + 2 * kDecTile * RS;                  // [2][64][RS]
-  __shared__ __align__(16) float Qs[GRP * HD];
-  __shared__ __align__(16) float S[kDecTile][GRP];   // column-major: one vector load gives every head
-  __shared__ float m_run[GRP], l_run[GRP], alpha[GRP];
-  __shared__ float red[CQ][GRP][HD];
-  __shared__ float sm_m[GRP], sm_l[GRP];
-  __shared__ int is_last;
+// ---- warp-level tensor-core helpers for the decode attention
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t* r) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// D[16x8] += A[16x16] * B[16x8], bf16 operands, fp32 accumulate
+__device__ __forceinline__ void mma_bf16_16816(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  return static_cast<uint32_t>(f_to_bf16(lo)) | (static_cast<uint32_t>(f_to_bf16(hi)) << 16);
+}
+// x ~= hi + lo with hi = bf16(x), lo = bf16(x - hi): a product of a bf16 value
+// with hi and lo, summed in fp32, carries about 16 significant bits of x
+__device__ __forceinline__ void split_bf16(float x, float& hi, float& lo) {
+  hi = bf16_to_f(f_to_bf16(x));
+  lo = x - hi;
+}
 
+// ============================================================================
+// decode attention over one cache (lazy base at loop 1, or the dense
+// baseline's own per-loop KV): grid (n*Hkv, splits), 128 threads (4 warps).
+// Each CTA takes the group's query heads (<= 8) over a range of 64-column
+// tiles.  K/V tiles arrive by TMA (128-byte swizzle) in a ring of kDecStages.
+// Scores S = tau * K q^T and the update O += P V are warp-level bf16 tensor-core
+// products with fp32 accumulation: q and P are carried as hi + lo bf16 pairs
+// (the lo half of P rides in the spare rows of the 16-row operand), the cache
+// values are bf16 already, so the products keep about fp32 accuracy.  The
+// online softmax runs on the score fragments.  The last CTA of a (token, KV
+// head) -- an atomic ticket, no waiting -- merges the splits' (max, sum,
+// unnormalised output) and writes O, lse.
+// ============================================================================
+template <int HD, int GRP>
+__global__ void __launch_bounds__(128, 2) k_attn_decode(const __grid_constant__ CUtensorMap kvmap, const AttnDecArgs a) {
+  constexpr int NB = HD / 64;                       // 128-byte TMA boxes per row
+  constexpr int BOX_BYTES = kDecTile * 128;         // one box of a 64-row tile
+  constexpr int TILE_BYTES = NB * BOX_BYTES;        // K or V of one tile
+  constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  constexpr int KSTEPS = HD / 16;                   // k-steps of the score product
+  constexpr int NTW = HD / 32;                      // 8-dim output tiles per warp
+  static_assert(GRP <= 8 && NTW % 2 == 0, "decode attention shape");
+  extern __shared__ uint8_t sm_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[kDecStages];
+  __shared__ __align__(128) uint16_t Pt[16 * 64];   // P^T operand: rows hi heads 0-7, lo heads 0-7; 64 columns
+  __shared__ float red_max[4][8];
+  __shared__ float alpha_s[8];
+  __shared__ float red_l[4][8];
+  __shared__ float sm_m[8], sm_l[8];
+  __shared__ int flag;
+
+  pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int i = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv, sp = blockIdx.y;
+  if (tid == 0) {
+    for (int s = 0; s < kDecStages; ++s) mbar_init(smem_u32(&full[s]), 1);
+    fence_mbar_init();
+    flag = 0;
+  }
+  pdl_wait();
   const int tok = a.idx ? a.idx[i] : i;
   const int b = a.seq[tok], P = a.pos[tok];
-  const int c_begin = sp * a.split_len;
-  const int c_end = min(c_begin + a.split_len, P + 1);
+  const int ncols = P + 1;
+  const int nt = (ncols + kDecTile - 1) / kDecTile;
+  const int t_begin = static_cast<int>((static_cast<long long>(sp) * nt) / a.n_splits);
+  const int t_end = static_cast<int>((static_cast<long long>(sp + 1) * nt) / a.n_splits);
+  const int ntiles = t_end - t_begin;
   const CacheView& cv = a.cv;
-  const uint16_t* kbase = a.dense ? cv.dense_row(a.j, a.loop, 0, b, g, 0) : cv.base_row(a.j, 0, b, g, 0);
-  const uint16_t* vbase = a.dense ? cv.dense_row(a.j, a.loop, 1, b, g, 0) : cv.base_row(a.j, 1, b, g, 0);
-
-  for (int e = tid; e < GRP * HD; e += 256) Qs[e] = a.q_cur[(static_cast<size_t>(i) * a.H + g * GRP) * HD + e];
-  if (tid < GRP) {
-    m_run[tid] = -INFINITY;
-    l_run[tid] = 0.f;
-  }
-  // PV phase: thread -> dim pair dp, column group cq; all GRP heads
-  const int dp = tid % NP, cq = tid / NP;
-  float acc[GRP][2];
+  // first row of this (layer, loop, K/V, sequence, KV head) in the 2-D [rows][hd] view of the cache
+  const size_t bh = static_cast<size_t>(b) * cv.Hkv + g;
+  const size_t plane = static_cast<size_t>(cv.B) * cv.Hkv * cv.T;
+  const size_t rk = a.dense ? ((static_cast<size_t>(a.j) * cv.K + (a.loop - 1)) * 2) * plane + bh * cv.T
+                            : (static_cast<size_t>(a.j) * 2) * plane + bh * cv.T;
+  const int row_k = static_cast<int>(rk), row_v = static_cast<int>(rk + plane);
+  __syncthreads();   // barrier initialisation visible to every thread
+  auto issue = [&](int u) {
+    const int s = u % kDecStages;
+    const int y = (t_begin + u) * kDecTile;
+    uint8_t* st = ring + s * STAGE_BYTES;
+    const uint32_t fb = smem_u32(&full[s]);
+    mbar_arrive_expect_tx(fb, STAGE_BYTES);
 #pragma unroll
-  for (int h = 0; h < GRP; ++h) acc[h][0] = acc[h][1] = 0.f;
-
-  auto stage = [&](int buf, int c0) {
-    const int nc = min(kDecTile, c_end - c0);
-    for (int e = tid; e < kDecTile * CH; e += 256) {
-      const int r = e / CH, cc = e % CH;
-      const bool in = r < nc;
-      const size_t off = static_cast<size_t>(in ? c0 + r : c0) * HD + cc * 8;
-      cp_async16(smem_u32(Kst + (buf * kDecTile + r) * RS + cc * 8), kbase + off, in ? 16u : 0u);
-      cp_async16(smem_u32(Vst + (buf * kDecTile + r) * RS + cc * 8), vbase + off, in ? 16u : 0u);
+    for (int bx = 0; bx < NB; ++bx) {
+      tma_load_2d(smem_u32(st + bx * BOX_BYTES), &kvmap, fb, bx * 64, row_k + y);
+      tma_load_2d(smem_u32(st + TILE_BYTES + bx * BOX_BYTES), &kvmap, fb, bx * 64, row_v + y);
     }
-    cp_async_commit();
   };
+  if (tid == 0) {
+    tma_prefetch_desc(&kvmap);
+    for (int u = 0; u < kDecStages && u < ntiles; ++u) issue(u);
+  }
 
-  const int n_tiles = c_end > c_begin ? (c_end - c_begin + kDecTile - 1) / kDecTile : 0;
-  if (n_tiles > 0) stage(0, c_begin);
-  __syncthreads();
-  for (int t = 0; t < n_tiles; ++t) {
-    const int buf = t & 1;
-    const int c0 = c_begin + t * kDecTile;
-    const int nc = min(kDecTile, c_end - c0);
-    if (t + 1 < n_tiles) {
-      stage(buf ^ 1, c0 + kDecTile);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
+  // q^T as the B operand of the score product (k = dims, n = heads), tau folded
+  // in, split into hi and lo bf16 parts: lane holds head lane/4, dims 2(lane%4)+{0,1,8,9}
+  uint32_t qb_hi[KSTEPS][2], qb_lo[KSTEPS][2];
+  {
+    const int hn = lane >> 2;
+    const float* qh = a.q_cur + (static_cast<size_t>(i) * a.H + g * GRP + (hn < GRP ? hn : 0)) * HD;
+#pragma unroll
+    for (int ks = 0; ks < KSTEPS; ++ks) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int d = ks * 16 + 2 * (lane & 3) + r * 8;
+        float x0 = hn < GRP ? qh[d] * a.tau : 0.f, x1 = hn < GRP ? qh[d + 1] * a.tau : 0.f;
+        float h0, l0, h1, l1;
+        split_bf16(x0, h0, l0);
+        split_bf16(x1, h1, l1);
+        qb_hi[ks][r] = pack_bf16x2(h0, h1);
+        qb_lo[ks][r] = pack_bf16x2(l0, l1);
+      }
     }
+  }
+  // online-softmax state of this thread's two heads (2(lane%4), +1); every
+  // thread tracks the running maxima, the sums are per-thread partials
+  const int h0 = 2 * (lane & 3);
+  float m_run[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.f, 0.f};
+  float acc[NTW][4];
+#pragma unroll
+  for (int n = 0; n < NTW; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  const uint32_t pt_base = smem_u32(Pt);
+
+  int u_stop = ntiles;
+  for (int u = 0; u < ntiles; ++u) {
+    const int s = u % kDecStages;
+    if (tid == 0) flag = mbar_wait(smem_u32(&full[s]), (u / kDecStages) & 1, a.status) ? 0 : 1;
     __syncthreads();
-    const uint16_t* Ks = Kst + buf * kDecTile * RS;
-    const uint16_t* Vs = Vst + buf * kDecTile * RS;
-    // scores: lane -> column warp*8 + lane%8, dim quarter lane/8, every head.  A
-    // quarter-warp reads eight consecutive staged rows (distinct banks) and one
-    // broadcast q chunk; the four quarters are summed by shuffles.
+    if (flag) {
+      u_stop = u;
+      break;
+    }
+    mbar_try_wait(smem_u32(&full[s]), (u / kDecStages) & 1);   // completed: acquire the tile for this thread
+    const uint32_t Kt = smem_u32(ring + s * STAGE_BYTES);
+    const uint32_t Vt = Kt + TILE_BYTES;
+    const int nc = min(kDecTile, ncols - (t_begin + u) * kDecTile);
+    // ---- scores of this warp's 16 columns (rows of the product) x 8 heads
+    float sc[4];
     {
-      const int c = warp * 8 + (lane & 7), qd = lane >> 3;
-      float dot[GRP];
+      // four independent accumulation chains (hi / lo parts x even / odd k-steps), summed at the end
+      float s4[4][4] = {};
+      const int r = warp * 16 + (lane & 15);   // column row of the K tile this lane addresses
 #pragma unroll
-      for (int h = 0; h < GRP; ++h) dot[h] = 0.f;
-      const uint16_t* kr = Ks + c * RS + qd * DQ;
-#pragma unroll
-      for (int e = 0; e < DQ; e += 8) {
-        const uint4 u = *reinterpret_cast<const uint4*>(kr + e);
-        const float k0 = __uint_as_float(u.x << 16), k1 = __uint_as_float(u.x & 0xFFFF0000u);
-        const float k2 = __uint_as_float(u.y << 16), k3 = __uint_as_float(u.y & 0xFFFF0000u);
-        const float k4 = __uint_as_float(u.z << 16), k5 = __uint_as_float(u.z & 0xFFFF0000u);
-        const float k6 = __uint_as_float(u.w << 16), k7 = __uint_as_float(u.w & 0xFFFF0000u);
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) {
-          const float4 qa = *reinterpret_cast<const float4*>(&Qs[h * HD + qd * DQ + e]);
-          const float4 qb = *reinterpret_cast<const float4*>(&Qs[h * HD + qd * DQ + e + 4]);
-          dot[h] += qa.x * k0 + qa.y * k1 + qa.z * k2 + qa.w * k3 + qb.x * k4 + qb.y * k5 + qb.z * k6 + qb.w * k7;
-        }
+      for (int ks = 0; ks < KSTEPS; ++ks) {
+        const int q = ks * 2 + (lane >> 4);   // 16-byte chunk (8 dims)
+        uint32_t af[4];
+        ldsm_x4(Kt + (q >> 3) * BOX_BYTES + r * 128 + (((q & 7) ^ (r & 7)) << 4), af);
+        mma_bf16_16816(s4[(ks & 1) * 2], af, qb_hi[ks][0], qb_hi[ks][1]);
+        mma_bf16_16816(s4[(ks & 1) * 2 + 1], af, qb_lo[ks][0], qb_lo[ks][1]);
       }
 #pragma unroll
-      for (int h = 0; h < GRP; ++h) {
-        float v = dot[h];
-        v += __shfl_xor_sync(0xffffffffu, v, 8);
-        v += __shfl_xor_sync(0xffffffffu, v, 16);
-        if (qd == 0) S[c][h] = c < nc ? v * a.tau : -INFINITY;
-      }
+      for (int e = 0; e < 4; ++e) sc[e] = (s4[0][e] + s4[2][e]) + (s4[1][e] + s4[3][e]);
+    }
+    // fragment: sc[0..1] column c0 = warp*16 + lane/4, heads h0, h0+1; sc[2..3] column c0 + 8
+    const int c0 = warp * 16 + (lane >> 2), c1 = c0 + 8;
+    if (c0 >= nc) sc[0] = sc[1] = -INFINITY;
+    if (c1 >= nc) sc[2] = sc[3] = -INFINITY;
+    float tm0 = fmaxf(sc[0], sc[2]), tm1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      tm0 = fmaxf(tm0, __shfl_xor_sync(0xffffffffu, tm0, o));
+      tm1 = fmaxf(tm1, __shfl_xor_sync(0xffffffffu, tm1, o));
+    }
+    if (lane < 4) {
+      red_max[warp][h0] = tm0;
+      red_max[warp][h0 + 1] = tm1;
     }
     __syncthreads();
-    // online softmax per head: warp h handles head h
-    for (int h = warp; h < GRP; h += 8) {
-      const float s0 = S[lane][h], s1 = S[lane + 32][h];
-      const float tmax = warp_max(fmaxf(s0, s1));
-      const float mnew = fmaxf(m_run[h], tmax);
-      const float p0 = s0 == -INFINITY ? 0.f : expf(s0 - mnew);
-      const float p1 = s1 == -INFINITY ? 0.f : expf(s1 - mnew);
-      const float psum = warp_sum(p0 + p1);
-      S[lane][h] = p0;
-      S[lane + 32][h] = p1;
-      __syncwarp();
-      if (lane == 0) {
-        const float al = m_run[h] == -INFINITY ? 0.f : expf(m_run[h] - mnew);
-        alpha[h] = al;
-        l_run[h] = l_run[h] * al + psum;
-        m_run[h] = mnew;
-      }
+    float mn[2], al[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const float tmx = fmaxf(fmaxf(red_max[0][h0 + e], red_max[1][h0 + e]), fmaxf(red_max[2][h0 + e], red_max[3][h0 + e]));
+      mn[e] = fmaxf(m_run[e], tmx);
+      al[e] = m_run[e] == -INFINITY ? 0.f : expf(m_run[e] - mn[e]);
+      m_run[e] = mn[e];
+    }
+    float p[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) p[e] = sc[e] == -INFINITY ? 0.f : expf(sc[e] - mn[e & 1]);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) l_part[e] = l_part[e] * al[e] + (p[e] + p[e + 2]);
+    if (lane < 4) {
+      alpha_s[h0] = al[0];
+      alpha_s[h0 + 1] = al[1];
+    }
+    // P^T rows: hi part of head h at row h, lo part at row 8 + h; column c
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int hh = h0 + (e & 1), c = (e < 2) ? c0 : c1;
+      float ph, pl;
+      split_bf16(p[e], ph, pl);
+      const int rh = hh, rl = 8 + hh;
+      Pt[rh * 64 + ((((c >> 3) ^ (rh & 7)) << 3) | (c & 7))] = f_to_bf16(ph);
+      Pt[rl * 64 + ((((c >> 3) ^ (rl & 7)) << 3) | (c & 7))] = f_to_bf16(pl);
     }
     __syncthreads();
-    // PV: this thread's dim pair over its column group, every head
+    // ---- O[16 rows (hi/lo heads) x this warp's HD/4 dims] += P^T V
+    const float arow = alpha_s[lane >> 2];
 #pragma unroll
-    for (int h = 0; h < GRP; ++h) {
-      acc[h][0] *= alpha[h];
-      acc[h][1] *= alpha[h];
+    for (int n = 0; n < NTW; ++n) {
+      acc[n][0] *= arow;
+      acc[n][1] *= arow;
+      acc[n][2] *= arow;
+      acc[n][3] *= arow;
     }
-    for (int c = cq; c < kDecTile; c += CQ) {
-      const uint32_t u = *reinterpret_cast<const uint32_t*>(Vs + c * RS + 2 * dp);
-      const float v0 = __uint_as_float(u << 16), v1 = __uint_as_float(u & 0xFFFF0000u);
-      float p[GRP];
-      if (GRP % 4 == 0) {
 #pragma unroll
-        for (int h = 0; h < GRP; h += 4) {
-          const float4 q4 = *reinterpret_cast<const float4*>(&S[c][h]);
-          p[h] = q4.x; p[(h + 1) % GRP] = q4.y; p[(h + 2) % GRP] = q4.z; p[(h + 3) % GRP] = q4.w;
-        }
-      } else {
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) p[h] = S[c][h];
+    for (int ks = 0; ks < 4; ++ks) {   // 16 columns per step
+      uint32_t pf[4];
+      {
+        const int r = lane & 15, q = ks * 2 + (lane >> 4);
+        ldsm_x4(pt_base + r * 128 + ((q ^ (r & 7)) << 4), pf);
       }
+      const int vr = ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;   // V row (column index)
 #pragma unroll
-      for (int h = 0; h < GRP; ++h) {
-        acc[h][0] += p[h] * v0;
-        acc[h][1] += p[h] * v1;
+      for (int n2 = 0; n2 < NTW / 2; ++n2) {
+        const int q = (warp * NTW + n2 * 2 + (lane >> 4));   // 8-dim chunk of this lane's address
+        uint32_t vf[4];
+        ldsm_x4_t(Vt + (q >> 3) * BOX_BYTES + vr * 128 + (((q & 7) ^ (vr & 7)) << 4), vf);
+        mma_bf16_16816(acc[n2 * 2], pf, vf[0], vf[1]);
+        mma_bf16_16816(acc[n2 * 2 + 1], pf, vf[2], vf[3]);
       }
     }
+    __syncthreads();   // the slot and P^T are free again
+    if (tid == 0 && u + kDecStages < ntiles) issue(u + kDecStages);
+  }
+  if (u_stop < ntiles) {
+    // a tile never arrived: let the copies still in flight land (bounded) before the CTA exits
+    if (tid == 0)
+      for (int u = u_stop; u < ntiles && u < u_stop + kDecStages; ++u)
+        mbar_wait(smem_u32(&full[u % kDecStages]), (u / kDecStages) & 1, nullptr);
     __syncthreads();
   }
-  // sum the column groups, then write this split's partial (m, l, unnormalised o)
+  // ---- this split's partial: per-head maxima (identical in every thread),
+  // sums over all threads, unnormalised output = hi row + lo row
 #pragma unroll
-  for (int h = 0; h < GRP; ++h) {
-    red[cq][h][2 * dp] = acc[h][0];
-    red[cq][h][2 * dp + 1] = acc[h][1];
+  for (int e = 0; e < 2; ++e) {
+    float l = l_part[e];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane < 4) red_l[warp][h0 + e] = l;
+  }
+  if (warp == 0 && lane < 4) {
+    sm_m[h0] = m_run[0];
+    sm_m[h0 + 1] = m_run[1];
   }
   __syncthreads();
+  if (tid < GRP) sm_l[tid] = (red_l[0][tid] + red_l[1][tid]) + (red_l[2][tid] + red_l[3][tid]);
+  const int hh = lane >> 2;
   const size_t pbase = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits + sp;
-  for (int e = tid; e < GRP * HD; e += 256) {
-    const int h = e / HD, d = e % HD;
-    float o = 0.f;
+  if (hh < GRP) {
 #pragma unroll
-    for (int q = 0; q < CQ; ++q) o += red[q][h][d];
-    a.part_o[(pbase * 8 + h) * HD + d] = o;
+    for (int n = 0; n < NTW; ++n) {
+      const int d = (warp * NTW + n) * 8 + 2 * (lane & 3);
+      float* dst = a.part_o + (pbase * 8 + hh) * HD + d;
+      dst[0] = acc[n][0] + acc[n][2];
+      dst[1] = acc[n][1] + acc[n][3];
+    }
   }
+  __syncthreads();
   if (tid < GRP) {
-    a.part_ml[(pbase * 8 + tid) * 2 + 0] = m_run[tid];
-    a.part_ml[(pbase * 8 + tid) * 2 + 1] = l_run[tid];
+    a.part_ml[(pbase * 8 + tid) * 2 + 0] = sm_m[tid];
+    a.part_ml[(pbase * 8 + tid) * 2 + 1] = sm_l[tid];
   }
   __threadfence();
   __syncthreads();
   if (tid == 0) {
     const int old = atomicAdd(&a.counters[i * a.Hkv + g], 1);
-    is_last = (old == a.n_splits - 1);
+    flag = (old == a.n_splits - 1);
   }
   __syncthreads();
-  if (!is_last) return;
+  if (!flag) return;
   __threadfence();
+  // merge in two rounds of loads: every split's (max, sum) at once, then every
+  // split's output for this thread's elements at once
   const size_t q0 = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits;
-  // merge: warp h finds head h's maximum and total over the splits (lanes over splits)
-  for (int h = warp; h < GRP; h += 8) {
-    float M = -INFINITY;
-    for (int s2 = lane; s2 < a.n_splits; s2 += 32) M = fmaxf(M, __ldcg(&a.part_ml[((q0 + s2) * 8 + h) * 2]));
-    M = warp_max(M);
-    float L = 0.f;
-    for (int s2 = lane; s2 < a.n_splits; s2 += 32) {
-      const float ms = __ldcg(&a.part_ml[((q0 + s2) * 8 + h) * 2]);
-      if (ms != -INFINITY) L += expf(ms - M) * __ldcg(&a.part_ml[((q0 + s2) * 8 + h) * 2 + 1]);
-    }
-    L = warp_sum(L);
-    if (lane == 0) {
-      sm_m[h] = M;
-      sm_l[h] = L;
-    }
+  float* ml = reinterpret_cast<float*>(ring);   // [splits][GRP][2], then weights
+  const int S = a.n_splits;
+  for (int e = tid; e < S * GRP; e += 128) {
+    const int s2 = e / GRP, h = e % GRP;
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(&a.part_ml[((q0 + s2) * 8 + h) * 2]));
+    ml[e * 2] = v.x;
+    ml[e * 2 + 1] = v.y;
   }
   __syncthreads();
-  for (int e = tid; e < GRP * HD; e += 256) {
-    const int h = e / HD, d = e % HD;
-    const float M = sm_m[h];
-    float o = 0.f;
-#pragma unroll 8
-    for (int s2 = 0; s2 < a.n_splits; ++s2) {
-      const float ms = __ldcg(&a.part_ml[((q0 + s2) * 8 + h) * 2]);
-      const float po = __ldcg(&a.part_o[((q0 + s2) * 8 + h) * HD + d]);
-      o += ms == -INFINITY ? 0.f : expf(ms - M) * po;
+  if (tid < GRP) {
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, ml[(s2 * GRP + tid) * 2]);
+    float L = 0.f;
+    for (int s2 = 0; s2 < S; ++s2) {
+      const float ms = ml[(s2 * GRP + tid) * 2];
+      const float w = ms == -INFINITY ? 0.f : expf(ms - M);
+      ml[(s2 * GRP + tid) * 2] = w;   // the split's weight replaces its maximum
+      L += w * ml[(s2 * GRP + tid) * 2 + 1];
     }
+    sm_m[tid] = M;
+    sm_l[tid] = L;
+  }
+  __syncthreads();
+  constexpr int EPT = (GRP * HD + 127) / 128;           // output elements per thread
+  constexpr int MB = 64 / EPT < 16 ? 64 / EPT : 16;      // splits whose outputs are requested together
+  float o[EPT];
+#pragma unroll
+  for (int t = 0; t < EPT; ++t) o[t] = 0.f;
+  for (int s0 = 0; s0 < S; s0 += MB) {
+    float pv[EPT][MB];
+#pragma unroll
+    for (int t = 0; t < EPT; ++t) {
+      const int e = tid + t * 128, h = e / HD, d = e % HD;
+#pragma unroll
+      for (int u = 0; u < MB; ++u)
+        pv[t][u] = (e < GRP * HD && s0 + u < S) ? __ldcg(&a.part_o[((q0 + s0 + u) * 8 + h) * HD + d]) : 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < EPT; ++t) {
+      const int e = tid + t * 128, h = e < GRP * HD ? e / HD : 0;
+#pragma unroll
+      for (int u = 0; u < MB; ++u)
+        if (s0 + u < S) o[t] += ml[((s0 + u) * GRP + h) * 2] * pv[t][u];
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < EPT; ++t) {
+    const int e = tid + t * 128;
+    if (e >= GRP * HD) break;
+    const int h = e / HD, d = e % HD;
     const int hq = g * GRP + h;
-    const float ov = o / sm_l[h];
+    const float ov = o[t] / sm_l[h];
     if (a.o_state) a.o_state[(static_cast<size_t>(tok) * a.H + hq) * HD + d] = ov;
     a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + d] = f_to_bf16(ov);
-    if (d == 0 && a.lse_state) a.lse_state[static_cast<size_t>(tok) * a.H + hq] = M + logf(sm_l[h]);
+    if (d == 0 && a.lse_state) a.lse_state[static_cast<size_t>(tok) * a.H + hq] = sm_m[h] + logf(sm_l[h]);
   }
   if (tid == 0) a.counters[i * a.Hkv + g] = 0;
 }
@@ -862,25 +1011,31 @@ __global__ void __launch_bounds__(1024) k_plan_tiles(const int32_t* __restrict__
   block_plan(idx, n_sel, tile, has_c, plan);
 }
 
-// One lazy loop's token bookkeeping for a call of at most blockDim.x tokens
-// (decode), in one CTA: the change keys of the previous loop (against h_in
-// after loop 1, against the selected rows' snapshot after a lazy loop, zero for
-// carried tokens), the previously selected tokens' `last` and tile flags, the
-// top-n_sel selection (or the forced one), the selection slots, the snapshot
-// of the selected rows and the query-tile plan.
+// One lazy loop's token bookkeeping for a call of at most kSelectStepMax tokens
+// (decode, short prefills), in one CTA: the change keys of the previous loop
+// (against h_in after loop 1, against the selected rows' snapshot after a lazy
+// loop, zero for carried tokens), the previously selected tokens' `last` and
+// tile flags, the top-n_sel selection (or the forced one), the selection slots,
+// the snapshot of the selected rows, optionally the first layer's input norm,
+// and the query-tile plan.  Keys, the selection, tiles, slots and tile flags
+// stay in shared memory, so the dependent steps do not go back to global memory.
 __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
   pdl_trigger();
   pdl_wait();
+  __shared__ float s_key[kSelectStepMax];
+  __shared__ int32_t s_idx[kSelectStepMax];
+  __shared__ int s_tile[kSelectStepMax], s_slot[kSelectStepMax], s_hasc[kSelectStepMax];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int t = threadIdx.x; t < a.N; t += blockDim.x) {
+    s_tile[t] = a.tile[t];
+    s_slot[t] = a.loop == 2 ? -1 : a.sel_slot[t];
+  }
+  for (int t = threadIdx.x; t < a.n_tiles; t += blockDim.x) s_hasc[t] = a.has_c[t];
+  __syncthreads();
   for (int t = warp; t < a.N; t += nw) {
-    const float* other = nullptr;
-    int slot = -1;
-    if (a.loop == 2) {
-      other = a.h_in + static_cast<size_t>(t) * a.d;
-    } else {
-      slot = a.sel_slot[t];
-      if (slot >= 0) other = a.h_snap + static_cast<size_t>(slot) * a.d;
-    }
+    const int slot = s_slot[t];
+    const float* other = a.loop == 2 ? a.h_in + static_cast<size_t>(t) * a.d
+                                     : (slot >= 0 ? a.h_snap + static_cast<size_t>(slot) * a.d : nullptr);
     float acc = 0.f;
     if (other) {
       const float* hr = a.h + static_cast<size_t>(t) * a.d;
@@ -893,38 +1048,62 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
       acc = warp_sum(acc);
     }
     if (lane == 0) {
+      s_key[t] = acc;
       a.key[t] = acc;
       a.keys_trace[t] = acc;
       if (slot >= 0) {
         a.last[t] = a.loop - 1;
-        a.has_c[a.tile[t]] = 1;
+        s_hasc[s_tile[t]] = 1;
+        a.has_c[s_tile[t]] = 1;
       }
     }
   }
   __syncthreads();
   if (a.forced_on && a.forced_on[0]) {
-    for (int i = threadIdx.x; i < a.n_sel; i += blockDim.x) a.idx[i] = a.forced[i];
-    __syncthreads();
+    for (int i = threadIdx.x; i < a.n_sel; i += blockDim.x) s_idx[i] = a.forced[i];
   } else {
-    block_topk(a.key, a.N, a.n_sel, a.idx);
+    block_topk(s_key, a.N, a.n_sel, s_idx);
   }
   __syncthreads();
+  for (int i = threadIdx.x; i < a.n_sel; i += blockDim.x) a.idx[i] = s_idx[i];
   for (int t = threadIdx.x; t < a.N; t += blockDim.x) {
     int lo = 0, hi = a.n_sel;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if (a.idx[mid] < t) lo = mid + 1; else hi = mid;
+      if (s_idx[mid] < t) lo = mid + 1; else hi = mid;
     }
-    a.sel_slot[t] = (lo < a.n_sel && a.idx[lo] == t) ? lo : -1;
+    a.sel_slot[t] = (lo < a.n_sel && s_idx[lo] == t) ? lo : -1;
   }
+  // snapshot of the selected rows (and, if asked, their normalised bf16 copy):
+  // one warp per row, the row read once for the copy and the sum of squares
+  const bool norm = a.norm_gain != nullptr;
   for (int r = warp; r < a.n_sel; r += nw) {
-    const float* src = a.h + static_cast<size_t>(a.idx[r]) * a.d;
+    const float* src = a.h + static_cast<size_t>(s_idx[r]) * a.d;
     float* dst = a.h_snap + static_cast<size_t>(r) * a.d;
-    for (int c = lane * 4; c < a.d; c += 128)
-      *reinterpret_cast<float4*>(dst + c) = *reinterpret_cast<const float4*>(src + c);
+    float ss = 0.f;
+    for (int c = lane * 4; c < a.d; c += 128) {
+      const float4 v = *reinterpret_cast<const float4*>(src + c);
+      *reinterpret_cast<float4*>(dst + c) = v;
+      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    }
+    if (!norm) continue;
+    const float inv = rsqrtf(warp_sum(ss) / static_cast<float>(a.d) + a.eps);
+    uint16_t* xr = a.x + static_cast<size_t>(r) * a.d;
+    for (int c = lane * 4; c < a.d; c += 128) {
+      const float4 v = *reinterpret_cast<const float4*>(src + c);
+      const float4 gv = *reinterpret_cast<const float4*>(a.norm_gain + c);
+      const uint32_t lo = f_to_bf16(v.x * inv * gv.x) | (static_cast<uint32_t>(f_to_bf16(v.y * inv * gv.y)) << 16);
+      const uint32_t hi = f_to_bf16(v.z * inv * gv.z) | (static_cast<uint32_t>(f_to_bf16(v.w * inv * gv.w)) << 16);
+      *reinterpret_cast<uint2*>(xr + c) = make_uint2(lo, hi);
+    }
   }
-  __syncthreads();
-  block_plan(a.idx, a.n_sel, a.tile, a.has_c, a.plan);
+  if (norm) {
+    for (int r = a.n_sel + warp; r < a.x_rows; r += nw) {
+      uint16_t* xr = a.x + static_cast<size_t>(r) * a.d;
+      for (int c = lane * 4; c < a.d; c += 128) *reinterpret_cast<uint2*>(xr + c) = make_uint2(0u, 0u);
+    }
+  }
+  block_plan(s_idx, a.n_sel, s_tile, s_hasc, a.plan);
 }
 
 // ============================================================================
@@ -1398,14 +1577,15 @@ cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* i
 }
 cudaError_t launch_quantize_rows(const float* r, int rows, int width, int g, int bits, uint8_t* codes,
                                  uint16_t* scales, cudaStream_t s) {
+  // 8 warps per CTA, 4 row chunks per warp
   if (width % 128 == 0) {
-    const int warps = rows * (width / 128);
-    return launch_k(false, k_quantize_rows<4>, dim3((warps + 3) / 4), dim3(128), 0, s, r, rows, width, g, bits,
-                    codes, scales);
+    const long long items = static_cast<long long>(rows) * (width / 128);
+    return launch_k(false, k_quantize_rows<4>, dim3(static_cast<unsigned>((items + 31) / 32)), dim3(256), 0, s, r,
+                    rows, width, g, bits, codes, scales);
   }
-  const int warps = rows * (width / 64);
-  return launch_k(false, k_quantize_rows<2>, dim3((warps + 3) / 4), dim3(128), 0, s, r, rows, width, g, bits, codes,
-                  scales);
+  const long long items = static_cast<long long>(rows) * (width / 64);
+  return launch_k(false, k_quantize_rows<2>, dim3(static_cast<unsigned>((items + 31) / 32)), dim3(256), 0, s, r,
+                  rows, width, g, bits, codes, scales);
 }
 cudaError_t launch_rmsnorm_rows(const float* h, const int* idx, int n, int n_pad, int d, const float* gain, float eps,
                                 uint16_t* x, cudaStream_t s) {
@@ -1416,15 +1596,15 @@ cudaError_t launch_qkv_post(const QkvPostArgs& a, cudaStream_t s) {
   if (a.hd == 128) return launch_k(g_pdl, k_qkv_post<4>, dim3((warps + 3) / 4), dim3(128), 0, s, a);
   return launch_k(g_pdl, k_qkv_post<2>, dim3((warps + 3) / 4), dim3(128), 0, s, a);
 }
-size_t attn_decode_smem(int hd) { return static_cast<size_t>(2) * 2 * kDecTile * (hd + kDecPad) * 2; }
-cudaError_t launch_attn_decode(const AttnDecArgs& a, int n, cudaStream_t s) {
+size_t attn_decode_smem(int hd) { return 1024 + static_cast<size_t>(kDecStages) * 2 * kDecTile * hd * 2; }
+cudaError_t launch_attn_decode(const CUtensorMap& kv, const AttnDecArgs& a, int n, cudaStream_t s) {
   dim3 grid(n * a.Hkv, a.n_splits);
   const size_t sm = attn_decode_smem(a.hd);
   const int grp = a.H / a.Hkv;
-#define FL_ATT(G)                                                                           \
-  case G:                                                                                   \
-    return a.hd == 128 ? launch_k(g_pdl, k_attn_decode<128, G>, grid, dim3(256), sm, s, a)  \
-                       : launch_k(g_pdl, k_attn_decode<64, G>, grid, dim3(256), sm, s, a);
+#define FL_ATT(G)                                                                              \
+  case G:                                                                                      \
+    return a.hd == 128 ? launch_k(g_pdl, k_attn_decode<128, G>, grid, dim3(128), sm, s, kv, a) \
+                       : launch_k(g_pdl, k_attn_decode<64, G>, grid, dim3(128), sm, s, kv, a);
   switch (grp) {
     FL_ATT(1)
     FL_ATT(2)
@@ -1571,7 +1751,10 @@ cudaError_t kernels_init_attrs() {
   if (done == cudaSuccess) return done;
   cudaError_t e = cudaSuccess;
   auto set = [&](auto* kern, int bytes) {
-    const cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    // all of the unified L1/shared storage as shared memory, so CTAs with large rings pair up on an SM
+    if (r == cudaSuccess && bytes > 48 * 1024)
+      r = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e == cudaSuccess) e = r;
   };
   set(k_attn_decode<128, 1>, static_cast<int>(attn_decode_smem(128)));

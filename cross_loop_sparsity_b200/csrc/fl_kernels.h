@@ -38,13 +38,14 @@ struct AttnDecArgs {
   int j, loop, dense;
   int H, Hkv, hd;
   float tau;
-  int split_len, n_splits;
+  int n_splits;       // CTAs per (token, KV head); split sp takes column tiles [sp*nt/n_splits, (sp+1)*nt/n_splits)
   float* part_o;      // [n][Hkv][splits][8][hd]
   float* part_ml;     // [n][Hkv][splits][8][2]
   int* counters;      // [n][Hkv], zero between launches
   float* o_state;     // [N][H][hd] token order (nullptr for the dense baseline)
   float* lse_state;   // [N][H]
   uint16_t* o_bf16;   // [n][H*hd] GEMM order
+  int* status;        // error bits (a bounded wait that ran out)
 };
 
 struct AttnPreArgs {
@@ -72,6 +73,7 @@ struct SelectStepArgs {
   float* h_snap;         // [n_sel][d] loop-start rows of the selected tokens (read, then rewritten)
   int* sel_slot;         // [N] slot of each token in the selection, or -1 (read, then rewritten)
   int N, d, loop, n_sel;
+  int n_tiles;           // query tiles of the call (tile flags read and set)
   float* key;            // [N]
   float* keys_trace;     // [N] this loop's keys, kept for read-back
   int32_t* idx;          // [n_sel] this loop's selection
@@ -81,6 +83,13 @@ struct SelectStepArgs {
   const int* forced_on;
   const int32_t* forced;
   TilePlan plan;
+  // optional: the first layer's attention RMSNorm of the selected rows,
+  // x[r] = bf16(h[idx[r]] * rsqrt(mean(h^2) + eps) * gain) for r < n_sel and
+  // zero rows for n_sel <= r < x_rows (nullptr gain: not fused)
+  const float* norm_gain;
+  uint16_t* x;
+  int x_rows;
+  float eps;
 };
 
 struct DScoreArgs {
@@ -138,6 +147,7 @@ struct CorrectArgs {
 cudaError_t kernels_init_attrs();
 
 constexpr int kLensByValue = 256;
+constexpr int kSelectStepMax = 1024;   // tokens (and query tiles) the one-CTA selection kernel handles
 struct LensArg {
   int n;
   int v[kLensByValue];
@@ -153,7 +163,9 @@ cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* i
 cudaError_t launch_rmsnorm_rows(const float* h, const int* idx, int n, int n_pad, int d, const float* gain, float eps,
                                 uint16_t* x, cudaStream_t s);
 cudaError_t launch_qkv_post(const QkvPostArgs& a, cudaStream_t s);
-cudaError_t launch_attn_decode(const AttnDecArgs& a, int n, cudaStream_t s);
+// kv: the cache's bf16 rows ([rows][hd], 64 x 64 boxes, 128-byte swizzle) in
+// the layout the context uses (lazy base or dense per-loop)
+cudaError_t launch_attn_decode(const CUtensorMap& kv, const AttnDecArgs& a, int n, cudaStream_t s);
 cudaError_t launch_attn_prefill(const AttnPreArgs& a, int B, cudaStream_t s);
 cudaError_t launch_setup_call(int N, int decode, int T, int tiles_per_seq, int q_tile, const int* seq_len, int* seq,
                               int* pos, int* tile, int* last, int n_tiles, int* has_c, cudaStream_t s);

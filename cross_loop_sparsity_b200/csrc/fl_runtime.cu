@@ -37,7 +37,7 @@ struct flashloop_ctx {
   CacheView cv{};
   bool lazy = true;
   int qkv_rows = 0, N_max = 0, N_pad = 0, n_tiles_max = 0, max_need = 0;
-  int dec_splits = 1, dec_split_len = 64;
+  int dec_splits = 1;   // decode attention: column-tile ranges per (token, KV head)
   // workspace regions
   float *rope_cos = nullptr, *rope_sin = nullptr;
   int *seq_len = nullptr, *status = nullptr;
@@ -67,11 +67,14 @@ struct flashloop_ctx {
   float* gemm_partial = nullptr;
   size_t gemm_partial_cap = 0;
   int* gemm_counters = nullptr;
+  float* ss_part = nullptr;      // [ss_tiles][kSsLd] per-tile sums of squares of updated rows
+  int ss_tiles = 0;
   float* logits_ws = nullptr;
   // descriptors
   CUtensorMap tm_qkv, tm_o, tm_gate, tm_up, tm_down, tm_out;
   CUtensorMap tm_x_a, tm_obf_a, tm_act_a;
   CUtensorMap tm_x_b[3], tm_obf_b[3], tm_act_b[3];
+  CUtensorMap tm_kv;   // the cache's bf16 rows for the decode attention
   // host state
   std::vector<int> lens;
   std::vector<int> graph_b;
@@ -95,7 +98,8 @@ constexpr int kNumSM = 148;
 // get narrow splits for parallelism; many (prefill) get wide ones.
 constexpr int kCorrColsSmall = 16, kCorrColsBig = 128, kCorrSmallQueries = 64;
 // Calls of at most this many tokens do a lazy loop's bookkeeping in one CTA.
-constexpr int kSelectStepMaxTokens = 1024;
+constexpr int kSelectStepMaxNorm = 64;   // selected rows the one-CTA selection kernel also normalises
+constexpr int kSsLd = 64;                // tokens per row of the sums-of-squares table (swap GEMMs: <= 64)
 constexpr int kCountersGemm = 4096;
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
@@ -219,12 +223,10 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   uint8_t* forced_scales = take(std::max<size_t>(fc_rows * (lazy ? hd / c.group_size : 1) * 2, 16));
   uint8_t* forced_codes_on = take(16);
   // decode attention split partials
-  int splits = ceil_div(4 * kNumSM, c.max_batch * Hkv);
+  int splits = (2 * kNumSM) / (c.max_batch * Hkv);   // decode attention: about two CTAs per SM
   const int max_splits = ceil_div(c.max_ctx, 64);
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
-  const int split_len = ceil_div(ceil_div(c.max_ctx, splits), 64) * 64;
-  splits = ceil_div(c.max_ctx, split_len);
   uint8_t* part_o = take(B * Hkv * splits * 8 * hd * 4);
   uint8_t* part_ml = take(B * Hkv * splits * 8 * 2 * 4);
   uint8_t* attn_counters = take(B * Hkv * 4);
@@ -262,6 +264,8 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   }
   uint8_t* gpart = take((gp > 0 ? gp : 1) * 4);
   uint8_t* gcnt = take(kCountersGemm * 4);
+  const int ss_tiles = ceil_div(d, 128);
+  uint8_t* ssp = take(static_cast<size_t>(ss_tiles) * kSsLd * 4);
   uint8_t* logits = take(B * c.vocab * 4);
   if (x) {
     x->lazy = lazy;
@@ -271,7 +275,6 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->n_tiles_max = n_tiles;
     x->max_need = max_need;
     x->dec_splits = splits;
-    x->dec_split_len = split_len;
     x->cv.M = M; x->cv.K = K; x->cv.B = c.max_batch; x->cv.Hkv = Hkv; x->cv.T = c.max_ctx; x->cv.hd = hd;
     x->cv.g = lazy ? c.group_size : hd;
     x->cv.bits = lazy ? c.resid_bits : 16;
@@ -330,6 +333,8 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->gemm_partial = reinterpret_cast<float*>(gpart);
     x->gemm_partial_cap = gp;
     x->gemm_counters = reinterpret_cast<int*>(gcnt);
+    x->ss_part = reinterpret_cast<float*>(ssp);
+    x->ss_tiles = ss_tiles;
     x->logits_ws = reinterpret_cast<float*>(logits);
   }
   return off;
@@ -346,10 +351,23 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
 
 enum GemmOpKind { kOpQKV, kOpO, kOpGU, kOpDown, kOpOut };
 
-fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, cudaStream_t s) {
+// RMSNorm of a GEMM's input rows built inside the GEMM from the fp32 hidden
+// state and the per-tile sums of squares the previous residual GEMM left.
+struct InNorm {
+  const float* gain = nullptr;   // nullptr: the input is the bf16 buffer, loaded by TMA
+  const int* idx = nullptr;      // hidden-state row of each GEMM token (nullptr: identity)
+};
+
+// Launch one GEMM of the block.  `in` (QKV, gate/up, LM head): the input
+// RMSNorm runs inside the GEMM (swap orientation only).  *ss_written (O and
+// down projections): whether the epilogue left the sums of squares of its
+// updated rows for the next norm (the cluster split-K path only).
+fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, cudaStream_t s,
+               const InNorm& in = InNorm{}, bool* ss_written = nullptr) {
   const flashloop_config& c = ctx->cfg;
   GemmLaunch g{};
   GemmArgs& a = g.args;
+  if (ss_written) *ss_written = false;
   const CUtensorMap *w0 = nullptr, *w1 = nullptr, *xa = nullptr;
   const CUtensorMap* xb = nullptr;
   int feat = 0, K = 0;
@@ -395,7 +413,16 @@ fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, 
     a.partial = ctx->gemm_partial; a.counters = ctx->gemm_counters;
     g.bn = bn;
     g.grid = dim3(tiles, 1, splits);
+    if (ss_written && a.epi == kEpiResid && splits > 1 && ceil_div(feat, 128) <= ctx->ss_tiles) {
+      a.ss_out = ctx->ss_part; a.ss_ld = kSsLd;
+      *ss_written = true;
+    }
+    if (in.gain) {
+      a.in_h = ctx->h; a.in_idx = in.idx; a.in_gain = in.gain; a.ss_in = ctx->ss_part; a.ss_ld = kSsLd;
+      a.in_ld = K; a.ss_parts = ceil_div(K, 128); a.in_eps = c.rms_eps;
+    }
   } else {
+    if (in.gain) return FL_ERR_UNSUPPORTED;   // the caller builds the input with the norm kernel instead
     g.a0 = xa; g.a1 = nullptr; g.b0 = w0; g.b1 = w1;
     g.a_3d = 0; g.b_3d = w3d;
     a.a_z = 0; a.b_z = j; a.swap = 0; a.splits = 1;
@@ -503,22 +530,33 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
   FL_LAUNCH(FL_KIND_OTHER, launch_setup_call(N, decode, T, tiles_per_seq, q_tile, ctx->seq_len, ctx->seq, ctx->pos,
                                              ctx->tile, ctx->last, n_tiles, ctx->has_c, s));
   FL_TRY(cudaMemcpyAsync(ctx->h, ctx->h_in, static_cast<size_t>(N) * d * 4, cudaMemcpyDeviceToDevice, s));
+  // How the next GEMM's normed input is produced: the norm kernel, already in
+  // x (the selection kernel normalised it), or inside the GEMM from the sums of
+  // squares the previous residual GEMM left.
+  enum XIn { kXNorm, kXReady, kXSums };
+  XIn carry = kXNorm;   // state at the end of the previous loop (dense loops keep their rows)
+  bool final_sums = false;
   for (int l = 1; l <= K; ++l) {
     const bool full = !lazy || l == 1;
     const int32_t* idx = ctx->idx_all;
     int n = N;
-    if (!full && N <= kSelectStepMaxTokens) {
+    XIn xs = (l > 1 && !lazy) ? carry : kXNorm;
+    if (!full && N <= kSelectStepMax && n_tiles <= kSelectStepMax) {
       // few tokens (decode): keys, selection, snapshot and tile plan in one kernel
       int32_t* sel = ctx->idx_sel + static_cast<size_t>(l - 2) * ctx->N_max;
       SelectStepArgs sa{};
       sa.h = ctx->h; sa.h_in = ctx->h_in; sa.h_snap = ctx->h_snap; sa.sel_slot = ctx->sel_slot;
-      sa.N = N; sa.d = d; sa.loop = l; sa.n_sel = n_sel; sa.key = ctx->key;
+      sa.N = N; sa.d = d; sa.loop = l; sa.n_sel = n_sel; sa.key = ctx->key; sa.n_tiles = n_tiles;
       sa.keys_trace = ctx->keys_trace + static_cast<size_t>(l - 2) * ctx->N_max; sa.idx = sel;
       sa.last = ctx->last; sa.tile = ctx->tile; sa.has_c = ctx->has_c; sa.forced_on = ctx->forced_on;
       sa.forced = ctx->forced_sel + static_cast<size_t>(l - 2) * ctx->N_max; sa.plan = ctx->plan;
+      if (n_sel <= kSelectStepMaxNorm) {   // the first layer's attention norm of the few selected rows
+        sa.norm_gain = ctx->w.attn_norm; sa.x = ctx->x; sa.x_rows = pad(n_sel); sa.eps = c.rms_eps;
+      }
       FL_LAUNCH(FL_KIND_SELECT, launch_select_step(sa, s));
       idx = sel;
       n = n_sel;
+      if (sa.norm_gain) xs = kXReady;
     } else if (!full) {
       int32_t* sel = ctx->idx_sel + static_cast<size_t>(l - 2) * ctx->N_max;
       FL_TRY(cudaMemcpyAsync(ctx->keys_trace + static_cast<size_t>(l - 2) * ctx->N_max, ctx->key,
@@ -535,9 +573,16 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
       float* l_st = lazy ? ctx->lse_state + j * st_l : nullptr;
       float* ql = lazy ? ctx->q_last + j * st_o : nullptr;
       // attention branch
-      FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d,
-                                                  ctx->w.attn_norm + static_cast<size_t>(j) * d, c.rms_eps, ctx->x, s));
-      FL_GEMM(gemm(ctx, kOpQKV, j, n, idx, s));
+      InNorm attn_in;
+      if (xs == kXNorm)
+        FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d,
+                                                    ctx->w.attn_norm + static_cast<size_t>(j) * d, c.rms_eps, ctx->x,
+                                                    s));
+      if (xs == kXSums) {
+        attn_in.gain = ctx->w.attn_norm + static_cast<size_t>(j) * d;
+        attn_in.idx = idx;
+      }
+      FL_GEMM(gemm(ctx, kOpQKV, j, n, idx, s, attn_in));
       QkvPostArgs qa{};
       qa.qkv = ctx->qkv; qa.ldq = ctx->qkv_rows; qa.idx = idx; qa.n = n; qa.seq = ctx->seq; qa.pos = ctx->pos;
       qa.H = H; qa.Hkv = Hkv; qa.hd = hd; qa.rope_cos = ctx->rope_cos; qa.rope_sin = ctx->rope_sin;
@@ -548,12 +593,14 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
       if (full) {
         if (decode) {
           AttnDecArgs aa{};
-          aa.q_cur = ctx->q_cur; aa.idx = idx; aa.seq = ctx->seq; aa.pos = ctx->pos; aa.cv = ctx->cv;
+          // a full loop covers every token in order: no index indirection
+          aa.q_cur = ctx->q_cur; aa.idx = idx == ctx->idx_all ? nullptr : idx; aa.seq = ctx->seq; aa.pos = ctx->pos;
+          aa.cv = ctx->cv;
           aa.j = j; aa.loop = l; aa.dense = lazy ? 0 : 1; aa.H = H; aa.Hkv = Hkv; aa.hd = hd; aa.tau = tau;
-          aa.split_len = ctx->dec_split_len; aa.n_splits = ctx->dec_splits;
+          aa.n_splits = ctx->dec_splits;
           aa.part_o = ctx->part_o; aa.part_ml = ctx->part_ml; aa.counters = ctx->attn_counters;
-          aa.o_state = o_st; aa.lse_state = l_st; aa.o_bf16 = ctx->obf;
-          FL_LAUNCH(FL_KIND_ATTN, launch_attn_decode(aa, n, s));
+          aa.o_state = o_st; aa.lse_state = l_st; aa.o_bf16 = ctx->obf; aa.status = ctx->status;
+          FL_LAUNCH(FL_KIND_ATTN, launch_attn_decode(ctx->tm_kv, aa, n, s));
         } else {
           AttnPreArgs pa{};
           pa.q_cur = ctx->q_cur; pa.cv = ctx->cv; pa.j = j; pa.loop = l; pa.dense = lazy ? 0 : 1;
@@ -584,14 +631,26 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
         FL_LAUNCH(FL_KIND_SELECT, launch_select_cols(sa, max_need, s));
         FL_LAUNCH(FL_KIND_CORRECT, launch_correct(ca, n, s));
       }
-      FL_GEMM(gemm(ctx, kOpO, j, n, idx, s));
+      bool sums = false;
+      FL_GEMM(gemm(ctx, kOpO, j, n, idx, s, InNorm{}, &sums));
       // MLP branch
-      FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d,
-                                                  ctx->w.mlp_norm + static_cast<size_t>(j) * d, c.rms_eps, ctx->x, s));
-      FL_GEMM(gemm(ctx, kOpGU, j, n, idx, s));
-      FL_GEMM(gemm(ctx, kOpDown, j, n, idx, s));
+      InNorm mlp_in;
+      if (sums) {
+        mlp_in.gain = ctx->w.mlp_norm + static_cast<size_t>(j) * d;
+        mlp_in.idx = idx;
+      } else {
+        FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d,
+                                                    ctx->w.mlp_norm + static_cast<size_t>(j) * d, c.rms_eps, ctx->x,
+                                                    s));
+      }
+      FL_GEMM(gemm(ctx, kOpGU, j, n, idx, s, mlp_in));
+      FL_GEMM(gemm(ctx, kOpDown, j, n, idx, s, InNorm{}, &sums));
+      xs = sums ? kXSums : kXNorm;
     }
-    if (lazy && l < K && N > kSelectStepMaxTokens)
+    carry = xs;
+    // the final norm can use the last down projection's sums when it covered every output row
+    final_sums = decode && l == K && full && xs == kXSums;
+    if (lazy && l < K && !(N <= kSelectStepMax && n_tiles <= kSelectStepMax))
       FL_LAUNCH(FL_KIND_OTHER, launch_change_keys(ctx->h, l == 1 ? ctx->h_in : ctx->h_snap, ctx->sel_slot, N, d, l,
                                                   ctx->key, ctx->last, ctx->tile, ctx->has_c, s));
   }
@@ -602,8 +661,14 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
                                       ctx->idx_last));
     rows = ctx->idx_last;
   }
-  FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, rows, B, pad(B), d, ctx->w.final_norm, c.rms_eps, ctx->x, s));
-  FL_GEMM(gemm(ctx, kOpOut, 0, B, rows, s));
+  InNorm out_in;
+  if (final_sums) {
+    out_in.gain = ctx->w.final_norm;
+    out_in.idx = rows;
+  } else {
+    FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, rows, B, pad(B), d, ctx->w.final_norm, c.rms_eps, ctx->x, s));
+  }
+  FL_GEMM(gemm(ctx, kOpOut, 0, B, rows, s, out_in));
   FL_LAUNCH(FL_KIND_OTHER, launch_set_lens(B, ctx->seq_len, decode ? 1 : 0, T, s));
   return FL_OK;
 }
@@ -623,6 +688,10 @@ bool build_tmaps(flashloop_ctx* ctx) {
   ok &= encode_tmap_bf16(&ctx->tm_x_a, ctx->x, d, R, 0, 128);
   ok &= encode_tmap_bf16(&ctx->tm_obf_a, ctx->obf, hq, R, 0, 128);
   ok &= encode_tmap_bf16(&ctx->tm_act_a, ctx->act, f, R, 0, 128);
+  // the cache as [rows][hd] bf16: lazy base [M][2][B][Hkv][T], dense [M][K][2][B][Hkv][T]
+  const uint64_t kv_rows = static_cast<uint64_t>(ctx->cv.M) * (ctx->cv.dense ? ctx->cv.K : 1) * 2 * ctx->cv.B *
+                           ctx->cv.Hkv * ctx->cv.T;
+  ok &= encode_tmap_bf16(&ctx->tm_kv, ctx->cv.base, ctx->cv.hd, kv_rows, 0, 64);
   const uint32_t bns[3] = {16, 32, 64};
   for (int i = 0; i < 3; ++i) {
     ok &= encode_tmap_bf16(&ctx->tm_x_b[i], ctx->x, d, R, 0, bns[i]);
@@ -1089,6 +1158,7 @@ fl_status fl_test_quantize(const float* r, int rows, int width, int g, int bits,
   if (width % g) return FL_ERR_INVALID_ARG;
   if (width % 128 != 0 && width != 64) return FL_ERR_INVALID_ARG;
   if (width == 64 && g > 64) return FL_ERR_INVALID_ARG;
+  if (!aligned16(r)) return FL_ERR_INVALID_ARG;   // rows are read as 16- or 8-byte vectors
   if (rows == 0) return FL_OK;
   return record(launch_quantize_rows(r, rows, width, g, bits, codes, scales, reinterpret_cast<cudaStream_t>(stream)));
 }

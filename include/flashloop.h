@@ -210,7 +210,9 @@ fl_status fl_test_topk(const float* keys, int n_seg, int n, int k, int32_t* idx,
 /* Per-group absmax quantiser: r fp32 [rows][width] (width % g == 0); writes
  * packed codes [rows][width*bits/8] and fp16 scale bits [rows][width/g]:
  * s = fp16_RU(fp32(absmax/qmax)), code = clamp(rint(fp32(r/s))) (KV-residual
- * quantisation, "FlashLoop ...", abstract).  bits 4 or 2; g multiple of 32. */
+ * quantisation, "FlashLoop ...", abstract).  bits 4 or 2; g in {32, 64,
+ * 128}; width a multiple of 128, or 64 with g <= 64; r 16-byte aligned.
+ * Anything else returns FL_ERR_INVALID_ARG before any launch. */
 fl_status fl_test_quantize(const float* r, int rows, int width, int g, int bits,
                            uint8_t* codes, uint16_t* scales, fl_stream_t stream);
 
