@@ -897,9 +897,19 @@ __global__ void k_reset_lens(const LensArg a, int* seq_len) {
 
 // slot of each token in the selection (or -1), and the snapshot of selected rows
 __global__ void k_after_select(const int32_t* __restrict__ idx, int n_sel, int N, int d, int* sel_slot,
-                               const float* __restrict__ h, float* __restrict__ h_snap, int slot_blocks) {
+                               const float* __restrict__ h, float* __restrict__ h_snap, int slot_blocks,
+                               const int* seq, const int* tile, const int* last, const int* pos, SelMeta* meta) {
   pdl_trigger();
   pdl_wait();
+  if (blockIdx.x == 0) {
+    for (int r = threadIdx.x; r < n_sel; r += blockDim.x) {
+      const int t = idx[r];
+      SelMeta m;
+      m.tok = t; m.seq = seq[t]; m.tile = tile[t]; m.last = last[t]; m.pos = pos[t];
+      m.pad0 = m.pad1 = m.pad2 = 0;
+      meta[r] = m;
+    }
+  }
   if (static_cast<int>(blockIdx.x) < slot_blocks) {
     const int t = blockIdx.x * blockDim.x + threadIdx.x;
     if (t >= N) return;
@@ -1024,11 +1034,12 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
   pdl_wait();
   __shared__ float s_key[kSelectStepMax];
   __shared__ int32_t s_idx[kSelectStepMax];
-  __shared__ int s_tile[kSelectStepMax], s_slot[kSelectStepMax], s_hasc[kSelectStepMax];
+  __shared__ int s_tile[kSelectStepMax], s_slot[kSelectStepMax], s_hasc[kSelectStepMax], s_last[kSelectStepMax];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int t = threadIdx.x; t < a.N; t += blockDim.x) {
     s_tile[t] = a.tile[t];
     s_slot[t] = a.loop == 2 ? -1 : a.sel_slot[t];
+    s_last[t] = a.last[t];
   }
   for (int t = threadIdx.x; t < a.n_tiles; t += blockDim.x) s_hasc[t] = a.has_c[t];
   __syncthreads();
@@ -1053,6 +1064,7 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
       a.keys_trace[t] = acc;
       if (slot >= 0) {
         a.last[t] = a.loop - 1;
+        s_last[t] = a.loop - 1;
         s_hasc[s_tile[t]] = 1;
         a.has_c[s_tile[t]] = 1;
       }
@@ -1065,7 +1077,14 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
     block_topk(s_key, a.N, a.n_sel, s_idx);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < a.n_sel; i += blockDim.x) a.idx[i] = s_idx[i];
+  for (int i = threadIdx.x; i < a.n_sel; i += blockDim.x) {
+    const int t = s_idx[i];
+    a.idx[i] = t;
+    SelMeta m;
+    m.tok = t; m.seq = a.seq[t]; m.tile = s_tile[t]; m.last = s_last[t]; m.pos = a.pos[t];
+    m.pad0 = m.pad1 = m.pad2 = 0;
+    a.meta[i] = m;
+  }
   for (int t = threadIdx.x; t < a.N; t += blockDim.x) {
     int lo = 0, hi = a.n_sel;
     while (lo < hi) {
@@ -1074,35 +1093,73 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
     }
     a.sel_slot[t] = (lo < a.n_sel && s_idx[lo] == t) ? lo : -1;
   }
-  // snapshot of the selected rows (and, if asked, their normalised bf16 copy):
-  // one warp per row, the row read once for the copy and the sum of squares
+  // snapshot of the selected rows (and, if asked, their normalised bf16 copy).
+  // Work items are 512-element slices of a row, one per warp at a time; a
+  // slice's loads are all issued before its stores (the snapshot may not be
+  // assumed apart from h), so a row costs one memory round trip per pass.
+  constexpr int SL = 512;
+  const int nsl = (a.d + SL - 1) / SL;
   const bool norm = a.norm_gain != nullptr;
-  for (int r = warp; r < a.n_sel; r += nw) {
+  __shared__ float s_ss[kSelectStepMaxNorm * kSelectStepSlices];
+  for (int it = warp; it < a.n_sel * nsl; it += nw) {
+    const int r = it / nsl, c0 = (it % nsl) * SL;
     const float* src = a.h + static_cast<size_t>(s_idx[r]) * a.d;
     float* dst = a.h_snap + static_cast<size_t>(r) * a.d;
-    float ss = 0.f;
-    for (int c = lane * 4; c < a.d; c += 128) {
-      const float4 v = *reinterpret_cast<const float4*>(src + c);
-      *reinterpret_cast<float4*>(dst + c) = v;
-      ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+    float4 v[SL / 128];
+#pragma unroll
+    for (int u = 0; u < SL / 128; ++u) {
+      const int c = c0 + u * 128 + lane * 4;
+      v[u] = c < a.d ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (!norm) continue;
-    const float inv = rsqrtf(warp_sum(ss) / static_cast<float>(a.d) + a.eps);
-    uint16_t* xr = a.x + static_cast<size_t>(r) * a.d;
-    for (int c = lane * 4; c < a.d; c += 128) {
-      const float4 v = *reinterpret_cast<const float4*>(src + c);
-      const float4 gv = *reinterpret_cast<const float4*>(a.norm_gain + c);
-      const uint32_t lo = f_to_bf16(v.x * inv * gv.x) | (static_cast<uint32_t>(f_to_bf16(v.y * inv * gv.y)) << 16);
-      const uint32_t hi = f_to_bf16(v.z * inv * gv.z) | (static_cast<uint32_t>(f_to_bf16(v.w * inv * gv.w)) << 16);
-      *reinterpret_cast<uint2*>(xr + c) = make_uint2(lo, hi);
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < SL / 128; ++u) {
+      const int c = c0 + u * 128 + lane * 4;
+      if (c < a.d) *reinterpret_cast<float4*>(dst + c) = v[u];
+      ss += v[u].x * v[u].x + v[u].y * v[u].y + v[u].z * v[u].z + v[u].w * v[u].w;
+    }
+    if (norm) {
+      ss = warp_sum(ss);
+      if (lane == 0) s_ss[it] = ss;
     }
   }
   if (norm) {
-    for (int r = a.n_sel + warp; r < a.x_rows; r += nw) {
+    __syncthreads();
+    for (int it = warp; it < a.x_rows * nsl; it += nw) {
+      const int r = it / nsl, c0 = (it % nsl) * SL;
       uint16_t* xr = a.x + static_cast<size_t>(r) * a.d;
-      for (int c = lane * 4; c < a.d; c += 128) *reinterpret_cast<uint2*>(xr + c) = make_uint2(0u, 0u);
+      if (r >= a.n_sel) {
+#pragma unroll
+        for (int u = 0; u < SL / 128; ++u) {
+          const int c = c0 + u * 128 + lane * 4;
+          if (c < a.d) *reinterpret_cast<uint2*>(xr + c) = make_uint2(0u, 0u);
+        }
+        continue;
+      }
+      float tot = 0.f;
+      for (int q = 0; q < nsl; ++q) tot += s_ss[r * nsl + q];
+      const float inv = rsqrtf(tot / static_cast<float>(a.d) + a.eps);
+      const float* src = a.h + static_cast<size_t>(s_idx[r]) * a.d;
+      float4 v[SL / 128], gv[SL / 128];
+#pragma unroll
+      for (int u = 0; u < SL / 128; ++u) {
+        const int c = c0 + u * 128 + lane * 4;
+        v[u] = c < a.d ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        gv[u] = c < a.d ? *reinterpret_cast<const float4*>(a.norm_gain + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < SL / 128; ++u) {
+        const int c = c0 + u * 128 + lane * 4;
+        if (c >= a.d) continue;
+        const uint32_t lo =
+            f_to_bf16(v[u].x * inv * gv[u].x) | (static_cast<uint32_t>(f_to_bf16(v[u].y * inv * gv[u].y)) << 16);
+        const uint32_t hi =
+            f_to_bf16(v[u].z * inv * gv[u].z) | (static_cast<uint32_t>(f_to_bf16(v[u].w * inv * gv[u].w)) << 16);
+        *reinterpret_cast<uint2*>(xr + c) = make_uint2(lo, hi);
+      }
     }
   }
+  __syncthreads();
   block_plan(s_idx, a.n_sel, s_tile, s_hasc, a.plan);
 }
 
@@ -1137,14 +1194,25 @@ __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
   const int nc = min(CC, maxpos + 1 - c0);
   const int grp = a.H / a.Hkv;
   const CacheView& cv = a.cv;
-  // reconstruct K of loop l and the base for this column chunk
-  for (int rr = warp; rr < nc; rr += 8) {
-    float lo[EPL], hi[EPL];
-    chain_lane2<EPL, KM>(cv, a.j, 0, b, g, c0 + rr, 1, a.loop, lane, lo, hi);
+  // reconstruct K of loop l and the base for this column chunk: a warp's rows
+  // are requested together, then stored
+  {
+    constexpr int RW = CC / 8;   // rows per warp
+    float lo[RW][EPL], hi[RW][EPL];
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      Kb[rr * (HD + 1) + lane * EPL + e] = lo[e];
-      Kn[rr * (HD + 1) + lane * EPL + e] = hi[e];
+    for (int u = 0; u < RW; ++u) {
+      const int rr = warp + u * 8;
+      if (rr < nc) chain_lane2<EPL, KM>(cv, a.j, 0, b, g, c0 + rr, 1, a.loop, lane, lo[u], hi[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < RW; ++u) {
+      const int rr = warp + u * 8;
+      if (rr >= nc) continue;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) {
+        Kb[rr * (HD + 1) + lane * EPL + e] = lo[u][e];
+        Kn[rr * (HD + 1) + lane * EPL + e] = hi[u][e];
+      }
     }
   }
   const int c = tid % CC, slot = tid / CC;
@@ -1380,13 +1448,15 @@ __global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
 
 // ============================================================================
 // The correction for few selected queries (decode): the column slices of one
-// (query, KV group) are the CTAs of one cluster.  Each warp takes two columns
-// at a time with every K and V chain load of both issued before any
-// arithmetic.  Each CTA leaves its piece (per-head max, denominator,
-// numerator) in shared memory; after the cluster barrier rank 0 merges the
-// pieces of every rank, in rank order, over distributed shared memory,
-// together with the stored (O, lse) term.  No global scratch, fence or ticket.
-// grid (kCorrCluster, n_sel * Hkv).
+// (query, KV group) are the CTAs of one cluster (kCorrCluster CTAs of
+// kCorrWarps warps).  The query's slot record, its column-set count and the
+// first column ids are requested together; warp w of rank r takes columns
+// r*per + w + u*kCorrWarps of the set, two at a time, with every K and V chain
+// load of both issued before any arithmetic.  The warps' pieces (per-head max,
+// denominator, numerator) are merged in the CTA with one weight per (warp,
+// head); then rank r merges outputs [r*E/CS, (r+1)*E/CS) of every rank, in rank
+// order, over distributed shared memory, together with the stored (O, lse)
+// term.  No global scratch, fence or ticket.  grid (kCorrCluster, n_sel * Hkv).
 // ============================================================================
 template <int EPL, int GRP>
 __device__ __forceinline__ void corr_column(const float (&qn)[GRP][EPL], const float (&qo)[GRP][EPL],
@@ -1414,26 +1484,31 @@ __device__ __forceinline__ void corr_column(const float (&qn)[GRP][EPL], const f
 }
 
 template <int HD, int EPL, int GRP, int KM>
-__global__ void __launch_bounds__(256) k_correct_cluster(const CorrectArgs a) {
+__global__ void __launch_bounds__(32 * kCorrWarps) k_correct_cluster(const CorrectArgs a) {
   pdl_trigger();
-  pdl_wait();
-  constexpr int NW = 8, CS = kCorrCluster;
-  __shared__ float sm_m[NW][GRP], sm_z[NW][GRP];
-  __shared__ float sm_acc[NW][GRP][HD];
+  constexpr int NW = kCorrWarps, CS = kCorrCluster, E = GRP * HD, NT = 32 * NW;
+  extern __shared__ float sm_acc[];   // [NW][GRP][HD]
+  __shared__ float sm_m[NW][GRP], sm_z[NW][GRP], sm_w[NW][GRP];
   __shared__ float pm[GRP], pz[GRP];
   __shared__ float pacc[GRP][HD];
   cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rank = static_cast<int>(cluster.block_rank());
   const int i = blockIdx.y / a.Hkv, g = blockIdx.y % a.Hkv;
-  const int tok = a.idx[i];
-  const int b = a.seq[tok], tl = a.tile[tok];
-  const int m_old = a.last[tok];
+  pdl_wait();
+  const SelMeta mt = a.meta[i];
+  const int tok = mt.tok, b = mt.seq, m_old = mt.last;
   const CacheView& cv = a.cv;
-  const size_t cset = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
+  const size_t cset = (static_cast<size_t>(a.j) * a.n_tiles + mt.tile) * a.Hkv + g;
   const int32_t* C = a.cols + cset * a.c;
-  // a decode token is its own tile, so every column of its set is causal
+  // a decode token is its own tile, so every column of its set is causal; the
+  // slice bounds use the set's capacity so the column ids need not wait for its count
+  const int per = (a.c + CS - 1) / CS;
+  const int k0 = rank * per, k1 = min(a.c, k0 + per);
   const int nvalid = a.ncols[cset];
+  int col_first[2];
+#pragma unroll
+  for (int u = 0; u < 2; ++u) col_first[u] = k0 + warp + u * NW < k1 ? C[k0 + warp + u * NW] : -1;
   float qn[GRP][EPL], qo[GRP][EPL];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
@@ -1444,21 +1519,18 @@ __global__ void __launch_bounds__(256) k_correct_cluster(const CorrectArgs a) {
       qo[h][e] = a.q_last[(static_cast<size_t>(tok) * a.H + hq) * HD + lane * EPL + e];
     }
   }
-  // rank 0 requests the stored state it will merge into now, not after the barrier
-  float st_o[2] = {0.f, 0.f}, st_l[2] = {0.f, 0.f};
-  if (rank == 0) {
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int e = tid + r * 256;
-      if (e < GRP * HD) {
-        const size_t so = static_cast<size_t>(tok) * a.H + g * GRP + e / HD;
-        st_o[r] = a.o_state[so * HD + e % HD];
-        st_l[r] = a.lse_state[so];
-      }
-    }
+  // rank r merges elements [r*E/CS, (r+1)*E/CS) of the (head, dim) outputs at the
+  // end; the stored state it merges into is requested now, not after the barrier
+  const int me = (rank * E) / CS + tid;
+  const bool merger = me < ((rank + 1) * E) / CS;
+  float st_o = 0.f, st_l = 0.f, q_now = 0.f;
+  if (merger) {
+    const size_t so = static_cast<size_t>(tok) * a.H + g * GRP + me / HD;
+    st_o = a.o_state[so * HD + me % HD];
+    st_l = a.lse_state[so];
+    q_now = a.q_cur[(static_cast<size_t>(i) * a.H + g * GRP + me / HD) * HD + me % HD];
   }
-  const int per = (nvalid + CS - 1) / CS;
-  const int k0 = rank * per, k1 = min(nvalid, k0 + per);
+  const int k1v = min(k1, nvalid);
   float m[GRP], z[GRP], acc[GRP][EPL];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
@@ -1467,12 +1539,23 @@ __global__ void __launch_bounds__(256) k_correct_cluster(const CorrectArgs a) {
 #pragma unroll
     for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
   }
-  for (int k = k0 + warp; k < k1; k += NW) {
-    const int col = C[k];
-    float klo[EPL], khi[EPL], vlo[EPL], vhi[EPL];
-    chain_lane2<EPL, KM>(cv, a.j, 0, b, g, col, m_old, a.loop, lane, klo, khi);
-    chain_lane2<EPL, KM>(cv, a.j, 1, b, g, col, m_old, a.loop, lane, vlo, vhi);
-    corr_column<EPL, GRP>(qn, qo, klo, khi, vlo, vhi, a.tau, m, z, acc);
+  for (int kb = k0 + warp; kb < k1v; kb += 2 * NW) {
+    int col[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int k = kb + u * NW;
+      col[u] = k < k1v ? (kb == k0 + warp ? col_first[u] : C[k]) : -1;
+    }
+    float klo[2][EPL], khi[2][EPL], vlo[2][EPL], vhi[2][EPL];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (col[u] < 0) continue;
+      chain_lane2<EPL, KM>(cv, a.j, 0, b, g, col[u], m_old, a.loop, lane, klo[u], khi[u]);
+      chain_lane2<EPL, KM>(cv, a.j, 1, b, g, col[u], m_old, a.loop, lane, vlo[u], vhi[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+      if (col[u] >= 0) corr_column<EPL, GRP>(qn, qo, klo[u], khi[u], vlo[u], vhi[u], a.tau, m, z, acc);
   }
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
@@ -1481,67 +1564,65 @@ __global__ void __launch_bounds__(256) k_correct_cluster(const CorrectArgs a) {
       sm_z[warp][h] = z[h];
     }
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) sm_acc[warp][h][lane * EPL + e] = acc[h][e];
+    for (int e = 0; e < EPL; ++e) sm_acc[(warp * GRP + h) * HD + lane * EPL + e] = acc[h][e];
   }
   __syncthreads();
-  for (int e = tid; e < GRP * HD; e += 256) {
-    const int h = e / HD, dd = e % HD;
+  // this CTA's piece: one weight per (warp, head), then the weighted sums in warp order
+  if (tid < GRP) {
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][h]);
-    float A = 0.f, Z = 0.f;
-    if (M != -INFINITY)
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][tid]);
+    float Z = 0.f;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) {
-        if (sm_m[w][h] == -INFINITY) continue;
-        const float f = expf(sm_m[w][h] - M);
-        A += sm_acc[w][h][dd] * f;
-        Z += sm_z[w][h] * f;
-      }
-    pacc[h][dd] = A;
-    if (dd == 0) {
-      pm[h] = M;
-      pz[h] = Z;
+    for (int w = 0; w < NW; ++w) {
+      const float f = sm_m[w][tid] == -INFINITY ? 0.f : expf(sm_m[w][tid] - M);
+      sm_w[w][tid] = f;
+      Z += f * sm_z[w][tid];
     }
+    pm[tid] = M;
+    pz[tid] = Z;
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += NT) {
+    const int h = e / HD, dd = e % HD;
+    float A = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) A += sm_w[w][h] * sm_acc[(w * GRP + h) * HD + dd];
+    pacc[h][dd] = A;
   }
   cluster.sync();
-  if (rank == 0) {
+  if (merger) {
+    const int h = me / HD, dd = me % HD;
+    const int hq = g * GRP + h;
+    const size_t so = static_cast<size_t>(tok) * a.H + hq;
+    // every rank's piece is requested before any is used, so the distributed
+    // shared-memory round trips overlap; the merge itself runs in rank order
+    float rm[CS], rz[CS], ra[CS];
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      const int e = tid + rr * 256;
-      if (e >= GRP * HD) break;
-      const int h = e / HD, dd = e % HD;
-      const int hq = g * GRP + h;
-      const size_t so = static_cast<size_t>(tok) * a.H + hq;
-      const float L = st_l[rr];
-      // every rank's piece is requested before any is used, so the distributed
-      // shared-memory round trips overlap; the merge itself runs in rank order
-      float rm[CS], rz[CS], ra[CS];
-#pragma unroll
-      for (int r = 0; r < CS; ++r) {
-        rm[r] = *cluster.map_shared_rank(&pm[h], r);
-        rz[r] = *cluster.map_shared_rank(&pz[h], r);
-        ra[r] = *cluster.map_shared_rank(&pacc[h][dd], r);
-      }
-      float M = L;
-#pragma unroll
-      for (int r = 0; r < CS; ++r) M = fmaxf(M, rm[r]);
-      const float el = expf(L - M);
-      float Z = el, N = el * st_o[rr];
-#pragma unroll
-      for (int r = 0; r < CS; ++r) {
-        if (rm[r] == -INFINITY) continue;
-        const float f = expf(rm[r] - M);
-        Z += f * rz[r];
-        N += f * ra[r];
-      }
-      if (!(Z > 0.f) && a.status) atomicOr(a.status, kErrBadIndex);
-      const float ov = N / Z;
-      a.o_state[so * HD + dd] = ov;
-      a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + dd] = f_to_bf16(ov);
-      a.q_last[so * HD + dd] = a.q_cur[(static_cast<size_t>(i) * a.H + hq) * HD + dd];
-      if (dd == 0) a.lse_state[so] = M + logf(Z);
+    for (int r = 0; r < CS; ++r) {
+      rm[r] = *cluster.map_shared_rank(&pm[h], r);
+      rz[r] = *cluster.map_shared_rank(&pz[h], r);
+      ra[r] = *cluster.map_shared_rank(&pacc[h][dd], r);
     }
+    const float L = st_l;
+    float M = L;
+#pragma unroll
+    for (int r = 0; r < CS; ++r) M = fmaxf(M, rm[r]);
+    const float el = expf(L - M);
+    float Z = el, N = el * st_o;
+#pragma unroll
+    for (int r = 0; r < CS; ++r) {
+      if (rm[r] == -INFINITY) continue;
+      const float f = expf(rm[r] - M);
+      Z += f * rz[r];
+      N += f * ra[r];
+    }
+    if (!(Z > 0.f) && a.status) atomicOr(a.status, kErrBadIndex);
+    const float ov = N / Z;
+    a.o_state[so * HD + dd] = ov;
+    a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + dd] = f_to_bf16(ov);
+    a.q_last[so * HD + dd] = q_now;
+    if (dd == 0) a.lse_state[so] = M + logf(Z);
   }
   cluster.sync();
 }
@@ -1636,10 +1717,11 @@ cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s) {
   return launch_k(false, k_reset_lens, dim3(1), dim3(kLensByValue), 0, s, a, seq_len);
 }
 cudaError_t launch_after_select(const int32_t* idx, int n_sel, int N, int d, int* sel_slot, const float* h,
-                                float* h_snap, cudaStream_t s) {
+                                float* h_snap, const int* seq, const int* tile, const int* last, const int* pos,
+                                SelMeta* meta, cudaStream_t s) {
   const int slot_blocks = (N + 255) / 256;
   return launch_k(g_pdl, k_after_select, dim3(slot_blocks + n_sel), dim3(256), 0, s, idx, n_sel, N, d, sel_slot, h,
-                  h_snap, slot_blocks);
+                  h_snap, slot_blocks, seq, tile, last, pos, meta);
 }
 cudaError_t launch_change_keys(const float* h, const float* ref, const int* sel_slot, int N, int d, int loop,
                                float* key, int* last, const int* tile, int* has_c, cudaStream_t s) {
@@ -1675,12 +1757,13 @@ cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cud
 cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t s) {
   return launch_k(g_pdl, k_select_cols, dim3(max_need * a.Hkv), dim3(1024), 0, s, a);
 }
+size_t corr_cluster_smem(int hd, int grp) { return static_cast<size_t>(kCorrWarps) * grp * hd * 4; }
 template <typename K, typename A>
-cudaError_t launch_cluster(K kern, dim3 grid, dim3 block, int cluster_x, cudaStream_t s, const A& a) {
+cudaError_t launch_cluster(K kern, dim3 grid, dim3 block, int cluster_x, size_t smem, cudaStream_t s, const A& a) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1698,7 +1781,8 @@ template <int HD, int EPL, int GRP, int KM>
 cudaError_t launch_correct_t(const CorrectArgs& a, int n_sel, cudaStream_t s) {
   if (a.cluster) {
     dim3 grid(kCorrCluster, n_sel * a.Hkv);
-    return launch_cluster(k_correct_cluster<HD, EPL, GRP, KM>, grid, dim3(256), kCorrCluster, s, a);
+    return launch_cluster(k_correct_cluster<HD, EPL, GRP, KM>, grid, dim3(32 * kCorrWarps), kCorrCluster,
+                          corr_cluster_smem(HD, GRP), s, a);
   }
   dim3 grid(n_sel * a.Hkv, a.n_splits);
   return launch_k(g_pdl, k_correct<HD, EPL, GRP, KM>, grid, dim3(256), 0, s, a);
@@ -1733,7 +1817,12 @@ cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
 // 16-CTA clusters are beyond the portable size: opt every instantiation in.
 template <int HD, int EPL, int GRP, int KM>
 cudaError_t allow_big_cluster() {
-  return cudaFuncSetAttribute(k_correct_cluster<HD, EPL, GRP, KM>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaError_t e =
+      cudaFuncSetAttribute(k_correct_cluster<HD, EPL, GRP, KM>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_correct_cluster<HD, EPL, GRP, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(corr_cluster_smem(HD, GRP)));
+  return e;
 }
 template <int HD, int EPL, int GRP>
 cudaError_t allow_big_cluster_km() {

@@ -67,6 +67,13 @@ struct TilePlan {
   int* counts;  // [0] entries, [1] entries needing a column set
 };
 
+// One selected slot of the current loop, written by the selection step: the
+// token and what the attention-side kernels need about it, in one 32-byte record
+// (last = the loop whose KV the token's attention state was computed with).
+struct alignas(32) SelMeta {
+  int tok, seq, tile, last, pos, pad0, pad1, pad2;
+};
+
 struct SelectStepArgs {
   const float* h;        // [N][d] current hidden states
   const float* h_in;     // [N][d] call inputs (change after loop 1)
@@ -83,6 +90,9 @@ struct SelectStepArgs {
   const int* forced_on;
   const int32_t* forced;
   TilePlan plan;
+  const int* seq;        // [N] sequence of each token
+  const int* pos;        // [N] position of each token
+  SelMeta* meta;         // [n_sel] written for the selected slots
   // optional: the first layer's attention RMSNorm of the selected rows,
   // x[r] = bf16(h[idx[r]] * rsqrt(mean(h^2) + eps) * gain) for r < n_sel and
   // zero rows for n_sel <= r < x_rows (nullptr gain: not fused)
@@ -132,6 +142,7 @@ struct CorrectArgs {
   uint16_t* o_bf16;
   const int32_t* cols;
   const int* ncols;
+  const SelMeta* meta;          // [n_sel] per selected slot (the clustered path reads this)
   CacheView cv;
   int j, loop, H, Hkv, hd, c, n_tiles;
   float tau;
@@ -148,11 +159,14 @@ cudaError_t kernels_init_attrs();
 
 constexpr int kLensByValue = 256;
 constexpr int kSelectStepMax = 1024;   // tokens (and query tiles) the one-CTA selection kernel handles
+constexpr int kSelectStepMaxNorm = 64;   // selected rows it also normalises (first layer's input)
+constexpr int kSelectStepSlices = 16;    // 512-element slices of a row it normalises (d <= 8192)
 struct LensArg {
   int n;
   int v[kLensByValue];
 };
 cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s);
+constexpr int kCorrWarps = 16;   // warps per CTA of the clustered correction
 constexpr int kCorrCluster = 16;  // CTAs per (query, KV group) in the clustered correction (non-portable size)
 // Launches made while this is on (the kernels of one call) are programmatic
 // dependents of the previous kernel; thread-local.
@@ -170,8 +184,11 @@ cudaError_t launch_attn_prefill(const AttnPreArgs& a, int B, cudaStream_t s);
 cudaError_t launch_setup_call(int N, int decode, int T, int tiles_per_seq, int q_tile, const int* seq_len, int* seq,
                               int* pos, int* tile, int* last, int n_tiles, int* has_c, cudaStream_t s);
 cudaError_t launch_set_lens(int B, int* seq_len, int add, int value, cudaStream_t s);
+// selection slots, snapshot of the selected rows and their SelMeta records
+// (the path for calls too large for the one-CTA selection step)
 cudaError_t launch_after_select(const int32_t* idx, int n_sel, int N, int d, int* sel_slot, const float* h,
-                                float* h_snap, cudaStream_t s);
+                                float* h_snap, const int* seq, const int* tile, const int* last, const int* pos,
+                                SelMeta* meta, cudaStream_t s);
 cudaError_t launch_change_keys(const float* h, const float* ref, const int* sel_slot, int N, int d, int loop,
                                float* key, int* last, const int* tile, int* has_c, cudaStream_t s);
 cudaError_t launch_select_step(const SelectStepArgs& a, cudaStream_t s);

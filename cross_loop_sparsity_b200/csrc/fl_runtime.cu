@@ -68,6 +68,7 @@ struct flashloop_ctx {
   size_t gemm_partial_cap = 0;
   int* gemm_counters = nullptr;
   float* ss_part = nullptr;      // [ss_tiles][kSsLd] per-tile sums of squares of updated rows
+  SelMeta* sel_meta = nullptr;   // [N] records of the current loop's selected slots
   int ss_tiles = 0;
   float* logits_ws = nullptr;
   // descriptors
@@ -98,7 +99,6 @@ constexpr int kNumSM = 148;
 // get narrow splits for parallelism; many (prefill) get wide ones.
 constexpr int kCorrColsSmall = 16, kCorrColsBig = 128, kCorrSmallQueries = 64;
 // Calls of at most this many tokens do a lazy loop's bookkeeping in one CTA.
-constexpr int kSelectStepMaxNorm = 64;   // selected rows the one-CTA selection kernel also normalises
 constexpr int kSsLd = 64;                // tokens per row of the sums-of-squares table (swap GEMMs: <= 64)
 constexpr int kCountersGemm = 4096;
 
@@ -265,6 +265,7 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   uint8_t* gpart = take((gp > 0 ? gp : 1) * 4);
   uint8_t* gcnt = take(kCountersGemm * 4);
   const int ss_tiles = ceil_div(d, 128);
+  uint8_t* smeta = take(static_cast<size_t>(N) * sizeof(SelMeta));
   uint8_t* ssp = take(static_cast<size_t>(ss_tiles) * kSsLd * 4);
   uint8_t* logits = take(B * c.vocab * 4);
   if (x) {
@@ -334,6 +335,7 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->gemm_partial_cap = gp;
     x->gemm_counters = reinterpret_cast<int*>(gcnt);
     x->ss_part = reinterpret_cast<float*>(ssp);
+    x->sel_meta = reinterpret_cast<SelMeta*>(smeta);
     x->ss_tiles = ss_tiles;
     x->logits_ws = reinterpret_cast<float*>(logits);
   }
@@ -547,10 +549,11 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
       SelectStepArgs sa{};
       sa.h = ctx->h; sa.h_in = ctx->h_in; sa.h_snap = ctx->h_snap; sa.sel_slot = ctx->sel_slot;
       sa.N = N; sa.d = d; sa.loop = l; sa.n_sel = n_sel; sa.key = ctx->key; sa.n_tiles = n_tiles;
+      sa.seq = ctx->seq; sa.pos = ctx->pos; sa.meta = ctx->sel_meta;
       sa.keys_trace = ctx->keys_trace + static_cast<size_t>(l - 2) * ctx->N_max; sa.idx = sel;
       sa.last = ctx->last; sa.tile = ctx->tile; sa.has_c = ctx->has_c; sa.forced_on = ctx->forced_on;
       sa.forced = ctx->forced_sel + static_cast<size_t>(l - 2) * ctx->N_max; sa.plan = ctx->plan;
-      if (n_sel <= kSelectStepMaxNorm) {   // the first layer's attention norm of the few selected rows
+      if (n_sel <= kSelectStepMaxNorm && d <= 512 * kSelectStepSlices) {   // first layer's norm of the few selected rows
         sa.norm_gain = ctx->w.attn_norm; sa.x = ctx->x; sa.x_rows = pad(n_sel); sa.eps = c.rms_eps;
       }
       FL_LAUNCH(FL_KIND_SELECT, launch_select_step(sa, s));
@@ -563,7 +566,8 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
                              static_cast<size_t>(N) * 4, cudaMemcpyDeviceToDevice, s));
       FL_LAUNCH(FL_KIND_SELECT, launch_select_tokens(ctx->key, N, n_sel, sel, ctx->forced_on,
                                                      ctx->forced_sel + static_cast<size_t>(l - 2) * ctx->N_max, s));
-      FL_LAUNCH(FL_KIND_SELECT, launch_after_select(sel, n_sel, N, d, ctx->sel_slot, ctx->h, ctx->h_snap, s));
+      FL_LAUNCH(FL_KIND_SELECT, launch_after_select(sel, n_sel, N, d, ctx->sel_slot, ctx->h, ctx->h_snap, ctx->seq,
+                                                    ctx->tile, ctx->last, ctx->pos, ctx->sel_meta, s));
       FL_LAUNCH(FL_KIND_SELECT, launch_plan_tiles(sel, n_sel, ctx->tile, ctx->has_c, ctx->plan, s));
       idx = sel;
       n = n_sel;
@@ -612,7 +616,7 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
         CorrectArgs ca{};
         ca.idx = idx; ca.seq = ctx->seq; ca.pos = ctx->pos; ca.tile = ctx->tile; ca.last = ctx->last;
         ca.q_cur = ctx->q_cur; ca.q_last = ql; ca.o_state = o_st; ca.lse_state = l_st; ca.o_bf16 = ctx->obf;
-        ca.cols = ctx->cols; ca.ncols = ctx->ncols; ca.cv = ctx->cv; ca.j = j; ca.loop = l; ca.H = H; ca.Hkv = Hkv;
+        ca.cols = ctx->cols; ca.ncols = ctx->ncols; ca.meta = ctx->sel_meta; ca.cv = ctx->cv; ca.j = j; ca.loop = l; ca.H = H; ca.Hkv = Hkv;
         ca.hd = hd; ca.c = c.c_cols; ca.n_tiles = ctx->n_tiles_max; ca.tau = tau; ca.status = ctx->status;
         ca.cols_per_cta = n_sel <= kCorrSmallQueries ? kCorrColsSmall : kCorrColsBig;
         ca.n_splits = ceil_div(c.c_cols, ca.cols_per_cta);
