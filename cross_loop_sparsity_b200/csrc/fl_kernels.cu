@@ -1182,13 +1182,14 @@ __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
   float* Qn = Kb + CC * (HD + 1);                // [QP][HD]
   float* Qo = Qn + QP * HD;                      // [QP][HD]
   float* Mx = Qo + QP * HD;                      // [4][CC]
+  __shared__ int Qpos[QP];                       // position of each staged pair's query
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int seg = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
-  if (seg >= a.plan.counts[1]) return;
-  const int p = a.plan.need[seg];
+  const int cnt = a.plan.counts[1], p = a.plan.need[seg];   // requested together
+  if (seg >= cnt) return;
   const int qb = a.plan.qb[p], qe = a.plan.qe[p];
-  const int tok_last = a.idx[qe - 1];
-  const int b = a.seq[tok_last], maxpos = a.pos[tok_last];
+  const SelMeta ml = a.meta[qe - 1];
+  const int b = ml.seq, maxpos = ml.pos;
   const int c0 = blockIdx.y * CC;
   if (c0 > maxpos) return;
   const int nc = min(CC, maxpos + 1 - c0);
@@ -1224,15 +1225,15 @@ __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
     for (int e = tid; e < np * HD; e += 256) {
       const int pr = e / HD, dd = e % HD;
       const int qi = qb + (pb + pr) / grp, hh = g * grp + (pb + pr) % grp;
-      const int tk = a.idx[qi];
+      const SelMeta mq = a.meta[qi];
       Qn[pr * HD + dd] = a.q_cur[(static_cast<size_t>(qi) * a.H + hh) * HD + dd];
-      Qo[pr * HD + dd] = a.q_last[(static_cast<size_t>(tk) * a.H + hh) * HD + dd];
+      Qo[pr * HD + dd] = a.q_last[(static_cast<size_t>(mq.tok) * a.H + hh) * HD + dd];
+      if (dd == 0) Qpos[pr] = mq.pos;
     }
     __syncthreads();
     if (c < nc) {
       for (int pr = slot; pr < np; pr += 4) {
-        const int qi = qb + (pb + pr) / grp;
-        if (a.pos[a.idx[qi]] < c0 + c) continue;
+        if (Qpos[pr] < c0 + c) continue;
         float dn = 0.f, db = 0.f;
         const float* kn = &Kn[c * (HD + 1)];
         const float* kb = &Kb[c * (HD + 1)];
@@ -1259,12 +1260,12 @@ __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
 __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
   pdl_trigger();
   pdl_wait();
+  extern __shared__ float keys_sm[];   // [min(max_cols, kSelColsSmemKeys)]
   const int seg = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
-  if (seg >= a.plan.counts[1]) return;
-  const int p = a.plan.need[seg];
+  const int cnt = a.plan.counts[1], p = a.plan.need[seg];   // requested together
+  if (seg >= cnt) return;
   const int tl = a.plan.tile[p];
-  const int tok_last = a.idx[a.plan.qe[p] - 1];
-  const int n = a.pos[tok_last] + 1;
+  const int n = a.meta[a.plan.qe[p] - 1].pos + 1;
   int32_t* out = a.cols + ((static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g) * a.c;
   int* nout = a.ncols + (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
   if (a.forced_on && a.forced_on[0]) {
@@ -1274,7 +1275,26 @@ __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
     if (threadIdx.x == 0) *nout = fn;
     return;
   }
-  const int got = block_topk(a.col_keys + (static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols, n, a.c, out);
+  const float* keys = a.col_keys + (static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols;
+  if (n <= kSelColsSmemKeys) {
+    // the radix passes read every key several times: stage them once, four loads in flight per thread
+    for (int e0 = 0; e0 < n; e0 += 4 * blockDim.x) {
+      float v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * blockDim.x + threadIdx.x;
+        v[u] = e < n ? keys[e] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e0 + u * blockDim.x + threadIdx.x;
+        if (e < n) keys_sm[e] = v[u];
+      }
+    }
+    __syncthreads();
+    keys = keys_sm;
+  }
+  const int got = block_topk(keys, n, a.c, out);
   if (threadIdx.x == 0) *nout = got;
 }
 
@@ -1754,8 +1774,11 @@ cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cud
   }
 #undef FL_DS
 }
+size_t select_cols_smem(int max_cols) {
+  return static_cast<size_t>(max_cols < kSelColsSmemKeys ? max_cols : kSelColsSmemKeys) * 4;
+}
 cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t s) {
-  return launch_k(g_pdl, k_select_cols, dim3(max_need * a.Hkv), dim3(1024), 0, s, a);
+  return launch_k(g_pdl, k_select_cols, dim3(max_need * a.Hkv), dim3(1024), select_cols_smem(a.max_cols), s, a);
 }
 size_t corr_cluster_smem(int hd, int grp) { return static_cast<size_t>(kCorrWarps) * grp * hd * 4; }
 template <typename K, typename A>
@@ -1854,6 +1877,7 @@ cudaError_t kernels_init_attrs() {
   set(k_attn_decode<64, 2>, static_cast<int>(attn_decode_smem(64)));
   set(k_attn_decode<64, 4>, static_cast<int>(attn_decode_smem(64)));
   set(k_attn_decode<64, 8>, static_cast<int>(attn_decode_smem(64)));
+  set(k_select_cols, static_cast<int>(select_cols_smem(kSelColsSmemKeys)));
   set(k_attn_prefill<128>, static_cast<int>(attn_prefill_smem(128)));
   set(k_attn_prefill<64>, static_cast<int>(attn_prefill_smem(64)));
   set(k_dscore<128, 4, 2>, static_cast<int>(dscore_smem(128)));

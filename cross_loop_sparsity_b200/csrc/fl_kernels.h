@@ -107,6 +107,7 @@ struct DScoreArgs {
   const int32_t* idx;
   const int* seq;
   const int* pos;
+  const SelMeta* meta;  // [n_sel] per selected slot
   const float* q_cur;   // GEMM order
   const float* q_last;  // token order (this layer)
   CacheView cv;
@@ -120,6 +121,7 @@ struct SelColsArgs {
   TilePlan plan;
   const int32_t* idx;
   const int* pos;
+  const SelMeta* meta;  // [n_sel] per selected slot
   const float* col_keys;
   int max_cols, Hkv, c, j, n_tiles;
   int32_t* cols;        // [M][n_tiles][Hkv][c]
@@ -166,7 +168,8 @@ struct LensArg {
   int v[kLensByValue];
 };
 cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s);
-constexpr int kCorrWarps = 16;   // warps per CTA of the clustered correction
+constexpr int kCorrWarps = 16;
+constexpr int kSelColsSmemKeys = 16384;   // column keys the top-c kernel stages in shared memory (64 KB)   // warps per CTA of the clustered correction
 constexpr int kCorrCluster = 16;  // CTAs per (query, KV group) in the clustered correction (non-portable size)
 // Launches made while this is on (the kernels of one call) are programmatic
 // dependents of the previous kernel; thread-local.

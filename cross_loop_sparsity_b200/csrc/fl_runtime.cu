@@ -623,12 +623,13 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
         ca.part_acc = ctx->corr_acc; ca.part_mz = ctx->corr_mz; ca.counters = ctx->corr_counters;
         ca.cluster = (decode && n_sel <= kCorrSmallQueries) ? 1 : 0;
         DScoreArgs da{};
-        da.plan = ctx->plan; da.idx = idx; da.seq = ctx->seq; da.pos = ctx->pos; da.q_cur = ctx->q_cur;
+        da.plan = ctx->plan; da.idx = idx; da.seq = ctx->seq; da.pos = ctx->pos; da.meta = ctx->sel_meta;
+        da.q_cur = ctx->q_cur;
         da.q_last = ql; da.cv = ctx->cv; da.j = j; da.loop = l; da.H = H; da.Hkv = Hkv; da.hd = hd; da.tau = tau;
         da.col_keys = ctx->col_keys; da.max_cols = c.max_ctx;
         FL_LAUNCH(FL_KIND_DSCORE, launch_dscore(da, max_need, max_chunks, s));
         SelColsArgs sa{};
-        sa.plan = ctx->plan; sa.idx = idx; sa.pos = ctx->pos; sa.col_keys = ctx->col_keys;
+        sa.plan = ctx->plan; sa.idx = idx; sa.pos = ctx->pos; sa.meta = ctx->sel_meta; sa.col_keys = ctx->col_keys;
         sa.max_cols = c.max_ctx; sa.Hkv = Hkv; sa.c = c.c_cols; sa.j = j; sa.n_tiles = ctx->n_tiles_max;
         sa.cols = ctx->cols; sa.ncols = ctx->ncols; sa.forced_on = ctx->forced_on;
         sa.forced_cols = ctx->forced_cols; sa.forced_ncols = ctx->forced_ncols;
