@@ -65,7 +65,8 @@ __device__ __forceinline__ float block_sum(float v, float* buf /*[32]*/) {
 // ============================================================================
 
 __device__ int block_topk(const float* __restrict__ keys, int n, int k, int32_t* __restrict__ out) {
-  __shared__ int hist[256];
+  __shared__ int whist[16 * 256];   // digit histograms, one per pair of warps (one per warp below 16 warps)
+  __shared__ int wgt[32], weq[32], wtot[256];
   __shared__ int sh_sel, sh_cum;
   __shared__ int scan_buf[33];
   __shared__ uint32_t small_keys[1024];
@@ -97,57 +98,159 @@ __device__ int block_topk(const float* __restrict__ keys, int n, int k, int32_t*
     __syncthreads();
     return k;
   }
+  // radix select: warp w owns keys [w*chunk, (w+1)*chunk) and shares a
+  // 256-bin histogram per 8-bit digit with at most one other warp (no
+  // block-wide atomics); one warp finds the digit holding the k_rem-th largest
+  // key; two block barriers per digit
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int nh = nw < 16 ? nw : 16;
+  const int chunk = (n + nw - 1) / nw;
+  const int lo = min(n, w * chunk), hi = min(n, lo + chunk);
+  int* wh = whist + (w % nh) * 256;
   uint32_t prefix = 0, mask = 0;
   int k_rem = k;
   for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    if (w < nh)
+#pragma unroll
+      for (int b = lane; b < 256; b += 32) wh[b] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t u = kb[i];
-      if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 0xFF], 1);
+    for (int i0 = lo; i0 < hi; i0 += 32) {
+      // keys of similar magnitude share their leading digits: when every
+      // candidate lane of the warp hits the same bin, one atomic adds them all
+      const int i = i0 + lane;
+      const uint32_t u = i < hi ? kb[i] : 0u;
+      const bool in = i < hi && (u & mask) == prefix;
+      const int bin = static_cast<int>((u >> shift) & 0xFF);
+      const unsigned inb = __ballot_sync(0xffffffffu, in);
+      if (inb == 0u) continue;
+      const int b0 = __shfl_sync(0xffffffffu, bin, __ffs(inb) - 1);
+      if (__all_sync(0xffffffffu, !in || bin == b0)) {
+        if (lane == 0) atomicAdd(&wh[b0], __popc(inb));
+      } else if (in) {
+        atomicAdd(&wh[bin], 1);
+      }
     }
     __syncthreads();
-    // the digit holding the k_rem-th largest key: a scan over the bins in
-    // descending digit order (thread t < 256 holds digit 255 - t)
-    const int cnt = threadIdx.x < 256 ? hist[255 - threadIdx.x] : 0;
-    int tot;
-    const int before = block_exclusive_scan(cnt, &tot, scan_buf);
-    if (threadIdx.x < 256 && before < k_rem && before + cnt >= k_rem) {
-      sh_sel = 255 - threadIdx.x;
-      sh_cum = before;
+    // fold the histograms: thread t < 256 totals digit t
+    if (threadIdx.x < 256) {
+      int c = 0;
+      for (int ww = 0; ww < nh; ++ww) c += whist[ww * 256 + threadIdx.x];
+      wtot[threadIdx.x] = c;
+    }
+    __syncthreads();
+    if (w == 0) {
+      // lane L totals digits 255-8L .. 248-8L (descending), then a warp scan
+      int cnt[8], tot = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        cnt[e] = wtot[255 - 8 * lane - e];
+        tot += cnt[e];
+      }
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int before = incl - tot;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if (before < k_rem && before + cnt[e] >= k_rem) {
+          sh_sel = 255 - 8 * lane - e;
+          sh_cum = before;
+        }
+        before += cnt[e];
+      }
     }
     __syncthreads();
     k_rem -= sh_cum;
     prefix |= static_cast<uint32_t>(sh_sel) << shift;
     mask |= 0xFFu << shift;
-    __syncthreads();
   }
-  // prefix = bit pattern of the k-th largest key; take k_rem of the keys equal to it.
-  int eq_off = 0, out_off = 0;
-  for (int base = 0; base < n; base += blockDim.x) {
-    const int i = base + threadIdx.x;
-    const uint32_t u = i < n ? kb[i] : 0u;
-    const int gt = (i < n && u > prefix) ? 1 : 0;
-    const int eq = (i < n && u == prefix) ? 1 : 0;
-    int eq_total;
-    const int eq_rank = eq_off + block_exclusive_scan(eq, &eq_total, scan_buf);
-    const int take = gt | (eq & (eq_rank < k_rem ? 1 : 0));
-    int take_total;
-    const int pos = out_off + block_exclusive_scan(take, &take_total, scan_buf);
-    if (take) out[pos] = i;
-    eq_off += eq_total;
-    out_off += take_total;
+  // prefix = bit pattern of the k-th largest key: take every key above it and
+  // the k_rem lowest-index keys equal to it, in index order.  Each warp counts
+  // its range, one warp turns the counts into offsets, each warp writes.
+  int gt_n = 0, eq_n = 0;
+  for (int i0 = lo; i0 < hi; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t u = i < hi ? kb[i] : 0u;
+    gt_n += __popc(__ballot_sync(0xffffffffu, i < hi && u > prefix));
+    eq_n += __popc(__ballot_sync(0xffffffffu, i < hi && u == prefix));
+  }
+  if (lane == 0) {
+    wgt[w] = gt_n;
+    weq[w] = eq_n;
+  }
+  __syncthreads();
+  if (w == 0) {
+    const int g0 = lane < nw ? wgt[lane] : 0, e0 = lane < nw ? weq[lane] : 0;
+    int ge = e0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, ge, o);
+      if (lane >= o) ge += y;
+    }
+    const int eq_before = ge - e0;
+    const int take_eq = max(0, min(e0, k_rem - eq_before));
+    int tk = g0 + take_eq, incl = tk;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane < nw) {
+      weq[lane] = eq_before;         // equal keys in earlier warps
+      wgt[lane] = incl - tk;         // output slots taken by earlier warps
+    }
+  }
+  __syncthreads();
+  int eq_seen = weq[w], pos0 = wgt[w];
+  const unsigned lt = (1u << lane) - 1u;
+  for (int i0 = lo; i0 < hi; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t u = i < hi ? kb[i] : 0u;
+    const bool eq = i < hi && u == prefix;
+    const unsigned eqb = __ballot_sync(0xffffffffu, eq);
+    const bool take = (i < hi && u > prefix) || (eq && eq_seen + __popc(eqb & lt) < k_rem);
+    const unsigned tb = __ballot_sync(0xffffffffu, take);
+    if (take) out[pos0 + __popc(tb & lt)] = i;
+    eq_seen += __popc(eqb);
+    pos0 += __popc(tb);
   }
   __syncthreads();
   return k;
+}
+
+// copy n keys into shared memory, four loads in flight per thread
+__device__ __forceinline__ void stage_keys(const float* __restrict__ src, int n, float* dst) {
+  for (int e0 = 0; e0 < n; e0 += 4 * blockDim.x) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = e0 + u * blockDim.x + threadIdx.x;
+      v[u] = e < n ? src[e] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = e0 + u * blockDim.x + threadIdx.x;
+      if (e < n) dst[e] = v[u];
+    }
+  }
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(1024) k_topk_segments(const float* __restrict__ keys, int n, int k,
                                                         int32_t* __restrict__ idx) {
   pdl_trigger();
   pdl_wait();
+  extern __shared__ float keys_sm[];   // [n] when n <= kSelColsSmemKeys
   const int s = blockIdx.x;
-  block_topk(keys + static_cast<size_t>(s) * n, n, k, idx + static_cast<size_t>(s) * (k < n ? k : n));
+  const float* src = keys + static_cast<size_t>(s) * n;
+  if (n <= kSelColsSmemKeys) {
+    stage_keys(src, n, keys_sm);
+    src = keys_sm;
+  }
+  block_topk(src, n, k, idx + static_cast<size_t>(s) * (k < n ? k : n));
 }
 
 // Token selection of a lazy loop: top-n_sel over the N keys, or the forced
@@ -1100,7 +1203,7 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
   constexpr int SL = 512;
   const int nsl = (a.d + SL - 1) / SL;
   const bool norm = a.norm_gain != nullptr;
-  __shared__ float s_ss[kSelectStepMaxNorm * kSelectStepSlices];
+  float* s_ss = s_key;   // [kSelectStepMaxNorm * kSelectStepSlices]; the keys are dead after the selection
   for (int it = warp; it < a.n_sel * nsl; it += nw) {
     const int r = it / nsl, c0 = (it % nsl) * SL;
     const float* src = a.h + static_cast<size_t>(s_idx[r]) * a.d;
@@ -1276,22 +1379,8 @@ __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
     return;
   }
   const float* keys = a.col_keys + (static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols;
-  if (n <= kSelColsSmemKeys) {
-    // the radix passes read every key several times: stage them once, four loads in flight per thread
-    for (int e0 = 0; e0 < n; e0 += 4 * blockDim.x) {
-      float v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e0 + u * blockDim.x + threadIdx.x;
-        v[u] = e < n ? keys[e] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e0 + u * blockDim.x + threadIdx.x;
-        if (e < n) keys_sm[e] = v[u];
-      }
-    }
-    __syncthreads();
+  if (n <= kSelColsSmemKeys) {   // the radix passes read every key several times: stage them once
+    stage_keys(keys, n, keys_sm);
     keys = keys_sm;
   }
   const int got = block_topk(keys, n, a.c, out);
@@ -1670,7 +1759,8 @@ thread_local bool g_pdl = false;
 void set_pdl(bool on) { g_pdl = on; }
 
 cudaError_t launch_topk(const float* keys, int n_seg, int n, int k, int32_t* idx, cudaStream_t s) {
-  return launch_k(false, k_topk_segments, dim3(n_seg), dim3(1024), 0, s, keys, n, k, idx);
+  const size_t sm = n <= kSelColsSmemKeys ? static_cast<size_t>(n) * 4 : 0;
+  return launch_k(false, k_topk_segments, dim3(n_seg), dim3(1024), sm, s, keys, n, k, idx);
 }
 cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* idx, const int* forced_on,
                                  const int32_t* forced, cudaStream_t s) {
@@ -1878,6 +1968,7 @@ cudaError_t kernels_init_attrs() {
   set(k_attn_decode<64, 4>, static_cast<int>(attn_decode_smem(64)));
   set(k_attn_decode<64, 8>, static_cast<int>(attn_decode_smem(64)));
   set(k_select_cols, static_cast<int>(select_cols_smem(kSelColsSmemKeys)));
+  set(k_topk_segments, static_cast<int>(select_cols_smem(kSelColsSmemKeys)));
   set(k_attn_prefill<128>, static_cast<int>(attn_prefill_smem(128)));
   set(k_attn_prefill<64>, static_cast<int>(attn_prefill_smem(64)));
   set(k_dscore<128, 4, 2>, static_cast<int>(dscore_smem(128)));

@@ -163,6 +163,7 @@ constexpr int kLensByValue = 256;
 constexpr int kSelectStepMax = 1024;   // tokens (and query tiles) the one-CTA selection kernel handles
 constexpr int kSelectStepMaxNorm = 64;   // selected rows it also normalises (first layer's input)
 constexpr int kSelectStepSlices = 16;    // 512-element slices of a row it normalises (d <= 8192)
+static_assert(kSelectStepMaxNorm * kSelectStepSlices <= kSelectStepMax, "norm sums reuse the key array");
 struct LensArg {
   int n;
   int v[kLensByValue];

@@ -1152,6 +1152,8 @@ static fl_status record(cudaError_t e) {
 fl_status fl_test_topk(const float* keys, int n_seg, int n, int k, int32_t* idx, fl_stream_t stream) {
   if (!keys || !idx || n_seg < 0 || n < 0 || k < 0) return FL_ERR_INVALID_ARG;
   if (n_seg == 0 || n == 0 || k == 0) return FL_OK;
+  const cudaError_t e = kernels_init_attrs();   // shared-memory opt-ins, once
+  if (e != cudaSuccess) return record(e);
   return record(launch_topk(keys, n_seg, n, k, idx, reinterpret_cast<cudaStream_t>(stream)));
 }
 

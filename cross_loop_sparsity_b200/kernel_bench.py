@@ -7,6 +7,9 @@
   5632), TFLOP/s against the measured dense bf16 peak.
 * ``gemm_skinny``: the split-K swap-AB GEMM at the decode shapes (8 tokens),
   weight GB/s against the measured HBM bandwidth.
+* ``topk``: the top-c column selection (bit pattern descending, index
+  ascending) of one decode layer's column keys (4 KV heads x 4097 keys,
+  c = 256) and of a 65537-key row (c = 1024); microseconds per launch.
 * ``quantize``: the KV-residual quantiser over a residual shaped like the
   65536-token context (65536 tokens x 4 layers x 2 (K, V) x 4 KV heads rows of
   128 fp32, int4 / int2, group 64), bytes moved against HBM.
@@ -104,6 +107,21 @@ def gemm_skinny(reps):
     return out
 
 
+def topk(reps):
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl, synth
+    out = []
+    for n_seg, n, k in ((4, 4097, 256), (4, 65537, 1024)):
+        keys = torch.from_numpy(np.stack([synth.make_keys(3 + s, n, "distinct") for s in range(n_seg)])).cuda()
+
+        def run(i):
+            fl.topk(keys, k)
+        ms = _time(run, reps)
+        out.append({"kernel": "topk", "shape": f"{n_seg} rows x {n} keys, k={k}", "ms": ms, "us": ms * 1e3,
+                    "note": "includes the output allocation of the binding"})
+    return out
+
+
 def quantize(reps):
     import ctypes
     import torch
@@ -136,7 +154,7 @@ def main():
     args = ap.parse_args()
     from cross_loop_sparsity_b200 import build
     build.build()
-    for fn in (gemm_wide, gemm_skinny, quantize):
+    for fn in (gemm_wide, gemm_skinny, topk, quantize):
         for line in fn(args.reps):
             print(json.dumps(line), flush=True)
 
