@@ -108,7 +108,7 @@ void set_last_error(const std::string& why);
 struct SelectSeg;  // fwd
 
 cudaError_t launch_topk(const float* keys, int n_seg, int n, int k, int32_t* idx, cudaStream_t s);
-cudaError_t launch_quantize_rows(const float* r, int rows, int width, int g, int bits, uint8_t* codes,
-                                 uint16_t* scales, cudaStream_t s);
+cudaError_t launch_quantize_rows(const float* r, const uint16_t* prev, int rows, int width, int g, int bits,
+                                 uint8_t* codes, uint16_t* scales, cudaStream_t s);
 
 }  // namespace fl

@@ -360,39 +360,57 @@ __device__ __forceinline__ void store_lane_codes(uint8_t* row, int bits, int lan
   }
 }
 
+// Rows of residuals, quantised and packed: r = x (prev == nullptr) or
+// r = fp32(x) - fp32(prev) with prev bf16 (the residual of a new KV row
+// against the previous loop's).  Each warp takes PER row chunks of 32 * EPL
+// values, all loads issued before any arithmetic.  Item indices are 32-bit
+// (the entry point bounds rows * chunks).
 template <int EPL>
-__global__ void __launch_bounds__(256) k_quantize_rows(const float* __restrict__ r, int rows, int width, int g,
+__global__ void __launch_bounds__(256) k_quantize_rows(const float* __restrict__ x,
+                                                       const uint16_t* __restrict__ prev, int rows, int width, int g,
                                                        int bits, uint8_t* __restrict__ codes,
                                                        uint16_t* __restrict__ scales) {
   pdl_trigger();
   pdl_wait();
   constexpr int PER = 4;   // row chunks per warp, loaded together
   const int lane = threadIdx.x & 31;
-  const int chunks = width / (32 * EPL);
-  const long long total = static_cast<long long>(rows) * chunks;
-  const long long w0 = (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * PER;
+  const unsigned chunks = static_cast<unsigned>(width / (32 * EPL));
+  const unsigned total = static_cast<unsigned>(rows) * chunks;
+  const unsigned w0 = (blockIdx.x * 8u + (threadIdx.x >> 5)) * PER;
   float v[PER][EPL];
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
-    const long long w = w0 + u;
-    if (w < total) {
-      const int row = static_cast<int>(w / chunks), ch = static_cast<int>(w % chunks);
-      const float* src = r + static_cast<size_t>(row) * width + ch * 32 * EPL + lane * EPL;
+    const unsigned w = w0 + u;
+    if (w >= total) continue;
+    const unsigned row = chunks == 1u ? w : w / chunks, ch = chunks == 1u ? 0u : w % chunks;
+    const size_t off = static_cast<size_t>(row) * width + ch * 32 * EPL + lane * EPL;
+    if (EPL == 4) {
+      const float4 q = *reinterpret_cast<const float4*>(x + off);
+      v[u][0] = q.x; v[u][EPL > 1 ? 1 : 0] = q.y; v[u][EPL > 2 ? 2 : 0] = q.z; v[u][EPL > 3 ? 3 : 0] = q.w;
+    } else {
+      const float2 q = *reinterpret_cast<const float2*>(x + off);
+      v[u][0] = q.x; v[u][EPL > 1 ? 1 : 0] = q.y;
+    }
+    if (prev) {
       if (EPL == 4) {
-        const float4 x = *reinterpret_cast<const float4*>(src);
-        v[u][0] = x.x; v[u][EPL > 1 ? 1 : 0] = x.y; v[u][EPL > 2 ? 2 : 0] = x.z; v[u][EPL > 3 ? 3 : 0] = x.w;
+        const uint2 pb = *reinterpret_cast<const uint2*>(prev + off);
+        v[u][0] = __fsub_rn(v[u][0], bf16_to_f(pb.x & 0xFFFF));
+        v[u][EPL > 1 ? 1 : 0] = __fsub_rn(v[u][EPL > 1 ? 1 : 0], bf16_to_f(pb.x >> 16));
+        v[u][EPL > 2 ? 2 : 0] = __fsub_rn(v[u][EPL > 2 ? 2 : 0], bf16_to_f(pb.y & 0xFFFF));
+        v[u][EPL > 3 ? 3 : 0] = __fsub_rn(v[u][EPL > 3 ? 3 : 0], bf16_to_f(pb.y >> 16));
       } else {
-        const float2 x = *reinterpret_cast<const float2*>(src);
-        v[u][0] = x.x; v[u][EPL > 1 ? 1 : 0] = x.y;
+        const uint32_t pb = *reinterpret_cast<const uint32_t*>(prev + off);
+        v[u][0] = __fsub_rn(v[u][0], bf16_to_f(pb & 0xFFFF));
+        v[u][EPL > 1 ? 1 : 0] = __fsub_rn(v[u][EPL > 1 ? 1 : 0], bf16_to_f(pb >> 16));
       }
     }
   }
   const int GL = g / EPL;
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
-    const long long w = w0 + u;
+    const unsigned w = w0 + u;
     if (w >= total) break;   // warp-uniform
-    const int row = static_cast<int>(w / chunks), ch = static_cast<int>(w % chunks);
+    const unsigned row = chunks == 1u ? w : w / chunks, ch = chunks == 1u ? 0u : w % chunks;
     int c[EPL];
     const uint16_t sc = quantize_lane<EPL>(v[u], g, bits, c);
     uint8_t* crow = codes + (static_cast<size_t>(row) * width + ch * 32 * EPL) * bits / 8;
@@ -1766,17 +1784,17 @@ cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* i
                                  const int32_t* forced, cudaStream_t s) {
   return launch_k(g_pdl, k_select_tokens, dim3(1), dim3(1024), 0, s, keys, N, n_sel, idx, forced_on, forced);
 }
-cudaError_t launch_quantize_rows(const float* r, int rows, int width, int g, int bits, uint8_t* codes,
-                                 uint16_t* scales, cudaStream_t s) {
+cudaError_t launch_quantize_rows(const float* r, const uint16_t* prev, int rows, int width, int g, int bits,
+                                 uint8_t* codes, uint16_t* scales, cudaStream_t s) {
   // 8 warps per CTA, 4 row chunks per warp
   if (width % 128 == 0) {
     const long long items = static_cast<long long>(rows) * (width / 128);
     return launch_k(false, k_quantize_rows<4>, dim3(static_cast<unsigned>((items + 31) / 32)), dim3(256), 0, s, r,
-                    rows, width, g, bits, codes, scales);
+                    prev, rows, width, g, bits, codes, scales);
   }
   const long long items = static_cast<long long>(rows) * (width / 64);
   return launch_k(false, k_quantize_rows<2>, dim3(static_cast<unsigned>((items + 31) / 32)), dim3(256), 0, s, r,
-                  rows, width, g, bits, codes, scales);
+                  prev, rows, width, g, bits, codes, scales);
 }
 cudaError_t launch_rmsnorm_rows(const float* h, const int* idx, int n, int n_pad, int d, const float* gain, float eps,
                                 uint16_t* x, cudaStream_t s) {

@@ -1157,17 +1157,34 @@ fl_status fl_test_topk(const float* keys, int n_seg, int n, int k, int32_t* idx,
   return record(launch_topk(keys, n_seg, n, k, idx, reinterpret_cast<cudaStream_t>(stream)));
 }
 
-fl_status fl_test_quantize(const float* r, int rows, int width, int g, int bits, uint8_t* codes, uint16_t* scales,
-                           fl_stream_t stream) {
-  if (!r || !codes || !scales || rows < 0 || width <= 0) return FL_ERR_INVALID_ARG;
+namespace {
+// the checks and the launch shared by the two quantiser entry points
+fl_status quantize_entry(const float* x, const uint16_t* prev, int rows, int width, int g, int bits, uint8_t* codes,
+                         uint16_t* scales, fl_stream_t stream) {
+  if (!x || !codes || !scales || rows < 0 || width <= 0) return FL_ERR_INVALID_ARG;
   if (bits != 2 && bits != 4) return FL_ERR_INVALID_ARG;
   if (g != 32 && g != 64 && g != 128) return FL_ERR_INVALID_ARG;
   if (width % g) return FL_ERR_INVALID_ARG;
   if (width % 128 != 0 && width != 64) return FL_ERR_INVALID_ARG;
   if (width == 64 && g > 64) return FL_ERR_INVALID_ARG;
-  if (!aligned16(r)) return FL_ERR_INVALID_ARG;   // rows are read as 16- or 8-byte vectors
+  if (!aligned16(x)) return FL_ERR_INVALID_ARG;   // rows are read as 16- or 8-byte vectors
+  if (prev && !aligned16(prev)) return FL_ERR_INVALID_ARG;
+  if (static_cast<long long>(rows) * (width / 64) >= (1LL << 31)) return FL_ERR_CAPACITY;
   if (rows == 0) return FL_OK;
-  return record(launch_quantize_rows(r, rows, width, g, bits, codes, scales, reinterpret_cast<cudaStream_t>(stream)));
+  return record(
+      launch_quantize_rows(x, prev, rows, width, g, bits, codes, scales, reinterpret_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+fl_status fl_test_quantize(const float* r, int rows, int width, int g, int bits, uint8_t* codes, uint16_t* scales,
+                           fl_stream_t stream) {
+  return quantize_entry(r, nullptr, rows, width, g, bits, codes, scales, stream);
+}
+
+fl_status fl_test_quantize_residual(const float* x, const uint16_t* prev, int rows, int width, int g, int bits,
+                                    uint8_t* codes, uint16_t* scales, fl_stream_t stream) {
+  if (!prev) return FL_ERR_INVALID_ARG;
+  return quantize_entry(x, prev, rows, width, g, bits, codes, scales, stream);
 }
 
 size_t fl_test_gemm_scratch_bytes(int m, int n, int k, int swap_ab) {

@@ -72,6 +72,7 @@ _SIG = {
     "flashloop_kernels_per_call": (_I, [_P]),
     "fl_test_topk": (_I, [_P, _I, _I, _I, _P, _P]),
     "fl_test_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
+    "fl_test_quantize_residual": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
     "fl_test_gemm_scratch_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "fl_test_gemm": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, ctypes.c_size_t, _P]),
     "fl_gemm_skinny_noalloc": (_I, [_P, _P, _P, _I, _I, _I, _P]),
@@ -341,6 +342,18 @@ def quantize(r, g: int, bits: int, stream=None):
     scales = torch.empty((rows, width // g), dtype=torch.int16, device=r.device)
     _check(lib().fl_test_quantize(_ptr(r), rows, width, g, bits, _ptr(codes), _ptr(scales), _stream_ptr(stream)),
            "fl_test_quantize")
+    return codes, scales
+
+
+def quantize_residual(x, prev, g: int, bits: int, stream=None):
+    """x: cuda float32 [rows, width], prev: cuda bf16 (or int16 bits) [rows, width]; quantises
+    r = x - prev; returns (packed codes uint8, fp16 scale bits int16)."""
+    import torch
+    rows, width = x.shape
+    codes = torch.empty((rows, width * bits // 8), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((rows, width // g), dtype=torch.int16, device=x.device)
+    _check(lib().fl_test_quantize_residual(_ptr(x), _ptr(prev), rows, width, g, bits, _ptr(codes), _ptr(scales),
+                                           _stream_ptr(stream)), "fl_test_quantize_residual")
     return codes, scales
 
 

@@ -10,6 +10,16 @@
 * ``topk``: the top-c column selection (bit pattern descending, index
   ascending) of one decode layer's column keys (4 KV heads x 4097 keys,
   c = 256) and of a 65537-key row (c = 1024); microseconds per launch.
+* ``attn_decode``: the loop-1 decode attention measured in situ inside the
+  decode step (CUDA events around each kernel of the replayed graph) at the
+  long-context decode shape (1 token, 65536-token context, 4 KV heads x 128,
+  134 MB of K and V per launch) and at the 8 x 4096 shape (67 MB per launch);
+  the cache is the zero-initialised workspace at full length (the values do
+  not change the work).
+* ``quantize_residual``: the residual quantiser on a c5-shaped KV update
+  (65536 tokens x 4 layers x 4 KV heads x (K, V) rows of 128): reads the new
+  fp32 rows and the previous bf16 rows (1.61 GB), writes packed int4 codes and
+  fp16 scales (0.14 GB); bytes moved against HBM.
 * ``quantize``: the KV-residual quantiser over a residual shaped like the
   65536-token context (65536 tokens x 4 layers x 2 (K, V) x 4 KV heads rows of
   128 fp32, int4 / int2, group 64), bytes moved against HBM.
@@ -148,13 +158,72 @@ def quantize(reps):
     return out
 
 
+def attn_decode(reps):
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl, synth
+    hbm, tc, src = _peaks()
+    out = []
+    for name in ("c5", "c2"):
+        cfg = synth.config(name)
+        w = synth.make_weights(cfg)
+        stream = torch.cuda.Stream()
+        eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=cfg.batch, max_ctx=cfg.ctx_len + 1, stream=stream)
+        lens = [cfg.ctx_len] * cfg.batch
+        h0 = torch.from_numpy(synth.make_h0(cfg, w["rng"], cfg.batch)).cuda()
+        logits = torch.empty((cfg.batch, cfg.vocab), dtype=torch.float32, device="cuda")
+        eng.set_option(fl.FL_OPT_PROFILE, 1)
+        acc, n = 0.0, 0
+        for i in range(reps + 2):
+            eng.reset(lens, stream=stream)
+            eng.decode_step(h0, cfg.batch, None, logits, stream=stream)
+            p = eng.profile(stream)
+            if i >= 2 and "attn" in p:
+                acc += p["attn"][0]
+                n = p["attn"][1]
+        ms = acc / reps / max(1, n)
+        moved = cfg.batch * cfg.n_kv_heads * (cfg.ctx_len + 1) * cfg.head_dim * 2 * 2
+        gbs = moved / (ms * 1e-3) / 1e9
+        out.append({"kernel": "attn_decode", "shape": f"{name}: {cfg.batch} token(s) x {cfg.ctx_len + 1} keys, "
+                    f"{cfg.n_kv_heads} KV heads x {cfg.head_dim}", "ms": ms, "bytes": moved, "achieved": gbs,
+                    "unit": "GB/s", "peak": hbm, "frac": gbs / hbm, "peak_source": f"{src} hbm_gbs",
+                    "note": "in situ, event-bracketed launch inside the replayed decode graph"})
+        eng.close()
+        del eng, w
+        torch.cuda.empty_cache()
+    return out
+
+
+def quantize_residual(reps):
+    import ctypes
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    hbm, tc, src = _peaks()
+    L = fl.lib()
+    rows, width, g, bits = 65536 * 4 * 4 * 2, 128, 64, 4
+    x = torch.randn((rows, width), device="cuda")
+    prev = (x + 0.05 * torch.randn_like(x)).to(torch.bfloat16)
+    codes = torch.empty((rows, width * bits // 8), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((rows, width // g), dtype=torch.int16, device="cuda")
+
+    def run(i):
+        st = L.fl_test_quantize_residual(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(prev.data_ptr()), rows, width,
+                                         g, bits, ctypes.c_void_p(codes.data_ptr()), ctypes.c_void_p(scales.data_ptr()),
+                                         None)
+        assert st == 0
+    ms = _time(run, reps)
+    moved = rows * width * (4 + 2) + rows * width * bits // 8 + rows * (width // g) * 2
+    gbs = moved / (ms * 1e-3) / 1e9
+    return [{"kernel": "quantize_residual", "shape": f"int{bits}: {rows} rows x {width}, g{g}", "ms": ms,
+             "achieved": gbs, "unit": "GB/s", "peak": hbm, "frac": gbs / hbm, "peak_source": f"{src} hbm_gbs"}]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--reps", type=int, default=20)
     args = ap.parse_args()
     from cross_loop_sparsity_b200 import build
     build.build()
-    for fn in (gemm_wide, gemm_skinny, topk, quantize):
+    for fn in (gemm_wide, gemm_skinny, topk, attn_decode, quantize_residual, quantize):
         for line in fn(args.reps):
             print(json.dumps(line), flush=True)
 

@@ -216,6 +216,14 @@ fl_status fl_test_topk(const float* keys, int n_seg, int n, int k, int32_t* idx,
 fl_status fl_test_quantize(const float* r, int rows, int width, int g, int bits,
                            uint8_t* codes, uint16_t* scales, fl_stream_t stream);
 
+/* The quantiser applied to the residual of new KV rows against the previous
+ * loop's reconstruction: r = fp32(x) - fp32(prev) (IEEE round-to-nearest), then
+ * exactly as fl_test_quantize (KV-residual quantisation, "FlashLoop ...",
+ * abstract).  x fp32 [rows][width], prev bf16 [rows][width], both 16-byte
+ * aligned; the other arguments, limits and errors as fl_test_quantize. */
+fl_status fl_test_quantize_residual(const float* x, const uint16_t* prev, int rows, int width, int g, int bits,
+                                    uint8_t* codes, uint16_t* scales, fl_stream_t stream);
+
 /* tcgen05 GEMM: D[m][n] = sum_k A[m][k] * B[n][k] (bf16 operands, fp32
  * accumulate); A [m][k] and B [n][k] row-major bf16, D fp32 [m][n]; k % 8 == 0,
  * all pointers 16-byte aligned.  swap_ab = 0: A's rows on the MMA M side

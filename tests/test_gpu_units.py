@@ -48,6 +48,24 @@ def test_quantize_bit_exact(env, width, g, bits):
     assert np.array_equal(codes, orc.pack_codes(want_c, bits))
 
 
+@pytest.mark.parametrize("width,g,bits", [(128, 64, 4), (128, 32, 2), (64, 32, 4), (256, 128, 2)])
+def test_quantize_residual_bit_exact(env, width, g, bits):
+    # r = x - prev in IEEE fp32 (exact rounding on both sides), then the quantiser
+    torch, fl, orc = env
+    rows = 1500
+    rng = np.random.default_rng(11 + width + g + bits)
+    x = rng.standard_normal((rows, width)).astype(np.float32)
+    prev = (x + 0.05 * rng.standard_normal((rows, width))).astype(np.float32)
+    prev_bits = orc.bf16_round(prev.astype(np.float64)).astype(np.float32).view(np.uint32) >> 16
+    prev_b = prev_bits.astype(np.uint16)
+    r = x - prev_b.astype(np.uint32).__lshift__(16).view(np.float32)
+    codes, scales = fl.quantize_residual(torch.from_numpy(x).cuda(), torch.from_numpy(prev_b.view(np.int16)).cuda(),
+                                         g, bits)
+    want_c, want_s = orc.quantize_groups(r, bits, g)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint16), want_s.view(np.uint16))
+    assert np.array_equal(codes.cpu().numpy(), orc.pack_codes(want_c, bits))
+
+
 def _bf16(torch, rng, shape, scale=1.0):
     x = torch.from_numpy((rng.standard_normal(shape) * scale).astype(np.float32))
     return x.to(torch.bfloat16).cuda()
