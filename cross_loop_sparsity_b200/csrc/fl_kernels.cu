@@ -254,13 +254,13 @@ __global__ void __launch_bounds__(1024) k_topk_segments(const float* __restrict_
 }
 
 // Token selection of a lazy loop: top-n_sel over the N keys, or the forced
-// indices when forced_on[0] is set.
+// indices when forced_on[0] has kForceSel set.
 __global__ void __launch_bounds__(1024) k_select_tokens(const float* __restrict__ keys, int N, int n_sel,
                                                         int32_t* __restrict__ idx, const int* forced_on,
                                                         const int32_t* __restrict__ forced) {
   pdl_trigger();
   pdl_wait();
-  if (forced_on && forced_on[0]) {
+  if (forced_on && (forced_on[0] & kForceSel)) {
     for (int i = threadIdx.x; i < n_sel; i += blockDim.x) idx[i] = forced[i];
     return;
   }
@@ -1192,7 +1192,7 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
     }
   }
   __syncthreads();
-  if (a.forced_on && a.forced_on[0]) {
+  if (a.forced_on && (a.forced_on[0] & kForceSel)) {
     for (int i = threadIdx.x; i < a.n_sel; i += blockDim.x) s_idx[i] = a.forced[i];
   } else {
     block_topk(s_key, a.N, a.n_sel, s_idx);
@@ -1389,7 +1389,7 @@ __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
   const int n = a.meta[a.plan.qe[p] - 1].pos + 1;
   int32_t* out = a.cols + ((static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g) * a.c;
   int* nout = a.ncols + (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
-  if (a.forced_on && a.forced_on[0]) {
+  if (a.forced_on && (a.forced_on[0] & kForceCols)) {
     const size_t off = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
     const int fn = a.forced_ncols[off];
     for (int e = threadIdx.x; e < fn; e += blockDim.x) out[e] = a.forced_cols[off * a.c + e];

@@ -159,6 +159,9 @@ struct CorrectArgs {
 
 cudaError_t kernels_init_attrs();
 
+// forced_on bits: the token selections, the column sets
+constexpr int kForceSel = 1, kForceCols = 2;
+
 constexpr int kLensByValue = 256;
 constexpr int kSelectStepMax = 1024;   // tokens (and query tiles) the one-CTA selection kernel handles
 constexpr int kSelectStepMaxNorm = 64;   // selected rows it also normalises (first layer's input)

@@ -1071,13 +1071,16 @@ fl_status flashloop_force_selection(flashloop_ctx* ctx, const int32_t* sel, int 
                                     const int32_t* cols, const int32_t* ncols, int n_tiles) {
   if (!ctx || !ctx->lazy) return FL_ERR_INVALID_ARG;
   const flashloop_config& c = ctx->cfg;
-  const int on = (sel && cols && ncols) ? 1 : 0;
-  if (on) {
-    if (n_sel_loops != c.n_loops - 1 || n_sel < 1 || n_sel > ctx->N_max || n_tiles < 1 || n_tiles > ctx->n_tiles_max)
-      return FL_ERR_INVALID_ARG;
+  if ((cols == nullptr) != (ncols == nullptr)) return FL_ERR_INVALID_ARG;
+  const int on = (sel ? kForceSel : 0) | (cols ? kForceCols : 0);
+  if ((on & kForceSel) && (n_sel_loops != c.n_loops - 1 || n_sel < 1 || n_sel > ctx->N_max))
+    return FL_ERR_INVALID_ARG;
+  if ((on & kForceCols) && (n_tiles < 1 || n_tiles > ctx->n_tiles_max)) return FL_ERR_INVALID_ARG;
+  if (on & kForceSel)
     for (int l = 0; l < n_sel_loops; ++l)
       FL_TRY(cudaMemcpy(ctx->forced_sel + static_cast<size_t>(l) * ctx->N_max, sel + static_cast<size_t>(l) * n_sel,
                         static_cast<size_t>(n_sel) * 4, cudaMemcpyHostToDevice));
+  if (on & kForceCols) {
     const size_t per_tile = static_cast<size_t>(c.n_kv_heads) * c.c_cols;
     for (int j = 0; j < c.n_layers; ++j) {
       FL_TRY(cudaMemcpy(ctx->forced_cols + static_cast<size_t>(j) * ctx->n_tiles_max * per_tile,

@@ -286,16 +286,23 @@ class FlashLoop:
         return codes.cpu().numpy(), scales.cpu().numpy().view(np.float16)
 
     def force_selection(self, sel=None, cols=None, ncols=None, n_tiles: int = 0):
-        if sel is None:
-            _check(lib().flashloop_force_selection(self.ctx, None, 0, 0, None, None, 0), "force_selection")
-            return
-        sel = np.ascontiguousarray(sel, np.int32)
-        cols = np.ascontiguousarray(cols, np.int32)
-        ncols = np.ascontiguousarray(ncols, np.int32)
-        self._forced_keep = (sel, cols, ncols)
-        _check(lib().flashloop_force_selection(self.ctx, sel.ctypes.data_as(ctypes.c_void_p), sel.shape[0],
-                                               sel.shape[1], cols.ctypes.data_as(ctypes.c_void_p),
-                                               ncols.ctypes.data_as(ctypes.c_void_p), n_tiles),
+        """sel int32 [K-1][n_sel] and/or cols int32 [M][n_tiles][Hkv][c] with
+        ncols [M][n_tiles][Hkv]; a part left None stays free; all None clears."""
+        sel_p, n_loops, n_sel = None, 0, 0
+        cols_p = ncols_p = None
+        keep = []
+        if sel is not None:
+            sel = np.ascontiguousarray(sel, np.int32)
+            keep.append(sel)
+            sel_p, n_loops, n_sel = sel.ctypes.data_as(ctypes.c_void_p), sel.shape[0], sel.shape[1]
+        if cols is not None:
+            cols = np.ascontiguousarray(cols, np.int32)
+            ncols = np.ascontiguousarray(ncols, np.int32)
+            keep += [cols, ncols]
+            cols_p, ncols_p = cols.ctypes.data_as(ctypes.c_void_p), ncols.ctypes.data_as(ctypes.c_void_p)
+        self._forced_keep = keep
+        _check(lib().flashloop_force_selection(self.ctx, sel_p, n_loops, n_sel, cols_p, ncols_p,
+                                               n_tiles if cols is not None else 0),
                "force_selection", self.ctx)
 
     def force_codes(self, codes=None, scales=None):

@@ -175,9 +175,12 @@ fl_status flashloop_export_slice(const flashloop_ctx* ctx, int layer, int loop, 
 /* Force the selections of the next call (checks only): sel [K-1][n_sel]
  * ascending token indices for loops 2..K; cols [M][n_tiles][Hkv][c_cols]
  * ascending column indices with ncols [M][n_tiles][Hkv] valid entries (host
- * arrays; NULL clears).  n_tiles is B for decode, B*ceil(T/q_tile) for
- * prefill.  The kernels still compute every key; only the chosen indices are
- * replaced. */
+ * arrays).  Either part may be NULL: sel NULL leaves the token selection free,
+ * cols and ncols NULL (both) leave the column sets free; all NULL clears.
+ * n_tiles is B for decode, B*ceil(T/q_tile) for prefill.  The kernels still
+ * compute every key; only the chosen indices are replaced.  cols without ncols
+ * (or the reverse), or sizes outside the context's capacity, return
+ * FL_ERR_INVALID_ARG. */
 fl_status flashloop_force_selection(flashloop_ctx* ctx, const int32_t* sel, int n_sel_loops, int n_sel,
                                     const int32_t* cols, const int32_t* ncols, int n_tiles);
 

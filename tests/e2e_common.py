@@ -105,6 +105,8 @@ def load_context(eng, cfg, ctx, dense=False):
 
 
 def run_decode(cfg, lens, forced=True, dense=False, steps=1, extra_ctx=0):
+    """forced: True hands over selections, column sets and codes; "sel" hands
+    over selections and codes only; False hands over nothing."""
     import torch
     from cross_loop_sparsity_b200 import flashloop as fl
     from oracle import flashloop_oracle as orc
@@ -125,7 +127,11 @@ def run_decode(cfg, lens, forced=True, dense=False, steps=1, extra_ctx=0):
         pos = cache.lens[:B].copy()
         ref = orc.decode_step(cfg, W, cache, h0, bf16_ops=bf16_ops(cfg))
         if forced and not dense and cfg.n_loops > 1:
-            eng.force_selection(*forced_arrays(cfg, ref.trace, B), n_tiles=B)
+            sel, cols, ncols = forced_arrays(cfg, ref.trace, B)
+            if forced == "sel":   # token selections and codes handed over, column sets left free
+                eng.force_selection(sel)
+            else:
+                eng.force_selection(sel, cols, ncols, n_tiles=B)
             eng.force_codes(*forced_codes(cfg, cache, ref.trace, np.arange(B), pos))
         h_out = torch.empty((B, cfg.d_model), dtype=torch.float32, device="cuda")
         logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")

@@ -99,6 +99,57 @@ def test_decode_c2_full_size_forced():
         _check_keys(cfg, ref, out, cfg.batch)
 
 
+def _check_free_column_sets(cfg, ref, out, max_swaps, key_tol):
+    """The library chose every column set itself: each has the oracle's size,
+    and the two differ only in columns whose oracle keys lie within key_tol x
+    the largest key of the c-th key (the boundary, where the two sides' fp32
+    and fp64 scores may order near-ties differently).  Returns (sets that agree
+    exactly, largest swap count, largest boundary distance / largest key)."""
+    exact, worst_swaps, worst_dist = 0, 0, 0.0
+    for (j, t, g), C in ref.trace["cols"].items():
+        n = int(out["ncols"][j, t, g])
+        assert n == len(C), (j, t, g)
+        G = out["cols"][j, t, g, :n]
+        assert np.all(np.diff(G) > 0) and G[0] >= 0
+        ck = ref.trace["col_keys"][(j, t, g)].astype(np.float64)
+        diff = np.setxor1d(G, C)
+        assert len(diff) <= 2 * max_swaps, (j, t, g, len(diff))
+        if len(diff):
+            kth = np.sort(ck)[::-1][len(C) - 1]
+            dist = float(np.max(np.abs(ck[diff] - kth)) / np.max(ck))
+            assert dist <= key_tol, (j, t, g, dist)
+            worst_dist = max(worst_dist, dist)
+        worst_swaps = max(worst_swaps, len(diff) // 2)
+        exact += len(diff) == 0
+    return exact, worst_swaps, worst_dist
+
+
+def test_decode_c2_free_column_sets():
+    """Selections and codes handed over, column sets left free: the library's
+    delta-score keys and top-c choose every set (tile-first recomputation)."""
+    cfg = synth.config("c2")
+    cfg, cache, eng, results = E.run_decode(cfg, [cfg.ctx_len] * cfg.batch, forced="sel")
+    for ref, out in results:
+        assert out["status"] == 0
+        n_sets = len(ref.trace["cols"])
+        exact, swaps, dist = _check_free_column_sets(cfg, ref, out, max_swaps=cfg.c_cols // 16, key_tol=2e-2)
+        print(f"column sets: {exact} of {n_sets} identical to the oracle's; at most {swaps} swaps, "
+              f"boundary distance <= {dist:.2e} of the largest key")
+        _check_outputs(ref, out, tol=2 * E.TOL)
+
+
+def test_decode_ragged_free_column_sets():
+    """The same with ragged contexts shorter than c (the whole causal prefix is
+    the set) and longer ones, several selected tokens and two steps."""
+    cfg = synth.config("c1").with_(mode="decode", batch=5, rho=0.4, c_cols=24, seed=23, seq_len=0)
+    cfg, cache, eng, results = E.run_decode(cfg, [150, 12, 1, 77, 300], forced="sel", steps=2)
+    for ref, out in results:
+        assert out["status"] == 0
+        exact, swaps, dist = _check_free_column_sets(cfg, ref, out, max_swaps=2, key_tol=2e-2)
+        print(f"column sets: {exact} of {len(ref.trace['cols'])} identical; at most {swaps} swaps, "
+              f"boundary distance <= {dist:.2e}")
+
+
 def test_decode_c2_dense_baseline():
     cfg = synth.config("c2").with_(ctx_len=1024)
     cfg, cache, eng, results = E.run_decode(cfg, [1024] * cfg.batch, dense=True)
