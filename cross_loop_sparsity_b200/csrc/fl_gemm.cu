@@ -492,6 +492,254 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
   }
 }
 
+// ============================================================================
+// Persistent GEMM of the wide (prefill) orientation: D[m][n] = sum_k A[m][k]
+// B[n][k] with A the token rows and B the weights, both bf16 K-major.  Output
+// tiles are 128 tokens x 256 features (one N = 256 MMA per k-step), or with two
+// weight operands 128 x (128 + 128) (two N = 128 MMAs into adjacent
+// accumulator columns, for SiLU(gate) * up).  One CTA per SM walks the tiles
+// t = blockIdx.x, blockIdx.x + gridDim.x, ... (feature tile fastest); the ring
+// runs continuously across tile boundaries, and two 256-column TMEM
+// accumulators let the epilogue of one tile overlap the MMAs of the next.
+//   warp 0: TMA producer; warp 1: TMEM owner and MMA issuer; warps 2-5: epilogue
+// ============================================================================
+constexpr int kWideBN = 256;                                 // accumulator columns per tile
+constexpr int kWideStageBytes = kABytes + kWideBN * kBoxK * 2;   // 16 KB tokens + 32 KB weights
+constexpr int kWideStages = 4;
+constexpr int kWideSmemBytes = 1024 + kWideStages * kWideStageBytes + 256;
+
+// Epilogue of 16 consecutive features of one token row (vector stores when the
+// 16 lie inside the output and the row is 16-byte aligned).
+__device__ __forceinline__ void epi_wide16(const GemmArgs& p, int tok, int f0, const float* v0, const float* v1) {
+  if (tok >= p.n_tok || f0 >= p.n_feat) return;
+  const bool full = f0 + 16 <= p.n_feat;
+  if (p.epi == kEpiStore) {
+    float* dst = p.out + static_cast<size_t>(tok) * p.ldo + f0;
+    if (full && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+#pragma unroll
+      for (int c = 0; c < 16; c += 4)
+        *reinterpret_cast<float4*>(dst + c) = make_float4(v0[c], v0[c + 1], v0[c + 2], v0[c + 3]);
+    } else {
+      for (int c = 0; c < 16 && f0 + c < p.n_feat; ++c) dst[c] = v0[c];
+    }
+  } else if (p.epi == kEpiResid) {
+    const int r = p.idx ? p.idx[tok] : tok;
+    float* dst = p.h + static_cast<size_t>(r) * p.ldh + f0;
+    if (full && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+      float4 hv[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) hv[c] = *reinterpret_cast<const float4*>(dst + 4 * c);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        *reinterpret_cast<float4*>(dst + 4 * c) =
+            make_float4(hv[c].x + p.scale * v0[4 * c], hv[c].y + p.scale * v0[4 * c + 1],
+                        hv[c].z + p.scale * v0[4 * c + 2], hv[c].w + p.scale * v0[4 * c + 3]);
+    } else {
+      for (int c = 0; c < 16 && f0 + c < p.n_feat; ++c) dst[c] = dst[c] + p.scale * v0[c];
+    }
+  } else {
+    uint16_t* dst = p.act + static_cast<size_t>(tok) * p.ld_act + f0;
+    if (full && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+      uint32_t w[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        w[c] = f_to_bf16(silu_f(v0[2 * c]) * v1[2 * c]) |
+               (static_cast<uint32_t>(f_to_bf16(silu_f(v0[2 * c + 1]) * v1[2 * c + 1])) << 16);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(dst + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+    } else {
+      for (int c = 0; c < 16 && f0 + c < p.n_feat; ++c) dst[c] = f_to_bf16(silu_f(v0[c]) * v1[c]);
+    }
+  }
+}
+
+template <bool DB>
+__global__ void __launch_bounds__(kThreads, 1)
+k_gemm_wide(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB0,
+            const __grid_constant__ CUtensorMap tmB1, const GemmArgs p, const int b_3d, const int tiles_m,
+            const int tiles_n) {
+  constexpr int kFeatPerTile = DB ? kWideBN / 2 : kWideBN;   // output features of one tile
+  constexpr int kHalfB = 128 * kBoxK * 2;                      // one 128-row weight box
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kWideStages * kWideStageBytes);
+  uint64_t* empty = full + kWideStages;
+  uint64_t* acc_full = empty + kWideStages;   // [2] the MMAs of a tile have completed
+  uint64_t* acc_empty = acc_full + 2;         // [2] the epilogue has read the accumulator
+  uint64_t* done = acc_empty + 2;             // teardown: every issued MMA has completed
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* issued_out = abort_flag + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = tiles_m * tiles_n, nch = p.k_chunks;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kWideStages; ++s) {
+      mbar_init(smem_u32(&full[s]), 1);
+      mbar_init(smem_u32(&empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&acc_full[b]), 1);
+      mbar_init(smem_u32(&acc_empty[b]), 4);   // one arrival per epilogue warp
+    }
+    mbar_init(smem_u32(done), 1);
+    *abort_flag = 0;
+    *issued_out = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(const_cast<uint32_t*>(tmem_slot)), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // dependents may start only now: a dependent CTA that took TMEM on this SM
+  // before this CTA's allocation would wait for this grid while holding it
+  pdl_trigger();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB0);
+    if (DB) tma_prefetch_desc(&tmB1);
+    auto load_w = [&](int tile_n, int i, uint8_t* st, uint32_t fb) {
+      const int kx = i * kBoxK;
+      uint8_t* sb = st + kABytes;
+      const int r0 = DB ? tile_n * 128 : tile_n * 256;
+      const int r1 = DB ? r0 : r0 + 128;
+      const CUtensorMap* m1 = DB ? &tmB1 : &tmB0;
+      if (b_3d) {
+        tma_load_3d(smem_u32(sb), &tmB0, fb, kx, r0, p.b_z);
+        tma_load_3d(smem_u32(sb + kHalfB), m1, fb, kx, r1, p.b_z);
+      } else {
+        tma_load_2d(smem_u32(sb), &tmB0, fb, kx, r0);
+        tma_load_2d(smem_u32(sb + kHalfB), m1, fb, kx, r1);
+      }
+    };
+    // the weights of the first tile's first ring slots do not depend on the
+    // predecessor grid: request them before waiting on it
+    int it = 0, pre = 0;
+    if (static_cast<int>(blockIdx.x) < n_tiles) {
+      pre = nch < kWideStages ? nch : kWideStages;
+      for (int i = 0; i < pre; ++i) {
+        const uint32_t fb = smem_u32(&full[i]);
+        mbar_arrive_expect_tx(fb, kWideStageBytes);
+        load_w(static_cast<int>(blockIdx.x) % tiles_n, i, smem + i * kWideStageBytes, fb);
+      }
+    }
+    pdl_wait();
+    for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x) {
+      const int tile_n = t % tiles_n, tile_m = t / tiles_n;
+      for (int i = 0; i < nch; ++i, ++it) {
+        const int s = it % kWideStages;
+        uint8_t* st = smem + s * kWideStageBytes;
+        const uint32_t fb = smem_u32(&full[s]);
+        if (it >= pre) {
+          if (it >= kWideStages &&
+              !mbar_wait(smem_u32(&empty[s]), ((it / kWideStages) & 1) ^ 1u, p.status)) {
+            *abort_flag = 1;
+            break;
+          }
+          mbar_arrive_expect_tx(fb, kWideStageBytes);
+          load_w(tile_n, i, st, fb);
+        }
+        tma_load_2d(smem_u32(st), &tmA, fb, i * kBoxK, tile_m * 128);
+      }
+    }
+    *issued_out = it > pre ? it : pre;
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc = umma_idesc_bf16(128, DB ? 128 : 256);
+    int it = 0, tl = 0;
+    for (int t = blockIdx.x; t < n_tiles && !*abort_flag; t += gridDim.x, ++tl) {
+      const int b = tl & 1;
+      // accumulator b was last used by local tile tl - 2: wait until the epilogue has read it
+      if (tl >= 2 && !mbar_wait(smem_u32(&acc_empty[b]), ((tl >> 1) & 1) ^ 1u, p.status)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t acc = tmem + b * kWideBN;
+      bool ok = true;
+      for (int i = 0; i < nch; ++i, ++it) {
+        const int s = it % kWideStages;
+        if (!mbar_wait(smem_u32(&full[s]), (it / kWideStages) & 1, p.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(smem + s * kWideStageBytes);
+        const uint32_t b0 = a0 + kABytes;
+#pragma unroll
+        for (int kk = 0; kk < kBoxK / 16; ++kk) {
+          const uint32_t accf = (i > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t da = umma_desc_sw128(a0 + kk * 32);
+          tc_mma_bf16(acc, da, umma_desc_sw128(b0 + kk * 32), idesc, accf);
+          if (DB) tc_mma_bf16(acc + 128, da, umma_desc_sw128(b0 + kHalfB + kk * 32), idesc, accf);
+        }
+        tc_commit(smem_u32(&empty[s]));
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_commit(smem_u32(&acc_full[b]));
+    }
+  } else if (warp >= 2) {
+    // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. +31
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    pdl_wait();
+    int tl = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
+      const int b = tl & 1;
+      if (!mbar_wait(smem_u32(&acc_full[b]), (tl >> 1) & 1, p.status)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int tile_n = t % tiles_n, tile_m = t / tiles_n;
+      const uint32_t tb = tmem + b * kWideBN + (static_cast<uint32_t>(q * 32) << 16);
+      const int tok = tile_m * 128 + row;
+#pragma unroll 1
+      for (int c = 0; c < kFeatPerTile; c += 16) {
+        float v0[16], v1[16];
+        tmem_ld16(tb + c, v0);
+        if (DB) tmem_ld16(tb + 128 + c, v1);
+        tc_wait_ld();
+        epi_wide16(p, tok, tile_n * kFeatPerTile + c, v0, v1);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[b]));
+    }
+  }
+  __syncthreads();
+  if (*abort_flag) {
+    // a wait ran out: let every issued MMA complete and the copies still in
+    // flight land (both bounded) before TMEM and the ring are released
+    if (warp == 1 && lane == 0) {
+      tc_commit(smem_u32(done));
+      mbar_wait(smem_u32(done), 0, nullptr);
+    }
+    if (warp == 0 && lane == 0) {
+      const int issued = *issued_out;
+      for (int i = (issued > kWideStages ? issued - kWideStages : 0); i < issued; ++i)
+        mbar_wait(smem_u32(&full[i % kWideStages]), (i / kWideStages) & 1, nullptr);
+    }
+    __syncthreads();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
 template <int BN, bool DA, bool DB, bool SWAP>
 cudaError_t launch_one(const GemmLaunch& g, cudaStream_t stream) {
   using C = Cfg<BN, DA, DB>;
@@ -519,6 +767,34 @@ cudaError_t launch_one(const GemmLaunch& g, cudaStream_t stream) {
                   g.a_3d, g.b_3d);
 }
 
+template <bool DB>
+cudaError_t launch_wide(const GemmLaunch& g, cudaStream_t stream) {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+  }
+  constexpr int kFeat = DB ? kWideBN / 2 : kWideBN;
+  const int tiles_m = (g.args.n_tok + 127) / 128;
+  const int tiles_n = (g.args.n_feat + kFeat - 1) / kFeat;
+  const int tiles = tiles_m * tiles_n;
+  if (tiles <= 0) return cudaSuccess;
+  const CUtensorMap& b1 = g.b1 ? *g.b1 : *g.b0;
+  return launch_k(g.pdl, k_gemm_wide<DB>, dim3(tiles < sms ? tiles : sms), dim3(kThreads), kWideSmemBytes, stream,
+                  *g.a0, *g.b0, b1, g.args, g.b_3d, tiles_m, tiles_n);
+}
+
+template <bool DB>
+cudaError_t set_attr_wide() {
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_wide<DB>, cudaFuncAttributeMaxDynamicSharedMemorySize, kWideSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_wide<DB>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+  return e;
+}
+
 template <int BN, bool DA, bool DB, bool SWAP>
 cudaError_t set_attr() {
   auto kern = k_gemm_tc<BN, DA, DB, SWAP>;
@@ -537,10 +813,10 @@ cudaError_t set_attr() {
 cudaError_t gemm_init_attrs() {
   static cudaError_t done = cudaErrorNotReady;
   if (done == cudaSuccess) return done;
-  const cudaError_t r[8] = {set_attr<16, true, false, true>(),   set_attr<16, false, false, true>(),
-                            set_attr<32, true, false, true>(),   set_attr<32, false, false, true>(),
-                            set_attr<64, true, false, true>(),   set_attr<64, false, false, true>(),
-                            set_attr<128, false, true, false>(), set_attr<128, false, false, false>()};
+  const cudaError_t r[8] = {set_attr<16, true, false, true>(), set_attr<16, false, false, true>(),
+                            set_attr<32, true, false, true>(), set_attr<32, false, false, true>(),
+                            set_attr<64, true, false, true>(), set_attr<64, false, false, true>(),
+                            set_attr_wide<true>(),             set_attr_wide<false>()};
   done = cudaSuccess;
   for (cudaError_t e : r)
     if (e != cudaSuccess) done = e;
@@ -564,8 +840,8 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
       default: return cudaErrorInvalidValue;
     }
   }
-  if (da || g.bn != 128 || g.args.splits != 1) return cudaErrorInvalidValue;
-  return db ? launch_one<128, false, true, false>(g, stream) : launch_one<128, false, false, false>(g, stream);
+  if (da || g.bn != 128 || g.args.splits != 1 || g.a_3d) return cudaErrorInvalidValue;
+  return db ? launch_wide<true>(g, stream) : launch_wide<false>(g, stream);
 }
 
 // ---------------------------------------------------------------- tensor maps
