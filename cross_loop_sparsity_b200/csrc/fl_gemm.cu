@@ -1,16 +1,24 @@
 // fl_gemm.cu -- the shared-block GEMMs on 5th-generation tensor cores.
 //
-// One CTA computes one 128 x BN output tile (or one K-split of it):
-//   warp 0      : TMA producer (one thread) filling a STAGES-deep shared-memory ring
+// Both kernels split one CTA into three roles:
+//   warp 0      : TMA producer (one thread) filling a shared-memory ring
 //   warp 1      : TMEM owner and MMA issuer (one thread issues tcgen05.mma)
 //   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4) .. +31 with tcgen05.ld
 // Operands are bf16, K-major, 128-byte swizzled (64 elements per row of a box),
 // accumulation is fp32 in TMEM.  The epilogue is fused: plain fp32 store (QKV,
 // logits), scaled residual scatter-add into the fp32 hidden state (O-proj,
 // down-proj), or SiLU(gate) * up into the bf16 MLP activation (gate/up, which
-// keeps two accumulators).  Split-K partials go to a scratch buffer and the
-// last CTA of a tile (an atomic ticket, no waiting) reduces them in split
-// order, so results do not depend on CTA timing.
+// keeps two accumulators).
+//
+// k_gemm_tc (decode, at most 64 tokens): weights on the MMA M side, tokens on
+// the N side (BN = 16/32/64); the K range is split over about one CTA per SM,
+// the splits of a tile forming one cluster whose partials are summed over
+// distributed shared memory in rank order (or, for callers without a cluster,
+// through global scratch and an atomic ticket), so results do not depend on
+// CTA timing.  It can build its token operand itself from fp32 hidden rows
+// (input RMSNorm).
+// k_gemm_wide (prefill): persistent, 128 x 256 output tiles, two TMEM
+// accumulators so that a tile's epilogue overlaps the next tile's MMAs.
 #include <cooperative_groups.h>
 
 #include "fl_device.cuh"
@@ -25,25 +33,24 @@ namespace {
 constexpr int kThreads = 192;
 constexpr int kBoxK = 64;             // bf16 elements per 128-byte swizzled row
 constexpr int kABytes = 128 * kBoxK * 2;
-// Shared-memory ring budget: the skinny (decode) orientation keeps two CTAs per
-// SM so that a dependent GEMM can become resident and start streaming its
-// weights while the previous kernel still runs; the 128x128 orientation uses
-// one deep ring per SM.  Two skinny CTAs fit one SM's 228 KB with the 1 KB the
-// hardware reserves per CTA and this kernel's 1.25 KB of slack and barriers:
-// 2 * (ring + 2304 + 1024) <= 233472.
+// Shared-memory ring budget of the skinny (decode) kernel: two CTAs per SM, so
+// that a dependent GEMM can become resident and start streaming its weights
+// while the previous kernel still runs.  Two CTAs fit one SM's 228 KB with the
+// 1 KB the hardware reserves per CTA and this kernel's 1.25 KB of slack and
+// barriers: 2 * (ring + 2304 + 1024) <= 233472.
 constexpr int kSmemBudgetSkinny = 113408;
-constexpr int kSmemBudgetWide = 200 * 1024;
 
-template <int BN, bool DA, bool DB>
+// Ring and TMEM layout of the skinny kernel for BN token columns, with one or
+// two (DA: gate and up) weight operands.
+template <int BN, bool DA>
 struct Cfg {
-  static constexpr int kSmemBudget = BN <= 64 ? kSmemBudgetSkinny : kSmemBudgetWide;
+  static constexpr int kSmemBudget = kSmemBudgetSkinny;
   static constexpr int kNA = DA ? 2 : 1;
-  static constexpr int kNB = DB ? 2 : 1;
   static constexpr int kBBytes = BN * kBoxK * 2;
-  static constexpr int kStageBytes = kNA * kABytes + kNB * kBBytes;
+  static constexpr int kStageBytes = kNA * kABytes + kBBytes;
   static constexpr int kStagesRaw = kSmemBudget / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr int kNAcc = (DA || DB) ? 2 : 1;
+  static constexpr int kNAcc = DA ? 2 : 1;
   static constexpr int kColsNeeded = kNAcc * BN;
   static constexpr uint32_t kTmemCols = kColsNeeded <= 32 ? 32 : kColsNeeded <= 64 ? 64
                                         : kColsNeeded <= 128 ? 128 : kColsNeeded <= 256 ? 256 : 512;
@@ -57,20 +64,13 @@ struct Cfg {
 
 __device__ __forceinline__ float silu_f(float x) { return x / (1.0f + expf(-x)); }
 
-template <bool SWAP>
-__device__ __forceinline__ void epi_apply(const GemmArgs& p, int row, int col0, int tile_m, int tile_n, int BN,
-                                          const float* v0, const float* v1) {
-  // row: accumulator row within the 128-row tile; columns col0 .. col0+15
+// Epilogue of the skinny kernel: accumulator row `row` of weight tile tile_m is
+// output feature tile_m * 128 + row; columns col0 .. col0+15 are tokens.
+__device__ __forceinline__ void epi_apply(const GemmArgs& p, int row, int col0, int tile_m, const float* v0,
+                                          const float* v1) {
 #pragma unroll
   for (int c = 0; c < 16; ++c) {
-    int tok, feat;
-    if (SWAP) {
-      feat = tile_m * 128 + row;
-      tok = col0 + c;
-    } else {
-      tok = tile_m * 128 + row;
-      feat = tile_n * BN + col0 + c;
-    }
+    const int feat = tile_m * 128 + row, tok = col0 + c;
     if (tok >= p.n_tok || feat >= p.n_feat) continue;
     if (p.epi == kEpiStore) {
       p.out[static_cast<size_t>(tok) * p.ldo + feat] = v0[c];
@@ -87,17 +87,8 @@ __device__ __forceinline__ void epi_apply(const GemmArgs& p, int row, int col0, 
 // The epilogue of one accumulator element (row, column col).  Returns the
 // updated hidden-state value of a residual epilogue (0 otherwise or if the
 // element is outside the output).
-template <bool SWAP>
-__device__ __forceinline__ float epi_one(const GemmArgs& p, int row, int col, int tile_m, int tile_n, int BN, float v0,
-                                         float v1) {
-  int tok, feat;
-  if (SWAP) {
-    feat = tile_m * 128 + row;
-    tok = col;
-  } else {
-    tok = tile_m * 128 + row;
-    feat = tile_n * BN + col;
-  }
+__device__ __forceinline__ float epi_one(const GemmArgs& p, int row, int col, int tile_m, float v0, float v1) {
+  const int feat = tile_m * 128 + row, tok = col;
   if (tok >= p.n_tok || feat >= p.n_feat) return 0.f;
   if (p.epi == kEpiStore) {
     p.out[static_cast<size_t>(tok) * p.ldo + feat] = v0;
@@ -207,12 +198,11 @@ __device__ __forceinline__ bool build_tokens(const GemmArgs& p, uint8_t* smem, u
   return true;
 }
 
-template <int BN, bool DA, bool DB, bool SWAP>
+template <int BN, bool DA>
 __global__ void __launch_bounds__(kThreads, 2)
 k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-          const __grid_constant__ CUtensorMap tmB0, const __grid_constant__ CUtensorMap tmB1,
-          const GemmArgs p, const int a_3d, const int b_3d) {
-  using C = Cfg<BN, DA, DB>;
+          const __grid_constant__ CUtensorMap tmB0, const GemmArgs p, const int a_3d, const int b_3d) {
+  using C = Cfg<BN, DA>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
@@ -223,7 +213,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
   uint8_t* tail = smem + C::kStages * C::kStageBytes;
   float* tok_scale = reinterpret_cast<float*>(tail + 256);   // [BN] input-norm scales
   float* ssum = reinterpret_cast<float*>(tail + 512);        // [4] per-warp sums of squares
-  const bool in_norm = SWAP && p.in_h != nullptr;
+  const bool in_norm = p.in_h != nullptr;
 
   pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -260,35 +250,19 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
     // activation tiles follow once it has completed.
     auto load_w = [&](int i, uint8_t* st, uint32_t fb) {
       const int kx = (c0 + i) * kBoxK;
-      if (SWAP) {
-        if (a_3d) {
-          tma_load_3d(smem_u32(st), &tmA0, fb, kx, tile_m * 128, p.a_z);
-          if (DA) tma_load_3d(smem_u32(st + kABytes), &tmA1, fb, kx, tile_m * 128, p.a_z);
-        } else {
-          tma_load_2d(smem_u32(st), &tmA0, fb, kx, tile_m * 128);
-          if (DA) tma_load_2d(smem_u32(st + kABytes), &tmA1, fb, kx, tile_m * 128);
-        }
+      if (a_3d) {
+        tma_load_3d(smem_u32(st), &tmA0, fb, kx, tile_m * 128, p.a_z);
+        if (DA) tma_load_3d(smem_u32(st + kABytes), &tmA1, fb, kx, tile_m * 128, p.a_z);
       } else {
-        uint8_t* sb = st + C::kNA * kABytes;
-        if (b_3d) {
-          tma_load_3d(smem_u32(sb), &tmB0, fb, kx, tile_n * BN, p.b_z);
-          if (DB) tma_load_3d(smem_u32(sb + C::kBBytes), &tmB1, fb, kx, tile_n * BN, p.b_z);
-        } else {
-          tma_load_2d(smem_u32(sb), &tmB0, fb, kx, tile_n * BN);
-          if (DB) tma_load_2d(smem_u32(sb + C::kBBytes), &tmB1, fb, kx, tile_n * BN);
-        }
+        tma_load_2d(smem_u32(st), &tmA0, fb, kx, tile_m * 128);
+        if (DA) tma_load_2d(smem_u32(st + kABytes), &tmA1, fb, kx, tile_m * 128);
       }
     };
     auto load_x = [&](int i, uint8_t* st, uint32_t fb) {
       const int kx = (c0 + i) * kBoxK;
-      if (SWAP) {
-        uint8_t* sb = st + C::kNA * kABytes;
-        if (b_3d) tma_load_3d(smem_u32(sb), &tmB0, fb, kx, tile_n * BN, p.b_z);
-        else tma_load_2d(smem_u32(sb), &tmB0, fb, kx, tile_n * BN);
-      } else {
-        if (a_3d) tma_load_3d(smem_u32(st), &tmA0, fb, kx, tile_m * 128, p.a_z);
-        else tma_load_2d(smem_u32(st), &tmA0, fb, kx, tile_m * 128);
-      }
+      uint8_t* sb = st + C::kNA * kABytes;
+      if (b_3d) tma_load_3d(smem_u32(sb), &tmB0, fb, kx, tile_n * BN, p.b_z);
+      else tma_load_2d(smem_u32(sb), &tmB0, fb, kx, tile_n * BN);
     };
     // with an input norm the token operand is built in shared memory, so the
     // producer moves weights only and never waits on the predecessor grid
@@ -338,18 +312,12 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
       const uint32_t a0 = smem_u32(smem + s * C::kStageBytes);
       const uint32_t a1 = a0 + kABytes;
       const uint32_t b0 = a0 + C::kNA * kABytes;
-      const uint32_t b1 = b0 + C::kBBytes;
 #pragma unroll
       for (int kk = 0; kk < kBoxK / 16; ++kk) {
         const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-        const uint64_t da = umma_desc_sw128(a0 + kk * 32);
         const uint64_t db = umma_desc_sw128(b0 + kk * 32);
-        tc_mma_bf16(tmem, da, db, idesc, acc);
-        if (C::kNAcc == 2) {
-          const uint64_t da1 = DA ? umma_desc_sw128(a1 + kk * 32) : da;
-          const uint64_t db1 = DB ? umma_desc_sw128(b1 + kk * 32) : db;
-          tc_mma_bf16(tmem + BN, da1, db1, idesc, acc);
-        }
+        tc_mma_bf16(tmem, umma_desc_sw128(a0 + kk * 32), db, idesc, acc);
+        if (DA) tc_mma_bf16(tmem + BN, umma_desc_sw128(a1 + kk * 32), db, idesc, acc);
       }
       tc_commit(smem_u32(&empty[s]));
     }
@@ -376,7 +344,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
         tmem_ld16(tbase + c, v0);
         if (C::kNAcc == 2) tmem_ld16(tbase + BN + c, v1);
         tc_wait_ld();
-        if (valid) epi_apply<SWAP>(p, row, c, tile_m, tile_n, BN, v0, v1);
+        if (valid) epi_apply(p, row, c, tile_m, v0, v1);
       }
     } else if (p.cluster) {
       // cluster split-K: park this split's partial tile in shared memory
@@ -431,7 +399,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
               if (C::kNAcc == 2) v1[j] += __ldcg(src + static_cast<size_t>(BN + c + j) * 128 + row);
             }
           }
-          epi_apply<SWAP>(p, row, c, tile_m, tile_n, BN, v0, v1);
+          epi_apply(p, row, c, tile_m, v0, v1);
         }
         if (warp == 2 && lane == 0) p.counters[tile_m] = 0;
       }
@@ -469,7 +437,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
           v0s += pv0[q];
           v1s += pv1[q];
         }
-        const float hn = epi_one<SWAP>(p, row, cc, tile_m, tile_n, BN, v0s, v1s);
+        const float hn = epi_one(p, row, cc, tile_m, v0s, v1s);
         if (p.ss_out) {
           // this tile's share of the token's sum of squares, in a fixed order
           const float qs = warp_sum(hn * hn);
@@ -740,12 +708,11 @@ k_gemm_wide(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   }
 }
 
-template <int BN, bool DA, bool DB, bool SWAP>
+template <int BN, bool DA>
 cudaError_t launch_one(const GemmLaunch& g, cudaStream_t stream) {
-  using C = Cfg<BN, DA, DB>;
-  auto kern = k_gemm_tc<BN, DA, DB, SWAP>;
+  using C = Cfg<BN, DA>;
+  auto kern = k_gemm_tc<BN, DA>;
   const CUtensorMap& a1 = g.a1 ? *g.a1 : *g.a0;
-  const CUtensorMap& b1 = g.b1 ? *g.b1 : *g.b0;
   if (g.args.cluster && g.args.splits > 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = g.grid;
@@ -761,10 +728,10 @@ cudaError_t launch_one(const GemmLaunch& g, cudaStream_t stream) {
     attr[1].val.programmaticStreamSerializationAllowed = g.pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, kern, *g.a0, a1, *g.b0, b1, g.args, g.a_3d, g.b_3d);
+    return cudaLaunchKernelEx(&cfg, kern, *g.a0, a1, *g.b0, g.args, g.a_3d, g.b_3d);
   }
-  return launch_k(g.pdl, kern, g.grid, dim3(kThreads), C::kSmemBytes, stream, *g.a0, a1, *g.b0, b1, g.args,
-                  g.a_3d, g.b_3d);
+  return launch_k(g.pdl, kern, g.grid, dim3(kThreads), C::kSmemBytes, stream, *g.a0, a1, *g.b0, g.args, g.a_3d,
+                  g.b_3d);
 }
 
 template <bool DB>
@@ -795,15 +762,15 @@ cudaError_t set_attr_wide() {
   return e;
 }
 
-template <int BN, bool DA, bool DB, bool SWAP>
+template <int BN, bool DA>
 cudaError_t set_attr() {
-  auto kern = k_gemm_tc<BN, DA, DB, SWAP>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN, DA, DB>::kSmemBytes);
+  auto kern = k_gemm_tc<BN, DA>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN, DA>::kSmemBytes);
   // all of the SM's unified L1/shared storage as shared memory, so two skinny CTAs are resident
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   // split-K clusters of the skinny orientation may hold up to 16 CTAs
-  if (e == cudaSuccess && SWAP) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   return e;
 }
 
@@ -813,10 +780,8 @@ cudaError_t set_attr() {
 cudaError_t gemm_init_attrs() {
   static cudaError_t done = cudaErrorNotReady;
   if (done == cudaSuccess) return done;
-  const cudaError_t r[8] = {set_attr<16, true, false, true>(), set_attr<16, false, false, true>(),
-                            set_attr<32, true, false, true>(), set_attr<32, false, false, true>(),
-                            set_attr<64, true, false, true>(), set_attr<64, false, false, true>(),
-                            set_attr_wide<true>(),             set_attr_wide<false>()};
+  const cudaError_t r[8] = {set_attr<16, true>(), set_attr<16, false>(), set_attr<32, true>(), set_attr<32, false>(),
+                            set_attr<64, true>(), set_attr<64, false>(), set_attr_wide<true>(), set_attr_wide<false>()};
   done = cudaSuccess;
   for (cudaError_t e : r)
     if (e != cudaSuccess) done = e;
@@ -834,9 +799,9 @@ cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream) {
   if (g.args.swap) {
     if (db) return cudaErrorInvalidValue;
     switch (g.bn) {
-      case 16: return da ? launch_one<16, true, false, true>(g, stream) : launch_one<16, false, false, true>(g, stream);
-      case 32: return da ? launch_one<32, true, false, true>(g, stream) : launch_one<32, false, false, true>(g, stream);
-      case 64: return da ? launch_one<64, true, false, true>(g, stream) : launch_one<64, false, false, true>(g, stream);
+      case 16: return da ? launch_one<16, true>(g, stream) : launch_one<16, false>(g, stream);
+      case 32: return da ? launch_one<32, true>(g, stream) : launch_one<32, false>(g, stream);
+      case 64: return da ? launch_one<64, true>(g, stream) : launch_one<64, false>(g, stream);
       default: return cudaErrorInvalidValue;
     }
   }

@@ -220,10 +220,15 @@ def quantize_residual(reps):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--only", default="", help="comma-separated subset, e.g. gemm_wide,topk")
     args = ap.parse_args()
     from cross_loop_sparsity_b200 import build
     build.build()
-    for fn in (gemm_wide, gemm_skinny, topk, attn_decode, quantize_residual, quantize):
+    fns = (gemm_wide, gemm_skinny, topk, attn_decode, quantize_residual, quantize)
+    only = {x for x in args.only.split(",") if x}
+    for fn in fns:
+        if only and fn.__name__ not in only:
+            continue
         for line in fn(args.reps):
             print(json.dumps(line), flush=True)
 
