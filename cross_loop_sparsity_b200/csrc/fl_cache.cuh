@@ -18,6 +18,7 @@ namespace fl {
 
 struct CacheView {
   int M, K, B, Hkv, T, hd, g, bits, dense;
+  int lg;   // log2(g): g is a power of two (32, 64, 128, or hd)
   uint16_t* base;
   uint8_t* codes;
   uint16_t* scales;
@@ -37,7 +38,7 @@ struct CacheView {
     return codes + res_index(j, l, kv, b, h, t) * row_bytes_codes();
   }
   __host__ __device__ uint16_t* scale_row(int j, int l, int kv, int b, int h, int t) const {
-    return scales + res_index(j, l, kv, b, h, t) * (hd / g);
+    return scales + res_index(j, l, kv, b, h, t) * (hd >> lg);
   }
 };
 
@@ -85,7 +86,7 @@ __device__ __forceinline__ void chain_lane(const CacheView& cv, int j, int kv, i
     out[0] = bf16_to_f(u & 0xFFFF);
     out[1] = bf16_to_f(u >> 16);
   }
-  const int gi = (lane * EPL) / cv.g;
+  const int gi = (lane * EPL) >> cv.lg;
   for (int l = 2; l <= m; ++l) {
     int c[EPL];
     lane_codes<EPL>(cv.code_row(j, l, kv, b, h, t), cv.bits, lane, c);
@@ -117,8 +118,8 @@ __device__ __forceinline__ void chain_lane2(const CacheView& cv, int j, int kv, 
   } else {
     braw[0] = *reinterpret_cast<const uint32_t*>(br);
   }
-  const int gi = (lane * EPL) / cv.g;
-  const size_t rb = cv.row_bytes_codes(), ns = cv.hd / cv.g;
+  const int gi = (lane * EPL) >> cv.lg;
+  const size_t rb = cv.row_bytes_codes(), ns = cv.hd >> cv.lg;
   const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * cv.T;   // rows between consecutive loops
   const size_t r0 = cv.res_index(j, 2, kv, b, h, t);
   uint32_t craw[KM - 1];

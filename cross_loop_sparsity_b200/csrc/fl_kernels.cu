@@ -304,13 +304,20 @@ __global__ void __launch_bounds__(256) k_rmsnorm_rows(const float* __restrict__ 
 
 // ============================================================================
 // residual quantiser of one group, lane-distributed: the group is GL = g/EPL
-// consecutive lanes.  s = fp16_RU(fp32(absmax / qmax)) (0 if absmax is 0),
+// consecutive lanes, g = 2^lg.  s = fp16_RU(fp32(absmax / qmax)) (0 if absmax is 0),
 // code = clamp(rint(fp32(r / s)), -qmax, qmax), ties to even.
 // Returns the lane's codes and the group's fp16 scale bits.
 // ============================================================================
+// The hardware reciprocal approximation (PTX rcp.approx, within 1 ulp of 1/x).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int EPL>
-__device__ __forceinline__ uint16_t quantize_lane(const float* r, int g, int bits, int* code) {
-  const int GL = g / EPL;
+__device__ __forceinline__ uint16_t quantize_lane(const float* r, int lg, int bits, int* code) {
+  const int GL = 1 << (lg - (EPL == 4 ? 2 : 1));
   float am = 0.f;
 #pragma unroll
   for (int e = 0; e < EPL; ++e) am = fmaxf(am, fabsf(r[e]));
@@ -318,22 +325,24 @@ __device__ __forceinline__ uint16_t quantize_lane(const float* r, int g, int bit
   const int qm = (1 << (bits - 1)) - 1;
   const __half sh = __float2half_ru(__fdiv_rn(am, static_cast<float>(qm)));
   const float s = __half2float(sh);
-  // code = rint of the correctly rounded quotient r/s.  r * (1/s), with 1/s
-  // correctly rounded, is within 2 ulp of that quotient (|r/s| <= qmax + tiny,
-  // so an ulp is at most 2^-21); the nearest integers can differ only when the
-  // product lies within a few ulp of a half-integer, and only then is the
-  // quotient computed exactly.
-  const float inv = s > 0.f ? __frcp_rn(s) : 0.f;
+  // code = rint of the correctly rounded quotient Q = RN(r/s).  Since s >=
+  // absmax/qmax up to one fp32 rounding, |r/s| < 7.01.  q = r * rcp_approx(s)
+  // then lies within 7.01 * 1.5 * 2^-23 of r/s, and so within 1.6 * 2^-20 of Q.
+  // When q is farther than 2^-18 from every half-integer, q and Q round to the
+  // same integer; otherwise Q itself is computed.  Rounding to an integer: the
+  // sum q + 1.5 * 2^23 lies in [2^23, 2^24), where the fp32 spacing is 1, so the
+  // addition rounds q to the nearest integer (ties to even) and leaves it, offset
+  // by 2^22, in the low bits of the sum.
+  const float inv = s > 0.f ? rcp_approx(s) : 0.f;
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
 #pragma unroll
   for (int e = 0; e < EPL; ++e) {
-    int c = 0;
-    if (s > 0.f) {
-      float q = r[e] * inv;
-      if (fabsf(q - (floorf(q) + 0.5f)) <= 0x1p-18f) q = __fdiv_rn(r[e], s);
-      c = __float2int_rn(q);
-      c = c > qm ? qm : (c < -qm ? -qm : c);
-    }
-    code[e] = c;
+    const float q = r[e] * inv;
+    float t = __fadd_rn(q, kMagic);
+    const float d = __fsub_rn(q, __fsub_rn(t, kMagic));   // q - rint(q), exact
+    if (fabsf(d) >= 0.5f - 0x1p-18f && s > 0.f) t = __fadd_rn(__fdiv_rn(r[e], s), kMagic);
+    const int c = __float_as_int(t) - 0x4B400000;
+    code[e] = c > qm ? qm : (c < -qm ? -qm : c);
   }
   return __half_as_ushort(sh);
 }
@@ -405,17 +414,19 @@ __global__ void __launch_bounds__(256) k_quantize_rows(const float* __restrict__
       }
     }
   }
-  const int GL = g / EPL;
+  // g is a power of two (the entry point admits 32, 64, 128): shifts, not divisions
+  const int lg = __ffs(g) - 1, lgl = lg - (EPL == 4 ? 2 : 1);
 #pragma unroll
   for (int u = 0; u < PER; ++u) {
     const unsigned w = w0 + u;
     if (w >= total) break;   // warp-uniform
     const unsigned row = chunks == 1u ? w : w / chunks, ch = chunks == 1u ? 0u : w % chunks;
     int c[EPL];
-    const uint16_t sc = quantize_lane<EPL>(v[u], g, bits, c);
-    uint8_t* crow = codes + (static_cast<size_t>(row) * width + ch * 32 * EPL) * bits / 8;
+    const uint16_t sc = quantize_lane<EPL>(v[u], lg, bits, c);
+    uint8_t* crow = codes + ((static_cast<size_t>(row) * width + ch * 32 * EPL) * bits >> 3);
     store_lane_codes<EPL>(crow, bits, lane, c);
-    if ((lane % GL) == 0) scales[static_cast<size_t>(row) * (width / g) + (ch * 32 * EPL) / g + lane / GL] = sc;
+    if ((lane & ((1 << lgl) - 1)) == 0)
+      scales[(static_cast<size_t>(row) * width >> lg) + ((ch * 32 * EPL) >> lg) + (lane >> lgl)] = sc;
   }
 }
 
@@ -479,7 +490,7 @@ __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
     }
     if (a.lazy) {
       const int rb = static_cast<int>(cv.row_bytes_codes());
-      const int ns = hd / cv.g;
+      const int ns = hd >> cv.lg;
       for (int l = 2; l <= cv.K; ++l) {
         uint8_t* cr = cv.code_row(a.j, l, kv, b, gk, t);
         for (int o = lane; o < rb; o += 32) cr[o] = 0;
@@ -497,18 +508,18 @@ __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
                            a.Hkv + gk;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) c[e] = a.forced_codes[row * hd + lane * EPL + e];
-    s = a.forced_scales[row * (hd / cv.g) + (lane * EPL) / cv.g];
+    s = a.forced_scales[row * (hd >> cv.lg) + ((lane * EPL) >> cv.lg)];
   } else {
     float prev[EPL];
     chain_lane<EPL>(cv, a.j, kv, b, gk, t, a.loop - 1, lane, prev);
     float r[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) r[e] = __fsub_rn(x[e], prev[e]);
-    s = quantize_lane<EPL>(r, cv.g, cv.bits, c);
+    s = quantize_lane<EPL>(r, cv.lg, cv.bits, c);
   }
   store_lane_codes<EPL>(cv.code_row(a.j, a.loop, kv, b, gk, t), cv.bits, lane, c);
-  const int GL = cv.g / EPL;
-  if ((lane % GL) == 0) cv.scale_row(a.j, a.loop, kv, b, gk, t)[lane / GL] = s;
+  const int lgl = cv.lg - (EPL == 4 ? 2 : 1);   // log2 of the lanes per group
+  if ((lane & ((1 << lgl) - 1)) == 0) cv.scale_row(a.j, a.loop, kv, b, gk, t)[lane >> lgl] = s;
 }
 
 constexpr int kDecTile = 64;

@@ -278,6 +278,8 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->dec_splits = splits;
     x->cv.M = M; x->cv.K = K; x->cv.B = c.max_batch; x->cv.Hkv = Hkv; x->cv.T = c.max_ctx; x->cv.hd = hd;
     x->cv.g = lazy ? c.group_size : hd;
+    x->cv.lg = 0;
+    while ((1 << x->cv.lg) < x->cv.g) ++x->cv.lg;
     x->cv.bits = lazy ? c.resid_bits : 16;
     x->cv.dense = lazy ? 0 : 1;
     x->cv.base = reinterpret_cast<uint16_t*>(base);

@@ -48,6 +48,39 @@ def test_quantize_bit_exact(env, width, g, bits):
     assert np.array_equal(codes, orc.pack_codes(want_c, bits))
 
 
+def _tie_residuals(seed, rows, width, g, bits):
+    """Rows whose quotients r/s sit exactly on, and one fp32 ulp either side
+    of, half-integers: each group's first element is qmax * s0 for an fp16
+    value s0 (so s = s0 exactly), the others (k + 1/2) * s0 nudged by -1, 0 or
+    +1 ulp, or a random multiple of s0."""
+    rng = np.random.default_rng(seed)
+    qm = (1 << (bits - 1)) - 1
+    s0 = (2.0 ** rng.integers(-14, 6, size=(rows, width // g, 1))
+          * rng.integers(1024, 2048, size=(rows, width // g, 1)) / 1024.0).astype(np.float16).astype(np.float32)
+    k = rng.integers(-qm, qm, size=(rows, width // g, g)).astype(np.float32)
+    r = ((k + np.float32(0.5)) * s0).astype(np.float32)
+    nudge = rng.integers(-1, 2, size=r.shape)
+    r = np.where(nudge > 0, np.nextafter(r, np.float32(np.inf)),
+                 np.where(nudge < 0, np.nextafter(r, np.float32(-np.inf)), r)).astype(np.float32)
+    rand = rng.random(r.shape) < 0.3
+    r[rand] = (rng.uniform(-qm, qm, size=r.shape).astype(np.float32) * s0 * np.ones_like(r))[rand]
+    r[:, :, 0] = (qm * s0[:, :, 0]).astype(np.float32)
+    r[rng.random(rows) < 0.02] = 0.0
+    return r.reshape(rows, width).astype(np.float32)
+
+
+@pytest.mark.parametrize("width,g,bits", [(128, 64, 4), (128, 32, 2), (64, 32, 4), (256, 128, 4)])
+def test_quantize_ties_bit_exact(env, width, g, bits):
+    """Quotients on and next to half-integers: rint ties to even of the correctly
+    rounded quotient, as the oracle takes it."""
+    torch, fl, orc = env
+    r = _tie_residuals(3 + width + g + bits, 3000, width, g, bits)
+    codes, scales = fl.quantize(torch.from_numpy(r).cuda(), g, bits)
+    want_c, want_s = orc.quantize_groups(r, bits, g)
+    assert np.array_equal(scales.cpu().numpy().view(np.uint16), want_s.view(np.uint16))
+    assert np.array_equal(codes.cpu().numpy(), orc.pack_codes(want_c, bits))
+
+
 @pytest.mark.parametrize("width,g,bits", [(128, 64, 4), (128, 32, 2), (64, 32, 4), (256, 128, 2)])
 def test_quantize_residual_bit_exact(env, width, g, bits):
     # r = x - prev in IEEE fp32 (exact rounding on both sides), then the quantiser
