@@ -315,15 +315,17 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
-template <int EPL>
-__device__ __forceinline__ uint16_t quantize_lane(const float* r, int lg, int bits, int* code) {
+// BITS = 4 or 2 fixes the code width at compile time; 0 takes it from `bits`.
+template <int EPL, int BITS = 0>
+__device__ __forceinline__ uint16_t quantize_lane(const float* r, int lg, int bits_rt, int* code) {
+  const int bits = BITS ? BITS : bits_rt;
   const int GL = 1 << (lg - (EPL == 4 ? 2 : 1));
   float am = 0.f;
 #pragma unroll
   for (int e = 0; e < EPL; ++e) am = fmaxf(am, fabsf(r[e]));
   for (int o = GL >> 1; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
   const int qm = (1 << (bits - 1)) - 1;
-  const __half sh = __float2half_ru(__fdiv_rn(am, static_cast<float>(qm)));
+  const __half sh = __float2half_ru(qm == 1 ? am : __fdiv_rn(am, static_cast<float>(qm)));
   const float s = __half2float(sh);
   // code = rint of the correctly rounded quotient Q = RN(r/s).  Since s >=
   // absmax/qmax up to one fp32 rounding, |r/s| < 7.01.  q = r * rcp_approx(s)
@@ -340,7 +342,7 @@ __device__ __forceinline__ uint16_t quantize_lane(const float* r, int lg, int bi
     const float q = r[e] * inv;
     float t = __fadd_rn(q, kMagic);
     const float d = __fsub_rn(q, __fsub_rn(t, kMagic));   // q - rint(q), exact
-    if (fabsf(d) >= 0.5f - 0x1p-18f && s > 0.f) t = __fadd_rn(__fdiv_rn(r[e], s), kMagic);
+    if (fabsf(d) >= 0.5f - 0x1p-18f) t = __fadd_rn(__fdiv_rn(r[e], s), kMagic);   // (s > 0 here: else q = 0)
     const int c = __float_as_int(t) - 0x4B400000;
     code[e] = c > qm ? qm : (c < -qm ? -qm : c);
   }
@@ -349,8 +351,9 @@ __device__ __forceinline__ uint16_t quantize_lane(const float* r, int lg, int bi
 
 // Pack the lane's codes (two's complement, element order low bits first) and
 // store them into a packed row; for EPL=2 with 2-bit codes two lanes share a byte.
-template <int EPL>
-__device__ __forceinline__ void store_lane_codes(uint8_t* row, int bits, int lane, const int* c) {
+template <int EPL, int BITS = 0>
+__device__ __forceinline__ void store_lane_codes(uint8_t* row, int bits_rt, int lane, const int* c) {
+  const int bits = BITS ? BITS : bits_rt;
   if (EPL == 4) {
     if (bits == 4) {
       const uint32_t u = (c[0] & 0xF) | ((c[1] & 0xF) << 4) | ((c[2] & 0xF) << 8) | ((c[3] & 0xF) << 12);
@@ -374,7 +377,7 @@ __device__ __forceinline__ void store_lane_codes(uint8_t* row, int bits, int lan
 // against the previous loop's).  Each warp takes PER row chunks of 32 * EPL
 // values, all loads issued before any arithmetic.  Item indices are 32-bit
 // (the entry point bounds rows * chunks).
-template <int EPL>
+template <int EPL, int BITS>
 __global__ void __launch_bounds__(256) k_quantize_rows(const float* __restrict__ x,
                                                        const uint16_t* __restrict__ prev, int rows, int width, int g,
                                                        int bits, uint8_t* __restrict__ codes,
@@ -422,9 +425,9 @@ __global__ void __launch_bounds__(256) k_quantize_rows(const float* __restrict__
     if (w >= total) break;   // warp-uniform
     const unsigned row = chunks == 1u ? w : w / chunks, ch = chunks == 1u ? 0u : w % chunks;
     int c[EPL];
-    const uint16_t sc = quantize_lane<EPL>(v[u], lg, bits, c);
-    uint8_t* crow = codes + ((static_cast<size_t>(row) * width + ch * 32 * EPL) * bits >> 3);
-    store_lane_codes<EPL>(crow, bits, lane, c);
+    const uint16_t sc = quantize_lane<EPL, BITS>(v[u], lg, BITS, c);
+    uint8_t* crow = codes + ((static_cast<size_t>(row) * width + ch * 32 * EPL) * BITS >> 3);
+    store_lane_codes<EPL, BITS>(crow, BITS, lane, c);
     if ((lane & ((1 << lgl) - 1)) == 0)
       scales[(static_cast<size_t>(row) * width >> lg) + ((ch * 32 * EPL) >> lg) + (lane >> lgl)] = sc;
   }
@@ -1797,15 +1800,19 @@ cudaError_t launch_select_tokens(const float* keys, int N, int n_sel, int32_t* i
 }
 cudaError_t launch_quantize_rows(const float* r, const uint16_t* prev, int rows, int width, int g, int bits,
                                  uint8_t* codes, uint16_t* scales, cudaStream_t s) {
-  // 8 warps per CTA, 4 row chunks per warp
-  if (width % 128 == 0) {
-    const long long items = static_cast<long long>(rows) * (width / 128);
-    return launch_k(false, k_quantize_rows<4>, dim3(static_cast<unsigned>((items + 31) / 32)), dim3(256), 0, s, r,
-                    prev, rows, width, g, bits, codes, scales);
-  }
-  const long long items = static_cast<long long>(rows) * (width / 64);
-  return launch_k(false, k_quantize_rows<2>, dim3(static_cast<unsigned>((items + 31) / 32)), dim3(256), 0, s, r,
-                  prev, rows, width, g, bits, codes, scales);
+  // 8 warps per CTA, 4 row chunks per warp; the code width is a template parameter
+  const bool wide = width % 128 == 0;
+  const long long items = static_cast<long long>(rows) * (wide ? width / 128 : width / 64);
+  const dim3 grid(static_cast<unsigned>((items + 31) / 32));
+  if (wide)
+    return bits == 4 ? launch_k(false, k_quantize_rows<4, 4>, grid, dim3(256), 0, s, r, prev, rows, width, g, bits,
+                                codes, scales)
+                     : launch_k(false, k_quantize_rows<4, 2>, grid, dim3(256), 0, s, r, prev, rows, width, g, bits,
+                                codes, scales);
+  return bits == 4 ? launch_k(false, k_quantize_rows<2, 4>, grid, dim3(256), 0, s, r, prev, rows, width, g, bits,
+                              codes, scales)
+                   : launch_k(false, k_quantize_rows<2, 2>, grid, dim3(256), 0, s, r, prev, rows, width, g, bits,
+                              codes, scales);
 }
 cudaError_t launch_rmsnorm_rows(const float* h, const int* idx, int n, int n_pad, int d, const float* gain, float eps,
                                 uint16_t* x, cudaStream_t s) {
