@@ -63,9 +63,9 @@ struct GemmLaunch {
   const CUtensorMap* a1;   // second A operand (dual, swap: gate / up weights) or nullptr
   const CUtensorMap* b0;
   const CUtensorMap* b1;   // second B operand (dual, normal: gate / up weights) or nullptr
-  int bn;                  // 16, 32, 64 (swap) or 128 (normal)
+  int bn;                  // token columns of a swap tile: 16, 32 or 64; 128 tags the normal orientation
   int a_3d, b_3d;          // operand maps are layer-stacked (rank 3)
-  dim3 grid;
+  dim3 grid;               // swap orientation; the persistent normal-orientation kernel sizes its own
   GemmArgs args;
   bool pdl = false;        // launched as a programmatic dependent of the previous kernel
 };

@@ -430,8 +430,7 @@ fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, 
     g.a0 = xa; g.a1 = nullptr; g.b0 = w0; g.b1 = w1;
     g.a_3d = 0; g.b_3d = w3d;
     a.a_z = 0; a.b_z = j; a.swap = 0; a.splits = 1;
-    g.bn = 128;
-    g.grid = dim3(ceil_div(n, 128), ceil_div(feat, 128), 1);
+    g.bn = 128;   // the normal orientation (the persistent kernel sizes its own grid)
   }
   g.pdl = ctx->pdl;
   FL_TRY(launch_gemm(g, s));
@@ -1238,9 +1237,8 @@ fl_status fl_test_gemm(const uint16_t* A, const uint16_t* B, float* D, int m, in
     g.grid = dim3(tiles, 1, splits);
   } else {
     if (!encode_tmap_bf16(&ta, A, k, m, 0, 128) || !encode_tmap_bf16(&tb, B, k, n, 0, 128)) return FL_ERR_INVALID_ARG;
-    g.a0 = &ta; g.b0 = &tb; g.bn = 128;
+    g.a0 = &ta; g.b0 = &tb; g.bn = 128;   // the normal orientation (the persistent kernel sizes its own grid)
     a.swap = 0; a.splits = 1;
-    g.grid = dim3(ceil_div(m, 128), ceil_div(n, 128), 1);
   }
   return record(launch_gemm(g, s));
 }
