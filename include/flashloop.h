@@ -229,8 +229,9 @@ fl_status fl_test_quantize_residual(const float* x, const uint16_t* prev, int ro
 
 /* tcgen05 GEMM: D[m][n] = sum_k A[m][k] * B[n][k] (bf16 operands, fp32
  * accumulate); A [m][k] and B [n][k] row-major bf16, D fp32 [m][n]; k % 8 == 0,
- * all pointers 16-byte aligned.  swap_ab = 0: A's rows on the MMA M side
- * (128-row tiles), B in 128-row tiles.  swap_ab = 1: the skinny orientation
+ * all pointers 16-byte aligned.  swap_ab = 0: the persistent prefill kernel,
+ * A's rows on the MMA M side (128-row tiles) and B in 256-row tiles, one CTA
+ * per SM walking the output tiles.  swap_ab = 1: the skinny orientation
  * used for decode (B's rows on the MMA M side, m <= 64 rows of A as the MMA N
  * side), with the reduction split across CTAs; `scratch` must then hold
  * fl_test_gemm_scratch_bytes() bytes (caller-allocated device memory). */
