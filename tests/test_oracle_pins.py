@@ -430,6 +430,211 @@ def test_lazy_prefill_matches_materialised_brute_force(seed, T, qt, c):
     assert np.max(np.abs(res.h - bh)) <= 1e-9 * np.sqrt(np.mean(bh ** 2))
 
 
+def _brute_lazy_call(cfg, W, h0, seq, pos, tile, ctx, quant):
+    """A lazy call over N tokens of B sequences, each query's attention held as an
+    explicit score vector and value rows over its causal columns.
+
+    seq / pos / tile: per call token (flat index = position in the call, the
+    pooled ranking's tie-break).  ctx: None (empty sequences, prefill) or a
+    synthetic context (bf16 base bits, int8 codes, fp16 scales of loops 2..K)
+    whose rows before each sequence's length hold that sequence's history.
+    Every KV level of every column is kept materialised: level m of a context
+    column is its base plus the dequantised residuals of loops 2..m, added one at
+    a time in fp32; a call token's level m is its level m-1 plus the residual it
+    stored at loop m (zero when carried).  A recomputed query overwrites the
+    entries of its tile's column set with the new loop's scores and values; the
+    set is the top-c columns by max |new score - stored score| over the tile's
+    selected queries and the group's heads, chosen once per tile.  Written
+    without the running (O, lse) form and without the oracle's cache class.
+    Returns h, selections, column sets and the residual codes stored per
+    (layer, loop, token, K/V).
+    """
+    H, Hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
+    grp, tau, M, K = H // Hkv, 1 / math.sqrt(hd), cfg.n_layers, cfg.n_loops
+    N = len(seq)
+    B = int(max(seq)) + 1
+    tlen = [int(max(pos[i] for i in range(N) if seq[i] == b)) + 1 for b in range(B)]
+    # lev[j][b][m]: (K, V) of level m = 1..K, [Hkv, tlen_b, hd] float32
+    lev = [[[None] + [(np.zeros((Hkv, tlen[b], hd), F32), np.zeros((Hkv, tlen[b], hd), F32)) for _ in range(K)]
+            for b in range(B)] for _ in range(M)]
+    if ctx is not None:
+        f32 = lambda bits: (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(F32)
+        g = cfg.group_size
+        for j in range(M):
+            for b in range(B):
+                n = int(ctx["lens"][b])
+                kb, vb = f32(ctx["base_k"][j, b][:, :n]), f32(ctx["base_v"][j, b][:, :n])
+                lev[j][b][1][0][:, :n], lev[j][b][1][1][:, :n] = kb, vb
+                for m in range(2, K + 1):
+                    for w, nm in enumerate(("k", "v")):
+                        codes = ctx["codes_" + nm][j, m - 2, b][:, :n].astype(F32)
+                        sc = np.repeat(ctx["scales_" + nm][j, m - 2, b][:, :n].astype(F32), g, axis=-1)
+                        lev[j][b][m][w][:, :n] = (lev[j][b][m - 1][w][:, :n] + codes * sc).astype(F32)
+    h = np.asarray(h0, np.float64).copy()
+    scores = [[np.zeros((H, pos[i] + 1)) for i in range(N)] for _ in range(M)]
+    values = [[np.zeros((H, pos[i] + 1, hd)) for i in range(N)] for _ in range(M)]
+    stored = {}
+
+    def out_of(j, i):
+        s = scores[j][i]
+        w = np.exp(s - s.max(axis=1, keepdims=True))
+        w /= w.sum(axis=1, keepdims=True)
+        return np.einsum("ht,htd->hd", w, values[j][i])
+
+    def layer_tail(lw, hs, o):
+        hs = hs + cfg.resid_scale * (o.reshape(len(hs), H * hd) @ lw["w_o"].T)
+        return orc._mlp_update(cfg, lw, hs)
+
+    for j, lw in enumerate(W["layers"]):
+        q, k, v = orc._qkv(cfg, lw, h, pos)
+        for i in range(N):
+            b, p = seq[i], pos[i]
+            for m in range(1, K + 1):      # a new token's later levels start equal to its base
+                lev[j][b][m][0][:, p] = orc.bf16_round(k[i])
+                lev[j][b][m][1][:, p] = orc.bf16_round(v[i])
+        for i in range(N):
+            b, p = seq[i], pos[i]
+            for hh in range(H):
+                scores[j][i][hh] = tau * (lev[j][b][1][0][hh // grp, :p + 1].astype(np.float64) @ q[i, hh])
+                values[j][i][hh] = lev[j][b][1][1][hh // grp, :p + 1]
+        o = np.stack([out_of(j, i) for i in range(N)])
+        h = layer_tail(lw, h, o)
+    key = np.sum((h - h0) ** 2, axis=1).astype(F32)
+    n_sel = max(1, min(N, math.ceil(cfg.rho * N - 1e-9)))
+    sels, colset = {}, {}
+    for l in range(2, K + 1):
+        kbits = key.view(np.uint32)
+        S = np.array(sorted(sorted(range(N), key=lambda t: (-int(kbits[t]), t))[:n_sel]))
+        sels[l] = S
+        hprev = h[S].copy()
+        for j, lw in enumerate(W["layers"]):
+            q, k, v = orc._qkv(cfg, lw, h[S], pos[S])
+            for i in range(N):          # carried: level l = level l-1 (a zero residual)
+                b, p = seq[i], pos[i]
+                for w in (0, 1):
+                    lev[j][b][l][w][:, p] = lev[j][b][l - 1][w][:, p]
+            for a, i in enumerate(S):
+                b, p = seq[i], pos[i]
+                for w, new in ((0, k[a]), (1, v[a])):
+                    prev = lev[j][b][l - 1][w][:, p]
+                    r = (new.astype(F32) - prev).astype(F32)
+                    c, s = quant(r)
+                    stored[(j, l, int(i), w)] = (c, s)
+                    lev[j][b][l][w][:, p] = (prev + orc.dequant_groups(c, s, cfg.group_size)).astype(F32)
+            for tl in sorted(set(int(tile[i]) for i in S)):
+                if (j, tl) in colset:
+                    continue
+                mem = [a for a, i in enumerate(S) if tile[i] == tl]
+                b = seq[S[mem[0]]]
+                mp = max(pos[S[a]] for a in mem)
+                kn = lev[j][b][l][0].astype(np.float64)
+                for gk in range(Hkv):
+                    ck = np.full(mp + 1, -np.inf)
+                    for a in mem:
+                        i, p = S[a], pos[S[a]]
+                        for hh in range(gk * grp, (gk + 1) * grp):
+                            d = np.abs(tau * (kn[gk, :p + 1] @ q[a, hh]) - scores[j][i][hh])
+                            ck[:p + 1] = np.maximum(ck[:p + 1], d)
+                    ck = ck.astype(F32)
+                    if mp + 1 <= cfg.c_cols:
+                        colset[(j, tl, gk)] = np.arange(mp + 1)
+                    else:
+                        b2 = ck.view(np.uint32)
+                        colset[(j, tl, gk)] = np.array(sorted(sorted(range(mp + 1),
+                                                                     key=lambda c: (-int(b2[c]), c))[:cfg.c_cols]))
+                colset[(j, tl)] = True
+            for a, i in enumerate(S):
+                b, p = seq[i], pos[i]
+                for hh in range(H):
+                    C = colset[(j, int(tile[i]), hh // grp)]
+                    C = C[C <= p]
+                    scores[j][i][hh, C] = tau * (lev[j][b][l][0][hh // grp, C].astype(np.float64) @ q[a, hh])
+                    values[j][i][hh, C] = lev[j][b][l][1][hh // grp, C]
+            o = np.stack([out_of(j, i) for i in S])
+            h[S] = layer_tail(lw, h[S], o)
+        key = np.zeros(N, F32)
+        key[S] = np.sum((h[S] - hprev) ** 2, axis=1).astype(F32)
+    return h, sels, {k_: v_ for k_, v_ in colset.items() if len(k_) == 3}, stored
+
+
+def _compare_with_brute(cfg, res, cache, seq, pos, bh, bsel, bcols, bstored):
+    assert set(res.trace["sel"]) == set(bsel)
+    for l, S in bsel.items():
+        assert np.array_equal(res.trace["sel"][l], S), l
+    assert set(res.trace["cols"]) == set(bcols)
+    for key_, C in res.trace["cols"].items():
+        assert np.array_equal(C, bcols[key_]), key_
+    for (j, l, i, w), (c, s) in bstored.items():
+        nm = "k" if w == 0 else "v"
+        assert np.array_equal(getattr(cache, "codes_" + nm)[j, l - 2, seq[i], :, pos[i]], c)
+        assert np.array_equal(getattr(cache, "scales_" + nm)[j, l - 2, seq[i], :, pos[i]].view(np.uint16),
+                              np.asarray(s, np.float16).view(np.uint16))
+    assert np.max(np.abs(res.h - bh)) <= 1e-9 * np.sqrt(np.mean(bh ** 2))
+
+
+@pytest.mark.parametrize("seed,bits,lens,rho,c", [(61, 4, [9, 4, 13], 0.5, 3), (62, 2, [6, 11, 1, 8], 0.5, 4),
+                                                  (63, 4, [12, 12], 1.0, 5), (64, 2, [3, 15, 7], 0.3, 2)])
+def test_lazy_decode_over_residual_context_matches_materialised_brute_force(seed, bits, lens, rho, c):
+    """Decode over a context whose tokens already hold residual levels 2..K,
+    pooled over ragged sequences, rho < 1 and c below the context length."""
+    cfg = _tiny_cfg(seed=seed, rho=rho, c_cols=c, resid_bits=bits, mode="decode", batch=len(lens), seq_len=0,
+                    ctx_len=max(lens), n_loops=4)
+    W, rng = _weights(cfg)
+    ctx = synth.make_context(cfg, rng, lens)
+    tmax = max(lens) + 1
+    cache = orc.KVCache.from_context(cfg, ctx, tmax)
+    h0 = synth.make_h0(cfg, rng, len(lens))
+    res = orc.decode_step(cfg, W, cache, h0)
+    B = len(lens)
+    seq, pos = np.arange(B), np.asarray(lens)
+    quant = lambda r: orc.quantize_groups(r, cfg.resid_bits, cfg.group_size)
+    bh, bsel, bcols, bstored = _brute_lazy_call(cfg, W, h0, seq, pos, seq.copy(), ctx, quant)
+    assert len(bstored) == cfg.n_layers * (cfg.n_loops - 1) * 2 * orc.n_select(rho, B)
+    _compare_with_brute(cfg, res, cache, seq, pos, bh, bsel, bcols, bstored)
+
+
+def test_lazy_decode_pooled_ties_go_to_the_lower_sequence():
+    """Identical sequences (same context, same input row) give bit-identical
+    change keys, so the pooled ranking is decided by the tie-break alone: the
+    lower flat index (sequence) wins, in the oracle and in the brute force."""
+    B, n = 4, 9
+    cfg = _tiny_cfg(seed=65, rho=0.5, c_cols=3, resid_bits=4, mode="decode", batch=B, seq_len=0, ctx_len=n,
+                    n_loops=3)
+    W, rng = _weights(cfg)
+    ctx = synth.make_context(cfg, rng, [n] * B)
+    for name in ("base_k", "base_v"):
+        ctx[name][:, 1:] = ctx[name][:, :1]
+    for name in ("codes_k", "codes_v", "scales_k", "scales_v"):
+        ctx[name][:, :, 1:] = ctx[name][:, :, :1]
+    h0 = np.repeat(synth.make_h0(cfg, rng, 1), B, axis=0)
+    cache = orc.KVCache.from_context(cfg, ctx, n + 1)
+    res = orc.decode_step(cfg, W, cache, h0)
+    seq, pos = np.arange(B), np.full(B, n)
+    quant = lambda r: orc.quantize_groups(r, cfg.resid_bits, cfg.group_size)
+    bh, bsel, bcols, bstored = _brute_lazy_call(cfg, W, h0, seq, pos, seq.copy(), ctx, quant)
+    assert len(set(res.trace["keys"][2].tolist())) == 1           # every key ties
+    assert np.array_equal(bsel[2], [0, 1])
+    _compare_with_brute(cfg, res, cache, seq, pos, bh, bsel, bcols, bstored)
+
+
+@pytest.mark.parametrize("seed,B,T,qt,c,bits", [(71, 2, 10, 4, 2, 4), (72, 3, 7, 8, 3, 2)])
+def test_lazy_prefill_pooled_sequences_match_materialised_brute_force(seed, B, T, qt, c, bits):
+    """Prefill of several sequences: the ranking pools all B*T tokens by flat
+    index b*T + t and query tiles never span two sequences."""
+    cfg = _tiny_cfg(seed=seed, seq_len=T, batch=B, q_tile=qt, c_cols=c, rho=0.3, n_loops=4, resid_bits=bits)
+    W, rng = _weights(cfg)
+    h0 = synth.make_h0(cfg, rng, B * T)
+    cache = orc.KVCache(cfg, B, T)
+    res = orc.prefill(cfg, W, cache, h0, B, T)
+    seq, pos = np.repeat(np.arange(B), T), np.tile(np.arange(T), B)
+    tile = seq * ((T + qt - 1) // qt) + pos // qt
+    quant = lambda r: orc.quantize_groups(r, cfg.resid_bits, cfg.group_size)
+    bh, bsel, bcols, bstored = _brute_lazy_call(cfg, W, h0, seq, pos, tile, None, quant)
+    _compare_with_brute(cfg, res, cache, seq, pos, bh, bsel, bcols, bstored)
+    # the pooled selection really crosses sequences (some loop takes tokens of two sequences)
+    assert any(len(set(seq[S])) > 1 for S in bsel.values())
+
+
 # ----------------------------------------------------------------------------
 # invariants of the lazy path
 # ----------------------------------------------------------------------------
