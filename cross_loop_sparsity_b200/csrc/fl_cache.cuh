@@ -96,6 +96,38 @@ __device__ __forceinline__ void chain_lane(const CacheView& cv, int j, int kv, i
   }
 }
 
+// ---------------------------------------------------------------- residual quantiser
+// The hardware reciprocal approximation (PTX rcp.approx, within 1 ulp of 1/x).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// The group scale s = fp16_RU(RN(absmax / qmax)) (0 for an all-zero group) as fp16 bits.
+__device__ __forceinline__ uint16_t quant_scale(float absmax, int qm) {
+  return __half_as_ushort(__float2half_ru(qm == 1 ? absmax : __fdiv_rn(absmax, static_cast<float>(qm))));
+}
+
+// code = clamp(rint(RN(r / s)), -qm, qm), ties to even, for the group scale s
+// (inv = rcp_approx(s), or 0 when s = 0).  Since s >= absmax / qmax up to one
+// fp32 rounding, |r / s| < 7.01; q = r * inv then lies within 7.01 * 1.5 * 2^-23
+// of r / s, and so within 1.6 * 2^-20 of the correctly rounded quotient Q.  When
+// q is farther than 2^-18 from every half-integer, q and Q round to the same
+// integer; otherwise Q itself is computed.  Rounding to an integer: q + 1.5 * 2^23
+// lies in [2^23, 2^24), where the fp32 spacing is 1, so the addition rounds q to
+// the nearest integer (ties to even) and leaves it, offset by 2^22, in the low
+// bits of the sum.  (With s = 0, q = 0 and the exact branch is never taken.)
+__device__ __forceinline__ int quant_code(float r, float s, float inv, int qm) {
+  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
+  const float q = r * inv;
+  float t = __fadd_rn(q, kMagic);
+  const float d = __fsub_rn(q, __fsub_rn(t, kMagic));   // q - rint(q), exact
+  if (fabsf(d) >= 0.5f - 0x1p-18f) t = __fadd_rn(__fdiv_rn(r, s), kMagic);
+  const int c = __float_as_int(t) - 0x4B400000;
+  return c > qm ? qm : (c < -qm ? -qm : c);
+}
+
 // Largest loop count K a context supports; kernels that reconstruct the chain
 // are instantiated for KM in {2, 4, 8, 16}, the smallest power of two >= K, so
 // the unrolled reconstruction issues no work for loops that cannot exist.

@@ -6,7 +6,38 @@
 #include <cstdint>
 #include <string>
 
+#include "fl_cache.cuh"
+
 namespace fl {
+
+// RoPE and the KV write of freshly projected rows: the separate kernel
+// (k_qkv_post) takes these, and so does the QKV GEMM when it does the same work
+// in its epilogue.
+struct QkvPostArgs {
+  const float* qkv;   // [n][(H+2Hkv)*hd] fp32, GEMM row order
+  int ldq;
+  const int* idx;     // GEMM row -> call token (nullptr = identity)
+  int n;
+  const int* seq;     // call token -> sequence
+  const int* pos;     // call token -> position
+  int H, Hkv, hd;
+  const float* rope_cos;  // [max_ctx][hd/2]
+  const float* rope_sin;
+  CacheView cv;
+  int j, loop, lazy;
+  float* q_cur;       // [n][H][hd] GEMM order
+  float* q_last;      // [N][H][hd] token order (this layer), written at loop 1
+  const int* forced_on;           // forced residual codes (checks): [0] != 0 when on
+  const int8_t* forced_codes;     // [M][K-1][ns][2][Hkv][hd]
+  const uint16_t* forced_scales;  // [M][K-1][ns][2][Hkv][hd/g]
+  int forced_ns;                  // selection-slot stride ns
+  // checks only: the rotated fp32 K/V rows each lazy loop quantised,
+  // [M][K-1][trace_ns][2][Hkv][hd] by (layer, loop 2..K, selection slot, K/V,
+  // KV head); slots >= trace_ns are not written (nullptr: off)
+  float* trace_kv;
+  int trace_ns;
+};
+
 
 // ------------------------------------------------------------------ GEMM
 // D = A * B^T on tcgen05 (bf16 operands, fp32 accumulate in TMEM).  A and B
@@ -50,6 +81,12 @@ struct GemmArgs {
   // memory from fp32 hidden rows instead of loaded by TMA:
   //   x[t][k] = bf16(h[r_t][k] * rsqrt(sum_p ss_in[p * ss_ld + t] / K + in_eps) * in_gain[k])
   // with r_t = in_idx ? in_idx[t] : t, p < ss_parts, and zero rows t >= n_tok.
+  // RoPE and the KV write in the epilogue (swap orientation, cluster split-K
+  // path, hd dividing 128): instead of storing fp32 rows, the epilogue rotates
+  // q and k, writes q (and q_last at loop 1 of the lazy path) and stores or
+  // quantises the K/V rows exactly as k_qkv_post does.
+  int post_on;
+  QkvPostArgs post;
   const float* in_h;   // nullptr: TMA operand
   const int* in_idx;
   const float* in_gain;
@@ -71,6 +108,19 @@ struct GemmLaunch {
 };
 
 constexpr int kMaxClusterSplits = 16;  // non-portable cluster size, opted in per kernel
+constexpr int kNumSM = 148;            // B200 streaming multiprocessors
+
+// Token columns of a skinny (swap-orientation) tile for n <= 64 tokens.
+inline int swap_bn(int n) { return n <= 16 ? 16 : n <= 32 ? 32 : 64; }
+
+// Split-K factor of a skinny GEMM with `tiles` 128-row feature tiles and
+// k_chunks 64-wide k-chunks: about one CTA per SM, at most one split per chunk.
+inline int split_factor(int tiles, int k_chunks) {
+  if (tiles >= kNumSM) return 1;
+  int s = kNumSM / tiles;
+  if (s > k_chunks) s = k_chunks;
+  return s < 1 ? 1 : s;
+}
 cudaError_t launch_gemm(const GemmLaunch& g, cudaStream_t stream);
 
 // Launch a kernel, with programmatic stream serialisation when `pdl` is set

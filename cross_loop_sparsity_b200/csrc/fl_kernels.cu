@@ -308,14 +308,6 @@ __global__ void __launch_bounds__(256) k_rmsnorm_rows(const float* __restrict__ 
 // code = clamp(rint(fp32(r / s)), -qmax, qmax), ties to even.
 // Returns the lane's codes and the group's fp16 scale bits.
 // ============================================================================
-// The hardware reciprocal approximation (PTX rcp.approx, within 1 ulp of 1/x).
-__device__ __forceinline__ float rcp_approx(float x) {
-  float y;
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// BITS = 4 or 2 fixes the code width at compile time; 0 takes it from `bits`.
 template <int EPL, int BITS = 0>
 __device__ __forceinline__ uint16_t quantize_lane(const float* r, int lg, int bits_rt, int* code) {
   const int bits = BITS ? BITS : bits_rt;
@@ -325,28 +317,12 @@ __device__ __forceinline__ uint16_t quantize_lane(const float* r, int lg, int bi
   for (int e = 0; e < EPL; ++e) am = fmaxf(am, fabsf(r[e]));
   for (int o = GL >> 1; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
   const int qm = (1 << (bits - 1)) - 1;
-  const __half sh = __float2half_ru(qm == 1 ? am : __fdiv_rn(am, static_cast<float>(qm)));
-  const float s = __half2float(sh);
-  // code = rint of the correctly rounded quotient Q = RN(r/s).  Since s >=
-  // absmax/qmax up to one fp32 rounding, |r/s| < 7.01.  q = r * rcp_approx(s)
-  // then lies within 7.01 * 1.5 * 2^-23 of r/s, and so within 1.6 * 2^-20 of Q.
-  // When q is farther than 2^-18 from every half-integer, q and Q round to the
-  // same integer; otherwise Q itself is computed.  Rounding to an integer: the
-  // sum q + 1.5 * 2^23 lies in [2^23, 2^24), where the fp32 spacing is 1, so the
-  // addition rounds q to the nearest integer (ties to even) and leaves it, offset
-  // by 2^22, in the low bits of the sum.
+  const uint16_t sh = quant_scale(am, qm);
+  const float s = half_bits_to_f(sh);
   const float inv = s > 0.f ? rcp_approx(s) : 0.f;
-  constexpr float kMagic = 12582912.0f;   // 1.5 * 2^23
 #pragma unroll
-  for (int e = 0; e < EPL; ++e) {
-    const float q = r[e] * inv;
-    float t = __fadd_rn(q, kMagic);
-    const float d = __fsub_rn(q, __fsub_rn(t, kMagic));   // q - rint(q), exact
-    if (fabsf(d) >= 0.5f - 0x1p-18f) t = __fadd_rn(__fdiv_rn(r[e], s), kMagic);   // (s > 0 here: else q = 0)
-    const int c = __float_as_int(t) - 0x4B400000;
-    code[e] = c > qm ? qm : (c < -qm ? -qm : c);
-  }
-  return __half_as_ushort(sh);
+  for (int e = 0; e < EPL; ++e) code[e] = quant_code(r[e], s, inv, qm);
+  return sh;
 }
 
 // Pack the lane's codes (two's complement, element order low bits first) and
@@ -466,7 +442,8 @@ __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
     const float* cs = a.rope_cos + static_cast<size_t>(t) * half + ai;
     const float* sn = a.rope_sin + static_cast<size_t>(t) * half + ai;
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) x[e] = lane < 16 ? x[e] * cs[e] - y[e] * sn[e] : x[e] * cs[e] + y[e] * sn[e];
+    for (int e = 0; e < EPL; ++e)   // explicit roundings: the GEMM epilogue's rotation matches bit for bit
+      x[e] = lane < 16 ? __fmaf_rn(x[e], cs[e], -__fmul_rn(y[e], sn[e])) : __fmaf_rn(x[e], cs[e], __fmul_rn(y[e], sn[e]));
   }
   if (hh < a.H) {
     float* dq = a.q_cur + (static_cast<size_t>(i) * a.H + hh) * hd + lane * EPL;
@@ -513,6 +490,12 @@ __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
     for (int e = 0; e < EPL; ++e) c[e] = a.forced_codes[row * hd + lane * EPL + e];
     s = a.forced_scales[row * (hd >> cv.lg) + ((lane * EPL) >> cv.lg)];
   } else {
+    if (a.trace_kv && i < a.trace_ns) {
+      float* tr = a.trace_kv + ((((static_cast<size_t>(a.j) * (cv.K - 1) + (a.loop - 2)) * a.trace_ns + i) * 2 + kv) *
+                                    a.Hkv + gk) * hd + lane * EPL;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) tr[e] = x[e];
+    }
     float prev[EPL];
     chain_lane<EPL>(cv, a.j, kv, b, gk, t, a.loop - 1, lane, prev);
     float r[EPL];
@@ -828,51 +811,71 @@ __global__ void __launch_bounds__(128, 2) k_attn_decode(const __grid_constant__ 
     ml[e * 2 + 1] = v.y;
   }
   __syncthreads();
-  if (tid < GRP) {
+  // warp w takes heads w, w + 4: its lanes stride over the splits
+  for (int h = warp; h < GRP; h += 4) {
     float M = -INFINITY;
-    for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, ml[(s2 * GRP + tid) * 2]);
+    for (int s2 = lane; s2 < S; s2 += 32) M = fmaxf(M, ml[(s2 * GRP + h) * 2]);
+    M = warp_max(M);
     float L = 0.f;
-    for (int s2 = 0; s2 < S; ++s2) {
-      const float ms = ml[(s2 * GRP + tid) * 2];
+    for (int s2 = lane; s2 < S; s2 += 32) {
+      const float ms = ml[(s2 * GRP + h) * 2];
       const float w = ms == -INFINITY ? 0.f : expf(ms - M);
-      ml[(s2 * GRP + tid) * 2] = w;   // the split's weight replaces its maximum
-      L += w * ml[(s2 * GRP + tid) * 2 + 1];
+      ml[(s2 * GRP + h) * 2] = w;   // the split's weight replaces its maximum
+      L += w * ml[(s2 * GRP + h) * 2 + 1];
     }
-    sm_m[tid] = M;
-    sm_l[tid] = L;
+    L = warp_sum(L);
+    if (lane == 0) {
+      sm_m[h] = M;
+      sm_l[h] = L;
+    }
   }
   __syncthreads();
-  constexpr int EPT = (GRP * HD + 127) / 128;           // output elements per thread
-  constexpr int MB = 64 / EPT < 16 ? 64 / EPT : 16;      // splits whose outputs are requested together
-  float o[EPT];
+  // each thread folds four consecutive output elements (one head), the
+  // splits' partial rows read as 16-byte vectors, MB splits requested together
+  constexpr int E4 = (GRP * HD / 4 + 127) / 128;        // 4-element groups per thread
+  constexpr int MB = 16 / E4 < 16 ? (16 / E4 > 0 ? 16 / E4 : 1) : 16;
+  float4 o[E4];
 #pragma unroll
-  for (int t = 0; t < EPT; ++t) o[t] = 0.f;
+  for (int t = 0; t < E4; ++t) o[t] = make_float4(0.f, 0.f, 0.f, 0.f);
   for (int s0 = 0; s0 < S; s0 += MB) {
-    float pv[EPT][MB];
+    float4 pv[E4][MB];
 #pragma unroll
-    for (int t = 0; t < EPT; ++t) {
-      const int e = tid + t * 128, h = e / HD, d = e % HD;
+    for (int t = 0; t < E4; ++t) {
+      const int e = (tid + t * 128) * 4, h = e / HD, d = e % HD;
 #pragma unroll
       for (int u = 0; u < MB; ++u)
-        pv[t][u] = (e < GRP * HD && s0 + u < S) ? __ldcg(&a.part_o[((q0 + s0 + u) * 8 + h) * HD + d]) : 0.f;
+        pv[t][u] = (e < GRP * HD && s0 + u < S)
+                       ? __ldcg(reinterpret_cast<const float4*>(&a.part_o[((q0 + s0 + u) * 8 + h) * HD + d]))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 #pragma unroll
-    for (int t = 0; t < EPT; ++t) {
-      const int e = tid + t * 128, h = e < GRP * HD ? e / HD : 0;
+    for (int t = 0; t < E4; ++t) {
+      const int e = (tid + t * 128) * 4, h = e < GRP * HD ? e / HD : 0;
 #pragma unroll
       for (int u = 0; u < MB; ++u)
-        if (s0 + u < S) o[t] += ml[((s0 + u) * GRP + h) * 2] * pv[t][u];
+        if (s0 + u < S) {
+          const float w = ml[((s0 + u) * GRP + h) * 2];
+          o[t].x += w * pv[t][u].x;
+          o[t].y += w * pv[t][u].y;
+          o[t].z += w * pv[t][u].z;
+          o[t].w += w * pv[t][u].w;
+        }
     }
   }
 #pragma unroll
-  for (int t = 0; t < EPT; ++t) {
-    const int e = tid + t * 128;
+  for (int t = 0; t < E4; ++t) {
+    const int e = (tid + t * 128) * 4;
     if (e >= GRP * HD) break;
     const int h = e / HD, d = e % HD;
     const int hq = g * GRP + h;
-    const float ov = o[t] / sm_l[h];
-    if (a.o_state) a.o_state[(static_cast<size_t>(tok) * a.H + hq) * HD + d] = ov;
-    a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + d] = f_to_bf16(ov);
+    const float L = sm_l[h];
+    const float ov[4] = {o[t].x / L, o[t].y / L, o[t].z / L, o[t].w / L};
+    if (a.o_state)
+      *reinterpret_cast<float4*>(&a.o_state[(static_cast<size_t>(tok) * a.H + hq) * HD + d]) =
+          make_float4(ov[0], ov[1], ov[2], ov[3]);
+    uint16_t* ob = a.o_bf16 + static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + d;
+    *reinterpret_cast<uint2*>(ob) = make_uint2(f_to_bf16(ov[0]) | (static_cast<uint32_t>(f_to_bf16(ov[1])) << 16),
+                                               f_to_bf16(ov[2]) | (static_cast<uint32_t>(f_to_bf16(ov[3])) << 16));
     if (d == 0 && a.lse_state) a.lse_state[static_cast<size_t>(tok) * a.H + hq] = sm_m[h] + logf(sm_l[h]);
   }
   if (tid == 0) a.counters[i * a.Hkv + g] = 0;
@@ -1388,6 +1391,9 @@ __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
   if (tid < nc) {
     const float v = fmaxf(fmaxf(Mx[tid], Mx[CC + tid]), fmaxf(Mx[2 * CC + tid], Mx[3 * CC + tid]));
     a.col_keys[(static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols + c0 + tid] = v;
+    const int tl = a.plan.tile[p];
+    if (a.trace_ck && tl < a.trace_tiles)
+      a.trace_ck[((static_cast<size_t>(a.j) * a.trace_tiles + tl) * a.Hkv + g) * a.max_cols + c0 + tid] = v;
   }
 }
 

@@ -9,25 +9,6 @@
 
 namespace fl {
 
-struct QkvPostArgs {
-  const float* qkv;   // [n][(H+2Hkv)*hd] fp32, GEMM row order
-  int ldq;
-  const int* idx;     // GEMM row -> call token (nullptr = identity)
-  int n;
-  const int* seq;     // call token -> sequence
-  const int* pos;     // call token -> position
-  int H, Hkv, hd;
-  const float* rope_cos;  // [max_ctx][hd/2]
-  const float* rope_sin;
-  CacheView cv;
-  int j, loop, lazy;
-  float* q_cur;       // [n][H][hd] GEMM order
-  float* q_last;      // [N][H][hd] token order (this layer), written at loop 1
-  const int* forced_on;           // forced residual codes (checks): [0] != 0 when on
-  const int8_t* forced_codes;     // [M][K-1][ns][2][Hkv][hd]
-  const uint16_t* forced_scales;  // [M][K-1][ns][2][Hkv][hd/g]
-  int forced_ns;                  // selection-slot stride ns
-};
 
 struct AttnDecArgs {
   const float* q_cur;
@@ -115,6 +96,10 @@ struct DScoreArgs {
   float tau;
   float* col_keys;      // [max_need][Hkv][max_cols]
   int max_cols;
+  // checks only: every tile's keys by query tile, [M][trace_tiles][Hkv][max_cols]
+  // (tiles >= trace_tiles are not written; nullptr: off)
+  float* trace_ck;
+  int trace_tiles;
 };
 
 struct SelColsArgs {

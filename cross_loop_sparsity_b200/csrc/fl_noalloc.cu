@@ -62,12 +62,11 @@ fl_status fl_gemm_skinny_noalloc(const uint16_t* A, const uint16_t* B, float* D,
     return fail(FL_ERR_INVALID_ARG, "A, B, D must be non-NULL; 1 <= m <= 64; k >= 8 and a multiple of 8");
   if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(B) | reinterpret_cast<uintptr_t>(D)) & 15)
     return fail(FL_ERR_INVALID_ARG, "A, B and D must be 16-byte aligned");
-  const int bn = m <= 16 ? 16 : m <= 32 ? 32 : 64;
+  // the same tile width and split rule as fl_test_gemm, so both give the same product bit for bit
+  const int bn = fl::swap_bn(m);
   const int tiles = ceil_div(n, 128);
   const int k_chunks = ceil_div(k, 64);
-  int splits = tiles >= 148 ? 1 : 148 / tiles;
-  if (splits > k_chunks) splits = k_chunks;
-  if (splits < 1) splits = 1;
+  const int splits = fl::split_factor(tiles, k_chunks);
   const size_t need = fl::gemm_partial_floats(bn, 0, tiles, splits) * sizeof(float);
   if (need > kPartialBytes || static_cast<size_t>(tiles) * sizeof(int) > kTicketBytes)
     return fail(FL_ERR_CAPACITY, "this shape needs " + std::to_string(need) + " bytes of split-K scratch; the "

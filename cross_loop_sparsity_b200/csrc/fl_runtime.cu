@@ -84,17 +84,22 @@ struct flashloop_ctx {
   int use_graph = 1;
   int pdl = 1;                        // FL_OPT_PDL
   int prof = 0;                       // FL_OPT_PROFILE
+  int fuse_qkv = 0;                   // FL_OPT_FUSE_QKV
   std::vector<cudaEvent_t> ev;        // start/end pairs of the last profiled call
   std::vector<int> ev_kind;
   int ev_used = 0;
   int launches = 0;                   // kernels enqueued by the last call
   std::string last_err;
   int last_N = 0, last_nsel = 0, last_decode = 0, last_tiles = 0;
+  // check buffers (caller device memory; nullptr: off)
+  float* trace_kv = nullptr;
+  int trace_ns = 0;
+  float* trace_ck = nullptr;
+  int trace_tiles = 0;
 };
 
 namespace {
 
-constexpr int kNumSM = 148;
 // Sparse-column correction: columns per CTA.  Few selected queries (decode)
 // get narrow splits for parallelism; many (prefill) get wide ones.
 constexpr int kCorrColsSmall = 16, kCorrColsBig = 128, kCorrSmallQueries = 64;
@@ -137,15 +142,6 @@ bool valid_config(const flashloop_config* c) {
   return true;
 }
 
-int swap_bn(int n) { return n <= 16 ? 16 : n <= 32 ? 32 : 64; }
-
-// split-K factor of a skinny GEMM with `tiles` 128-row feature tiles
-int split_factor(int tiles, int k_chunks) {
-  if (tiles >= kNumSM) return 1;
-  int s = kNumSM / tiles;
-  if (s > k_chunks) s = k_chunks;
-  return s < 1 ? 1 : s;
-}
 
 // Walk the workspace regions; assign pointers when ctx is given.  Returns the byte total.
 size_t layout(const flashloop_config& c, flashloop_ctx* x) {
@@ -367,11 +363,13 @@ struct InNorm {
 // down projections): whether the epilogue left the sums of squares of its
 // updated rows for the next norm (the cluster split-K path only).
 fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, cudaStream_t s,
-               const InNorm& in = InNorm{}, bool* ss_written = nullptr) {
+               const InNorm& in = InNorm{}, bool* ss_written = nullptr, const QkvPostArgs* post = nullptr,
+               bool* post_done = nullptr) {
   const flashloop_config& c = ctx->cfg;
   GemmLaunch g{};
   GemmArgs& a = g.args;
   if (ss_written) *ss_written = false;
+  if (post_done) *post_done = false;
   const CUtensorMap *w0 = nullptr, *w1 = nullptr, *xa = nullptr;
   const CUtensorMap* xb = nullptr;
   int feat = 0, K = 0;
@@ -424,6 +422,12 @@ fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, 
     if (in.gain) {
       a.in_h = ctx->h; a.in_idx = in.idx; a.in_gain = in.gain; a.ss_in = ctx->ss_part; a.ss_ld = kSsLd;
       a.in_ld = K; a.ss_parts = ceil_div(K, 128); a.in_eps = c.rms_eps;
+    }
+    // RoPE and the KV write in the epilogue of the cluster split-K path
+    if (post && post_done && ctx->fuse_qkv && splits > 1 && 128 % c.head_dim == 0) {
+      a.post_on = 1;
+      a.post = *post;
+      *post_done = true;
     }
   } else {
     if (in.gain) return FL_ERR_UNSUPPORTED;   // the caller builds the input with the norm kernel instead
@@ -587,14 +591,16 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
         attn_in.gain = ctx->w.attn_norm + static_cast<size_t>(j) * d;
         attn_in.idx = idx;
       }
-      FL_GEMM(gemm(ctx, kOpQKV, j, n, idx, s, attn_in));
       QkvPostArgs qa{};
       qa.qkv = ctx->qkv; qa.ldq = ctx->qkv_rows; qa.idx = idx; qa.n = n; qa.seq = ctx->seq; qa.pos = ctx->pos;
       qa.H = H; qa.Hkv = Hkv; qa.hd = hd; qa.rope_cos = ctx->rope_cos; qa.rope_sin = ctx->rope_sin;
       qa.cv = ctx->cv; qa.j = j; qa.loop = l; qa.lazy = lazy ? 1 : 0; qa.q_cur = ctx->q_cur; qa.q_last = ql;
       qa.forced_on = ctx->forced_codes_on; qa.forced_codes = ctx->forced_codes;
       qa.forced_scales = ctx->forced_scales; qa.forced_ns = ctx->nsel_max;
-      FL_LAUNCH(FL_KIND_KV, launch_qkv_post(qa, s));
+      qa.trace_kv = ctx->trace_kv; qa.trace_ns = ctx->trace_ns;
+      bool post_done = false;
+      FL_GEMM(gemm(ctx, kOpQKV, j, n, idx, s, attn_in, nullptr, &qa, &post_done));
+      if (!post_done) FL_LAUNCH(FL_KIND_KV, launch_qkv_post(qa, s));
       if (full) {
         if (decode) {
           AttnDecArgs aa{};
@@ -628,6 +634,7 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
         da.q_cur = ctx->q_cur;
         da.q_last = ql; da.cv = ctx->cv; da.j = j; da.loop = l; da.H = H; da.Hkv = Hkv; da.hd = hd; da.tau = tau;
         da.col_keys = ctx->col_keys; da.max_cols = c.max_ctx;
+        da.trace_ck = ctx->trace_ck; da.trace_tiles = ctx->trace_tiles;
         FL_LAUNCH(FL_KIND_DSCORE, launch_dscore(da, max_need, max_chunks, s));
         SelColsArgs sa{};
         sa.plan = ctx->plan; sa.idx = idx; sa.pos = ctx->pos; sa.meta = ctx->sel_meta; sa.col_keys = ctx->col_keys;
@@ -824,6 +831,10 @@ fl_status flashloop_set_option(flashloop_ctx* ctx, fl_option opt, int value) {
     ctx->pdl = value ? 1 : 0;
     return FL_OK;
   }
+  if (opt == FL_OPT_FUSE_QKV) {
+    ctx->fuse_qkv = value ? 1 : 0;
+    return FL_OK;
+  }
   return FL_ERR_INVALID_ARG;
 }
 
@@ -860,7 +871,7 @@ fl_status flashloop_decode_step(flashloop_ctx* ctx, const float* h0, int B, floa
   FL_TRY(cudaMemcpyAsync(ctx->h_in, h0, static_cast<size_t>(B) * c.d_model * 4, cudaMemcpyDefault, s));
   // A decode step's launch sequence depends on B only; after one direct run it
   // is captured once into a CUDA graph and replayed (not on the legacy stream).
-  const int gkey = B * 4 + (ctx->prof ? 1 : 0) + (ctx->pdl ? 2 : 0);
+  const int gkey = B * 8 + (ctx->prof ? 1 : 0) + (ctx->pdl ? 2 : 0) + (ctx->fuse_qkv ? 4 : 0);
   size_t gi = 0;
   while (gi < ctx->graph_b.size() && ctx->graph_b[gi] != gkey) ++gi;
   bool seen = false;
@@ -1114,6 +1125,22 @@ fl_status flashloop_force_codes(flashloop_ctx* ctx, const int8_t* codes, const u
     }
   }
   FL_TRY(cudaMemcpy(ctx->forced_codes_on, &on, 4, cudaMemcpyHostToDevice));
+  return FL_OK;
+}
+
+fl_status flashloop_set_trace(flashloop_ctx* ctx, float* kv_rows, int n_slots, float* col_keys, int n_tiles) {
+  if (!ctx || !ctx->lazy) return FL_ERR_INVALID_ARG;
+  if ((kv_rows && n_slots < 1) || (col_keys && n_tiles < 1)) return FL_ERR_INVALID_ARG;
+  if ((kv_rows && !aligned16(kv_rows)) || (col_keys && !aligned16(col_keys))) return FL_ERR_INVALID_ARG;
+  ctx->trace_kv = kv_rows;
+  ctx->trace_ns = kv_rows ? n_slots : 0;
+  ctx->trace_ck = col_keys;
+  ctx->trace_tiles = col_keys ? n_tiles : 0;
+  // captured decode graphs hold the old pointers: capture again
+  for (cudaGraphExec_t e : ctx->graph_exec)
+    if (e) cudaGraphExecDestroy(e);
+  ctx->graph_exec.clear();
+  ctx->graph_b.clear();
   return FL_OK;
 }
 

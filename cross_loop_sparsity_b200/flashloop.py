@@ -18,6 +18,8 @@ LIB_PATH = os.path.join(_HERE, "libflashloop.so")
 FL_OK = 0
 FL_OPT_USE_GRAPH = 1
 FL_OPT_PROFILE = 2
+FL_OPT_PDL = 3
+FL_OPT_FUSE_QKV = 4
 KINDS = ["gemm", "attn", "dscore", "correct", "kv", "select", "norm", "other"]
 STATUS = {0: "ok", 1: "invalid argument", 2: "capacity exceeded", 3: "workspace", 4: "cuda error",
           5: "timeout", 6: "nonfinite", 7: "unsupported"}
@@ -66,6 +68,7 @@ _SIG = {
     "flashloop_export_slice": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "flashloop_force_selection": (_I, [_P, _P, _I, _I, _P, _P, _I]),
     "flashloop_read_trace": (_I, [_P, _P, _P, _P, _P, _P]),
+    "flashloop_set_trace": (_I, [_P, _P, _I, _P, _I]),
     "flashloop_force_codes": (_I, [_P, _P, _P, _I]),
     "flashloop_set_option": (_I, [_P, _I, _I]),
     "flashloop_profile": (_I, [_P, _P, _P, _P]),
@@ -267,6 +270,20 @@ class FlashLoop:
         self.reset([int(x) for x in lens])
         torch.cuda.synchronize()
 
+    def load_context_device(self, lens, seed=None, dense: bool = False):
+        """Import a synthetic context drawn on the device (``synth.context_slices_device``)
+        slice by slice, then set the lengths."""
+        import torch
+        from cross_loop_sparsity_b200 import synth
+        for sl in synth.context_slices_device(self.cfg, lens, seed=seed, dense=dense):
+            if dense:
+                self.import_dense(*sl)
+            else:
+                self.import_lazy(*sl)
+            torch.cuda.synchronize()    # the import copies read the drawn tensors
+        self.reset([int(x) for x in lens])
+        torch.cuda.synchronize()
+
     def export_slice(self, layer, loop, seq, which, n, stream=None):
         """Returns (codes, scales) numpy arrays; loop 1 (or dense) returns (bf16 bits [Hkv][n][hd], None)."""
         import torch
@@ -316,6 +333,15 @@ class FlashLoop:
         _check(lib().flashloop_force_codes(self.ctx, codes.ctypes.data_as(ctypes.c_void_p),
                                            scales.ctypes.data_as(ctypes.c_void_p), codes.shape[2]),
                "force_codes", self.ctx)
+
+    def set_trace(self, kv_rows=None, n_slots: int = 0, col_keys=None, n_tiles: int = 0):
+        """Check buffers (cuda float32 tensors, or None): kv_rows [M][K-1][n_slots][2][Hkv][hd]
+        receives the new K/V rows each lazy loop quantised; col_keys [M][n_tiles][Hkv][max_ctx]
+        the delta-score keys of every column set the call chose."""
+        self._trace_keep = (kv_rows, col_keys)
+        _check(lib().flashloop_set_trace(self.ctx, None if kv_rows is None else _ptr(kv_rows), n_slots,
+                                         None if col_keys is None else _ptr(col_keys), n_tiles),
+               "set_trace", self.ctx)
 
     def read_trace(self, N: int, n_sel: int, n_tiles: int, stream=None):
         c = self.c

@@ -44,7 +44,7 @@ typedef enum {
   FL_ERR_WORKSPACE = 3,   /* workspace smaller than flashloop_workspace_bytes() or misaligned */
   FL_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (see flashloop_last_cuda_error) */
   FL_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out; the kernel returned early */
-  FL_ERR_NONFINITE = 6,   /* reserved: non-finite value detected by a checking build */
+  FL_ERR_NONFINITE = 6,   /* a corrected softmax denominator was not positive (non-finite result) */
   FL_ERR_UNSUPPORTED = 7  /* a configuration this build does not implement */
 } fl_status;
 
@@ -194,6 +194,22 @@ fl_status flashloop_force_selection(flashloop_ctx* ctx, const int32_t* sel, int 
  * bit-exactly on identical inputs (fl_test_quantize). */
 fl_status flashloop_force_codes(flashloop_ctx* ctx, const int8_t* codes, const uint16_t* scales, int n_sel);
 
+/* Check buffers written by the following calls (device pointers, caller-owned;
+ * NULL turns each off).  kv_rows: fp32 [M][K-1][n_slots][2][Hkv][hd], the
+ * rotated new K (0) and V (1) rows that a lazy loop l >= 2 quantised, by (layer,
+ * loop, selection slot, K/V, KV head) -- the inputs of the KV-residual quantiser
+ * ("FlashLoop ...", abstract: KV residuals between adjacent loops in low-bit
+ * form); rows are written only where the library quantised them itself (not
+ * under flashloop_force_codes) and only for slots < n_slots.  col_keys: fp32
+ * [M][n_tiles][Hkv][max_ctx], the delta-score key of every eligible column of
+ * each query tile whose column set the call chose ("FlashLoop ...", abstract:
+ * the sparse, stable subset of key columns), by global query tile (decode: the
+ * sequence; prefill: b * ceil(T / q_tile) + t / q_tile); tiles >= n_tiles are not
+ * written.  Pointers must be 16-byte aligned.  Captured decode graphs are
+ * dropped and captured again.  FL_ERR_INVALID_ARG for a dense context, a
+ * non-positive capacity or a misaligned pointer. */
+fl_status flashloop_set_trace(flashloop_ctx* ctx, float* kv_rows, int n_slots, float* col_keys, int n_tiles);
+
 /* Read back the last call's choices (host buffers): sel [K-1][n_sel]; keys
  * [K-1][N] fp32 selection keys of loops 2..K; cols/ncols as above.  Any may be
  * NULL.  Synchronises `stream`. */
@@ -260,7 +276,10 @@ fl_status fl_test_gemm(const uint16_t* A, const uint16_t* B, float* D, int m, in
  *    fl_test_gemm with caller scratch for those.
  *  - Every call shares the one array and leaves its contents behind; the
  *    tickets are cleared on the call's stream before each launch.  Calls that
- *    overlap on the GPU (other streams, other host threads) race on it. */
+ *    overlap on the GPU (other streams, other host threads) race on it.
+ *  - There is no context to report a kernel's failure through: if a bounded
+ *    wait inside the kernel runs out, the affected output tile is written as
+ *    NaN, never as a silently wrong product. */
 #define FL_NOALLOC_SCRATCH_BYTES (2u << 20)
 fl_status fl_gemm_skinny_noalloc(const uint16_t* A, const uint16_t* B, float* D, int m, int n, int k,
                                  fl_stream_t stream);
@@ -269,8 +288,11 @@ fl_status fl_gemm_skinny_noalloc(const uint16_t* A, const uint16_t* B, float* D,
 typedef enum {
   FL_OPT_USE_GRAPH = 1, /* 1 (default): capture decode steps into CUDA graphs; 0: launch directly */
   FL_OPT_PROFILE = 2,   /* 1: bracket every kernel of a call with CUDA events (read with flashloop_profile) */
-  FL_OPT_PDL = 3        /* 1 (default): launch each kernel of a call as a programmatic dependent of the
+  FL_OPT_PDL = 3,       /* 1 (default): launch each kernel of a call as a programmatic dependent of the
                            previous one, so its launch and set-up overlap the predecessor */
+  FL_OPT_FUSE_QKV = 4   /* 0 (default): RoPE and the KV write run in their own kernel; 1: in the QKV GEMM's
+                           epilogue wherever the decode GEMM is split over a cluster (bit-identical results;
+                           measured slower on the decode workload, so off) */
 } fl_option;
 fl_status flashloop_set_option(flashloop_ctx* ctx, fl_option opt, int value);
 

@@ -193,6 +193,49 @@ def test_decode_graph_replay_matches_direct_launches():
         assert np.array_equal(a, b)
 
 
+def test_decode_fused_rope_kv_matches_separate_kernel():
+    """RoPE, q and the KV store / residual quantise done in the QKV GEMM's
+    epilogue give bit for bit what the separate kernel gives: logits, hidden
+    states and every exported KV slice, free running over two steps."""
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    cfg = synth.config("c2").with_(ctx_len=700, rho=0.5, seed=29)
+    B = cfg.batch
+    lens = [700, 5, 300, 64, 1, 640, 129, 12][:B]
+    outs = []
+    for fuse in (1, 0):
+        w = synth.make_weights(cfg)
+        rng = w["rng"]
+        ctx = synth.make_context(cfg, rng, lens)
+        eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=max(lens) + 2)
+        E.load_context(eng, cfg, ctx)
+        eng.set_option(fl.FL_OPT_FUSE_QKV, fuse)
+        s = torch.cuda.Stream()
+        res = []
+        for _ in range(2):
+            h0 = torch.from_numpy(synth.make_h0(cfg, rng, B)).cuda()
+            h_out = torch.empty((B, cfg.d_model), dtype=torch.float32, device="cuda")
+            lg = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+            torch.cuda.synchronize()
+            eng.decode_step(h0, B, h_out, lg, stream=s)
+            s.synchronize()
+            res += [lg.cpu().numpy(), h_out.cpu().numpy()]
+        assert eng.sync_status(s) == 0
+        for layer in range(cfg.n_layers):
+            for loop in range(1, cfg.n_loops + 1):
+                for b in (0, 4, 5):
+                    for which in (0, 1):
+                        c_, s_ = eng.export_slice(layer, loop, b, which, lens[b] + 2)
+                        res.append(c_)
+                        if s_ is not None:
+                            res.append(s_.view(np.uint16))
+        outs.append(res)
+        eng.close()
+    assert len(outs[0]) == len(outs[1])
+    for a, b in zip(*outs):
+        assert np.array_equal(a, b)
+
+
 def test_decode_free_running_selection_and_column_sets_are_valid():
     cfg = synth.config("c1").with_(mode="decode", batch=6, rho=0.4, c_cols=20, seed=19, seq_len=0)
     lens = [90, 33, 7, 64, 120, 1]

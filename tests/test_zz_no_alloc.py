@@ -32,14 +32,26 @@ def _operands(torch, m, n, k, seed):
 
 def test_no_alloc_gemm_matches_the_caller_scratch_gemm_on_two_calls(env):
     torch, fl = env
-    # two calls in a row with different split counts: the second must not see the first's tickets
-    for m, n, k, seed in ((8, 3072, 2048, 1), (16, 2048, 5632, 2)):
-        A, B = _operands(torch, m, n, k, seed)
-        want = fl.gemm(A, B, swap_ab=True)
-        got = fl.gemm_noalloc(A, B)
+    # Both entry points run the same kernel with the same tile width, split
+    # count and ordered ticket reduction, so the products must agree bit for bit.
+    # Two calls in a row with different split counts: the second must not see
+    # the first's tickets or partials.
+    shapes = ((8, 3072, 2048, 1), (16, 2048, 5632, 2))
+    ops = [_operands(torch, m, n, k, seed) for m, n, k, seed in shapes]
+    wants = [fl.gemm(A, B, swap_ab=True) for A, B in ops]
+    outs = [torch.empty((m, n), dtype=torch.float32, device="cuda") for m, n, _, _ in shapes]
+    fl.gemm_noalloc(*ops[0], out=outs[0])      # first call on this device: looks up the array's address
+    torch.cuda.synchronize()
+    free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
+    for (A, B), out, want in zip(ops, outs, wants):
+        out.fill_(float("nan"))
+        got = fl.gemm_noalloc(A, B, out=out)
         torch.cuda.synchronize()
-        bound = (A.double().abs() @ B.double().abs().T) * (k * 2.0 ** -23) + 1e-6
-        assert torch.all((got.double() - want.double()).abs() <= bound)
+        assert got.data_ptr() == out.data_ptr()
+        assert torch.equal(got, want)
+    # the calls allocated nothing: neither the device's free memory nor torch's pool moved
+    assert torch.cuda.mem_get_info()[0] == free0
+    assert torch.cuda.memory_allocated() == alloc0
 
 
 def test_no_alloc_gemm_refuses_shapes_beyond_its_scratch(env):
