@@ -29,12 +29,8 @@ integer -- the quantiser (residual, scale and code are taken in IEEE fp32, as
 the kernels take them) and the selection keys (rounded to fp32 and ordered by
 their bit pattern).  The residual chain is defined as fp32 accumulation in loop
 order, base first; bf16 storage of base / per-loop KV is modelled by
-round-to-nearest-even.  For workloads that declare bf16 compute, ``bf16_ops``
-rounds the four GEMM input activations (the pre-norm outputs fed to QKV and
-gate/up, the attention output fed to O, the SwiGLU output fed to down) to
-bf16, the operands bf16 compute multiplies: the quantiser's codes are decided
-from the keys those operands give, so both sides take that integer decision in
-the same precision.  Accumulation and every other step stay fp64.
+round-to-nearest-even.  Activations are never rounded: the oracle is the plain
+high-precision statement of the step, whatever precision the GPU computes in.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_pins.py``
 against a definition other than itself (dense limit, brute force, closed
@@ -226,15 +222,10 @@ def prepare_weights(w: dict) -> dict:
     return out
 
 
-def _op(x, bf16_ops):
-    """A GEMM input activation: as is, or rounded to bf16 for bf16-compute workloads."""
-    return bf16_round(x) if bf16_ops else x
-
-
-def _qkv(cfg, lw, h, pos, bf16_ops=False):
+def _qkv(cfg, lw, h, pos):
     """Pre-norm, fused QKV projection, RoPE on q and k.  Returns q [n,H,hd], k, v [n,Hkv,hd]."""
     H, Hkv, hd = cfg.n_heads, cfg.n_kv_heads, cfg.head_dim
-    x = _op(rmsnorm(h, lw["attn_norm"], cfg.rms_eps), bf16_ops)
+    x = rmsnorm(h, lw["attn_norm"], cfg.rms_eps)
     y = x @ lw["w_qkv"].T
     q = y[:, :H * hd].reshape(-1, H, hd)
     k = y[:, H * hd:(H + Hkv) * hd].reshape(-1, Hkv, hd)
@@ -242,10 +233,10 @@ def _qkv(cfg, lw, h, pos, bf16_ops=False):
     return apply_rope(q, pos, cfg.rope_theta), apply_rope(k, pos, cfg.rope_theta), v
 
 
-def _mlp_update(cfg, lw, h, bf16_ops=False):
+def _mlp_update(cfg, lw, h):
     """h + s * W_down(silu(W_gate x) * W_up x), x = RMSNorm(h)."""
-    x = _op(rmsnorm(h, lw["mlp_norm"], cfg.rms_eps), bf16_ops)
-    a = _op(silu(x @ lw["w_gate"].T) * (x @ lw["w_up"].T), bf16_ops)
+    x = rmsnorm(h, lw["mlp_norm"], cfg.rms_eps)
+    a = silu(x @ lw["w_gate"].T) * (x @ lw["w_up"].T)
     return h + cfg.resid_scale * (a @ lw["w_down"].T)
 
 
@@ -364,12 +355,12 @@ class Result:
         self.h, self.logits, self.trace = h, logits, trace
 
 
-def _logits(cfg, W, h_rows, bf16_ops=False):
-    x = _op(rmsnorm(h_rows, W["final_norm"], cfg.rms_eps), bf16_ops)
+def _logits(cfg, W, h_rows):
+    x = rmsnorm(h_rows, W["final_norm"], cfg.rms_eps)
     return x @ W["w_out"].T
 
 
-def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None, bf16_ops=False):
+def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None):
     """The lazy-update looped forward over the call's N tokens.
 
     Loop 1 is dense.  At loops l = 2..K: select the top-n_sel tokens by the
@@ -396,7 +387,7 @@ def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None, bf16_ops=
 
     # ---- loop 1: every token, full causal attention over the base KV ----
     for j, lw in enumerate(W["layers"]):
-        q, k, v = _qkv(cfg, lw, h, pos, bf16_ops)
+        q, k, v = _qkv(cfg, lw, h, pos)
         for i in range(N):
             cache.base_k[j, seq[i], :, pos[i]] = cache.store_kv(k[i])
             cache.base_v[j, seq[i], :, pos[i]] = cache.store_kv(v[i])
@@ -406,8 +397,8 @@ def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None, bf16_ops=
             vv = cache.chain("v", j, 1, seq[i], rows)
             O[j, i], lse[j, i] = _attn_full(q[i], kk, vv, tau)
         qlast[j] = q
-        h = h + s_res * (_op(O[j].reshape(N, H * hd), bf16_ops) @ lw["w_o"].T)
-        h = _mlp_update(cfg, lw, h, bf16_ops)
+        h = h + s_res * (O[j].reshape(N, H * hd) @ lw["w_o"].T)
+        h = _mlp_update(cfg, lw, h)
         trace["applications"] += 1
     key = np.sum((h - np.asarray(h0, F64)) ** 2, axis=1).astype(F32)
     trace["h"] = {1: h.copy()}
@@ -422,7 +413,7 @@ def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None, bf16_ops=
         trace["sel"][l] = S.astype(np.int32)
         h_prev = h[S].copy()
         for j, lw in enumerate(W["layers"]):
-            q, k, v = _qkv(cfg, lw, h[S], pos[S], bf16_ops)
+            q, k, v = _qkv(cfg, lw, h[S], pos[S])
             # residual rows of loop l: zero for every token of the call ...
             for i in range(N):
                 for nm in ("k", "v"):
@@ -499,8 +490,8 @@ def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None, bf16_ops=
                     O[j, i, hh] = num / z
                     lse[j, i, hh] = mx + math.log(z)
                 qlast[j, i] = q[a]
-            hs = h[S] + s_res * (_op(O[j, S].reshape(len(S), H * hd), bf16_ops) @ lw["w_o"].T)
-            h[S] = _mlp_update(cfg, lw, hs, bf16_ops)
+            hs = h[S] + s_res * (O[j, S].reshape(len(S), H * hd) @ lw["w_o"].T)
+            h[S] = _mlp_update(cfg, lw, hs)
             trace["applications"] += 1
         last[S] = l
         key = np.zeros(N, F32)
@@ -510,7 +501,7 @@ def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None, bf16_ops=
     return h, trace
 
 
-def _run_dense(cfg, W, cache: KVCache, h0, seq, pos, bf16_ops=False):
+def _run_dense(cfg, W, cache: KVCache, h0, seq, pos):
     """Dense looped forward with a per-loop KV cache: h_l = block(h_{l-1}), l = 1..K.
 
     "Looped Transformer 教程", 第一步 and 第四步 (per_loop KV); "循环Transformer
@@ -524,7 +515,7 @@ def _run_dense(cfg, W, cache: KVCache, h0, seq, pos, bf16_ops=False):
     apps = 0
     for l in range(1, cfg.n_loops + 1):
         for j, lw in enumerate(W["layers"]):
-            q, k, v = _qkv(cfg, lw, h, pos, bf16_ops)
+            q, k, v = _qkv(cfg, lw, h, pos)
             for i in range(N):
                 cache.kv_k[j, l - 1, seq[i], :, pos[i]] = cache.store_kv(k[i])
                 cache.kv_v[j, l - 1, seq[i], :, pos[i]] = cache.store_kv(v[i])
@@ -533,19 +524,19 @@ def _run_dense(cfg, W, cache: KVCache, h0, seq, pos, bf16_ops=False):
                 kk = cache.kv_k[j, l - 1, seq[i]][:, :pos[i] + 1]
                 vv = cache.kv_v[j, l - 1, seq[i]][:, :pos[i] + 1]
                 O[i], _ = _attn_full(q[i], kk, vv, tau)
-            h = h + cfg.resid_scale * (_op(O.reshape(N, H * hd), bf16_ops) @ lw["w_o"].T)
-            h = _mlp_update(cfg, lw, h, bf16_ops)
+            h = h + cfg.resid_scale * (O.reshape(N, H * hd) @ lw["w_o"].T)
+            h = _mlp_update(cfg, lw, h)
             apps += 1
     return h, {"applications": apps}
 
 
-def _call(cfg, W, cache, h0, seq, pos, tile, forced, bf16_ops):
+def _call(cfg, W, cache, h0, seq, pos, tile, forced):
     if cache.dense:
-        return _run_dense(cfg, W, cache, h0, seq, pos, bf16_ops)
-    return _run_lazy(cfg, W, cache, h0, seq, pos, tile, forced, bf16_ops)
+        return _run_dense(cfg, W, cache, h0, seq, pos)
+    return _run_lazy(cfg, W, cache, h0, seq, pos, tile, forced)
 
 
-def prefill(cfg, W, cache: KVCache, h0: np.ndarray, B: int, T: int, forced=None, bf16_ops=False) -> Result:
+def prefill(cfg, W, cache: KVCache, h0: np.ndarray, B: int, T: int, forced=None) -> Result:
     """Prefill T tokens for each of B empty sequences; h0 is [B*T, d] (sequence-major).
 
     Query tiles are q_tile consecutive positions of one sequence; the token
@@ -556,13 +547,13 @@ def prefill(cfg, W, cache: KVCache, h0: np.ndarray, B: int, T: int, forced=None,
     seq = np.repeat(np.arange(B), T)
     pos = np.tile(np.arange(T), B)
     tile = seq * ((T + cfg.q_tile - 1) // cfg.q_tile) + pos // cfg.q_tile
-    h, trace = _call(cfg, W, cache, h0, seq, pos, tile, forced, bf16_ops)
+    h, trace = _call(cfg, W, cache, h0, seq, pos, tile, forced)
     cache.lens[:B] = T
     last_rows = np.arange(B) * T + (T - 1)
-    return Result(h, _logits(cfg, W, h[last_rows], bf16_ops), trace)
+    return Result(h, _logits(cfg, W, h[last_rows]), trace)
 
 
-def decode_step(cfg, W, cache: KVCache, h0: np.ndarray, forced=None, bf16_ops=False) -> Result:
+def decode_step(cfg, W, cache: KVCache, h0: np.ndarray, forced=None) -> Result:
     """Append one token to each of the B sequences; h0 is [B, d].
 
     Each new token is its own query tile; the token ranking pools the B new
@@ -572,6 +563,6 @@ def decode_step(cfg, W, cache: KVCache, h0: np.ndarray, forced=None, bf16_ops=Fa
     seq = np.arange(B)
     pos = cache.lens[:B].copy()
     assert np.all(pos < cache.tmax)
-    h, trace = _call(cfg, W, cache, h0, seq, pos, seq.copy(), forced, bf16_ops)
+    h, trace = _call(cfg, W, cache, h0, seq, pos, seq.copy(), forced)
     cache.lens[:B] += 1
-    return Result(h, _logits(cfg, W, h, bf16_ops), trace)
+    return Result(h, _logits(cfg, W, h), trace)

@@ -17,17 +17,6 @@ from cross_loop_sparsity_b200 import synth
 
 TOL = 2e-2   # max |gpu - oracle| <= TOL * RMS(oracle), for hidden states and logits
 
-# Workloads that declare bf16 compute: the oracle rounds the GEMM input
-# activations to bf16 (the operands bf16 compute multiplies), so the
-# quantiser's integer decisions are taken on keys of the same precision on both
-# sides.  The fp32 tiny workload keeps the plain fp64 oracle.
-BF16_WORKLOADS = {"c2", "c3", "c4", "c5", "c5_int2"}
-
-
-def bf16_ops(cfg):
-    return cfg.name in BF16_WORKLOADS
-
-
 def rel_err(got, want):
     want = np.asarray(want, np.float64)
     rms = float(np.sqrt(np.mean(want ** 2)))
@@ -80,7 +69,7 @@ def run_prefill(cfg, B, T, forced=True, dense=False):
     h0 = synth.make_h0(cfg, w["rng"], B * T)
     W = orc.prepare_weights(w)
     ocache = orc.KVCache(cfg, B, T)
-    ref = orc.prefill(cfg, W, ocache, h0, B, T, bf16_ops=bf16_ops(cfg))
+    ref = orc.prefill(cfg, W, ocache, h0, B, T)
     eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=T, max_tokens=B * T)
     n_tiles = B * ((T + cfg.q_tile - 1) // cfg.q_tile)
     if forced and not dense and cfg.n_loops > 1:
@@ -125,7 +114,7 @@ def run_decode(cfg, lens, forced=True, dense=False, steps=1, extra_ctx=0):
     for _ in range(steps):
         h0 = synth.make_h0(cfg, rng, B)
         pos = cache.lens[:B].copy()
-        ref = orc.decode_step(cfg, W, cache, h0, bf16_ops=bf16_ops(cfg))
+        ref = orc.decode_step(cfg, W, cache, h0)
         if forced and not dense and cfg.n_loops > 1:
             sel, cols, ncols = forced_arrays(cfg, ref.trace, B)
             if forced == "sel":   # token selections and codes handed over, column sets left free
