@@ -20,11 +20,7 @@ import hashlib
 import json
 import math
 import os
-import re
-import statistics
-import subprocess
 import sys
-import tempfile
 import time
 
 import numpy as np
@@ -33,10 +29,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from cross_loop_sparsity_b200 import synth  # noqa: E402
+from cross_loop_sparsity_b200.clocks import ClockSampler  # noqa: E402
 
 WORKLOAD = "c2"
 METRIC = "looped decode tokens/s at K loops; KV-cache bytes/token; % of HBM/TC roofline"
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "gemm_decode_c2.md")
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "gemm_decode_c2_traffic.json")
 GEMM_SOURCE = os.path.join(ROOT, "cross_loop_sparsity_b200", "csrc", "fl_gemm.cu")
 
 
@@ -48,6 +45,12 @@ def parse():
     ap.add_argument("--impl", choices=["flashloop", "reference"], default="flashloop")
     ap.add_argument("--no-dense", action="store_true", help="skip the dense-looped GPU baseline")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
+    ap.add_argument("--workload", default=None, choices=["c1", "c2", "c3", "c4", "c5", "c5_int2"],
+                    help="time this one workload as the line's headline (default: c2, with every other "
+                         "workload summarised under per_config)")
+    ap.add_argument("--no-per-config", action="store_true", help="time the headline workload only")
+    ap.add_argument("--resid-layout", choices=["sparse", "dense"], default="sparse",
+                    help="lazy-path KV residual storage: rows for recomputed tokens only (sparse) or every position")
     return ap.parse_args()
 
 
@@ -66,18 +69,15 @@ def measured_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
-def gemm_traffic():
-    """Per-launch DRAM bytes of the decode GEMM from the committed ncu summary,
-    or None when the summary is missing or the GEMM source changed since."""
-    if not os.path.exists(PROFILE_SUMMARY):
+def gemm_traffic_ratio():
+    """DRAM bytes per algorithmic byte of the decode GEMM, from the committed
+    ncu capture (profiles/gemm_decode_c2_traffic.json), or None when the file
+    is missing or the GEMM source changed since it was taken."""
+    if not os.path.exists(TRAFFIC_JSON):
         return None
-    txt = open(PROFILE_SUMMARY).read()
-    m = re.search(r"gemm_source_sha256:\s*([0-9a-f]{64})", txt)
-    t = re.search(r"traffic_bytes_per_step:\s*([0-9.eE+]+)", txt)
-    if not m or not t:
-        return None
+    d = json.load(open(TRAFFIC_JSON))
     cur = hashlib.sha256(open(GEMM_SOURCE, "rb").read()).hexdigest()
-    return float(t.group(1)) if m.group(1) == cur else None
+    return float(d["dram_bytes_per_algorithmic_byte"]) if d.get("gemm_source_sha256") == cur else None
 
 
 def gemm_algorithmic_bytes(cfg, n_first, n_sel):
@@ -97,57 +97,6 @@ def gemm_algorithmic_bytes(cfg, n_first, n_sel):
     return total
 
 
-class ClockSampler:
-    """nvidia-smi clocks / throttle reasons every 200 ms while running."""
-
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-
-    def start(self):
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
-                                         stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
-
-    def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.f.flush()
-        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
-        os.unlink(self.f.name)
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            r = [x.strip() for x in r]
-            if len(r) < 9:
-                continue
-            try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names, r[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
-
-
 # ------------------------------------------------------------------ replicas (one per GPU)
 from cross_loop_sparsity_b200 import replicas  # noqa: E402
 
@@ -156,6 +105,12 @@ max_over_ranks = replicas.max_over_ranks
 
 
 # ------------------------------------------------------------------ the library arm
+def lazy_cfg(cfg, layout):
+    """The lazy arm's config: sparse residual storage sized to the synthetic
+    context's recompute rate plus the batch's new tokens, or every position."""
+    return cfg.with_(resid_rows=synth.sparse_rows(cfg, cfg.batch)) if layout == "sparse" else cfg
+
+
 def setup_engine(cfg, dense, stream):
     import torch
     from cross_loop_sparsity_b200 import flashloop as fl
@@ -202,31 +157,25 @@ def run_library(args, world, rank, local):
     from cross_loop_sparsity_b200 import build
     from cross_loop_sparsity_b200 import flashloop as fl
     build.build()
-    cfg = synth.config(WORKLOAD)
-    B = cfg.batch
     stream = torch.cuda.Stream()
+    if args.workload and args.workload != WORKLOAD:
+        return run_single(args.workload, args, world, rank, local, stream)
+    cfg = lazy_cfg(synth.config(WORKLOAD), args.resid_layout)
+    B = cfg.batch
     eng, lens, h0, w = setup_engine(cfg, False, stream)
     h0_dev = torch.from_numpy(h0).cuda()
     logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
     sampler = ClockSampler(local)
+    # the GEMMs stamp their own start (dependency released) and end on the GPU's
+    # global timer during the timed replays: two atomics per CTA
+    eng.set_option(fl.FL_OPT_GEMM_TIMES, 1)
     ms, clocks = time_steps(eng, lens, h0_dev, logits, stream, args.steps, args.warmup, world, sampler)
     ms_step = ms / args.steps
     assert eng.sync_status(stream) == 0, "a kernel reported an error"
     launches_per_step = eng.kernels_per_call() + 1          # + the length-reset kernel
-
-    # profiled pass: per-kind device time from CUDA events around each kernel
-    prof, prof_mode = None, None
-    for use_graph in (1, 0):
-        try:
-            prof = profile_pass(eng, fl, lens, h0_dev, logits, stream, max(3, min(10, args.steps)), use_graph)
-            prof_mode = "graph replay with event-record nodes" if use_graph else "direct launches"
-            break
-        except Exception as e:  # graph event nodes refused: profile direct launches instead
-            print(f"profile pass ({'graph' if use_graph else 'direct'}) failed: {e}", file=sys.stderr)
-            torch.cuda.synchronize()
-    eng.set_option(fl.FL_OPT_PROFILE, 0)
-    eng.set_option(fl.FL_OPT_USE_GRAPH, 1)
-    prof = prof or {}
+    gemm_ms, gemm_n = gemm_time_per_step(eng, lens, h0_dev, logits, stream, args.steps)
+    assert gemm_ms <= ms_step * 1.001, (gemm_ms, ms_step)   # launches never overlap in the sum
+    eng.set_option(fl.FL_OPT_GEMM_TIMES, 0)
 
     # end to end through the C ABI with pinned host buffers (copies inside the timed region)
     h0_host = torch.from_numpy(h0).pin_memory()
@@ -242,7 +191,7 @@ def run_library(args, world, rank, local):
 
     dense = None
     if not args.no_dense:
-        deng, dlens, dh0, _ = setup_engine(cfg, True, stream)
+        deng, dlens, dh0, _ = setup_engine(cfg.with_(resid_rows=0), True, stream)
         dms, _ = time_steps(deng, dlens, torch.from_numpy(dh0).cuda(), logits, stream, max(5, args.steps // 2),
                             max(3, args.warmup // 2), world)
         dsteps = max(5, args.steps // 2)
@@ -254,16 +203,19 @@ def run_library(args, world, rank, local):
         torch.cuda.empty_cache()
 
     hbm, tc, peak_kind = measured_peaks()
-    gemm = prof.get("gemm", {"ms_per_step": float("nan"), "launches_per_step": 0})
     gbytes = gemm_algorithmic_bytes(cfg, B, n_sel)
-    achieved = gbytes / (gemm["ms_per_step"] / 1e3) / 1e9
-    n_launch = max(1, gemm["launches_per_step"])
-    traffic = gemm_traffic()
+    achieved = gbytes / (gemm_ms / 1e3) / 1e9
+    n_launch = max(1, gemm_n)
+    ratio = gemm_traffic_ratio()
     roofline = {"kernel": "k_gemm_tc (all tcgen05 GEMMs of the step: QKV, O, gate/up, down, LM head)",
                 "bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "peak_source": f"{peak_kind} hbm_gbs", "traffic": None if traffic is None else traffic / n_launch,
+                "peak_source": f"{peak_kind} hbm_gbs",
+                "traffic": None if ratio is None else ratio * gbytes / n_launch,
                 "algorithmic_bytes_per_launch": gbytes / n_launch, "launches_per_step": n_launch,
-                "avg_launch_us": gemm["ms_per_step"] * 1e3 / n_launch}
+                "avg_launch_us": gemm_ms * 1e3 / n_launch, "gemm_ms_per_step": gemm_ms,
+                "gemm_share_of_step": gemm_ms / ms_step,
+                "timing": "per launch: last CTA's end - first CTA's return from the dependency wait, stamped by "
+                          "the kernel on the global timer during graph replays of the timed step; summed per step"}
     step_bytes = gbytes + kv_bytes_read(cfg, n_sel)
     whole = {"bytes_per_step": step_bytes, "roofline_ms": step_bytes / hbm / 1e6,
              "frac_of_hbm_roofline": (step_bytes / hbm / 1e6) / ms_step}
@@ -281,7 +233,7 @@ def run_library(args, world, rank, local):
                    "graph": "decode step captured as one CUDA graph, replayed"},
         "kv_bytes": {"per_token_per_layer": per, "dense_per_token_per_layer": dense_per,
                      "reduction": dense_per / per, "cache_total": tot},
-        "roofline": roofline, "whole_step": whole, "profile": prof, "profile_mode": prof_mode,
+        "roofline": roofline, "whole_step": whole,
         "e2e": {"value": e2e_tps, "unit": "tokens/s", "h2d_bytes_per_step": B * cfg.d_model * 4,
                 "d2h_bytes_per_step": B * cfg.vocab * 4},
         "gpu_launches": launches_per_step * args.steps, "gpu_launches_per_step": launches_per_step,
@@ -289,24 +241,63 @@ def run_library(args, world, rank, local):
         "speedup_vs_dense": None if dense is None else (world * B / (ms_step / 1e3)) / dense["tokens_per_s"],
         "cpu_baseline": cpu, "clocks": clocks,
     }
+    # every other workload: lazy and dense-looped throughput, speedup, KV bytes, roofline, clocks
+    per = {WORKLOAD: {"workload": workload_desc(cfg), "unit": "tokens/s",
+                      "lazy": {"tokens_per_s": out["value"], "ms_per_step": ms_step,
+                               "kv_bytes_per_token_per_layer": out["kv_bytes"]["per_token_per_layer"],
+                               "roofline": decode_roofline(cfg, ms_step, n_sel), "clocks": clocks},
+                      "dense_looped": None if dense is None else {
+                          "tokens_per_s": dense["tokens_per_s"], "ms_per_step": dense["ms_per_step"],
+                          "kv_bytes_per_token_per_layer": dense_per,
+                          "roofline": decode_roofline(cfg, dense["ms_per_step"], B, True)},
+                      "speedup_vs_dense": out["speedup_vs_dense"],
+                      "kv_bytes_reduction": out["kv_bytes"]["reduction"]}}
+    if not args.no_per_config and args.workload is None:
+        for nm in PER_CONFIG:
+            try:
+                per[nm] = measure_workload(nm, args, world, local, stream)
+            except Exception as e:     # one workload failing must not hide the others
+                per[nm] = {"error": f"{type(e).__name__}: {e}"}
+                torch.cuda.synchronize()
+                torch.cuda.empty_cache()
+    out["per_config"] = per
     if rank == 0:
         print(json.dumps(out), flush=True)
 
 
-def profile_pass(eng, fl, lens, h0_dev, logits, stream, steps, use_graph):
-    eng.set_option(fl.FL_OPT_USE_GRAPH, use_graph)
-    eng.set_option(fl.FL_OPT_PROFILE, 1)
-    acc = {}
-    for i in range(steps + 2):
+def run_single(name, args, world, rank, local, stream):
+    """One workload as the line's headline (its lazy throughput), with its dense-looped baseline."""
+    r = measure_workload(name, args, world, local, stream)
+    lazy = r["lazy"]
+    ms = lazy.get("ms_per_step", lazy.get("ms_per_call"))
+    cfg = synth.config(name)
+    units = cfg.batch if cfg.mode == "decode" else cfg.batch * cfg.seq_len
+    rl = lazy["roofline"]
+    out = {"metric": METRIC, "value": lazy["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
+           "steps": r.get("timed_steps", r.get("timed_calls")), "warmup": args.warmup, "ms_per_step": ms,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+           "data": "synthetic (device-drawn weights and context)",
+           "config": {"workload": r["workload"], "global_batch": world * cfg.batch, "units_per_step": units,
+                      "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+           "roofline": {"kernel": "whole step", "bound": rl["bound"], "frac": rl["frac"], "peak": rl["peak"],
+                        "peak_source": rl["peak_source"]},
+           "gpu_launches": None, "speedup_vs_dense": r["speedup_vs_dense"], "dense_baseline": r["dense_looped"],
+           "kv_bytes_reduction": r["kv_bytes_reduction"], "clocks": lazy["clocks"], "detail": r}
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def gemm_time_per_step(eng, lens, h0_dev, logits, stream, steps):
+    """Mean over `steps` replays of the step's summed GEMM device time (the
+    kernels' own global-timer stamps), and the GEMM launches per step."""
+    tot, n = 0.0, 0
+    reps = max(3, min(steps, 20))
+    for _ in range(reps):
         eng.reset(lens, stream=stream)
         eng.decode_step(h0_dev, len(lens), None, logits, stream=stream)
-        p = eng.profile(stream)
-        if i >= 2:
-            for k, (t, n) in p.items():
-                a = acc.setdefault(k, [0.0, 0])
-                a[0] += t
-                a[1] = n
-    return {k: {"ms_per_step": v[0] / steps, "launches_per_step": v[1]} for k, v in acc.items()}
+        ms, n = eng.gemm_times(stream)
+        tot += ms
+    return tot / reps, n
 
 
 def kv_bytes_read(cfg, n_sel):
@@ -321,6 +312,165 @@ def kv_bytes_read(cfg, n_sel):
     for l in range(2, cfg.n_loops + 1):
         corr += M * n_sel * Hkv * cfg.c_cols * 2 * (hd * 2 + (l - 1) * res) * 2
     return base + dscore + corr
+
+
+# ------------------------------------------------------------------ every workload (per_config)
+PER_CONFIG = ["c1", "c3", "c4", "c5", "c5_int2"]
+
+
+def dense_kv_bytes_read(cfg):
+    """KV bytes a dense-looped decode step reads: every loop's own K/V of every column."""
+    return cfg.n_layers * cfg.n_loops * cfg.batch * cfg.n_kv_heads * (cfg.ctx_len + 1) * cfg.head_dim * 2 * 2
+
+
+def decode_roofline(cfg, ms, n_sel, dense=False):
+    """Whole-step algorithmic bytes against the HBM peak (decode is bandwidth-bound)."""
+    hbm, _, kind = measured_peaks()
+    B = cfg.batch
+    if dense:
+        nbytes = gemm_algorithmic_bytes(cfg, B, B) + dense_kv_bytes_read(cfg)
+    else:
+        nbytes = gemm_algorithmic_bytes(cfg, B, n_sel) + kv_bytes_read(cfg, n_sel)
+    t_roof = nbytes / hbm / 1e6
+    return {"bound": "hbm", "bytes_per_step": nbytes, "roofline_ms": t_roof, "frac": t_roof / ms,
+            "peak": hbm, "peak_source": f"{kind} hbm_gbs"}
+
+
+def prefill_flops(cfg, sel=None):
+    """Algorithmic FLOPs of one prefill call.  Dense (sel None): K loops of every
+    token's GEMMs and causal attention.  Lazy: loop 1 dense; each later loop the
+    recomputed tokens' GEMMs, the delta-score products of tiles choosing their
+    column set (q_l.K_l and q_last.K_last over the query's causal columns) and
+    the correction over c columns; every call ends with the last rows' LM head."""
+    d, f, hq, qkv, H, hd = cfg.d_model, cfg.ffn_dim, cfg.n_heads * cfg.head_dim, cfg.qkv_rows, cfg.n_heads, cfg.head_dim
+    B, T, M, K = cfg.batch, cfg.seq_len, cfg.n_layers, cfg.n_loops
+    gemm_tok = 2 * (d * qkv + hq * d + 2 * d * f + f * d)
+    attn = 4 * H * hd * B * T * (T + 1) / 2
+    head = 2 * d * cfg.vocab * B
+    if sel is None:
+        return K * M * (B * T * gemm_tok + attn) + head
+    total = M * (B * T * gemm_tok + attn) + head
+    tps = (T + cfg.q_tile - 1) // cfg.q_tile
+    chosen = set()
+    for l in range(2, K + 1):
+        S = np.asarray(sel[l - 2])
+        tiles = (S // T) * tps + (S % T) // cfg.q_tile
+        new = [t for t in np.unique(tiles) if t not in chosen]
+        pos = S % T
+        for t in new:
+            total += M * 4 * hd * H * float(np.sum(pos[tiles == t] + 1))
+        chosen.update(new)
+        total += M * len(S) * (gemm_tok + 8 * H * hd * cfg.c_cols)
+    return total
+
+
+def measure_decode(name, args, world, local, stream):
+    """Lazy and dense-looped decode steps of one workload on device-drawn inputs."""
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    cfg = lazy_cfg(synth.config(name), args.resid_layout)
+    B, d = cfg.batch, cfg.d_model
+    lens = [cfg.ctx_len] * B
+    steps, warm = (10, 3) if cfg.n_layers * cfg.d_model > 65536 else (20, 5)
+    w = synth.make_weights_device(cfg)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(cfg.seed + 11)
+    h0 = torch.randn((B, d), generator=g, device="cuda", dtype=torch.float32)
+    logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    res = {"workload": workload_desc(cfg), "unit": "tokens/s", "timed_steps": steps}
+    for dense in (False, True):
+        ecfg = cfg.with_(resid_rows=0) if dense else cfg
+        eng = fl.FlashLoop(ecfg, w, max_batch=B, max_ctx=cfg.ctx_len + 1, resid_bits=16 if dense else None,
+                           stream=stream)
+        eng.load_context_device(lens, dense=dense)
+        ms, clocks = time_steps(eng, lens, h0, logits, stream, steps, warm, world, ClockSampler(local))
+        assert eng.sync_status(stream) == 0, f"{name}: a kernel reported an error"
+        ms_step = ms / steps
+        tot, per, dense_per = eng.kv_bytes()
+        n_sel = B if dense else max(1, min(B, math.ceil(cfg.rho * B - 1e-9)))
+        part = {"tokens_per_s": replicas.job_throughput(world, B, ms_step), "ms_per_step": ms_step,
+                "kv_bytes_per_token_per_layer": per, "roofline": decode_roofline(cfg, ms_step, n_sel, dense),
+                "gpu_launches_per_step": eng.kernels_per_call() + 1, "clocks": clocks}
+        eng.close()
+        del eng
+        torch.cuda.empty_cache()
+        res["dense_looped" if dense else "lazy"] = part
+    res["speedup_vs_dense"] = res["lazy"]["tokens_per_s"] / res["dense_looped"]["tokens_per_s"]
+    res["kv_bytes_reduction"] = (res["dense_looped"]["kv_bytes_per_token_per_layer"] /
+                                 res["lazy"]["kv_bytes_per_token_per_layer"])
+    del w
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_prefill(name, args, world, local, stream):
+    """Lazy and dense-looped prefill calls of one workload (B sequences of T tokens)."""
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    cfg = synth.config(name)
+    if args.resid_layout == "sparse":   # room for every recomputed token of the call in one sequence's pool
+        cfg = cfg.with_(resid_rows=min(cfg.seq_len, int(math.ceil(cfg.rho * cfg.batch * cfg.seq_len - 1e-9))))
+    B, T, d = cfg.batch, cfg.seq_len, cfg.d_model
+    big = B * T * cfg.n_layers > 100000
+    steps, warm = (3, 1) if big else (20, 5)
+    w = synth.make_weights_device(cfg)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(cfg.seed + 13)
+    h0 = torch.randn((B * T, d), generator=g, device="cuda", dtype=torch.float32)
+    logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+    _, tc, kind = measured_peaks()
+    res = {"workload": (f"prefill, B={B} x {T} tokens, d_model={d}, {cfg.n_heads}q/{cfg.n_kv_heads}kv heads x "
+                        f"{cfg.head_dim}, ffn={cfg.ffn_dim}, {cfg.n_layers} shared layers x K={cfg.n_loops} loops, "
+                        f"rho={cfg.rho}, c={cfg.c_cols} per {cfg.q_tile}-query tile, int{cfg.resid_bits} g"
+                        f"{cfg.group_size}"), "unit": "tokens/s", "timed_calls": steps}
+    for dense in (False, True):
+        eng = fl.FlashLoop(cfg.with_(resid_rows=0) if dense else cfg, w, max_batch=B, max_ctx=T, max_tokens=B * T,
+                           resid_bits=16 if dense else None, stream=stream)
+        for _ in range(warm):
+            eng.reset(None, stream=stream)
+            eng.prefill(h0, B, T, None, logits, stream=stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        sampler = ClockSampler(local)
+        sampler.start()
+        time.sleep(0.3)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            eng.reset(None, stream=stream)
+            eng.prefill(h0, B, T, None, logits, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        clocks = sampler.stop()
+        ms = max_over_ranks(world, e0.elapsed_time(e1)) / steps
+        assert eng.sync_status(stream) == 0, f"{name}: a kernel reported an error"
+        sel = None
+        if not dense and cfg.n_loops > 1:
+            n_sel = max(1, min(B * T, math.ceil(cfg.rho * B * T - 1e-9)))
+            sel, _, _, _ = eng.read_trace(B * T, n_sel, B * ((T + cfg.q_tile - 1) // cfg.q_tile), stream=stream)
+        flops = prefill_flops(cfg, None if dense else sel)
+        _, per, _ = eng.kv_bytes()
+        t_roof = flops / (tc * 1e12) * 1e3
+        res["dense_looped" if dense else "lazy"] = {
+            "tokens_per_s": replicas.job_throughput(world, B * T, ms), "ms_per_call": ms,
+            "kv_bytes_per_token_per_layer": per, "gpu_launches_per_call": eng.kernels_per_call() + 1,
+            "roofline": {"bound": "tensor", "flops_per_call": flops, "roofline_ms": t_roof, "frac": t_roof / ms,
+                         "peak": tc, "peak_source": f"{kind} bf16_tflops"},
+            "clocks": clocks}
+        eng.close()
+        del eng
+        torch.cuda.empty_cache()
+    res["speedup_vs_dense"] = res["lazy"]["tokens_per_s"] / res["dense_looped"]["tokens_per_s"]
+    res["kv_bytes_reduction"] = (res["dense_looped"]["kv_bytes_per_token_per_layer"] /
+                                 res["lazy"]["kv_bytes_per_token_per_layer"])
+    del w
+    torch.cuda.empty_cache()
+    return res
+
+
+def measure_workload(name, args, world, local, stream):
+    return (measure_prefill if synth.config(name).mode == "prefill" else measure_decode)(name, args, world, local,
+                                                                                       stream)
 
 
 # ------------------------------------------------------------------ the oracle on the host
@@ -366,8 +516,9 @@ def run_reference(args, world, rank):
     w = synth.make_weights(cfg)
     rng = w["rng"]
     W = orc.prepare_weights(w)
-    # each step is a bounded sample: one sequence of the batch (its token through all K loops)
-    sample_b = 1
+    # each step is one full decode step of the workload: all B tokens through all K loops
+    # (about a second on the host cores, so the driver's warm-up + timed steps stay within a minute)
+    sample_b = cfg.batch
     lens = [cfg.ctx_len] * sample_b
     ctx = synth.make_context(cfg, rng, lens)
     cache = orc.KVCache.from_context(cfg, ctx, cfg.ctx_len + 1)
@@ -382,8 +533,8 @@ def run_reference(args, world, rank):
         orc.decode_step(cfg, W, cache, h0)
     dt = time.perf_counter() - t0
     tps = sample_b * args.steps / dt
-    sample = (f"each step: one sequence of the {cfg.batch}-sequence batch ({sample_b} token through all "
-              f"{cfg.n_loops} loops over the {cfg.ctx_len}-token context), fp64 numpy oracle")
+    sample = (f"each step: the full decode step of the workload ({sample_b} tokens through all {cfg.n_loops} "
+              f"loops over the {cfg.ctx_len}-token context), fp64 numpy oracle")
     out = {"impl": "reference", "metric": METRIC, "value": tps, "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",

@@ -3,10 +3,15 @@
 //
 // Lazy layout (resid_bits 4 or 2):
 //   base   bf16  [M][2][B][Hkv][T][hd]            loop-1 K (0) and V (1)
-//   codes  u8    [M][K-1][2][B][Hkv][T][hd*b/8]   residual codes of loops 2..K
-//   scales fp16  [M][K-1][2][B][Hkv][T][hd/g]     per-group scales of loops 2..K
-// Dense per-loop layout (resid_bits 16):
-//   base   bf16  [M][K][2][B][Hkv][T][hd]
+//   codes  u8    [M][K-1][2][B][Hkv][R][hd*b/8]   residual codes of loops 2..K
+//   scales fp16  [M][K-1][2][B][Hkv][R][hd/g]     per-group scales of loops 2..K
+// with R = T (one residual row per position) or, with sparse residual storage,
+// R = rows: a pool of rows per (layer, loop, K/V, sequence, KV head) holding the
+// residuals of the tokens that loop recomputed only, and an index
+//   ridx   int32 [M][K-1][B][T]  pool row of (layer, loop, sequence, position), -1 = zero residual
+//   rcount int32 [M][K-1][B]     pool rows in use (rows are taken in position order)
+// Dense layout (resid_bits 16): per_loop [M][K][2][B][Hkv][T][hd]; last_loop keeps
+// one loop slot, [M][1][2][B][Hkv][T][hd], which every loop overwrites
 // Tokens of one (sequence, KV head) are contiguous so a decode step streams them.
 // The reconstructed KV of loop m is base + code*scale of loops 2..m, added in
 // loop order in fp32 ("FlashLoop ...", abstract: KV residuals between
@@ -22,23 +27,38 @@ struct CacheView {
   uint16_t* base;
   uint8_t* codes;
   uint16_t* scales;
+  int rows;          // sparse residual storage: pool rows per (layer, loop, K/V, sequence, KV head); 0: R = T
+  int32_t* ridx;     // sparse: [M][K-1][B][T]
+  int* rcount;       // sparse: [M][K-1][B]
+
+  __host__ __device__ int pool_rows() const { return rows ? rows : T; }
+  __host__ __device__ size_t ridx_index(int j, int l, int b, int t) const {
+    return ((static_cast<size_t>(j) * (K - 1) + (l - 2)) * B + b) * T + t;
+  }
+  // pool row of the loop-l residual of (layer j, sequence b, position t); -1: zero residual
+  __device__ __forceinline__ int res_row(int j, int l, int b, int t) const {
+    return rows ? ridx[ridx_index(j, l, b, t)] : t;
+  }
 
   __host__ __device__ size_t row_bytes_codes() const { return static_cast<size_t>(hd) * bits / 8; }
   __host__ __device__ uint16_t* base_row(int j, int kv, int b, int h, int t) const {
     return base + ((((static_cast<size_t>(j) * 2 + kv) * B + b) * Hkv + h) * T + t) * hd;
   }
-  // dense per-loop KV, loop l in 1..K
+  // dense KV of loop l in 1..K: per-loop slots, or (K == 1, last_loop mode) one
+  // slot that every loop overwrites
+  __host__ __device__ int dense_slot(int l) const { return K == 1 ? 0 : l - 1; }
   __host__ __device__ uint16_t* dense_row(int j, int l, int kv, int b, int h, int t) const {
-    return base + (((((static_cast<size_t>(j) * K + (l - 1)) * 2 + kv) * B + b) * Hkv + h) * T + t) * hd;
+    return base + (((((static_cast<size_t>(j) * K + dense_slot(l)) * 2 + kv) * B + b) * Hkv + h) * T + t) * hd;
   }
-  __host__ __device__ size_t res_index(int j, int l, int kv, int b, int h, int t) const {
-    return ((((static_cast<size_t>(j) * (K - 1) + (l - 2)) * 2 + kv) * B + b) * Hkv + h) * T + t;
+  // residual row r of a pool (r = the position t without sparse storage)
+  __host__ __device__ size_t res_index(int j, int l, int kv, int b, int h, int r) const {
+    return ((((static_cast<size_t>(j) * (K - 1) + (l - 2)) * 2 + kv) * B + b) * Hkv + h) * pool_rows() + r;
   }
-  __host__ __device__ uint8_t* code_row(int j, int l, int kv, int b, int h, int t) const {
-    return codes + res_index(j, l, kv, b, h, t) * row_bytes_codes();
+  __host__ __device__ uint8_t* code_row(int j, int l, int kv, int b, int h, int r) const {
+    return codes + res_index(j, l, kv, b, h, r) * row_bytes_codes();
   }
-  __host__ __device__ uint16_t* scale_row(int j, int l, int kv, int b, int h, int t) const {
-    return scales + res_index(j, l, kv, b, h, t) * (hd >> lg);
+  __host__ __device__ uint16_t* scale_row(int j, int l, int kv, int b, int h, int r) const {
+    return scales + res_index(j, l, kv, b, h, r) * (hd >> lg);
   }
 };
 
@@ -88,15 +108,18 @@ __device__ __forceinline__ void chain_lane(const CacheView& cv, int j, int kv, i
   }
   const int gi = (lane * EPL) >> cv.lg;
   for (int l = 2; l <= m; ++l) {
+    const int r = cv.res_row(j, l, b, t);
+    if (r < 0) continue;   // no residual stored: zero
     int c[EPL];
-    lane_codes<EPL>(cv.code_row(j, l, kv, b, h, t), cv.bits, lane, c);
-    const float s = half_bits_to_f(cv.scale_row(j, l, kv, b, h, t)[gi]);
+    lane_codes<EPL>(cv.code_row(j, l, kv, b, h, r), cv.bits, lane, c);
+    const float s = half_bits_to_f(cv.scale_row(j, l, kv, b, h, r)[gi]);
 #pragma unroll
     for (int e = 0; e < EPL; ++e) out[e] = __fadd_rn(out[e], __fmul_rn(static_cast<float>(c[e]), s));
   }
 }
 
 // ---------------------------------------------------------------- residual quantiser
+// (the quantiser's scale and code rules, shared by its kernels)
 // The hardware reciprocal approximation (PTX rcp.approx, within 1 ulp of 1/x).
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
@@ -152,16 +175,38 @@ __device__ __forceinline__ void chain_lane2(const CacheView& cv, int j, int kv, 
   }
   const int gi = (lane * EPL) >> cv.lg;
   const size_t rb = cv.row_bytes_codes(), ns = cv.hd >> cv.lg;
-  const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * cv.T;   // rows between consecutive loops
-  const size_t r0 = cv.res_index(j, 2, kv, b, h, t);
+  // residual row of every level: one row per position (consecutive levels a
+  // fixed stride apart), or with sparse storage the pool row from the index
+  // (all index loads first), -1 for none
+  const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * cv.pool_rows();   // rows between loops
+  size_t ridx_lv[KM - 1];
+  bool have[KM - 1];
+  if (!cv.rows) {
+    const size_t r0 = cv.res_index(j, 2, kv, b, h, t);
+#pragma unroll
+    for (int q = 0; q < KM - 1; ++q) {
+      ridx_lv[q] = r0 + q * step;
+      have[q] = q + 2 <= m_hi;
+    }
+  } else {
+    int rr[KM - 1];
+#pragma unroll
+    for (int q = 0; q < KM - 1; ++q) rr[q] = q + 2 <= m_hi ? cv.res_row(j, q + 2, b, t) : -1;
+#pragma unroll
+    for (int q = 0; q < KM - 1; ++q) {
+      have[q] = rr[q] >= 0;
+      ridx_lv[q] = have[q] ? cv.res_index(j, q + 2, kv, b, h, rr[q]) : 0;
+    }
+  }
   uint32_t craw[KM - 1];
   uint16_t sraw[KM - 1];
 #pragma unroll
   for (int q = 0; q < KM - 1; ++q) {
     craw[q] = 0u;
     sraw[q] = 0;
-    if (q + 2 <= m_hi) {
-      const uint8_t* row = cv.codes + (r0 + q * step) * rb;
+    if (have[q]) {
+      const size_t ri = ridx_lv[q];
+      const uint8_t* row = cv.codes + ri * rb;
       if (EPL == 4) {
         craw[q] = cv.bits == 4 ? static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(row + lane * 2))
                                : static_cast<uint32_t>(row[lane]);
@@ -169,7 +214,7 @@ __device__ __forceinline__ void chain_lane2(const CacheView& cv, int j, int kv, 
         craw[q] = cv.bits == 4 ? static_cast<uint32_t>(row[lane])
                                : static_cast<uint32_t>((row[lane >> 1] >> ((lane & 1) * 4)) & 0xF);
       }
-      sraw[q] = cv.scales[(r0 + q * step) * ns + gi];
+      sraw[q] = cv.scales[ri * ns + gi];
     }
   }
   float acc[EPL];

@@ -11,7 +11,7 @@
 namespace fl {
 
 // Error bits a kernel records in the context status word.
-enum : int { kErrWaitTimeout = 1, kErrBadIndex = 2 };
+enum : int { kErrWaitTimeout = 1, kErrBadIndex = 2, kErrCapacity = 4 };
 
 // A bounded wait gives up after this many SM clock cycles (about 1 s at
 // 1.9 GHz), records kErrWaitTimeout and lets the kernel return.
@@ -161,6 +161,13 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
 // Both are no-ops for a kernel launched without the attribute.
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// The GPU's global nanosecond timer (the same clock on every SM).
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
 
 // ---------------------------------------------------------------- misc
 __device__ __forceinline__ float warp_sum(float v) {

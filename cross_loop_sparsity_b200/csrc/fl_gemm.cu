@@ -106,118 +106,6 @@ __device__ __forceinline__ float epi_one(const GemmArgs& p, int row, int col, in
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 2, 128;" ::: "memory"); }
 
-// RoPE and the KV write of one GEMM row (token slot) cc of a QKV tile, in the
-// epilogue: the 128 epilogue threads hold the tile's 128 features (whole heads,
-// hd dividing 128), thread `row` feature tile_m * 128 + row with value x.  The
-// same arithmetic as the separate RoPE/KV kernel (k_qkv_post): rotate q and k
-// heads; write q (and q_last at loop 1 of the lazy path); store the bf16 K/V row
-// (dense, or the lazy base at loop 1, zeroing the residual rows of later loops),
-// or quantise its residual against the loop-(l-1) reconstruction.  Every thread
-// takes every barrier, whatever its head kind.  xs: 128 floats, gmax: 4 floats
-// of shared scratch.
-__device__ __forceinline__ void post_qkv(const GemmArgs& p, int row, int cc, int tile_m, float x, float* xs,
-                                         float* gmax, int lane) {
-  const QkvPostArgs& a = p.post;
-  const CacheView& cv = a.cv;
-  const int hd = a.hd, half = hd >> 1, lhd = hd == 128 ? 7 : 6;
-  const int f = tile_m * 128 + row;
-  const int hh = f >> lhd, d = f & (hd - 1);
-  const bool valid = cc < p.n_tok && f < p.n_feat;
-  // rotation partner (dimension d +- hd/2) through shared memory
-  xs[row] = x;
-  epi_bar();
-  const float y = xs[row ^ half];
-  epi_bar();
-  int tok = 0, b = 0, t = 0;
-  if (valid) {
-    tok = a.idx ? a.idx[cc] : cc;
-    b = a.seq[tok];
-    t = a.pos[tok];
-  }
-  const bool is_q = hh < a.H, is_v = hh >= a.H + a.Hkv;
-  if (valid && !is_v) {
-    const int ai = d & (half - 1);
-    const float cs = a.rope_cos[static_cast<size_t>(t) * half + ai];
-    const float sn = a.rope_sin[static_cast<size_t>(t) * half + ai];
-    x = d < half ? __fmaf_rn(x, cs, -__fmul_rn(y, sn)) : __fmaf_rn(x, cs, __fmul_rn(y, sn));   // as k_qkv_post
-  }
-  const int kv = is_v ? 1 : 0;
-  const int gk = is_v ? hh - a.H - a.Hkv : hh - a.H;
-  const bool quant = valid && !is_q && a.lazy && a.loop > 1;
-  const bool forced = a.forced_on && a.forced_on[0];
-  // residual against the loop-(l-1) reconstruction, and its group's absmax
-  // (a group of g = 2^lg dimensions is g/32 consecutive warps of the epilogue)
-  float r = 0.f;
-  if (quant && !forced) {
-    float pv = bf16_to_f(cv.base_row(a.j, kv, b, gk, t)[d]);
-    const int gi = d >> cv.lg;
-    for (int l2 = 2; l2 < a.loop; ++l2) {
-      const uint8_t* cr = cv.code_row(a.j, l2, kv, b, gk, t);
-      const int bitpos = d * cv.bits;
-      const int code = sext((cr[bitpos >> 3] >> (bitpos & 7)) & ((1 << cv.bits) - 1), cv.bits);
-      const float sc = half_bits_to_f(cv.scale_row(a.j, l2, kv, b, gk, t)[gi]);
-      pv = __fadd_rn(pv, __fmul_rn(static_cast<float>(code), sc));
-    }
-    r = __fsub_rn(x, pv);
-  }
-  float am = fabsf(r);
-  for (int o = 16; o > 0; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-  const int wq = row >> 5;   // the warp's 32-row quarter of the tile
-  if (lane == 0) gmax[wq] = am;
-  epi_bar();
-  {
-    const int gw = (1 << cv.lg) >> 5;   // warps per group (g >= 32)
-    const int w0 = (wq / gw) * gw;
-    float m = 0.f;
-    for (int w = w0; w < w0 + gw; ++w) m = fmaxf(m, gmax[w]);
-    am = m;
-  }
-  epi_bar();
-  if (!valid) return;
-  if (is_q) {
-    a.q_cur[(static_cast<size_t>(cc) * a.H + hh) * hd + d] = x;
-    if (a.lazy && a.loop == 1 && a.q_last) a.q_last[(static_cast<size_t>(tok) * a.H + hh) * hd + d] = x;
-    return;
-  }
-  if (!a.lazy || a.loop == 1) {
-    uint16_t* dst = a.lazy ? cv.base_row(a.j, kv, b, gk, t) : cv.dense_row(a.j, a.loop, kv, b, gk, t);
-    dst[d] = f_to_bf16(x);
-    if (a.lazy) {
-      const int rb = static_cast<int>(cv.row_bytes_codes()), ns = hd >> cv.lg;
-      for (int l = 2; l <= cv.K; ++l) {
-        if (d < rb) cv.code_row(a.j, l, kv, b, gk, t)[d] = 0;
-        if (d < ns) cv.scale_row(a.j, l, kv, b, gk, t)[d] = 0;
-      }
-    }
-    return;
-  }
-  int c;
-  uint16_t sh;
-  if (forced) {
-    // checks only: the caller's codes for this selection slot
-    const size_t fr = (((static_cast<size_t>(a.j) * (cv.K - 1) + (a.loop - 2)) * a.forced_ns + cc) * 2 + kv) *
-                          a.Hkv + gk;
-    c = a.forced_codes[fr * hd + d];
-    sh = a.forced_scales[fr * (hd >> cv.lg) + (d >> cv.lg)];
-  } else {
-    if (a.trace_kv && cc < a.trace_ns)
-      a.trace_kv[((((static_cast<size_t>(a.j) * (cv.K - 1) + (a.loop - 2)) * a.trace_ns + cc) * 2 + kv) * a.Hkv + gk) *
-                     hd + d] = x;
-    const int qm = (1 << (cv.bits - 1)) - 1;
-    sh = quant_scale(am, qm);
-    const float sc = half_bits_to_f(sh);
-    c = quant_code(r, sc, sc > 0.f ? rcp_approx(sc) : 0.f, qm);
-  }
-  // pack: two's complement fields, element order low bits first
-  uint8_t* crow = cv.code_row(a.j, a.loop, kv, b, gk, t);
-  const int per_byte = 8 / cv.bits, fm = (1 << cv.bits) - 1;
-  uint32_t byte = static_cast<uint32_t>(c & fm);
-  for (int e = 1; e < per_byte; ++e)
-    byte |= static_cast<uint32_t>(__shfl_down_sync(0xffffffffu, c, e) & fm) << (e * cv.bits);
-  if ((d & (per_byte - 1)) == 0) crow[d / per_byte] = static_cast<uint8_t>(byte);
-  if ((d & ((1 << cv.lg) - 1)) == 0) cv.scale_row(a.j, a.loop, kv, b, gk, t)[d >> cv.lg] = sh;
-}
-
 // The token operand of a swap-orientation GEMM with an input RMSNorm, built by
 // the four epilogue warps (t4 = 0..127) while the TMA producer streams only
 // weights.  For ring slot s of k-chunk i the BN x 64 bf16 tile is written in
@@ -439,6 +327,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
     const int q = warp & 3;
     const int row = q * 32 + lane;
     pdl_wait();
+    if (p.stamp_start && warp == 2 && lane == 0) atomicMin(p.stamp_start, globaltimer_ns());
     if (in_norm) {
       if (!build_tokens<BN, C::kStages, C::kStageBytes, C::kNA * kABytes>(
               p, smem, full, empty, tok_scale, reinterpret_cast<float*>(tail + 768), flags + 2, c0, nch,
@@ -553,12 +442,6 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
           v0s += pv0[q];
           v1s += pv1[q];
         }
-        if (p.post_on) {
-          // RoPE and the KV write of this token column (every epilogue thread takes part)
-          post_qkv(p, row, cc, tile_m, v0s, reinterpret_cast<float*>(tail + 768), reinterpret_cast<float*>(tail + 256),
-                   lane);
-          continue;
-        }
         const float hn = epi_one(p, row, cc, tile_m, v0s, v1s);
         if (p.ss_out) {
           // this tile's share of the token's sum of squares, in a fixed order
@@ -575,6 +458,7 @@ k_gemm_tc(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUte
   }
   tc_fence_before();
   __syncthreads();
+  if (p.stamp_end && threadIdx.x == 0) atomicMax(p.stamp_end, globaltimer_ns());
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
@@ -782,6 +666,7 @@ k_gemm_wide(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     const int q = warp & 3;
     const int row = q * 32 + lane;
     pdl_wait();
+    if (p.stamp_start && warp == 2 && lane == 0) atomicMin(p.stamp_start, globaltimer_ns());
     int tl = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
       const int b = tl & 1;
@@ -823,6 +708,7 @@ k_gemm_wide(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   }
   tc_fence_before();
   __syncthreads();
+  if (p.stamp_end && threadIdx.x == 0) atomicMax(p.stamp_end, globaltimer_ns());
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

@@ -6,38 +6,7 @@
 #include <cstdint>
 #include <string>
 
-#include "fl_cache.cuh"
-
 namespace fl {
-
-// RoPE and the KV write of freshly projected rows: the separate kernel
-// (k_qkv_post) takes these, and so does the QKV GEMM when it does the same work
-// in its epilogue.
-struct QkvPostArgs {
-  const float* qkv;   // [n][(H+2Hkv)*hd] fp32, GEMM row order
-  int ldq;
-  const int* idx;     // GEMM row -> call token (nullptr = identity)
-  int n;
-  const int* seq;     // call token -> sequence
-  const int* pos;     // call token -> position
-  int H, Hkv, hd;
-  const float* rope_cos;  // [max_ctx][hd/2]
-  const float* rope_sin;
-  CacheView cv;
-  int j, loop, lazy;
-  float* q_cur;       // [n][H][hd] GEMM order
-  float* q_last;      // [N][H][hd] token order (this layer), written at loop 1
-  const int* forced_on;           // forced residual codes (checks): [0] != 0 when on
-  const int8_t* forced_codes;     // [M][K-1][ns][2][Hkv][hd]
-  const uint16_t* forced_scales;  // [M][K-1][ns][2][Hkv][hd/g]
-  int forced_ns;                  // selection-slot stride ns
-  // checks only: the rotated fp32 K/V rows each lazy loop quantised,
-  // [M][K-1][trace_ns][2][Hkv][hd] by (layer, loop 2..K, selection slot, K/V,
-  // KV head); slots >= trace_ns are not written (nullptr: off)
-  float* trace_kv;
-  int trace_ns;
-};
-
 
 // ------------------------------------------------------------------ GEMM
 // D = A * B^T on tcgen05 (bf16 operands, fp32 accumulate in TMEM).  A and B
@@ -72,6 +41,11 @@ struct GemmArgs {
   int cluster;      // split-K through a (1,1,splits) cluster and distributed shared memory
                     // instead of global partials and tickets (splits <= kMaxClusterSplits)
   int* status;
+  // Launch timing (nullptr: off): the earliest time any CTA's dependency wait
+  // returned (atomicMin) and the time the last CTA finished (atomicMax), from
+  // the global nanosecond timer.
+  unsigned long long* stamp_start;
+  unsigned long long* stamp_end;
   // Sums of squares for the next RMSNorm, written by a residual epilogue of the
   // cluster split-K path: ss_out[tile_m * ss_ld + tok] = sum over the tile's
   // 128 features of the updated h[r_tok][feat]^2 (nullptr: not written).
@@ -81,12 +55,6 @@ struct GemmArgs {
   // memory from fp32 hidden rows instead of loaded by TMA:
   //   x[t][k] = bf16(h[r_t][k] * rsqrt(sum_p ss_in[p * ss_ld + t] / K + in_eps) * in_gain[k])
   // with r_t = in_idx ? in_idx[t] : t, p < ss_parts, and zero rows t >= n_tok.
-  // RoPE and the KV write in the epilogue (swap orientation, cluster split-K
-  // path, hd dividing 128): instead of storing fp32 rows, the epilogue rotates
-  // q and k, writes q (and q_last at loop 1 of the lazy path) and stores or
-  // quantises the K/V rows exactly as k_qkv_post does.
-  int post_on;
-  QkvPostArgs post;
   const float* in_h;   // nullptr: TMA operand
   const int* in_idx;
   const float* in_gain;

@@ -3,6 +3,7 @@
 // decode and prefill attention, delta-score column keys, sparse-column
 // correction, and the per-token change keys.  Method: "FlashLoop: Fast and
 // Memory-Efficient Looped Transformers via Lazy Updates" (abstract).
+#include <algorithm>
 #include <cooperative_groups.h>
 
 #include "fl_cache.cuh"
@@ -131,11 +132,11 @@ __device__ int block_topk(const float* __restrict__ keys, int n, int k, int32_t*
       }
     }
     __syncthreads();
-    // fold the histograms: thread t < 256 totals digit t
-    if (threadIdx.x < 256) {
+    // fold the histograms: thread t totals digits t, t + blockDim.x, ...
+    for (int dg = threadIdx.x; dg < 256; dg += blockDim.x) {
       int c = 0;
-      for (int ww = 0; ww < nh; ++ww) c += whist[ww * 256 + threadIdx.x];
-      wtot[threadIdx.x] = c;
+      for (int ww = 0; ww < nh; ++ww) c += whist[ww * 256 + dg];
+      wtot[dg] = c;
     }
     __syncthreads();
     if (w == 0) {
@@ -468,7 +469,7 @@ __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
     } else {
       *reinterpret_cast<uint32_t*>(dst) = f_to_bf16(x[0]) | (static_cast<uint32_t>(f_to_bf16(x[1])) << 16);
     }
-    if (a.lazy) {
+    if (a.lazy && !cv.rows) {   // (with sparse storage the selection marks unrecomputed rows instead)
       const int rb = static_cast<int>(cv.row_bytes_codes());
       const int ns = hd >> cv.lg;
       for (int l = 2; l <= cv.K; ++l) {
@@ -503,9 +504,11 @@ __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
     for (int e = 0; e < EPL; ++e) r[e] = __fsub_rn(x[e], prev[e]);
     s = quantize_lane<EPL>(r, cv.lg, cv.bits, c);
   }
-  store_lane_codes<EPL>(cv.code_row(a.j, a.loop, kv, b, gk, t), cv.bits, lane, c);
+  const int r = cv.res_row(a.j, a.loop, b, t);   // the pool row the selection gave this token
+  if (r < 0) return;                               // (no room: the selection recorded the overflow)
+  store_lane_codes<EPL>(cv.code_row(a.j, a.loop, kv, b, gk, r), cv.bits, lane, c);
   const int lgl = cv.lg - (EPL == 4 ? 2 : 1);   // log2 of the lanes per group
-  if ((lane & ((1 << lgl) - 1)) == 0) cv.scale_row(a.j, a.loop, kv, b, gk, t)[lane >> lgl] = s;
+  if ((lane & ((1 << lgl) - 1)) == 0) cv.scale_row(a.j, a.loop, kv, b, gk, r)[lane >> lgl] = s;
 }
 
 constexpr int kDecTile = 64;
@@ -600,7 +603,7 @@ __global__ void __launch_bounds__(128, 2) k_attn_decode(const __grid_constant__ 
   // first row of this (layer, loop, K/V, sequence, KV head) in the 2-D [rows][hd] view of the cache
   const size_t bh = static_cast<size_t>(b) * cv.Hkv + g;
   const size_t plane = static_cast<size_t>(cv.B) * cv.Hkv * cv.T;
-  const size_t rk = a.dense ? ((static_cast<size_t>(a.j) * cv.K + (a.loop - 1)) * 2) * plane + bh * cv.T
+  const size_t rk = a.dense ? ((static_cast<size_t>(a.j) * cv.K + cv.dense_slot(a.loop)) * 2) * plane + bh * cv.T
                             : (static_cast<size_t>(a.j) * 2) * plane + bh * cv.T;
   const int row_k = static_cast<int>(rk), row_v = static_cast<int>(rk + plane);
   __syncthreads();   // barrier initialisation visible to every thread
@@ -905,8 +908,11 @@ __global__ void __launch_bounds__(256) k_attn_prefill(const AttnPreArgs a) {
   const int T = a.T;
   const int r = tid >> 2, c4 = tid & 3;
   const int q0 = qb * BQ;
-  const int qpos = q0 + r;
+  const int qpos = q0 + r;   // query index within the chunk
   const CacheView& cv = a.cv;
+  // the chunk starts after the L positions the sequence already holds: query
+  // qpos sits at position L + qpos and sees keys 0 .. L + qpos
+  const int L = a.pos[static_cast<size_t>(b) * T];
 
   for (int e = tid; e < BQ * HD; e += 256) {
     const int rr = e / HD, dd = e % HD;
@@ -917,7 +923,7 @@ __global__ void __launch_bounds__(256) k_attn_prefill(const AttnPreArgs a) {
   float acc[DV];
 #pragma unroll
   for (int e = 0; e < DV; ++e) acc[e] = 0.f;
-  const int kt_end = min(T, q0 + BQ);
+  const int kt_end = L + min(T, q0 + BQ);
   for (int k0 = 0; k0 < kt_end; k0 += BK) {
     __syncthreads();
     constexpr int CH = HD / 8;
@@ -925,7 +931,7 @@ __global__ void __launch_bounds__(256) k_attn_prefill(const AttnPreArgs a) {
       const int rr = e / CH, cc = e % CH;
       const int kp = k0 + rr;
       uint4 ku = make_uint4(0, 0, 0, 0), vu = make_uint4(0, 0, 0, 0);
-      if (kp < T) {
+      if (kp < kt_end) {
         const uint16_t* kr = a.dense ? cv.dense_row(a.j, a.loop, 0, b, g, kp) : cv.base_row(a.j, 0, b, g, kp);
         const uint16_t* vr = a.dense ? cv.dense_row(a.j, a.loop, 1, b, g, kp) : cv.base_row(a.j, 1, b, g, kp);
         ku = *reinterpret_cast<const uint4*>(kr + cc * 8);
@@ -949,7 +955,7 @@ __global__ void __launch_bounds__(256) k_attn_prefill(const AttnPreArgs a) {
         const uint32_t u = *reinterpret_cast<const uint32_t*>(kr + e);
         dot += q[e] * bf16_to_f(u & 0xFFFF) + q[e + 1] * bf16_to_f(u >> 16);
       }
-      s[j] = (kp <= qpos && kp < T && qpos < T) ? dot * a.tau : -INFINITY;
+      s[j] = (kp <= L + qpos && qpos < T) ? dot * a.tau : -INFINITY;
       tmax = fmaxf(tmax, s[j]);
     }
     tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
@@ -995,23 +1001,265 @@ __global__ void __launch_bounds__(256) k_attn_prefill(const AttnPreArgs a) {
 }
 
 // ============================================================================
+// prefill causal attention on the tensor cores (loop 1 of the lazy path; every
+// loop of the dense baseline; the prelude / coda layers).  grid (ceil(T/64), H,
+// B), 128 threads: warp w owns queries q0 + 16w .. +15 of a 64-query tile, over
+// 64-key tiles of the sequence's cache (the context before a chunk, then the
+// chunk up to each query's own position).  K and V tiles arrive by TMA
+// (128-byte swizzle, 64-row boxes) in a ring of kPreStages.  S = tau * Q K^T
+// and O += P V are warp-level bf16 products with fp32 accumulation: Q and P are
+// carried as bf16 hi + lo pairs (two products into one accumulator, about 16
+// significant bits, as the fp32 kernel), P straight from the score registers
+// (the accumulator layout of two 8-key score tiles is the A-operand layout of
+// one 16-key step), V's fragments from ldmatrix with transposition.  The
+// online softmax runs on the score fragments; a row's statistics live in the
+// four threads of a quad.
+// ============================================================================
+constexpr int kPreStages = 3;
+constexpr int kDscoreSMs = 148;   // the Δscore grid: two CTAs per SM of the B200
+
+template <int HD>
+__global__ void __launch_bounds__(128, 2) k_attn_prefill_tc(const __grid_constant__ CUtensorMap kvmap,
+                                                            const AttnPreArgs a) {
+  constexpr int NB = HD / 64;                   // 128-byte boxes per cache row
+  constexpr int BOX_BYTES = 64 * 128;
+  constexpr int TILE_BYTES = NB * BOX_BYTES;    // K or V of one 64-key tile
+  constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  constexpr int KS = HD / 16;                   // k-steps of the score product
+  constexpr int NDT = HD / 8;                   // 8-dim output tiles per warp
+  extern __shared__ uint8_t sm_raw[];
+  uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t full[kPreStages];
+  __shared__ int flag;
+
+  pdl_trigger();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int qb = gridDim.x - 1 - blockIdx.x;    // the longest causal ranges start first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (a.H / a.Hkv);
+  const int T = a.T;
+  if (tid == 0) {
+    for (int st = 0; st < kPreStages; ++st) mbar_init(smem_u32(&full[st]), 1);
+    fence_mbar_init();
+    flag = 0;
+  }
+  pdl_wait();
+  const CacheView& cv = a.cv;
+  // the chunk starts after the L positions the sequence already holds: query
+  // t of the chunk sits at position L + t and sees keys 0 .. L + t
+  const int L = a.pos[static_cast<size_t>(b) * T];
+  const int q0 = qb * 64;
+  const int kt_end = L + min(T, q0 + 64);
+  const int ntiles = (kt_end + 63) / 64;
+  const size_t plane = static_cast<size_t>(cv.B) * cv.Hkv * cv.T;
+  const size_t bh = static_cast<size_t>(b) * cv.Hkv + g;
+  const size_t rk = a.dense ? ((static_cast<size_t>(a.j) * cv.K + cv.dense_slot(a.loop)) * 2) * plane + bh * cv.T
+                            : (static_cast<size_t>(a.j) * 2) * plane + bh * cv.T;
+  const int row_k = static_cast<int>(rk), row_v = static_cast<int>(rk + plane);
+  __syncthreads();
+  auto issue = [&](int u) {
+    const int st = u % kPreStages;
+    uint8_t* dst = ring + st * STAGE_BYTES;
+    const uint32_t fb = smem_u32(&full[st]);
+    mbar_arrive_expect_tx(fb, STAGE_BYTES);
+#pragma unroll
+    for (int bx = 0; bx < NB; ++bx) {
+      tma_load_2d(smem_u32(dst + bx * BOX_BYTES), &kvmap, fb, bx * 64, row_k + u * 64);
+      tma_load_2d(smem_u32(dst + TILE_BYTES + bx * BOX_BYTES), &kvmap, fb, bx * 64, row_v + u * 64);
+    }
+  };
+  if (tid == 0) {
+    tma_prefetch_desc(&kvmap);
+    for (int u = 0; u < kPreStages && u < ntiles; ++u) issue(u);
+  }
+  // Q fragments (A operand, rows = queries, k = dims), tau folded in, hi + lo
+  const int r0 = q0 + warp * 16 + (lane >> 2), r1 = r0 + 8;   // chunk-relative query indices
+  const int P0 = L + r0, P1 = L + r1;                          // their positions
+  uint32_t qh[KS][4], ql[KS][4];
+  {
+    const float* q0p = a.q_cur + ((static_cast<size_t>(b) * T + min(r0, T - 1)) * a.H + h) * HD;
+    const float* q1p = a.q_cur + ((static_cast<size_t>(b) * T + min(r1, T - 1)) * a.H + h) * HD;
+    const bool v0 = r0 < T, v1 = r1 < T;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      const int d = ks * 16 + 2 * (lane & 3);
+      float x[8];
+      x[0] = v0 ? q0p[d] : 0.f;     x[1] = v0 ? q0p[d + 1] : 0.f;
+      x[2] = v1 ? q1p[d] : 0.f;     x[3] = v1 ? q1p[d + 1] : 0.f;
+      x[4] = v0 ? q0p[d + 8] : 0.f; x[5] = v0 ? q0p[d + 9] : 0.f;
+      x[6] = v1 ? q1p[d + 8] : 0.f; x[7] = v1 ? q1p[d + 9] : 0.f;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        float h0, l0, h1, l1;
+        split_bf16(x[2 * r] * a.tau, h0, l0);
+        split_bf16(x[2 * r + 1] * a.tau, h1, l1);
+        qh[ks][r] = pack_bf16x2(h0, h1);
+        ql[ks][r] = pack_bf16x2(l0, l1);
+      }
+    }
+  }
+  float o[NDT][4];
+#pragma unroll
+  for (int n = 0; n < NDT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.f, 0.f};
+
+  int u_stop = ntiles;
+  for (int u = 0; u < ntiles; ++u) {
+    const int st = u % kPreStages;
+    if (tid == 0) flag = mbar_wait(smem_u32(&full[st]), (u / kPreStages) & 1, a.status) ? 0 : 1;
+    __syncthreads();
+    if (flag) {
+      u_stop = u;
+      break;
+    }
+    mbar_try_wait(smem_u32(&full[st]), (u / kPreStages) & 1);   // completed: acquire the tile for this thread
+    const uint32_t Kt = smem_u32(ring + st * STAGE_BYTES);
+    const uint32_t Vt = Kt + TILE_BYTES;
+    const int k0 = u * 64;
+    // ---- scores of this warp's 16 queries x 64 keys (8 tiles of 8 keys)
+    float sc[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+      for (int np = 0; np < 4; ++np) {
+        const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+        const int ch = 2 * ks + ((lane >> 3) & 1);   // 16-byte chunk (8 dims) of the key row
+        uint32_t kb[4];
+        ldsm_x4(Kt + (ch >> 3) * BOX_BYTES + key * 128 + (((ch & 7) ^ (key & 7)) << 4), kb);
+        mma_bf16_16816(sc[2 * np], qh[ks], kb[0], kb[1]);
+        mma_bf16_16816(sc[2 * np], ql[ks], kb[0], kb[1]);
+        mma_bf16_16816(sc[2 * np + 1], qh[ks], kb[2], kb[3]);
+        mma_bf16_16816(sc[2 * np + 1], ql[ks], kb[2], kb[3]);
+      }
+    }
+    // causal mask: key c is visible to the query at position P when c <= P
+    float tm[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = k0 + nt * 8 + 2 * (lane & 3) + e;
+        if (c > P0 || r0 >= T) sc[nt][e] = -INFINITY;
+        if (c > P1 || r1 >= T) sc[nt][2 + e] = -INFINITY;
+        tm[0] = fmaxf(tm[0], sc[nt][e]);
+        tm[1] = fmaxf(tm[1], sc[nt][2 + e]);
+      }
+    }
+    float alpha[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      tm[r] = fmaxf(tm[r], __shfl_xor_sync(0xffffffffu, tm[r], 1));
+      tm[r] = fmaxf(tm[r], __shfl_xor_sync(0xffffffffu, tm[r], 2));
+      const float mn = fmaxf(m_run[r], tm[r]);
+      alpha[r] = (m_run[r] == -INFINITY || mn == -INFINITY) ? (m_run[r] == -INFINITY ? 0.f : 1.f)
+                                                             : expf(m_run[r] - mn);
+      m_run[r] = mn;
+    }
+    float rs[2] = {0.f, 0.f};
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float mr = m_run[e >> 1];
+        const float pv = (sc[nt][e] == -INFINITY) ? 0.f : expf(sc[nt][e] - mr);
+        sc[nt][e] = pv;
+        rs[e >> 1] += pv;
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) l_part[r] = l_part[r] * alpha[r] + rs[r];
+#pragma unroll
+    for (int n = 0; n < NDT; ++n) {
+      o[n][0] *= alpha[0];
+      o[n][1] *= alpha[0];
+      o[n][2] *= alpha[1];
+      o[n][3] *= alpha[1];
+    }
+    // ---- O += P V over the tile's 64 keys (4 steps of 16); P as a bf16 hi + lo pair
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      uint32_t ph[4], pl[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float* src = sc[2 * kk + (r >> 1)] + 2 * (r & 1);   // (row, row+8) x (keys 0-7, 8-15)
+        float h0, l0, h1, l1;
+        split_bf16(src[0], h0, l0);
+        split_bf16(src[1], h1, l1);
+        ph[r] = pack_bf16x2(h0, h1);
+        pl[r] = pack_bf16x2(l0, l1);
+      }
+      const int vr = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;   // V row (key) this lane addresses
+#pragma unroll
+      for (int n2 = 0; n2 < NDT / 2; ++n2) {
+        const int ch = n2 * 2 + (lane >> 4);                          // 8-dim chunk
+        uint32_t vf[4];
+        ldsm_x4_t(Vt + (ch >> 3) * BOX_BYTES + vr * 128 + (((ch & 7) ^ (vr & 7)) << 4), vf);
+        mma_bf16_16816(o[2 * n2], ph, vf[0], vf[1]);
+        mma_bf16_16816(o[2 * n2], pl, vf[0], vf[1]);
+        mma_bf16_16816(o[2 * n2 + 1], ph, vf[2], vf[3]);
+        mma_bf16_16816(o[2 * n2 + 1], pl, vf[2], vf[3]);
+      }
+    }
+    __syncthreads();   // every warp is done with the slot
+    if (tid == 0 && u + kPreStages < ntiles) issue(u + kPreStages);
+  }
+  if (u_stop < ntiles) {
+    // a tile never arrived: let the copies still in flight land (bounded) before the CTA exits
+    if (tid == 0)
+      for (int u = u_stop; u < ntiles && u < u_stop + kPreStages; ++u)
+        mbar_wait(smem_u32(&full[u % kPreStages]), (u / kPreStages) & 1, nullptr);
+    __syncthreads();
+    return;
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 1);
+    l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 2);
+  }
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int qi = r ? r1 : r0;
+    if (qi >= T) continue;
+    const size_t tok = static_cast<size_t>(b) * T + qi;
+    const float inv = 1.f / l_part[r];
+#pragma unroll
+    for (int n = 0; n < NDT; ++n) {
+      const int d = n * 8 + 2 * (lane & 3);
+      const float o0 = o[n][2 * r] * inv, o1 = o[n][2 * r + 1] * inv;
+      if (a.o_state) *reinterpret_cast<float2*>(a.o_state + (tok * a.H + h) * HD + d) = make_float2(o0, o1);
+      *reinterpret_cast<uint32_t*>(a.o_bf16 + tok * a.H * HD + static_cast<size_t>(h) * HD + d) = pack_bf16x2(o0, o1);
+    }
+    if ((lane & 3) == 0 && a.lse_state) a.lse_state[tok * a.H + h] = m_run[r] + logf(l_part[r]);
+  }
+}
+
+// ============================================================================
 // per-call token bookkeeping
 // ============================================================================
 __global__ void k_setup_call(int N, int mode_decode, int T, int tiles_per_seq, int q_tile,
                              const int* __restrict__ seq_len, int* seq, int* pos, int* tile, int* last,
-                             int n_tiles, int* has_c) {
+                             int n_tiles, int* has_c, unsigned long long* stamps, int n_stamps) {
   pdl_trigger();
   pdl_wait();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (stamps)   // GEMM launch stamps of this call: starts to the largest value (atomicMin), ends to zero
+    for (int i = t; i < n_stamps; i += gridDim.x * blockDim.x) {
+      stamps[i] = ~0ULL;
+      stamps[n_stamps + i] = 0ULL;
+    }
   if (t < N) {
     if (mode_decode) {
       seq[t] = t;
       pos[t] = seq_len[t];
       tile[t] = t;
     } else {
+      // a prefill chunk continues each sequence after its current length; its
+      // query tiles count q_tile positions from the chunk's first token
       const int b = t / T, p = t % T;
       seq[t] = b;
-      pos[t] = p;
+      pos[t] = seq_len[b] + p;
       tile[t] = b * tiles_per_seq + p / q_tile;
     }
     last[t] = 1;
@@ -1019,11 +1267,11 @@ __global__ void k_setup_call(int N, int mode_decode, int T, int tiles_per_seq, i
   if (t < n_tiles) has_c[t] = 0;
 }
 
-__global__ void k_set_lens(int B, int* seq_len, int add, int value) {
+__global__ void k_set_lens(int B, int* seq_len, int add) {
   pdl_trigger();
   pdl_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
-  if (b < B) seq_len[b] = add ? seq_len[b] + 1 : value;
+  if (b < B) seq_len[b] += add;
 }
 
 __global__ void k_reset_lens(const LensArg a, int* seq_len) {
@@ -1031,6 +1279,34 @@ __global__ void k_reset_lens(const LensArg a, int* seq_len) {
   pdl_wait();
   const int b = blockIdx.x * blockDim.x + threadIdx.x;
   if (b < a.n) seq_len[b] = a.v[b];
+}
+
+// The state a token enters a loop with: h[r] += e (the loop embedding, when
+// given) + gamma * x[r] (input injection: x is the state that entered the
+// loop stack), r = idx ? idx[i] : i, for the loop's n token rows.
+__global__ void __launch_bounds__(256) k_loop_input(float* __restrict__ h, const int* __restrict__ idx, int n, int d,
+                                                    const float* __restrict__ e, float gamma,
+                                                    const float* __restrict__ x) {
+  pdl_trigger();
+  pdl_wait();
+  const int i = blockIdx.x;
+  if (i >= n) return;
+  const int r = idx ? idx[i] : i;
+  float* hr = h + static_cast<size_t>(r) * d;
+  const float* xr = x + static_cast<size_t>(r) * d;
+  for (int c = threadIdx.x * 4; c < d; c += blockDim.x * 4) {
+    float4 v = *reinterpret_cast<const float4*>(hr + c);
+    if (e) {
+      const float4 ev = *reinterpret_cast<const float4*>(e + c);
+      v.x += ev.x; v.y += ev.y; v.z += ev.z; v.w += ev.w;
+    }
+    if (gamma != 0.f) {
+      const float4 xv = *reinterpret_cast<const float4*>(xr + c);
+      v.x = __fmaf_rn(gamma, xv.x, v.x); v.y = __fmaf_rn(gamma, xv.y, v.y);
+      v.z = __fmaf_rn(gamma, xv.z, v.z); v.w = __fmaf_rn(gamma, xv.w, v.w);
+    }
+    *reinterpret_cast<float4*>(hr + c) = v;
+  }
 }
 
 // slot of each token in the selection (or -1), and the snapshot of selected rows
@@ -1159,6 +1435,91 @@ __global__ void __launch_bounds__(1024) k_plan_tiles(const int32_t* __restrict__
   block_plan(idx, n_sel, tile, has_c, plan);
 }
 
+// Sparse residual storage: the pool rows of one call token at lazy loop l, for
+// every layer.  A recomputed token gets row rcount[j][l][b] + rank, rank = its
+// position among the call's recomputed tokens of sequence b (they are taken in
+// position order); others get -1 (zero residual).  A row beyond the pool is not
+// given (-1) and kErrCapacity is recorded.  The counts grow afterwards
+// (rows_advance), once every token of the call has read them.
+__device__ __forceinline__ void rows_assign(const CacheView& cv, int l, int b, int p, int rank, int* status) {
+  for (int j = 0; j < cv.M; ++j) {
+    int r = -1;
+    if (rank >= 0) {
+      r = cv.rcount[(static_cast<size_t>(j) * (cv.K - 1) + (l - 2)) * cv.B + b] + rank;
+      if (r >= cv.rows) {
+        r = -1;
+        if (status) atomicOr(status, kErrCapacity);
+      }
+    }
+    cv.ridx[cv.ridx_index(j, l, b, p)] = r;
+  }
+}
+__device__ __forceinline__ void rows_advance(const CacheView& cv, int l, int b, int n_b) {
+  for (int j = 0; j < cv.M; ++j) {
+    int* rc = cv.rcount + (static_cast<size_t>(j) * (cv.K - 1) + (l - 2)) * cv.B + b;
+    *rc = min(cv.rows, *rc + n_b);
+  }
+}
+// first index i in the ascending array v[0..n) with v[i] >= key
+__device__ __forceinline__ int lower_bound_i(const int32_t* v, int n, int key) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (v[mid] < key) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// The same for calls too large for the one-CTA selection step: CTA b takes
+// sequence b's call tokens [b*Tc, (b+1)*Tc), whose selection slots (-1 when not
+// recomputed) are in sel_slot.
+__global__ void __launch_bounds__(1024) k_assign_rows(const CacheView cv, int loop, int Tc, const int* sel_slot,
+                                                      const int* pos, int* status) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int scan_buf[33];
+  __shared__ int base;
+  const int b = blockIdx.x;
+  if (threadIdx.x == 0) base = 0;
+  __syncthreads();
+  for (int t0 = 0; t0 < Tc; t0 += blockDim.x) {
+    const int t = b * Tc + t0 + threadIdx.x;
+    const int sel = (t0 + threadIdx.x < Tc && sel_slot[t] >= 0) ? 1 : 0;
+    int tot;
+    const int rank = base + block_exclusive_scan(sel, &tot, scan_buf);
+    if (t0 + threadIdx.x < Tc) rows_assign(cv, loop, b, pos[t], sel ? rank : -1, status);
+    __syncthreads();
+    if (threadIdx.x == 0) base += tot;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) rows_advance(cv, loop, b, base);
+}
+
+// After a length reset: a sequence's pool holds the rows of its positions below
+// the new length, taken in position order, so its count is one past the row of
+// the last recomputed position below it.  One warp per (layer, loop, sequence).
+__global__ void k_reset_rows(const CacheView cv, const int* seq_len) {
+  pdl_trigger();
+  pdl_wait();
+  const int w = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  const int n_pairs = cv.M * (cv.K - 1) * cv.B;
+  if (w >= n_pairs) return;
+  const int b = w % cv.B, jl = w / cv.B;
+  const int32_t* ri = cv.ridx + static_cast<size_t>(jl) * cv.B * cv.T + static_cast<size_t>(b) * cv.T;
+  int cnt = 0;
+  for (int p0 = seq_len[b] - 1; p0 >= 0; p0 -= 32) {
+    const int p = p0 - lane;
+    const int r = p >= 0 ? ri[p] : -1;
+    const unsigned hit = __ballot_sync(0xffffffffu, r >= 0);
+    if (hit) {
+      const int first = __ffs(hit) - 1;   // the lane nearest the top
+      cnt = __shfl_sync(0xffffffffu, r, first) + 1;
+      break;
+    }
+  }
+  if (lane == 0) cv.rcount[static_cast<size_t>(jl) * cv.B + b] = cnt;
+}
+
 // One lazy loop's token bookkeeping for a call of at most kSelectStepMax tokens
 // (decode, short prefills), in one CTA: the change keys of the previous loop
 // (against h_in after loop 1, against the selected rows' snapshot after a lazy
@@ -1224,12 +1585,19 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
     a.meta[i] = m;
   }
   for (int t = threadIdx.x; t < a.N; t += blockDim.x) {
-    int lo = 0, hi = a.n_sel;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (s_idx[mid] < t) lo = mid + 1; else hi = mid;
+    const int lo = lower_bound_i(s_idx, a.n_sel, t);
+    const int sl = (lo < a.n_sel && s_idx[lo] == t) ? lo : -1;
+    a.sel_slot[t] = sl;
+    if (a.cv.rows) {   // sparse residual storage: pool rows of this loop's recomputed tokens
+      const int Tc = a.N / a.B_call, b = t / Tc;
+      rows_assign(a.cv, a.loop, b, a.pos[t], sl >= 0 ? sl - lower_bound_i(s_idx, a.n_sel, b * Tc) : -1, a.status);
     }
-    a.sel_slot[t] = (lo < a.n_sel && s_idx[lo] == t) ? lo : -1;
+  }
+  if (a.cv.rows) {
+    __syncthreads();   // every token has read the counts
+    const int Tc = a.N / a.B_call;
+    for (int b = threadIdx.x; b < a.B_call; b += blockDim.x)
+      rows_advance(a.cv, a.loop, b, lower_bound_i(s_idx, a.n_sel, (b + 1) * Tc) - lower_bound_i(s_idx, a.n_sel, b * Tc));
   }
   // snapshot of the selected rows (and, if asked, their normalised bf16 copy).
   // Work items are 512-element slices of a row, one per warp at a time; a
@@ -1301,6 +1669,46 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
   block_plan(s_idx, a.n_sel, s_tile, s_hasc, a.plan);
 }
 
+// The column set of one (tile, KV head) row from its n <= kSelColsSmemKeys keys
+// (staged in keys_sm), or the forced set: top-c by (bit pattern desc, column
+// asc), ascending.  Every thread of the CTA takes part.
+__device__ void select_row(const SelColsArgs& a, int seg, int g, int tl, int n, float* keys_sm) {
+  int32_t* out = a.cols + ((static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g) * a.c;
+  int* nout = a.ncols + (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
+  if (a.forced_on && (a.forced_on[0] & kForceCols)) {
+    const size_t off = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
+    const int fn = a.forced_ncols[off];
+    for (int e = threadIdx.x; e < fn; e += blockDim.x) out[e] = a.forced_cols[off * a.c + e];
+    if (threadIdx.x == 0) *nout = fn;
+    return;
+  }
+  const float* keys = a.col_keys + (static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols;
+  for (int e = threadIdx.x; e < n; e += blockDim.x) keys_sm[e] = __ldcg(keys + e);
+  __syncthreads();
+  const int got = block_topk(keys_sm, n, a.c, out);
+  if (threadIdx.x == 0) *nout = got;
+}
+
+// After a delta-score item: the CTA that wrote the last chunk of its row (an
+// atomic ticket over the row's chunks, no waiting) selects the row's column
+// set, so the selection needs no launch of its own.
+__device__ __forceinline__ void fold_select(const DScoreArgs& a, int seg, int g, int tl, int n, float* keys_sm,
+                                            int* last_flag) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int nch = (n + 63) / 64;
+    const int old = atomicAdd(&a.row_tickets[seg * a.Hkv + g], 1);
+    *last_flag = old == nch - 1;
+  }
+  __syncthreads();
+  if (!*last_flag) return;
+  __threadfence();
+  select_row(a.sel, seg, g, tl, n, keys_sm);
+  if (threadIdx.x == 0) a.row_tickets[seg * a.Hkv + g] = 0;
+  __syncthreads();
+}
+
 // ============================================================================
 // delta-score column keys of tiles recomputed for the first time:
 //   key[k] = max over the tile's selected queries i (with k <= pos(i)) and the
@@ -1321,15 +1729,21 @@ __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
   float* Qo = Qn + QP * HD;                      // [QP][HD]
   float* Mx = Qo + QP * HD;                      // [4][CC]
   __shared__ int Qpos[QP];                       // position of each staged pair's query
+  __shared__ int fold_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int seg = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
-  const int cnt = a.plan.counts[1], p = a.plan.need[seg];   // requested together
-  if (seg >= cnt) return;
+  // work items (tile needing a set, KV head, 64-column chunk), taken grid-stride
+  // by a grid sized to the GPU, so a loop whose tiles all have their sets
+  // (every lazy loop after the first, mostly) costs one launch, not a grid of
+  // empty CTAs sized for the longest row
+  const int cnt = a.plan.counts[1];
+  for (int it = blockIdx.x; it < cnt * a.Hkv * a.max_chunks; it += gridDim.x) {
+  const int seg = it / (a.Hkv * a.max_chunks), g = (it / a.max_chunks) % a.Hkv, chunk = it % a.max_chunks;
+  const int p = a.plan.need[seg];
   const int qb = a.plan.qb[p], qe = a.plan.qe[p];
   const SelMeta ml = a.meta[qe - 1];
   const int b = ml.seq, maxpos = ml.pos;
-  const int c0 = blockIdx.y * CC;
-  if (c0 > maxpos) return;
+  const int c0 = chunk * CC;
+  if (c0 > maxpos) continue;   // (uniform over the CTA)
   const int nc = min(CC, maxpos + 1 - c0);
   const int grp = a.H / a.Hkv;
   const CacheView& cv = a.cv;
@@ -1395,21 +1809,197 @@ __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
     if (a.trace_ck && tl < a.trace_tiles)
       a.trace_ck[((static_cast<size_t>(a.j) * a.trace_tiles + tl) * a.Hkv + g) * a.max_cols + c0 + tid] = v;
   }
+  __syncthreads();   // the staged rows and Mx are reused by the next item
+  if (a.fold) fold_select(a, seg, g, a.plan.tile[p], maxpos + 1, reinterpret_cast<float*>(sm), &fold_last);
+  }
 }
 
-// top-c columns of each (tile, KV head) that needs a column set
+// ============================================================================
+// delta-score column keys of prefill tiles on the tensor cores.  The same keys
+// as k_dscore -- key[k] = max over the tile's selected queries (k <= their
+// position) and the group's heads of |tau (q_l . K_l[k] - q_last . K_base[k])|
+// -- with the products as warp-level bf16 MMAs with fp32 accumulation.  At a
+// tile's first recomputation every member was last computed at loop 1, so the
+// old keys are the bf16 base exactly; the new keys (base + residuals, fp32) are
+// split into bf16 hi + lo, the queries too, and the difference accumulates in
+// one register set:  Qh Kh + Ql Kh + Qh Kl - Qoh Kb - Qol Kb  (the Ql Kl term,
+// below 2^-16 relative, is dropped).  Items (tile, KV head, 64-column chunk)
+// are taken grid-stride; a CTA's 4 warps take 16 (query, head) rows each, 64
+// rows per pass, and their column maxima meet in shared memory (max of
+// non-negative floats = max of their bit patterns, in any order).
+// ============================================================================
+template <int HD, int KM>
+__global__ void __launch_bounds__(128) k_dscore_tc(const DScoreArgs a) {
+  static_assert(HD == 128, "the staging gives each lane four dims of a 128-dim row");
+  pdl_trigger();
+  pdl_wait();
+  constexpr int CC = 64, BOX = 64 * 128, NB = HD / 64, TILE = NB * BOX, KS = HD / 16;
+  extern __shared__ uint8_t sm_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* knh = sm;   // new keys (hi, lo) and the base keys, one 64 x HD bf16 tile each
+
+  uint8_t* knl = sm + TILE;
+  uint8_t* kbs = sm + 2 * TILE;
+  __shared__ unsigned colmax[CC];
+  __shared__ int fold_last;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int grp = a.H / a.Hkv;
+  const int cnt = a.plan.counts[1];
+  const CacheView& cv = a.cv;
+  for (int it = blockIdx.x; it < cnt * a.Hkv * a.max_chunks; it += gridDim.x) {
+    const int seg = it / (a.Hkv * a.max_chunks), g = (it / a.max_chunks) % a.Hkv, chunk = it % a.max_chunks;
+    const int p = a.plan.need[seg];
+    const int qb = a.plan.qb[p], qe = a.plan.qe[p];
+    const SelMeta ml = a.meta[qe - 1];
+    const int b = ml.seq, maxpos = ml.pos;
+    const int c0 = chunk * CC;
+    if (c0 > maxpos) continue;   // (uniform over the CTA)
+    const int nc = min(CC, maxpos + 1 - c0);
+    if (tid < CC) colmax[tid] = 0u;
+    // stage the chunk's keys: row r = column c0 + r, 16-byte chunk ch at
+    // (ch / 8) * BOX + r * 128 + ((ch % 8) ^ (r % 8)) * 16 (the 128-byte swizzle)
+    {
+      constexpr int RW = CC / 4;   // rows per warp
+      for (int u = 0; u < RW; ++u) {
+        const int rr = warp * RW + u;
+        float lo[4], hi[4];
+        if (rr < nc) {
+          chain_lane2<4, KM>(cv, a.j, 0, b, g, c0 + rr, 1, a.loop, lane, lo, hi);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) lo[e] = hi[e] = 0.f;
+        }
+        // lane holds dims 4*lane .. +3: 8 bytes of a 16-byte chunk
+        const int ch = lane >> 1;
+        const uint32_t off = (ch >> 3) * BOX + rr * 128 + ((((ch & 7) ^ (rr & 7)) << 4) | ((lane & 1) << 3));
+        float h[4], l[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split_bf16(hi[e], h[e], l[e]);
+        *reinterpret_cast<uint2*>(knh + off) = make_uint2(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]));
+        *reinterpret_cast<uint2*>(knl + off) = make_uint2(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]));
+        *reinterpret_cast<uint2*>(kbs + off) = make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
+      }
+    }
+    __syncthreads();
+    const int npairs = (qe - qb) * grp;
+    for (int pb = 0; pb < npairs; pb += 64) {
+      // this warp's 16 (query, head) rows: r0 = lane/4, r1 = r0 + 8
+      int qpos[2];
+      uint32_t qnh[KS][4], qnl[KS][4], qoh[KS][4], qol[KS][4];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int pr = pb + warp * 16 + (lane >> 2) + 8 * r;
+        qpos[r] = -1;
+        if (pr < npairs) qpos[r] = a.meta[qb + pr / grp].pos;
+      }
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        float xn[8], xo[8];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int pr = min(pb + warp * 16 + (lane >> 2) + 8 * r, npairs - 1);
+          const int qi = qb + pr / grp, hh = g * grp + pr % grp;
+          const float* qn = a.q_cur + (static_cast<size_t>(qi) * a.H + hh) * HD;
+          const float* qo = a.q_last + (static_cast<size_t>(a.meta[qi].tok) * a.H + hh) * HD;
+          const int d = ks * 16 + 2 * (lane & 3);
+          const bool v = qpos[r] >= 0;
+          // A fragment order: (r0, d), (r1, d), (r0, d+8), (r1, d+8), two values each
+          xn[2 * r] = v ? qn[d] * a.tau : 0.f;         xn[2 * r + 1] = v ? qn[d + 1] * a.tau : 0.f;
+          xn[4 + 2 * r] = v ? qn[d + 8] * a.tau : 0.f; xn[4 + 2 * r + 1] = v ? qn[d + 9] * a.tau : 0.f;
+          xo[2 * r] = v ? -qo[d] * a.tau : 0.f;         xo[2 * r + 1] = v ? -qo[d + 1] * a.tau : 0.f;
+          xo[4 + 2 * r] = v ? -qo[d + 8] * a.tau : 0.f; xo[4 + 2 * r + 1] = v ? -qo[d + 9] * a.tau : 0.f;
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          float h0, l0, h1, l1;
+          split_bf16(xn[2 * r], h0, l0);
+          split_bf16(xn[2 * r + 1], h1, l1);
+          qnh[ks][r] = pack_bf16x2(h0, h1);
+          qnl[ks][r] = pack_bf16x2(l0, l1);
+          split_bf16(xo[2 * r], h0, l0);
+          split_bf16(xo[2 * r + 1], h1, l1);
+          qoh[ks][r] = pack_bf16x2(h0, h1);
+          qol[ks][r] = pack_bf16x2(l0, l1);
+        }
+      }
+      float acc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const int ch = 2 * ks + ((lane >> 3) & 1);
+          const uint32_t off = (ch >> 3) * BOX + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
+          uint32_t fh[4], fl[4], fb[4];
+          ldsm_x4(smem_u32(knh) + off, fh);
+          ldsm_x4(smem_u32(knl) + off, fl);
+          ldsm_x4(smem_u32(kbs) + off, fb);
+#pragma unroll
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            float* c = acc[2 * np + hlf];
+            mma_bf16_16816(c, qnh[ks], fh[2 * hlf], fh[2 * hlf + 1]);
+            mma_bf16_16816(c, qnl[ks], fh[2 * hlf], fh[2 * hlf + 1]);
+            mma_bf16_16816(c, qnh[ks], fl[2 * hlf], fl[2 * hlf + 1]);
+            mma_bf16_16816(c, qoh[ks], fb[2 * hlf], fb[2 * hlf + 1]);
+            mma_bf16_16816(c, qol[ks], fb[2 * hlf], fb[2 * hlf + 1]);
+          }
+        }
+      }
+      // |delta| of causal columns, max over this warp's rows, then over the CTA
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int col = nt * 8 + 2 * (lane & 3) + e;
+          float m = 0.f;
+          if (c0 + col <= qpos[0]) m = fmaxf(m, fabsf(acc[nt][e]));
+          if (c0 + col <= qpos[1]) m = fmaxf(m, fabsf(acc[nt][2 + e]));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+          if (lane < 4 && m > 0.f) atomicMax(&colmax[col], __float_as_uint(m));
+        }
+      }
+    }
+    __syncthreads();
+    if (tid < nc) {
+      const float v = __uint_as_float(colmax[tid]);
+      a.col_keys[(static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols + c0 + tid] = v;
+      const int tl = a.plan.tile[p];
+      if (a.trace_ck && tl < a.trace_tiles)
+        a.trace_ck[((static_cast<size_t>(a.j) * a.trace_tiles + tl) * a.Hkv + g) * a.max_cols + c0 + tid] = v;
+    }
+    __syncthreads();   // the staged keys and colmax are reused by the next item
+    if (a.fold) fold_select(a, seg, g, a.plan.tile[p], maxpos + 1, reinterpret_cast<float*>(sm), &fold_last);
+  }
+}
+
+// top-c columns of each (tile, KV head) that needs a column set.  A row of n
+// keys is split into slices of kSelColsSmemKeys (grid.y); the radix passes read
+// every key several times, so each slice is staged in shared memory once.  One
+// slice: its top-c is the answer.  Several: each slice writes its own top-c
+// (keys and ascending column ids) as candidates, and the last slice CTA of the
+// row (an atomic ticket, no waiting) takes the top-c of the candidates, laid
+// out in ascending column order: every member of the row's top-c is in its
+// slice's top-c, and equal keys still go to the lower column.
 __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
   pdl_trigger();
   pdl_wait();
-  extern __shared__ float keys_sm[];   // [min(max_cols, kSelColsSmemKeys)]
-  const int seg = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv;
+  extern __shared__ float keys_sm[];   // [kSelColsSmemKeys]
+  __shared__ int last_cta;
+  const int seg = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv, sl = blockIdx.y;
   const int cnt = a.plan.counts[1], p = a.plan.need[seg];   // requested together
   if (seg >= cnt) return;
   const int tl = a.plan.tile[p];
   const int n = a.meta[a.plan.qe[p] - 1].pos + 1;
+  const int slices = select_cols_slices(n);
+  if (sl >= slices) return;
   int32_t* out = a.cols + ((static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g) * a.c;
   int* nout = a.ncols + (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
   if (a.forced_on && (a.forced_on[0] & kForceCols)) {
+    if (sl != 0) return;
     const size_t off = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
     const int fn = a.forced_ncols[off];
     for (int e = threadIdx.x; e < fn; e += blockDim.x) out[e] = a.forced_cols[off * a.c + e];
@@ -1417,12 +2007,55 @@ __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
     return;
   }
   const float* keys = a.col_keys + (static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols;
-  if (n <= kSelColsSmemKeys) {   // the radix passes read every key several times: stage them once
-    stage_keys(keys, n, keys_sm);
-    keys = keys_sm;
+  if (slices == 1) {
+    select_row(a, seg, g, tl, n, keys_sm);
+    return;
   }
-  const int got = block_topk(keys, n, a.c, out);
-  if (threadIdx.x == 0) *nout = got;
+  // this slice's own top-c, as candidates
+  const int k0 = sl * kSelColsSmemKeys, ns = min(kSelColsSmemKeys, n - k0);
+  const size_t row = static_cast<size_t>(seg) * a.Hkv + g;
+  float* ck = a.cand_keys + (row * a.max_slices + sl) * a.c;
+  int32_t* ci = a.cand_idx + (row * a.max_slices + sl) * a.c;
+  stage_keys(keys + k0, ns, keys_sm);
+  const int kept = block_topk(keys_sm, ns, a.c, ci);   // slice positions, ascending
+  for (int e = threadIdx.x; e < kept; e += blockDim.x) {
+    const int q = ci[e];
+    ck[e] = keys_sm[q];
+    ci[e] = k0 + q;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int old = atomicAdd(&a.cand_counters[row], 1);
+    last_cta = old == slices - 1;
+  }
+  __syncthreads();
+  if (!last_cta) return;
+  __threadfence();
+  // the union, in slice order (= ascending column ids): every slice but the
+  // last kept c candidates (c < kSelColsSmemKeys), so the union is contiguous
+  const float* cand = a.cand_keys + row * a.max_slices * a.c;
+  const int m = (slices - 1) * a.c + min(a.c, n - (slices - 1) * kSelColsSmemKeys);
+  const float* src = cand;
+  if (m <= kSelColsSmemKeys) {
+    for (int e = threadIdx.x; e < m; e += blockDim.x) keys_sm[e] = __ldcg(cand + e);
+    __syncthreads();
+    src = keys_sm;
+  }
+  const int got = block_topk(src, m, a.c, out);   // positions among the candidates, ascending
+  // map positions to column ids (out is rewritten in place, in chunks of 1024)
+  for (int e0 = 0; e0 < got; e0 += 1024) {
+    const int e = e0 + threadIdx.x;
+    int col = 0;
+    if (e < got) col = __ldcg(a.cand_idx + row * a.max_slices * a.c + out[e]);
+    __syncthreads();
+    if (e < got) out[e] = col;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    *nout = got;
+    a.cand_counters[row] = 0;
+  }
 }
 
 // ============================================================================
@@ -1790,11 +2423,104 @@ __global__ void k_pack_codes(const int8_t* __restrict__ src, int rows, int hd, i
   store_lane_codes<EPL>(dst + static_cast<size_t>(w) * dst_row_stride, bits, lane, c);
 }
 
+// Sparse residual storage: one (layer, sequence) slice of an imported lazy
+// context.  CTA l-2 takes loop l: the positions whose codes or scales are not
+// all zero take pool rows in position order and their codes are packed into
+// them; the other positions get -1.  codes int8 [K-1][Hkv][n][hd], scales fp16
+// bits [K-1][Hkv][n][hd/g] (K, V).  A position beyond the pool records
+// kErrCapacity and keeps no row.
+__global__ void __launch_bounds__(256) k_import_rows(const CacheView cv, int j, int b, int n, const int8_t* ck,
+                                                     const int8_t* cvv, const uint16_t* sk, const uint16_t* sv,
+                                                     int* status) {
+  __shared__ int scan_buf[33];
+  __shared__ int base;
+  const int l = blockIdx.x + 2, hd = cv.hd, ns = hd >> cv.lg;
+  const size_t lrow = static_cast<size_t>(blockIdx.x) * cv.Hkv;   // [K-1][Hkv] row block of this loop
+  if (threadIdx.x == 0) base = 0;
+  __syncthreads();
+  for (int t0 = 0; t0 < n; t0 += blockDim.x) {
+    const int t = t0 + threadIdx.x;
+    int nz = 0;
+    if (t < n)
+      for (int kv = 0; kv < 2 && !nz; ++kv)
+        for (int h = 0; h < cv.Hkv && !nz; ++h) {
+          const size_t row = (lrow + h) * n + t;
+          const int8_t* c = (kv ? cvv : ck) + row * hd;
+          const uint16_t* sc = (kv ? sv : sk) + row * ns;
+          for (int e = 0; e < hd && !nz; ++e) nz = c[e] != 0;
+          for (int e = 0; e < ns && !nz; ++e) nz = sc[e] != 0;
+        }
+    int tot;
+    const int rank = base + block_exclusive_scan(nz, &tot, scan_buf);
+    if (t < n) {
+      int r = -1;
+      if (nz) {
+        r = rank;
+        if (r >= cv.rows) {
+          r = -1;
+          if (status) atomicOr(status, kErrCapacity);
+        }
+      }
+      cv.ridx[cv.ridx_index(j, l, b, t)] = r;
+      if (r >= 0)
+        for (int kv = 0; kv < 2; ++kv)
+          for (int h = 0; h < cv.Hkv; ++h) {
+            const size_t row = (lrow + h) * n + t;
+            const int8_t* c = (kv ? cvv : ck) + row * hd;
+            uint8_t* dst = cv.code_row(j, l, kv, b, h, r);
+            const int per = 8 / cv.bits, fm = (1 << cv.bits) - 1;
+            for (int o = 0; o < hd / per; ++o) {
+              uint32_t byte = 0;
+              for (int e = 0; e < per; ++e) byte |= static_cast<uint32_t>(c[o * per + e] & fm) << (e * cv.bits);
+              dst[o] = static_cast<uint8_t>(byte);
+            }
+            const uint16_t* sc = (kv ? sv : sk) + row * ns;
+            uint16_t* sd = cv.scale_row(j, l, kv, b, h, r);
+            for (int e = 0; e < ns; ++e) sd[e] = sc[e];
+          }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) base += tot;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) cv.rcount[(static_cast<size_t>(j) * (cv.K - 1) + (l - 2)) * cv.B + b] = min(base, cv.rows);
+}
+
+// Sparse residual storage: positions 0..n-1 of one (layer, loop, K/V, sequence)
+// as dense rows (zero where no row is kept): codes [Hkv][n][hd*b/8], scales
+// [Hkv][n][hd/g].  One thread per (head, position).
+__global__ void k_export_rows(const CacheView cv, int j, int l, int kv, int b, int n, uint8_t* codes,
+                              uint16_t* scales) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= cv.Hkv * n) return;
+  const int h = i / n, t = i % n;
+  const int rb = static_cast<int>(cv.row_bytes_codes()), ns = cv.hd >> cv.lg;
+  const int r = cv.ridx[cv.ridx_index(j, l, b, t)];
+  uint8_t* cd = codes + static_cast<size_t>(i) * rb;
+  uint16_t* sd = scales + static_cast<size_t>(i) * ns;
+  for (int o = 0; o < rb; ++o) cd[o] = r >= 0 ? cv.code_row(j, l, kv, b, h, r)[o] : 0;
+  for (int e = 0; e < ns; ++e) sd[e] = r >= 0 ? cv.scale_row(j, l, kv, b, h, r)[e] : 0;
+}
+
+cudaError_t launch_import_rows(const CacheView& cv, int j, int b, int n, const int8_t* ck, const int8_t* cvv,
+                               const uint16_t* sk, const uint16_t* sv, int* status, cudaStream_t s) {
+  return launch_k(false, k_import_rows, dim3(cv.K - 1), dim3(256), 0, s, cv, j, b, n, ck, cvv, sk, sv, status);
+}
+cudaError_t launch_export_rows(const CacheView& cv, int j, int l, int kv, int b, int n, uint8_t* codes,
+                               uint16_t* scales, cudaStream_t s) {
+  const int items = cv.Hkv * n;
+  return launch_k(false, k_export_rows, dim3((items + 255) / 256), dim3(256), 0, s, cv, j, l, kv, b, n, codes,
+                  scales);
+}
+
 // ============================================================================
 // launchers
 // ============================================================================
 thread_local bool g_pdl = false;
 void set_pdl(bool on) { g_pdl = on; }
+// prefill attention on the tensor-core kernel (1) or the fp32 SIMT one (0); thread-local
+thread_local bool kv_tc_prefill = true;
+void set_tc_prefill(bool on) { kv_tc_prefill = on; }
 
 cudaError_t launch_topk(const float* keys, int n_seg, int n, int k, int32_t* idx, cudaStream_t s) {
   const size_t sm = n <= kSelColsSmemKeys ? static_cast<size_t>(n) * 4 : 0;
@@ -1850,20 +2576,31 @@ cudaError_t launch_attn_decode(const CUtensorMap& kv, const AttnDecArgs& a, int 
 size_t attn_prefill_smem(int hd) {
   return static_cast<size_t>(64) * (hd + 1) * 4 + 64 * 65 * 4 + 2 * 64 * (hd + kDecPad) * 2;
 }
-cudaError_t launch_attn_prefill(const AttnPreArgs& a, int B, cudaStream_t s) {
+size_t attn_prefill_tc_smem(int hd) { return 1024 + static_cast<size_t>(kPreStages) * 2 * 64 * hd * 2; }
+cudaError_t launch_attn_prefill(const CUtensorMap& kv, const AttnPreArgs& a, int B, cudaStream_t s) {
   dim3 grid((a.T + 63) / 64, a.H, B);
+  if (kv_tc_prefill) {
+    const size_t sm = attn_prefill_tc_smem(a.hd);
+    if (a.hd == 128) return launch_k(g_pdl, k_attn_prefill_tc<128>, grid, dim3(128), sm, s, kv, a);
+    return launch_k(g_pdl, k_attn_prefill_tc<64>, grid, dim3(128), sm, s, kv, a);
+  }
   const size_t sm = attn_prefill_smem(a.hd);
   if (a.hd == 128) return launch_k(g_pdl, k_attn_prefill<128>, grid, dim3(256), sm, s, a);
   return launch_k(g_pdl, k_attn_prefill<64>, grid, dim3(256), sm, s, a);
 }
 cudaError_t launch_setup_call(int N, int decode, int T, int tiles_per_seq, int q_tile, const int* seq_len, int* seq,
-                              int* pos, int* tile, int* last, int n_tiles, int* has_c, cudaStream_t s) {
+                              int* pos, int* tile, int* last, int n_tiles, int* has_c, unsigned long long* stamps,
+                              int n_stamps, cudaStream_t s) {
   const int n = N > n_tiles ? N : n_tiles;
   return launch_k(g_pdl, k_setup_call, dim3((n + 255) / 256), dim3(256), 0, s, N, decode, T, tiles_per_seq, q_tile,
-                  seq_len, seq, pos, tile, last, n_tiles, has_c);
+                  seq_len, seq, pos, tile, last, n_tiles, has_c, stamps, n_stamps);
 }
-cudaError_t launch_set_lens(int B, int* seq_len, int add, int value, cudaStream_t s) {
-  return launch_k(g_pdl, k_set_lens, dim3((B + 127) / 128), dim3(128), 0, s, B, seq_len, add, value);
+cudaError_t launch_loop_input(float* h, const int* idx, int n, int d, const float* e, float gamma, const float* x,
+                              cudaStream_t s) {
+  return launch_k(g_pdl, k_loop_input, dim3(n), dim3(256), 0, s, h, idx, n, d, e, gamma, x);
+}
+cudaError_t launch_set_lens(int B, int* seq_len, int add, cudaStream_t s) {
+  return launch_k(g_pdl, k_set_lens, dim3((B + 127) / 128), dim3(128), 0, s, B, seq_len, add);
 }
 cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s) {
   return launch_k(false, k_reset_lens, dim3(1), dim3(kLensByValue), 0, s, a, seq_len);
@@ -1880,6 +2617,14 @@ cudaError_t launch_change_keys(const float* h, const float* ref, const int* sel_
   return launch_k(g_pdl, k_change_keys, dim3((N + 3) / 4), dim3(128), 0, s, h, ref, sel_slot, N, d, loop, key, last,
                   tile, has_c);
 }
+cudaError_t launch_assign_rows(const CacheView& cv, int loop, int B, int Tc, const int* sel_slot, const int* pos,
+                               int* status, cudaStream_t s) {
+  return launch_k(g_pdl, k_assign_rows, dim3(B), dim3(1024), 0, s, cv, loop, Tc, sel_slot, pos, status);
+}
+cudaError_t launch_reset_rows(const CacheView& cv, const int* seq_len, cudaStream_t s) {
+  const int warps = cv.M * (cv.K - 1) * cv.B;
+  return launch_k(false, k_reset_rows, dim3((warps + 7) / 8), dim3(256), 0, s, cv, seq_len);
+}
 cudaError_t launch_select_step(const SelectStepArgs& a, cudaStream_t s) {
   return launch_k(g_pdl, k_select_step, dim3(1), dim3(1024), 0, s, a);
 }
@@ -1887,16 +2632,33 @@ cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, co
                               cudaStream_t s) {
   return launch_k(g_pdl, k_plan_tiles, dim3(1), dim3(1024), 0, s, idx, n_sel, tile, has_c, p);
 }
+// (both also stage one row of column keys, up to kSelColsSmemKeys, for the folded selection)
+size_t dscore_tc_smem() { return std::max<size_t>(1024 + 3 * 64 * 128 * 2, kSelColsSmemKeys * 4 + 1024); }
 size_t dscore_smem(int hd) {
-  return (static_cast<size_t>(2) * 64 * (hd + 1) + 2 * 16 * hd + 4 * 64) * 4;
+  return std::max<size_t>((static_cast<size_t>(2) * 64 * (hd + 1) + 2 * 16 * hd + 4 * 64) * 4, kSelColsSmemKeys * 4);
 }
 cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s) {
-  dim3 grid(max_need * a.Hkv, max_chunks);
+  // grid-stride over (tile, KV head, chunk) items: at most two CTAs per SM
+  const int items = max_need * a.Hkv * max_chunks;
+  dim3 grid(items < 2 * kDscoreSMs ? items : 2 * kDscoreSMs);
   const size_t sm = dscore_smem(a.hd);
+  DScoreArgs b = a;
+  b.max_chunks = max_chunks;
+  if (a.tc && a.hd == 128) {   // prefill tiles: the tensor-core kernel, four CTAs per SM
+    const dim3 g4(items < 4 * kDscoreSMs ? items : 4 * kDscoreSMs);
+    const size_t smt = dscore_tc_smem();
+    switch (chain_km(a.cv.K)) {
+      case 2: return launch_k(g_pdl, k_dscore_tc<128, 2>, g4, dim3(128), smt, s, b);
+      case 4: return launch_k(g_pdl, k_dscore_tc<128, 4>, g4, dim3(128), smt, s, b);
+      case 8: return launch_k(g_pdl, k_dscore_tc<128, 8>, g4, dim3(128), smt, s, b);
+      case 16: return launch_k(g_pdl, k_dscore_tc<128, 16>, g4, dim3(128), smt, s, b);
+      default: return cudaErrorInvalidValue;
+    }
+  }
 #define FL_DS(KMv)                                                                           \
   case KMv:                                                                                  \
-    return a.hd == 128 ? launch_k(g_pdl, k_dscore<128, 4, KMv>, grid, dim3(256), sm, s, a)  \
-                       : launch_k(g_pdl, k_dscore<64, 2, KMv>, grid, dim3(256), sm, s, a);
+    return a.hd == 128 ? launch_k(g_pdl, k_dscore<128, 4, KMv>, grid, dim3(256), sm, s, b)  \
+                       : launch_k(g_pdl, k_dscore<64, 2, KMv>, grid, dim3(256), sm, s, b);
   switch (chain_km(a.cv.K)) {
     FL_DS(2)
     FL_DS(4)
@@ -1909,8 +2671,10 @@ cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cud
 size_t select_cols_smem(int max_cols) {
   return static_cast<size_t>(max_cols < kSelColsSmemKeys ? max_cols : kSelColsSmemKeys) * 4;
 }
-cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t s) {
-  return launch_k(g_pdl, k_select_cols, dim3(max_need * a.Hkv), dim3(1024), select_cols_smem(a.max_cols), s, a);
+cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, int max_cols_now, cudaStream_t s) {
+  const int slices = select_cols_slices(max_cols_now);
+  return launch_k(g_pdl, k_select_cols, dim3(max_need * a.Hkv, slices), dim3(1024),
+                  select_cols_smem(kSelColsSmemKeys), s, a);
 }
 size_t corr_cluster_smem(int hd, int grp) { return static_cast<size_t>(kCorrWarps) * grp * hd * 4; }
 template <typename K, typename A>
@@ -2013,6 +2777,12 @@ cudaError_t kernels_init_attrs() {
   set(k_topk_segments, static_cast<int>(select_cols_smem(kSelColsSmemKeys)));
   set(k_attn_prefill<128>, static_cast<int>(attn_prefill_smem(128)));
   set(k_attn_prefill<64>, static_cast<int>(attn_prefill_smem(64)));
+  set(k_attn_prefill_tc<128>, static_cast<int>(attn_prefill_tc_smem(128)));
+  set(k_attn_prefill_tc<64>, static_cast<int>(attn_prefill_tc_smem(64)));
+  set(k_dscore_tc<128, 2>, static_cast<int>(dscore_tc_smem()));
+  set(k_dscore_tc<128, 4>, static_cast<int>(dscore_tc_smem()));
+  set(k_dscore_tc<128, 8>, static_cast<int>(dscore_tc_smem()));
+  set(k_dscore_tc<128, 16>, static_cast<int>(dscore_tc_smem()));
   set(k_dscore<128, 4, 2>, static_cast<int>(dscore_smem(128)));
   set(k_dscore<128, 4, 4>, static_cast<int>(dscore_smem(128)));
   set(k_dscore<128, 4, 8>, static_cast<int>(dscore_smem(128)));

@@ -9,6 +9,32 @@
 
 namespace fl {
 
+// RoPE and the KV write of freshly projected rows (k_qkv_post).
+struct QkvPostArgs {
+  const float* qkv;   // [n][(H+2Hkv)*hd] fp32, GEMM row order
+  int ldq;
+  const int* idx;     // GEMM row -> call token (nullptr = identity)
+  int n;
+  const int* seq;     // call token -> sequence
+  const int* pos;     // call token -> position
+  int H, Hkv, hd;
+  const float* rope_cos;  // [max_ctx][hd/2]
+  const float* rope_sin;
+  CacheView cv;
+  int j, loop, lazy;
+  float* q_cur;       // [n][H][hd] GEMM order
+  float* q_last;      // [N][H][hd] token order (this layer), written at loop 1
+  const int* forced_on;           // forced residual codes (checks): [0] != 0 when on
+  const int8_t* forced_codes;     // [M][K-1][ns][2][Hkv][hd]
+  const uint16_t* forced_scales;  // [M][K-1][ns][2][Hkv][hd/g]
+  int forced_ns;                  // selection-slot stride ns
+  // checks only: the rotated fp32 K/V rows each lazy loop quantised,
+  // [M][K-1][trace_ns][2][Hkv][hd] by (layer, loop 2..K, selection slot, K/V,
+  // KV head); slots >= trace_ns are not written (nullptr: off)
+  float* trace_kv;
+  int trace_ns;
+};
+
 
 struct AttnDecArgs {
   const float* q_cur;
@@ -31,6 +57,7 @@ struct AttnDecArgs {
 
 struct AttnPreArgs {
   const float* q_cur;  // [B*T][H][hd] token order
+  const int* pos;      // [B*T] absolute position of each call token (chunk after the context)
   CacheView cv;
   int j, loop, dense;
   int T, H, Hkv, hd;
@@ -38,6 +65,7 @@ struct AttnPreArgs {
   float* o_state;
   float* lse_state;
   uint16_t* o_bf16;
+  int* status;         // error bits (a bounded wait that ran out)
 };
 
 struct TilePlan {
@@ -81,6 +109,31 @@ struct SelectStepArgs {
   uint16_t* x;
   int x_rows;
   float eps;
+  // sparse residual storage (cv.rows > 0): pool rows of the recomputed tokens
+  CacheView cv;
+  int B_call;            // sequences of the call (its N tokens are B_call runs of N / B_call)
+  int* status;
+};
+
+struct SelColsArgs {
+  TilePlan plan;
+  const int32_t* idx;
+  const int* pos;
+  const SelMeta* meta;  // [n_sel] per selected slot
+  const float* col_keys;
+  int max_cols, Hkv, c, j, n_tiles;
+  int32_t* cols;        // [M][n_tiles][Hkv][c]
+  int* ncols;           // [M][n_tiles][Hkv]
+  const int* forced_on;
+  const int32_t* forced_cols;
+  const int* forced_ncols;
+  // rows longer than kSelColsSmemKeys: each slice of kSelColsSmemKeys keys
+  // keeps its own top-c (grid.y = slices), the last slice CTA of a row (ticket)
+  // takes the top-c of their union
+  float* cand_keys;     // [max_need][Hkv][max_slices][c]
+  int32_t* cand_idx;    // [max_need][Hkv][max_slices][c] ascending global column ids
+  int* cand_counters;   // [max_need][Hkv], zero between launches
+  int max_slices;
 };
 
 struct DScoreArgs {
@@ -96,25 +149,20 @@ struct DScoreArgs {
   float tau;
   float* col_keys;      // [max_need][Hkv][max_cols]
   int max_cols;
+  int max_chunks;       // 64-column chunks of the longest row (set by the launcher)
+  int tc;               // 1: the tensor-core kernel (prefill tiles, head_dim 128)
+  // 1: the CTA finishing a row's last chunk also selects its column set (rows of
+  // at most kSelColsSmemKeys columns), with `sel`; row_tickets [max_need][Hkv]
+  // count finished chunks (zero between launches)
+  int fold;
+  SelColsArgs sel;
+  int* row_tickets;
   // checks only: every tile's keys by query tile, [M][trace_tiles][Hkv][max_cols]
   // (tiles >= trace_tiles are not written; nullptr: off)
   float* trace_ck;
   int trace_tiles;
 };
 
-struct SelColsArgs {
-  TilePlan plan;
-  const int32_t* idx;
-  const int* pos;
-  const SelMeta* meta;  // [n_sel] per selected slot
-  const float* col_keys;
-  int max_cols, Hkv, c, j, n_tiles;
-  int32_t* cols;        // [M][n_tiles][Hkv][c]
-  int* ncols;           // [M][n_tiles][Hkv]
-  const int* forced_on;
-  const int32_t* forced_cols;
-  const int* forced_ncols;
-};
 
 struct CorrectArgs {
   const int32_t* idx;
@@ -157,8 +205,8 @@ struct LensArg {
   int v[kLensByValue];
 };
 cudaError_t launch_reset_lens(const LensArg& a, int* seq_len, cudaStream_t s);
-constexpr int kCorrWarps = 16;
-constexpr int kSelColsSmemKeys = 16384;   // column keys the top-c kernel stages in shared memory (64 KB)   // warps per CTA of the clustered correction
+constexpr int kCorrWarps = 16;            // warps per CTA of the clustered correction
+constexpr int kSelColsSmemKeys = 16384;   // column keys the top-c selection stages in shared memory (64 KB)
 constexpr int kCorrCluster = 16;  // CTAs per (query, KV group) in the clustered correction (non-portable size)
 // Launches made while this is on (the kernels of one call) are programmatic
 // dependents of the previous kernel; thread-local.
@@ -172,10 +220,18 @@ cudaError_t launch_qkv_post(const QkvPostArgs& a, cudaStream_t s);
 // kv: the cache's bf16 rows ([rows][hd], 64 x 64 boxes, 128-byte swizzle) in
 // the layout the context uses (lazy base or dense per-loop)
 cudaError_t launch_attn_decode(const CUtensorMap& kv, const AttnDecArgs& a, int n, cudaStream_t s);
-cudaError_t launch_attn_prefill(const AttnPreArgs& a, int B, cudaStream_t s);
+// kv: the cache's bf16 rows ([rows][hd], 64 x 64 boxes, 128-byte swizzle), as for the decode attention
+cudaError_t launch_attn_prefill(const CUtensorMap& kv, const AttnPreArgs& a, int B, cudaStream_t s);
+// Prefill attention kernel choice for launches from this thread: tensor cores (default) or fp32 SIMT.
+void set_tc_prefill(bool on);
+// stamps (nullptr: none): the call's GEMM launch stamps [2][n_stamps], cleared here
 cudaError_t launch_setup_call(int N, int decode, int T, int tiles_per_seq, int q_tile, const int* seq_len, int* seq,
-                              int* pos, int* tile, int* last, int n_tiles, int* has_c, cudaStream_t s);
-cudaError_t launch_set_lens(int B, int* seq_len, int add, int value, cudaStream_t s);
+                              int* pos, int* tile, int* last, int n_tiles, int* has_c, unsigned long long* stamps,
+                              int n_stamps, cudaStream_t s);
+cudaError_t launch_set_lens(int B, int* seq_len, int add, cudaStream_t s);
+// h[r] += e + gamma * x[r] for the n rows r = idx ? idx[i] : i (e may be nullptr)
+cudaError_t launch_loop_input(float* h, const int* idx, int n, int d, const float* e, float gamma, const float* x,
+                              cudaStream_t s);
 // selection slots, snapshot of the selected rows and their SelMeta records
 // (the path for calls too large for the one-CTA selection step)
 cudaError_t launch_after_select(const int32_t* idx, int n_sel, int N, int d, int* sel_slot, const float* h,
@@ -184,10 +240,24 @@ cudaError_t launch_after_select(const int32_t* idx, int n_sel, int N, int d, int
 cudaError_t launch_change_keys(const float* h, const float* ref, const int* sel_slot, int N, int d, int loop,
                                float* key, int* last, const int* tile, int* has_c, cudaStream_t s);
 cudaError_t launch_select_step(const SelectStepArgs& a, cudaStream_t s);
+// sparse residual storage: pool rows of a lazy loop's recomputed tokens (calls
+// too large for the selection step), and the pool counts after a length reset
+cudaError_t launch_assign_rows(const CacheView& cv, int loop, int B, int Tc, const int* sel_slot, const int* pos,
+                               int* status, cudaStream_t s);
+cudaError_t launch_reset_rows(const CacheView& cv, const int* seq_len, cudaStream_t s);
+// sparse residual storage: import one (layer, sequence) slice of a lazy context
+// (int8 codes, fp16 scales by position), and export one (layer, loop, K/V,
+// sequence) slice back to packed rows by position
+cudaError_t launch_import_rows(const CacheView& cv, int j, int b, int n, const int8_t* ck, const int8_t* cvv,
+                               const uint16_t* sk, const uint16_t* sv, int* status, cudaStream_t s);
+cudaError_t launch_export_rows(const CacheView& cv, int j, int l, int kv, int b, int n, uint8_t* codes,
+                               uint16_t* scales, cudaStream_t s);
 cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, const int* has_c, const TilePlan& p,
                               cudaStream_t s);
 cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s);
-cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, cudaStream_t s);
+cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, int max_cols_now, cudaStream_t s);
+// slices of a row of column keys the top-c selection splits it into
+__host__ __device__ inline int select_cols_slices(int n) { return n <= kSelColsSmemKeys ? 1 : (n + kSelColsSmemKeys - 1) / kSelColsSmemKeys; }
 cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s);
 
 

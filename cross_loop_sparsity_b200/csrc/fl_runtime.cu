@@ -53,6 +53,11 @@ struct flashloop_ctx {
   int32_t* cols = nullptr;
   int* ncols = nullptr;
   float* col_keys = nullptr;
+  float* cand_keys = nullptr;     // slice candidates of long column-key rows
+  int32_t* cand_idx = nullptr;
+  int* cand_cnt = nullptr;
+  int* row_tickets = nullptr;     // finished chunks of each column-key row (the folded selection)
+  int max_slices = 1;
   int* forced_on = nullptr;
   int32_t *forced_sel = nullptr, *forced_cols = nullptr;
   int* forced_ncols = nullptr;
@@ -71,8 +76,12 @@ struct flashloop_ctx {
   SelMeta* sel_meta = nullptr;   // [N] records of the current loop's selected slots
   int ss_tiles = 0;
   float* logits_ws = nullptr;
+  // prelude / coda (independent layers, one-pass KV each) and loop-input variants
+  CacheView cvx{};            // their KV: dense layout with one loop slot, n_prelude + n_coda layers
   // descriptors
   CUtensorMap tm_qkv, tm_o, tm_gate, tm_up, tm_down, tm_out;
+  CUtensorMap tm_x_qkv[2], tm_x_o[2], tm_x_gate[2], tm_x_up[2], tm_x_down[2];   // prelude [0], coda [1]
+  CUtensorMap tm_kvx;         // the independent layers' KV rows for the decode attention
   CUtensorMap tm_x_a, tm_obf_a, tm_act_a;
   CUtensorMap tm_x_b[3], tm_obf_b[3], tm_act_b[3];
   CUtensorMap tm_kv;   // the cache's bf16 rows for the decode attention
@@ -84,7 +93,11 @@ struct flashloop_ctx {
   int use_graph = 1;
   int pdl = 1;                        // FL_OPT_PDL
   int prof = 0;                       // FL_OPT_PROFILE
-  int fuse_qkv = 0;                   // FL_OPT_FUSE_QKV
+  int gemm_times = 0;                 // FL_OPT_GEMM_TIMES
+  int tc_prefill = 1;                 // FL_OPT_TC_PREFILL
+  int corr_cluster = 1;               // FL_OPT_CORR_CLUSTER
+  unsigned long long* stamps = nullptr;   // [2][kMaxStamps]: launch start (min), end (max) per GEMM of a call
+  int stamp_slots = 0;                // GEMM launches of the last call (capped at kMaxStamps)
   std::vector<cudaEvent_t> ev;        // start/end pairs of the last profiled call
   std::vector<int> ev_kind;
   int ev_used = 0;
@@ -106,6 +119,7 @@ constexpr int kCorrColsSmall = 16, kCorrColsBig = 128, kCorrSmallQueries = 64;
 // Calls of at most this many tokens do a lazy loop's bookkeeping in one CTA.
 constexpr int kSsLd = 64;                // tokens per row of the sums-of-squares table (swap GEMMs: <= 64)
 constexpr int kCountersGemm = 4096;
+constexpr int kMaxStamps = 4096;         // GEMM launches of one call that are timed
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 int ceil_div(int a, int b) { return (a + b - 1) / b; }
@@ -137,6 +151,12 @@ bool valid_config(const flashloop_config* c) {
     if (c->group_size > c->head_dim || c->head_dim % c->group_size) return false;
     if (c->q_tile < 1) return false;
   }
+  if (c->n_prelude < 0 || c->n_coda < 0 || (c->loop_embed != 0 && c->loop_embed != 1)) return false;
+  if (!(c->inject_scale == c->inject_scale)) return false;   // NaN
+  if (c->resid_rows < 0 || c->resid_rows > c->max_ctx) return false;
+  if (c->resid_rows > 0 && c->resid_bits == 16) return false;   // a lazy-path layout
+  if (c->kv_mode != 0 && c->kv_mode != 1) return false;
+  if (c->kv_mode == 1 && c->resid_bits != 16) return false;   // last_loop is a dense-path KV mode
   if (c->vocab < 1 || c->max_batch < 1 || c->max_ctx < 1 || c->max_tokens < 0) return false;
   if (!(c->rms_eps > 0.f) || !(c->rope_theta > 0.f)) return false;
   return true;
@@ -147,6 +167,7 @@ bool valid_config(const flashloop_config* c) {
 size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   const int M = c.n_layers, K = c.n_loops, Hkv = c.n_kv_heads, H = c.n_heads, hd = c.head_dim, d = c.d_model;
   const bool lazy = c.resid_bits != 16;
+  const int KS = (!lazy && c.kv_mode == 1) ? 1 : K;   // KV loops stored by the dense path (last_loop: one)
   const size_t B = c.max_batch, T = c.max_ctx;
   const int N = c.max_tokens > c.max_batch ? c.max_tokens : c.max_batch;
   const int Npad = ceil_div(N > 64 ? N : 64, 128) * 128;
@@ -166,13 +187,23 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   // KV cache
   const size_t rows = static_cast<size_t>(M) * 2 * B * Hkv * T;
   uint8_t *base, *codes = nullptr, *scales = nullptr;
+  // residual rows per pool: every position, or (sparse storage) resid_rows
+  const size_t R = (lazy && c.resid_rows > 0) ? static_cast<size_t>(c.resid_rows) : T;
+  const size_t res_rows = static_cast<size_t>(M) * 2 * B * Hkv * R;
+  uint8_t *ridx = nullptr, *rcount = nullptr;
   if (lazy) {
     base = take(rows * hd * 2);
-    codes = take(rows * (K - 1) * (static_cast<size_t>(hd) * c.resid_bits / 8));
-    scales = take(rows * (K - 1) * (hd / c.group_size) * 2);
+    codes = take(res_rows * (K - 1) * (static_cast<size_t>(hd) * c.resid_bits / 8));
+    scales = take(res_rows * (K - 1) * (hd / c.group_size) * 2);
+    if (c.resid_rows > 0 && K > 1) {
+      ridx = take(static_cast<size_t>(M) * (K - 1) * B * T * 4);
+      rcount = take(static_cast<size_t>(M) * (K - 1) * B * 4);
+    }
   } else {
-    base = take(rows * K * hd * 2);
+    base = take(rows * KS * hd * 2);
   }
+  const int X = c.n_prelude + c.n_coda;
+  uint8_t* xkv = X ? take(static_cast<size_t>(X) * 2 * B * Hkv * T * hd * 2) : nullptr;
   uint8_t* rc = take(T * (hd / 2) * 4);
   uint8_t* rs = take(T * (hd / 2) * 4);
   uint8_t* seq_len = take(B * 4);
@@ -210,6 +241,13 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   uint8_t* cols = take(static_cast<size_t>(M) * n_tiles * Hkv * cc * 4);
   uint8_t* ncols = take(static_cast<size_t>(M) * n_tiles * Hkv * 4);
   uint8_t* col_keys = take(lazy ? static_cast<size_t>(max_need) * Hkv * T * 4 : 4);
+  // top-c candidates of the slices of column-key rows longer than one slice
+  const int max_slices = lazy ? select_cols_slices(c.max_ctx) : 1;
+  const size_t n_cand = max_slices > 1 ? static_cast<size_t>(max_need) * Hkv * max_slices * cc : 1;
+  uint8_t* cand_keys = take(n_cand * 4);
+  uint8_t* cand_idx = take(n_cand * 4);
+  uint8_t* cand_cnt = take(static_cast<size_t>(std::max(max_need, 1)) * Hkv * 4);
+  uint8_t* row_tk = take(static_cast<size_t>(std::max(max_need, 1)) * Hkv * 4);
   uint8_t* forced_on = take(16);
   uint8_t* forced_sel = take(static_cast<size_t>(K) * N * 4);
   uint8_t* forced_cols = take(static_cast<size_t>(M) * n_tiles * Hkv * cc * 4);
@@ -264,6 +302,7 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   uint8_t* smeta = take(static_cast<size_t>(N) * sizeof(SelMeta));
   uint8_t* ssp = take(static_cast<size_t>(ss_tiles) * kSsLd * 4);
   uint8_t* logits = take(B * c.vocab * 4);
+  uint8_t* stamps = take(2 * kMaxStamps * 8);
   if (x) {
     x->lazy = lazy;
     x->qkv_rows = qkv_rows;
@@ -272,13 +311,26 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->n_tiles_max = n_tiles;
     x->max_need = max_need;
     x->dec_splits = splits;
-    x->cv.M = M; x->cv.K = K; x->cv.B = c.max_batch; x->cv.Hkv = Hkv; x->cv.T = c.max_ctx; x->cv.hd = hd;
+    x->cv.M = M; x->cv.K = KS; x->cv.B = c.max_batch; x->cv.Hkv = Hkv; x->cv.T = c.max_ctx; x->cv.hd = hd;
     x->cv.g = lazy ? c.group_size : hd;
     x->cv.lg = 0;
     while ((1 << x->cv.lg) < x->cv.g) ++x->cv.lg;
     x->cv.bits = lazy ? c.resid_bits : 16;
     x->cv.dense = lazy ? 0 : 1;
     x->cv.base = reinterpret_cast<uint16_t*>(base);
+    x->cv.rows = ridx ? c.resid_rows : 0;
+    x->cv.ridx = reinterpret_cast<int32_t*>(ridx);
+    x->cv.rcount = reinterpret_cast<int*>(rcount);
+    x->cvx = x->cv;
+    x->cvx.rows = 0;
+    x->cvx.ridx = nullptr;
+    x->cvx.rcount = nullptr;
+    x->cvx.M = X; x->cvx.K = 1; x->cvx.g = hd; x->cvx.lg = x->cv.lg; x->cvx.bits = 16; x->cvx.dense = 1;
+    while ((1 << x->cvx.lg) < hd) ++x->cvx.lg;
+    while (x->cvx.lg > 0 && (1 << x->cvx.lg) > hd) --x->cvx.lg;
+    x->cvx.base = reinterpret_cast<uint16_t*>(xkv);
+    x->cvx.codes = nullptr;
+    x->cvx.scales = nullptr;
     x->cv.codes = codes;
     x->cv.scales = reinterpret_cast<uint16_t*>(scales);
     x->rope_cos = reinterpret_cast<float*>(rc);
@@ -315,6 +367,11 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->cols = reinterpret_cast<int32_t*>(cols);
     x->ncols = reinterpret_cast<int*>(ncols);
     x->col_keys = reinterpret_cast<float*>(col_keys);
+    x->cand_keys = reinterpret_cast<float*>(cand_keys);
+    x->cand_idx = reinterpret_cast<int32_t*>(cand_idx);
+    x->cand_cnt = reinterpret_cast<int*>(cand_cnt);
+    x->row_tickets = reinterpret_cast<int*>(row_tk);
+    x->max_slices = max_slices;
     x->forced_on = reinterpret_cast<int*>(forced_on);
     x->forced_sel = reinterpret_cast<int32_t*>(forced_sel);
     x->forced_cols = reinterpret_cast<int32_t*>(forced_cols);
@@ -336,6 +393,7 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->sel_meta = reinterpret_cast<SelMeta*>(smeta);
     x->ss_tiles = ss_tiles;
     x->logits_ws = reinterpret_cast<float*>(logits);
+    x->stamps = reinterpret_cast<unsigned long long*>(stamps);
   }
   return off;
 }
@@ -351,6 +409,21 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
 
 enum GemmOpKind { kOpQKV, kOpO, kOpGU, kOpDown, kOpOut };
 
+// One stack of layers' weights: the shared block, the prelude or the coda.
+struct StackW {
+  const CUtensorMap *qkv, *o, *gate, *up, *down;   // layer-stacked (rank-3) maps
+  const float *attn_norm, *mlp_norm;               // [layers][d]
+};
+StackW stack_w(const flashloop_ctx* ctx, int stack) {
+  if (stack == 0)
+    return StackW{&ctx->tm_qkv, &ctx->tm_o, &ctx->tm_gate, &ctx->tm_up, &ctx->tm_down, ctx->w.attn_norm,
+                  ctx->w.mlp_norm};
+  const int x = stack - 1;
+  const flashloop_layers& L = x == 0 ? ctx->w.prelude : ctx->w.coda;
+  return StackW{&ctx->tm_x_qkv[x], &ctx->tm_x_o[x], &ctx->tm_x_gate[x], &ctx->tm_x_up[x], &ctx->tm_x_down[x],
+                L.attn_norm, L.mlp_norm};
+}
+
 // RMSNorm of a GEMM's input rows built inside the GEMM from the fp32 hidden
 // state and the per-tile sums of squares the previous residual GEMM left.
 struct InNorm {
@@ -362,32 +435,30 @@ struct InNorm {
 // RMSNorm runs inside the GEMM (swap orientation only).  *ss_written (O and
 // down projections): whether the epilogue left the sums of squares of its
 // updated rows for the next norm (the cluster split-K path only).
-fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, cudaStream_t s,
-               const InNorm& in = InNorm{}, bool* ss_written = nullptr, const QkvPostArgs* post = nullptr,
-               bool* post_done = nullptr) {
+fl_status gemm(flashloop_ctx* ctx, const StackW& W, GemmOpKind op, int j, int n, const int* idx, cudaStream_t s,
+               const InNorm& in = InNorm{}, bool* ss_written = nullptr) {
   const flashloop_config& c = ctx->cfg;
   GemmLaunch g{};
   GemmArgs& a = g.args;
   if (ss_written) *ss_written = false;
-  if (post_done) *post_done = false;
   const CUtensorMap *w0 = nullptr, *w1 = nullptr, *xa = nullptr;
   const CUtensorMap* xb = nullptr;
   int feat = 0, K = 0;
   switch (op) {
     case kOpQKV:
-      w0 = &ctx->tm_qkv; feat = ctx->qkv_rows; K = c.d_model; xa = &ctx->tm_x_a; xb = ctx->tm_x_b;
+      w0 = W.qkv; feat = ctx->qkv_rows; K = c.d_model; xa = &ctx->tm_x_a; xb = ctx->tm_x_b;
       a.epi = kEpiStore; a.out = ctx->qkv; a.ldo = ctx->qkv_rows;
       break;
     case kOpO:
-      w0 = &ctx->tm_o; feat = c.d_model; K = c.n_heads * c.head_dim; xa = &ctx->tm_obf_a; xb = ctx->tm_obf_b;
+      w0 = W.o; feat = c.d_model; K = c.n_heads * c.head_dim; xa = &ctx->tm_obf_a; xb = ctx->tm_obf_b;
       a.epi = kEpiResid; a.h = ctx->h; a.idx = idx; a.scale = c.resid_scale; a.ldh = c.d_model;
       break;
     case kOpGU:
-      w0 = &ctx->tm_gate; w1 = &ctx->tm_up; feat = c.ffn_dim; K = c.d_model; xa = &ctx->tm_x_a; xb = ctx->tm_x_b;
+      w0 = W.gate; w1 = W.up; feat = c.ffn_dim; K = c.d_model; xa = &ctx->tm_x_a; xb = ctx->tm_x_b;
       a.epi = kEpiSwiglu; a.act = ctx->act; a.ld_act = c.ffn_dim;
       break;
     case kOpDown:
-      w0 = &ctx->tm_down; feat = c.d_model; K = c.ffn_dim; xa = &ctx->tm_act_a; xb = ctx->tm_act_b;
+      w0 = W.down; feat = c.d_model; K = c.ffn_dim; xa = &ctx->tm_act_a; xb = ctx->tm_act_b;
       a.epi = kEpiResid; a.h = ctx->h; a.idx = idx; a.scale = c.resid_scale; a.ldh = c.d_model;
       break;
     case kOpOut:
@@ -399,6 +470,11 @@ fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, 
   a.n_feat = feat;
   a.n_tok = n;
   a.status = ctx->status;
+  if (ctx->gemm_times && ctx->stamp_slots < kMaxStamps) {
+    a.stamp_start = ctx->stamps + ctx->stamp_slots;
+    a.stamp_end = ctx->stamps + kMaxStamps + ctx->stamp_slots;
+    ++ctx->stamp_slots;
+  }
   const int w3d = op != kOpOut;
   if (n <= 64) {
     const int bn = swap_bn(n);
@@ -422,12 +498,6 @@ fl_status gemm(flashloop_ctx* ctx, GemmOpKind op, int j, int n, const int* idx, 
     if (in.gain) {
       a.in_h = ctx->h; a.in_idx = in.idx; a.in_gain = in.gain; a.ss_in = ctx->ss_part; a.ss_ld = kSsLd;
       a.in_ld = K; a.ss_parts = ceil_div(K, 128); a.in_eps = c.rms_eps;
-    }
-    // RoPE and the KV write in the epilogue of the cluster split-K path
-    if (post && post_done && ctx->fuse_qkv && splits > 1 && 128 % c.head_dim == 0) {
-      a.post_on = 1;
-      a.post = *post;
-      *post_done = true;
     }
   } else {
     if (in.gain) return FL_ERR_UNSUPPORTED;   // the caller builds the input with the norm kernel instead
@@ -511,37 +581,181 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
 // previous kernel.
 fl_status run_call(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s) {
   set_pdl(ctx->pdl != 0);
+  set_tc_prefill(ctx->tc_prefill != 0);
   const fl_status st = run_call_body(ctx, decode, B, T, s);
   set_pdl(false);
   return st;
 }
 
+// How the next GEMM's normed input is produced: the norm kernel, already in x
+// (the selection kernel normalised it), or inside the GEMM from the sums of
+// squares the previous residual GEMM left.
+enum XIn { kXNorm, kXReady, kXSums };
+
+// The call's fixed shapes, shared by every layer.
+struct CallShape {
+  int decode, B, T, N, n_sel, max_need, max_chunks;
+  float tau;
+  int col_span;   // columns a query tile can see
+};
+
+// One layer applied to `n` token rows (`idx`, or every call token): the
+// attention branch (pre-norm, QKV + RoPE + KV write, dense attention or the
+// sparse-column correction, O-projection with the scaled residual add) and the
+// MLP branch (pre-norm, SwiGLU, down-projection with the scaled residual add).
+struct LayerRef {
+  StackW W;                  // weights of the layer's stack
+  int z;                     // layer index within the stack
+  const CacheView* cv;       // the KV cache the layer writes and reads
+  const CUtensorMap* kvmap;  // that cache's rows for the decode attention
+  int cj;                    // layer index within the cache
+  int loop;                  // loop number of the KV write (1 for independent layers)
+  bool lazy;                 // the lazy layout: base + residuals (the shared block on the lazy path)
+  bool full;                 // dense attention (otherwise the correction over column sets)
+  float *o_st, *l_st, *ql;   // per-query attention state (lazy path), or nullptr
+};
+
+fl_status run_layer(flashloop_ctx* ctx, const LayerRef& L, const CallShape& cs, const int32_t* idx, int n, XIn& xs,
+                    cudaStream_t s) {
+  const flashloop_config& c = ctx->cfg;
+  const int d = c.d_model, H = c.n_heads, Hkv = c.n_kv_heads, hd = c.head_dim;
+  auto pad = [&](int m) { return m <= 64 ? swap_bn(m) : ceil_div(m, 128) * 128; };
+  const float* attn_gain = L.W.attn_norm + static_cast<size_t>(L.z) * d;
+  const float* mlp_gain = L.W.mlp_norm + static_cast<size_t>(L.z) * d;
+  // attention branch
+  InNorm attn_in;
+  if (xs == kXNorm)
+    FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d, attn_gain, c.rms_eps, ctx->x, s));
+  if (xs == kXSums) {
+    attn_in.gain = attn_gain;
+    attn_in.idx = idx;
+  }
+  QkvPostArgs qa{};
+  qa.qkv = ctx->qkv; qa.ldq = ctx->qkv_rows; qa.idx = idx; qa.n = n; qa.seq = ctx->seq; qa.pos = ctx->pos;
+  qa.H = H; qa.Hkv = Hkv; qa.hd = hd; qa.rope_cos = ctx->rope_cos; qa.rope_sin = ctx->rope_sin;
+  qa.cv = *L.cv; qa.j = L.cj; qa.loop = L.loop; qa.lazy = L.lazy ? 1 : 0; qa.q_cur = ctx->q_cur; qa.q_last = L.ql;
+  qa.forced_on = ctx->forced_codes_on; qa.forced_codes = ctx->forced_codes;
+  qa.forced_scales = ctx->forced_scales; qa.forced_ns = ctx->nsel_max;
+  qa.trace_kv = ctx->trace_kv; qa.trace_ns = ctx->trace_ns;
+  FL_GEMM(gemm(ctx, L.W, kOpQKV, L.z, n, idx, s, attn_in));
+  FL_LAUNCH(FL_KIND_KV, launch_qkv_post(qa, s));
+  if (L.full) {
+    if (cs.decode) {
+      AttnDecArgs aa{};
+      // a full loop covers every token in order: no index indirection
+      aa.q_cur = ctx->q_cur; aa.idx = idx == ctx->idx_all ? nullptr : idx; aa.seq = ctx->seq; aa.pos = ctx->pos;
+      aa.cv = *L.cv;
+      aa.j = L.cj; aa.loop = L.loop; aa.dense = L.lazy ? 0 : 1; aa.H = H; aa.Hkv = Hkv; aa.hd = hd; aa.tau = cs.tau;
+      aa.n_splits = ctx->dec_splits;
+      aa.part_o = ctx->part_o; aa.part_ml = ctx->part_ml; aa.counters = ctx->attn_counters;
+      aa.o_state = L.o_st; aa.lse_state = L.l_st; aa.o_bf16 = ctx->obf; aa.status = ctx->status;
+      FL_LAUNCH(FL_KIND_ATTN, launch_attn_decode(*L.kvmap, aa, n, s));
+    } else {
+      AttnPreArgs pa{};
+      pa.q_cur = ctx->q_cur; pa.pos = ctx->pos; pa.cv = *L.cv; pa.j = L.cj; pa.loop = L.loop;
+      pa.dense = L.lazy ? 0 : 1;
+      pa.T = cs.T; pa.H = H; pa.Hkv = Hkv; pa.hd = hd; pa.tau = cs.tau;
+      pa.o_state = L.o_st; pa.lse_state = L.l_st; pa.o_bf16 = ctx->obf; pa.status = ctx->status;
+      FL_LAUNCH(FL_KIND_ATTN, launch_attn_prefill(*L.kvmap, pa, cs.B, s));
+    }
+  } else {
+    CorrectArgs ca{};
+    ca.idx = idx; ca.seq = ctx->seq; ca.pos = ctx->pos; ca.tile = ctx->tile; ca.last = ctx->last;
+    ca.q_cur = ctx->q_cur; ca.q_last = L.ql; ca.o_state = L.o_st; ca.lse_state = L.l_st; ca.o_bf16 = ctx->obf;
+    ca.cols = ctx->cols; ca.ncols = ctx->ncols; ca.meta = ctx->sel_meta; ca.cv = *L.cv; ca.j = L.cj; ca.loop = L.loop;
+    ca.H = H; ca.Hkv = Hkv;
+    ca.hd = hd; ca.c = c.c_cols; ca.n_tiles = ctx->n_tiles_max; ca.tau = cs.tau; ca.status = ctx->status;
+    ca.cols_per_cta = cs.n_sel <= kCorrSmallQueries ? kCorrColsSmall : kCorrColsBig;
+    ca.n_splits = ceil_div(c.c_cols, ca.cols_per_cta);
+    ca.part_acc = ctx->corr_acc; ca.part_mz = ctx->corr_mz; ca.counters = ctx->corr_counters;
+    ca.cluster = (cs.decode && cs.n_sel <= kCorrSmallQueries && ctx->corr_cluster) ? 1 : 0;
+    SelColsArgs sa{};
+    sa.plan = ctx->plan; sa.idx = idx; sa.pos = ctx->pos; sa.meta = ctx->sel_meta; sa.col_keys = ctx->col_keys;
+    sa.max_cols = c.max_ctx; sa.Hkv = Hkv; sa.c = c.c_cols; sa.j = L.cj; sa.n_tiles = ctx->n_tiles_max;
+    sa.cols = ctx->cols; sa.ncols = ctx->ncols; sa.forced_on = ctx->forced_on;
+    sa.forced_cols = ctx->forced_cols; sa.forced_ncols = ctx->forced_ncols;
+    sa.cand_keys = ctx->cand_keys; sa.cand_idx = ctx->cand_idx; sa.cand_counters = ctx->cand_cnt;
+    sa.max_slices = ctx->max_slices;
+    DScoreArgs da{};
+    da.plan = ctx->plan; da.idx = idx; da.seq = ctx->seq; da.pos = ctx->pos; da.meta = ctx->sel_meta;
+    da.q_cur = ctx->q_cur;
+    da.q_last = L.ql; da.cv = *L.cv; da.j = L.cj; da.loop = L.loop; da.H = H; da.Hkv = Hkv; da.hd = hd;
+    da.tau = cs.tau;
+    da.col_keys = ctx->col_keys; da.max_cols = c.max_ctx;
+    da.trace_ck = ctx->trace_ck; da.trace_tiles = ctx->trace_tiles;
+    da.tc = (!cs.decode && ctx->tc_prefill) ? 1 : 0;   // many queries per tile: tensor-core products
+    // rows that fit shared memory: the delta-score kernel also selects the column sets
+    da.fold = cs.col_span <= kSelColsSmemKeys ? 1 : 0;
+    da.sel = sa;
+    da.row_tickets = ctx->row_tickets;
+    FL_LAUNCH(FL_KIND_DSCORE, launch_dscore(da, cs.max_need, cs.max_chunks, s));
+    if (!da.fold) FL_LAUNCH(FL_KIND_SELECT, launch_select_cols(sa, cs.max_need, cs.col_span, s));
+    FL_LAUNCH(FL_KIND_CORRECT, launch_correct(ca, n, s));
+  }
+  bool sums = false;
+  FL_GEMM(gemm(ctx, L.W, kOpO, L.z, n, idx, s, InNorm{}, &sums));
+  // MLP branch
+  InNorm mlp_in;
+  if (sums) {
+    mlp_in.gain = mlp_gain;
+    mlp_in.idx = idx;
+  } else {
+    FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d, mlp_gain, c.rms_eps, ctx->x, s));
+  }
+  FL_GEMM(gemm(ctx, L.W, kOpGU, L.z, n, idx, s, mlp_in));
+  FL_GEMM(gemm(ctx, L.W, kOpDown, L.z, n, idx, s, InNorm{}, &sums));
+  xs = sums ? kXSums : kXNorm;
+  return FL_OK;
+}
+
+// The prelude (stack 1) or coda (stack 2) layers over every call token: dense
+// attention over their own one-pass KV.
+fl_status run_independent(flashloop_ctx* ctx, int stack, const CallShape& cs, XIn& xs, cudaStream_t s) {
+  const flashloop_config& c = ctx->cfg;
+  const int count = stack == 1 ? c.n_prelude : c.n_coda;
+  for (int z = 0; z < count; ++z) {
+    LayerRef L{stack_w(ctx, stack), z, &ctx->cvx, &ctx->tm_kvx, stack == 1 ? z : c.n_prelude + z, 1, false, true,
+               nullptr, nullptr, nullptr};
+    FL_STEP(run_layer(ctx, L, cs, ctx->idx_all, cs.N, xs, s));
+  }
+  return FL_OK;
+}
+
 fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream_t s) {
   const flashloop_config& c = ctx->cfg;
-  const int M = c.n_layers, K = c.n_loops, d = c.d_model, H = c.n_heads, Hkv = c.n_kv_heads, hd = c.head_dim;
+  const int M = c.n_layers, K = c.n_loops, d = c.d_model, H = c.n_heads, hd = c.head_dim;
   const bool lazy = ctx->lazy;
   const int N = decode ? B : B * T;
   const int q_tile = lazy ? c.q_tile : 128;
   const int tiles_per_seq = decode ? 1 : ceil_div(T, q_tile);
   const int n_tiles = decode ? B : B * tiles_per_seq;
   const int n_sel = lazy ? n_select(c.rho, N) : N;
-  const float tau = 1.0f / std::sqrt(static_cast<float>(hd));
   const size_t st_o = static_cast<size_t>(ctx->N_max) * H * hd, st_l = static_cast<size_t>(ctx->N_max) * H;
   auto pad = [&](int n) { return n <= 64 ? swap_bn(n) : ceil_div(n, 128) * 128; };
-  const int max_need = n_sel < n_tiles ? n_sel : n_tiles;
-  const int col_span = decode ? c.max_ctx : T;   // columns a query tile can see
-  const int max_chunks = ceil_div(col_span, 64);
+  int max_len = 0;   // longest context before the call (a prefill chunk continues after it)
+  for (int b = 0; b < B; ++b) max_len = std::max(max_len, ctx->lens[b]);
+  const int col_span = decode ? c.max_ctx : max_len + T;   // columns a query tile can see
+  CallShape cs{decode, B, T, N, n_sel, n_sel < n_tiles ? n_sel : n_tiles, ceil_div(col_span, 64),
+               1.0f / std::sqrt(static_cast<float>(hd)), col_span};
+  // the loop input h + e_l + gamma * x (loop embedding, input injection), x = the
+  // state entering the loop stack, kept in h_in
+  const bool loop_input = c.loop_embed || c.inject_scale != 0.f;
 
   ctx->launches = 0;
   ctx->ev_used = 0;
+  ctx->stamp_slots = 0;
+  // (the setup kernel also clears the GEMM launch stamps when they are on)
   FL_LAUNCH(FL_KIND_OTHER, launch_setup_call(N, decode, T, tiles_per_seq, q_tile, ctx->seq_len, ctx->seq, ctx->pos,
-                                             ctx->tile, ctx->last, n_tiles, ctx->has_c, s));
+                                             ctx->tile, ctx->last, n_tiles, ctx->has_c,
+                                             ctx->gemm_times ? ctx->stamps : nullptr, kMaxStamps, s));
   FL_TRY(cudaMemcpyAsync(ctx->h, ctx->h_in, static_cast<size_t>(N) * d * 4, cudaMemcpyDeviceToDevice, s));
-  // How the next GEMM's normed input is produced: the norm kernel, already in
-  // x (the selection kernel normalised it), or inside the GEMM from the sums of
-  // squares the previous residual GEMM left.
-  enum XIn { kXNorm, kXReady, kXSums };
   XIn carry = kXNorm;   // state at the end of the previous loop (dense loops keep their rows)
+  if (c.n_prelude) {
+    FL_STEP(run_independent(ctx, 1, cs, carry, s));
+    // the prelude's output is the state entering the loop stack: the loop-1
+    // change keys and the input injection measure from it
+    FL_TRY(cudaMemcpyAsync(ctx->h_in, ctx->h, static_cast<size_t>(N) * d * 4, cudaMemcpyDeviceToDevice, s));
+  }
   bool final_sums = false;
   for (int l = 1; l <= K; ++l) {
     const bool full = !lazy || l == 1;
@@ -558,7 +772,9 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
       sa.keys_trace = ctx->keys_trace + static_cast<size_t>(l - 2) * ctx->N_max; sa.idx = sel;
       sa.last = ctx->last; sa.tile = ctx->tile; sa.has_c = ctx->has_c; sa.forced_on = ctx->forced_on;
       sa.forced = ctx->forced_sel + static_cast<size_t>(l - 2) * ctx->N_max; sa.plan = ctx->plan;
-      if (n_sel <= kSelectStepMaxNorm && d <= 512 * kSelectStepSlices) {   // first layer's norm of the few selected rows
+      sa.cv = ctx->cv; sa.B_call = B; sa.status = ctx->status;
+      // first layer's norm of the few selected rows (not when the loop input changes them first)
+      if (!loop_input && n_sel <= kSelectStepMaxNorm && d <= 512 * kSelectStepSlices) {
         sa.norm_gain = ctx->w.attn_norm; sa.x = ctx->x; sa.x_rows = pad(n_sel); sa.eps = c.rms_eps;
       }
       FL_LAUNCH(FL_KIND_SELECT, launch_select_step(sa, s));
@@ -573,99 +789,37 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
                                                      ctx->forced_sel + static_cast<size_t>(l - 2) * ctx->N_max, s));
       FL_LAUNCH(FL_KIND_SELECT, launch_after_select(sel, n_sel, N, d, ctx->sel_slot, ctx->h, ctx->h_snap, ctx->seq,
                                                     ctx->tile, ctx->last, ctx->pos, ctx->sel_meta, s));
+      if (ctx->cv.rows)
+        FL_LAUNCH(FL_KIND_SELECT, launch_assign_rows(ctx->cv, l, B, N / B, ctx->sel_slot, ctx->pos, ctx->status, s));
       FL_LAUNCH(FL_KIND_SELECT, launch_plan_tiles(sel, n_sel, ctx->tile, ctx->has_c, ctx->plan, s));
       idx = sel;
       n = n_sel;
     }
+    if (loop_input) {
+      // after the selection's snapshot: the change keys compare loop outputs
+      FL_LAUNCH(FL_KIND_OTHER, launch_loop_input(ctx->h, idx == ctx->idx_all ? nullptr : idx, n, d,
+                                                 c.loop_embed ? ctx->w.loop_embed + static_cast<size_t>(l - 1) * d
+                                                              : nullptr,
+                                                 c.inject_scale, ctx->h_in, s));
+      xs = kXNorm;
+    }
     for (int j = 0; j < M; ++j) {
-      float* o_st = lazy ? ctx->o_state + j * st_o : nullptr;
-      float* l_st = lazy ? ctx->lse_state + j * st_l : nullptr;
-      float* ql = lazy ? ctx->q_last + j * st_o : nullptr;
-      // attention branch
-      InNorm attn_in;
-      if (xs == kXNorm)
-        FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d,
-                                                    ctx->w.attn_norm + static_cast<size_t>(j) * d, c.rms_eps, ctx->x,
-                                                    s));
-      if (xs == kXSums) {
-        attn_in.gain = ctx->w.attn_norm + static_cast<size_t>(j) * d;
-        attn_in.idx = idx;
-      }
-      QkvPostArgs qa{};
-      qa.qkv = ctx->qkv; qa.ldq = ctx->qkv_rows; qa.idx = idx; qa.n = n; qa.seq = ctx->seq; qa.pos = ctx->pos;
-      qa.H = H; qa.Hkv = Hkv; qa.hd = hd; qa.rope_cos = ctx->rope_cos; qa.rope_sin = ctx->rope_sin;
-      qa.cv = ctx->cv; qa.j = j; qa.loop = l; qa.lazy = lazy ? 1 : 0; qa.q_cur = ctx->q_cur; qa.q_last = ql;
-      qa.forced_on = ctx->forced_codes_on; qa.forced_codes = ctx->forced_codes;
-      qa.forced_scales = ctx->forced_scales; qa.forced_ns = ctx->nsel_max;
-      qa.trace_kv = ctx->trace_kv; qa.trace_ns = ctx->trace_ns;
-      bool post_done = false;
-      FL_GEMM(gemm(ctx, kOpQKV, j, n, idx, s, attn_in, nullptr, &qa, &post_done));
-      if (!post_done) FL_LAUNCH(FL_KIND_KV, launch_qkv_post(qa, s));
-      if (full) {
-        if (decode) {
-          AttnDecArgs aa{};
-          // a full loop covers every token in order: no index indirection
-          aa.q_cur = ctx->q_cur; aa.idx = idx == ctx->idx_all ? nullptr : idx; aa.seq = ctx->seq; aa.pos = ctx->pos;
-          aa.cv = ctx->cv;
-          aa.j = j; aa.loop = l; aa.dense = lazy ? 0 : 1; aa.H = H; aa.Hkv = Hkv; aa.hd = hd; aa.tau = tau;
-          aa.n_splits = ctx->dec_splits;
-          aa.part_o = ctx->part_o; aa.part_ml = ctx->part_ml; aa.counters = ctx->attn_counters;
-          aa.o_state = o_st; aa.lse_state = l_st; aa.o_bf16 = ctx->obf; aa.status = ctx->status;
-          FL_LAUNCH(FL_KIND_ATTN, launch_attn_decode(ctx->tm_kv, aa, n, s));
-        } else {
-          AttnPreArgs pa{};
-          pa.q_cur = ctx->q_cur; pa.cv = ctx->cv; pa.j = j; pa.loop = l; pa.dense = lazy ? 0 : 1;
-          pa.T = T; pa.H = H; pa.Hkv = Hkv; pa.hd = hd; pa.tau = tau;
-          pa.o_state = o_st; pa.lse_state = l_st; pa.o_bf16 = ctx->obf;
-          FL_LAUNCH(FL_KIND_ATTN, launch_attn_prefill(pa, B, s));
-        }
-      } else {
-        CorrectArgs ca{};
-        ca.idx = idx; ca.seq = ctx->seq; ca.pos = ctx->pos; ca.tile = ctx->tile; ca.last = ctx->last;
-        ca.q_cur = ctx->q_cur; ca.q_last = ql; ca.o_state = o_st; ca.lse_state = l_st; ca.o_bf16 = ctx->obf;
-        ca.cols = ctx->cols; ca.ncols = ctx->ncols; ca.meta = ctx->sel_meta; ca.cv = ctx->cv; ca.j = j; ca.loop = l; ca.H = H; ca.Hkv = Hkv;
-        ca.hd = hd; ca.c = c.c_cols; ca.n_tiles = ctx->n_tiles_max; ca.tau = tau; ca.status = ctx->status;
-        ca.cols_per_cta = n_sel <= kCorrSmallQueries ? kCorrColsSmall : kCorrColsBig;
-        ca.n_splits = ceil_div(c.c_cols, ca.cols_per_cta);
-        ca.part_acc = ctx->corr_acc; ca.part_mz = ctx->corr_mz; ca.counters = ctx->corr_counters;
-        ca.cluster = (decode && n_sel <= kCorrSmallQueries) ? 1 : 0;
-        DScoreArgs da{};
-        da.plan = ctx->plan; da.idx = idx; da.seq = ctx->seq; da.pos = ctx->pos; da.meta = ctx->sel_meta;
-        da.q_cur = ctx->q_cur;
-        da.q_last = ql; da.cv = ctx->cv; da.j = j; da.loop = l; da.H = H; da.Hkv = Hkv; da.hd = hd; da.tau = tau;
-        da.col_keys = ctx->col_keys; da.max_cols = c.max_ctx;
-        da.trace_ck = ctx->trace_ck; da.trace_tiles = ctx->trace_tiles;
-        FL_LAUNCH(FL_KIND_DSCORE, launch_dscore(da, max_need, max_chunks, s));
-        SelColsArgs sa{};
-        sa.plan = ctx->plan; sa.idx = idx; sa.pos = ctx->pos; sa.meta = ctx->sel_meta; sa.col_keys = ctx->col_keys;
-        sa.max_cols = c.max_ctx; sa.Hkv = Hkv; sa.c = c.c_cols; sa.j = j; sa.n_tiles = ctx->n_tiles_max;
-        sa.cols = ctx->cols; sa.ncols = ctx->ncols; sa.forced_on = ctx->forced_on;
-        sa.forced_cols = ctx->forced_cols; sa.forced_ncols = ctx->forced_ncols;
-        FL_LAUNCH(FL_KIND_SELECT, launch_select_cols(sa, max_need, s));
-        FL_LAUNCH(FL_KIND_CORRECT, launch_correct(ca, n, s));
-      }
-      bool sums = false;
-      FL_GEMM(gemm(ctx, kOpO, j, n, idx, s, InNorm{}, &sums));
-      // MLP branch
-      InNorm mlp_in;
-      if (sums) {
-        mlp_in.gain = ctx->w.mlp_norm + static_cast<size_t>(j) * d;
-        mlp_in.idx = idx;
-      } else {
-        FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, idx, n, pad(n), d,
-                                                    ctx->w.mlp_norm + static_cast<size_t>(j) * d, c.rms_eps, ctx->x,
-                                                    s));
-      }
-      FL_GEMM(gemm(ctx, kOpGU, j, n, idx, s, mlp_in));
-      FL_GEMM(gemm(ctx, kOpDown, j, n, idx, s, InNorm{}, &sums));
-      xs = sums ? kXSums : kXNorm;
+      LayerRef L{stack_w(ctx, 0), j, &ctx->cv, &ctx->tm_kv, j, l, lazy, full,
+                 lazy ? ctx->o_state + j * st_o : nullptr, lazy ? ctx->lse_state + j * st_l : nullptr,
+                 lazy ? ctx->q_last + j * st_o : nullptr};
+      FL_STEP(run_layer(ctx, L, cs, idx, n, xs, s));
     }
     carry = xs;
-    // the final norm can use the last down projection's sums when it covered every output row
-    final_sums = decode && l == K && full && xs == kXSums;
     if (lazy && l < K && !(N <= kSelectStepMax && n_tiles <= kSelectStepMax))
       FL_LAUNCH(FL_KIND_OTHER, launch_change_keys(ctx->h, l == 1 ? ctx->h_in : ctx->h_snap, ctx->sel_slot, N, d, l,
                                                   ctx->key, ctx->last, ctx->tile, ctx->has_c, s));
+    // the final norm can use the last down projection's sums when it covered every output row
+    final_sums = decode && l == K && full && xs == kXSums;
+  }
+  if (c.n_coda) {
+    XIn xc = (lazy && K > 1) ? kXNorm : carry;   // after a lazy loop the sums cover the selected rows only
+    FL_STEP(run_independent(ctx, 2, cs, xc, s));
+    final_sums = decode && xc == kXSums;
   }
   // final norm + LM head on the output rows
   const int32_t* rows = ctx->idx_all;
@@ -681,8 +835,8 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
   } else {
     FL_LAUNCH(FL_KIND_NORM, launch_rmsnorm_rows(ctx->h, rows, B, pad(B), d, ctx->w.final_norm, c.rms_eps, ctx->x, s));
   }
-  FL_GEMM(gemm(ctx, kOpOut, 0, B, rows, s, out_in));
-  FL_LAUNCH(FL_KIND_OTHER, launch_set_lens(B, ctx->seq_len, decode ? 1 : 0, T, s));
+  FL_GEMM(gemm(ctx, stack_w(ctx, 0), kOpOut, 0, B, rows, s, out_in));
+  FL_LAUNCH(FL_KIND_OTHER, launch_set_lens(B, ctx->seq_len, decode ? 1 : T, s));
   return FL_OK;
 }
 
@@ -697,6 +851,19 @@ bool build_tmaps(flashloop_ctx* ctx) {
   ok &= encode_tmap_bf16(&ctx->tm_up, w.w_up, d, f, M, 128);
   ok &= encode_tmap_bf16(&ctx->tm_down, w.w_down, f, d, M, 128);
   ok &= encode_tmap_bf16(&ctx->tm_out, w.w_out, d, c.vocab, 0, 128);
+  for (int x = 0; x < 2; ++x) {   // the prelude and coda stacks
+    const uint64_t L = x == 0 ? c.n_prelude : c.n_coda;
+    if (L == 0) continue;
+    const flashloop_layers& S = x == 0 ? w.prelude : w.coda;
+    ok &= encode_tmap_bf16(&ctx->tm_x_qkv[x], S.w_qkv, d, ctx->qkv_rows, L, 128);
+    ok &= encode_tmap_bf16(&ctx->tm_x_o[x], S.w_o, hq, d, L, 128);
+    ok &= encode_tmap_bf16(&ctx->tm_x_gate[x], S.w_gate, d, f, L, 128);
+    ok &= encode_tmap_bf16(&ctx->tm_x_up[x], S.w_up, d, f, L, 128);
+    ok &= encode_tmap_bf16(&ctx->tm_x_down[x], S.w_down, f, d, L, 128);
+  }
+  if (ctx->cvx.M > 0)   // the independent layers' KV as [rows][hd]: [X][1][2][B][Hkv][T]
+    ok &= encode_tmap_bf16(&ctx->tm_kvx, ctx->cvx.base, ctx->cvx.hd,
+                           static_cast<uint64_t>(ctx->cvx.M) * 2 * ctx->cvx.B * ctx->cvx.Hkv * ctx->cvx.T, 0, 64);
   const uint64_t R = ctx->N_pad;
   ok &= encode_tmap_bf16(&ctx->tm_x_a, ctx->x, d, R, 0, 128);
   ok &= encode_tmap_bf16(&ctx->tm_obf_a, ctx->obf, hq, R, 0, 128);
@@ -756,6 +923,14 @@ fl_status flashloop_init(const flashloop_config* cfg, const flashloop_weights* w
                        w->w_out};
   for (const void* p : wp)
     if (!p || !aligned16(p)) return FL_ERR_INVALID_ARG;
+  for (int x = 0; x < 2; ++x) {
+    if ((x == 0 ? cfg->n_prelude : cfg->n_coda) == 0) continue;
+    const flashloop_layers& S = x == 0 ? w->prelude : w->coda;
+    const void* sp[7] = {S.attn_norm, S.w_qkv, S.w_o, S.mlp_norm, S.w_gate, S.w_up, S.w_down};
+    for (const void* p : sp)
+      if (!p || !aligned16(p)) return FL_ERR_INVALID_ARG;
+  }
+  if (cfg->loop_embed && (!w->loop_embed || !aligned16(w->loop_embed))) return FL_ERR_INVALID_ARG;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255)) return FL_ERR_WORKSPACE;
   const size_t need = layout(*cfg, nullptr);
   if (workspace_bytes < need) return FL_ERR_WORKSPACE;
@@ -786,6 +961,11 @@ fl_status flashloop_init(const flashloop_config* cfg, const flashloop_weights* w
 
   if (!build_tmaps(ctx)) return fail(FL_ERR_CUDA);
   if (cudaMemsetAsync(ctx->ws, 0, need, s) != cudaSuccess) return fail(FL_ERR_CUDA);
+  if (ctx->cv.rows &&   // sparse residual storage: no position holds a residual row yet
+      cudaMemsetAsync(ctx->cv.ridx, 0xFF,
+                      static_cast<size_t>(cfg->n_layers) * (cfg->n_loops - 1) * cfg->max_batch * cfg->max_ctx * 4,
+                      s) != cudaSuccess)
+    return fail(FL_ERR_CUDA);
   // RoPE table: angle = pos * theta^(-2i/hd), computed in double, stored fp32
   const int half = cfg->head_dim / 2;
   std::vector<float> rc(static_cast<size_t>(cfg->max_ctx) * half), rs(rc.size());
@@ -831,8 +1011,16 @@ fl_status flashloop_set_option(flashloop_ctx* ctx, fl_option opt, int value) {
     ctx->pdl = value ? 1 : 0;
     return FL_OK;
   }
-  if (opt == FL_OPT_FUSE_QKV) {
-    ctx->fuse_qkv = value ? 1 : 0;
+  if (opt == FL_OPT_GEMM_TIMES) {
+    ctx->gemm_times = value ? 1 : 0;
+    return FL_OK;
+  }
+  if (opt == FL_OPT_TC_PREFILL) {
+    ctx->tc_prefill = value ? 1 : 0;
+    return FL_OK;
+  }
+  if (opt == FL_OPT_CORR_CLUSTER) {
+    ctx->corr_cluster = value ? 1 : 0;
     return FL_OK;
   }
   return FL_ERR_INVALID_ARG;
@@ -844,7 +1032,7 @@ fl_status flashloop_prefill(flashloop_ctx* ctx, const float* h0, int B, int T, f
   const flashloop_config& c = ctx->cfg;
   if (B > c.max_batch || static_cast<long long>(B) * T > c.max_tokens || T > c.max_ctx) return FL_ERR_CAPACITY;
   for (int b = 0; b < B; ++b)
-    if (ctx->lens[b] != 0) return FL_ERR_INVALID_ARG;
+    if (ctx->lens[b] + T > c.max_ctx) return FL_ERR_CAPACITY;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t bytes = static_cast<size_t>(B) * T * c.d_model * 4;
   FL_TRY(cudaMemcpyAsync(ctx->h_in, h0, bytes, cudaMemcpyDefault, s));
@@ -852,7 +1040,7 @@ fl_status flashloop_prefill(flashloop_ctx* ctx, const float* h0, int B, int T, f
   if (h_out) FL_TRY(cudaMemcpyAsync(h_out, ctx->h, bytes, cudaMemcpyDefault, s));
   if (logits_last)
     FL_TRY(cudaMemcpyAsync(logits_last, ctx->logits_ws, static_cast<size_t>(B) * c.vocab * 4, cudaMemcpyDefault, s));
-  for (int b = 0; b < B; ++b) ctx->lens[b] = T;
+  for (int b = 0; b < B; ++b) ctx->lens[b] += T;
   ctx->last_N = B * T;
   ctx->last_nsel = ctx->lazy ? n_select(c.rho, B * T) : B * T;
   ctx->last_decode = 0;
@@ -871,7 +1059,8 @@ fl_status flashloop_decode_step(flashloop_ctx* ctx, const float* h0, int B, floa
   FL_TRY(cudaMemcpyAsync(ctx->h_in, h0, static_cast<size_t>(B) * c.d_model * 4, cudaMemcpyDefault, s));
   // A decode step's launch sequence depends on B only; after one direct run it
   // is captured once into a CUDA graph and replayed (not on the legacy stream).
-  const int gkey = B * 8 + (ctx->prof ? 1 : 0) + (ctx->pdl ? 2 : 0) + (ctx->fuse_qkv ? 4 : 0);
+  const int gkey = B * 32 + (ctx->prof ? 1 : 0) + (ctx->pdl ? 2 : 0) + (ctx->gemm_times ? 8 : 0) +
+                   (ctx->corr_cluster ? 16 : 0);
   size_t gi = 0;
   while (gi < ctx->graph_b.size() && ctx->graph_b[gi] != gkey) ++gi;
   bool seen = false;
@@ -916,12 +1105,23 @@ fl_status flashloop_kv_bytes_for(const flashloop_config* cfg, size_t* total, dou
   const flashloop_config& c = *cfg;
   const double hd = c.head_dim, kv = 2.0 * c.n_kv_heads;
   const double dense = kv * c.n_loops * hd * 2.0;
-  double per = dense;
-  if (c.resid_bits != 16)
-    per = kv * (hd * 2.0 + (c.n_loops - 1) * (hd * c.resid_bits / 8.0 + (hd / c.group_size) * 2.0));
+  double per = c.kv_mode == 1 ? kv * hd * 2.0 : dense;   // last_loop keeps one pass of KV
+  if (c.resid_bits != 16) {
+    // the bf16 base, plus K-1 residual rows (packed codes and fp16 scales) per
+    // position, or with sparse storage resid_rows per pool and a 4-byte row index
+    const double row = hd * c.resid_bits / 8.0 + (hd / c.group_size) * 2.0;
+    per = kv * hd * 2.0;
+    if (c.resid_rows > 0)
+      per += (c.n_loops - 1) * (kv * row * static_cast<double>(c.resid_rows) / c.max_ctx + 4.0);
+    else
+      per += (c.n_loops - 1) * kv * row;
+  }
   if (per_token_per_layer) *per_token_per_layer = per;
   if (dense_per_token_per_layer) *dense_per_token_per_layer = dense;
-  if (total) *total = static_cast<size_t>(per * c.n_layers * c.max_batch * static_cast<double>(c.max_ctx));
+  // the looped layers' cache plus one pass of KV for each prelude / coda layer
+  const double extra = (c.n_prelude + c.n_coda) * kv * hd * 2.0;
+  if (total)
+    *total = static_cast<size_t>((per * c.n_layers + extra) * c.max_batch * static_cast<double>(c.max_ctx));
   return FL_OK;
 }
 
@@ -950,6 +1150,8 @@ fl_status flashloop_reset(flashloop_ctx* ctx, const int* seq_len, fl_stream_t st
     FL_TRY(cudaMemcpyAsync(ctx->seq_len, v.data(), B * 4, cudaMemcpyHostToDevice, s));
     FL_TRY(cudaStreamSynchronize(s));
   }
+  // sparse residual storage: the pools keep the rows of the positions below the new lengths
+  if (ctx->cv.rows) FL_TRY(launch_reset_rows(ctx->cv, ctx->seq_len, s));
   ctx->lens = v;
   return FL_OK;
 }
@@ -973,6 +1175,27 @@ fl_status flashloop_profile(flashloop_ctx* ctx, fl_stream_t stream, float* ms, i
 
 int flashloop_kernels_per_call(const flashloop_ctx* ctx) { return ctx ? ctx->launches : 0; }
 
+fl_status flashloop_gemm_times(flashloop_ctx* ctx, fl_stream_t stream, double* total_ms, int* launches) {
+  if (!ctx || !total_ms || !launches) return FL_ERR_INVALID_ARG;
+  *total_ms = 0.0;
+  *launches = 0;
+  if (!ctx->gemm_times) return FL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  FL_TRY(cudaStreamSynchronize(s));
+  const int n = ctx->stamp_slots;
+  std::vector<unsigned long long> st(n), en(n);
+  if (n) {
+    FL_TRY(cudaMemcpy(st.data(), ctx->stamps, static_cast<size_t>(n) * 8, cudaMemcpyDeviceToHost));
+    FL_TRY(cudaMemcpy(en.data(), ctx->stamps + kMaxStamps, static_cast<size_t>(n) * 8, cudaMemcpyDeviceToHost));
+  }
+  double sum = 0.0;
+  for (int i = 0; i < n; ++i)
+    if (en[i] > st[i] && st[i] != ~0ULL) sum += static_cast<double>(en[i] - st[i]);
+  *total_ms = sum * 1e-6;
+  *launches = n;
+  return FL_OK;
+}
+
 fl_status flashloop_sync_status(flashloop_ctx* ctx, fl_stream_t stream) {
   if (!ctx) return FL_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -984,6 +1207,7 @@ fl_status flashloop_sync_status(flashloop_ctx* ctx, fl_stream_t stream) {
     FL_TRY(cudaMemcpy(ctx->status, &zero, 4, cudaMemcpyHostToDevice));
   }
   if (st & kErrWaitTimeout) return FL_ERR_TIMEOUT;
+  if (st & kErrCapacity) return FL_ERR_CAPACITY;
   if (st) return FL_ERR_NONFINITE;
   return FL_OK;
 }
@@ -1001,6 +1225,15 @@ fl_status flashloop_import_lazy(flashloop_ctx* ctx, int layer, int seq, int n, c
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const int Hkv = c.n_kv_heads, hd = c.head_dim, ns = hd / c.group_size;
   const CacheView& cv = ctx->cv;
+  if (cv.rows) {   // sparse residual storage: rows for the positions that hold a residual
+    for (int kv = 0; kv < 2; ++kv)
+      for (int h = 0; h < Hkv; ++h)
+        FL_TRY(cudaMemcpyAsync(cv.base_row(layer, kv, seq, h, 0), (kv ? base_v : base_k) + static_cast<size_t>(h) * n * hd,
+                               static_cast<size_t>(n) * hd * 2, cudaMemcpyDefault, s));
+    if (c.n_loops > 1)
+      FL_TRY(launch_import_rows(cv, layer, seq, n, codes_k, codes_v, scales_k, scales_v, ctx->status, s));
+    return FL_OK;
+  }
   for (int kv = 0; kv < 2; ++kv) {
     const uint16_t* base = kv ? base_v : base_k;
     for (int h = 0; h < Hkv; ++h)
@@ -1031,12 +1264,27 @@ fl_status flashloop_import_dense(flashloop_ctx* ctx, int layer, int seq, int n, 
   const int Hkv = c.n_kv_heads, hd = c.head_dim;
   for (int kv = 0; kv < 2; ++kv) {
     const uint16_t* src = kv ? kv_v : kv_k;
-    for (int l = 1; l <= c.n_loops; ++l)
+    for (int l = 1; l <= ctx->cv.K; ++l)   // the stored loops (one in last_loop mode)
       for (int h = 0; h < Hkv; ++h)
         FL_TRY(cudaMemcpyAsync(ctx->cv.dense_row(layer, l, kv, seq, h, 0),
                                src + (static_cast<size_t>(l - 1) * Hkv + h) * n * hd, static_cast<size_t>(n) * hd * 2,
                                cudaMemcpyDefault, s));
   }
+  return FL_OK;
+}
+
+fl_status flashloop_import_extra(flashloop_ctx* ctx, int x, int seq, int n, const uint16_t* kv_k,
+                                 const uint16_t* kv_v, fl_stream_t stream) {
+  if (!ctx || !kv_k || !kv_v) return FL_ERR_INVALID_ARG;
+  const flashloop_config& c = ctx->cfg;
+  if (x < 0 || x >= c.n_prelude + c.n_coda || seq < 0 || seq >= c.max_batch || n < 0 || n > c.max_ctx)
+    return FL_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int Hkv = c.n_kv_heads, hd = c.head_dim;
+  for (int kv = 0; kv < 2 && n > 0; ++kv)
+    for (int h = 0; h < Hkv; ++h)
+      FL_TRY(cudaMemcpyAsync(ctx->cvx.dense_row(x, 1, kv, seq, h, 0), (kv ? kv_v : kv_k) + static_cast<size_t>(h) * n * hd,
+                             static_cast<size_t>(n) * hd * 2, cudaMemcpyDefault, s));
   return FL_OK;
 }
 
@@ -1063,6 +1311,14 @@ fl_status flashloop_export_slice(const flashloop_ctx* ctx, int layer, int loop, 
     return FL_OK;
   }
   if (!scales) return FL_ERR_INVALID_ARG;
+  if (cv.rows) {   // sparse residual storage: gathered by position, zero where no row is kept
+    if (n > 0 && launch_export_rows(cv, layer, loop, which, seq, n, static_cast<uint8_t*>(codes),
+                                    static_cast<uint16_t*>(scales), s) != cudaSuccess) {
+      mctx->last_err = "export gather failed";
+      return FL_ERR_CUDA;
+    }
+    return FL_OK;
+  }
   const size_t rb = cv.row_bytes_codes();
   const int ns = hd / c.group_size;
   for (int h = 0; h < Hkv; ++h) {

@@ -19,7 +19,9 @@ FL_OK = 0
 FL_OPT_USE_GRAPH = 1
 FL_OPT_PROFILE = 2
 FL_OPT_PDL = 3
-FL_OPT_FUSE_QKV = 4
+FL_OPT_GEMM_TIMES = 5
+FL_OPT_TC_PREFILL = 6
+FL_OPT_CORR_CLUSTER = 7
 KINDS = ["gemm", "attn", "dscore", "correct", "kv", "select", "norm", "other"]
 STATUS = {0: "ok", 1: "invalid argument", 2: "capacity exceeded", 3: "workspace", 4: "cuda error",
           5: "timeout", 6: "nonfinite", 7: "unsupported"}
@@ -38,12 +40,21 @@ class Config(ctypes.Structure):
                 ("q_tile", ctypes.c_int), ("resid_bits", ctypes.c_int), ("group_size", ctypes.c_int),
                 ("resid_scale", ctypes.c_float), ("rms_eps", ctypes.c_float), ("rope_theta", ctypes.c_float),
                 ("vocab", ctypes.c_int), ("max_batch", ctypes.c_int), ("max_ctx", ctypes.c_int),
-                ("max_tokens", ctypes.c_int)]
+                ("max_tokens", ctypes.c_int), ("kv_mode", ctypes.c_int), ("n_prelude", ctypes.c_int),
+                ("n_coda", ctypes.c_int), ("loop_embed", ctypes.c_int), ("inject_scale", ctypes.c_float),
+                ("resid_rows", ctypes.c_int)]
+
+
+LAYER_FIELDS = ("attn_norm", "w_qkv", "w_o", "mlp_norm", "w_gate", "w_up", "w_down")
+
+
+class Layers(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in LAYER_FIELDS]
 
 
 class Weights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("attn_norm", "w_qkv", "w_o", "mlp_norm", "w_gate", "w_up",
-                                               "w_down", "final_norm", "w_out")]
+    _fields_ = [(n, ctypes.c_void_p) for n in LAYER_FIELDS + ("final_norm", "w_out")] + [
+        ("prelude", Layers), ("coda", Layers), ("loop_embed", ctypes.c_void_p)]
 
 
 _P = ctypes.c_void_p
@@ -65,6 +76,7 @@ _SIG = {
     "flashloop_last_cuda_error": (ctypes.c_char_p, [_P]),
     "flashloop_import_lazy": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P]),
     "flashloop_import_dense": (_I, [_P, _I, _I, _I, _P, _P, _P]),
+    "flashloop_import_extra": (_I, [_P, _I, _I, _I, _P, _P, _P]),
     "flashloop_export_slice": (_I, [_P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "flashloop_force_selection": (_I, [_P, _P, _I, _I, _P, _P, _I]),
     "flashloop_read_trace": (_I, [_P, _P, _P, _P, _P, _P]),
@@ -73,6 +85,7 @@ _SIG = {
     "flashloop_set_option": (_I, [_P, _I, _I]),
     "flashloop_profile": (_I, [_P, _P, _P, _P]),
     "flashloop_kernels_per_call": (_I, [_P]),
+    "flashloop_gemm_times": (_I, [_P, _P, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(_I)]),
     "fl_test_topk": (_I, [_P, _I, _I, _I, _P, _P]),
     "fl_test_quantize": (_I, [_P, _I, _I, _I, _I, _P, _P, _P]),
     "fl_test_quantize_residual": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P]),
@@ -111,7 +124,10 @@ def make_config(cfg, max_batch: int, max_ctx: int, max_tokens: int = 0, resid_bi
     return Config(cfg.d_model, cfg.n_heads, cfg.n_kv_heads, cfg.head_dim, cfg.ffn_dim, cfg.n_layers, cfg.n_loops,
                   float(cfg.rho), cfg.c_cols, cfg.q_tile, cfg.resid_bits if resid_bits is None else resid_bits,
                   cfg.group_size, float(cfg.resid_scale), float(cfg.rms_eps), float(cfg.rope_theta), cfg.vocab,
-                  max_batch, max_ctx, max_tokens)
+                  max_batch, max_ctx, max_tokens, int(getattr(cfg, "kv_mode", 0)),
+                  int(getattr(cfg, "n_prelude", 0)), int(getattr(cfg, "n_coda", 0)),
+                  int(getattr(cfg, "loop_embed", 0)), float(getattr(cfg, "inject_scale", 0.0)),
+                  int(getattr(cfg, "resid_rows", 0)))
 
 
 def workspace_bytes(c: Config) -> int:
@@ -137,19 +153,24 @@ def upload_weights(w: dict, device="cuda"):
     """Stack the generator's per-layer weights into device tensors (bf16 bits as int16)."""
     import torch
 
-    def stack(name, dt=np.uint16):
-        a = np.stack([lw[name] for lw in w["layers"]]).astype(dt, copy=False)
+    def stack(layers, name, dt=np.uint16):
+        a = np.stack([lw[name] for lw in layers]).astype(dt, copy=False)
         if dt == np.uint16:
             return torch.from_numpy(a.view(np.int16)).to(device)
         return torch.from_numpy(a).to(device)
 
-    return {
-        "attn_norm": stack("attn_norm", np.float32), "w_qkv": stack("w_qkv"), "w_o": stack("w_o"),
-        "mlp_norm": stack("mlp_norm", np.float32), "w_gate": stack("w_gate"), "w_up": stack("w_up"),
-        "w_down": stack("w_down"),
-        "final_norm": torch.from_numpy(np.asarray(w["final_norm"], np.float32)).to(device),
-        "w_out": torch.from_numpy(np.asarray(w["w_out"]).view(np.int16)).to(device),
-    }
+    def layer_stack(layers):
+        return {n: stack(layers, n, np.float32 if n.endswith("norm") else np.uint16) for n in LAYER_FIELDS}
+
+    out = layer_stack(w["layers"])
+    out["final_norm"] = torch.from_numpy(np.asarray(w["final_norm"], np.float32)).to(device)
+    out["w_out"] = torch.from_numpy(np.asarray(w["w_out"]).view(np.int16)).to(device)
+    for part in ("prelude", "coda"):
+        if w.get(part):
+            out[part] = layer_stack(w[part])
+    if "loop_embed" in w:
+        out["loop_embed"] = torch.from_numpy(np.asarray(w["loop_embed"], np.float32)).to(device)
+    return out
 
 
 class FlashLoop:
@@ -168,7 +189,12 @@ class FlashLoop:
         off = (-self.workspace.data_ptr()) % 256
         self._ws_ptr = self.workspace.data_ptr() + off
         self._ws_bytes = nbytes
-        wt = Weights(*[dev_weights[n].data_ptr() for n, _ in Weights._fields_])
+        def layers(d):
+            return Layers(*[d[n].data_ptr() for n in LAYER_FIELDS]) if d else Layers()
+
+        wt = Weights(*[dev_weights[n].data_ptr() for n in LAYER_FIELDS + ("final_norm", "w_out")],
+                     layers(dev_weights.get("prelude")), layers(dev_weights.get("coda")),
+                     dev_weights["loop_embed"].data_ptr() if "loop_embed" in dev_weights else None)
         self._wstruct = wt
         ctx = ctypes.c_void_p()
         st = lib().flashloop_init(ctypes.byref(self.c), ctypes.byref(wt), ctypes.c_void_p(self._ws_ptr),
@@ -222,6 +248,13 @@ class FlashLoop:
         _check(lib().flashloop_profile(self.ctx, _stream_ptr(stream), ms, n), "flashloop_profile", self.ctx)
         return {k: (float(ms[i]), int(n[i])) for i, k in enumerate(KINDS)}
 
+    def gemm_times(self, stream=None):
+        """(summed device ms, launches) of the last call's GEMMs (FL_OPT_GEMM_TIMES on)."""
+        ms, n = ctypes.c_double(), ctypes.c_int()
+        _check(lib().flashloop_gemm_times(self.ctx, _stream_ptr(stream), ctypes.byref(ms), ctypes.byref(n)),
+               "gemm_times", self.ctx)
+        return ms.value, n.value
+
     def kernels_per_call(self) -> int:
         return int(lib().flashloop_kernels_per_call(self.ctx))
 
@@ -266,6 +299,17 @@ class FlashLoop:
                 self.import_lazy(j, b, a["base_k"], a["base_v"], a["codes_k"], a["codes_v"], a["scales_k"],
                                  a["scales_v"])
                 torch.cuda.synchronize()   # the import copies read the staged tensors
+        if "extra_k" in ctx:             # the prelude / coda layers' one-pass KV
+            for x in range(ctx["extra_k"].shape[0]):
+                for b, n in enumerate(lens):
+                    n = int(n)
+                    if n == 0:
+                        continue
+                    kk = torch.from_numpy(np.ascontiguousarray(ctx["extra_k"][x, b, :, :n]).view(np.int16)).cuda()
+                    vv = torch.from_numpy(np.ascontiguousarray(ctx["extra_v"][x, b, :, :n]).view(np.int16)).cuda()
+                    _check(lib().flashloop_import_extra(self.ctx, x, b, n, _ptr(kk), _ptr(vv), None),
+                           "flashloop_import_extra", self.ctx)
+                    torch.cuda.synchronize()
         torch.cuda.synchronize()
         self.reset([int(x) for x in lens])
         torch.cuda.synchronize()

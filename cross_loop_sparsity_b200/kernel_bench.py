@@ -2,9 +2,10 @@
 
   python -m cross_loop_sparsity_b200.kernel_bench [--reps N]
 
-* ``gemm_wide``: the 128x128 tcgen05 GEMM at the long-prefill shapes
-  (16384 tokens x d_model 2048: QKV 3072, O 2048, gate or up 5632, down from
-  5632), TFLOP/s against the measured dense bf16 peak.
+* ``gemm_wide``: the persistent tcgen05 GEMM (128 x 256 output tiles, two TMEM
+  accumulators) at the long-prefill shapes (16384 tokens x d_model 2048: QKV
+  3072, O 2048, gate or up 5632, down from 5632), TFLOP/s against the measured
+  dense bf16 peak.
 * ``gemm_skinny``: the split-K swap-AB GEMM at the decode shapes (8 tokens),
   weight GB/s against the measured HBM bandwidth.
 * ``topk``: the top-c column selection (bit pattern descending, index
@@ -26,7 +27,8 @@
 
 Every operand set is rotated over copies whose total exceeds L2 (126 MB), so
 each timed launch reads from HBM; times are CUDA events around ``reps``
-launches after warm-up, on one stream.
+launches after warm-up, on one stream.  Every line carries the SM clocks and
+throttle reasons sampled while its kernel group ran (``clocks``).
 """
 from __future__ import annotations
 
@@ -217,6 +219,26 @@ def quantize_residual(reps):
              "achieved": gbs, "unit": "GB/s", "peak": hbm, "frac": gbs / hbm, "peak_source": f"{src} hbm_gbs"}]
 
 
+def decode_step_capture(reps):
+    """One decode step at the decode workload's GEMM shapes (8 tokens, d_model
+    2048, ffn 5632, vocab 32000) with one shared layer and a 512-token context,
+    kernels launched directly (no graph), for an ncu capture of the first GEMM
+    launches: a few GB on the device.  Prints no measurement."""
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl, synth
+    cfg = synth.config("c2").with_(n_layers=1, ctx_len=512)
+    w = synth.make_weights(cfg)
+    eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=cfg.batch, max_ctx=cfg.ctx_len + 1)
+    eng.load_context(synth.make_context(cfg, w["rng"], [cfg.ctx_len] * cfg.batch))
+    eng.set_option(fl.FL_OPT_USE_GRAPH, 0)
+    h0 = torch.from_numpy(synth.make_h0(cfg, w["rng"], cfg.batch)).cuda()
+    eng.decode_step(h0, cfg.batch)
+    torch.cuda.synchronize()
+    assert eng.sync_status() == 0
+    eng.close()
+    return []
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--reps", type=int, default=20)
@@ -224,12 +246,21 @@ def main():
     args = ap.parse_args()
     from cross_loop_sparsity_b200 import build
     build.build()
-    fns = (gemm_wide, gemm_skinny, topk, attn_decode, quantize_residual, quantize)
+    import time
+    import torch
+    from cross_loop_sparsity_b200.clocks import ClockSampler
+    fns = (gemm_wide, gemm_skinny, topk, attn_decode, quantize_residual, quantize, decode_step_capture)
     only = {x for x in args.only.split(",") if x}
     for fn in fns:
-        if only and fn.__name__ not in only:
+        if (only and fn.__name__ not in only) or (not only and fn is decode_step_capture):
             continue
-        for line in fn(args.reps):
+        sampler = ClockSampler(torch.cuda.current_device())
+        sampler.start()
+        time.sleep(0.3)
+        lines = fn(args.reps)
+        clocks = sampler.stop()
+        for line in lines:
+            line["clocks"] = clocks
             print(json.dumps(line), flush=True)
 
 

@@ -36,7 +36,7 @@ import numpy as np
 __all__ = [
     "LoopConfig", "CONFIGS", "config", "bf16_bits", "bf16_bits_to_f32",
     "make_weights", "make_h0", "make_context", "make_dense_context",
-    "make_keys", "make_residuals",
+    "make_keys", "make_residuals", "make_weights_device", "context_slices_device",
 ]
 
 
@@ -66,6 +66,14 @@ class LoopConfig:
     batch: int = 1
     seq_len: int = 0       # prefill tokens per sequence
     ctx_len: int = 0       # existing context per sequence (decode)
+    kv_mode: int = 0       # dense path: 0 per_loop KV, 1 last_loop (one KV per layer, overwritten each loop)
+    # variants around the looped core: independent layers before (prelude) and
+    # after (coda) the loop, a per-loop input embedding, and input injection
+    n_prelude: int = 0
+    n_coda: int = 0
+    loop_embed: int = 0        # 1: loop k's input is h + e_k
+    inject_scale: float = 0.0  # gamma: loop k's input also adds gamma * (the state entering the loop)
+    resid_rows: int = 0        # sparse residual storage: rows per pool (0: one row per position)
 
     @property
     def qkv_rows(self) -> int:
@@ -113,6 +121,13 @@ def config(name: str, **overrides) -> LoopConfig:
     return cfg.with_(**overrides) if overrides else cfg
 
 
+def sparse_rows(cfg: LoopConfig, extra: int) -> int:
+    """Rows per sparse residual pool for a cache of cfg.max_ctx positions whose
+    tokens were recomputed at rate rho (the synthetic context's rate), plus
+    `extra` rows for tokens appended later."""
+    return min(cfg.max_ctx, int(math.ceil(cfg.rho * cfg.max_ctx - 1e-9)) + extra)
+
+
 # ----------------------------------------------------------------------------
 # bfloat16 bit patterns (input preparation: weights and KV are bf16 data)
 # ----------------------------------------------------------------------------
@@ -146,25 +161,37 @@ def _normal_bf16(rng: np.random.Generator, shape, sigma: float) -> np.ndarray:
 def make_weights(cfg: LoopConfig, rng: np.random.Generator | None = None) -> dict:
     """All block weights as bfloat16 bit patterns; norm gains are float32 ones."""
     rng = np.random.default_rng(cfg.seed) if rng is None else rng
-    d, f = cfg.d_model, cfg.ffn_dim
-    hq = cfg.n_heads * cfg.head_dim
-    layers = []
-    for _ in range(cfg.n_layers):
-        lw = {}
-        lw["attn_norm"] = np.ones(d, np.float32)
-        lw["w_qkv"] = _normal_bf16(rng, (cfg.qkv_rows, d), cfg.sigma)
-        lw["w_o"] = _normal_bf16(rng, (d, hq), cfg.sigma)
-        lw["mlp_norm"] = np.ones(d, np.float32)
-        lw["w_gate"] = _normal_bf16(rng, (f, d), cfg.sigma)
-        lw["w_up"] = _normal_bf16(rng, (f, d), cfg.sigma)
-        lw["w_down"] = _normal_bf16(rng, (d, f), cfg.sigma)
-        layers.append(lw)
-    return {
-        "layers": layers,
+    d = cfg.d_model
+    out = {
+        "layers": [_draw_layer(cfg, rng) for _ in range(cfg.n_layers)],
         "final_norm": np.ones(d, np.float32),
         "w_out": _normal_bf16(rng, (cfg.vocab, d), cfg.sigma),
         "rng": rng,
     }
+    # variants, drawn after everything above so the plain looped block's draws
+    # do not move: prelude layers, coda layers, then the loop embeddings
+    # e_1..e_K ~ N(0, 1) float32 (the scale of the residual stream)
+    if cfg.n_prelude:
+        out["prelude"] = [_draw_layer(cfg, rng) for _ in range(cfg.n_prelude)]
+    if cfg.n_coda:
+        out["coda"] = [_draw_layer(cfg, rng) for _ in range(cfg.n_coda)]
+    if cfg.loop_embed:
+        out["loop_embed"] = rng.standard_normal(size=(cfg.n_loops, d), dtype=np.float32)
+    return out
+
+
+def _draw_layer(cfg: LoopConfig, rng: np.random.Generator) -> dict:
+    """One layer's weights in the draw order of the recipe."""
+    d, f, hq = cfg.d_model, cfg.ffn_dim, cfg.n_heads * cfg.head_dim
+    lw = {}
+    lw["attn_norm"] = np.ones(d, np.float32)
+    lw["w_qkv"] = _normal_bf16(rng, (cfg.qkv_rows, d), cfg.sigma)
+    lw["w_o"] = _normal_bf16(rng, (d, hq), cfg.sigma)
+    lw["mlp_norm"] = np.ones(d, np.float32)
+    lw["w_gate"] = _normal_bf16(rng, (f, d), cfg.sigma)
+    lw["w_up"] = _normal_bf16(rng, (f, d), cfg.sigma)
+    lw["w_down"] = _normal_bf16(rng, (d, f), cfg.sigma)
+    return lw
 
 
 def make_h0(cfg: LoopConfig, rng: np.random.Generator, n_tokens: int) -> np.ndarray:
@@ -207,15 +234,36 @@ def make_context(cfg: LoopConfig, rng: np.random.Generator, ctx_lens) -> dict:
                                                    dtype=np.int8)
                     s_view[:, rows] = rng.uniform(0.01, 0.03, size=(Hkv, len(rows), hd // g)
                                                   ).astype(np.float16)
-    return {"lens": lens, "base_k": base_k, "base_v": base_v, "codes_k": codes_k, "codes_v": codes_v,
-            "scales_k": scales_k, "scales_v": scales_v}
+    out = {"lens": lens, "base_k": base_k, "base_v": base_v, "codes_k": codes_k, "codes_v": codes_v,
+           "scales_k": scales_k, "scales_v": scales_v}
+    out.update(_extra_context(cfg, rng, lens))
+    return out
+
+
+def _extra_context(cfg: LoopConfig, rng: np.random.Generator, lens) -> dict:
+    """KV of the prelude and coda layers (one pass each): uint16 bf16 bits
+    [P+Q, B, Hkv, T, hd] of N(0, 1), drawn after the looped layers' context."""
+    X = cfg.n_prelude + cfg.n_coda
+    if X == 0:
+        return {}
+    B, T = len(lens), int(max(lens)) if len(lens) else 0
+    xk = np.zeros((X, B, cfg.n_kv_heads, T, cfg.head_dim), np.uint16)
+    xv = np.zeros_like(xk)
+    for x in range(X):
+        for b in range(B):
+            n = int(lens[b])
+            xk[x, b, :, :n] = _normal_bf16(rng, (cfg.n_kv_heads, n, cfg.head_dim), 1.0)
+            xv[x, b, :, :n] = _normal_bf16(rng, (cfg.n_kv_heads, n, cfg.head_dim), 1.0)
+    return {"extra_k": xk, "extra_v": xv}
 
 
 def make_dense_context(cfg: LoopConfig, rng: np.random.Generator, ctx_lens) -> dict:
-    """Per-loop bf16 K/V context for the dense looped baseline: uint16 [M, K, B, Hkv, T, hd]."""
+    """bf16 K/V context for the dense looped baseline: uint16 [M, KS, B, Hkv, T, hd],
+    KS = K loop slots (per_loop) or 1 (last_loop)."""
     lens = np.asarray(ctx_lens, dtype=np.int64)
     B, T = len(lens), int(lens.max()) if len(lens) else 0
-    M, K, Hkv, hd = cfg.n_layers, cfg.n_loops, cfg.n_kv_heads, cfg.head_dim
+    M, Hkv, hd = cfg.n_layers, cfg.n_kv_heads, cfg.head_dim
+    K = 1 if cfg.kv_mode == 1 else cfg.n_loops
     kv_k = np.zeros((M, K, B, Hkv, T, hd), np.uint16)
     kv_v = np.zeros_like(kv_k)
     for j in range(M):
@@ -224,7 +272,9 @@ def make_dense_context(cfg: LoopConfig, rng: np.random.Generator, ctx_lens) -> d
                 n = int(lens[b])
                 kv_k[j, l, b, :, :n] = _normal_bf16(rng, (Hkv, n, hd), 1.0)
                 kv_v[j, l, b, :, :n] = _normal_bf16(rng, (Hkv, n, hd), 1.0)
-    return {"lens": lens, "kv_k": kv_k, "kv_v": kv_v}
+    out = {"lens": lens, "kv_k": kv_k, "kv_v": kv_v}
+    out.update(_extra_context(cfg, rng, lens))
+    return out
 
 
 # ----------------------------------------------------------------------------
@@ -255,3 +305,87 @@ def make_residuals(seed: int, n_rows: int, width: int, scale_mix: bool = True) -
         zero_rows = rng.random(n_rows) < 0.05
         r[zero_rows] = 0.0
     return r.astype(np.float32)
+
+
+# ----------------------------------------------------------------------------
+# device-drawn inputs for benchmark workloads too large to draw on the host
+# ----------------------------------------------------------------------------
+# The same distributions as above, drawn on the GPU with torch's seeded
+# generator (Philox) instead of PCG64, so the 17 GB of deep-recurrence weights
+# or a 65536-token context take seconds, not minutes.  The parity tests use the
+# host draws; the benchmark's timings do not depend on which generator drew the
+# values.
+
+def _dev_gen(seed: int, device):
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def _dev_normal_bf16(g, shape, sigma: float, device):
+    import torch
+    x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+    if sigma != 1.0:
+        x.mul_(sigma)
+    return x.to(torch.bfloat16).view(torch.int16)     # round to nearest even, bit patterns
+
+
+def make_weights_device(cfg: LoopConfig, device="cuda", seed: int | None = None) -> dict:
+    """Block weights stacked over layers on the device (bf16 bits as int16,
+    gains float32 ones), in the layout ``flashloop.upload_weights`` returns."""
+    import torch
+    g = _dev_gen(cfg.seed if seed is None else seed, device)
+    M, d, f, hq = cfg.n_layers, cfg.d_model, cfg.ffn_dim, cfg.n_heads * cfg.head_dim
+    out = {"attn_norm": torch.ones((M, d), dtype=torch.float32, device=device),
+           "mlp_norm": torch.ones((M, d), dtype=torch.float32, device=device),
+           "final_norm": torch.ones((d,), dtype=torch.float32, device=device)}
+    shapes = {"w_qkv": (cfg.qkv_rows, d), "w_o": (d, hq), "w_gate": (f, d), "w_up": (f, d), "w_down": (d, f)}
+    for name, shp in shapes.items():
+        t = torch.empty((M,) + shp, dtype=torch.int16, device=device)
+        for j in range(M):              # one layer at a time keeps the fp32 draw small
+            t[j] = _dev_normal_bf16(g, shp, cfg.sigma, device)
+        out[name] = t
+    out["w_out"] = _dev_normal_bf16(g, (cfg.vocab, d), cfg.sigma, device)
+    return out
+
+
+def context_slices_device(cfg: LoopConfig, ctx_lens, device="cuda", seed: int | None = None, dense: bool = False):
+    """Yield one (layer, sequence) slice of a synthetic decode context at a time,
+    drawn on the device, in the import layout of ``flashloop_import_lazy``
+    (``dense``: ``flashloop_import_dense``):
+      lazy : (j, b, base_k, base_v, codes_k, codes_v, scales_k, scales_v) with base
+             bf16 bits [Hkv][n][hd], codes int8 [K-1][Hkv][n][hd], scales fp16 bits
+             [K-1][Hkv][n][hd/g]; for each loop a uniformly random ceil(rho*n)
+             subset of the rows carries codes uniform in [-qmax, qmax] and scales
+             U[0.01, 0.03], the other rows zero (the recipe of ``make_context``)
+      dense: (j, b, kv_k, kv_v) with bf16 bits [KS][Hkv][n][hd], N(0, 1), KS = K loop
+             slots (per_loop) or 1 (last_loop)."""
+    import torch
+    g = _dev_gen((cfg.seed if seed is None else seed) + 7919, device)
+    M, K, Hkv, hd = cfg.n_layers, cfg.n_loops, cfg.n_kv_heads, cfg.head_dim
+    KS = 1 if (dense and cfg.kv_mode == 1) else K
+    for j in range(M):
+        for b, n in enumerate(ctx_lens):
+            n = int(n)
+            if n == 0:
+                continue
+            if dense:
+                yield (j, b, _dev_normal_bf16(g, (KS, Hkv, n, hd), 1.0, device),
+                       _dev_normal_bf16(g, (KS, Hkv, n, hd), 1.0, device))
+                continue
+            ng = hd // cfg.group_size
+            qmax = (1 << (cfg.resid_bits - 1)) - 1
+            m = min(n, int(math.ceil(cfg.rho * n - 1e-9)))
+            base = [_dev_normal_bf16(g, (Hkv, n, hd), 1.0, device) for _ in range(2)]
+            codes = [torch.zeros((max(K - 1, 0), Hkv, n, hd), dtype=torch.int8, device=device) for _ in range(2)]
+            scales = [torch.zeros((max(K - 1, 0), Hkv, n, ng), dtype=torch.float16, device=device) for _ in range(2)]
+            for li in range(K - 1):
+                rows = torch.sort(torch.randperm(n, generator=g, device=device)[:m]).values
+                for w in range(2):
+                    codes[w][li][:, rows] = torch.randint(-qmax, qmax + 1, (Hkv, m, hd), generator=g, device=device,
+                                                          dtype=torch.int8)
+                    scales[w][li][:, rows] = (torch.rand((Hkv, m, ng), generator=g, device=device) * 0.02 + 0.01
+                                              ).to(torch.float16)
+            yield (j, b, base[0], base[1], codes[0], codes[1], scales[0].view(torch.int16),
+                   scales[1].view(torch.int16))

@@ -40,7 +40,8 @@ typedef struct CUstream_st* fl_stream_t; /* a cudaStream_t; NULL = legacy defaul
 typedef enum {
   FL_OK = 0,
   FL_ERR_INVALID_ARG = 1, /* a NULL/misaligned pointer, an out-of-range size or knob */
-  FL_ERR_CAPACITY = 2,    /* batch > max_batch, tokens > max_tokens, or context > max_ctx */
+  FL_ERR_CAPACITY = 2,    /* batch > max_batch, tokens > max_tokens, context > max_ctx, or (from
+                             flashloop_sync_status) a sparse residual pool ran out of rows */
   FL_ERR_WORKSPACE = 3,   /* workspace smaller than flashloop_workspace_bytes() or misaligned */
   FL_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (see flashloop_last_cuda_error) */
   FL_ERR_TIMEOUT = 5,     /* a kernel's bounded wait ran out; the kernel returned early */
@@ -71,7 +72,34 @@ typedef struct {
   int max_batch;    /* sequences held in the cache */
   int max_ctx;      /* positions per sequence held in the cache */
   int max_tokens;   /* largest B*T of one prefill call (decode needs max_batch) */
+  int kv_mode;      /* dense path only: 0 = per_loop (every loop keeps its own KV), 1 = last_loop (one KV
+                       per layer that every loop overwrites, "Looped Transformer 教程", 第四步:
+                       recurrent_kv_cache_mode); must be 0 on the lazy path */
+  /* Variants around the looped core ("从'堆层数'到'循环复用'：FlashLoop 到底在解决什么问题",
+   * §3.1, §3.2, §4.1; "Looped Transformer 教程", 第三步).  All zero: the plain looped block. */
+  int n_prelude;    /* P independent layers before the loop, applied once to every token, own KV */
+  int n_coda;       /* Q independent layers after the loop, likewise */
+  int loop_embed;   /* 1: loop k's input is h + e_k (weights.loop_embed) */
+  float inject_scale; /* gamma: loop k's input also adds gamma * x, x = the state entering the loop */
+  /* Sparse residual storage (lazy path): 0 = one residual row per position and loop; R > 0 = residual rows
+   * are kept only for the tokens a loop recomputed, in a pool of R rows per (layer, loop, K/V, sequence,
+   * KV head) plus a 4-byte row index per (layer, loop, sequence, position) -- the KV-cache memory
+   * reduction of "FlashLoop ...", abstract.  Rows are taken in position order; a call that needs more
+   * than R rows keeps no residual for the excess tokens and flashloop_sync_status reports
+   * FL_ERR_CAPACITY.  0 <= R <= max_ctx. */
+  int resid_rows;
 } flashloop_config;
+
+/* A stack of L layers' weights (device pointers, stacked over layers). */
+typedef struct {
+  const float* attn_norm;     /* [L][d] fp32 gains */
+  const uint16_t* w_qkv;      /* [L][(H+2Hkv)*hd][d] bf16; rows: q heads, k heads, v heads */
+  const uint16_t* w_o;        /* [L][d][H*hd] bf16 */
+  const float* mlp_norm;      /* [L][d] fp32 gains */
+  const uint16_t* w_gate;     /* [L][ffn][d] bf16 */
+  const uint16_t* w_up;       /* [L][ffn][d] bf16 */
+  const uint16_t* w_down;     /* [L][d][ffn] bf16 */
+} flashloop_layers;
 
 /* Device pointers to the weights (borrowed for the context's lifetime). */
 typedef struct {
@@ -84,6 +112,9 @@ typedef struct {
   const uint16_t* w_down;     /* [M][d][ffn] bf16 */
   const float* final_norm;    /* [d] fp32 gains */
   const uint16_t* w_out;      /* [V][d] bf16 */
+  flashloop_layers prelude;   /* n_prelude layers (ignored when 0) */
+  flashloop_layers coda;      /* n_coda layers (ignored when 0) */
+  const float* loop_embed;    /* [K][d] fp32 loop embeddings e_1..e_K (loop_embed = 1; else ignored) */
 } flashloop_weights;
 
 typedef struct flashloop_ctx flashloop_ctx;
@@ -102,13 +133,24 @@ fl_status flashloop_init(const flashloop_config* cfg, const flashloop_weights* w
                          void* workspace, size_t workspace_bytes, fl_stream_t stream,
                          flashloop_ctx** out);
 
-/* Prefill T tokens into each of B empty sequences (lengths must be 0).
+/* Prefill a chunk of T tokens onto each of sequences 0..B-1: token t of
+ * sequence b sits at position len_b + t, after whatever the sequence already
+ * holds (len_b = 0 for a fresh prompt; a later chunk continues a prompt, or
+ * follows decode steps).  The looped block over the call's tokens: loop 1 runs
+ * every token with causal attention over the cache's positions 0..len_b + t;
+ * loops 2..K recompute the top ceil(rho*B*T) tokens by change norm (pooled over
+ * the call, ties to the lower flat index b*T+t) with their attention corrected
+ * over the fixed top-c key columns of their query tile ("FlashLoop: Fast and
+ * Memory-Efficient Looped Transformers via Lazy Updates", abstract: token-sparse
+ * updates, sparse stable key columns, KV residuals); query tiles are q_tile
+ * consecutive tokens of one sequence's chunk, counted from its first token,
+ * and see every earlier column of the sequence.
  * h0: [B*T][d] fp32 input hidden states, sequence-major (host or device).
  * h_out: [B*T][d] fp32 final hidden states after K loops (host or device, may be NULL).
  * logits_last: [B][V] fp32 logits of each sequence's last position (host or device, may be NULL).
- * Loop 1 is dense; loops 2..K recompute ceil(rho*B*T) tokens (pooled over the
- * call, ties to the lower flat index b*T+t).  Query tiles are q_tile
- * positions of one sequence.  On return the sequences' lengths are T. */
+ * Errors: FL_ERR_INVALID_ARG (NULL h0, B or T < 1), FL_ERR_CAPACITY (B >
+ * max_batch, B*T > max_tokens, or len_b + T > max_ctx), FL_ERR_CUDA.  On
+ * return the sequences' lengths have grown by T. */
 fl_status flashloop_prefill(flashloop_ctx* ctx, const float* h0, int B, int T,
                             float* h_out, float* logits_last, fl_stream_t stream);
 
@@ -120,9 +162,14 @@ fl_status flashloop_prefill(flashloop_ctx* ctx, const float* h0, int B, int T,
 fl_status flashloop_decode_step(flashloop_ctx* ctx, const float* h0, int B,
                                 float* h_out, float* logits, fl_stream_t stream);
 
-/* KV-cache bytes: *total = bytes of the allocated cache layout; per token and
- * layer: *per_token_per_layer for this config and *dense_per_token_per_layer
- * for dense per-loop bf16 KV (K * 2 * Hkv * hd * 2 bytes).  Host arithmetic. */
+/* KV-cache bytes ("FlashLoop ...", abstract: the KV-cache memory the residual
+ * form saves): *total = bytes of the allocated cache layout (looped layers, plus
+ * one pass for each prelude / coda layer); per token and looped layer:
+ * *per_token_per_layer for this config (lazy: the bf16 base plus K-1 packed
+ * residual rows and their fp16 scales; dense per_loop: K passes; last_loop:
+ * one) and *dense_per_token_per_layer for dense per-loop bf16 KV (K * 2 * Hkv *
+ * hd * 2 bytes), the reference the reduction is quoted against.  Host
+ * arithmetic; FL_ERR_INVALID_ARG for a NULL context. */
 fl_status flashloop_kv_bytes(const flashloop_ctx* ctx, size_t* total, double* per_token_per_layer,
                              double* dense_per_token_per_layer);
 
@@ -160,10 +207,17 @@ fl_status flashloop_import_lazy(flashloop_ctx* ctx, int layer, int seq, int n,
                                 const uint16_t* scales_k, const uint16_t* scales_v,
                                 fl_stream_t stream);
 
-/* Load one (layer, sequence) slice of a dense per-loop cache: kv_k/kv_v
- * [K][Hkv][n][hd] bf16.  resid_bits 16 only. */
+/* Load one (layer, sequence) slice of a dense cache: kv_k/kv_v [KS][Hkv][n][hd]
+ * bf16, KS = K loops (per_loop) or 1 (last_loop).  resid_bits 16 only. */
 fl_status flashloop_import_dense(flashloop_ctx* ctx, int layer, int seq, int n,
                                  const uint16_t* kv_k, const uint16_t* kv_v, fl_stream_t stream);
+
+/* Load one (independent layer, sequence) slice of the prelude / coda KV: x in
+ * [0, n_prelude) for the prelude, n_prelude + i for coda layer i; kv_k/kv_v
+ * [Hkv][n][hd] bf16 (device buffers).  FL_ERR_INVALID_ARG when x, seq or n is out
+ * of range or a pointer is NULL. */
+fl_status flashloop_import_extra(flashloop_ctx* ctx, int x, int seq, int n, const uint16_t* kv_k,
+                                 const uint16_t* kv_v, fl_stream_t stream);
 
 /* Copy one (layer, loop, sequence) slice of the residual store to device
  * buffers: codes [Hkv][n][hd*bits/8] packed bytes, scales [Hkv][n][hd/g] fp16
@@ -290,9 +344,13 @@ typedef enum {
   FL_OPT_PROFILE = 2,   /* 1: bracket every kernel of a call with CUDA events (read with flashloop_profile) */
   FL_OPT_PDL = 3,       /* 1 (default): launch each kernel of a call as a programmatic dependent of the
                            previous one, so its launch and set-up overlap the predecessor */
-  FL_OPT_FUSE_QKV = 4   /* 0 (default): RoPE and the KV write run in their own kernel; 1: in the QKV GEMM's
-                           epilogue wherever the decode GEMM is split over a cluster (bit-identical results;
-                           measured slower on the decode workload, so off) */
+  FL_OPT_GEMM_TIMES = 5, /* 1: every GEMM launch of a call stamps, from the GPU's global nanosecond timer, when
+                           its first CTA's dependency wait returned and when its last CTA finished (read with
+                           flashloop_gemm_times); 0 (default): off */
+  FL_OPT_TC_PREFILL = 6, /* 1 (default): prefill attention and prefill delta scores on warp-level bf16
+                           tensor-core products (fp32 operands as bf16 hi + lo pairs); 0: the fp32 SIMT kernels */
+  FL_OPT_CORR_CLUSTER = 7 /* 1 (default): a decode query's column correction runs as one 16-CTA cluster merged
+                           over distributed shared memory; 0: column slices merged by an atomic ticket */
 } fl_option;
 fl_status flashloop_set_option(flashloop_ctx* ctx, fl_option opt, int value);
 
@@ -317,6 +375,15 @@ fl_status flashloop_profile(flashloop_ctx* ctx, fl_stream_t stream, float* ms, i
 
 /* Number of kernels the last prefill / decode call enqueued (all kinds). */
 int flashloop_kernels_per_call(const flashloop_ctx* ctx);
+
+/* Device time of the GEMMs of the last call made with FL_OPT_GEMM_TIMES on
+ * (the shared-block projections and the LM head, "FlashLoop ...", abstract:
+ * the recomputed tokens' block): synchronises `stream`, then *total_ms = the
+ * sum over the call's GEMM launches of (last CTA's end - first return from the
+ * dependency wait), so launches never overlap in the sum and it cannot exceed
+ * the call's duration; *launches = the GEMM launches timed.  FL_ERR_INVALID_ARG
+ * when the option is off or a pointer is NULL. */
+fl_status flashloop_gemm_times(flashloop_ctx* ctx, fl_stream_t stream, double* total_ms, int* launches);
 
 #ifdef __cplusplus
 }

@@ -219,6 +219,12 @@ def prepare_weights(w: dict) -> dict:
         })
     out["final_norm"] = np.asarray(w["final_norm"], F64)
     out["w_out"] = f(w["w_out"])
+    for part in ("prelude", "coda"):
+        if part in w:
+            out[part] = prepare_weights({"layers": w[part], "final_norm": w["final_norm"],
+                                         "w_out": w["w_out"][:1]})["layers"]
+    if "loop_embed" in w:
+        out["loop_embed"] = np.asarray(w["loop_embed"], F64)
     return out
 
 
@@ -268,7 +274,10 @@ class KVCache:
       base_k/v [M, B, Hkv, T, hd]   -- loop-1 KV (bf16 values unless exact)
       codes_k/v [M, K-1, B, Hkv, T, hd] int8 and scales_k/v [.., hd/g] float16
       res_k/v  [M, K-1, B, Hkv, T, hd] -- dequantised residual (fp32, or fp64 when exact)
-    Dense layout (bits 16): kv_k/v [M, K, B, Hkv, T, hd] (bf16 values unless exact).
+    Dense layout (bits 16): kv_k/v [M, KS, B, Hkv, T, hd] (bf16 values unless
+    exact), KS = K with per-loop KV ("Looped Transformer 教程", 第四步:
+    per_loop), or 1 in last_loop mode, where each loop overwrites the one slot
+    with its own KV and only the last pass is kept (第四步: last_loop).
     """
 
     def __init__(self, cfg, B: int, tmax: int, kv_exact: bool = False):
@@ -276,9 +285,14 @@ class KVCache:
         self.kv_exact = kv_exact
         self.lens = np.zeros(B, dtype=np.int64)
         M, K, Hkv, hd = cfg.n_layers, cfg.n_loops, cfg.n_kv_heads, cfg.head_dim
+        # prelude and coda layers: one pass of KV each, [P+Q, B, Hkv, T, hd]
+        X = getattr(cfg, "n_prelude", 0) + getattr(cfg, "n_coda", 0)
+        self.xk = np.zeros((X, B, Hkv, tmax, hd), F64)
+        self.xv = np.zeros_like(self.xk)
         self.dense = cfg.resid_bits == 16
         if self.dense:
-            self.kv_k = np.zeros((M, K, B, Hkv, tmax, hd), F64)
+            self.last_loop = getattr(cfg, "kv_mode", 0) == 1
+            self.kv_k = np.zeros((M, 1 if self.last_loop else K, B, Hkv, tmax, hd), F64)
             self.kv_v = np.zeros_like(self.kv_k)
         else:
             exact = cfg.resid_bits == 32
@@ -310,8 +324,15 @@ class KVCache:
             getattr(c, "codes_" + name)[..., :T, :] = codes
             getattr(c, "scales_" + name)[..., :T, :] = scales
             getattr(c, "res_" + name)[..., :T, :] = dequant_groups(codes, scales, g)
+        c._load_extra(ctx, T)
         c.lens[:] = lens
         return c
+
+    def _load_extra(self, ctx, T):
+        if "extra_k" in ctx:
+            to64 = lambda b: (b.astype(np.uint32) << 16).view(F32).astype(F64)
+            self.xk[..., :T, :] = to64(ctx["extra_k"])
+            self.xv[..., :T, :] = to64(ctx["extra_v"])
 
     @classmethod
     def from_dense_context(cls, cfg, ctx: dict, tmax: int):
@@ -321,8 +342,13 @@ class KVCache:
         to64 = lambda b: (b.astype(np.uint32) << 16).view(F32).astype(F64)
         c.kv_k[..., :T, :] = to64(ctx["kv_k"])
         c.kv_v[..., :T, :] = to64(ctx["kv_v"])
+        c._load_extra(ctx, T)
         c.lens[:] = lens
         return c
+
+    def slot(self, l: int) -> int:
+        """Dense KV slot of loop l (1..K): its own, or the single last_loop slot."""
+        return 0 if self.last_loop else l - 1
 
     # -- storage rules -----------------------------------------------------
     def store_kv(self, x: np.ndarray) -> np.ndarray:
@@ -344,6 +370,55 @@ class KVCache:
             r = res[j, l - 2, b][:, rows]
             acc = (acc + r) if exact else (acc + r).astype(F32)
         return acc.astype(F64)
+
+
+# ============================================================================
+# variants around the looped core
+# ============================================================================
+
+def _independent_layer(cfg, lw, cache: KVCache, x: int, h, seq, pos):
+    """One prelude or coda layer: applied once to every token, its own weights
+    and its own one-pass KV (slot x of cache.xk / xv), otherwise the same
+    pre-norm layer as the shared block ("从'堆层数'到'循环复用'", §3.1: the
+    independent first P and last Q layers around the R looped layers)."""
+    tau = 1.0 / math.sqrt(cfg.head_dim)
+    N = h.shape[0]
+    q, k, v = _qkv(cfg, lw, h, pos)
+    for i in range(N):
+        cache.xk[x, seq[i], :, pos[i]] = cache.store_kv(k[i])
+        cache.xv[x, seq[i], :, pos[i]] = cache.store_kv(v[i])
+    O = np.zeros((N, cfg.n_heads, cfg.head_dim))
+    for i in range(N):
+        O[i], _ = _attn_full(q[i], cache.xk[x, seq[i]][:, :pos[i] + 1], cache.xv[x, seq[i]][:, :pos[i] + 1], tau)
+    h = h + cfg.resid_scale * (O.reshape(N, -1) @ lw["w_o"].T)
+    return _mlp_update(cfg, lw, h)
+
+
+def _loop_input(cfg, W, l: int, h_rows, x_rows):
+    """The state a token enters loop l with: h + e_l when loop embeddings are on
+    (same page, §3.2 and §4.1: each loop's input adds a learned loop
+    embedding) + gamma * x with input injection ("Looped Transformer 教程",
+    第三步: every loop also receives the input representation), x being the
+    token's state when it entered the loop stack."""
+    u = np.asarray(h_rows, F64)
+    if "loop_embed" in W:
+        u = u + W["loop_embed"][l - 1]
+    if getattr(cfg, "inject_scale", 0.0):
+        u = u + cfg.inject_scale * np.asarray(x_rows, F64)
+    return u
+
+
+def _prelude(cfg, W, cache, h, seq, pos):
+    for x, lw in enumerate(W.get("prelude", [])):
+        h = _independent_layer(cfg, lw, cache, x, h, seq, pos)
+    return h
+
+
+def _coda(cfg, W, cache, h, seq, pos):
+    P = len(W.get("prelude", []))
+    for x, lw in enumerate(W.get("coda", [])):
+        h = _independent_layer(cfg, lw, cache, P + x, h, seq, pos)
+    return h
 
 
 # ============================================================================
@@ -377,7 +452,9 @@ def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None):
     M, K, s_res = cfg.n_layers, cfg.n_loops, cfg.resid_scale
     exact = cfg.resid_bits == 32
     N = h0.shape[0]
-    h = np.asarray(h0, F64).copy()
+    h = _prelude(cfg, W, cache, np.asarray(h0, F64).copy(), seq, pos)
+    x_in = h.copy()                     # the state entering the loop stack
+    h = _loop_input(cfg, W, 1, h, x_in)
     O = np.zeros((M, N, H, hd))
     lse = np.zeros((M, N, H))
     qlast = np.zeros((M, N, H, hd))
@@ -400,7 +477,7 @@ def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None):
         h = h + s_res * (O[j].reshape(N, H * hd) @ lw["w_o"].T)
         h = _mlp_update(cfg, lw, h)
         trace["applications"] += 1
-    key = np.sum((h - np.asarray(h0, F64)) ** 2, axis=1).astype(F32)
+    key = np.sum((h - x_in) ** 2, axis=1).astype(F32)
     trace["h"] = {1: h.copy()}
 
     n_sel = n_select(cfg.rho, N)
@@ -412,6 +489,7 @@ def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None):
             S = select_top(key, n_sel).astype(np.int64)
         trace["sel"][l] = S.astype(np.int32)
         h_prev = h[S].copy()
+        h[S] = _loop_input(cfg, W, l, h[S], x_in[S])
         for j, lw in enumerate(W["layers"]):
             q, k, v = _qkv(cfg, lw, h[S], pos[S])
             # residual rows of loop l: zero for every token of the call ...
@@ -498,6 +576,8 @@ def _run_lazy(cfg, W, cache: KVCache, h0, seq, pos, tile, forced=None):
         key[S] = np.sum((h[S] - h_prev) ** 2, axis=1).astype(F32)
         trace["h"][l] = h.copy()
     trace["O"], trace["lse"] = O, lse
+    h = _coda(cfg, W, cache, h, seq, pos)
+    trace["independent"] = len(W.get("prelude", [])) + len(W.get("coda", []))
     return h, trace
 
 
@@ -511,23 +591,27 @@ def _run_dense(cfg, W, cache: KVCache, h0, seq, pos):
     H, hd = cfg.n_heads, cfg.head_dim
     tau = 1.0 / math.sqrt(hd)
     N = h0.shape[0]
-    h = np.asarray(h0, F64).copy()
+    h = _prelude(cfg, W, cache, np.asarray(h0, F64).copy(), seq, pos)
+    x_in = h.copy()
     apps = 0
     for l in range(1, cfg.n_loops + 1):
+        h = _loop_input(cfg, W, l, h, x_in)
         for j, lw in enumerate(W["layers"]):
             q, k, v = _qkv(cfg, lw, h, pos)
+            sl = cache.slot(l)
             for i in range(N):
-                cache.kv_k[j, l - 1, seq[i], :, pos[i]] = cache.store_kv(k[i])
-                cache.kv_v[j, l - 1, seq[i], :, pos[i]] = cache.store_kv(v[i])
+                cache.kv_k[j, sl, seq[i], :, pos[i]] = cache.store_kv(k[i])
+                cache.kv_v[j, sl, seq[i], :, pos[i]] = cache.store_kv(v[i])
             O = np.zeros((N, H, hd))
             for i in range(N):
-                kk = cache.kv_k[j, l - 1, seq[i]][:, :pos[i] + 1]
-                vv = cache.kv_v[j, l - 1, seq[i]][:, :pos[i] + 1]
+                kk = cache.kv_k[j, sl, seq[i]][:, :pos[i] + 1]
+                vv = cache.kv_v[j, sl, seq[i]][:, :pos[i] + 1]
                 O[i], _ = _attn_full(q[i], kk, vv, tau)
             h = h + cfg.resid_scale * (O.reshape(N, H * hd) @ lw["w_o"].T)
             h = _mlp_update(cfg, lw, h)
             apps += 1
-    return h, {"applications": apps}
+    h = _coda(cfg, W, cache, h, seq, pos)
+    return h, {"applications": apps, "independent": len(W.get("prelude", [])) + len(W.get("coda", []))}
 
 
 def _call(cfg, W, cache, h0, seq, pos, tile, forced):
@@ -537,18 +621,23 @@ def _call(cfg, W, cache, h0, seq, pos, tile, forced):
 
 
 def prefill(cfg, W, cache: KVCache, h0: np.ndarray, B: int, T: int, forced=None) -> Result:
-    """Prefill T tokens for each of B empty sequences; h0 is [B*T, d] (sequence-major).
-
-    Query tiles are q_tile consecutive positions of one sequence; the token
-    ranking pools all B*T tokens by flat index b*T + t.  Logits are for the
-    last position of each sequence.
+    """Prefill a chunk of T tokens onto each of sequences 0..B-1; h0 is [B*T, d]
+    (sequence-major).  Token t of sequence b sits at position lens[b] + t, after
+    what the sequence already holds (nothing for a fresh prompt; a later chunk
+    of the prompt, or decoded tokens, otherwise) and attends to every earlier
+    position.  Query tiles are q_tile consecutive tokens of one sequence's
+    chunk, counted from the chunk's first token; the token ranking pools all
+    B*T tokens by flat index b*T + t.  Logits are for the last position of each
+    sequence.
     """
-    assert np.all(cache.lens[:B] == 0), "prefill needs empty sequences"
+    start = cache.lens[:B].copy()
+    assert np.all(start + T <= cache.tmax), "the chunk does not fit the cache"
     seq = np.repeat(np.arange(B), T)
-    pos = np.tile(np.arange(T), B)
-    tile = seq * ((T + cfg.q_tile - 1) // cfg.q_tile) + pos // cfg.q_tile
+    rel = np.tile(np.arange(T), B)
+    pos = start[seq] + rel
+    tile = seq * ((T + cfg.q_tile - 1) // cfg.q_tile) + rel // cfg.q_tile
     h, trace = _call(cfg, W, cache, h0, seq, pos, tile, forced)
-    cache.lens[:B] = T
+    cache.lens[:B] = start + T
     last_rows = np.arange(B) * T + (T - 1)
     return Result(h, _logits(cfg, W, h[last_rows]), trace)
 

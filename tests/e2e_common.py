@@ -60,6 +60,8 @@ def forced_codes(cfg, cache, trace, seq, pos):
 
 
 def run_prefill(cfg, B, T, forced=True, dense=False):
+    """forced: True hands over selections, column sets and codes; "sel" hands
+    over selections and codes only; False hands over nothing."""
     import torch
     from cross_loop_sparsity_b200 import flashloop as fl
     from oracle import flashloop_oracle as orc
@@ -73,7 +75,11 @@ def run_prefill(cfg, B, T, forced=True, dense=False):
     eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=T, max_tokens=B * T)
     n_tiles = B * ((T + cfg.q_tile - 1) // cfg.q_tile)
     if forced and not dense and cfg.n_loops > 1:
-        eng.force_selection(*forced_arrays(cfg, ref.trace, n_tiles), n_tiles=n_tiles)
+        sel, cols, ncols = forced_arrays(cfg, ref.trace, n_tiles)
+        if forced == "sel":   # token selections and codes handed over, column sets left free
+            eng.force_selection(sel)
+        else:
+            eng.force_selection(sel, cols, ncols, n_tiles=n_tiles)
         seq, pos = np.repeat(np.arange(B), T), np.tile(np.arange(T), B)
         eng.force_codes(*forced_codes(cfg, ocache, ref.trace, seq, pos))
     h_out = torch.empty((B * T, cfg.d_model), dtype=torch.float32, device="cuda")
@@ -93,9 +99,10 @@ def load_context(eng, cfg, ctx, dense=False):
     eng.load_context(ctx, dense)
 
 
-def run_decode(cfg, lens, forced=True, dense=False, steps=1, extra_ctx=0):
+def run_decode(cfg, lens, forced=True, dense=False, steps=1, extra_ctx=0, options=None):
     """forced: True hands over selections, column sets and codes; "sel" hands
-    over selections and codes only; False hands over nothing."""
+    over selections and codes only; False hands over nothing.  options: library
+    options (FL_OPT_*) set on the context first."""
     import torch
     from cross_loop_sparsity_b200 import flashloop as fl
     from oracle import flashloop_oracle as orc
@@ -109,6 +116,8 @@ def run_decode(cfg, lens, forced=True, dense=False, steps=1, extra_ctx=0):
     ctx = synth.make_dense_context(cfg, rng, lens) if dense else synth.make_context(cfg, rng, lens)
     cache = orc.KVCache.from_dense_context(cfg, ctx, tmax) if dense else orc.KVCache.from_context(cfg, ctx, tmax)
     eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=tmax, max_tokens=0)
+    for opt, val in (options or {}).items():
+        eng.set_option(opt, val)
     load_context(eng, cfg, ctx, dense)
     results = []
     for _ in range(steps):
@@ -132,3 +141,65 @@ def run_decode(cfg, lens, forced=True, dense=False, steps=1, extra_ctx=0):
             out["sel"], out["keys"], out["cols"], out["ncols"] = eng.read_trace(B, n_sel, B)
         results.append((ref, out))
     return cfg, cache, eng, results
+
+
+def run_calls(cfg, B, ctx_lens, chunks, dense=False, decode_after=0, forced=True):
+    """Oracle and library through the same calls: an optional synthetic context,
+    prefill chunks of the given sizes, then decode steps."""
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    from oracle import flashloop_oracle as orc
+    if dense:
+        cfg = cfg.with_(resid_bits=16)
+    w = synth.make_weights(cfg)
+    rng = w["rng"]
+    W = orc.prepare_weights(w)
+    tmax = max(ctx_lens) + sum(chunks) + decode_after
+    if max(ctx_lens) > 0:
+        ctx = synth.make_dense_context(cfg, rng, ctx_lens) if dense else synth.make_context(cfg, rng, ctx_lens)
+        cache = (orc.KVCache.from_dense_context if dense else orc.KVCache.from_context)(cfg, ctx, tmax)
+    else:
+        ctx, cache = None, orc.KVCache(cfg, B, tmax)
+    eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=tmax, max_tokens=B * max(chunks, default=0))
+    if ctx is not None:
+        eng.load_context(ctx, dense)
+    out = []
+    for T in chunks:
+        h0 = synth.make_h0(cfg, rng, B * T)
+        start = cache.lens[:B].copy()
+        ref = orc.prefill(cfg, W, cache, h0, B, T)
+        n_tiles = B * ((T + cfg.q_tile - 1) // cfg.q_tile)
+        if forced and not dense and cfg.n_loops > 1:
+            eng.force_selection(*forced_arrays(cfg, ref.trace, n_tiles), n_tiles=n_tiles)
+            seq = np.repeat(np.arange(B), T)
+            pos = start[seq] + np.tile(np.arange(T), B)
+            eng.force_codes(*forced_codes(cfg, cache, ref.trace, seq, pos))
+        h_out = torch.empty((B * T, cfg.d_model), dtype=torch.float32, device="cuda")
+        logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+        eng.prefill(torch.from_numpy(h0).cuda(), B, T, h_out, logits)
+        torch.cuda.synchronize()
+        out.append((ref, {"h": h_out.cpu().numpy(), "logits": logits.cpu().numpy(), "status": eng.sync_status()}))
+    for _ in range(decode_after):
+        h0 = synth.make_h0(cfg, rng, B)
+        pos = cache.lens[:B].copy()
+        ref = orc.decode_step(cfg, W, cache, h0)
+        if forced and not dense and cfg.n_loops > 1:
+            sel, cols, ncols = forced_arrays(cfg, ref.trace, B)
+            eng.force_selection(sel, cols, ncols, n_tiles=B)
+            eng.force_codes(*forced_codes(cfg, cache, ref.trace, np.arange(B), pos))
+        h_out = torch.empty((B, cfg.d_model), dtype=torch.float32, device="cuda")
+        logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+        eng.decode_step(torch.from_numpy(h0).cuda(), B, h_out, logits)
+        torch.cuda.synchronize()
+        out.append((ref, {"h": h_out.cpu().numpy(), "logits": logits.cpu().numpy(), "status": eng.sync_status()}))
+    eng.close()
+    return out
+
+
+def check_all(results, tol=TOL):
+    """Every call's hidden states and logits within tol x RMS of the oracle's."""
+    for ref, o in results:
+        assert o["status"] == 0
+        eh, el = rel_err(o["h"], ref.h), rel_err(o["logits"], ref.logits)
+        assert eh <= tol, eh
+        assert el <= tol, el

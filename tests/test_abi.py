@@ -98,3 +98,41 @@ def test_unit_entry_points_reject_bad_sizes(L):
     assert L.fl_test_topk(None, 1, 10, 3, None, None) == 1
     assert L.fl_test_gemm(None, None, None, 1, 1, 8, 0, None, 0, None) == 1
     assert L.fl_test_gemm_scratch_bytes(65, 128, 64, 1) == 0
+
+
+def test_last_loop_kv_bytes_are_one_pass(L):
+    """last_loop keeps one pass of dense KV: K times fewer bytes than per_loop."""
+    from cross_loop_sparsity_b200 import flashloop as fl
+    cfg = synth.config("c2").with_(resid_bits=16)
+    per = fl.kv_bytes_for(fl.make_config(cfg, 8, 4097))
+    last = fl.kv_bytes_for(fl.make_config(cfg.with_(kv_mode=1), 8, 4097))
+    assert per[1] == per[2] == cfg.n_loops * last[1]
+    assert last[2] == per[2] and per[0] == cfg.n_loops * last[0]
+    # last_loop is a dense-path mode: the lazy path rejects it
+    bad = fl.make_config(cfg.with_(resid_bits=4, kv_mode=1), 8, 4097)
+    assert L.flashloop_workspace_bytes(bad) == 0
+
+
+@pytest.mark.parametrize("name,floor", [("c2", 3.5), ("c5", 5.0), ("c5_int2", 5.0)])
+def test_sparse_residual_storage_kv_bytes(L, name, floor):
+    """Residual rows for the recomputed tokens only (a pool sized to the
+    context's recompute rate plus the batch's new tokens) and a 4-byte row index
+    per (layer, loop, position): bf16 base + (K-1) x (pool fraction x row bytes
+    + 4) per token and layer."""
+    cfg = synth.config(name)
+    rows = synth.sparse_rows(cfg, cfg.batch)
+    c = fl.make_config(cfg.with_(resid_rows=rows), cfg.batch, cfg.max_ctx)
+    tot, per, dense = fl.kv_bytes_for(c)
+    kv, hd, K = 2 * cfg.n_kv_heads, cfg.head_dim, cfg.n_loops
+    row = hd * cfg.resid_bits / 8 + (hd // cfg.group_size) * 2
+    assert per == pytest.approx(kv * hd * 2 + (K - 1) * (kv * row * rows / cfg.max_ctx + 4))
+    assert dense / per >= floor
+    # the dense layout of the same config keeps every position's residual rows
+    _, per_dense_layout, _ = fl.kv_bytes_for(fl.make_config(cfg, cfg.batch, cfg.max_ctx))
+    assert per < per_dense_layout
+    assert L.flashloop_workspace_bytes(ctypes.byref(c)) > 0
+    # the pool cannot be larger than the context, and is a lazy-path layout
+    assert L.flashloop_workspace_bytes(ctypes.byref(fl.make_config(cfg.with_(resid_rows=cfg.max_ctx + 1), cfg.batch,
+                                                                   cfg.max_ctx))) == 0
+    assert L.flashloop_workspace_bytes(ctypes.byref(fl.make_config(cfg.with_(resid_rows=rows, resid_bits=16),
+                                                                   cfg.batch, cfg.max_ctx))) == 0

@@ -84,9 +84,13 @@ def test_prefill_single_loop_is_a_plain_block():
 
 
 # ---------------------------------------------------------------- decode
-def test_decode_ragged_lengths_forced():
+@pytest.mark.parametrize("cluster", [1, 0])
+def test_decode_ragged_lengths_forced(cluster):
+    """cluster 0: the decode correction's column slices merged by an atomic
+    ticket instead of over a cluster's distributed shared memory."""
+    from cross_loop_sparsity_b200 import flashloop as fl
     cfg = synth.config("c1").with_(mode="decode", batch=3, rho=0.5, c_cols=24, seed=7, seq_len=0)
-    cfg, cache, eng, results = E.run_decode(cfg, [300, 77, 1], steps=2)
+    cfg, cache, eng, results = E.run_decode(cfg, [300, 77, 1], steps=2, options={fl.FL_OPT_CORR_CLUSTER: cluster})
     for ref, out in results:
         _check_outputs(ref, out)
 
@@ -136,6 +140,20 @@ def test_decode_c2_free_column_sets():
         print(f"column sets: {exact} of {n_sets} identical to the oracle's; at most {swaps} swaps, "
               f"boundary distance <= {dist:.2e} of the largest key")
         _check_outputs(ref, out, tol=2 * E.TOL)
+
+
+def test_prefill_long_block_free_column_sets():
+    """Prefill tiles of the long-prefill block (head_dim 128: the tensor-core
+    delta-score kernel) choose their own column sets from the oracle's
+    selections and codes: each set has the oracle's size and differs only at
+    the top-c boundary."""
+    cfg = synth.config("c3").with_(n_layers=2, seq_len=1024, seed=131)
+    cfg, ref, eng, out = E.run_prefill(cfg, 1, 1024, forced="sel")
+    assert out["status"] == 0
+    exact, swaps, dist = _check_free_column_sets(cfg, ref, out, max_swaps=cfg.c_cols // 16, key_tol=2e-2)
+    print(f"column sets: {exact} of {len(ref.trace['cols'])} identical; at most {swaps} swaps, boundary "
+          f"distance <= {dist:.2e} of the largest key")
+    _check_outputs(ref, out, tol=2 * E.TOL)
 
 
 def test_decode_ragged_free_column_sets():
@@ -193,49 +211,6 @@ def test_decode_graph_replay_matches_direct_launches():
         assert np.array_equal(a, b)
 
 
-def test_decode_fused_rope_kv_matches_separate_kernel():
-    """RoPE, q and the KV store / residual quantise done in the QKV GEMM's
-    epilogue give bit for bit what the separate kernel gives: logits, hidden
-    states and every exported KV slice, free running over two steps."""
-    import torch
-    from cross_loop_sparsity_b200 import flashloop as fl
-    cfg = synth.config("c2").with_(ctx_len=700, rho=0.5, seed=29)
-    B = cfg.batch
-    lens = [700, 5, 300, 64, 1, 640, 129, 12][:B]
-    outs = []
-    for fuse in (1, 0):
-        w = synth.make_weights(cfg)
-        rng = w["rng"]
-        ctx = synth.make_context(cfg, rng, lens)
-        eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=max(lens) + 2)
-        E.load_context(eng, cfg, ctx)
-        eng.set_option(fl.FL_OPT_FUSE_QKV, fuse)
-        s = torch.cuda.Stream()
-        res = []
-        for _ in range(2):
-            h0 = torch.from_numpy(synth.make_h0(cfg, rng, B)).cuda()
-            h_out = torch.empty((B, cfg.d_model), dtype=torch.float32, device="cuda")
-            lg = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
-            torch.cuda.synchronize()
-            eng.decode_step(h0, B, h_out, lg, stream=s)
-            s.synchronize()
-            res += [lg.cpu().numpy(), h_out.cpu().numpy()]
-        assert eng.sync_status(s) == 0
-        for layer in range(cfg.n_layers):
-            for loop in range(1, cfg.n_loops + 1):
-                for b in (0, 4, 5):
-                    for which in (0, 1):
-                        c_, s_ = eng.export_slice(layer, loop, b, which, lens[b] + 2)
-                        res.append(c_)
-                        if s_ is not None:
-                            res.append(s_.view(np.uint16))
-        outs.append(res)
-        eng.close()
-    assert len(outs[0]) == len(outs[1])
-    for a, b in zip(*outs):
-        assert np.array_equal(a, b)
-
-
 def test_decode_free_running_selection_and_column_sets_are_valid():
     cfg = synth.config("c1").with_(mode="decode", batch=6, rho=0.4, c_cols=20, seed=19, seq_len=0)
     lens = [90, 33, 7, 64, 120, 1]
@@ -255,3 +230,43 @@ def test_decode_free_running_selection_and_column_sets_are_valid():
                     assert n == min(cfg.c_cols, P + 1)
                     C = out["cols"][j, t, g, :n]
                     assert np.all(np.diff(C) > 0) and C[0] >= 0 and C[-1] <= P
+
+
+@pytest.mark.parametrize("name,B,T,ctx", [("c1", 2, 200, 0), ("c3", 1, 700, 0), ("c3", 1, 300, 500)])
+def test_prefill_attention_tensor_core_and_simt_agree(name, B, T, ctx):
+    """The tensor-core prefill attention (bf16 products, Q and P as hi + lo
+    pairs) and the fp32 SIMT kernel give the same call within the end-to-end
+    tolerance of the oracle and within 2e-3 x RMS of each other, head_dim 64 and
+    128, a fresh prompt and a chunk onto a residual context."""
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl
+    from oracle import flashloop_oracle as orc
+    cfg = synth.config(name).with_(seed=111, n_layers=2, n_loops=2, seq_len=T)
+    w = synth.make_weights(cfg)
+    rng = w["rng"]
+    W = orc.prepare_weights(w)
+    ctx_arr = synth.make_context(cfg, rng, [ctx] * B) if ctx else None
+    h0 = synth.make_h0(cfg, rng, B * T)
+    cache = orc.KVCache.from_context(cfg, ctx_arr, ctx + T) if ctx else orc.KVCache(cfg, B, T)
+    ref = orc.prefill(cfg, W, cache, h0, B, T)
+    n_tiles = B * ((T + cfg.q_tile - 1) // cfg.q_tile)
+    seq = np.repeat(np.arange(B), T)
+    pos = ctx + np.tile(np.arange(T), B)
+    outs = []
+    for tc in (1, 0):
+        eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=ctx + T, max_tokens=B * T)
+        if ctx:
+            eng.load_context(ctx_arr)
+        eng.set_option(fl.FL_OPT_TC_PREFILL, tc)
+        eng.force_selection(*E.forced_arrays(cfg, ref.trace, n_tiles), n_tiles=n_tiles)
+        eng.force_codes(*E.forced_codes(cfg, cache, ref.trace, seq, pos))
+        h_out = torch.empty((B * T, cfg.d_model), dtype=torch.float32, device="cuda")
+        logits = torch.empty((B, cfg.vocab), dtype=torch.float32, device="cuda")
+        eng.prefill(torch.from_numpy(h0).cuda(), B, T, h_out, logits)
+        torch.cuda.synchronize()
+        assert eng.sync_status() == 0
+        outs.append(h_out.cpu().numpy())
+        assert E.rel_err(outs[-1], ref.h) <= E.TOL
+        assert E.rel_err(logits.cpu().numpy(), ref.logits) <= E.TOL
+        eng.close()
+    assert E.rel_err(outs[0], outs[1]) <= 2e-3

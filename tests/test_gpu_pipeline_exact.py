@@ -19,10 +19,9 @@ inputs and the library's exported cache:
   asc), checked with a plain sort.
 * Token selections: a valid top-n_sel of the library's own change keys.
 
-Prefill goes through the wide GEMM and the separate RoPE / KV kernel; decode
-through the QKV GEMM whose epilogue quantises (and, switched off, the separate
-kernel), so both quantiser sites are covered, int4 and int2, head_dim 64 and
-128, groups 32 and 64, loops 2..8.
+Prefill (wide GEMM) and decode (split-K GEMM) both feed the RoPE / KV kernel,
+whose quantiser is covered at int4 and int2, head_dim 64 and 128 (two and four
+values per lane), groups 32 and 64, loops 2..8.
 """
 import numpy as np
 import pytest
@@ -123,23 +122,31 @@ def _traces(torch, cfg, n_slots, n_tiles, max_ctx):
     return kv, ck
 
 
-@pytest.mark.parametrize("case", ["c1_two_sequences", "c3_block_1024"])
+@pytest.mark.parametrize("case", ["c1_two_sequences", "c3_block_1024", "c1_chunk_onto_context"])
 def test_prefill_free_running_codes_and_column_sets_bit_exact(case):
     import torch
     from cross_loop_sparsity_b200 import flashloop as fl
     from oracle import flashloop_oracle as orc
+    lens = None
     if case == "c1_two_sequences":
         cfg, B, T = synth.config("c1").with_(seq_len=200, seed=41), 2, 200
-    else:
+    elif case == "c3_block_1024":
         cfg, B, T = synth.config("c3").with_(n_layers=2, n_loops=3, seq_len=1024, seed=43), 1, 1024
+    else:   # a chunk continuing sequences whose context already holds residual levels
+        cfg, B, T, lens = synth.config("c1").with_(seq_len=150, seed=45, c_cols=24), 2, 150, [220, 60]
     w = synth.make_weights(cfg)
-    h0 = synth.make_h0(cfg, w["rng"], B * T)
-    eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=T, max_tokens=B * T)
+    rng = w["rng"]
+    ctx = synth.make_context(cfg, rng, lens) if lens else None
+    h0 = synth.make_h0(cfg, rng, B * T)
+    lens = lens or [0] * B
+    eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=max(lens) + T, max_tokens=B * T)
+    if ctx is not None:
+        eng.load_context(ctx)
     N = B * T
     n_sel = orc.n_select(cfg.rho, N)
     tps = (T + cfg.q_tile - 1) // cfg.q_tile
     n_tiles = B * tps
-    kv, ck = _traces(torch, cfg, n_sel, n_tiles, T)
+    kv, ck = _traces(torch, cfg, n_sel, n_tiles, max(lens) + T)
     eng.set_trace(kv, n_sel, ck, n_tiles)
     eng.prefill(torch.from_numpy(h0).cuda(), B, T)
     torch.cuda.synchronize()
@@ -147,9 +154,10 @@ def test_prefill_free_running_codes_and_column_sets_bit_exact(case):
     sel, keys, cols, ncols = eng.read_trace(N, n_sel, n_tiles)
     for l in range(2, cfg.n_loops + 1):
         assert E.top_valid(keys[l - 2], n_sel, sel[l - 2]), l
-    seq_of, pos_of = np.repeat(np.arange(B), T), np.tile(np.arange(T), B)
-    tile_of = seq_of * tps + pos_of // cfg.q_tile
-    n = _check_codes(cfg, eng, sel, kv.cpu().numpy(), seq_of, pos_of, list(range(N)), [T] * B)
+    seq_of, rel = np.repeat(np.arange(B), T), np.tile(np.arange(T), B)
+    pos_of = np.asarray(lens)[seq_of] + rel
+    tile_of = seq_of * tps + rel // cfg.q_tile
+    n = _check_codes(cfg, eng, sel, kv.cpu().numpy(), seq_of, pos_of, list(range(N)), [l + T for l in lens])
     assert n == cfg.n_layers * (cfg.n_loops - 1) * 2 * n_sel
     assert _check_column_sets(cfg, sel, cols, ncols, ck.cpu().numpy(), tile_of, pos_of) > 0
     eng.close()
@@ -158,13 +166,18 @@ def test_prefill_free_running_codes_and_column_sets_bit_exact(case):
 DECODE_CASES = {
     # tiny block, int4 g32, head_dim 64, ragged contexts, several recomputed tokens
     "c1_ragged": (synth.config("c1").with_(mode="decode", batch=3, rho=0.5, c_cols=24, seed=47, seq_len=0),
-                  [300, 77, 1], 2, 1),
-    # the full decode workload: 8 x 4096, int4 g64, head_dim 128 (quantised in the QKV epilogue)
-    "c2_full": (synth.config("c2"), [4096] * 8, 1, 1),
-    # the same through the separate RoPE / KV kernel
-    "c2_separate_kernel": (synth.config("c2").with_(ctx_len=1500, seed=53), [1500, 700, 3, 1200], 1, 0),
+                  [300, 77, 1], 2),
+    # the full decode workload: 8 x 4096, int4 g64, head_dim 128
+    "c2_full": (synth.config("c2"), [4096] * 8, 1),
+    # ragged contexts of the decode block, two recomputed tokens per loop
+    "c2_ragged": (synth.config("c2").with_(ctx_len=1500, seed=53, rho=0.5), [1500, 700, 3, 1200], 1),
     # K = 8 loops, int2, ragged contexts, two recomputed tokens per loop
-    "c5_int2_ragged": (synth.config("c5_int2").with_(batch=3, rho=0.5, ctx_len=3000, seed=59), [3000, 1700, 64], 2, 1),
+    "c5_int2_ragged": (synth.config("c5_int2").with_(batch=3, rho=0.5, ctx_len=3000, seed=59), [3000, 1700, 64], 2),
+    # contexts longer than one shared-memory slice of column keys: the top-c is
+    # taken per slice and then over the slices' candidates
+    "c5_long_slices": (synth.config("c5").with_(batch=2, rho=0.5, ctx_len=40000, seed=61), [40000, 20001], 1),
+    # the full decode workload with sparse residual storage (rows for recomputed tokens only)
+    "c2_full_sparse": (synth.config("c2").with_(resid_rows=synth.sparse_rows(synth.config("c2"), 8)), [4096] * 8, 1),
 }
 
 
@@ -173,7 +186,7 @@ def test_decode_free_running_codes_and_column_sets_bit_exact(case):
     import torch
     from cross_loop_sparsity_b200 import flashloop as fl
     from oracle import flashloop_oracle as orc
-    cfg, lens, steps, fuse = DECODE_CASES[case]
+    cfg, lens, steps = DECODE_CASES[case]
     B = len(lens)
     w = synth.make_weights(cfg)
     rng = w["rng"]
@@ -182,7 +195,6 @@ def test_decode_free_running_codes_and_column_sets_bit_exact(case):
     eng = fl.FlashLoop(cfg, fl.upload_weights(w), max_batch=B, max_ctx=max_ctx)
     eng.load_context(ctx)
     del ctx
-    eng.set_option(fl.FL_OPT_FUSE_QKV, fuse)
     n_sel = orc.n_select(cfg.rho, B)
     kv, ck = _traces(torch, cfg, n_sel, B, max_ctx)
     eng.set_trace(kv, n_sel, ck, B)

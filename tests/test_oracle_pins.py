@@ -618,6 +618,195 @@ def test_lazy_prefill_pooled_sequences_match_materialised_brute_force(seed, B, T
 
 
 # ----------------------------------------------------------------------------
+# chunked prefill onto an existing cache, and the last_loop KV mode
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed,lens,T,qt,c,bits", [(81, [7, 3], 6, 4, 3, 4), (82, [5, 9, 2], 5, 8, 4, 2)])
+def test_lazy_chunked_prefill_over_residual_context_matches_materialised_brute_force(seed, lens, T, qt, c, bits):
+    """A prefill chunk continues sequences that already hold tokens with
+    residual levels: positions lens[b] + t, tiles counted from the chunk start,
+    columns over the whole causal prefix (context and chunk)."""
+    B = len(lens)
+    cfg = _tiny_cfg(seed=seed, seq_len=T, batch=B, q_tile=qt, c_cols=c, rho=0.3, n_loops=4, resid_bits=bits,
+                    ctx_len=max(lens))
+    W, rng = _weights(cfg)
+    ctx = synth.make_context(cfg, rng, lens)
+    cache = orc.KVCache.from_context(cfg, ctx, max(lens) + T)
+    h0 = synth.make_h0(cfg, rng, B * T)
+    res = orc.prefill(cfg, W, cache, h0, B, T)
+    assert np.array_equal(cache.lens, np.asarray(lens) + T)
+    seq = np.repeat(np.arange(B), T)
+    rel = np.tile(np.arange(T), B)
+    pos = np.asarray(lens)[seq] + rel
+    tile = seq * ((T + qt - 1) // qt) + rel // qt
+    quant = lambda r: orc.quantize_groups(r, cfg.resid_bits, cfg.group_size)
+    bh, bsel, bcols, bstored = _brute_lazy_call(cfg, W, h0, seq, pos, tile, ctx, quant)
+    _compare_with_brute(cfg, res, cache, seq, pos, bh, bsel, bcols, bstored)
+    # the column sets really reach into the context
+    assert any(C.min() < min(lens) for C in bcols.values())
+
+
+def test_lazy_chunked_prefill_dense_limit():
+    """rho = 1, every column and an exact residual: a chunk over a residual
+    context equals the dense per-loop chunk over the same context."""
+    lens, T = np.array([6, 2]), 5
+    cfg = _tiny_cfg(rho=1.0, c_cols=10 ** 6, resid_bits=32, seq_len=T, batch=2, n_loops=3, q_tile=4)
+    W, rng = _weights(cfg)
+    M, K, Hkv, hd = cfg.n_layers, cfg.n_loops, cfg.n_kv_heads, cfg.head_dim
+    tmax = int(lens.max()) + T
+    lazy_c = orc.KVCache(cfg, 2, tmax, kv_exact=True)
+    dcfg = cfg.with_(resid_bits=16)
+    dense_c = orc.KVCache(dcfg, 2, tmax, kv_exact=True)
+    base_k, base_v = (rng.standard_normal((M, 2, Hkv, tmax, hd)) for _ in range(2))
+    res_k, res_v = (rng.standard_normal((M, K - 1, 2, Hkv, tmax, hd)) * 0.1 for _ in range(2))
+    for b in range(2):
+        base_k[:, b, :, lens[b]:] = base_v[:, b, :, lens[b]:] = 0
+        res_k[:, :, b, :, lens[b]:] = res_v[:, :, b, :, lens[b]:] = 0
+    lazy_c.base_k[:], lazy_c.base_v[:], lazy_c.res_k[:], lazy_c.res_v[:] = base_k, base_v, res_k, res_v
+    dense_c.kv_k[:, 0], dense_c.kv_v[:, 0] = base_k, base_v
+    dense_c.kv_k[:, 1:] = base_k[:, None] + np.cumsum(res_k, axis=1)
+    dense_c.kv_v[:, 1:] = base_v[:, None] + np.cumsum(res_v, axis=1)
+    lazy_c.lens[:] = dense_c.lens[:] = lens
+    h0 = synth.make_h0(cfg, rng, 2 * T)
+    a = orc.prefill(cfg, W, lazy_c, h0, 2, T)
+    b = orc.prefill(dcfg, W, dense_c, h0, 2, T)
+    assert np.max(np.abs(a.h - b.h)) <= 1e-9 * np.sqrt(np.mean(b.h ** 2))
+    np.testing.assert_allclose(a.logits, b.logits, atol=1e-9 * np.abs(b.logits).max())
+
+
+def test_dense_chunked_prefill_equals_the_whole_prompt():
+    """The dense looped forward is causal through every loop, so a prompt
+    prefilled in chunks gives the same states, caches and logits as in one call."""
+    cfg = _tiny_cfg(resid_bits=16, n_loops=3, seq_len=12, batch=2, seed=83)
+    W, rng = _weights(cfg)
+    T = cfg.seq_len
+    h0 = synth.make_h0(cfg, rng, 2 * T)
+    whole_c = orc.KVCache(cfg, 2, T)
+    whole = orc.prefill(cfg, W, whole_c, h0, 2, T)
+    parts_c = orc.KVCache(cfg, 2, T)
+    hp = h0.reshape(2, T, -1)
+    outs = []
+    for a, b in ((0, 5), (5, 9), (9, 12)):
+        r = orc.prefill(cfg, W, parts_c, hp[:, a:b].reshape(-1, cfg.d_model), 2, b - a)
+        outs.append(r.h.reshape(2, b - a, -1))
+    scale = np.abs(whole.h).max()
+    np.testing.assert_allclose(np.concatenate(outs, axis=1).reshape(2 * T, -1), whole.h, atol=1e-12 * scale)
+    np.testing.assert_allclose(r.logits, whole.logits, atol=1e-12 * np.abs(whole.logits).max())
+    np.testing.assert_allclose(parts_c.kv_k, whole_c.kv_k, atol=1e-12 * np.abs(whole_c.kv_k).max())
+
+
+def test_last_loop_prefill_of_a_fresh_prompt_equals_per_loop():
+    """Within one call every token is at the same loop, so overwriting one KV
+    slot per loop (last_loop) gives exactly the per-loop result."""
+    cfg = _tiny_cfg(resid_bits=16, n_loops=3, seq_len=10, batch=2, seed=84)
+    W, rng = _weights(cfg)
+    h0 = synth.make_h0(cfg, rng, 20)
+    per = orc.prefill(cfg, W, orc.KVCache(cfg, 2, 10), h0, 2, 10)
+    lcfg = cfg.with_(kv_mode=1)
+    lc = orc.KVCache(lcfg, 2, 10)
+    last = orc.prefill(lcfg, W, lc, h0, 2, 10)
+    assert np.array_equal(per.h, last.h) and np.array_equal(per.logits, last.logits)
+    assert lc.kv_k.shape[1] == 1
+
+
+def test_last_loop_decode_sees_the_context_last_pass_at_every_loop():
+    """Over a context, last_loop attends to the context's one stored pass at
+    every loop: the same as per_loop with every loop slot holding that pass."""
+    cfg = _tiny_cfg(resid_bits=16, n_loops=3, mode="decode", batch=3, seq_len=0, ctx_len=8, seed=85, kv_mode=1)
+    W, rng = _weights(cfg)
+    lens = [8, 3, 6]
+    ctx = synth.make_dense_context(cfg, rng, lens)
+    assert ctx["kv_k"].shape[1] == 1
+    last_c = orc.KVCache.from_dense_context(cfg, ctx, 9)
+    pcfg = cfg.with_(kv_mode=0)
+    rep = {"lens": ctx["lens"], "kv_k": np.repeat(ctx["kv_k"], cfg.n_loops, axis=1),
+           "kv_v": np.repeat(ctx["kv_v"], cfg.n_loops, axis=1)}
+    per_c = orc.KVCache.from_dense_context(pcfg, rep, 9)
+    h0 = synth.make_h0(cfg, rng, 3)
+    a = orc.decode_step(cfg, W, last_c, h0)
+    b = orc.decode_step(pcfg, W, per_c, h0)
+    assert np.array_equal(a.h, b.h)
+    # and the new token's stored pass is its last loop's KV
+    np.testing.assert_array_equal(last_c.kv_k[:, 0, :, :, 8], per_c.kv_k[:, -1, :, :, 8])
+
+
+# ----------------------------------------------------------------------------
+# variants around the looped core: prelude / coda layers, loop embedding,
+# input injection
+# ----------------------------------------------------------------------------
+
+def test_sandwich_depth_golden():
+    """The page's worked example: applications of independent and shared layers
+    add up to the effective depth; the weights are P + R + Q layers."""
+    rows = [tuple(int(v) for v in ln.split()) for ln in open(
+        __file__.replace("test_oracle_pins.py", "golden/sandwich_depth.txt"))
+        if ln.strip() and not ln.startswith("#")]
+    for P, R, K, Q, depth, weight_layers in rows:
+        cfg = _tiny_cfg(d_model=16, n_heads=2, n_kv_heads=1, head_dim=8, ffn_dim=16, n_layers=R, n_loops=K,
+                        n_prelude=P, n_coda=Q, seq_len=4, q_tile=4, rho=0.5, c_cols=2, group_size=8)
+        w = synth.make_weights(cfg)
+        W = orc.prepare_weights(w)
+        h0 = synth.make_h0(cfg, w["rng"], 4)
+        res = orc.prefill(cfg, W, orc.KVCache(cfg, 1, 4), h0, 1, 4)
+        assert res.trace["applications"] + res.trace["independent"] == depth
+        assert len(W["prelude"]) + len(W["layers"]) + len(W["coda"]) == weight_layers
+        dense = orc.prefill(cfg.with_(resid_bits=16), W, orc.KVCache(cfg.with_(resid_bits=16), 1, 4), h0, 1, 4)
+        assert dense.trace["applications"] + dense.trace["independent"] == depth
+
+
+@pytest.mark.parametrize("embed,gamma", [(0, 0.0), (1, 0.0), (1, 0.5), (0, 0.7)])
+def test_sandwich_with_loop_embedding_and_injection_matches_torch(embed, gamma):
+    """Dense variants against a torch restatement: the prelude, then per loop
+    the shared stack applied to h + e_k + gamma * x (x: the prelude output),
+    then the coda, each stack a plain pre-norm block sequence."""
+    cfg = _tiny_cfg(resid_bits=16, n_loops=3, n_prelude=2, n_coda=1, loop_embed=embed, inject_scale=gamma, seed=87,
+                    seq_len=10)
+    w = synth.make_weights(cfg)
+    W = orc.prepare_weights(w)
+    h0 = synth.make_h0(cfg, w["rng"], 10)
+    res = orc.prefill(cfg, W, orc.KVCache(cfg, 1, 10, kv_exact=True), h0, 1, 10)
+    sub = lambda layers: {"layers": layers}
+    x = _torch_block_forward(cfg, sub(W["prelude"]), np.asarray(h0, np.float64))
+    h = x.copy()
+    for k in range(cfg.n_loops):
+        u = h + (W["loop_embed"][k] if embed else 0.0) + gamma * x
+        h = _torch_block_forward(cfg, W, u)
+    want = _torch_block_forward(cfg, sub(W["coda"]), h)
+    np.testing.assert_allclose(res.h, want, rtol=0, atol=1e-11 * np.abs(want).max())
+    if embed or gamma:      # the variant really changes the result
+        plain = orc.prefill(cfg.with_(loop_embed=0, inject_scale=0.0), {k_: v_ for k_, v_ in W.items()
+                            if k_ != "loop_embed"}, orc.KVCache(cfg, 1, 10, kv_exact=True), h0, 1, 10)
+        assert np.max(np.abs(plain.h - res.h)) > 1e-3 * np.abs(want).max()
+
+
+@pytest.mark.parametrize("mode", ["prefill", "decode"])
+def test_lazy_variants_dense_limit(mode):
+    """rho = 1, every column, exact residuals: the lazy path with prelude, coda,
+    loop embedding and input injection equals the dense one."""
+    cfg = _tiny_cfg(rho=1.0, c_cols=10 ** 6, resid_bits=32, n_loops=3, n_prelude=1, n_coda=2, loop_embed=1,
+                    inject_scale=0.4, seed=88, seq_len=9, batch=2)
+    dcfg = cfg.with_(resid_bits=16)
+    w = synth.make_weights(cfg)
+    rng = w["rng"]
+    W = orc.prepare_weights(w)
+    if mode == "prefill":
+        h0 = synth.make_h0(cfg, rng, 18)
+        a = orc.prefill(cfg, W, orc.KVCache(cfg, 2, 9, kv_exact=True), h0, 2, 9)
+        b = orc.prefill(dcfg, W, orc.KVCache(dcfg, 2, 9, kv_exact=True), h0, 2, 9)
+    else:
+        lazy_c = orc.KVCache(cfg, 2, 12, kv_exact=True)
+        dense_c = orc.KVCache(dcfg, 2, 12, kv_exact=True)
+        pre = synth.make_h0(cfg, rng, 18)       # a dense prompt fills both caches identically
+        orc.prefill(cfg, W, lazy_c, pre, 2, 9)
+        orc.prefill(dcfg, W, dense_c, pre, 2, 9)
+        h0 = synth.make_h0(cfg, rng, 2)
+        a = orc.decode_step(cfg, W, lazy_c, h0)
+        b = orc.decode_step(dcfg, W, dense_c, h0)
+    assert np.max(np.abs(a.h - b.h)) <= 1e-9 * np.sqrt(np.mean(b.h ** 2))
+    np.testing.assert_allclose(a.logits, b.logits, atol=1e-9 * np.abs(b.logits).max())
+
+
+# ----------------------------------------------------------------------------
 # invariants of the lazy path
 # ----------------------------------------------------------------------------
 
