@@ -14,8 +14,8 @@
 // one loop slot, [M][1][2][B][Hkv][T][hd], which every loop overwrites
 // Tokens of one (sequence, KV head) are contiguous so a decode step streams them.
 // The reconstructed KV of loop m is base + code*scale of loops 2..m, added in
-// loop order in fp32 ("FlashLoop ...", abstract: KV residuals between
-// adjacent loops).  code*scale is exact in fp32 (|code| <= 7, 11-bit scale).
+// loop order in fp32 ("FlashLoop ...", abstract: each loop's KV as a
+// low-bit residual over the previous loop's).  code*scale is exact in fp32 (|code| <= 7, 11-bit scale).
 #pragma once
 #include "fl_device.cuh"
 
@@ -158,12 +158,22 @@ constexpr int kMaxLoops = 16;
 inline int chain_km(int K) { return K <= 2 ? 2 : K <= 4 ? 4 : K <= 8 ? 8 : 16; }
 
 // Reconstructions to loop m_lo and to loop m_hi (m_lo <= m_hi <= KM) of one
-// row; lane holds EPL values of each.  All loads (base row, residual codes and
+// row; lane holds EPL values of each; SP: the sparse residual layout, whose
+// pool rows (from chain_rows) may be passed in when K and V of a position are
+// both rebuilt.  All loads (base row, residual codes and
 // scales of loops 2..m_hi) are issued before any arithmetic so their latencies
 // overlap; the adds then run in loop order, as the definition requires.
-template <int EPL, int KM = kMaxLoops>
+// Sparse layout: the pool rows of levels 2..m_hi of position t (-1 for none),
+// shared by K, V and every KV head of the position.
+template <int KM>
+__device__ __forceinline__ void chain_rows(const CacheView& cv, int j, int b, int t, int m_hi, int* rr) {
+#pragma unroll
+  for (int q = 0; q < KM - 1; ++q) rr[q] = q + 2 <= m_hi ? cv.ridx[cv.ridx_index(j, q + 2, b, t)] : -1;
+}
+
+template <int EPL, int KM, bool SP>
 __device__ __forceinline__ void chain_lane2(const CacheView& cv, int j, int kv, int b, int h, int t, int m_lo,
-                                            int m_hi, int lane, float* lo, float* hi) {
+                                            int m_hi, int lane, float* lo, float* hi, const int* rows_in = nullptr) {
   const uint16_t* br = cv.base_row(j, kv, b, h, t) + lane * EPL;
   uint32_t braw[EPL == 4 ? 2 : 1];
   if (EPL == 4) {
@@ -175,46 +185,48 @@ __device__ __forceinline__ void chain_lane2(const CacheView& cv, int j, int kv, 
   }
   const int gi = (lane * EPL) >> cv.lg;
   const size_t rb = cv.row_bytes_codes(), ns = cv.hd >> cv.lg;
-  // residual row of every level: one row per position (consecutive levels a
-  // fixed stride apart), or with sparse storage the pool row from the index
-  // (all index loads first), -1 for none
-  const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * cv.pool_rows();   // rows between loops
-  size_t ridx_lv[KM - 1];
-  bool have[KM - 1];
-  if (!cv.rows) {
-    const size_t r0 = cv.res_index(j, 2, kv, b, h, t);
-#pragma unroll
-    for (int q = 0; q < KM - 1; ++q) {
-      ridx_lv[q] = r0 + q * step;
-      have[q] = q + 2 <= m_hi;
-    }
-  } else {
-    int rr[KM - 1];
-#pragma unroll
-    for (int q = 0; q < KM - 1; ++q) rr[q] = q + 2 <= m_hi ? cv.res_row(j, q + 2, b, t) : -1;
-#pragma unroll
-    for (int q = 0; q < KM - 1; ++q) {
-      have[q] = rr[q] >= 0;
-      ridx_lv[q] = have[q] ? cv.res_index(j, q + 2, kv, b, h, rr[q]) : 0;
-    }
-  }
+  // residual row of level q + 2: SP false (one row per position), the row of
+  // level 2 plus q * step; SP true (sparse storage), the pool row from the
+  // index, all index loads first, -1 for none.  A level without a row
+  // contributes code 0 x scale 0, as a stored zero row does.  The layout is a
+  // template parameter so the dense layout's walk carries no index registers.
   uint32_t craw[KM - 1];
   uint16_t sraw[KM - 1];
+  auto load_level = [&](int q, size_t ri) {
+    const uint8_t* row = cv.codes + ri * rb;
+    if (EPL == 4) {
+      craw[q] = cv.bits == 4 ? static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(row + lane * 2))
+                             : static_cast<uint32_t>(row[lane]);
+    } else {
+      craw[q] = cv.bits == 4 ? static_cast<uint32_t>(row[lane])
+                             : static_cast<uint32_t>((row[lane >> 1] >> ((lane & 1) * 4)) & 0xF);
+    }
+    sraw[q] = cv.scales[ri * ns + gi];
+  };
+  if (!SP) {
+    const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * cv.T;   // rows between consecutive loops
+    const size_t r0 = ((((static_cast<size_t>(j) * (cv.K - 1)) * 2 + kv) * cv.B + b) * cv.Hkv + h) * cv.T + t;
 #pragma unroll
-  for (int q = 0; q < KM - 1; ++q) {
-    craw[q] = 0u;
-    sraw[q] = 0;
-    if (have[q]) {
-      const size_t ri = ridx_lv[q];
-      const uint8_t* row = cv.codes + ri * rb;
-      if (EPL == 4) {
-        craw[q] = cv.bits == 4 ? static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(row + lane * 2))
-                               : static_cast<uint32_t>(row[lane]);
-      } else {
-        craw[q] = cv.bits == 4 ? static_cast<uint32_t>(row[lane])
-                               : static_cast<uint32_t>((row[lane >> 1] >> ((lane & 1) * 4)) & 0xF);
-      }
-      sraw[q] = cv.scales[ri * ns + gi];
+    for (int q = 0; q < KM - 1; ++q) {
+      craw[q] = 0u;
+      sraw[q] = 0;
+      if (q + 2 <= m_hi) load_level(q, r0 + q * step);
+    }
+  } else {
+    const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * cv.rows;
+    const size_t q0 = ((((static_cast<size_t>(j) * (cv.K - 1)) * 2 + kv) * cv.B + b) * cv.Hkv + h) * cv.rows;
+    int rr[KM - 1];
+    if (rows_in) {
+#pragma unroll
+      for (int q = 0; q < KM - 1; ++q) rr[q] = rows_in[q];
+    } else {
+      chain_rows<KM>(cv, j, b, t, m_hi, rr);
+    }
+#pragma unroll
+    for (int q = 0; q < KM - 1; ++q) {
+      craw[q] = 0u;
+      sraw[q] = 0;
+      if (rr[q] >= 0) load_level(q, q0 + q * step + static_cast<size_t>(rr[q]));
     }
   }
   float acc[EPL];

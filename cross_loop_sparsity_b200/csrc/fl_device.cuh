@@ -11,7 +11,7 @@
 namespace fl {
 
 // Error bits a kernel records in the context status word.
-enum : int { kErrWaitTimeout = 1, kErrBadIndex = 2, kErrCapacity = 4 };
+enum : int { kErrWaitTimeout = 1, kErrNonfinite = 2, kErrCapacity = 4 };
 
 // A bounded wait gives up after this many SM clock cycles (about 1 s at
 // 1.9 GHz), records kErrWaitTimeout and lets the kernel return.

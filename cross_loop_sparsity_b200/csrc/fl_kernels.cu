@@ -1689,15 +1689,15 @@ __device__ void select_row(const SelColsArgs& a, int seg, int g, int tl, int n, 
   if (threadIdx.x == 0) *nout = got;
 }
 
-// After a delta-score item: the CTA that wrote the last chunk of its row (an
-// atomic ticket over the row's chunks, no waiting) selects the row's column
-// set, so the selection needs no launch of its own.
+// After a delta-score item: the CTA that wrote the last unit of its row (an
+// atomic ticket over the row's units of unit_cols columns, no waiting) selects
+// the row's column set, so the selection needs no launch of its own.
 __device__ __forceinline__ void fold_select(const DScoreArgs& a, int seg, int g, int tl, int n, float* keys_sm,
-                                            int* last_flag) {
+                                            int* last_flag, int unit_cols) {
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
-    const int nch = (n + 63) / 64;
+    const int nch = (n + unit_cols - 1) / unit_cols;
     const int old = atomicAdd(&a.row_tickets[seg * a.Hkv + g], 1);
     *last_flag = old == nch - 1;
   }
@@ -1713,104 +1713,224 @@ __device__ __forceinline__ void fold_select(const DScoreArgs& a, int seg, int g,
 // delta-score column keys of tiles recomputed for the first time:
 //   key[k] = max over the tile's selected queries i (with k <= pos(i)) and the
 //   group's heads h of | tau*(q_l[i,h] . K_l[k] - q_last[i,h] . K_base[k]) |
-// ("attention-output differences are dominated by a sparse and stable subset
-// of key columns", "FlashLoop ...", abstract).  grid (max_need*Hkv, chunks).
+// ("FlashLoop ...", abstract: the change of a query's attention output
+// between loops comes from few key columns, and the same ones over loops).
+// At a tile's first
+// recomputation every member was last computed at loop 1, so the old keys are
+// the bf16 base rows.
+//
+// SIMT form, for few (query, head) pairs per tile (decode: one query per tile)
+// and head_dim 64 without tensor cores.  Work items are (tile, KV head, block of
+// 64, 128 or 256 columns -- the largest that still gives every CTA work); each
+// CTA takes a contiguous range of items, so the tile's pairs, staged in shared
+// memory kDsPairs at a time, are reused while (tile, KV head) stays the same,
+// and with sparse storage the item's pool rows of every level are staged
+// first, so each step needs one memory round trip.  A quad of lanes owns one
+// column: lane qd of the quad holds dims [qd*HD/4, (qd+1)*HD/4) of K_l and
+// K_base, all of whose loads (index rows first with sparse storage, then base,
+// codes and scales of every level) are issued before any is used; the quad's
+// partial dot products meet in two shuffles.
 // ============================================================================
-template <int HD, int EPL, int KM>
-__global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
+constexpr int kDsBlock = 256;   // largest columns per work item
+constexpr int kDsPairs = 8;     // (query, head) pairs held in registers per pass
+
+template <int HD, int KM, bool SP>
+__global__ void __launch_bounds__(256, 2) k_dscore(const DScoreArgs a) {
   pdl_trigger();
   pdl_wait();
-  constexpr int CC = 64;      // columns per CTA
-  constexpr int QP = 16;      // (query, head) pairs staged per batch
+  constexpr int DPL = HD / 4;              // dims per lane
+  constexpr int QS = DPL + 4;              // padded stride of one lane-quarter of a staged query row
   extern __shared__ __align__(16) uint8_t sm[];
-  float* Kn = reinterpret_cast<float*>(sm);      // [CC][HD+1]
-  float* Kb = Kn + CC * (HD + 1);                // [CC][HD+1]
-  float* Qn = Kb + CC * (HD + 1);                // [QP][HD]
-  float* Qo = Qn + QP * HD;                      // [QP][HD]
-  float* Mx = Qo + QP * HD;                      // [4][CC]
-  __shared__ int Qpos[QP];                       // position of each staged pair's query
+  float* qn_sm = reinterpret_cast<float*>(sm);       // [kDsPairs][4][QS]: tau * q_l
+  float* qo_sm = qn_sm + kDsPairs * 4 * QS;           // [kDsPairs][4][QS]: tau * q_last
+  __shared__ int qpos_sm[kDsPairs], qtok_sm[kDsPairs], qi_sm[kDsPairs];
+  __shared__ float best_sm[kDsBlock];            // the item's column keys so far (one owner quad per column)
+  __shared__ int rows_sm[SP ? (KM - 1) * kDsBlock : 1];   // sparse storage: pool rows of the item's columns
   __shared__ int fold_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  // work items (tile needing a set, KV head, 64-column chunk), taken grid-stride
-  // by a grid sized to the GPU, so a loop whose tiles all have their sets
-  // (every lazy loop after the first, mostly) costs one launch, not a grid of
-  // empty CTAs sized for the longest row
-  const int cnt = a.plan.counts[1];
-  for (int it = blockIdx.x; it < cnt * a.Hkv * a.max_chunks; it += gridDim.x) {
-  const int seg = it / (a.Hkv * a.max_chunks), g = (it / a.max_chunks) % a.Hkv, chunk = it % a.max_chunks;
-  const int p = a.plan.need[seg];
-  const int qb = a.plan.qb[p], qe = a.plan.qe[p];
-  const SelMeta ml = a.meta[qe - 1];
-  const int b = ml.seq, maxpos = ml.pos;
-  const int c0 = chunk * CC;
-  if (c0 > maxpos) continue;   // (uniform over the CTA)
-  const int nc = min(CC, maxpos + 1 - c0);
+  const int qd = lane & 3, col_in_warp = lane >> 2;
   const int grp = a.H / a.Hkv;
+  const int blk_cols = a.ds_block, nsteps = blk_cols / 64;   // columns per item (64, 128 or 256)
+  const int nblk = (a.max_cols + blk_cols - 1) / blk_cols;
+  const int cnt = a.plan.counts[1];
   const CacheView& cv = a.cv;
-  // reconstruct K of loop l and the base for this column chunk: a warp's rows
-  // are requested together, then stored
-  {
-    constexpr int RW = CC / 8;   // rows per warp
-    float lo[RW][EPL], hi[RW][EPL];
-#pragma unroll
-    for (int u = 0; u < RW; ++u) {
-      const int rr = warp + u * 8;
-      if (rr < nc) chain_lane2<EPL, KM>(cv, a.j, 0, b, g, c0 + rr, 1, a.loop, lane, lo[u], hi[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < RW; ++u) {
-      const int rr = warp + u * 8;
-      if (rr >= nc) continue;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        Kb[rr * (HD + 1) + lane * EPL + e] = lo[u][e];
-        Kn[rr * (HD + 1) + lane * EPL + e] = hi[u][e];
+  const int bits = cv.bits, gi = (qd * DPL) >> cv.lg;
+  const size_t rb = cv.row_bytes_codes(), ns = cv.hd >> cv.lg;
+  // each CTA takes a contiguous range of items, so consecutive items mostly
+  // share (tile, KV head) and their staged pairs are reused
+  const int total = cnt * a.Hkv * nblk, per_cta = (total + gridDim.x - 1) / gridDim.x;
+  const int it_end = min(total, (blockIdx.x + 1) * per_cta);
+  int staged = -1;
+  for (int it = blockIdx.x * per_cta; it < it_end; ++it) {
+    const int seg = it / (a.Hkv * nblk), g = (it / nblk) % a.Hkv, blk = it % nblk;
+    const int p = a.plan.need[seg];
+    const int qb = a.plan.qb[p], qe = a.plan.qe[p];
+    const SelMeta ml = a.meta[qe - 1];
+    const int b = ml.seq, maxpos = ml.pos;
+    const int c0 = blk * blk_cols;
+    if (c0 > maxpos) continue;   // (uniform over the CTA)
+    const int npairs = (qe - qb) * grp;
+    const bool one_group = npairs <= kDsPairs;
+    // every column of the item: this warp's 8 columns per step, nsteps steps
+    for (int pb = 0; pb < npairs; pb += kDsPairs) {
+      const int np = min(kDsPairs, npairs - pb);
+      __syncthreads();   // the previous pairs (and the previous item's keys) are no longer read
+      if (pb == 0) {
+        best_sm[tid] = 0.f;
+        if (SP)
+          for (int e = tid; e < (KM - 1) * blk_cols; e += blockDim.x) {
+            const int q = e / blk_cols, k = e % blk_cols, col = c0 + k;
+            rows_sm[q * kDsBlock + k] =
+                (col <= maxpos && q + 2 <= a.loop) ? cv.ridx[cv.ridx_index(a.j, q + 2, b, col)] : -1;
+          }
       }
-    }
-  }
-  const int c = tid % CC, slot = tid / CC;
-  float best = 0.f;
-  const int npairs = (qe - qb) * grp;
-  for (int pb = 0; pb < npairs; pb += QP) {
-    __syncthreads();
-    const int np = min(QP, npairs - pb);
-    for (int e = tid; e < np * HD; e += 256) {
-      const int pr = e / HD, dd = e % HD;
-      const int qi = qb + (pb + pr) / grp, hh = g * grp + (pb + pr) % grp;
-      const SelMeta mq = a.meta[qi];
-      Qn[pr * HD + dd] = a.q_cur[(static_cast<size_t>(qi) * a.H + hh) * HD + dd];
-      Qo[pr * HD + dd] = a.q_last[(static_cast<size_t>(mq.tok) * a.H + hh) * HD + dd];
-      if (dd == 0) Qpos[pr] = mq.pos;
-    }
-    __syncthreads();
-    if (c < nc) {
-      for (int pr = slot; pr < np; pr += 4) {
-        if (Qpos[pr] < c0 + c) continue;
-        float dn = 0.f, db = 0.f;
-        const float* kn = &Kn[c * (HD + 1)];
-        const float* kb = &Kb[c * (HD + 1)];
-        const float* qn = &Qn[pr * HD];
-        const float* qo = &Qo[pr * HD];
-#pragma unroll 8
-        for (int e = 0; e < HD; ++e) {
-          dn += kn[e] * qn[e];
-          db += kb[e] * qo[e];
+      const int key = seg * a.Hkv + g;
+      if (!(one_group && staged == key)) {
+        // the pairs' slots first, then every query element with its address known
+        if (tid < kDsPairs) {
+          const int pr = tid;
+          if (pr < np) {
+            const int qi = qb + (pb + pr) / grp;
+            const SelMeta mq = a.meta[qi];
+            qi_sm[pr] = qi;
+            qtok_sm[pr] = mq.tok;
+            qpos_sm[pr] = mq.pos;
+          } else {
+            qi_sm[pr] = qtok_sm[pr] = 0;
+            qpos_sm[pr] = -1;
+          }
         }
-        best = fmaxf(best, fabsf(a.tau * (dn - db)));
+        __syncthreads();
+#pragma unroll 4
+        for (int e = tid; e < kDsPairs * HD; e += blockDim.x) {
+          const int pr = e / HD, dd = e % HD;
+          float vn = 0.f, vo = 0.f;
+          if (pr < np) {
+            const int hh = g * grp + (pb + pr) % grp;
+            vn = a.tau * a.q_cur[(static_cast<size_t>(qi_sm[pr]) * a.H + hh) * HD + dd];
+            vo = a.tau * a.q_last[(static_cast<size_t>(qtok_sm[pr]) * a.H + hh) * HD + dd];
+          }
+          const int o = (pr * 4 + dd / DPL) * QS + dd % DPL;
+          qn_sm[o] = vn;
+          qo_sm[o] = vo;
+        }
+        staged = one_group ? key : -1;
+      }
+      __syncthreads();
+#pragma unroll 1
+      for (int s = 0; s < nsteps; ++s) {
+        const int col = c0 + s * 64 + warp * 8 + col_in_warp;
+        const bool valid = col <= maxpos;
+        // ---- loads: base dims of this lane, then every level's codes and scale
+        uint4 braw[DPL / 8];
+        uint4 craw[KM - 1];
+        uint16_t sraw[KM - 1];
+        if (valid) {
+          const uint4* br = reinterpret_cast<const uint4*>(cv.base_row(a.j, 0, b, g, col) + qd * DPL);
+#pragma unroll
+          for (int u = 0; u < DPL / 8; ++u) braw[u] = br[u];
+        } else {
+#pragma unroll
+          for (int u = 0; u < DPL / 8; ++u) braw[u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        int rr[KM - 1];
+#pragma unroll
+        for (int q = 0; q < KM - 1; ++q)
+          rr[q] = SP ? rows_sm[q * kDsBlock + (col - c0)] : ((valid && q + 2 <= a.loop) ? col : -1);
+        const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * (SP ? cv.rows : cv.T);
+        const size_t q0 = ((((static_cast<size_t>(a.j) * (cv.K - 1)) * 2) * cv.B + b) * cv.Hkv + g) *
+                          static_cast<size_t>(SP ? cv.rows : cv.T);
+#pragma unroll
+        for (int q = 0; q < KM - 1; ++q) {
+          craw[q] = make_uint4(0u, 0u, 0u, 0u);
+          sraw[q] = 0;
+          if (rr[q] >= 0) {
+            const size_t ri = q0 + q * step + static_cast<size_t>(rr[q]);
+            const int nb = DPL * bits / 8;   // code bytes of this lane's dims: 16, 8 or 4
+            const uint8_t* row = cv.codes + ri * rb + qd * nb;
+            if (nb == 16) {
+              craw[q] = *reinterpret_cast<const uint4*>(row);
+            } else if (nb == 8) {
+              const uint2 v = *reinterpret_cast<const uint2*>(row);
+              craw[q].x = v.x;
+              craw[q].y = v.y;
+            } else {
+              craw[q].x = *reinterpret_cast<const uint32_t*>(row);
+            }
+            sraw[q] = cv.scales[ri * ns + gi];
+          }
+        }
+        // ---- K_l = base + code * scale of loops 2..l, added in loop order in fp32
+        // (the base stays packed: two bf16 per word, widened where it is used)
+        uint32_t kb[DPL / 2];
+#pragma unroll
+        for (int u = 0; u < DPL / 8; ++u) {
+          kb[4 * u] = braw[u].x;
+          kb[4 * u + 1] = braw[u].y;
+          kb[4 * u + 2] = braw[u].z;
+          kb[4 * u + 3] = braw[u].w;
+        }
+        float kn[DPL];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) kn[e] = bf16_to_f(e & 1 ? kb[e / 2] >> 16 : kb[e / 2] & 0xFFFF);
+#pragma unroll
+        for (int q = 0; q < KM - 1; ++q) {
+          if (q + 2 > a.loop) break;
+          const float sc = half_bits_to_f(sraw[q]);
+          const uint32_t w[4] = {craw[q].x, craw[q].y, craw[q].z, craw[q].w};
+          if (bits == 4) {   // element e: nibble e % 8 of word e / 8 (low nibble first)
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) {
+              const int c = sext(static_cast<int>((w[e / 8] >> ((e % 8) * 4)) & 0xFu), 4);
+              kn[e] = __fadd_rn(kn[e], __fmul_rn(static_cast<float>(c), sc));
+            }
+          } else {           // element e: bits 2(e % 16) of word e / 16 (LSB first)
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) {
+              const int c = sext(static_cast<int>((w[e / 16] >> ((e % 16) * 2)) & 0x3u), 2);
+              kn[e] = __fadd_rn(kn[e], __fmul_rn(static_cast<float>(c), sc));
+            }
+          }
+        }
+        // ---- partial dot products of this lane's dims, one pair at a time
+        float m = 0.f;
+#pragma unroll 1
+        for (int pr = 0; pr < np; ++pr) {
+          const float* qn = qn_sm + (pr * 4 + qd) * QS;
+          const float* qo = qo_sm + (pr * 4 + qd) * QS;
+          float dn = 0.f, db = 0.f;
+#pragma unroll
+          for (int e = 0; e < DPL; e += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(qn + e);
+            const float4 y = *reinterpret_cast<const float4*>(qo + e);
+            dn += kn[e] * x.x + kn[e + 1] * x.y + kn[e + 2] * x.z + kn[e + 3] * x.w;
+            db += bf16_to_f(kb[e / 2] & 0xFFFF) * y.x + bf16_to_f(kb[e / 2] >> 16) * y.y +
+                  bf16_to_f(kb[e / 2 + 1] & 0xFFFF) * y.z + bf16_to_f(kb[e / 2 + 1] >> 16) * y.w;
+          }
+          float d = dn - db;
+          d += __shfl_xor_sync(0xffffffffu, d, 1);
+          d += __shfl_xor_sync(0xffffffffu, d, 2);
+          if (col <= qpos_sm[pr]) m = fmaxf(m, fabsf(d));
+        }
+        const int slot = s * 64 + warp * 8 + col_in_warp;
+        if (qd == 0) best_sm[slot] = fmaxf(best_sm[slot], m);
       }
     }
-  }
-  Mx[slot * CC + c] = best;
-  __syncthreads();
-  if (tid < nc) {
-    const float v = fmaxf(fmaxf(Mx[tid], Mx[CC + tid]), fmaxf(Mx[2 * CC + tid], Mx[3 * CC + tid]));
-    a.col_keys[(static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols + c0 + tid] = v;
-    const int tl = a.plan.tile[p];
-    if (a.trace_ck && tl < a.trace_tiles)
-      a.trace_ck[((static_cast<size_t>(a.j) * a.trace_tiles + tl) * a.Hkv + g) * a.max_cols + c0 + tid] = v;
-  }
-  __syncthreads();   // the staged rows and Mx are reused by the next item
-  if (a.fold) fold_select(a, seg, g, a.plan.tile[p], maxpos + 1, reinterpret_cast<float*>(sm), &fold_last);
+    // ---- this item's keys (each written by the lane that owns the column)
+    for (int s = 0; s < nsteps; ++s) {
+      const int slot = s * 64 + warp * 8 + col_in_warp, col = c0 + slot;
+      if (qd == 0 && col <= maxpos) {
+        const float v = best_sm[slot];
+        a.col_keys[(static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols + col] = v;
+        const int tl = a.plan.tile[p];
+        if (a.trace_ck && tl < a.trace_tiles)
+          a.trace_ck[((static_cast<size_t>(a.j) * a.trace_tiles + tl) * a.Hkv + g) * a.max_cols + col] = v;
+      }
+    }
+    if (a.fold) {
+      __syncthreads();   // the staged pairs are dead; the fold reuses the shared memory
+      fold_select(a, seg, g, a.plan.tile[p], maxpos + 1, reinterpret_cast<float*>(sm), &fold_last, blk_cols);
+    }
   }
 }
 
@@ -1823,156 +1943,246 @@ __global__ void __launch_bounds__(256) k_dscore(const DScoreArgs a) {
 // old keys are the bf16 base exactly; the new keys (base + residuals, fp32) are
 // split into bf16 hi + lo, the queries too, and the difference accumulates in
 // one register set:  Qh Kh + Ql Kh + Qh Kl - Qoh Kb - Qol Kb  (the Ql Kl term,
-// below 2^-16 relative, is dropped).  Items (tile, KV head, 64-column chunk)
-// are taken grid-stride; a CTA's 4 warps take 16 (query, head) rows each, 64
-// rows per pass, and their column maxima meet in shared memory (max of
-// non-negative floats = max of their bit patterns, in any order).
+// below 2^-16 relative, is dropped).
+//
+// Work items are (tile, KV head, unit of kDsTcUnit 64-column chunks), taken
+// grid-stride, one CTA per SM.  Per item and per pass of 64 (query, head)
+// pairs, the pairs are staged once in shared memory as the four bf16 operand
+// tiles (tau q_l hi / lo, -tau q_last hi / lo); the unit's chunks then stream
+// through: the base rows of chunk c + 1 are copied (cp.async, 128-byte swizzle)
+// while chunk c's new keys are built (base + the residual codes of loops
+// 2..l, loaded before the copy is awaited) and multiplied.  Warp w takes pair
+// rows 16 (w % 4) .. +15 against columns 32 (w / 4) .. +31 of the chunk; the
+// column maxima meet in shared memory (max of non-negative floats = max of
+// their bit patterns, in any order).
 // ============================================================================
-template <int HD, int KM>
-__global__ void __launch_bounds__(128) k_dscore_tc(const DScoreArgs a) {
-  static_assert(HD == 128, "the staging gives each lane four dims of a 128-dim row");
+constexpr int kDsTcUnit = 4;   // 64-column chunks per work item
+
+__device__ __forceinline__ uint32_t swz128(int row, int piece) {   // 16-byte piece of a 64 x 128-dim bf16 tile
+  return static_cast<uint32_t>((piece >> 3) * (64 * 128) + row * 128 + (((piece & 7) ^ (row & 7)) << 4));
+}
+
+template <int KM, bool SP>
+__global__ void __launch_bounds__(256, 1) k_dscore_tc(const DScoreArgs a) {
+  constexpr int HD = 128, TILE = 2 * 64 * 128, KS = HD / 16, UC = kDsTcUnit;
   pdl_trigger();
   pdl_wait();
-  constexpr int CC = 64, BOX = 64 * 128, NB = HD / 64, TILE = NB * BOX, KS = HD / 16;
   extern __shared__ uint8_t sm_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* knh = sm;   // new keys (hi, lo) and the base keys, one 64 x HD bf16 tile each
-
-  uint8_t* knl = sm + TILE;
-  uint8_t* kbs = sm + 2 * TILE;
-  __shared__ unsigned colmax[CC];
+  uint8_t* qt = sm;                    // [4][TILE]: tau q_l hi, lo; -tau q_last hi, lo (64 pair rows)
+  uint8_t* kbs = sm + 4 * TILE;        // [2][TILE]: base rows of the chunk (double-buffered)
+  uint8_t* knh = sm + 6 * TILE;        // new keys, hi
+  uint8_t* knl = sm + 7 * TILE;        // new keys, lo
+  __shared__ unsigned colmax[UC * 64];
+  __shared__ int qpos[64];
   __shared__ int fold_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rg = warp & 3, ch2 = warp >> 2;   // pair-row group, column half
   const int grp = a.H / a.Hkv;
   const int cnt = a.plan.counts[1];
+  const int nunit = (a.max_chunks + UC - 1) / UC;
   const CacheView& cv = a.cv;
-  for (int it = blockIdx.x; it < cnt * a.Hkv * a.max_chunks; it += gridDim.x) {
-    const int seg = it / (a.Hkv * a.max_chunks), g = (it / a.max_chunks) % a.Hkv, chunk = it % a.max_chunks;
+  const int bits = cv.bits;
+  const size_t rb = cv.row_bytes_codes(), ns = cv.hd >> cv.lg;
+  const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * (SP ? cv.rows : cv.T);
+  const uint32_t qt_s = smem_u32(qt), kbs_s = smem_u32(kbs), knh_s = smem_u32(knh), knl_s = smem_u32(knl);
+  for (int it = blockIdx.x; it < cnt * a.Hkv * nunit; it += gridDim.x) {
+    const int seg = it / (a.Hkv * nunit), g = (it / nunit) % a.Hkv, unit = it % nunit;
     const int p = a.plan.need[seg];
     const int qb = a.plan.qb[p], qe = a.plan.qe[p];
     const SelMeta ml = a.meta[qe - 1];
     const int b = ml.seq, maxpos = ml.pos;
-    const int c0 = chunk * CC;
-    if (c0 > maxpos) continue;   // (uniform over the CTA)
-    const int nc = min(CC, maxpos + 1 - c0);
-    if (tid < CC) colmax[tid] = 0u;
-    // stage the chunk's keys: row r = column c0 + r, 16-byte chunk ch at
-    // (ch / 8) * BOX + r * 128 + ((ch % 8) ^ (r % 8)) * 16 (the 128-byte swizzle)
-    {
-      constexpr int RW = CC / 4;   // rows per warp
-      for (int u = 0; u < RW; ++u) {
-        const int rr = warp * RW + u;
-        float lo[4], hi[4];
-        if (rr < nc) {
-          chain_lane2<4, KM>(cv, a.j, 0, b, g, c0 + rr, 1, a.loop, lane, lo, hi);
+    const int u0 = unit * UC * 64;
+    if (u0 > maxpos) continue;   // (uniform over the CTA)
+    const int nch = min(UC, (maxpos - u0) / 64 + 1);
+    const size_t q0 = ((((static_cast<size_t>(a.j) * (cv.K - 1)) * 2) * cv.B + b) * cv.Hkv + g) *
+                      static_cast<size_t>(SP ? cv.rows : cv.T);
+    const int npairs = (qe - qb) * grp;
+    // copy the base rows of chunk c (rows past the last eligible column read zero)
+    auto issue_base = [&](int c) {
+      const int c0 = u0 + c * 64;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = tid + 256 * u, r = e >> 4, pc = e & 15;
+        const bool ok = c0 + r <= maxpos;
+        const uint16_t* src = cv.base_row(a.j, 0, b, g, ok ? c0 + r : c0) + pc * 8;
+        cp_async16(kbs_s + (c & 1) * TILE + swz128(r, pc), src, ok ? 16u : 0u);
+      }
+      cp_async_commit();
+    };
+    for (int pb = 0; pb < npairs; pb += 64) {
+      __syncthreads();   // the previous pass (or item, or fold) no longer reads shared memory
+      // ---- the pass's pairs as operand tiles: thread -> (pair row, 8-dim piece) x 4
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = tid + 256 * u, r = e >> 4, pc = e & 15;
+        const int pr = pb + r;
+        float xn[8], xo[8];
+        if (pr < npairs) {
+          const int qi = qb + pr / grp, hh = g * grp + pr % grp;
+          const SelMeta mq = a.meta[qi];
+          const float4* qn = reinterpret_cast<const float4*>(a.q_cur + (static_cast<size_t>(qi) * a.H + hh) * HD) + pc * 2;
+          const float4* qo = reinterpret_cast<const float4*>(a.q_last + (static_cast<size_t>(mq.tok) * a.H + hh) * HD) + pc * 2;
+          const float4 n0 = qn[0], n1 = qn[1], o0 = qo[0], o1 = qo[1];
+          xn[0] = n0.x; xn[1] = n0.y; xn[2] = n0.z; xn[3] = n0.w; xn[4] = n1.x; xn[5] = n1.y; xn[6] = n1.z; xn[7] = n1.w;
+          xo[0] = o0.x; xo[1] = o0.y; xo[2] = o0.z; xo[3] = o0.w; xo[4] = o1.x; xo[5] = o1.y; xo[6] = o1.z; xo[7] = o1.w;
+          if (pc == 0) qpos[r] = mq.pos;
         } else {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) lo[e] = hi[e] = 0.f;
+          for (int k = 0; k < 8; ++k) xn[k] = xo[k] = 0.f;
+          if (pc == 0) qpos[r] = -1;
         }
-        // lane holds dims 4*lane .. +3: 8 bytes of a 16-byte chunk
-        const int ch = lane >> 1;
-        const uint32_t off = (ch >> 3) * BOX + rr * 128 + ((((ch & 7) ^ (rr & 7)) << 4) | ((lane & 1) << 3));
-        float h[4], l[4];
+        uint32_t wh[4], wl[4], woh[4], wol[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) split_bf16(hi[e], h[e], l[e]);
-        *reinterpret_cast<uint2*>(knh + off) = make_uint2(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]));
-        *reinterpret_cast<uint2*>(knl + off) = make_uint2(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]));
-        *reinterpret_cast<uint2*>(kbs + off) = make_uint2(pack_bf16x2(lo[0], lo[1]), pack_bf16x2(lo[2], lo[3]));
-      }
-    }
-    __syncthreads();
-    const int npairs = (qe - qb) * grp;
-    for (int pb = 0; pb < npairs; pb += 64) {
-      // this warp's 16 (query, head) rows: r0 = lane/4, r1 = r0 + 8
-      int qpos[2];
-      uint32_t qnh[KS][4], qnl[KS][4], qoh[KS][4], qol[KS][4];
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int pr = pb + warp * 16 + (lane >> 2) + 8 * r;
-        qpos[r] = -1;
-        if (pr < npairs) qpos[r] = a.meta[qb + pr / grp].pos;
-      }
-#pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
-        float xn[8], xo[8];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int pr = min(pb + warp * 16 + (lane >> 2) + 8 * r, npairs - 1);
-          const int qi = qb + pr / grp, hh = g * grp + pr % grp;
-          const float* qn = a.q_cur + (static_cast<size_t>(qi) * a.H + hh) * HD;
-          const float* qo = a.q_last + (static_cast<size_t>(a.meta[qi].tok) * a.H + hh) * HD;
-          const int d = ks * 16 + 2 * (lane & 3);
-          const bool v = qpos[r] >= 0;
-          // A fragment order: (r0, d), (r1, d), (r0, d+8), (r1, d+8), two values each
-          xn[2 * r] = v ? qn[d] * a.tau : 0.f;         xn[2 * r + 1] = v ? qn[d + 1] * a.tau : 0.f;
-          xn[4 + 2 * r] = v ? qn[d + 8] * a.tau : 0.f; xn[4 + 2 * r + 1] = v ? qn[d + 9] * a.tau : 0.f;
-          xo[2 * r] = v ? -qo[d] * a.tau : 0.f;         xo[2 * r + 1] = v ? -qo[d + 1] * a.tau : 0.f;
-          xo[4 + 2 * r] = v ? -qo[d + 8] * a.tau : 0.f; xo[4 + 2 * r + 1] = v ? -qo[d + 9] * a.tau : 0.f;
-        }
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
+        for (int k = 0; k < 4; ++k) {
           float h0, l0, h1, l1;
-          split_bf16(xn[2 * r], h0, l0);
-          split_bf16(xn[2 * r + 1], h1, l1);
-          qnh[ks][r] = pack_bf16x2(h0, h1);
-          qnl[ks][r] = pack_bf16x2(l0, l1);
-          split_bf16(xo[2 * r], h0, l0);
-          split_bf16(xo[2 * r + 1], h1, l1);
-          qoh[ks][r] = pack_bf16x2(h0, h1);
-          qol[ks][r] = pack_bf16x2(l0, l1);
+          split_bf16(a.tau * xn[2 * k], h0, l0);
+          split_bf16(a.tau * xn[2 * k + 1], h1, l1);
+          wh[k] = pack_bf16x2(h0, h1);
+          wl[k] = pack_bf16x2(l0, l1);
+          split_bf16(-a.tau * xo[2 * k], h0, l0);
+          split_bf16(-a.tau * xo[2 * k + 1], h1, l1);
+          woh[k] = pack_bf16x2(h0, h1);
+          wol[k] = pack_bf16x2(l0, l1);
         }
+        const uint32_t o = swz128(r, pc);
+        *reinterpret_cast<uint4*>(qt + o) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+        *reinterpret_cast<uint4*>(qt + TILE + o) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+        *reinterpret_cast<uint4*>(qt + 2 * TILE + o) = make_uint4(woh[0], woh[1], woh[2], woh[3]);
+        *reinterpret_cast<uint4*>(qt + 3 * TILE + o) = make_uint4(wol[0], wol[1], wol[2], wol[3]);
       }
-      float acc[8][4];
+      if (pb == 0) colmax[tid] = 0u;   // UC * 64 == 256 == blockDim.x
+      issue_base(0);
+      const bool rows_active = pb + 16 * rg < npairs;   // this warp's pair rows hold any pair
+      for (int c = 0; c < nch; ++c) {
+        const int c0 = u0 + c * 64;
+        // residual codes of this chunk's rows (loads issued before the copy is awaited)
+        uint32_t craw[4][KM - 1];
+        uint16_t sraw[4][KM - 1];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        for (int u = 0; u < 4; ++u) {
+          const int e = tid + 256 * u, r = e >> 4, pc = e & 15;
+          const int t = c0 + r;
+          int rr[KM - 1];
 #pragma unroll
-      for (int ks = 0; ks < KS; ++ks) {
+          for (int q = 0; q < KM - 1; ++q) rr[q] = (t <= maxpos && q + 2 <= a.loop) ? (SP ? 0 : t) : -1;
+          if (SP && t <= maxpos) chain_rows<KM>(cv, a.j, b, t, a.loop, rr);
 #pragma unroll
-        for (int np = 0; np < 4; ++np) {
-          const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
-          const int ch = 2 * ks + ((lane >> 3) & 1);
-          const uint32_t off = (ch >> 3) * BOX + key * 128 + (((ch & 7) ^ (key & 7)) << 4);
-          uint32_t fh[4], fl[4], fb[4];
-          ldsm_x4(smem_u32(knh) + off, fh);
-          ldsm_x4(smem_u32(knl) + off, fl);
-          ldsm_x4(smem_u32(kbs) + off, fb);
+          for (int q = 0; q < KM - 1; ++q) {
+            craw[u][q] = 0u;
+            sraw[u][q] = 0;
+            if (rr[q] >= 0) {
+              const size_t ri = q0 + q * step + static_cast<size_t>(rr[q]);
+              const uint8_t* row = cv.codes + ri * rb;
+              craw[u][q] = bits == 4 ? *reinterpret_cast<const uint32_t*>(row + pc * 4)
+                                     : static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(row + pc * 2));
+              sraw[u][q] = cv.scales[ri * ns + ((pc * 8) >> cv.lg)];
+            }
+          }
+        }
+        cp_async_wait<0>();
+        __syncthreads();   // chunk c's base rows are in; every warp is done with chunk c - 1
+        if (c + 1 < nch) issue_base(c + 1);   // into the buffer chunk c - 1 used
+        // ---- new keys: base + code * scale of loops 2..l in loop order (fp32), split hi / lo
+        const uint8_t* kb_c = kbs + (c & 1) * TILE;
 #pragma unroll
-          for (int hlf = 0; hlf < 2; ++hlf) {
-            float* c = acc[2 * np + hlf];
-            mma_bf16_16816(c, qnh[ks], fh[2 * hlf], fh[2 * hlf + 1]);
-            mma_bf16_16816(c, qnl[ks], fh[2 * hlf], fh[2 * hlf + 1]);
-            mma_bf16_16816(c, qnh[ks], fl[2 * hlf], fl[2 * hlf + 1]);
-            mma_bf16_16816(c, qoh[ks], fb[2 * hlf], fb[2 * hlf + 1]);
-            mma_bf16_16816(c, qol[ks], fb[2 * hlf], fb[2 * hlf + 1]);
+        for (int u = 0; u < 4; ++u) {
+          const int e = tid + 256 * u, r = e >> 4, pc = e & 15;
+          const uint32_t o = swz128(r, pc);
+          const uint4 bw = *reinterpret_cast<const uint4*>(kb_c + o);
+          const uint32_t w[4] = {bw.x, bw.y, bw.z, bw.w};
+          float x[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            x[2 * k] = bf16_to_f(w[k] & 0xFFFF);
+            x[2 * k + 1] = bf16_to_f(w[k] >> 16);
+          }
+#pragma unroll
+          for (int q = 0; q < KM - 1; ++q) {
+            if (q + 2 > a.loop) break;
+            const float sc = half_bits_to_f(sraw[u][q]);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int cd = bits == 4 ? sext(static_cast<int>((craw[u][q] >> (4 * k)) & 0xFu), 4)
+                                       : sext(static_cast<int>((craw[u][q] >> (2 * k)) & 0x3u), 2);
+              x[k] = __fadd_rn(x[k], __fmul_rn(static_cast<float>(cd), sc));
+            }
+          }
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float h0, l0, h1, l1;
+            split_bf16(x[2 * k], h0, l0);
+            split_bf16(x[2 * k + 1], h1, l1);
+            hw[k] = pack_bf16x2(h0, h1);
+            lw[k] = pack_bf16x2(l0, l1);
+          }
+          *reinterpret_cast<uint4*>(knh + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(knl + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+        __syncthreads();
+        if (rows_active) {
+          float acc[4][4];
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            uint32_t an[4], al[4], aoh[4], aol[4];
+            const uint32_t qo_ = swz128(16 * rg + (lane & 15), 2 * ks + (lane >> 4));
+            ldsm_x4(qt_s + qo_, an);
+            ldsm_x4(qt_s + TILE + qo_, al);
+            ldsm_x4(qt_s + 2 * TILE + qo_, aoh);
+            ldsm_x4(qt_s + 3 * TILE + qo_, aol);
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+              const int key = 32 * ch2 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
+              const uint32_t ko = swz128(key, 2 * ks + ((lane >> 3) & 1));
+              uint32_t fh[4], fl[4], fb[4];
+              ldsm_x4(knh_s + ko, fh);
+              ldsm_x4(knl_s + ko, fl);
+              ldsm_x4(kbs_s + (c & 1) * TILE + ko, fb);
+#pragma unroll
+              for (int hlf = 0; hlf < 2; ++hlf) {
+                float* d = acc[2 * np + hlf];
+                mma_bf16_16816(d, an, fh[2 * hlf], fh[2 * hlf + 1]);
+                mma_bf16_16816(d, al, fh[2 * hlf], fh[2 * hlf + 1]);
+                mma_bf16_16816(d, an, fl[2 * hlf], fl[2 * hlf + 1]);
+                mma_bf16_16816(d, aoh, fb[2 * hlf], fb[2 * hlf + 1]);
+                mma_bf16_16816(d, aol, fb[2 * hlf], fb[2 * hlf + 1]);
+              }
+            }
+          }
+          // |delta| of causal columns, max over this warp's rows, then over the CTA
+          const int p0 = qpos[16 * rg + (lane >> 2)], p1 = qpos[16 * rg + (lane >> 2) + 8];
+#pragma unroll
+          for (int nt = 0; nt < 4; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int col = 32 * ch2 + nt * 8 + 2 * (lane & 3) + e;
+              float m = 0.f;
+              if (c0 + col <= p0) m = fmaxf(m, fabsf(acc[nt][e]));
+              if (c0 + col <= p1) m = fmaxf(m, fabsf(acc[nt][2 + e]));
+              m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+              m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+              m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+              if (lane < 4 && m > 0.f) atomicMax(&colmax[c * 64 + col], __float_as_uint(m));
+            }
           }
         }
       }
-      // |delta| of causal columns, max over this warp's rows, then over the CTA
-#pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int col = nt * 8 + 2 * (lane & 3) + e;
-          float m = 0.f;
-          if (c0 + col <= qpos[0]) m = fmaxf(m, fabsf(acc[nt][e]));
-          if (c0 + col <= qpos[1]) m = fmaxf(m, fabsf(acc[nt][2 + e]));
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
-          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
-          if (lane < 4 && m > 0.f) atomicMax(&colmax[col], __float_as_uint(m));
-        }
-      }
     }
     __syncthreads();
-    if (tid < nc) {
-      const float v = __uint_as_float(colmax[tid]);
-      a.col_keys[(static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols + c0 + tid] = v;
-      const int tl = a.plan.tile[p];
-      if (a.trace_ck && tl < a.trace_tiles)
-        a.trace_ck[((static_cast<size_t>(a.j) * a.trace_tiles + tl) * a.Hkv + g) * a.max_cols + c0 + tid] = v;
+    {
+      const int col = u0 + tid;
+      if (col <= maxpos) {
+        const float v = __uint_as_float(colmax[tid]);
+        a.col_keys[(static_cast<size_t>(seg) * a.Hkv + g) * a.max_cols + col] = v;
+        const int tl = a.plan.tile[p];
+        if (a.trace_ck && tl < a.trace_tiles)
+          a.trace_ck[((static_cast<size_t>(a.j) * a.trace_tiles + tl) * a.Hkv + g) * a.max_cols + col] = v;
+      }
     }
-    __syncthreads();   // the staged keys and colmax are reused by the next item
-    if (a.fold) fold_select(a, seg, g, a.plan.tile[p], maxpos + 1, reinterpret_cast<float*>(sm), &fold_last);
+    if (a.fold) fold_select(a, seg, g, a.plan.tile[p], maxpos + 1, reinterpret_cast<float*>(sm), &fold_last, UC * 64);
   }
 }
 
@@ -2059,190 +2269,64 @@ __global__ void __launch_bounds__(1024) k_select_cols(const SelColsArgs a) {
 }
 
 // ============================================================================
-// sparse-column correction of (O, lse) for one selected query and KV group:
-//   Mx = max(lse, s_new, s_old) over the query's columns C (k <= pos)
+// sparse-column correction of one selected query and KV group.  With
+// s_new = tau q_l.K_l and s_old = tau q_last.K_last over the query's columns C
+// (k <= pos), the corrected denominator and numerator are
 //   Z' = e^(lse-Mx) - sum_C e^(s_old-Mx) + sum_C e^(s_new-Mx)
 //   N' = e^(lse-Mx) O - sum_C e^(s_old-Mx) V_last + sum_C e^(s_new-Mx) V_l
-//   O = N'/Z', lse = Mx + ln Z', q_last = q_l
-// with s_new = tau q_l.K_l, s_old = tau q_last.K_last.  The column set is
-// split across CTAs (grid.y); each warp takes one column at a time and keeps a
-// running per-head maximum, so the sums above are accumulated in pieces that
-// are rescaled to the common maximum when merged.  The last CTA of a (query,
-// group) -- an atomic ticket, no waiting -- merges the pieces with the stored
-// (O, lse) term and writes the new state.
+// and O = N'/Z'.  The first two terms -- the attention over the columns outside
+// C, "the rest" -- do not change while C is fixed, so they are formed once, at
+// the token's first recomputation (last = 1: the stored state is the loop-1
+// attention (O, lse), and K_last, V_last are the base rows), and kept as
+// (M_r, Z_r, N_r) in (lse_state, z_state, o_state).  At every later
+// recomputation Z' = e^(M_r-Mx) Z_r + sum_C e^(s_new-Mx) and N' likewise, so the
+// old chains are never rebuilt again.  This is the same sum as the step-by-step
+// update (the old term of loop l is the new term of the token's previous
+// recomputation, with the same C); it is only grouped differently.  q_last
+// therefore stays the loop-1 query, which is what the delta scores of a tile's
+// first recomputation read.  A non-positive Z' is reported as non-finite.
 // ============================================================================
-template <int HD, int EPL, int GRP, int KM>
-__global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
-  pdl_trigger();
-  pdl_wait();
-  constexpr int GMAX = 8, NW = 8;
-  __shared__ float sm_m[NW][GMAX], sm_z[NW][GMAX];
-  __shared__ float sm_acc[NW][GMAX][HD];
-  __shared__ int ncs, is_last;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int i = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv, sp = blockIdx.y;
-  constexpr int grp = GRP;
-  const int tok = a.idx[i];
-  const int b = a.seq[tok], P = a.pos[tok], tl = a.tile[tok];
-  const int m_old = a.last[tok];
-  const CacheView& cv = a.cv;
-  const size_t cset = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
-  const int32_t* C = a.cols + cset * a.c;
-  // C is ascending: the query's columns are its prefix with C[k] <= pos; only
-  // this CTA's slice of C is needed, so count within the slice in parallel
-  const int ncol_all = a.ncols[cset];
-  const int k0s = sp * a.cols_per_cta;
-  const int kend = min(ncol_all, k0s + a.cols_per_cta);
-  const int kk = k0s + tid;
-  const int in_slice = (kk < kend && C[kk] <= P) ? 1 : 0;
-  const int cnt = __syncthreads_count(in_slice);
-  if (tid == 0) ncs = k0s + cnt;
-  // the group's query heads (new and last) in registers
-  float qn[GRP][EPL], qo[GRP][EPL];
-#pragma unroll
-  for (int h = 0; h < GRP; ++h) {
-    const size_t hq = static_cast<size_t>(g * grp + h);
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      qn[h][e] = a.q_cur[(static_cast<size_t>(i) * a.H + hq) * HD + lane * EPL + e];
-      qo[h][e] = a.q_last[(static_cast<size_t>(tok) * a.H + hq) * HD + lane * EPL + e];
-    }
+// The EPL base (bf16) values of one row held by a lane.
+template <int EPL>
+__device__ __forceinline__ void base_lane(const uint16_t* row, int lane, float* out) {
+  if (EPL == 4) {
+    const uint2 u = *reinterpret_cast<const uint2*>(row + lane * 4);
+    out[0] = bf16_to_f(u.x & 0xFFFF);
+    out[1] = bf16_to_f(u.x >> 16);
+    out[EPL == 4 ? 2 : 0] = bf16_to_f(u.y & 0xFFFF);
+    out[EPL == 4 ? 3 : 1] = bf16_to_f(u.y >> 16);
+  } else {
+    const uint32_t u = *reinterpret_cast<const uint32_t*>(row + lane * 2);
+    out[0] = bf16_to_f(u & 0xFFFF);
+    out[1] = bf16_to_f(u >> 16);
   }
-  __syncthreads();
-  const int k0 = k0s, k1 = ncs;
-  float m[GRP], z[GRP], acc[GRP][EPL];
-#pragma unroll
-  for (int h = 0; h < GRP; ++h) {
-    m[h] = -INFINITY;
-    z[h] = 0.f;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
-  }
-  for (int k = k0 + warp; k < k1; k += NW) {
-    const int col = C[k];
-    float klo[EPL], khi[EPL], vlo[EPL], vhi[EPL];
-    chain_lane2<EPL, KM>(cv, a.j, 0, b, g, col, m_old, a.loop, lane, klo, khi);
-    chain_lane2<EPL, KM>(cv, a.j, 1, b, g, col, m_old, a.loop, lane, vlo, vhi);
-#pragma unroll
-    for (int h = 0; h < GRP; ++h) {
-      float dn = 0.f, dl = 0.f;
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) {
-        dn += qn[h][e] * khi[e];
-        dl += qo[h][e] * klo[e];
-      }
-      dn = warp_sum(dn) * a.tau;
-      dl = warp_sum(dl) * a.tau;
-      const float mn = fmaxf(m[h], fmaxf(dn, dl));
-      const float sc = m[h] == -INFINITY ? 0.f : expf(m[h] - mn);
-      const float en = expf(dn - mn), eo = expf(dl - mn);
-      z[h] = z[h] * sc + (en - eo);
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) acc[h][e] = acc[h][e] * sc + en * vhi[e] - eo * vlo[e];
-      m[h] = mn;
-    }
-  }
-  // merge the warps of this CTA
-#pragma unroll
-  for (int h = 0; h < GRP; ++h) {
-    if (lane == 0) {
-      sm_m[warp][h] = m[h];
-      sm_z[warp][h] = z[h];
-    }
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) sm_acc[warp][h][lane * EPL + e] = acc[h][e];
-  }
-  __syncthreads();
-  const size_t pbase = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits + sp;
-  for (int e = tid; e < grp * HD; e += 256) {
-    const int h = e / HD, dd = e % HD;
-    float M = -INFINITY;
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][h]);
-    float A = 0.f, Z = 0.f;
-    if (M != -INFINITY)
-      for (int w = 0; w < NW; ++w) {
-        if (sm_m[w][h] == -INFINITY) continue;
-        const float f = expf(sm_m[w][h] - M);
-        A += sm_acc[w][h][dd] * f;
-        Z += sm_z[w][h] * f;
-      }
-    a.part_acc[(pbase * GMAX + h) * HD + dd] = A;
-    if (dd == 0) {
-      a.part_mz[(pbase * GMAX + h) * 2 + 0] = M;
-      a.part_mz[(pbase * GMAX + h) * 2 + 1] = Z;
-    }
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) {
-    const int old = atomicAdd(&a.counters[i * a.Hkv + g], 1);
-    is_last = (old == a.n_splits - 1);
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  const size_t q0 = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits;
-  // merge: warp h finds head h's common maximum and denominator (lanes over splits)
-  __shared__ float mg[GMAX], zg[GMAX], eg[GMAX];
-  for (int h = warp; h < grp; h += NW) {
-    const size_t so = static_cast<size_t>(tok) * a.H + g * grp + h;
-    const float L = a.lse_state[so];
-    float M = L;
-    for (int s2 = lane; s2 < a.n_splits; s2 += 32) M = fmaxf(M, __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2]));
-    M = warp_max(M);
-    float Z = 0.f;
-    for (int s2 = lane; s2 < a.n_splits; s2 += 32) {
-      const float ms = __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2]);
-      if (ms != -INFINITY) Z += expf(ms - M) * __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2 + 1]);
-    }
-    Z = warp_sum(Z);
-    if (lane == 0) {
-      const float el = expf(L - M);
-      mg[h] = M;
-      eg[h] = el;
-      zg[h] = el + Z;
-    }
-  }
-  __syncthreads();
-  for (int e = tid; e < grp * HD; e += 256) {
-    const int h = e / HD, dd = e % HD;
-    const int hq = g * grp + h;
-    const size_t so = static_cast<size_t>(tok) * a.H + hq;
-    const float M = mg[h], Z = zg[h];
-    float N = eg[h] * a.o_state[so * HD + dd];
-#pragma unroll 8
-    for (int s2 = 0; s2 < a.n_splits; ++s2) {
-      const float ms = __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 2]);
-      const float pa = __ldcg(&a.part_acc[((q0 + s2) * GMAX + h) * HD + dd]);
-      N += ms == -INFINITY ? 0.f : expf(ms - M) * pa;
-    }
-    if (!(Z > 0.f) && a.status) atomicOr(a.status, kErrBadIndex);
-    const float ov = N / Z;
-    a.o_state[so * HD + dd] = ov;
-    a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + dd] = f_to_bf16(ov);
-    a.q_last[so * HD + dd] = a.q_cur[(static_cast<size_t>(i) * a.H + hq) * HD + dd];
-    if (dd == 0) a.lse_state[so] = M + logf(Z);
-  }
-  if (tid == 0) a.counters[i * a.Hkv + g] = 0;
 }
-
-// ============================================================================
-// The correction for few selected queries (decode): the column slices of one
-// (query, KV group) are the CTAs of one cluster (kCorrCluster CTAs of
-// kCorrWarps warps).  The query's slot record, its column-set count and the
-// first column ids are requested together; warp w of rank r takes columns
-// r*per + w + u*kCorrWarps of the set, two at a time, with every K and V chain
-// load of both issued before any arithmetic.  The warps' pieces (per-head max,
-// denominator, numerator) are merged in the CTA with one weight per (warp,
-// head); then rank r merges outputs [r*E/CS, (r+1)*E/CS) of every rank, in rank
-// order, over distributed shared memory, together with the stored (O, lse)
-// term.  No global scratch, fence or ticket.  grid (kCorrCluster, n_sel * Hkv).
-// ============================================================================
+// One column of the running sums (per head: max m, then e^(s - m)-weighted
+// denominators and numerators, rescaled when m grows): the new term only ...
 template <int EPL, int GRP>
-__device__ __forceinline__ void corr_column(const float (&qn)[GRP][EPL], const float (&qo)[GRP][EPL],
-                                            const float* klo, const float* khi, const float* vlo,
-                                            const float* vhi, float tau, float (&m)[GRP], float (&z)[GRP],
-                                            float (&acc)[GRP][EPL]) {
+__device__ __forceinline__ void corr_new(const float (&qn)[GRP][EPL], const float* khi, const float* vhi, float tau,
+                                         float (&m)[GRP], float (&zn)[GRP], float (&an)[GRP][EPL]) {
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    float dn = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) dn += qn[h][e] * khi[e];
+    dn = warp_sum(dn) * tau;
+    const float mn = fmaxf(m[h], dn);
+    const float sc = m[h] == -INFINITY ? 0.f : expf(m[h] - mn);
+    const float en = expf(dn - mn);
+    zn[h] = zn[h] * sc + en;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) an[h][e] = an[h][e] * sc + en * vhi[e];
+    m[h] = mn;
+  }
+}
+// ... or the new and the old terms, with one running max per head
+template <int EPL, int GRP>
+__device__ __forceinline__ void corr_both(const float (&qn)[GRP][EPL], const float (&qo)[GRP][EPL],
+                                          const float* klo, const float* khi, const float* vlo, const float* vhi,
+                                          float tau, float (&m)[GRP], float (&zn)[GRP], float (&an)[GRP][EPL],
+                                          float (&zo)[GRP], float (&ao)[GRP][EPL]) {
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
     float dn = 0.f, dl = 0.f;
@@ -2256,28 +2340,631 @@ __device__ __forceinline__ void corr_column(const float (&qn)[GRP][EPL], const f
     const float mn = fmaxf(m[h], fmaxf(dn, dl));
     const float sc = m[h] == -INFINITY ? 0.f : expf(m[h] - mn);
     const float en = expf(dn - mn), eo = expf(dl - mn);
-    z[h] = z[h] * sc + (en - eo);
+    zn[h] = zn[h] * sc + en;
+    zo[h] = zo[h] * sc + eo;
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[h][e] = acc[h][e] * sc + en * vhi[e] - eo * vlo[e];
+    for (int e = 0; e < EPL; ++e) {
+      an[h][e] = an[h][e] * sc + en * vhi[e];
+      ao[h][e] = ao[h][e] * sc + eo * vlo[e];
+    }
     m[h] = mn;
   }
 }
 
-template <int HD, int EPL, int GRP, int KM>
+// The state update of one output element (head h, dim dd) from the merged
+// pieces -- the new-term denominator zn and numerator nn relative to their
+// maximum Mn, the old-term ones (zo, no) relative to Mo -- and the stored
+// state, read before any of it is rewritten: on a first recomputation
+// (Ls, O) = the loop-1 (lse, O) element, otherwise (Ls, Zs, O) = the rest
+// (M_r, Z_r, N_r).  Returns the corrected output; on a first recomputation
+// also sets the rest to store.
+struct CorrRest {
+  float m, z, n;
+};
+__device__ __forceinline__ float corr_finish(bool first, float Mn, float zn, float nn, float Mo, float zo, float no,
+                                             float Ls, float Zs, float O, CorrRest& rest, int* status) {
+  float Mr, Zr, Nr;
+  if (first) {   // remove the loop-1 terms of C from the loop-1 attention
+    Mr = fmaxf(Ls, Mo);
+    const float es = expf(Ls - Mr), eo = Mo == -INFINITY ? 0.f : expf(Mo - Mr);
+    Zr = es - eo * zo;
+    Nr = es * O - eo * no;
+    rest.m = Mr;
+    rest.z = Zr;
+    rest.n = Nr;
+  } else {       // the stored rest
+    Mr = Ls;
+    Zr = Zs;
+    Nr = O;
+  }
+  const float M = fmaxf(Mr, Mn);
+  const float er = expf(Mr - M), en = Mn == -INFINITY ? 0.f : expf(Mn - M);
+  const float Z = er * Zr + en * zn;
+  if (!(Z > 0.f) && status) atomicOr(status, kErrNonfinite);
+  return (er * Nr + en * nn) / Z;
+}
+
+// The general form (prefill; decode with the ticket merge).  The column set is
+// split across CTAs (grid.y); each warp takes one column at a time and keeps a
+// running per-head maximum, so the sums are accumulated in pieces that are
+// rescaled to the common maximum when merged.  The last CTA of a (query,
+// group) -- an atomic ticket, no waiting -- merges the pieces with the stored
+// state.  Partials: part_acc [rows][2][8][hd] (new, old), part_mz [rows][8][3]
+// (max, new denominator, old denominator).
+template <int HD, int EPL, int GRP, int KM, bool SP>
+__global__ void __launch_bounds__(256) k_correct(const CorrectArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int GMAX = 8, NW = 8;
+  __shared__ float sm_m[NW][GMAX], sm_zn[NW][GMAX], sm_zo[NW][GMAX];
+  __shared__ float sm_acc[NW][GRP][HD];   // the warps' numerators: new term, then (first recomputation) old
+  __shared__ int ncs, is_last;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i = blockIdx.x / a.Hkv, g = blockIdx.x % a.Hkv, sp = blockIdx.y;
+  constexpr int grp = GRP;
+  const int tok = a.idx[i];
+  const int b = a.seq[tok], P = a.pos[tok], tl = a.tile[tok];
+  const int m_old = a.last[tok];
+  const bool first = m_old == 1;
+  const CacheView& cv = a.cv;
+  const size_t cset = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
+  const int32_t* C = a.cols + cset * a.c;
+  // C is ascending: the query's columns are its prefix with C[k] <= pos; only
+  // this CTA's slice of C is needed, so count within the slice in parallel
+  const int ncol_all = a.ncols[cset];
+  const int k0s = sp * a.cols_per_cta;
+  const int kend = min(ncol_all, k0s + a.cols_per_cta);
+  const int kk = k0s + tid;
+  const int in_slice = (kk < kend && C[kk] <= P) ? 1 : 0;
+  const int cnt = __syncthreads_count(in_slice);
+  if (tid == 0) ncs = k0s + cnt;
+  // the group's query heads (new, and on a first recomputation the loop-1 ones) in registers
+  float qn[GRP][EPL], qo[GRP][EPL];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    const size_t hq = static_cast<size_t>(g * grp + h);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      qn[h][e] = a.q_cur[(static_cast<size_t>(i) * a.H + hq) * HD + lane * EPL + e];
+      qo[h][e] = first ? a.q_last[(static_cast<size_t>(tok) * a.H + hq) * HD + lane * EPL + e] : 0.f;
+    }
+  }
+  __syncthreads();
+  const int k0 = k0s, k1 = ncs;
+  float m[GRP], zn[GRP], zo[GRP], an[GRP][EPL], ao[GRP][EPL];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    m[h] = -INFINITY;
+    zn[h] = zo[h] = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) an[h][e] = ao[h][e] = 0.f;
+  }
+  for (int k = k0 + warp; k < k1; k += NW) {
+    const int col = C[k];
+    float klo[EPL], khi[EPL], vlo[EPL], vhi[EPL];
+    int rr[KM - 1];   // sparse layout: the column's pool rows, shared by its K and V chains
+    if (SP) chain_rows<KM>(cv, a.j, b, col, a.loop, rr);
+    chain_lane2<EPL, KM, SP>(cv, a.j, 0, b, g, col, 1, a.loop, lane, klo, khi, SP ? rr : nullptr);
+    chain_lane2<EPL, KM, SP>(cv, a.j, 1, b, g, col, 1, a.loop, lane, vlo, vhi, SP ? rr : nullptr);
+    if (first)
+      corr_both<EPL, GRP>(qn, qo, klo, khi, vlo, vhi, a.tau, m, zn, an, zo, ao);
+    else
+      corr_new<EPL, GRP>(qn, khi, vhi, a.tau, m, zn, an);
+  }
+  // merge the warps of this CTA: the new-term numerators, then (first
+  // recomputation) the old-term ones through the same buffer
+  const size_t pbase = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits + sp;
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    if (lane == 0) {
+      sm_m[warp][h] = m[h];
+      sm_zn[warp][h] = zn[h];
+      sm_zo[warp][h] = zo[h];
+    }
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) sm_acc[warp][h][lane * EPL + e] = an[h][e];
+  }
+  for (int term = 0; term < (first ? 2 : 1); ++term) {
+    __syncthreads();
+    for (int e = tid; e < grp * HD; e += 256) {
+      const int h = e / HD, dd = e % HD;
+      float M = -INFINITY;
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][h]);
+      float A = 0.f, Zn = 0.f, Zo = 0.f;
+      if (M != -INFINITY)
+        for (int w = 0; w < NW; ++w) {
+          if (sm_m[w][h] == -INFINITY) continue;
+          const float f = expf(sm_m[w][h] - M);
+          A += sm_acc[w][h][dd] * f;
+          Zn += sm_zn[w][h] * f;
+          Zo += sm_zo[w][h] * f;
+        }
+      a.part_acc[((pbase * 2 + term) * GMAX + h) * HD + dd] = A;
+      if (dd == 0 && term == 0) {
+        a.part_mz[(pbase * GMAX + h) * 3 + 0] = M;
+        a.part_mz[(pbase * GMAX + h) * 3 + 1] = Zn;
+        a.part_mz[(pbase * GMAX + h) * 3 + 2] = Zo;
+      }
+    }
+    if (term == 0 && first) {
+      __syncthreads();
+#pragma unroll
+      for (int h = 0; h < GRP; ++h)
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) sm_acc[warp][h][lane * EPL + e] = ao[h][e];
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    const int old = atomicAdd(&a.counters[i * a.Hkv + g], 1);
+    is_last = (old == a.n_splits - 1);
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  const size_t q0 = (static_cast<size_t>(i) * a.Hkv + g) * a.n_splits;
+  // merge: warp h finds head h's common maximum and denominators (lanes over
+  // splits) and reads the head's stored scalars, before any is rewritten
+  __shared__ float mg[GMAX], zng[GMAX], zog[GMAX], lsg[GMAX], zsg[GMAX];
+  for (int h = warp; h < grp; h += NW) {
+    if (lane == 0) {
+      const size_t so = static_cast<size_t>(tok) * a.H + g * grp + h;
+      lsg[h] = a.lse_state[so];
+      zsg[h] = first ? 0.f : a.z_state[so];
+    }
+    float M = -INFINITY;
+    for (int s2 = lane; s2 < a.n_splits; s2 += 32) M = fmaxf(M, __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 3]));
+    M = warp_max(M);
+    float Zn = 0.f, Zo = 0.f;
+    if (M != -INFINITY)
+      for (int s2 = lane; s2 < a.n_splits; s2 += 32) {
+        const float ms = __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 3]);
+        if (ms == -INFINITY) continue;
+        const float f = expf(ms - M);
+        Zn += f * __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 3 + 1]);
+        Zo += f * __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 3 + 2]);
+      }
+    Zn = warp_sum(Zn);
+    Zo = warp_sum(Zo);
+    if (lane == 0) {
+      mg[h] = M;
+      zng[h] = Zn;
+      zog[h] = Zo;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < grp * HD; e += 256) {
+    const int h = e / HD, dd = e % HD;
+    const int hq = g * grp + h;
+    const size_t so = static_cast<size_t>(tok) * a.H + hq;
+    const float M = mg[h];
+    float Nn = 0.f, No = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll 4
+      for (int s2 = 0; s2 < a.n_splits; ++s2) {
+        const float ms = __ldcg(&a.part_mz[((q0 + s2) * GMAX + h) * 3]);
+        if (ms == -INFINITY) continue;
+        const float f = expf(ms - M);
+        Nn += f * __ldcg(&a.part_acc[(((q0 + s2) * 2 + 0) * GMAX + h) * HD + dd]);
+        if (first) No += f * __ldcg(&a.part_acc[(((q0 + s2) * 2 + 1) * GMAX + h) * HD + dd]);
+      }
+    }
+    CorrRest rest;
+    const float ov = corr_finish(first, M, zng[h], Nn, M, zog[h], No, lsg[h], zsg[h], a.o_state[so * HD + dd], rest,
+                                 a.status);
+    a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + dd] = f_to_bf16(ov);
+    if (first) {
+      a.o_state[so * HD + dd] = rest.n;
+      if (dd == 0) {
+        a.lse_state[so] = rest.m;
+        a.z_state[so] = rest.z;
+      }
+    }
+  }
+  if (tid == 0) a.counters[i * a.Hkv + g] = 0;
+}
+
+// ============================================================================
+// The correction for prefill tiles on the tensor cores (head_dim 128).  All
+// selected queries of a tile share the tile's column set, so the set's rows
+// are gathered once per (tile, KV head) and 64 of its (query, head) pairs at a
+// time are corrected together, as a small attention over the gathered columns:
+// S = tau Q K^T and O += P V with warp-level bf16 products (fp32 operands as
+// hi + lo pairs, as in the prefill attention), an online softmax per row, and
+// the causal rule C[k] <= pos per row.  Warps 0-3 take the new term (this
+// loop's queries against the rebuilt chains of the columns), warps 4-7 the old
+// term (the loop-1 queries against the base rows) of the same staged chunk,
+// for the pairs on their first recomputation; each warp owns 16 pair rows.  The
+// pieces then meet in shared memory and each element is finished with the
+// stored state as in the other correction kernels.  Items are (plan entry,
+// KV head, pass of 64 pairs), grid-stride, one CTA per SM.
+// ============================================================================
+template <int KM, bool SP>
+__global__ void __launch_bounds__(256, 1) k_correct_tc(const CorrectArgs a) {
+  constexpr int HD = 128, TILE = 64 * 128 * 2, KS = HD / 16, NDT = HD / 8;
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ uint8_t sm_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+  // [0,1]: tau q_l hi / lo; [2,3]: tau q_last hi / lo; [4..9]: K new hi / lo, K base, V new hi / lo, V base
+  const uint32_t sb = smem_u32(sm);
+  auto tile_s = [&](int t) { return sb + static_cast<uint32_t>(t * TILE); };
+  float* park = reinterpret_cast<float*>(sm + 4 * TILE);   // after the last chunk: old-term pieces [64][HD]
+  __shared__ int rpos[64], rtok[64], rfirst[64];
+  __shared__ int cpos[64];
+  __shared__ float pm_o[64], pz_o[64];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int wr = warp & 3;          // pair-row group
+  const bool old_warp = warp >= 4;  // the old term
+  const int grp = a.H / a.Hkv;
+  const int nent = a.plan.counts[0];
+  const int npass = (a.q_tile * grp + 63) / 64;
+  const CacheView& cv = a.cv;
+  const int bits = cv.bits;
+  const size_t rb = cv.row_bytes_codes(), ns = cv.hd >> cv.lg;
+  const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * (SP ? cv.rows : cv.T);
+  for (int it = blockIdx.x; it < nent * a.Hkv * npass; it += gridDim.x) {
+    const int p = it / (a.Hkv * npass), g = (it / npass) % a.Hkv, pass = it % npass;
+    const int qb = a.plan.qb[p], qe = a.plan.qe[p], tl = a.plan.tile[p];
+    const int npairs = (qe - qb) * grp, pb = pass * 64;
+    if (pb >= npairs) continue;   // (uniform over the CTA)
+    const size_t cset = (static_cast<size_t>(a.j) * a.n_tiles + tl) * a.Hkv + g;
+    const int32_t* C = a.cols + cset * a.c;
+    const int ncol = a.ncols[cset];
+    const int b = a.meta[qb].seq;
+    const size_t q0 = ((((static_cast<size_t>(a.j) * (cv.K - 1)) * 2) * cv.B + b) * cv.Hkv + g) *
+                      static_cast<size_t>(SP ? cv.rows : cv.T);
+    __syncthreads();   // the previous item no longer reads shared memory
+    // ---- stage the pass's pairs: thread -> (pair row, 8-dim piece) x 4
+    bool my_first = false;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = tid + 256 * u, r = e >> 4, pc = e & 15;
+      const int pr = pb + r;
+      float xn[8], xo[8];
+      if (pr < npairs) {
+        const int qi = qb + pr / grp, hh = g * grp + pr % grp;
+        const SelMeta mq = a.meta[qi];
+        const float4* qn = reinterpret_cast<const float4*>(a.q_cur + (static_cast<size_t>(qi) * a.H + hh) * HD) + pc * 2;
+        const float4* qo = reinterpret_cast<const float4*>(a.q_last + (static_cast<size_t>(mq.tok) * a.H + hh) * HD) + pc * 2;
+        const float4 n0 = qn[0], n1 = qn[1], o0 = qo[0], o1 = qo[1];
+        xn[0] = n0.x; xn[1] = n0.y; xn[2] = n0.z; xn[3] = n0.w; xn[4] = n1.x; xn[5] = n1.y; xn[6] = n1.z; xn[7] = n1.w;
+        xo[0] = o0.x; xo[1] = o0.y; xo[2] = o0.z; xo[3] = o0.w; xo[4] = o1.x; xo[5] = o1.y; xo[6] = o1.z; xo[7] = o1.w;
+        if (pc == 0) {
+          rpos[r] = mq.pos;
+          rtok[r] = mq.tok;
+          rfirst[r] = mq.last == 1;
+        }
+        my_first = my_first || mq.last == 1;
+      } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) xn[k] = xo[k] = 0.f;
+        if (pc == 0) {
+          rpos[r] = -1;
+          rtok[r] = -1;
+          rfirst[r] = 0;
+        }
+      }
+      uint32_t wh[4], wl[4], woh[4], wol[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float h0, l0, h1, l1;
+        split_bf16(a.tau * xn[2 * k], h0, l0);
+        split_bf16(a.tau * xn[2 * k + 1], h1, l1);
+        wh[k] = pack_bf16x2(h0, h1);
+        wl[k] = pack_bf16x2(l0, l1);
+        split_bf16(a.tau * xo[2 * k], h0, l0);
+        split_bf16(a.tau * xo[2 * k + 1], h1, l1);
+        woh[k] = pack_bf16x2(h0, h1);
+        wol[k] = pack_bf16x2(l0, l1);
+      }
+      const uint32_t o = swz128(r, pc);
+      *reinterpret_cast<uint4*>(sm + o) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+      *reinterpret_cast<uint4*>(sm + TILE + o) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+      *reinterpret_cast<uint4*>(sm + 2 * TILE + o) = make_uint4(woh[0], woh[1], woh[2], woh[3]);
+      *reinterpret_cast<uint4*>(sm + 3 * TILE + o) = make_uint4(wol[0], wol[1], wol[2], wol[3]);
+    }
+    const bool old_on = __syncthreads_or(my_first ? 1 : 0) != 0;   // any pair on its first recomputation
+    // this warp's rows: r0 = 16 wr + lane / 4 and r0 + 8
+    const int r0 = 16 * wr + (lane >> 2), r1 = r0 + 8;
+    const int P0 = rpos[r0], P1 = rpos[r1];
+    const bool active = pb + 16 * wr < npairs && (!old_warp || old_on);
+    const uint32_t qsh = tile_s(old_warp ? 2 : 0), qsl = tile_s(old_warp ? 3 : 1);
+    float o[NDT][4];
+#pragma unroll
+    for (int n = 0; n < NDT; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.f, 0.f};
+    for (int k0 = 0; k0 < ncol; k0 += 64) {
+      // ---- gather the chunk's columns: thread -> (column row, 8-dim piece) x 4, K and V
+      uint4 bk[4], bv[4];
+      int tcol[4];
+      uint32_t ck[4][KM - 1], cvv[4][KM - 1];
+      uint16_t sk[4][KM - 1], svv[4][KM - 1];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = tid + 256 * u, r = e >> 4, pc = e & 15;
+        const bool ok = k0 + r < ncol;
+        const int t = ok ? C[k0 + r] : 0;
+        tcol[u] = ok ? t : 0x7fffffff;
+        bk[u] = ok ? *reinterpret_cast<const uint4*>(cv.base_row(a.j, 0, b, g, t) + pc * 8) : make_uint4(0, 0, 0, 0);
+        bv[u] = ok ? *reinterpret_cast<const uint4*>(cv.base_row(a.j, 1, b, g, t) + pc * 8) : make_uint4(0, 0, 0, 0);
+        int rr[KM - 1];
+#pragma unroll
+        for (int q = 0; q < KM - 1; ++q) rr[q] = (ok && q + 2 <= a.loop) ? (SP ? 0 : t) : -1;
+        if (SP && ok) chain_rows<KM>(cv, a.j, b, t, a.loop, rr);
+#pragma unroll
+        for (int q = 0; q < KM - 1; ++q) {
+          ck[u][q] = cvv[u][q] = 0u;
+          sk[u][q] = svv[u][q] = 0;
+          if (rr[q] >= 0) {
+            const size_t rik = q0 + q * step + static_cast<size_t>(rr[q]);
+            const size_t riv = rik + static_cast<size_t>(cv.B) * cv.Hkv * (SP ? cv.rows : cv.T);   // kv = 1
+            const uint8_t* rowk = cv.codes + rik * rb;
+            const uint8_t* rowv = cv.codes + riv * rb;
+            ck[u][q] = bits == 4 ? *reinterpret_cast<const uint32_t*>(rowk + pc * 4)
+                                 : static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(rowk + pc * 2));
+            cvv[u][q] = bits == 4 ? *reinterpret_cast<const uint32_t*>(rowv + pc * 4)
+                                  : static_cast<uint32_t>(*reinterpret_cast<const uint16_t*>(rowv + pc * 2));
+            sk[u][q] = cv.scales[rik * ns + ((pc * 8) >> cv.lg)];
+            svv[u][q] = cv.scales[riv * ns + ((pc * 8) >> cv.lg)];
+          }
+        }
+      }
+      __syncthreads();   // every warp is done with the previous chunk's tiles
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = tid + 256 * u, r = e >> 4, pc = e & 15;
+        const uint32_t off = swz128(r, pc);
+        if (pc == 0) cpos[r] = tcol[u];
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint4 bw = kv ? bv[u] : bk[u];
+          const uint32_t w[4] = {bw.x, bw.y, bw.z, bw.w};
+          float x[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            x[2 * k] = bf16_to_f(w[k] & 0xFFFF);
+            x[2 * k + 1] = bf16_to_f(w[k] >> 16);
+          }
+#pragma unroll
+          for (int q = 0; q < KM - 1; ++q) {
+            if (q + 2 > a.loop) break;
+            const float sc = half_bits_to_f(kv ? svv[u][q] : sk[u][q]);
+            const uint32_t cw = kv ? cvv[u][q] : ck[u][q];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              const int cd = bits == 4 ? sext(static_cast<int>((cw >> (4 * k)) & 0xFu), 4)
+                                       : sext(static_cast<int>((cw >> (2 * k)) & 0x3u), 2);
+              x[k] = __fadd_rn(x[k], __fmul_rn(static_cast<float>(cd), sc));
+            }
+          }
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float h0, l0, h1, l1;
+            split_bf16(x[2 * k], h0, l0);
+            split_bf16(x[2 * k + 1], h1, l1);
+            hw[k] = pack_bf16x2(h0, h1);
+            lw[k] = pack_bf16x2(l0, l1);
+          }
+          uint8_t* t0 = sm + (4 + 3 * kv) * TILE;   // new hi, new lo, base
+          *reinterpret_cast<uint4*>(t0 + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(t0 + TILE + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          *reinterpret_cast<uint4*>(t0 + 2 * TILE + off) = bw;
+        }
+      }
+      __syncthreads();
+      if (!active) continue;
+      // ---- scores of this warp's 16 rows x 64 columns
+      const uint32_t kh = tile_s(4), kl = tile_s(5), kbt = tile_s(6);
+      float sc[8][4];
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t ah[4], al[4];
+        const uint32_t qo_ = swz128(16 * wr + (lane & 15), 2 * ks + (lane >> 4));
+        ldsm_x4(qsh + qo_, ah);
+        ldsm_x4(qsl + qo_, al);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+          const int key = np * 16 + (lane & 7) + ((lane >> 4) << 3);
+          const uint32_t ko = swz128(key, 2 * ks + ((lane >> 3) & 1));
+          uint32_t fh[4];
+          ldsm_x4((old_warp ? kbt : kh) + ko, fh);
+#pragma unroll
+          for (int hlf = 0; hlf < 2; ++hlf) {
+            mma_bf16_16816(sc[2 * np + hlf], ah, fh[2 * hlf], fh[2 * hlf + 1]);
+            mma_bf16_16816(sc[2 * np + hlf], al, fh[2 * hlf], fh[2 * hlf + 1]);
+          }
+          if (!old_warp) {
+            uint32_t fl[4];
+            ldsm_x4(kl + ko, fl);
+#pragma unroll
+            for (int hlf = 0; hlf < 2; ++hlf) mma_bf16_16816(sc[2 * np + hlf], ah, fl[2 * hlf], fl[2 * hlf + 1]);
+          }
+        }
+      }
+      // causal rule per row: column C[k] is visible at position P when C[k] <= P
+      float tm[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int cp = cpos[nt * 8 + 2 * (lane & 3) + e];
+          if (cp > P0) sc[nt][e] = -INFINITY;
+          if (cp > P1) sc[nt][2 + e] = -INFINITY;
+          tm[0] = fmaxf(tm[0], sc[nt][e]);
+          tm[1] = fmaxf(tm[1], sc[nt][2 + e]);
+        }
+      }
+      float alpha[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        tm[r] = fmaxf(tm[r], __shfl_xor_sync(0xffffffffu, tm[r], 1));
+        tm[r] = fmaxf(tm[r], __shfl_xor_sync(0xffffffffu, tm[r], 2));
+        const float mn = fmaxf(m_run[r], tm[r]);
+        alpha[r] = (m_run[r] == -INFINITY || mn == -INFINITY) ? (m_run[r] == -INFINITY ? 0.f : 1.f)
+                                                               : expf(m_run[r] - mn);
+        m_run[r] = mn;
+      }
+      float rs[2] = {0.f, 0.f};
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float mr = m_run[e >> 1];
+          const float pv = (sc[nt][e] == -INFINITY) ? 0.f : expf(sc[nt][e] - mr);
+          sc[nt][e] = pv;
+          rs[e >> 1] += pv;
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) l_part[r] = l_part[r] * alpha[r] + rs[r];
+#pragma unroll
+      for (int n = 0; n < NDT; ++n) {
+        o[n][0] *= alpha[0];
+        o[n][1] *= alpha[0];
+        o[n][2] *= alpha[1];
+        o[n][3] *= alpha[1];
+      }
+      // ---- O += P V over the chunk's 64 columns (4 steps of 16)
+      const uint32_t vh = tile_s(7), vl = tile_s(8), vbt = tile_s(9);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        uint32_t ph[4], pl[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float* src = sc[2 * kk + (r >> 1)] + 2 * (r & 1);
+          float h0, l0, h1, l1;
+          split_bf16(src[0], h0, l0);
+          split_bf16(src[1], h1, l1);
+          ph[r] = pack_bf16x2(h0, h1);
+          pl[r] = pack_bf16x2(l0, l1);
+        }
+        const int vr = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int n2 = 0; n2 < NDT / 2; ++n2) {
+          const uint32_t vo = swz128(vr, n2 * 2 + (lane >> 4));
+          uint32_t vf[4];
+          ldsm_x4_t((old_warp ? vbt : vh) + vo, vf);
+          mma_bf16_16816(o[2 * n2], ph, vf[0], vf[1]);
+          mma_bf16_16816(o[2 * n2], pl, vf[0], vf[1]);
+          mma_bf16_16816(o[2 * n2 + 1], ph, vf[2], vf[3]);
+          mma_bf16_16816(o[2 * n2 + 1], pl, vf[2], vf[3]);
+          if (!old_warp) {
+            ldsm_x4_t(vl + vo, vf);
+            mma_bf16_16816(o[2 * n2], ph, vf[0], vf[1]);
+            mma_bf16_16816(o[2 * n2 + 1], ph, vf[2], vf[3]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 1);
+      l_part[r] += __shfl_xor_sync(0xffffffffu, l_part[r], 2);
+    }
+    __syncthreads();   // the column tiles are dead: the old-term warps park their pieces there
+    if (old_warp && old_on) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = r ? r1 : r0;
+#pragma unroll
+        for (int n = 0; n < NDT; ++n) {
+          const int d = n * 8 + 2 * (lane & 3);
+          *reinterpret_cast<float2*>(park + row * HD + d) = make_float2(o[n][2 * r], o[n][2 * r + 1]);
+        }
+        if ((lane & 3) == 0) {
+          pm_o[row] = m_run[r];
+          pz_o[row] = l_part[r];
+        }
+      }
+    }
+    __syncthreads();
+    if (!old_warp && pb + 16 * wr < npairs) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = r ? r1 : r0;
+        const int pr = pb + row;
+        const bool valid = pr < npairs;
+        const int slot = qb + pr / grp, hq = g * grp + pr % grp;
+        const size_t so = valid ? static_cast<size_t>(rtok[row]) * a.H + hq : 0;
+        const bool first = valid && rfirst[row] != 0;
+        float Ls = 0.f, Zs = 0.f;
+        float st[NDT][2];
+        if (valid) {
+          Ls = a.lse_state[so];
+          Zs = first ? 0.f : a.z_state[so];
+#pragma unroll
+          for (int n = 0; n < NDT; ++n) {
+            const float2 v = *reinterpret_cast<const float2*>(a.o_state + so * HD + n * 8 + 2 * (lane & 3));
+            st[n][0] = v.x;
+            st[n][1] = v.y;
+          }
+        }
+        __syncwarp();   // the quad has read the stored scalars before any lane rewrites them
+        if (!valid) continue;
+        const float Mo = first ? pm_o[row] : -INFINITY, zo = first ? pz_o[row] : 0.f;
+#pragma unroll
+        for (int n = 0; n < NDT; ++n) {
+          const int d = n * 8 + 2 * (lane & 3);
+          float ov[2], rn[2];
+          CorrRest rest{};
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float no = first ? park[row * HD + d + e] : 0.f;
+            ov[e] = corr_finish(first, m_run[r], l_part[r], o[n][2 * r + e], Mo, zo, no, Ls, Zs, st[n][e], rest,
+                                a.status);
+            rn[e] = rest.n;
+          }
+          *reinterpret_cast<uint32_t*>(a.o_bf16 + static_cast<size_t>(slot) * a.H * HD +
+                                       static_cast<size_t>(hq) * HD + d) = pack_bf16x2(ov[0], ov[1]);
+          if (first) {
+            *reinterpret_cast<float2*>(a.o_state + so * HD + d) = make_float2(rn[0], rn[1]);
+            if (n == 0 && (lane & 3) == 0) {
+              a.lse_state[so] = rest.m;
+              a.z_state[so] = rest.z;
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
+// ============================================================================
+// The correction for few selected queries (decode): the column slices of one
+// (query, KV group) are the CTAs of one cluster (kCorrCluster CTAs of
+// kCorrWarps warps).  The query's slot record, its column-set count and the
+// first column ids are requested together; warp w of rank r takes columns
+// r*per + w + u*kCorrWarps of the set, two at a time (later recomputations:
+// the new chains only) or one at a time (a first recomputation: new and base
+// rows), with every K and V chain load issued before any arithmetic.  The
+// warps' pieces (per-head max, denominators, numerators) are merged in the CTA
+// with one weight per (warp, head); then rank r merges outputs
+// [r*E/CS, (r+1)*E/CS) of every rank, in rank order, over distributed shared
+// memory, with the stored state.  No global scratch, fence or ticket.
+// grid (kCorrCluster, n_sel * Hkv).
+// ============================================================================
+template <int HD, int EPL, int GRP, int KM, bool SP>
 __global__ void __launch_bounds__(32 * kCorrWarps) k_correct_cluster(const CorrectArgs a) {
   pdl_trigger();
   constexpr int NW = kCorrWarps, CS = kCorrCluster, E = GRP * HD, NT = 32 * NW;
-  extern __shared__ float sm_acc[];   // [NW][GRP][HD]
-  __shared__ float sm_m[NW][GRP], sm_z[NW][GRP], sm_w[NW][GRP];
-  __shared__ float pm[GRP], pz[GRP];
-  __shared__ float pacc[GRP][HD];
+  extern __shared__ float sm_acc[];   // [2][NW][GRP][HD]: new-term numerators, then old-term ones
+  __shared__ float sm_m[2][NW][GRP], sm_z[2][NW][GRP], sm_w[2][NW][GRP];
+  __shared__ float pm[2][GRP], pz[2][GRP];
+  __shared__ float pacc[2][GRP][HD];
   cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rank = static_cast<int>(cluster.block_rank());
   const int i = blockIdx.y / a.Hkv, g = blockIdx.y % a.Hkv;
   pdl_wait();
   const SelMeta mt = a.meta[i];
-  const int tok = mt.tok, b = mt.seq, m_old = mt.last;
+  const int tok = mt.tok, b = mt.seq;
+  const bool first = mt.last == 1;
+  const int nterm = first ? 2 : 1;
   const CacheView& cv = a.cv;
   const size_t cset = (static_cast<size_t>(a.j) * a.n_tiles + mt.tile) * a.Hkv + g;
   const int32_t* C = a.cols + cset * a.c;
@@ -2289,86 +2976,145 @@ __global__ void __launch_bounds__(32 * kCorrWarps) k_correct_cluster(const Corre
   int col_first[2];
 #pragma unroll
   for (int u = 0; u < 2; ++u) col_first[u] = k0 + warp + u * NW < k1 ? C[k0 + warp + u * NW] : -1;
-  float qn[GRP][EPL], qo[GRP][EPL];
-#pragma unroll
-  for (int h = 0; h < GRP; ++h) {
-    const size_t hq = static_cast<size_t>(g * GRP + h);
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) {
-      qn[h][e] = a.q_cur[(static_cast<size_t>(i) * a.H + hq) * HD + lane * EPL + e];
-      qo[h][e] = a.q_last[(static_cast<size_t>(tok) * a.H + hq) * HD + lane * EPL + e];
-    }
-  }
   // rank r merges elements [r*E/CS, (r+1)*E/CS) of the (head, dim) outputs at the
   // end; the stored state it merges into is requested now, not after the barrier
   const int me = (rank * E) / CS + tid;
   const bool merger = me < ((rank + 1) * E) / CS;
-  float st_o = 0.f, st_l = 0.f, q_now = 0.f;
+  float st_o = 0.f, st_l = 0.f, st_z = 0.f;
   if (merger) {
     const size_t so = static_cast<size_t>(tok) * a.H + g * GRP + me / HD;
     st_o = a.o_state[so * HD + me % HD];
     st_l = a.lse_state[so];
-    q_now = a.q_cur[(static_cast<size_t>(i) * a.H + g * GRP + me / HD) * HD + me % HD];
+    st_z = first ? 0.f : a.z_state[so];
   }
   const int k1v = min(k1, nvalid);
-  float m[GRP], z[GRP], acc[GRP][EPL];
+  auto col_at = [&](int k) { return k == k0 + warp ? col_first[0] : (k == k0 + warp + NW ? col_first[1] : C[k]); };
+  // sparse storage: the pool rows of this CTA's columns, staged once ([column][level])
+  __shared__ int rows_sm[SP ? 64 * (KM - 1) : 1];
+  const bool rows_staged = SP && per <= 64;
+  if (rows_staged) {
+    for (int e = tid; e < per * (KM - 1); e += NT) {
+      const int kk = e / (KM - 1), q = e % (KM - 1), k = k0 + kk;
+      const int col = k < k1v ? C[k] : -1;
+      rows_sm[e] = (col >= 0 && q + 2 <= a.loop) ? cv.ridx[cv.ridx_index(a.j, q + 2, b, col)] : -1;
+    }
+    __syncthreads();
+  }
+  float q[GRP][EPL], m[GRP], z[GRP], acc[GRP][EPL];
+  auto reset = [&]() {
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) {
+      m[h] = -INFINITY;
+      z[h] = 0.f;
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
+    }
+  };
+  auto park = [&](int term) {   // this warp's piece of one term, to shared memory
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) {
+      if (lane == 0) {
+        sm_m[term][warp][h] = m[h];
+        sm_z[term][warp][h] = z[h];
+      }
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) sm_acc[((term * NW + warp) * GRP + h) * HD + lane * EPL + e] = acc[h][e];
+    }
+  };
+  if (first) {
+    // old term: the loop-1 queries against the base rows (the loop-1 K, V)
+#pragma unroll
+    for (int h = 0; h < GRP; ++h) {
+      const size_t hq = static_cast<size_t>(g * GRP + h);
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) q[h][e] = a.q_last[(static_cast<size_t>(tok) * a.H + hq) * HD + lane * EPL + e];
+    }
+    reset();
+    for (int kb = k0 + warp; kb < k1v; kb += 2 * NW) {
+      float kr[2][EPL], vr[2][EPL];
+      int col[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        col[u] = kb + u * NW < k1v ? col_at(kb + u * NW) : -1;
+        if (col[u] < 0) continue;
+        base_lane<EPL>(cv.base_row(a.j, 0, b, g, col[u]), lane, kr[u]);
+        base_lane<EPL>(cv.base_row(a.j, 1, b, g, col[u]), lane, vr[u]);
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+        if (col[u] >= 0) corr_new<EPL, GRP>(q, kr[u], vr[u], a.tau, m, z, acc);
+    }
+    park(1);
+  }
+  // new term: this loop's queries against the rebuilt chains, CPI columns at
+  // a time (one with sparse storage, whose index rows would otherwise not fit
+  // in registers beside the chains)
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
-    m[h] = -INFINITY;
-    z[h] = 0.f;
+    const size_t hq = static_cast<size_t>(g * GRP + h);
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
+    for (int e = 0; e < EPL; ++e) q[h][e] = a.q_cur[(static_cast<size_t>(i) * a.H + hq) * HD + lane * EPL + e];
   }
-  for (int kb = k0 + warp; kb < k1v; kb += 2 * NW) {
-    int col[2];
+  reset();
+  {
+    constexpr int CPI = SP ? 1 : 2;
+    for (int kb = k0 + warp; kb < k1v; kb += CPI * NW) {
+      int col[CPI];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int k = kb + u * NW;
-      col[u] = k < k1v ? (kb == k0 + warp ? col_first[u] : C[k]) : -1;
+      for (int u = 0; u < CPI; ++u) col[u] = kb + u * NW < k1v ? col_at(kb + u * NW) : -1;
+      float klo[CPI][EPL], khi[CPI][EPL], vlo[CPI][EPL], vhi[CPI][EPL];
+      int rr[CPI][KM - 1];
+      if (SP) {
+#pragma unroll
+        for (int u = 0; u < CPI; ++u) {
+          if (col[u] < 0) continue;
+          if (rows_staged) {
+#pragma unroll
+            for (int q = 0; q < KM - 1; ++q) rr[u][q] = rows_sm[(kb + u * NW - k0) * (KM - 1) + q];
+          } else {
+            chain_rows<KM>(cv, a.j, b, col[u], a.loop, rr[u]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < CPI; ++u) {
+        if (col[u] < 0) continue;
+        chain_lane2<EPL, KM, SP>(cv, a.j, 0, b, g, col[u], a.loop, a.loop, lane, klo[u], khi[u],
+                                 SP ? rr[u] : nullptr);
+        chain_lane2<EPL, KM, SP>(cv, a.j, 1, b, g, col[u], a.loop, a.loop, lane, vlo[u], vhi[u],
+                                 SP ? rr[u] : nullptr);
+      }
+#pragma unroll
+      for (int u = 0; u < CPI; ++u)
+        if (col[u] >= 0) corr_new<EPL, GRP>(q, khi[u], vhi[u], a.tau, m, z, acc);
     }
-    float klo[2][EPL], khi[2][EPL], vlo[2][EPL], vhi[2][EPL];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      if (col[u] < 0) continue;
-      chain_lane2<EPL, KM>(cv, a.j, 0, b, g, col[u], m_old, a.loop, lane, klo[u], khi[u]);
-      chain_lane2<EPL, KM>(cv, a.j, 1, b, g, col[u], m_old, a.loop, lane, vlo[u], vhi[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-      if (col[u] >= 0) corr_column<EPL, GRP>(qn, qo, klo[u], khi[u], vlo[u], vhi[u], a.tau, m, z, acc);
   }
-#pragma unroll
-  for (int h = 0; h < GRP; ++h) {
-    if (lane == 0) {
-      sm_m[warp][h] = m[h];
-      sm_z[warp][h] = z[h];
-    }
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) sm_acc[(warp * GRP + h) * HD + lane * EPL + e] = acc[h][e];
-  }
+  park(0);
   __syncthreads();
-  // this CTA's piece: one weight per (warp, head), then the weighted sums in warp order
-  if (tid < GRP) {
+  // this CTA's piece of each term: one weight per (warp, head), then the
+  // weighted sums in warp order
+  if (tid < nterm * GRP) {
+    const int term = tid / GRP, h = tid % GRP;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[w][tid]);
+    for (int w = 0; w < NW; ++w) M = fmaxf(M, sm_m[term][w][h]);
     float Z = 0.f;
 #pragma unroll
     for (int w = 0; w < NW; ++w) {
-      const float f = sm_m[w][tid] == -INFINITY ? 0.f : expf(sm_m[w][tid] - M);
-      sm_w[w][tid] = f;
-      Z += f * sm_z[w][tid];
+      const float f = sm_m[term][w][h] == -INFINITY ? 0.f : expf(sm_m[term][w][h] - M);
+      sm_w[term][w][h] = f;
+      Z += f * sm_z[term][w][h];
     }
-    pm[tid] = M;
-    pz[tid] = Z;
+    pm[term][h] = M;
+    pz[term][h] = Z;
   }
   __syncthreads();
-  for (int e = tid; e < E; e += NT) {
-    const int h = e / HD, dd = e % HD;
+  for (int e = tid; e < nterm * E; e += NT) {
+    const int term = e / E, h = (e % E) / HD, dd = e % HD;
     float A = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) A += sm_w[w][h] * sm_acc[(w * GRP + h) * HD + dd];
-    pacc[h][dd] = A;
+    for (int w = 0; w < NW; ++w) A += sm_w[term][w][h] * sm_acc[((term * NW + w) * GRP + h) * HD + dd];
+    pacc[term][h][dd] = A;
   }
   cluster.sync();
   if (merger) {
@@ -2377,32 +3123,45 @@ __global__ void __launch_bounds__(32 * kCorrWarps) k_correct_cluster(const Corre
     const size_t so = static_cast<size_t>(tok) * a.H + hq;
     // every rank's piece is requested before any is used, so the distributed
     // shared-memory round trips overlap; the merge itself runs in rank order
-    float rm[CS], rz[CS], ra[CS];
+    float Mt[2], Zt[2], Nt[2];
 #pragma unroll
-    for (int r = 0; r < CS; ++r) {
-      rm[r] = *cluster.map_shared_rank(&pm[h], r);
-      rz[r] = *cluster.map_shared_rank(&pz[h], r);
-      ra[r] = *cluster.map_shared_rank(&pacc[h][dd], r);
+    for (int term = 0; term < 2; ++term) {
+      Mt[term] = -INFINITY;
+      Zt[term] = Nt[term] = 0.f;
+      if (term >= nterm) continue;
+      float rm[CS], rz[CS], ra[CS];
+#pragma unroll
+      for (int r = 0; r < CS; ++r) {
+        rm[r] = *cluster.map_shared_rank(&pm[term][h], r);
+        rz[r] = *cluster.map_shared_rank(&pz[term][h], r);
+        ra[r] = *cluster.map_shared_rank(&pacc[term][h][dd], r);
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < CS; ++r) M = fmaxf(M, rm[r]);
+      float Z = 0.f, N = 0.f;
+#pragma unroll
+      for (int r = 0; r < CS; ++r) {
+        if (rm[r] == -INFINITY) continue;
+        const float f = expf(rm[r] - M);
+        Z += f * rz[r];
+        N += f * ra[r];
+      }
+      Mt[term] = M;
+      Zt[term] = Z;
+      Nt[term] = N;
     }
-    const float L = st_l;
-    float M = L;
-#pragma unroll
-    for (int r = 0; r < CS; ++r) M = fmaxf(M, rm[r]);
-    const float el = expf(L - M);
-    float Z = el, N = el * st_o;
-#pragma unroll
-    for (int r = 0; r < CS; ++r) {
-      if (rm[r] == -INFINITY) continue;
-      const float f = expf(rm[r] - M);
-      Z += f * rz[r];
-      N += f * ra[r];
-    }
-    if (!(Z > 0.f) && a.status) atomicOr(a.status, kErrBadIndex);
-    const float ov = N / Z;
-    a.o_state[so * HD + dd] = ov;
+    CorrRest rest;
+    const float ov = corr_finish(first, Mt[0], Zt[0], Nt[0], Mt[1], Zt[1], Nt[1], st_l, st_z, st_o, rest, a.status);
     a.o_bf16[static_cast<size_t>(i) * a.H * HD + static_cast<size_t>(hq) * HD + dd] = f_to_bf16(ov);
-    a.q_last[so * HD + dd] = q_now;
-    if (dd == 0) a.lse_state[so] = M + logf(Z);
+    // every rank read the stored scalars before the first cluster barrier
+    if (first) {
+      a.o_state[so * HD + dd] = rest.n;
+      if (dd == 0) {
+        a.lse_state[so] = rest.m;
+        a.z_state[so] = rest.z;
+      }
+    }
   }
   cluster.sync();
 }
@@ -2633,32 +3392,48 @@ cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, co
   return launch_k(g_pdl, k_plan_tiles, dim3(1), dim3(1024), 0, s, idx, n_sel, tile, has_c, p);
 }
 // (both also stage one row of column keys, up to kSelColsSmemKeys, for the folded selection)
-size_t dscore_tc_smem() { return std::max<size_t>(1024 + 3 * 64 * 128 * 2, kSelColsSmemKeys * 4 + 1024); }
+size_t dscore_tc_smem() { return 1024 + 8 * 64 * 128 * 2; }   // 4 query tiles, 2 base stages, new hi / lo
 size_t dscore_smem(int hd) {
-  return std::max<size_t>((static_cast<size_t>(2) * 64 * (hd + 1) + 2 * 16 * hd + 4 * 64) * 4, kSelColsSmemKeys * 4);
+  return std::max<size_t>(static_cast<size_t>(2) * kDsPairs * 4 * (hd / 4 + 4) * 4, kSelColsSmemKeys * 4);
 }
 cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s) {
-  // grid-stride over (tile, KV head, chunk) items: at most two CTAs per SM
-  const int items = max_need * a.Hkv * max_chunks;
-  dim3 grid(items < 2 * kDscoreSMs ? items : 2 * kDscoreSMs);
-  const size_t sm = dscore_smem(a.hd);
   DScoreArgs b = a;
   b.max_chunks = max_chunks;
-  if (a.tc && a.hd == 128) {   // prefill tiles: the tensor-core kernel, four CTAs per SM
-    const dim3 g4(items < 4 * kDscoreSMs ? items : 4 * kDscoreSMs);
+  if (a.tc && a.hd == 128) {   // prefill tiles: the tensor-core kernel, one CTA per SM
+    // grid-stride over (tile, KV head, unit of kDsTcUnit chunks) items
+    const int items = max_need * a.Hkv * ((max_chunks + kDsTcUnit - 1) / kDsTcUnit);
+    const dim3 g1(items < kDscoreSMs ? items : kDscoreSMs);
     const size_t smt = dscore_tc_smem();
+    const bool sp = a.cv.rows != 0;
+#define FL_DST(KMv)                                                                                    \
+  case KMv:                                                                                            \
+    return sp ? launch_k(g_pdl, k_dscore_tc<KMv, true>, g1, dim3(256), smt, s, b)                      \
+              : launch_k(g_pdl, k_dscore_tc<KMv, false>, g1, dim3(256), smt, s, b);
     switch (chain_km(a.cv.K)) {
-      case 2: return launch_k(g_pdl, k_dscore_tc<128, 2>, g4, dim3(128), smt, s, b);
-      case 4: return launch_k(g_pdl, k_dscore_tc<128, 4>, g4, dim3(128), smt, s, b);
-      case 8: return launch_k(g_pdl, k_dscore_tc<128, 8>, g4, dim3(128), smt, s, b);
-      case 16: return launch_k(g_pdl, k_dscore_tc<128, 16>, g4, dim3(128), smt, s, b);
+      FL_DST(2)
+      FL_DST(4)
+      FL_DST(8)
+      FL_DST(16)
       default: return cudaErrorInvalidValue;
     }
+#undef FL_DST
   }
-#define FL_DS(KMv)                                                                           \
-  case KMv:                                                                                  \
-    return a.hd == 128 ? launch_k(g_pdl, k_dscore<128, 4, KMv>, grid, dim3(256), sm, s, b)  \
-                       : launch_k(g_pdl, k_dscore<64, 2, KMv>, grid, dim3(256), sm, s, b);
+  // items of (tile, KV head, block of columns): 256-column blocks, halved (to 64)
+  // while the items would not fill two CTAs per SM; two CTAs per SM
+  int blk = kDsBlock;
+  while (blk > 64 && max_need * a.Hkv * ((max_chunks * 64 + blk - 1) / blk) < 2 * kDscoreSMs) blk /= 2;
+  b.ds_block = blk;
+  const int items = max_need * a.Hkv * ((max_chunks * 64 + blk - 1) / blk);
+  const dim3 grid(items < 2 * kDscoreSMs ? items : 2 * kDscoreSMs);
+  const size_t sm = dscore_smem(a.hd);
+  const bool sp = a.cv.rows != 0;
+#define FL_DS(KMv)                                                                                     \
+  case KMv:                                                                                            \
+    if (sp)                                                                                            \
+      return a.hd == 128 ? launch_k(g_pdl, k_dscore<128, KMv, true>, grid, dim3(256), sm, s, b)        \
+                         : launch_k(g_pdl, k_dscore<64, KMv, true>, grid, dim3(256), sm, s, b);        \
+    return a.hd == 128 ? launch_k(g_pdl, k_dscore<128, KMv, false>, grid, dim3(256), sm, s, b)         \
+                       : launch_k(g_pdl, k_dscore<64, KMv, false>, grid, dim3(256), sm, s, b);
   switch (chain_km(a.cv.K)) {
     FL_DS(2)
     FL_DS(4)
@@ -2676,7 +3451,7 @@ cudaError_t launch_select_cols(const SelColsArgs& a, int max_need, int max_cols_
   return launch_k(g_pdl, k_select_cols, dim3(max_need * a.Hkv, slices), dim3(1024),
                   select_cols_smem(kSelColsSmemKeys), s, a);
 }
-size_t corr_cluster_smem(int hd, int grp) { return static_cast<size_t>(kCorrWarps) * grp * hd * 4; }
+size_t corr_cluster_smem(int hd, int grp) { return static_cast<size_t>(2) * kCorrWarps * grp * hd * 4; }
 template <typename K, typename A>
 cudaError_t launch_cluster(K kern, dim3 grid, dim3 block, int cluster_x, size_t smem, cudaStream_t s, const A& a) {
   cudaLaunchConfig_t cfg = {};
@@ -2696,15 +3471,40 @@ cudaError_t launch_cluster(K kern, dim3 grid, dim3 block, int cluster_x, size_t 
   return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
-template <int HD, int EPL, int GRP, int KM>
-cudaError_t launch_correct_t(const CorrectArgs& a, int n_sel, cudaStream_t s) {
+template <int HD, int EPL, int GRP, int KM, bool SP>
+cudaError_t launch_correct_sp(const CorrectArgs& a, int n_sel, cudaStream_t s) {
   if (a.cluster) {
     dim3 grid(kCorrCluster, n_sel * a.Hkv);
-    return launch_cluster(k_correct_cluster<HD, EPL, GRP, KM>, grid, dim3(32 * kCorrWarps), kCorrCluster,
+    return launch_cluster(k_correct_cluster<HD, EPL, GRP, KM, SP>, grid, dim3(32 * kCorrWarps), kCorrCluster,
                           corr_cluster_smem(HD, GRP), s, a);
   }
   dim3 grid(n_sel * a.Hkv, a.n_splits);
-  return launch_k(g_pdl, k_correct<HD, EPL, GRP, KM>, grid, dim3(256), 0, s, a);
+  return launch_k(g_pdl, k_correct<HD, EPL, GRP, KM, SP>, grid, dim3(256), 0, s, a);
+}
+template <int HD, int EPL, int GRP, int KM>
+cudaError_t launch_correct_t(const CorrectArgs& a, int n_sel, cudaStream_t s) {
+  return a.cv.rows ? launch_correct_sp<HD, EPL, GRP, KM, true>(a, n_sel, s)
+                   : launch_correct_sp<HD, EPL, GRP, KM, false>(a, n_sel, s);
+}
+size_t correct_tc_smem() { return 1024 + static_cast<size_t>(10) * 64 * 128 * 2; }
+// prefill tiles on the tensor cores: grid-stride over (plan entry, KV head, pass of 64 pairs)
+cudaError_t launch_correct_tc(const CorrectArgs& a, int max_entries, cudaStream_t s) {
+  const int npass = (a.q_tile * (a.H / a.Hkv) + 63) / 64;
+  const int items = max_entries * a.Hkv * npass;
+  const dim3 grid(items < kDscoreSMs ? items : kDscoreSMs);
+  const size_t sm = correct_tc_smem();
+  const bool sp = a.cv.rows != 0;
+  switch (chain_km(a.cv.K)) {
+    case 2: return sp ? launch_k(g_pdl, k_correct_tc<2, true>, grid, dim3(256), sm, s, a)
+                      : launch_k(g_pdl, k_correct_tc<2, false>, grid, dim3(256), sm, s, a);
+    case 4: return sp ? launch_k(g_pdl, k_correct_tc<4, true>, grid, dim3(256), sm, s, a)
+                      : launch_k(g_pdl, k_correct_tc<4, false>, grid, dim3(256), sm, s, a);
+    case 8: return sp ? launch_k(g_pdl, k_correct_tc<8, true>, grid, dim3(256), sm, s, a)
+                      : launch_k(g_pdl, k_correct_tc<8, false>, grid, dim3(256), sm, s, a);
+    case 16: return sp ? launch_k(g_pdl, k_correct_tc<16, true>, grid, dim3(256), sm, s, a)
+                       : launch_k(g_pdl, k_correct_tc<16, false>, grid, dim3(256), sm, s, a);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 template <int HD, int EPL, int GRP>
@@ -2720,6 +3520,7 @@ cudaError_t launch_correct_km(const CorrectArgs& a, int n_sel, cudaStream_t s) {
 
 cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
   const int grp = a.H / a.Hkv;
+  if (a.tc && a.hd == 128 && !a.cluster) return launch_correct_tc(a, a.max_entries, s);
 #define FL_CORR(G)                                                                   \
   case G:                                                                            \
     return a.hd == 128 ? launch_correct_km<128, 4, G>(a, n_sel, s) : launch_correct_km<64, 2, G>(a, n_sel, s);
@@ -2734,22 +3535,48 @@ cudaError_t launch_correct(const CorrectArgs& a, int n_sel, cudaStream_t s) {
 }
 
 // 16-CTA clusters are beyond the portable size: opt every instantiation in.
-template <int HD, int EPL, int GRP, int KM>
+template <int HD, int EPL, int GRP, int KM, bool SP>
 cudaError_t allow_big_cluster() {
   cudaError_t e =
-      cudaFuncSetAttribute(k_correct_cluster<HD, EPL, GRP, KM>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      cudaFuncSetAttribute(k_correct_cluster<HD, EPL, GRP, KM, SP>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_correct_cluster<HD, EPL, GRP, KM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_correct_cluster<HD, EPL, GRP, KM, SP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(corr_cluster_smem(HD, GRP)));
+  return e;
+}
+template <int HD, int EPL, int GRP, bool SP>
+cudaError_t allow_big_cluster_sp() {
+  cudaError_t e = allow_big_cluster<HD, EPL, GRP, 2, SP>();
+  if (e == cudaSuccess) e = allow_big_cluster<HD, EPL, GRP, 4, SP>();
+  if (e == cudaSuccess) e = allow_big_cluster<HD, EPL, GRP, 8, SP>();
+  if (e == cudaSuccess) e = allow_big_cluster<HD, EPL, GRP, 16, SP>();
   return e;
 }
 template <int HD, int EPL, int GRP>
 cudaError_t allow_big_cluster_km() {
-  cudaError_t e = allow_big_cluster<HD, EPL, GRP, 2>();
-  if (e == cudaSuccess) e = allow_big_cluster<HD, EPL, GRP, 4>();
-  if (e == cudaSuccess) e = allow_big_cluster<HD, EPL, GRP, 8>();
-  if (e == cudaSuccess) e = allow_big_cluster<HD, EPL, GRP, 16>();
+  cudaError_t e = allow_big_cluster_sp<HD, EPL, GRP, false>();
+  if (e == cudaSuccess) e = allow_big_cluster_sp<HD, EPL, GRP, true>();
   return e;
+}
+
+template <bool SP, typename Set>
+void set_dscore(Set& set) {
+  set(k_correct_tc<2, SP>, static_cast<int>(correct_tc_smem()));
+  set(k_correct_tc<4, SP>, static_cast<int>(correct_tc_smem()));
+  set(k_correct_tc<8, SP>, static_cast<int>(correct_tc_smem()));
+  set(k_correct_tc<16, SP>, static_cast<int>(correct_tc_smem()));
+  set(k_dscore_tc<2, SP>, static_cast<int>(dscore_tc_smem()));
+  set(k_dscore_tc<4, SP>, static_cast<int>(dscore_tc_smem()));
+  set(k_dscore_tc<8, SP>, static_cast<int>(dscore_tc_smem()));
+  set(k_dscore_tc<16, SP>, static_cast<int>(dscore_tc_smem()));
+  set(k_dscore<128, 2, SP>, static_cast<int>(dscore_smem(128)));
+  set(k_dscore<128, 4, SP>, static_cast<int>(dscore_smem(128)));
+  set(k_dscore<128, 8, SP>, static_cast<int>(dscore_smem(128)));
+  set(k_dscore<128, 16, SP>, static_cast<int>(dscore_smem(128)));
+  set(k_dscore<64, 2, SP>, static_cast<int>(dscore_smem(64)));
+  set(k_dscore<64, 4, SP>, static_cast<int>(dscore_smem(64)));
+  set(k_dscore<64, 8, SP>, static_cast<int>(dscore_smem(64)));
+  set(k_dscore<64, 16, SP>, static_cast<int>(dscore_smem(64)));
 }
 
 // Opt every large-shared-memory kernel in to its dynamic shared memory once,
@@ -2779,18 +3606,8 @@ cudaError_t kernels_init_attrs() {
   set(k_attn_prefill<64>, static_cast<int>(attn_prefill_smem(64)));
   set(k_attn_prefill_tc<128>, static_cast<int>(attn_prefill_tc_smem(128)));
   set(k_attn_prefill_tc<64>, static_cast<int>(attn_prefill_tc_smem(64)));
-  set(k_dscore_tc<128, 2>, static_cast<int>(dscore_tc_smem()));
-  set(k_dscore_tc<128, 4>, static_cast<int>(dscore_tc_smem()));
-  set(k_dscore_tc<128, 8>, static_cast<int>(dscore_tc_smem()));
-  set(k_dscore_tc<128, 16>, static_cast<int>(dscore_tc_smem()));
-  set(k_dscore<128, 4, 2>, static_cast<int>(dscore_smem(128)));
-  set(k_dscore<128, 4, 4>, static_cast<int>(dscore_smem(128)));
-  set(k_dscore<128, 4, 8>, static_cast<int>(dscore_smem(128)));
-  set(k_dscore<128, 4, 16>, static_cast<int>(dscore_smem(128)));
-  set(k_dscore<64, 2, 2>, static_cast<int>(dscore_smem(64)));
-  set(k_dscore<64, 2, 4>, static_cast<int>(dscore_smem(64)));
-  set(k_dscore<64, 2, 8>, static_cast<int>(dscore_smem(64)));
-  set(k_dscore<64, 2, 16>, static_cast<int>(dscore_smem(64)));
+  set_dscore<false>(set);
+  set_dscore<true>(set);
   {
     const cudaError_t r[8] = {allow_big_cluster_km<128, 4, 1>(), allow_big_cluster_km<128, 4, 2>(),
                               allow_big_cluster_km<128, 4, 4>(), allow_big_cluster_km<128, 4, 8>(),

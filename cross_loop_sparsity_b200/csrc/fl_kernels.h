@@ -150,6 +150,7 @@ struct DScoreArgs {
   float* col_keys;      // [max_need][Hkv][max_cols]
   int max_cols;
   int max_chunks;       // 64-column chunks of the longest row (set by the launcher)
+  int ds_block;         // columns per work item of the SIMT kernel (set by the launcher)
   int tc;               // 1: the tensor-core kernel (prefill tiles, head_dim 128)
   // 1: the CTA finishing a row's last chunk also selects its column set (rows of
   // at most kSelColsSmemKeys columns), with `sel`; row_tickets [max_need][Hkv]
@@ -171,9 +172,10 @@ struct CorrectArgs {
   const int* tile;
   const int* last;
   const float* q_cur;
-  float* q_last;
-  float* o_state;
-  float* lse_state;
+  const float* q_last;   // the loop-1 queries (token order)
+  float* o_state;               // loop-1 O, then (after the token's first recomputation) the rest's numerator
+  float* lse_state;             // loop-1 lse, then the rest's maximum
+  float* z_state;               // the rest's denominator
   uint16_t* o_bf16;
   const int32_t* cols;
   const int* ncols;
@@ -184,8 +186,11 @@ struct CorrectArgs {
   int cols_per_cta, n_splits;   // column split: grid.y = n_splits = ceil(c / cols_per_cta)
   int cluster;                  // decode (each query its own tile, few queries): one cluster per
                                 // (query, group), merged over distributed shared memory
-  float* part_acc;              // [n_sel][Hkv][n_splits][8][hd]
-  float* part_mz;               // [n_sel][Hkv][n_splits][8][2]
+  int tc;                       // prefill tiles, head_dim 128: the tensor-core kernel, per (tile, group)
+  TilePlan plan;                // (tc) the loop's query tiles and their selected slots
+  int q_tile, max_entries;      // (tc) query tile size; bound on the plan's entries
+  float* part_acc;              // [n_sel][Hkv][n_splits][2][8][hd]: new-term, old-term numerators
+  float* part_mz;               // [n_sel][Hkv][n_splits][8][3]: max, new-term, old-term denominators
   int* counters;                // [n_sel][Hkv], zero between launches
   int* status;
 };

@@ -44,7 +44,7 @@ struct flashloop_ctx {
   float *h = nullptr, *h_in = nullptr, *h_snap = nullptr;
   uint16_t *x = nullptr, *obf = nullptr, *act = nullptr;
   float *qkv = nullptr, *q_cur = nullptr;
-  float *o_state = nullptr, *lse_state = nullptr, *q_last = nullptr;
+  float *o_state = nullptr, *lse_state = nullptr, *z_state = nullptr, *q_last = nullptr;
   int *seq = nullptr, *pos = nullptr, *tile = nullptr, *last = nullptr, *sel_slot = nullptr;
   float *key = nullptr, *keys_trace = nullptr;
   int32_t *idx_all = nullptr, *idx_sel = nullptr, *idx_last = nullptr;
@@ -216,10 +216,11 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   uint8_t* act = take(static_cast<size_t>(Npad) * c.ffn_dim * 2);
   uint8_t* qkv = take(static_cast<size_t>(Npad) * qkv_rows * 4);
   uint8_t* q_cur = take(static_cast<size_t>(N) * H * hd * 4);
-  uint8_t *o_state = nullptr, *lse = nullptr, *q_last = nullptr;
+  uint8_t *o_state = nullptr, *lse = nullptr, *z_state = nullptr, *q_last = nullptr;
   if (lazy) {
     o_state = take(static_cast<size_t>(M) * N * H * hd * 4);
     lse = take(static_cast<size_t>(M) * N * H * 4);
+    z_state = take(static_cast<size_t>(M) * N * H * 4);
     q_last = take(static_cast<size_t>(M) * N * H * hd * 4);
   }
   uint8_t* seq = take(N * 4);
@@ -272,8 +273,8 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     const size_t big_rows = static_cast<size_t>(nsel_max) * Hkv * ns_big;
     cp_rows = std::max(small_rows, big_rows);
   }
-  uint8_t* corr_acc = take(std::max<size_t>(cp_rows, 1) * 8 * hd * 4);
-  uint8_t* corr_mz = take(std::max<size_t>(cp_rows, 1) * 8 * 2 * 4);
+  uint8_t* corr_acc = take(std::max<size_t>(cp_rows, 1) * 2 * 8 * hd * 4);
+  uint8_t* corr_mz = take(std::max<size_t>(cp_rows, 1) * 8 * 3 * 4);
   uint8_t* corr_counters = take(static_cast<size_t>(std::max(nsel_max, 1)) * Hkv * 4);
   // GEMM split-K partials (skinny orientation only)
   size_t gp = 0;
@@ -347,6 +348,7 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->q_cur = reinterpret_cast<float*>(q_cur);
     x->o_state = reinterpret_cast<float*>(o_state);
     x->lse_state = reinterpret_cast<float*>(lse);
+    x->z_state = reinterpret_cast<float*>(z_state);
     x->q_last = reinterpret_cast<float*>(q_last);
     x->seq = reinterpret_cast<int*>(seq);
     x->pos = reinterpret_cast<int*>(pos);
@@ -612,7 +614,7 @@ struct LayerRef {
   int loop;                  // loop number of the KV write (1 for independent layers)
   bool lazy;                 // the lazy layout: base + residuals (the shared block on the lazy path)
   bool full;                 // dense attention (otherwise the correction over column sets)
-  float *o_st, *l_st, *ql;   // per-query attention state (lazy path), or nullptr
+  float *o_st, *l_st, *z_st, *ql;   // per-query attention state (lazy path), or nullptr
 };
 
 fl_status run_layer(flashloop_ctx* ctx, const LayerRef& L, const CallShape& cs, const int32_t* idx, int n, XIn& xs,
@@ -661,7 +663,8 @@ fl_status run_layer(flashloop_ctx* ctx, const LayerRef& L, const CallShape& cs, 
   } else {
     CorrectArgs ca{};
     ca.idx = idx; ca.seq = ctx->seq; ca.pos = ctx->pos; ca.tile = ctx->tile; ca.last = ctx->last;
-    ca.q_cur = ctx->q_cur; ca.q_last = L.ql; ca.o_state = L.o_st; ca.lse_state = L.l_st; ca.o_bf16 = ctx->obf;
+    ca.q_cur = ctx->q_cur; ca.q_last = L.ql; ca.o_state = L.o_st; ca.lse_state = L.l_st; ca.z_state = L.z_st;
+    ca.o_bf16 = ctx->obf;
     ca.cols = ctx->cols; ca.ncols = ctx->ncols; ca.meta = ctx->sel_meta; ca.cv = *L.cv; ca.j = L.cj; ca.loop = L.loop;
     ca.H = H; ca.Hkv = Hkv;
     ca.hd = hd; ca.c = c.c_cols; ca.n_tiles = ctx->n_tiles_max; ca.tau = cs.tau; ca.status = ctx->status;
@@ -669,6 +672,8 @@ fl_status run_layer(flashloop_ctx* ctx, const LayerRef& L, const CallShape& cs, 
     ca.n_splits = ceil_div(c.c_cols, ca.cols_per_cta);
     ca.part_acc = ctx->corr_acc; ca.part_mz = ctx->corr_mz; ca.counters = ctx->corr_counters;
     ca.cluster = (cs.decode && cs.n_sel <= kCorrSmallQueries && ctx->corr_cluster) ? 1 : 0;
+    ca.tc = (!cs.decode && ctx->tc_prefill) ? 1 : 0;   // many queries per tile: tensor-core products
+    ca.plan = ctx->plan; ca.q_tile = c.q_tile; ca.max_entries = cs.max_need;   // plan entries <= min(n_sel, tiles)
     SelColsArgs sa{};
     sa.plan = ctx->plan; sa.idx = idx; sa.pos = ctx->pos; sa.meta = ctx->sel_meta; sa.col_keys = ctx->col_keys;
     sa.max_cols = c.max_ctx; sa.Hkv = Hkv; sa.c = c.c_cols; sa.j = L.cj; sa.n_tiles = ctx->n_tiles_max;
@@ -715,7 +720,7 @@ fl_status run_independent(flashloop_ctx* ctx, int stack, const CallShape& cs, XI
   const int count = stack == 1 ? c.n_prelude : c.n_coda;
   for (int z = 0; z < count; ++z) {
     LayerRef L{stack_w(ctx, stack), z, &ctx->cvx, &ctx->tm_kvx, stack == 1 ? z : c.n_prelude + z, 1, false, true,
-               nullptr, nullptr, nullptr};
+               nullptr, nullptr, nullptr, nullptr};
     FL_STEP(run_layer(ctx, L, cs, ctx->idx_all, cs.N, xs, s));
   }
   return FL_OK;
@@ -806,7 +811,7 @@ fl_status run_call_body(flashloop_ctx* ctx, int decode, int B, int T, cudaStream
     for (int j = 0; j < M; ++j) {
       LayerRef L{stack_w(ctx, 0), j, &ctx->cv, &ctx->tm_kv, j, l, lazy, full,
                  lazy ? ctx->o_state + j * st_o : nullptr, lazy ? ctx->lse_state + j * st_l : nullptr,
-                 lazy ? ctx->q_last + j * st_o : nullptr};
+                 lazy ? ctx->z_state + j * st_l : nullptr, lazy ? ctx->q_last + j * st_o : nullptr};
       FL_STEP(run_layer(ctx, L, cs, idx, n, xs, s));
     }
     carry = xs;

@@ -252,8 +252,8 @@ fl_status flashloop_force_codes(flashloop_ctx* ctx, const int8_t* codes, const u
  * NULL turns each off).  kv_rows: fp32 [M][K-1][n_slots][2][Hkv][hd], the
  * rotated new K (0) and V (1) rows that a lazy loop l >= 2 quantised, by (layer,
  * loop, selection slot, K/V, KV head) -- the inputs of the KV-residual quantiser
- * ("FlashLoop ...", abstract: KV residuals between adjacent loops in low-bit
- * form); rows are written only where the library quantised them itself (not
+ * ("FlashLoop ...", abstract: each loop's KV as a low-bit residual over the
+ * previous loop's); rows are written only where the library quantised them itself (not
  * under flashloop_force_codes) and only for slots < n_slots.  col_keys: fp32
  * [M][n_tiles][Hkv][max_ctx], the delta-score key of every eligible column of
  * each query tile whose column set the call chose ("FlashLoop ...", abstract:

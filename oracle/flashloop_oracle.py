@@ -9,8 +9,8 @@ Plain, slow and meant to be read against the pages:
 
 * "FlashLoop: Fast and Memory-Efficient Looped Transformers via Lazy Updates"
   (abstract) -- the method: token-sparse updates, sparse attention over a
-  stable subset of key columns, and KV residuals between adjacent loops stored
-  in low-bit form.  It gives no equations; the concrete rules below (ranking by
+  fixed small set of key columns, and each loop's KV kept as a low-bit
+  residual over the previous loop's.  It gives no equations; the concrete rules below (ranking by
   the squared change norm, top-c columns by |delta score|, per-group absmax
   int4/int2 codes) are the plainest reading of it, and every open point is
   listed with the reading taken in the design notes.
@@ -68,8 +68,8 @@ def select_top(keys: np.ndarray, k: int) -> np.ndarray:
     Order: the key's IEEE-754 bit pattern read as an unsigned integer,
     descending (so NaN sorts above +inf), ties to the lower index.  Used for
     the top-rho tokens and for the top-c key columns ("FlashLoop ...",
-    abstract: state changes concentrate on few tokens; attention-output
-    differences are dominated by a sparse subset of key columns).
+    abstract: few tokens carry most of a loop's state change, and few key
+    columns carry most of the change in attention output).
     """
     keys = np.ascontiguousarray(keys, dtype=F32)
     n = keys.shape[0]
@@ -360,7 +360,8 @@ class KVCache:
 
         base, then + residual of loops 2..m in that order; each add rounded to
         fp32 (fp64 in the exact mode).  KV_l = KV_{l-1} + deq(q(r_l))
-        ("FlashLoop ...", abstract: KV residuals between adjacent loops).
+        ("FlashLoop ...", abstract: each loop's KV as a residual over the
+        previous loop's).
         """
         base = getattr(self, "base_" + which)[j, b][:, rows]
         res = getattr(self, "res_" + which)

@@ -8,8 +8,8 @@ eligible column -- and the tests recompute every decision on the CPU from those
 inputs and the library's exported cache:
 
 * KV-residual quantisation ("FlashLoop: Fast and Memory-Efficient Looped
-  Transformers via Lazy Updates", abstract: KV residuals between adjacent loops
-  in low-bit form): the previous level is rebuilt from the exported base and
+  Transformers via Lazy Updates", abstract: each loop's KV kept as a low-bit
+  residual over the previous loop's): the previous level is rebuilt from the exported base and
   residual codes / scales of loops 2..l-1 (fp32 adds in loop order), r =
   fp32(x - prev), and the oracle's quantiser and packer must give the exported
   codes and scales bit for bit.  Tokens not recomputed at loop l must hold a
