@@ -1938,41 +1938,60 @@ __global__ void __launch_bounds__(256, 2) k_dscore(const DScoreArgs a) {
 // delta-score column keys of prefill tiles on the tensor cores.  The same keys
 // as k_dscore -- key[k] = max over the tile's selected queries (k <= their
 // position) and the group's heads of |tau (q_l . K_l[k] - q_last . K_base[k])|
-// -- with the products as warp-level bf16 MMAs with fp32 accumulation.  At a
-// tile's first recomputation every member was last computed at loop 1, so the
-// old keys are the bf16 base exactly; the new keys (base + residuals, fp32) are
-// split into bf16 hi + lo, the queries too, and the difference accumulates in
-// one register set:  Qh Kh + Ql Kh + Qh Kl - Qoh Kb - Qol Kb  (the Ql Kl term,
-// below 2^-16 relative, is dropped).
+// -- evaluated through the identity
+//   q_l . K_l - q_last . K_base = (q_l - q_last) . K_base + q_l . R,
+// R = K_l - K_base = the sum of code * scale of loops 2..l (fp32, loop order):
+// the difference of the queries is formed in fp32 before it is rounded, so two
+// single bf16 products with fp32 accumulation (K_base is bf16 exactly; R is
+// small) keep the key accurate where the direct form would cancel two large
+// terms.  (At a tile's first recomputation every member was last computed at
+// loop 1, so the old keys are the base rows.)
 //
 // Work items are (tile, KV head, unit of kDsTcUnit 64-column chunks), taken
-// grid-stride, one CTA per SM.  Per item and per pass of 64 (query, head)
-// pairs, the pairs are staged once in shared memory as the four bf16 operand
-// tiles (tau q_l hi / lo, -tau q_last hi / lo); the unit's chunks then stream
-// through: the base rows of chunk c + 1 are copied (cp.async, 128-byte swizzle)
-// while chunk c's new keys are built (base + the residual codes of loops
-// 2..l, loaded before the copy is awaited) and multiplied.  Warp w takes pair
-// rows 16 (w % 4) .. +15 against columns 32 (w / 4) .. +31 of the chunk; the
-// column maxima meet in shared memory (max of non-negative floats = max of
-// their bit patterns, in any order).
+// grid-stride, two CTAs per SM.  Per item and per pass of 64 (query, head)
+// pairs, the pairs are staged once in shared memory as two bf16 operand tiles
+// (tau (q_l - q_last), tau q_l); the unit's chunks then stream through: the
+// base rows of chunk c + 1 are copied (cp.async, 128-byte swizzle) while chunk
+// c's residual tile is built (codes loaded before the copy is awaited) and
+// multiplied.  Warp w takes pair rows 16 (w % 4) .. +15 against columns
+// 32 (w / 4) .. +31 of the chunk; the column maxima meet in shared memory (max
+// of non-negative floats = max of their bit patterns, in any order).
 // ============================================================================
 constexpr int kDsTcUnit = 4;   // 64-column chunks per work item
+
+// Dynamic work distribution: CTAs take items from a counter, so CTAs that drew
+// cheap or empty items take more; the last CTA to finish resets the counter
+// for the next launch.  (Items are numbered heaviest first by the callers.)
+__device__ __forceinline__ int next_item(int* work, int* s_item) {
+  __syncthreads();   // every thread has read the previous item
+  if (threadIdx.x == 0) *s_item = atomicAdd(&work[0], 1);
+  __syncthreads();
+  return *s_item;
+}
+__device__ __forceinline__ void finish_items(int* work) {
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&work[1], 1) == static_cast<int>(gridDim.x) - 1) {
+      work[0] = 0;
+      work[1] = 0;
+    }
+  }
+}
 
 __device__ __forceinline__ uint32_t swz128(int row, int piece) {   // 16-byte piece of a 64 x 128-dim bf16 tile
   return static_cast<uint32_t>((piece >> 3) * (64 * 128) + row * 128 + (((piece & 7) ^ (row & 7)) << 4));
 }
 
 template <int KM, bool SP>
-__global__ void __launch_bounds__(256, 1) k_dscore_tc(const DScoreArgs a) {
+__global__ void __launch_bounds__(256, 2) k_dscore_tc(const DScoreArgs a) {
   constexpr int HD = 128, TILE = 2 * 64 * 128, KS = HD / 16, UC = kDsTcUnit;
   pdl_trigger();
   pdl_wait();
   extern __shared__ uint8_t sm_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qt = sm;                    // [4][TILE]: tau q_l hi, lo; -tau q_last hi, lo (64 pair rows)
-  uint8_t* kbs = sm + 4 * TILE;        // [2][TILE]: base rows of the chunk (double-buffered)
-  uint8_t* knh = sm + 6 * TILE;        // new keys, hi
-  uint8_t* knl = sm + 7 * TILE;        // new keys, lo
+  uint8_t* qt = sm;                    // [2][TILE]: tau (q_l - q_last), tau q_l (64 pair rows)
+  uint8_t* kbs = sm + 2 * TILE;        // [2][TILE]: base rows of the chunk (double-buffered)
+  uint8_t* krs = sm + 4 * TILE;        // the chunk's residual sums R
   __shared__ unsigned colmax[UC * 64];
   __shared__ int qpos[64];
   __shared__ int fold_last;
@@ -1985,9 +2004,13 @@ __global__ void __launch_bounds__(256, 1) k_dscore_tc(const DScoreArgs a) {
   const int bits = cv.bits;
   const size_t rb = cv.row_bytes_codes(), ns = cv.hd >> cv.lg;
   const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * (SP ? cv.rows : cv.T);
-  const uint32_t qt_s = smem_u32(qt), kbs_s = smem_u32(kbs), knh_s = smem_u32(knh), knl_s = smem_u32(knl);
-  for (int it = blockIdx.x; it < cnt * a.Hkv * nunit; it += gridDim.x) {
-    const int seg = it / (a.Hkv * nunit), g = (it / nunit) % a.Hkv, unit = it % nunit;
+  const uint32_t qt_s = smem_u32(qt), kbs_s = smem_u32(kbs), krs_s = smem_u32(krs);
+  __shared__ int s_item;
+  for (;;) {
+    const int it = next_item(a.work, &s_item);
+    if (it >= cnt * a.Hkv * nunit) break;
+    // the longest rows (the last plan entries: the latest tiles) first
+    const int seg = cnt - 1 - it / (a.Hkv * nunit), g = (it / nunit) % a.Hkv, unit = it % nunit;
     const int p = a.plan.need[seg];
     const int qb = a.plan.qb[p], qe = a.plan.qe[p];
     const SelMeta ml = a.meta[qe - 1];
@@ -2013,7 +2036,7 @@ __global__ void __launch_bounds__(256, 1) k_dscore_tc(const DScoreArgs a) {
     for (int pb = 0; pb < npairs; pb += 64) {
       __syncthreads();   // the previous pass (or item, or fold) no longer reads shared memory
       // ---- the pass's pairs as operand tiles: thread -> (pair row, 8-dim piece) x 4
-#pragma unroll
+#pragma unroll 1
       for (int u = 0; u < 4; ++u) {
         const int e = tid + 256 * u, r = e >> 4, pc = e & 15;
         const int pr = pb + r;
@@ -2032,24 +2055,15 @@ __global__ void __launch_bounds__(256, 1) k_dscore_tc(const DScoreArgs a) {
           for (int k = 0; k < 8; ++k) xn[k] = xo[k] = 0.f;
           if (pc == 0) qpos[r] = -1;
         }
-        uint32_t wh[4], wl[4], woh[4], wol[4];
+        uint32_t wd[4], wn[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          float h0, l0, h1, l1;
-          split_bf16(a.tau * xn[2 * k], h0, l0);
-          split_bf16(a.tau * xn[2 * k + 1], h1, l1);
-          wh[k] = pack_bf16x2(h0, h1);
-          wl[k] = pack_bf16x2(l0, l1);
-          split_bf16(-a.tau * xo[2 * k], h0, l0);
-          split_bf16(-a.tau * xo[2 * k + 1], h1, l1);
-          woh[k] = pack_bf16x2(h0, h1);
-          wol[k] = pack_bf16x2(l0, l1);
+          wd[k] = pack_bf16x2(a.tau * (xn[2 * k] - xo[2 * k]), a.tau * (xn[2 * k + 1] - xo[2 * k + 1]));
+          wn[k] = pack_bf16x2(a.tau * xn[2 * k], a.tau * xn[2 * k + 1]);
         }
         const uint32_t o = swz128(r, pc);
-        *reinterpret_cast<uint4*>(qt + o) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-        *reinterpret_cast<uint4*>(qt + TILE + o) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
-        *reinterpret_cast<uint4*>(qt + 2 * TILE + o) = make_uint4(woh[0], woh[1], woh[2], woh[3]);
-        *reinterpret_cast<uint4*>(qt + 3 * TILE + o) = make_uint4(wol[0], wol[1], wol[2], wol[3]);
+        *reinterpret_cast<uint4*>(qt + o) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        *reinterpret_cast<uint4*>(qt + TILE + o) = make_uint4(wn[0], wn[1], wn[2], wn[3]);
       }
       if (pb == 0) colmax[tid] = 0u;   // UC * 64 == 256 == blockDim.x
       issue_base(0);
@@ -2083,20 +2097,13 @@ __global__ void __launch_bounds__(256, 1) k_dscore_tc(const DScoreArgs a) {
         cp_async_wait<0>();
         __syncthreads();   // chunk c's base rows are in; every warp is done with chunk c - 1
         if (c + 1 < nch) issue_base(c + 1);   // into the buffer chunk c - 1 used
-        // ---- new keys: base + code * scale of loops 2..l in loop order (fp32), split hi / lo
-        const uint8_t* kb_c = kbs + (c & 1) * TILE;
+        // ---- R = code * scale of loops 2..l summed in loop order (fp32), as bf16
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int e = tid + 256 * u, r = e >> 4, pc = e & 15;
-          const uint32_t o = swz128(r, pc);
-          const uint4 bw = *reinterpret_cast<const uint4*>(kb_c + o);
-          const uint32_t w[4] = {bw.x, bw.y, bw.z, bw.w};
           float x[8];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            x[2 * k] = bf16_to_f(w[k] & 0xFFFF);
-            x[2 * k + 1] = bf16_to_f(w[k] >> 16);
-          }
+          for (int k = 0; k < 8; ++k) x[k] = 0.f;
 #pragma unroll
           for (int q = 0; q < KM - 1; ++q) {
             if (q + 2 > a.loop) break;
@@ -2108,17 +2115,10 @@ __global__ void __launch_bounds__(256, 1) k_dscore_tc(const DScoreArgs a) {
               x[k] = __fadd_rn(x[k], __fmul_rn(static_cast<float>(cd), sc));
             }
           }
-          uint32_t hw[4], lw[4];
+          uint32_t w[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            float h0, l0, h1, l1;
-            split_bf16(x[2 * k], h0, l0);
-            split_bf16(x[2 * k + 1], h1, l1);
-            hw[k] = pack_bf16x2(h0, h1);
-            lw[k] = pack_bf16x2(l0, l1);
-          }
-          *reinterpret_cast<uint4*>(knh + o) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-          *reinterpret_cast<uint4*>(knl + o) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          for (int k = 0; k < 4; ++k) w[k] = pack_bf16x2(x[2 * k], x[2 * k + 1]);
+          *reinterpret_cast<uint4*>(krs + swz128(r, pc)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
         __syncthreads();
         if (rows_active) {
@@ -2127,28 +2127,22 @@ __global__ void __launch_bounds__(256, 1) k_dscore_tc(const DScoreArgs a) {
           for (int nt = 0; nt < 4; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
-            uint32_t an[4], al[4], aoh[4], aol[4];
+            uint32_t ad[4], an[4];
             const uint32_t qo_ = swz128(16 * rg + (lane & 15), 2 * ks + (lane >> 4));
-            ldsm_x4(qt_s + qo_, an);
-            ldsm_x4(qt_s + TILE + qo_, al);
-            ldsm_x4(qt_s + 2 * TILE + qo_, aoh);
-            ldsm_x4(qt_s + 3 * TILE + qo_, aol);
+            ldsm_x4(qt_s + qo_, ad);
+            ldsm_x4(qt_s + TILE + qo_, an);
 #pragma unroll
             for (int np = 0; np < 2; ++np) {
               const int key = 32 * ch2 + np * 16 + (lane & 7) + ((lane >> 4) << 3);
               const uint32_t ko = swz128(key, 2 * ks + ((lane >> 3) & 1));
-              uint32_t fh[4], fl[4], fb[4];
-              ldsm_x4(knh_s + ko, fh);
-              ldsm_x4(knl_s + ko, fl);
+              uint32_t fb[4], fr[4];
               ldsm_x4(kbs_s + (c & 1) * TILE + ko, fb);
+              ldsm_x4(krs_s + ko, fr);
 #pragma unroll
               for (int hlf = 0; hlf < 2; ++hlf) {
                 float* d = acc[2 * np + hlf];
-                mma_bf16_16816(d, an, fh[2 * hlf], fh[2 * hlf + 1]);
-                mma_bf16_16816(d, al, fh[2 * hlf], fh[2 * hlf + 1]);
-                mma_bf16_16816(d, an, fl[2 * hlf], fl[2 * hlf + 1]);
-                mma_bf16_16816(d, aoh, fb[2 * hlf], fb[2 * hlf + 1]);
-                mma_bf16_16816(d, aol, fb[2 * hlf], fb[2 * hlf + 1]);
+                mma_bf16_16816(d, ad, fb[2 * hlf], fb[2 * hlf + 1]);
+                mma_bf16_16816(d, an, fr[2 * hlf], fr[2 * hlf + 1]);
               }
             }
           }
@@ -2184,6 +2178,7 @@ __global__ void __launch_bounds__(256, 1) k_dscore_tc(const DScoreArgs a) {
     }
     if (a.fold) fold_select(a, seg, g, a.plan.tile[p], maxpos + 1, reinterpret_cast<float*>(sm), &fold_last, UC * 64);
   }
+  finish_items(a.work);
 }
 
 // top-c columns of each (tile, KV head) that needs a column set.  A row of n
@@ -2604,8 +2599,12 @@ __global__ void __launch_bounds__(256, 1) k_correct_tc(const CorrectArgs a) {
   const int bits = cv.bits;
   const size_t rb = cv.row_bytes_codes(), ns = cv.hd >> cv.lg;
   const size_t step = static_cast<size_t>(2) * cv.B * cv.Hkv * (SP ? cv.rows : cv.T);
-  for (int it = blockIdx.x; it < nent * a.Hkv * npass; it += gridDim.x) {
-    const int p = it / (a.Hkv * npass), g = (it / npass) % a.Hkv, pass = it % npass;
+  __shared__ int s_item;
+  for (;;) {
+    const int it = next_item(a.work, &s_item);
+    if (it >= nent * a.Hkv * npass) break;
+    // passes outermost (every plan entry has a first pass), the latest tiles (the longest rows) first
+    const int pass = it / (nent * a.Hkv), p = nent - 1 - (it / a.Hkv) % nent, g = it % a.Hkv;
     const int qb = a.plan.qb[p], qe = a.plan.qe[p], tl = a.plan.tile[p];
     const int npairs = (qe - qb) * grp, pb = pass * 64;
     if (pb >= npairs) continue;   // (uniform over the CTA)
@@ -2932,6 +2931,7 @@ __global__ void __launch_bounds__(256, 1) k_correct_tc(const CorrectArgs a) {
       }
     }
   }
+  finish_items(a.work);
 }
 
 // ============================================================================
@@ -3392,17 +3392,18 @@ cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, co
   return launch_k(g_pdl, k_plan_tiles, dim3(1), dim3(1024), 0, s, idx, n_sel, tile, has_c, p);
 }
 // (both also stage one row of column keys, up to kSelColsSmemKeys, for the folded selection)
-size_t dscore_tc_smem() { return 1024 + 8 * 64 * 128 * 2; }   // 4 query tiles, 2 base stages, new hi / lo
+// 2 query tiles, 2 base stages, the residual tile; at least the folded selection's key row
+size_t dscore_tc_smem() { return std::max<size_t>(1024 + 5 * 64 * 128 * 2, 1024 + kSelColsSmemKeys * 4); }
 size_t dscore_smem(int hd) {
   return std::max<size_t>(static_cast<size_t>(2) * kDsPairs * 4 * (hd / 4 + 4) * 4, kSelColsSmemKeys * 4);
 }
 cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s) {
   DScoreArgs b = a;
   b.max_chunks = max_chunks;
-  if (a.tc && a.hd == 128) {   // prefill tiles: the tensor-core kernel, one CTA per SM
+  if (a.tc && a.hd == 128) {   // prefill tiles: the tensor-core kernel, two CTAs per SM
     // grid-stride over (tile, KV head, unit of kDsTcUnit chunks) items
     const int items = max_need * a.Hkv * ((max_chunks + kDsTcUnit - 1) / kDsTcUnit);
-    const dim3 g1(items < kDscoreSMs ? items : kDscoreSMs);
+    const dim3 g1(items < 2 * kDscoreSMs ? items : 2 * kDscoreSMs);
     const size_t smt = dscore_tc_smem();
     const bool sp = a.cv.rows != 0;
 #define FL_DST(KMv)                                                                                    \

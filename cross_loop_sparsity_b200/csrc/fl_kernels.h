@@ -151,6 +151,7 @@ struct DScoreArgs {
   int max_cols;
   int max_chunks;       // 64-column chunks of the longest row (set by the launcher)
   int ds_block;         // columns per work item of the SIMT kernel (set by the launcher)
+  int* work;            // tensor-core kernel: [2] next work item, CTAs finished (zero between launches)
   int tc;               // 1: the tensor-core kernel (prefill tiles, head_dim 128)
   // 1: the CTA finishing a row's last chunk also selects its column set (rows of
   // at most kSelColsSmemKeys columns), with `sel`; row_tickets [max_need][Hkv]
@@ -189,6 +190,7 @@ struct CorrectArgs {
   int tc;                       // prefill tiles, head_dim 128: the tensor-core kernel, per (tile, group)
   TilePlan plan;                // (tc) the loop's query tiles and their selected slots
   int q_tile, max_entries;      // (tc) query tile size; bound on the plan's entries
+  int* work;                    // (tc) [2] next work item, CTAs finished (zero between launches)
   float* part_acc;              // [n_sel][Hkv][n_splits][2][8][hd]: new-term, old-term numerators
   float* part_mz;               // [n_sel][Hkv][n_splits][8][3]: max, new-term, old-term denominators
   int* counters;                // [n_sel][Hkv], zero between launches

@@ -69,6 +69,7 @@ struct flashloop_ctx {
   int* attn_counters = nullptr;
   float *corr_acc = nullptr, *corr_mz = nullptr;
   int* corr_counters = nullptr;
+  int* work_ctr = nullptr;        // [0..1] delta-score, [2..3] correction: next item, CTAs finished
   float* gemm_partial = nullptr;
   size_t gemm_partial_cap = 0;
   int* gemm_counters = nullptr;
@@ -276,6 +277,7 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
   uint8_t* corr_acc = take(std::max<size_t>(cp_rows, 1) * 2 * 8 * hd * 4);
   uint8_t* corr_mz = take(std::max<size_t>(cp_rows, 1) * 8 * 3 * 4);
   uint8_t* corr_counters = take(static_cast<size_t>(std::max(nsel_max, 1)) * Hkv * 4);
+  uint8_t* work_ctr = take(16 * 4);   // work-item counters of the tensor-core delta-score and correction
   // GEMM split-K partials (skinny orientation only)
   size_t gp = 0;
   if (N <= 64 || c.max_batch <= 64) {
@@ -388,6 +390,7 @@ size_t layout(const flashloop_config& c, flashloop_ctx* x) {
     x->corr_acc = reinterpret_cast<float*>(corr_acc);
     x->corr_mz = reinterpret_cast<float*>(corr_mz);
     x->corr_counters = reinterpret_cast<int*>(corr_counters);
+    x->work_ctr = reinterpret_cast<int*>(work_ctr);
     x->gemm_partial = reinterpret_cast<float*>(gpart);
     x->gemm_partial_cap = gp;
     x->gemm_counters = reinterpret_cast<int*>(gcnt);
@@ -674,6 +677,7 @@ fl_status run_layer(flashloop_ctx* ctx, const LayerRef& L, const CallShape& cs, 
     ca.cluster = (cs.decode && cs.n_sel <= kCorrSmallQueries && ctx->corr_cluster) ? 1 : 0;
     ca.tc = (!cs.decode && ctx->tc_prefill) ? 1 : 0;   // many queries per tile: tensor-core products
     ca.plan = ctx->plan; ca.q_tile = c.q_tile; ca.max_entries = cs.max_need;   // plan entries <= min(n_sel, tiles)
+    ca.work = ctx->work_ctr + 2;
     SelColsArgs sa{};
     sa.plan = ctx->plan; sa.idx = idx; sa.pos = ctx->pos; sa.meta = ctx->sel_meta; sa.col_keys = ctx->col_keys;
     sa.max_cols = c.max_ctx; sa.Hkv = Hkv; sa.c = c.c_cols; sa.j = L.cj; sa.n_tiles = ctx->n_tiles_max;
@@ -693,6 +697,7 @@ fl_status run_layer(flashloop_ctx* ctx, const LayerRef& L, const CallShape& cs, 
     da.fold = cs.col_span <= kSelColsSmemKeys ? 1 : 0;
     da.sel = sa;
     da.row_tickets = ctx->row_tickets;
+    da.work = ctx->work_ctr;
     FL_LAUNCH(FL_KIND_DSCORE, launch_dscore(da, cs.max_need, cs.max_chunks, s));
     if (!da.fold) FL_LAUNCH(FL_KIND_SELECT, launch_select_cols(sa, cs.max_need, cs.col_span, s));
     FL_LAUNCH(FL_KIND_CORRECT, launch_correct(ca, n, s));
