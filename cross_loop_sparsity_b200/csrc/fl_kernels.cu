@@ -1007,11 +1007,12 @@ __global__ void __launch_bounds__(256) k_attn_prefill(const AttnPreArgs a) {
 // 64-key tiles of the sequence's cache (the context before a chunk, then the
 // chunk up to each query's own position).  K and V tiles arrive by TMA
 // (128-byte swizzle, 64-row boxes) in a ring of kPreStages.  S = tau * Q K^T
-// and O += P V are warp-level bf16 products with fp32 accumulation: Q and P are
-// carried as bf16 hi + lo pairs (two products into one accumulator, about 16
-// significant bits, as the fp32 kernel), P straight from the score registers
-// (the accumulator layout of two 8-key score tiles is the A-operand layout of
-// one 16-key step), V's fragments from ldmatrix with transposition.  The
+// and O += P V are warp-level bf16 products with fp32 accumulation: Q is
+// carried as a bf16 hi + lo pair (two products into one accumulator, about 16
+// significant bits, so the scores are as accurate as the fp32 kernel's), P as
+// bf16 straight from the score registers (the accumulator layout of two 8-key
+// score tiles is the A-operand layout of one 16-key step), V's fragments from
+// ldmatrix with transposition.  The
 // online softmax runs on the score fragments; a row's statistics live in the
 // four threads of a quad.
 // ============================================================================
@@ -1177,18 +1178,16 @@ __global__ void __launch_bounds__(128, 2) k_attn_prefill_tc(const __grid_constan
       o[n][2] *= alpha[1];
       o[n][3] *= alpha[1];
     }
-    // ---- O += P V over the tile's 64 keys (4 steps of 16); P as a bf16 hi + lo pair
+    // ---- O += P V over the tile's 64 keys (4 steps of 16); P in [0, 1] as bf16
+    // (a relative rounding of 2^-9 per weight, which the weighted sum averages;
+    // the row sums l use the fp32 weights)
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
-      uint32_t ph[4], pl[4];
+      uint32_t ph[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const float* src = sc[2 * kk + (r >> 1)] + 2 * (r & 1);   // (row, row+8) x (keys 0-7, 8-15)
-        float h0, l0, h1, l1;
-        split_bf16(src[0], h0, l0);
-        split_bf16(src[1], h1, l1);
-        ph[r] = pack_bf16x2(h0, h1);
-        pl[r] = pack_bf16x2(l0, l1);
+        ph[r] = pack_bf16x2(src[0], src[1]);
       }
       const int vr = kk * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;   // V row (key) this lane addresses
 #pragma unroll
@@ -1197,9 +1196,7 @@ __global__ void __launch_bounds__(128, 2) k_attn_prefill_tc(const __grid_constan
         uint32_t vf[4];
         ldsm_x4_t(Vt + (ch >> 3) * BOX_BYTES + vr * 128 + (((ch & 7) ^ (vr & 7)) << 4), vf);
         mma_bf16_16816(o[2 * n2], ph, vf[0], vf[1]);
-        mma_bf16_16816(o[2 * n2], pl, vf[0], vf[1]);
         mma_bf16_16816(o[2 * n2 + 1], ph, vf[2], vf[3]);
-        mma_bf16_16816(o[2 * n2 + 1], pl, vf[2], vf[3]);
       }
     }
     __syncthreads();   // every warp is done with the slot
@@ -1588,16 +1585,32 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
     const int lo = lower_bound_i(s_idx, a.n_sel, t);
     const int sl = (lo < a.n_sel && s_idx[lo] == t) ? lo : -1;
     a.sel_slot[t] = sl;
-    if (a.cv.rows) {   // sparse residual storage: pool rows of this loop's recomputed tokens
-      const int Tc = a.N / a.B_call, b = t / Tc;
-      rows_assign(a.cv, a.loop, b, a.pos[t], sl >= 0 ? sl - lower_bound_i(s_idx, a.n_sel, b * Tc) : -1, a.status);
-    }
+    s_slot[t] = sl;   // (the previous slots are dead after the change keys)
   }
   if (a.cv.rows) {
+    // sparse residual storage: pool rows of this loop's recomputed tokens, one
+    // (token, layer) per thread so the layers' counts are read in parallel
+    __syncthreads();
+    const int Tc = a.N / a.B_call, M = a.cv.M;
+    for (int e = threadIdx.x; e < a.N * M; e += blockDim.x) {
+      const int t = e % a.N, j = e / a.N, b = t / Tc, sl = s_slot[t];
+      int r = -1;
+      if (sl >= 0) {
+        r = a.cv.rcount[(static_cast<size_t>(j) * (a.cv.K - 1) + (a.loop - 2)) * a.cv.B + b] + sl -
+            lower_bound_i(s_idx, a.n_sel, b * Tc);
+        if (r >= a.cv.rows) {
+          r = -1;
+          if (a.status) atomicOr(a.status, kErrCapacity);
+        }
+      }
+      a.cv.ridx[a.cv.ridx_index(j, a.loop, b, a.pos[t])] = r;
+    }
     __syncthreads();   // every token has read the counts
-    const int Tc = a.N / a.B_call;
-    for (int b = threadIdx.x; b < a.B_call; b += blockDim.x)
-      rows_advance(a.cv, a.loop, b, lower_bound_i(s_idx, a.n_sel, (b + 1) * Tc) - lower_bound_i(s_idx, a.n_sel, b * Tc));
+    for (int e = threadIdx.x; e < a.B_call * M; e += blockDim.x) {
+      const int b = e % a.B_call, j = e / a.B_call;
+      int* rc = a.cv.rcount + (static_cast<size_t>(j) * (a.cv.K - 1) + (a.loop - 2)) * a.cv.B + b;
+      *rc = min(a.cv.rows, *rc + lower_bound_i(s_idx, a.n_sel, (b + 1) * Tc) - lower_bound_i(s_idx, a.n_sel, b * Tc));
+    }
   }
   // snapshot of the selected rows (and, if asked, their normalised bf16 copy).
   // Work items are 512-element slices of a row, one per warp at a time; a
@@ -1607,6 +1620,9 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
   const int nsl = (a.d + SL - 1) / SL;
   const bool norm = a.norm_gain != nullptr;
   float* s_ss = s_key;   // [kSelectStepMaxNorm * kSelectStepSlices]; the keys are dead after the selection
+  // with at most one slice per warp the normalisation reuses the slice in registers
+  const bool keep = norm && a.n_sel * nsl <= nw;
+  float4 vk[SL / 128];
   for (int it = warp; it < a.n_sel * nsl; it += nw) {
     const int r = it / nsl, c0 = (it % nsl) * SL;
     const float* src = a.h + static_cast<size_t>(s_idx[r]) * a.d;
@@ -1627,6 +1643,10 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
     if (norm) {
       ss = warp_sum(ss);
       if (lane == 0) s_ss[it] = ss;
+    }
+    if (keep) {
+#pragma unroll
+      for (int u = 0; u < SL / 128; ++u) vk[u] = v[u];
     }
   }
   if (norm) {
@@ -1650,7 +1670,8 @@ __global__ void __launch_bounds__(1024) k_select_step(const SelectStepArgs a) {
 #pragma unroll
       for (int u = 0; u < SL / 128; ++u) {
         const int c = c0 + u * 128 + lane * 4;
-        v[u] = c < a.d ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+        // keep: item it of this loop is item it of the snapshot loop, held by this warp
+        v[u] = keep ? vk[u] : (c < a.d ? *reinterpret_cast<const float4*>(src + c) : make_float4(0.f, 0.f, 0.f, 0.f));
         gv[u] = c < a.d ? *reinterpret_cast<const float4*>(a.norm_gain + c) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
@@ -1725,7 +1746,10 @@ __device__ __forceinline__ void fold_select(const DScoreArgs& a, int seg, int g,
 // CTA takes a contiguous range of items, so the tile's pairs, staged in shared
 // memory kDsPairs at a time, are reused while (tile, KV head) stays the same,
 // and with sparse storage the item's pool rows of every level are staged
-// first, so each step needs one memory round trip.  A quad of lanes owns one
+// first, so each step needs one memory round trip.  The key is evaluated as
+// (q_l - q_last) . K_base + q_l . R, R = K_l - K_base = the residual sum: the
+// queries' difference is formed in fp32 when staged, and a column without
+// residual rows (most of them) costs one product per pair.  A quad of lanes owns one
 // column: lane qd of the quad holds dims [qd*HD/4, (qd+1)*HD/4) of K_l and
 // K_base, all of whose loads (index rows first with sparse storage, then base,
 // codes and scales of every level) are issued before any is used; the quad's
@@ -1742,7 +1766,7 @@ __global__ void __launch_bounds__(256, 2) k_dscore(const DScoreArgs a) {
   constexpr int QS = DPL + 4;              // padded stride of one lane-quarter of a staged query row
   extern __shared__ __align__(16) uint8_t sm[];
   float* qn_sm = reinterpret_cast<float*>(sm);       // [kDsPairs][4][QS]: tau * q_l
-  float* qo_sm = qn_sm + kDsPairs * 4 * QS;           // [kDsPairs][4][QS]: tau * q_last
+  float* qo_sm = qn_sm + kDsPairs * 4 * QS;           // [kDsPairs][4][QS]: tau * (q_l - q_last)
   __shared__ int qpos_sm[kDsPairs], qtok_sm[kDsPairs], qi_sm[kDsPairs];
   __shared__ float best_sm[kDsBlock];            // the item's column keys so far (one owner quad per column)
   __shared__ int rows_sm[SP ? (KM - 1) * kDsBlock : 1];   // sparse storage: pool rows of the item's columns
@@ -1807,8 +1831,9 @@ __global__ void __launch_bounds__(256, 2) k_dscore(const DScoreArgs a) {
           float vn = 0.f, vo = 0.f;
           if (pr < np) {
             const int hh = g * grp + (pb + pr) % grp;
-            vn = a.tau * a.q_cur[(static_cast<size_t>(qi_sm[pr]) * a.H + hh) * HD + dd];
-            vo = a.tau * a.q_last[(static_cast<size_t>(qtok_sm[pr]) * a.H + hh) * HD + dd];
+            const float xn = a.q_cur[(static_cast<size_t>(qi_sm[pr]) * a.H + hh) * HD + dd];
+            vn = a.tau * xn;
+            vo = a.tau * (xn - a.q_last[(static_cast<size_t>(qtok_sm[pr]) * a.H + hh) * HD + dd]);
           }
           const int o = (pr * 4 + dd / DPL) * QS + dd % DPL;
           qn_sm[o] = vn;
@@ -1860,35 +1885,42 @@ __global__ void __launch_bounds__(256, 2) k_dscore(const DScoreArgs a) {
             sraw[q] = cv.scales[ri * ns + gi];
           }
         }
-        // ---- K_l = base + code * scale of loops 2..l, added in loop order in fp32
-        // (the base stays packed: two bf16 per word, widened where it is used)
-        uint32_t kb[DPL / 2];
+        // ---- the key through (q_l - q_last) . K_base + q_l . R, R = the sum of
+        // code * scale of loops 2..l in loop order (fp32): one product per pair
+        // for a column without residual rows, two with
+        float kb[DPL], rs[DPL];
+        bool has_r = false;
+#pragma unroll
+        for (int q = 0; q < KM - 1; ++q) has_r = has_r || (q + 2 <= a.loop && rr[q] >= 0);
 #pragma unroll
         for (int u = 0; u < DPL / 8; ++u) {
-          kb[4 * u] = braw[u].x;
-          kb[4 * u + 1] = braw[u].y;
-          kb[4 * u + 2] = braw[u].z;
-          kb[4 * u + 3] = braw[u].w;
+          const uint32_t w[4] = {braw[u].x, braw[u].y, braw[u].z, braw[u].w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            kb[u * 8 + 2 * k] = bf16_to_f(w[k] & 0xFFFF);
+            kb[u * 8 + 2 * k + 1] = bf16_to_f(w[k] >> 16);
+          }
         }
-        float kn[DPL];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) kn[e] = bf16_to_f(e & 1 ? kb[e / 2] >> 16 : kb[e / 2] & 0xFFFF);
+        for (int e = 0; e < DPL; ++e) rs[e] = 0.f;
+        if (has_r) {
 #pragma unroll
-        for (int q = 0; q < KM - 1; ++q) {
-          if (q + 2 > a.loop) break;
-          const float sc = half_bits_to_f(sraw[q]);
-          const uint32_t w[4] = {craw[q].x, craw[q].y, craw[q].z, craw[q].w};
-          if (bits == 4) {   // element e: nibble e % 8 of word e / 8 (low nibble first)
+          for (int q = 0; q < KM - 1; ++q) {
+            if (q + 2 > a.loop) break;
+            const float sc = half_bits_to_f(sraw[q]);
+            const uint32_t w[4] = {craw[q].x, craw[q].y, craw[q].z, craw[q].w};
+            if (bits == 4) {   // element e: nibble e % 8 of word e / 8 (low nibble first)
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) {
-              const int c = sext(static_cast<int>((w[e / 8] >> ((e % 8) * 4)) & 0xFu), 4);
-              kn[e] = __fadd_rn(kn[e], __fmul_rn(static_cast<float>(c), sc));
-            }
-          } else {           // element e: bits 2(e % 16) of word e / 16 (LSB first)
+              for (int e = 0; e < DPL; ++e) {
+                const int c = sext(static_cast<int>((w[e / 8] >> ((e % 8) * 4)) & 0xFu), 4);
+                rs[e] = __fadd_rn(rs[e], __fmul_rn(static_cast<float>(c), sc));
+              }
+            } else {           // element e: bits 2(e % 16) of word e / 16 (LSB first)
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) {
-              const int c = sext(static_cast<int>((w[e / 16] >> ((e % 16) * 2)) & 0x3u), 2);
-              kn[e] = __fadd_rn(kn[e], __fmul_rn(static_cast<float>(c), sc));
+              for (int e = 0; e < DPL; ++e) {
+                const int c = sext(static_cast<int>((w[e / 16] >> ((e % 16) * 2)) & 0x3u), 2);
+                rs[e] = __fadd_rn(rs[e], __fmul_rn(static_cast<float>(c), sc));
+              }
             }
           }
         }
@@ -1897,17 +1929,21 @@ __global__ void __launch_bounds__(256, 2) k_dscore(const DScoreArgs a) {
 #pragma unroll 1
         for (int pr = 0; pr < np; ++pr) {
           const float* qn = qn_sm + (pr * 4 + qd) * QS;
-          const float* qo = qo_sm + (pr * 4 + qd) * QS;
-          float dn = 0.f, db = 0.f;
+          const float* qdl = qo_sm + (pr * 4 + qd) * QS;
+          float dd = 0.f, dr = 0.f;
 #pragma unroll
           for (int e = 0; e < DPL; e += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(qn + e);
-            const float4 y = *reinterpret_cast<const float4*>(qo + e);
-            dn += kn[e] * x.x + kn[e + 1] * x.y + kn[e + 2] * x.z + kn[e + 3] * x.w;
-            db += bf16_to_f(kb[e / 2] & 0xFFFF) * y.x + bf16_to_f(kb[e / 2] >> 16) * y.y +
-                  bf16_to_f(kb[e / 2 + 1] & 0xFFFF) * y.z + bf16_to_f(kb[e / 2 + 1] >> 16) * y.w;
+            const float4 y = *reinterpret_cast<const float4*>(qdl + e);
+            dd += kb[e] * y.x + kb[e + 1] * y.y + kb[e + 2] * y.z + kb[e + 3] * y.w;
           }
-          float d = dn - db;
+          if (has_r) {
+#pragma unroll
+            for (int e = 0; e < DPL; e += 4) {
+              const float4 x = *reinterpret_cast<const float4*>(qn + e);
+              dr += rs[e] * x.x + rs[e + 1] * x.y + rs[e + 2] * x.z + rs[e + 3] * x.w;
+            }
+          }
+          float d = dd + dr;
           d += __shfl_xor_sync(0xffffffffu, d, 1);
           d += __shfl_xor_sync(0xffffffffu, d, 2);
           if (col <= qpos_sm[pr]) m = fmaxf(m, fabsf(d));
@@ -3047,8 +3083,8 @@ __global__ void __launch_bounds__(32 * kCorrWarps) k_correct_cluster(const Corre
     park(1);
   }
   // new term: this loop's queries against the rebuilt chains, CPI columns at
-  // a time (one with sparse storage, whose index rows would otherwise not fit
-  // in registers beside the chains)
+  // a time (one for sparse chains longer than four levels, whose index rows
+  // would otherwise not fit in registers beside the chains)
 #pragma unroll
   for (int h = 0; h < GRP; ++h) {
     const size_t hq = static_cast<size_t>(g * GRP + h);
@@ -3057,7 +3093,7 @@ __global__ void __launch_bounds__(32 * kCorrWarps) k_correct_cluster(const Corre
   }
   reset();
   {
-    constexpr int CPI = SP ? 1 : 2;
+    constexpr int CPI = (SP && KM > 4) ? 1 : 2;
     for (int kb = k0 + warp; kb < k1v; kb += CPI * NW) {
       int col[CPI];
 #pragma unroll

@@ -1069,8 +1069,8 @@ fl_status flashloop_decode_step(flashloop_ctx* ctx, const float* h0, int B, floa
   FL_TRY(cudaMemcpyAsync(ctx->h_in, h0, static_cast<size_t>(B) * c.d_model * 4, cudaMemcpyDefault, s));
   // A decode step's launch sequence depends on B only; after one direct run it
   // is captured once into a CUDA graph and replayed (not on the legacy stream).
-  const int gkey = B * 32 + (ctx->prof ? 1 : 0) + (ctx->pdl ? 2 : 0) + (ctx->gemm_times ? 8 : 0) +
-                   (ctx->corr_cluster ? 16 : 0);
+  const int gkey = B * 128 + (ctx->prof ? 1 : 0) + (ctx->pdl ? 2 : 0) + (ctx->gemm_times ? 8 : 0) +
+                   (ctx->corr_cluster ? 16 : 0) + (ctx->tc_prefill ? 64 : 0);
   size_t gi = 0;
   while (gi < ctx->graph_b.size() && ctx->graph_b[gi] != gkey) ++gi;
   bool seen = false;

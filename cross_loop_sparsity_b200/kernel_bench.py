@@ -21,6 +21,8 @@
   (65536 tokens x 4 layers x 4 KV heads x (K, V) rows of 128): reads the new
   fp32 rows and the previous bf16 rows (1.61 GB), writes packed int4 codes and
   fp16 scales (0.14 GB); bytes moved against HBM.
+* ``lazy_call_capture`` (only on request, for ncu): one lazy call of
+  ``--workload`` with ``--layers`` shared layers, kernels launched directly.
 * ``quantize``: the KV-residual quantiser over a residual shaped like the
   65536-token context (65536 tokens x 4 layers x 2 (K, V) x 4 KV heads rows of
   128 fp32, int4 / int2, group 64), bytes moved against HBM.
@@ -239,20 +241,69 @@ def decode_step_capture(reps):
     return []
 
 
+CAPTURE = {"workload": "c3", "layers": 2}
+
+
+def lazy_call_capture(reps):
+    """One lazy call of a workload (prefill or decode, sparse residual storage,
+    kernels launched directly) after one warm-up call, for ncu captures of its
+    lazy-loop kernels: the workload's shapes with `--layers` shared layers, so
+    the device holds a few GB at most.  Prints the call's duration (under ncu:
+    not a measurement)."""
+    import math
+    import torch
+    from cross_loop_sparsity_b200 import flashloop as fl, synth
+    cfg = synth.config(CAPTURE["workload"])
+    if CAPTURE["layers"]:
+        cfg = cfg.with_(n_layers=CAPTURE["layers"])
+    w = synth.make_weights_device(cfg)
+    if cfg.mode == "prefill":
+        B, T = cfg.batch, cfg.seq_len
+        cfg = cfg.with_(resid_rows=min(T, int(math.ceil(cfg.rho * B * T - 1e-9))))
+        eng = fl.FlashLoop(cfg, w, max_batch=B, max_ctx=T, max_tokens=B * T)
+        h0 = torch.randn((B * T, cfg.d_model), device="cuda")
+        run = lambda: (eng.reset(None), eng.prefill(h0, B, T))
+    else:
+        B = cfg.batch
+        cfg = cfg.with_(resid_rows=synth.sparse_rows(cfg, B))
+        lens = [cfg.ctx_len] * B
+        eng = fl.FlashLoop(cfg, w, max_batch=B, max_ctx=cfg.ctx_len + 1)
+        eng.load_context_device(lens)
+        eng.set_option(fl.FL_OPT_USE_GRAPH, 0)
+        h0 = torch.randn((B, cfg.d_model), device="cuda")
+        run = lambda: (eng.reset(lens), eng.decode_step(h0, B))
+    run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    run()
+    b.record()
+    b.synchronize()
+    assert eng.sync_status() == 0
+    eng.close()
+    return [{"kernel": "lazy call", "workload": CAPTURE["workload"], "layers": cfg.n_layers,
+             "ms": a.elapsed_time(b), "note": "kernels launched directly, for ncu captures"}]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--only", default="", help="comma-separated subset, e.g. gemm_wide,topk")
+    ap.add_argument("--workload", default="c3", help="lazy_call_capture: the workload")
+    ap.add_argument("--layers", type=int, default=2, help="lazy_call_capture: shared layers (0: the workload's)")
     args = ap.parse_args()
+    CAPTURE.update(workload=args.workload, layers=args.layers)
     from cross_loop_sparsity_b200 import build
     build.build()
     import time
     import torch
     from cross_loop_sparsity_b200.clocks import ClockSampler
-    fns = (gemm_wide, gemm_skinny, topk, attn_decode, quantize_residual, quantize, decode_step_capture)
+    fns = (gemm_wide, gemm_skinny, topk, attn_decode, quantize_residual, quantize, decode_step_capture,
+           lazy_call_capture)
+    captures = (decode_step_capture, lazy_call_capture)
     only = {x for x in args.only.split(",") if x}
     for fn in fns:
-        if (only and fn.__name__ not in only) or (not only and fn is decode_step_capture):
+        if (only and fn.__name__ not in only) or (not only and fn in captures):
             continue
         sampler = ClockSampler(torch.cuda.current_device())
         sampler.start()

@@ -154,11 +154,16 @@ fl_status flashloop_init(const flashloop_config* cfg, const flashloop_weights* w
 fl_status flashloop_prefill(flashloop_ctx* ctx, const float* h0, int B, int T,
                             float* h_out, float* logits_last, fl_stream_t stream);
 
-/* Append one token to each of sequences 0..B-1 at position len_b.
+/* Append one token to each of sequences 0..B-1 at position len_b: the same
+ * lazy looped step as flashloop_prefill ("FlashLoop ...", abstract), or with
+ * resid_bits 16 the dense looped forward with one KV pass per loop ("Looped
+ * Transformer 教程：权重共享、循环次数与推理成本怎么读", 第一步 and 第四步).
  * h0: [B][d] fp32 (host or device); h_out: [B][d] fp32 or NULL; logits: [B][V]
  * fp32 or NULL (host or device).  The ranking pools the B new tokens; each new
  * token is its own query tile.  The step's kernels are captured once per B
- * into a CUDA graph and replayed.  Lengths advance by one. */
+ * into a CUDA graph and replayed.  Lengths advance by one.
+ * Errors: FL_ERR_INVALID_ARG (NULL h0, B < 1), FL_ERR_CAPACITY (B > max_batch,
+ * or a sequence at max_ctx), FL_ERR_CUDA. */
 fl_status flashloop_decode_step(flashloop_ctx* ctx, const float* h0, int B,
                                 float* h_out, float* logits, fl_stream_t stream);
 
@@ -185,7 +190,9 @@ fl_status flashloop_kv_bytes_for(const flashloop_config* cfg, size_t* total, dou
 fl_status flashloop_reset(flashloop_ctx* ctx, const int* seq_len, fl_stream_t stream);
 
 /* Synchronise `stream` and report the first error a kernel recorded since
- * the last call (FL_ERR_TIMEOUT for a bounded wait that ran out), clearing it. */
+ * the last call, clearing it: FL_ERR_TIMEOUT (a bounded wait ran out),
+ * FL_ERR_CAPACITY (a sparse residual pool was full), FL_ERR_NONFINITE (a
+ * corrected softmax denominator was not positive). */
 fl_status flashloop_sync_status(flashloop_ctx* ctx, fl_stream_t stream);
 
 void flashloop_destroy(flashloop_ctx* ctx);
@@ -347,8 +354,10 @@ typedef enum {
   FL_OPT_GEMM_TIMES = 5, /* 1: every GEMM launch of a call stamps, from the GPU's global nanosecond timer, when
                            its first CTA's dependency wait returned and when its last CTA finished (read with
                            flashloop_gemm_times); 0 (default): off */
-  FL_OPT_TC_PREFILL = 6, /* 1 (default): prefill attention and prefill delta scores on warp-level bf16
-                           tensor-core products (fp32 operands as bf16 hi + lo pairs); 0: the fp32 SIMT kernels */
+  FL_OPT_TC_PREFILL = 6, /* 1 (default): prefill attention, delta scores and correction on warp-level bf16
+                           tensor-core products with fp32 accumulation (attention and correction: queries
+                           as bf16 hi + lo pairs; delta scores: the fp32 query difference, rounded once);
+                           0: the fp32 SIMT kernels */
   FL_OPT_CORR_CLUSTER = 7 /* 1 (default): a decode query's column correction runs as one 16-CTA cluster merged
                            over distributed shared memory; 0: column slices merged by an atomic ticket */
 } fl_option;

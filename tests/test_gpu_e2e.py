@@ -235,9 +235,9 @@ def test_decode_free_running_selection_and_column_sets_are_valid():
 @pytest.mark.parametrize("name,B,T,ctx,M,K", [("c1", 2, 200, 0, 2, 2), ("c3", 1, 700, 0, 2, 2),
                                                ("c3", 1, 300, 500, 2, 2), ("c3", 1, 256, 0, 1, 1)])
 def test_prefill_attention_tensor_core_as_accurate_as_simt(name, B, T, ctx, M, K):
-    """The tensor-core prefill attention (bf16 products, Q and P as hi + lo
-    pairs, about 16 significant bits) is as close to the oracle as the fp32 SIMT
-    kernel: head_dim 64 and 128, a fresh prompt, a chunk onto a residual
+    """The tensor-core prefill attention (bf16 products; Q as a hi + lo pair,
+    about 16 significant bits; the softmax weights as bf16) is as close to the
+    oracle as the fp32 SIMT kernel: head_dim 64 and 128, a fresh prompt, a chunk onto a residual
     context, and a single plain layer.  The two GPU results are not compared
     with each other: both round the attention output to bf16 for the O
     projection, and at that rounding two accurate kernels already differ by
