@@ -64,60 +64,6 @@ struct CacheView {
 
 __device__ __forceinline__ int sext(int v, int bits) { return (v << (32 - bits)) >> (32 - bits); }
 
-// The EPL codes of one lane (elements lane*EPL .. +EPL-1) of a packed row.
-template <int EPL>
-__device__ __forceinline__ void lane_codes(const uint8_t* row, int bits, int lane, int* c) {
-  if (EPL == 4) {
-    if (bits == 4) {
-      const uint32_t u = *reinterpret_cast<const uint16_t*>(row + lane * 2);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) c[e] = sext((u >> (4 * e)) & 0xF, 4);
-    } else {
-      const uint32_t u = row[lane];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) c[e] = sext((u >> (2 * e)) & 0x3, 2);
-    }
-  } else {  // EPL == 2
-    if (bits == 4) {
-      const uint32_t u = row[lane];
-      c[0] = sext(u & 0xF, 4);
-      c[1] = sext((u >> 4) & 0xF, 4);
-    } else {
-      const uint32_t u = (row[lane >> 1] >> ((lane & 1) * 4)) & 0xF;
-      c[0] = sext(u & 0x3, 2);
-      c[1] = sext((u >> 2) & 0x3, 2);
-    }
-  }
-}
-
-// Reconstructed lazy KV of loop m (1 = base) for one row; lane holds EPL values.
-template <int EPL>
-__device__ __forceinline__ void chain_lane(const CacheView& cv, int j, int kv, int b, int h, int t, int m, int lane,
-                                           float* out) {
-  const uint16_t* br = cv.base_row(j, kv, b, h, t) + lane * EPL;
-  if (EPL == 4) {
-    const uint2 u = *reinterpret_cast<const uint2*>(br);
-    out[0] = bf16_to_f(u.x & 0xFFFF);
-    out[1] = bf16_to_f(u.x >> 16);
-    out[2] = bf16_to_f(u.y & 0xFFFF);
-    out[3] = bf16_to_f(u.y >> 16);
-  } else {
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(br);
-    out[0] = bf16_to_f(u & 0xFFFF);
-    out[1] = bf16_to_f(u >> 16);
-  }
-  const int gi = (lane * EPL) >> cv.lg;
-  for (int l = 2; l <= m; ++l) {
-    const int r = cv.res_row(j, l, b, t);
-    if (r < 0) continue;   // no residual stored: zero
-    int c[EPL];
-    lane_codes<EPL>(cv.code_row(j, l, kv, b, h, r), cv.bits, lane, c);
-    const float s = half_bits_to_f(cv.scale_row(j, l, kv, b, h, r)[gi]);
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) out[e] = __fadd_rn(out[e], __fmul_rn(static_cast<float>(c[e]), s));
-  }
-}
-
 // ---------------------------------------------------------------- residual quantiser
 // (the quantiser's scale and code rules, shared by its kernels)
 // The hardware reciprocal approximation (PTX rcp.approx, within 1 ulp of 1/x).

@@ -418,7 +418,7 @@ __global__ void __launch_bounds__(256) k_quantize_rows(const float* __restrict__
 //     lazy l=1: store bf16 base; zero the residual rows of loops 2..K
 //     lazy l>1: r = kv - reconstructed(loop l-1); quantise; store codes+scale
 // ============================================================================
-template <int EPL>
+template <int EPL, int KM, bool SP>
 __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
   pdl_trigger();
   pdl_wait();
@@ -497,8 +497,10 @@ __global__ void __launch_bounds__(128) k_qkv_post(const QkvPostArgs a) {
 #pragma unroll
       for (int e = 0; e < EPL; ++e) tr[e] = x[e];
     }
-    float prev[EPL];
-    chain_lane<EPL>(cv, a.j, kv, b, gk, t, a.loop - 1, lane, prev);
+    // the previous level, every level's loads issued together (levels without a
+    // row add code 0 x scale 0, as a stored zero row does)
+    float prev[EPL], unused[EPL];
+    chain_lane2<EPL, KM, SP>(cv, a.j, kv, b, gk, t, a.loop - 1, a.loop - 1, lane, unused, prev);
     float r[EPL];
 #pragma unroll
     for (int e = 0; e < EPL; ++e) r[e] = __fsub_rn(x[e], prev[e]);
@@ -1767,6 +1769,9 @@ __global__ void __launch_bounds__(256, 2) k_dscore(const DScoreArgs a) {
   extern __shared__ __align__(16) uint8_t sm[];
   float* qn_sm = reinterpret_cast<float*>(sm);       // [kDsPairs][4][QS]: tau * q_l
   float* qo_sm = qn_sm + kDsPairs * 4 * QS;           // [kDsPairs][4][QS]: tau * (q_l - q_last)
+  // each warp's base rows of its 8 columns, double-buffered: [warps][2][8][HD] bf16
+  constexpr int WBUF = 2 * 8 * HD * 2;
+  uint8_t* wbuf_all = sm + 2 * kDsPairs * 4 * QS * 4;
   __shared__ int qpos_sm[kDsPairs], qtok_sm[kDsPairs], qi_sm[kDsPairs];
   __shared__ float best_sm[kDsBlock];            // the item's column keys so far (one owner quad per column)
   __shared__ int rows_sm[SP ? (KM - 1) * kDsBlock : 1];   // sparse storage: pool rows of the item's columns
@@ -1842,21 +1847,43 @@ __global__ void __launch_bounds__(256, 2) k_dscore(const DScoreArgs a) {
         staged = one_group ? key : -1;
       }
       __syncthreads();
+      // the base rows of this warp's 8 columns of step s, copied into its buffer
+      // s & 1 (columns past the last eligible one read zero); step s + 1's copy
+      // is in flight while step s is computed
+      uint8_t* wbuf = wbuf_all + warp * WBUF;
+      auto issue_cols = [&](int st) {
+        const int cb = c0 + st * 64 + warp * 8;
+        const uint32_t dst = smem_u32(wbuf + (st & 1) * (WBUF / 2));
+        constexpr int PR = HD * 2 / 16;   // 16-byte pieces per row
+#pragma unroll
+        for (int k = lane; k < 8 * PR; k += 32) {
+          const int r = k / PR, pc = k % PR, cc = cb + r;
+          const bool ok = cc <= maxpos;
+          cp_async16(dst + k * 16, cv.base_row(a.j, 0, b, g, ok ? cc : c0) + pc * 8, ok ? 16u : 0u);
+        }
+        cp_async_commit();
+      };
+      issue_cols(0);
 #pragma unroll 1
       for (int s = 0; s < nsteps; ++s) {
         const int col = c0 + s * 64 + warp * 8 + col_in_warp;
         const bool valid = col <= maxpos;
-        // ---- loads: base dims of this lane, then every level's codes and scale
+        if (s + 1 < nsteps) {
+          issue_cols(s + 1);
+          cp_async_wait<1>();
+        } else {
+          cp_async_wait<0>();
+        }
+        __syncwarp();   // every lane's copies of step s are visible to the warp
+        // ---- base dims of this lane from the buffer, then every level's codes and scale
         uint4 braw[DPL / 8];
         uint4 craw[KM - 1];
         uint16_t sraw[KM - 1];
-        if (valid) {
-          const uint4* br = reinterpret_cast<const uint4*>(cv.base_row(a.j, 0, b, g, col) + qd * DPL);
+        {
+          const uint4* br = reinterpret_cast<const uint4*>(wbuf + (s & 1) * (WBUF / 2) + col_in_warp * HD * 2 +
+                                                           qd * DPL * 2);
 #pragma unroll
           for (int u = 0; u < DPL / 8; ++u) braw[u] = br[u];
-        } else {
-#pragma unroll
-          for (int u = 0; u < DPL / 8; ++u) braw[u] = make_uint4(0u, 0u, 0u, 0u);
         }
         int rr[KM - 1];
 #pragma unroll
@@ -1950,6 +1977,7 @@ __global__ void __launch_bounds__(256, 2) k_dscore(const DScoreArgs a) {
         }
         const int slot = s * 64 + warp * 8 + col_in_warp;
         if (qd == 0) best_sm[slot] = fmaxf(best_sm[slot], m);
+        __syncwarp();   // buffer s & 1 is read before step s + 2's copy reuses it
       }
     }
     // ---- this item's keys (each written by the lane that owns the column)
@@ -3345,10 +3373,25 @@ cudaError_t launch_rmsnorm_rows(const float* h, const int* idx, int n, int n_pad
                                 uint16_t* x, cudaStream_t s) {
   return launch_k(g_pdl, k_rmsnorm_rows, dim3(n_pad), dim3(256), 0, s, h, idx, n, d, gain, eps, x);
 }
+template <int EPL, int KM>
+cudaError_t launch_qkv_post_km(const QkvPostArgs& a, dim3 grid, cudaStream_t s) {
+  return a.cv.rows ? launch_k(g_pdl, k_qkv_post<EPL, KM, true>, grid, dim3(128), 0, s, a)
+                   : launch_k(g_pdl, k_qkv_post<EPL, KM, false>, grid, dim3(128), 0, s, a);
+}
+template <int EPL>
+cudaError_t launch_qkv_post_e(const QkvPostArgs& a, dim3 grid, cudaStream_t s) {
+  switch (chain_km(a.cv.K)) {
+    case 2: return launch_qkv_post_km<EPL, 2>(a, grid, s);
+    case 4: return launch_qkv_post_km<EPL, 4>(a, grid, s);
+    case 8: return launch_qkv_post_km<EPL, 8>(a, grid, s);
+    case 16: return launch_qkv_post_km<EPL, 16>(a, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
 cudaError_t launch_qkv_post(const QkvPostArgs& a, cudaStream_t s) {
   const int warps = a.n * (a.H + 2 * a.Hkv);
-  if (a.hd == 128) return launch_k(g_pdl, k_qkv_post<4>, dim3((warps + 3) / 4), dim3(128), 0, s, a);
-  return launch_k(g_pdl, k_qkv_post<2>, dim3((warps + 3) / 4), dim3(128), 0, s, a);
+  const dim3 grid((warps + 3) / 4);
+  return a.hd == 128 ? launch_qkv_post_e<4>(a, grid, s) : launch_qkv_post_e<2>(a, grid, s);
 }
 size_t attn_decode_smem(int hd) { return 1024 + static_cast<size_t>(kDecStages) * 2 * kDecTile * hd * 2; }
 cudaError_t launch_attn_decode(const CUtensorMap& kv, const AttnDecArgs& a, int n, cudaStream_t s) {
@@ -3430,8 +3473,9 @@ cudaError_t launch_plan_tiles(const int32_t* idx, int n_sel, const int* tile, co
 // (both also stage one row of column keys, up to kSelColsSmemKeys, for the folded selection)
 // 2 query tiles, 2 base stages, the residual tile; at least the folded selection's key row
 size_t dscore_tc_smem() { return std::max<size_t>(1024 + 5 * 64 * 128 * 2, 1024 + kSelColsSmemKeys * 4); }
-size_t dscore_smem(int hd) {
-  return std::max<size_t>(static_cast<size_t>(2) * kDsPairs * 4 * (hd / 4 + 4) * 4, kSelColsSmemKeys * 4);
+size_t dscore_smem(int hd) {   // staged pairs + the warps' column buffers, or the folded selection's key row
+  return std::max<size_t>(static_cast<size_t>(2) * kDsPairs * 4 * (hd / 4 + 4) * 4 + 8 * 2 * 8 * hd * 2,
+                          kSelColsSmemKeys * 4);
 }
 cudaError_t launch_dscore(const DScoreArgs& a, int max_need, int max_chunks, cudaStream_t s) {
   DScoreArgs b = a;
