@@ -169,7 +169,7 @@ def run_library(args, world, rank, local):
     ms, clocks = time_steps(eng, lens, h0_dev, logits, stream, args.steps, args.warmup, world, sampler)
     ms_step = ms / args.steps
     assert eng.sync_status(stream) == 0, "a kernel reported an error"
-    launches_per_step = eng.kernels_per_call() + 1          # + the length-reset kernel
+    launches_per_step = eng.kernels_per_call() + (2 if cfg.resid_rows else 1)   # + the reset (lengths, pool counts)
     # then, in replays of the same step after the timed region, the GEMMs stamp
     # their own start (dependency released) and end on the GPU's global timer:
     # two atomics per CTA, kept out of the timed steps
@@ -392,7 +392,7 @@ def measure_decode(name, args, world, local, stream):
         n_sel = B if dense else max(1, min(B, math.ceil(cfg.rho * B - 1e-9)))
         part = {"tokens_per_s": replicas.job_throughput(world, B, ms_step), "ms_per_step": ms_step,
                 "kv_bytes_per_token_per_layer": per, "roofline": decode_roofline(cfg, ms_step, n_sel, dense),
-                "gpu_launches_per_step": eng.kernels_per_call() + 1, "clocks": clocks}
+                "gpu_launches_per_step": eng.kernels_per_call() + (2 if ecfg.resid_rows else 1), "clocks": clocks}
         eng.close()
         del eng
         torch.cuda.empty_cache()
