@@ -21,11 +21,13 @@
   (65536 tokens x 4 layers x 4 KV heads x (K, V) rows of 128): reads the new
   fp32 rows and the previous bf16 rows (1.61 GB), writes packed int4 codes and
   fp16 scales (0.14 GB); bytes moved against HBM.
-* ``lazy_call_capture`` (only on request, for ncu): one lazy call of
-  ``--workload`` with ``--layers`` shared layers, kernels launched directly.
 * ``quantize``: the KV-residual quantiser over a residual shaped like the
   65536-token context (65536 tokens x 4 layers x 2 (K, V) x 4 KV heads rows of
   128 fp32, int4 / int2, group 64), bytes moved against HBM.
+* ``decode_step_capture`` and ``lazy_call_capture`` (only on request, for ncu;
+  no measurement): one decode step at the decode GEMM shapes with one shared
+  layer and a 512-token context, and one lazy call of ``--workload`` with
+  ``--layers`` shared layers; kernels launched directly, a few GB on the device.
 
 Every operand set is rotated over copies whose total exceeds L2 (126 MB), so
 each timed launch reads from HBM; times are CUDA events around ``reps``
