@@ -698,8 +698,15 @@ fl_status run_layer(flashloop_ctx* ctx, const LayerRef& L, const CallShape& cs, 
     da.sel = sa;
     da.row_tickets = ctx->row_tickets;
     da.work = ctx->work_ctr;
-    FL_LAUNCH(FL_KIND_DSCORE, launch_dscore(da, cs.max_need, cs.max_chunks, s));
-    if (!da.fold) FL_LAUNCH(FL_KIND_SELECT, launch_select_cols(sa, cs.max_need, cs.col_span, s));
+    // Column sets are chosen at a tile's first recomputation.  A decode call
+    // that recomputes every token at every lazy loop (n_sel = N) recomputes
+    // each one (its own tile) first at loop 2, so later loops have no tile to
+    // score and these launches would find no work.
+    const bool first_recomputations = !(cs.decode && cs.n_sel == cs.N && L.loop > 2);
+    if (first_recomputations) {
+      FL_LAUNCH(FL_KIND_DSCORE, launch_dscore(da, cs.max_need, cs.max_chunks, s));
+      if (!da.fold) FL_LAUNCH(FL_KIND_SELECT, launch_select_cols(sa, cs.max_need, cs.col_span, s));
+    }
     FL_LAUNCH(FL_KIND_CORRECT, launch_correct(ca, n, s));
   }
   bool sums = false;
