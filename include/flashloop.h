@@ -234,7 +234,9 @@ fl_status flashloop_export_slice(const flashloop_ctx* ctx, int layer, int loop, 
                                  int n, void* codes, void* scales, fl_stream_t stream);
 
 /* Force the selections of the next call (checks only): sel [K-1][n_sel]
- * ascending token indices for loops 2..K; cols [M][n_tiles][Hkv][c_cols]
+ * strictly ascending token indices in [0, N) of that call for loops 2..K
+ * (not checked on the host; n_sel must be the call's own selection count);
+ * cols [M][n_tiles][Hkv][c_cols]
  * ascending column indices with ncols [M][n_tiles][Hkv] valid entries (host
  * arrays).  Either part may be NULL: sel NULL leaves the token selection free,
  * cols and ncols NULL (both) leave the column sets free; all NULL clears.
